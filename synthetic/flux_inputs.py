@@ -1,0 +1,216 @@
+"""Seeded synthetic inputs for the FLUX.2-klein denoising transformer.
+
+This module only draws random numbers and lays bytes out.  It holds none of
+the model's arithmetic: both the CPU oracle (``oracle/``) and the CUDA path
+(``latent_flow_matching_b200``) receive the same arrays from here and compute
+independently.
+
+Recipe (every value is a bf16 number, stored as its 16 raw bits):
+
+* Each weight tensor ``i`` (index in blob order) is filled chunk by chunk; chunk
+  ``c`` (``CHUNK`` elements) comes from ``numpy.random.default_rng([seed, i, c])``
+  (PCG64 seeded through SeedSequence), ``standard_normal(float32)``, multiplied
+  by ``1/sqrt(fan_in)`` in float32, then rounded to bf16 (nearest, ties to even).
+  Gains of the QK-RMSNorm have ``fan_in = 1``; a bias uses its layer's fan-in.
+  Chunking keeps the values independent of the number of worker threads.
+* The latent ``[32, H/8, W/8]``, the text features ``[Nt, txt_dim]`` and the
+  reference latent come from ``default_rng([seed, INPUT_KEY + k])`` with
+  k = 0, 1, 2 respectively, N(0,1) rounded to bf16.
+
+Architecture facts behind the shapes: 5 double-stream and 20 single-stream
+blocks, width 3072, 24 heads of 128 (antirez flux pages, "Modellarchitektur und
+Leistung"; hakusoku "技術詳細"); 32-channel latent packed 2x2 into 128-channel
+tokens (mindverse FLUX.3 write-up, "Zweistufiger Transformer und Tokenisierung").
+"""
+from __future__ import annotations
+
+import dataclasses
+import struct
+from concurrent.futures import ThreadPoolExecutor
+import os
+
+import numpy as np
+
+CHUNK = 1 << 22           # elements per independently seeded chunk
+INPUT_KEY = 1_000_000     # seed-key offset of the latent / text / reference draws
+BLOB_MAGIC = b"FLUXDIT\0"
+BLOB_VERSION = 1
+HEADER_BYTES = 256
+ALIGN = 256
+
+
+@dataclasses.dataclass(frozen=True)
+class FluxDims:
+    n_double: int = 5
+    n_single: int = 20
+    hidden: int = 3072
+    heads: int = 24
+    head_dim: int = 128
+    mlp_hidden: int = 9216
+    in_ch: int = 128
+    txt_dim: int = 3072
+    t_freq_dim: int = 256
+    rope_theta: float = 10000.0
+    eps_ln: float = 1e-6
+    eps_rms: float = 1e-6
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One synthetic generation problem (batch 1)."""
+    name: str
+    seed: int
+    image: int            # square image side in pixels
+    n_txt: int
+    ref_image: int        # 0 = no reference image
+    n_steps: int
+    dims: FluxDims
+
+    @property
+    def grid(self) -> int:       # image tokens per side (16 px per token)
+        return self.image // 16
+
+    @property
+    def ref_grid(self) -> int:
+        return self.ref_image // 16
+
+    @property
+    def n_img(self) -> int:
+        return self.grid * self.grid
+
+    @property
+    def n_ref(self) -> int:
+        return self.ref_grid * self.ref_grid
+
+    @property
+    def n_tokens(self) -> int:
+        return self.n_txt + self.n_img + self.n_ref
+
+
+TINY_DIMS = FluxDims(n_double=1, n_single=1)
+FULL_DIMS = FluxDims()
+
+WORKLOADS = {
+    "tiny64": Workload("tiny64", 0, 64, 16, 0, 1, TINY_DIMS),
+    "t2i256": Workload("t2i256", 1, 256, 512, 0, 4, FULL_DIMS),
+    "t2i512": Workload("t2i512", 2, 512, 512, 0, 4, FULL_DIMS),
+    "t2i1024": Workload("t2i1024", 3, 1024, 512, 0, 4, FULL_DIMS),
+    "i2i1024": Workload("i2i1024", 4, 1024, 512, 1024, 4, FULL_DIMS),
+}
+
+
+def tensor_specs(d: FluxDims):
+    """Blob order: list of (name, shape, fan_in)."""
+    D, F, hd = d.hidden, d.mlp_hidden, d.head_dim
+    specs = [
+        ("time_in.w1", (D, d.t_freq_dim), d.t_freq_dim), ("time_in.b1", (D,), d.t_freq_dim),
+        ("time_in.w2", (D, D), D), ("time_in.b2", (D,), D),
+        ("img_in.w", (D, d.in_ch), d.in_ch), ("img_in.b", (D,), d.in_ch),
+        ("txt_in.w", (D, d.txt_dim), d.txt_dim), ("txt_in.b", (D,), d.txt_dim),
+    ]
+    for i in range(d.n_double):
+        for s in ("img", "txt"):
+            p = f"double.{i}.{s}."
+            specs += [
+                (p + "mod.w", (6 * D, D), D), (p + "mod.b", (6 * D,), D),
+                (p + "qkv.w", (3 * D, D), D), (p + "qkv.b", (3 * D,), D),
+                (p + "q_gain", (hd,), 1), (p + "k_gain", (hd,), 1),
+                (p + "proj.w", (D, D), D), (p + "proj.b", (D,), D),
+                (p + "mlp_in.w", (2 * F, D), D), (p + "mlp_in.b", (2 * F,), D),
+                (p + "mlp_out.w", (D, F), F), (p + "mlp_out.b", (D,), F),
+            ]
+    for i in range(d.n_single):
+        p = f"single.{i}."
+        specs += [
+            (p + "mod.w", (3 * D, D), D), (p + "mod.b", (3 * D,), D),
+            (p + "lin1.w", (3 * D + 2 * F, D), D), (p + "lin1.b", (3 * D + 2 * F,), D),
+            (p + "q_gain", (hd,), 1), (p + "k_gain", (hd,), 1),
+            (p + "lin2.w", (D, D + F), D + F), (p + "lin2.b", (D,), D + F),
+        ]
+    specs += [
+        ("final.mod.w", (2 * D, D), D), ("final.mod.b", (2 * D,), D),
+        ("final.out.w", (d.in_ch, D), D), ("final.out.b", (d.in_ch,), D),
+    ]
+    return specs
+
+
+def _align(x: int) -> int:
+    return (x + ALIGN - 1) // ALIGN * ALIGN
+
+
+def blob_layout(d: FluxDims):
+    """Byte offset (from the start of the blob) of every tensor, and total size."""
+    off = HEADER_BYTES
+    layout = []
+    for name, shape, fan_in in tensor_specs(d):
+        n = int(np.prod(shape))
+        layout.append((name, shape, fan_in, off, n))
+        off = _align(off + 2 * n)
+    return layout, off
+
+
+def round_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bit pattern (uint16), round to nearest, ties to even."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
+    return r.astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def _header(d: FluxDims, n_tensors: int, total: int) -> bytes:
+    h = BLOB_MAGIC + struct.pack(
+        "<II9i3fQQ", BLOB_VERSION, n_tensors,
+        d.n_double, d.n_single, d.hidden, d.heads, d.head_dim, d.mlp_hidden,
+        d.in_ch, d.txt_dim, d.t_freq_dim, d.rope_theta, d.eps_ln, d.eps_rms,
+        HEADER_BYTES, total - HEADER_BYTES)
+    return h + b"\0" * (HEADER_BYTES - len(h))
+
+
+def _fill(dst_u16: np.ndarray, seed: int, idx: int, chunk: int, scale: np.float32):
+    lo = chunk * CHUNK
+    hi = min(lo + CHUNK, dst_u16.size)
+    g = np.random.default_rng([seed, idx, chunk])
+    x = g.standard_normal(hi - lo, dtype=np.float32)
+    if scale != 1:
+        x *= scale
+    dst_u16[lo:hi] = round_to_bf16_bits(x)
+
+
+def make_weights(d: FluxDims, seed: int, threads: int | None = None):
+    """Return (blob: uint8 array, params: dict name -> uint16 view of bf16 bits)."""
+    layout, total = blob_layout(d)
+    blob = np.zeros(total, dtype=np.uint8)
+    blob[:HEADER_BYTES] = np.frombuffer(_header(d, len(layout), total), dtype=np.uint8)
+    params = {}
+    jobs = []
+    for idx, (name, shape, fan_in, off, n) in enumerate(layout):
+        view = blob[off:off + 2 * n].view(np.uint16)
+        params[name] = view.reshape(shape)
+        scale = np.float32(1.0 / np.sqrt(np.float32(fan_in)))
+        for c in range((n + CHUNK - 1) // CHUNK):
+            jobs.append((view, seed, idx, c, scale))
+    threads = threads or min(32, os.cpu_count() or 1)
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(lambda j: _fill(*j), jobs))
+    return blob, params
+
+
+def make_inputs(w: Workload):
+    """Latent, text and reference latent as float32 arrays holding bf16 values."""
+    def draw(k, shape):
+        g = np.random.default_rng([w.seed, INPUT_KEY + k])
+        x = g.standard_normal(int(np.prod(shape)), dtype=np.float32)
+        return bf16_bits_to_f32(round_to_bf16_bits(x)).reshape(shape)
+
+    h8 = w.image // 8
+    latent = draw(0, (32, h8, h8))
+    txt = draw(1, (w.n_txt, w.dims.txt_dim))
+    ref = None
+    if w.ref_image:
+        r8 = w.ref_image // 8
+        ref = draw(2, (32, r8, r8))
+    return latent, txt, ref
+

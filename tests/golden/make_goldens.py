@@ -1,0 +1,63 @@
+"""Write the oracle's sampled outputs for the full-size workloads to tests/golden/.
+
+Calls only ``synthetic`` (seeded inputs) and ``oracle`` (CPU definition).  For
+each workload it runs the whole Euler sampler in float32 (the precision of the
+pages' own C implementation) and stores, for a fixed set of token rows, every
+step's velocity and the final packed latent:
+
+    <workload>.npz: rows int32 [R], v float32 [S, R, 128], final float32 [R, 128]
+
+Row sets: all rows at 256^2, every 2nd at 512^2, every 8th at 1024^2.
+
+Usage: python tests/golden/make_goldens.py [workload ...]   (about an hour on 8 cores)
+"""
+import json
+import os
+import sys
+import time
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, os.path.dirname(os.path.dirname(HERE)))
+
+from synthetic import WORKLOADS, make_weights, make_inputs  # noqa: E402
+from oracle import flux_oracle as O  # noqa: E402
+
+ROW_STRIDE = {"t2i256": 1, "t2i512": 2, "t2i1024": 8, "i2i1024": 8}
+
+
+def rows_for(name):
+    w = WORKLOADS[name]
+    return np.arange(0, w.n_img, ROW_STRIDE[name], dtype=np.int32)
+
+
+def make(name):
+    w = WORKLOADS[name]
+    t0 = time.time()
+    _, p = make_weights(w.dims, w.seed)
+    lat, txt, ref = make_inputs(w)
+    rows = rows_for(name)
+    vs = []
+
+    def on_step(i, v):
+        vs.append(v[rows].float().numpy())
+        print(f"  {name} step {i} done at {time.time() - t0:.0f}s", flush=True)
+
+    with torch.no_grad():
+        final, _ = O.sample(p, O.hyper(w.dims), torch.from_numpy(lat), torch.from_numpy(txt),
+                            w.n_steps, None if ref is None else torch.from_numpy(ref),
+                            dtype=torch.float32, on_step=on_step)
+    final_tok = O.pack_latents(final)[rows].float().numpy()
+    meta = {"workload": name, "seed": w.seed, "oracle_dtype": "float32", "n_steps": w.n_steps,
+            "row_stride": ROW_STRIDE[name], "seconds": round(time.time() - t0, 1)}
+    np.savez(os.path.join(HERE, f"{name}.npz"), rows=rows, v=np.stack(vs), final=final_tok,
+             meta=np.array(json.dumps(meta)))
+    print(f"{name}: wrote {len(rows)} rows x {w.n_steps} steps in {time.time() - t0:.0f}s", flush=True)
+
+
+if __name__ == "__main__":
+    torch.set_grad_enabled(False)
+    for n in (sys.argv[1:] or list(ROW_STRIDE)):
+        make(n)
