@@ -1,0 +1,181 @@
+/*
+ * fluxdit.h -- C ABI of the B200 (sm_100a) FLUX.2-klein denoising transformer.
+ *
+ * The library evaluates the velocity field of the FLUX.2-klein image generator
+ * once per Euler flow-matching step: 5 double-stream blocks (separate text and
+ * image weights, joint attention over the concatenated sequence) and 20
+ * single-stream blocks, width 3072, 24 heads of 128 ("Flux 2 Klein: Reine
+ * C-basierte Inferenz", section "Modellarchitektur und Leistung"; hakusoku.com
+ * story 4662, section "技術詳細"), on image tokens that are 2x2 patches of a
+ * 32-channel, 8x-downsampled latent packed to 128 channels ("FLUX.3 Image Klein
+ * in Diffusers: Architektur, ...", section "Zweistufiger Transformer und
+ * Tokenisierung").
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, unless stated.
+ *     Layouts are row-major and dense.  "bf16" arrays are uint16_t bit patterns.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  Nothing synchronises the host except
+ *     flux_dit_create (blob upload) and flux_device_error.
+ *   - Return 0 on success or a negative errno-style code: FLUX_EINVAL for a bad
+ *     argument (null pointer, shape out of range), FLUX_ENOMEM when a device
+ *     allocation fails, FLUX_EIO for a CUDA launch or runtime error.  Pointer
+ *     returning calls return NULL on failure.  flux_get_error() then holds a
+ *     message for the calling thread.
+ *   - Kernels never trap: a pipeline wait that exceeds one second makes the
+ *     kernel stop, record a code in a device error word and return;
+ *     flux_device_error() reads and clears it.
+ */
+#ifndef FLUXDIT_H
+#define FLUXDIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FLUX_API __attribute__((visibility("default")))
+#else
+#define FLUX_API
+#endif
+
+#define FLUX_OK 0
+#define FLUX_EIO (-5)
+#define FLUX_ENOMEM (-12)
+#define FLUX_EINVAL (-22)
+
+typedef struct flux_dit flux_dit;
+
+/* Model hyper-parameters.  Defaults (FLUX.2-klein): 5, 20, 3072, 24, 128, 9216,
+ * 128, 3072, 256, 1e4, 1e-6, 1e-6.  hidden == heads * head_dim, head_dim == 128. */
+typedef struct {
+  int n_double, n_single, hidden, heads, head_dim, mlp_hidden, in_ch, txt_dim, t_freq_dim;
+  float rope_theta, eps_ln, eps_rms;
+} flux_dit_config;
+
+/* Last error message of the calling thread ("" if none).  Valid until the next call. */
+FLUX_API const char *flux_get_error(void);
+
+/* Bytes of a weight blob for `cfg` (header + tensors), or 0 if cfg is invalid.
+ *
+ * Blob format (little endian): a 256-byte header
+ *   char magic[8] = "FLUXDIT\0"; uint32 version = 1; uint32 n_tensors;
+ *   int32 n_double, n_single, hidden, heads, head_dim, mlp_hidden, in_ch, txt_dim, t_freq_dim;
+ *   float32 rope_theta, eps_ln, eps_rms; uint64 data_offset (= 256); uint64 data_bytes;
+ * then every tensor as bf16, row-major, each starting on a 256-byte boundary, in this order:
+ *   time_in.{w1 [D,256], b1 [D], w2 [D,D], b2 [D]}, img_in.{w [D,128], b [D]},
+ *   txt_in.{w [D,txt_dim], b [D]},
+ *   for each double block i, for stream s in (img, txt):
+ *     mod.{w [6D,D], b [6D]}        rows: shift1, scale1, gate1, shift2, scale2, gate2
+ *     qkv.{w [3D,D], b [3D]}        rows: q, k, v (head h = rows h*128 .. h*128+127)
+ *     q_gain [128], k_gain [128]    QK-RMSNorm gains
+ *     proj.{w [D,D], b [D]}
+ *     mlp_in.{w [2F,D], b [2F]}     rows: a, b of SwiGLU, silu(a) * b
+ *     mlp_out.{w [D,F], b [D]}
+ *   for each single block i:
+ *     mod.{w [3D,D], b [3D]}        rows: shift, scale, gate
+ *     lin1.{w [3D+2F,D], b}         rows: q, k, v, a, b
+ *     q_gain [128], k_gain [128]
+ *     lin2.{w [D,D+F], b [D]}       input: [attention output ; silu(a) * b]
+ *   final.mod.{w [2D,D], b [2D]}    rows: shift, scale
+ *   final.out.{w [128,D], b [128]}
+ * (D = hidden, F = mlp_hidden.) */
+FLUX_API size_t flux_blob_expected_bytes(const flux_dit_config *cfg);
+
+/* Create a model from a weight blob in HOST memory (format above).  The blob is
+ * copied to the device (and SwiGLU rows re-interleaved for the GEMM epilogue);
+ * the caller keeps ownership of `blob`.  `cfg` may be NULL (take the header's),
+ * otherwise it must equal the header's.  Synchronises `stream`.  NULL on error. */
+FLUX_API flux_dit *flux_dit_create(const void *blob, size_t blob_bytes, const flux_dit_config *cfg, void *stream);
+
+/* Release the model's device memory.  NULL is allowed. */
+FLUX_API void flux_dit_destroy(flux_dit *m);
+
+/* One transformer forward: the velocity of the image tokens at time t.
+ *   img_tok  fp32 [grid_h*grid_w, 128]    packed noisy latent tokens (flux_pack_latents)
+ *   txt      fp32 [n_txt, txt_dim]         text features
+ *   ref_tok  fp32 [ref_h*ref_w, 128] or NULL   packed reference-image tokens
+ *   v_out    fp32 [grid_h*grid_w, 128]    velocity (written)
+ * The joint sequence is text | image | reference; reference tokens use the image
+ * stream's weights, the same timestep, and RoPE coordinates (0, row, col, -1)
+ * (FLUX.3 Image Klein in Diffusers write-up, section "Modulation pro Token-Typ,
+ * Flow-Map-Destillation und 4D-RoPE"); only image tokens reach the output layer
+ * (section "Entkoppelte Vorverarbeitung und gemeinsame Attention-Blöcke").
+ * Shapes: 4 <= grid_h, grid_w <= 64 (64..1024 px in steps of 16 px, "Flux 2
+ * Klein: Reine C-basierte Inferenz", "Build und Ausführung"); ref_h = ref_w = 0
+ * or in 4..64; 0 <= n_txt <= 4096.  The first call with a larger sequence grows
+ * the model's workspace (cudaMalloc), so it must not be inside a stream capture. */
+FLUX_API int flux_dit_forward(flux_dit *m, const float *img_tok, int grid_h, int grid_w, const float *txt, int n_txt,
+                     const float *ref_tok, int ref_h, int ref_w, float t, float *v_out, void *stream);
+
+/* Diagnostic: run only the first n_double double blocks and n_single single
+ * blocks in later forwards (-1 = all).  Used to bisect parity; not a model change. */
+FLUX_API int flux_dit_set_active_blocks(flux_dit *m, int n_double, int n_single);
+
+/* The modulation vector for time t: SiLU(vec(t)) through every block's
+ * modulation linear, fp32 [flux_dit_modulation_size(m)], in blob order of the
+ * mod tensors (double i img, double i txt, ..., single i, ..., final). */
+FLUX_API size_t flux_dit_modulation_size(const flux_dit *m);
+FLUX_API int flux_dit_modulation(flux_dit *m, float t, float *mods_out, void *stream);
+
+/* Euler flow-matching update x += dt * v over n fp32 values, in place
+ * ("Flux 2 Klein: Reine C-basierte Inferenz", "Modellarchitektur und Leistung":
+ * 4 sampling steps; t_i = linspace(1, 0, S+1), dt = t_{i+1} - t_i). */
+FLUX_API int flux_euler_step(float *x, const float *v, size_t n, float dt, void *stream);
+
+/* 2x2 latent packing ("Zweistufiger Transformer und Tokenisierung"):
+ *   lat fp32 [32, h8, w8]  <->  tok fp32 [(h8/2)*(w8/2), 128],
+ *   tok[i*(w8/2)+j][c*4 + py*2 + px] = lat[c][2i+py][2j+px].  h8, w8 even, >= 2. */
+FLUX_API int flux_pack_latents(const float *lat, float *tok, int h8, int w8, void *stream);
+FLUX_API int flux_unpack_latents(const float *tok, float *lat, int h8, int w8, void *stream);
+
+/* Joint attention O = softmax(Q K^T * scale) V per head, no mask, non-causal
+ * (FLUX.3 Image Klein in Diffusers write-up, "Entkoppelte Vorverarbeitung und
+ * gemeinsame Attention-Blöcke").  q, k, v, o bf16 [n, heads, head_dim],
+ * head_dim == 128, n >= 1.  fp32 softmax statistics, bf16 P, fp32 accumulation. */
+FLUX_API int flux_joint_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, uint16_t *o, int n, int heads,
+                         int head_dim, float scale, void *stream);
+
+/* Kernel-level entry points of the forward's steps (for parity tests and reuse). */
+
+/* Linear layer on the tensor cores: acc = A W^T, A bf16 [m, k] (row stride lda
+ * elements), W bf16 [n, k] (nn.Linear layout), bias bf16 [n].  k % 64 == 0,
+ * n % 32 == 0, lda % 8 == 0.  mode:
+ *   0  out bf16 [m, ldo]: acc + bias
+ *   1  out fp32 [m, ldo]: acc + bias
+ *   2  out bf16 [m, ldo]: silu(a + bias_a) * (b + bias_b) for n/2 output columns;
+ *      W and bias rows in GEMM order: for output columns [128g, 128g+128) the
+ *      128 a-rows then the 128 matching b-rows; n % 256 == 0
+ *   3  out fp32 [m, ldo] residual: out += gate * (acc + bias), gate fp32 [n] */
+FLUX_API int flux_linear(const uint16_t *a, int m, int k, int lda, const uint16_t *w, int n, const uint16_t *bias, int mode,
+                void *out, int ldo, const float *gate, void *stream);
+
+/* y = LayerNorm(x) * (1 + scale) + shift per row (no learned affine; eps):
+ * x fp32 [rows, dim], shift/scale fp32 [dim], y bf16 [rows, dim]
+ * ("Modulation pro Token-Typ, Flow-Map-Destillation und 4D-RoPE"). */
+FLUX_API int flux_layernorm_modulate(const float *x, uint16_t *y, int rows, int dim, const float *shift, const float *scale,
+                            float eps, void *stream);
+
+/* RoPE (cos, sin) table for the joint sequence [n_txt text; gh x gw image;
+ * rh x rw reference], head_dim 128, axes (t, h, w, l) of 32 dims, frequency
+ * theta^(-2m/32): table fp32 [n, 64, 2] with n = n_txt + gh*gw + rh*rw. */
+FLUX_API int flux_rope_table(float *table, int n_txt, int gh, int gw, int rh, int rw, float theta, void *stream);
+
+/* In place on a bf16 [rows, ld] buffer: q = columns [0, heads*128), k = columns
+ * [k_col, k_col + heads*128).  Each head's 128 values are RMS-normalised and
+ * scaled by the gain (bf16 [128]), then rotated by the table (flux_rope_table). */
+FLUX_API int flux_qk_rmsnorm_rope(uint16_t *qkv, int rows, int ld, int k_col, int heads, const uint16_t *q_gain,
+                         const uint16_t *k_gain, const float *table, float eps, void *stream);
+
+/* Synchronise `stream`, then read and clear the kernels' device error words:
+ * 0 when no kernel gave up waiting, else the first nonzero code. */
+FLUX_API int flux_device_error(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLUXDIT_H */

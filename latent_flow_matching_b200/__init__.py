@@ -1,0 +1,268 @@
+"""Python binding of libfluxdit.so, the sm_100a FLUX.2-klein transformer library.
+
+Argument marshalling only: every function forwards device pointers of torch
+tensors (PyTorch owns the memory and the stream) to the C ABI declared in
+``include/fluxdit.h``.  All computation happens in the library's CUDA kernels;
+there is no CPU or PyTorch fallback.  Importing works without a GPU; calling a
+compute function without the built library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfluxdit.so")
+
+FLUX_OK, FLUX_EIO, FLUX_ENOMEM, FLUX_EINVAL = 0, -5, -12, -22
+
+EPI_BF16_BIAS, EPI_F32_BIAS, EPI_SWIGLU, EPI_RESID_GATE = 0, 1, 2, 3
+
+
+class FluxConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("n_double", "n_single", "hidden", "heads", "head_dim",
+                                            "mlp_hidden", "in_ch", "txt_dim", "t_freq_dim")] + \
+               [(n, ctypes.c_float) for n in ("rope_theta", "eps_ln", "eps_rms")]
+
+    @classmethod
+    def from_dims(cls, d):
+        return cls(*(getattr(d, f) for f, _ in cls._fields_))
+
+
+class FluxError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"fluxdit error {code}: {msg}")
+        self.code = code
+
+
+_P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_SIGS = {
+    "flux_get_error": (ctypes.c_char_p, []),
+    "flux_blob_expected_bytes": (_Z, [ctypes.POINTER(FluxConfig)]),
+    "flux_dit_create": (_P, [_P, _Z, ctypes.POINTER(FluxConfig), _P]),
+    "flux_dit_destroy": (None, [_P]),
+    "flux_dit_forward": (_I, [_P, _P, _I, _I, _P, _I, _P, _I, _I, _F, _P, _P]),
+    "flux_dit_set_active_blocks": (_I, [_P, _I, _I]),
+    "flux_dit_modulation_size": (_Z, [_P]),
+    "flux_dit_modulation": (_I, [_P, _F, _P, _P]),
+    "flux_euler_step": (_I, [_P, _P, _Z, _F, _P]),
+    "flux_pack_latents": (_I, [_P, _P, _I, _I, _P]),
+    "flux_unpack_latents": (_I, [_P, _P, _I, _I, _P]),
+    "flux_joint_attention": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P]),
+    "flux_linear": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _P]),
+    "flux_layernorm_modulate": (_I, [_P, _P, _I, _I, _P, _P, _F, _P]),
+    "flux_rope_table": (_I, [_P, _I, _I, _I, _I, _I, _F, _P]),
+    "flux_qk_rmsnorm_rope": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _F, _P]),
+    "flux_device_error": (_I, [_P]),
+}
+EXPORTED = tuple(_SIGS)
+
+_lib = None
+
+
+def lib():
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m latent_flow_matching_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def get_error() -> str:
+    return lib().flux_get_error().decode()
+
+
+def _check(rc):
+    if rc != FLUX_OK:
+        raise FluxError(rc, get_error())
+
+
+def _stream(stream):
+    if stream is not None:
+        return ctypes.c_void_p(stream if isinstance(stream, int) else stream.cuda_stream)
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t, dtype=None, what="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{what} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _bits(t, what):
+    """bf16 tensors are passed as their raw 16-bit patterns."""
+    import torch
+    if t.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
+        raise ValueError(f"{what} must be bf16")
+    return _ptr(t, None, what)
+
+
+def flux_blob_expected_bytes(dims) -> int:
+    cfg = FluxConfig.from_dims(dims)
+    return lib().flux_blob_expected_bytes(ctypes.byref(cfg))
+
+
+class FluxDiT:
+    """A model created from a weight blob (host bytes); see flux_dit_create."""
+
+    def __init__(self, blob: np.ndarray, dims=None, stream=None):
+        blob = np.ascontiguousarray(blob)
+        cfg = ctypes.byref(FluxConfig.from_dims(dims)) if dims is not None else None
+        h = lib().flux_dit_create(ctypes.c_void_p(blob.ctypes.data), blob.nbytes, cfg, _stream(stream))
+        if not h:
+            raise FluxError(FLUX_EINVAL, get_error())
+        self._h = ctypes.c_void_p(h)
+        self.dims = dims
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().flux_dit_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def forward(self, img_tok, grid_hw, txt, t, v_out, ref_tok=None, ref_hw=(0, 0), stream=None):
+        import torch
+        n_txt = 0 if txt is None else txt.shape[0]
+        _check(lib().flux_dit_forward(self._h, _ptr(img_tok, torch.float32, "img_tok"), grid_hw[0], grid_hw[1],
+                                      _ptr(txt, torch.float32, "txt"), n_txt,
+                                      _ptr(ref_tok, torch.float32, "ref_tok"), ref_hw[0], ref_hw[1],
+                                      float(t), _ptr(v_out, torch.float32, "v_out"), _stream(stream)))
+        return v_out
+
+    def set_active_blocks(self, n_double=-1, n_single=-1):
+        _check(lib().flux_dit_set_active_blocks(self._h, n_double, n_single))
+
+    def modulation_size(self) -> int:
+        return lib().flux_dit_modulation_size(self._h)
+
+    def modulation(self, t, out, stream=None):
+        import torch
+        _check(lib().flux_dit_modulation(self._h, float(t), _ptr(out, torch.float32, "mods"), _stream(stream)))
+        return out
+
+
+def euler_schedule(n_steps: int):
+    """t_0 = 1 > ... > t_S = 0 evenly spaced (float32 values)."""
+    return [float(np.float32(1.0 - i / n_steps)) for i in range(n_steps + 1)]
+
+
+def flux_euler_step(x, v, dt, stream=None):
+    import torch
+    _check(lib().flux_euler_step(_ptr(x, torch.float32, "x"), _ptr(v, torch.float32, "v"), x.numel(),
+                                 float(dt), _stream(stream)))
+    return x
+
+
+def flux_pack_latents(lat, tok, stream=None):
+    import torch
+    _check(lib().flux_pack_latents(_ptr(lat, torch.float32, "lat"), _ptr(tok, torch.float32, "tok"),
+                                   lat.shape[1], lat.shape[2], _stream(stream)))
+    return tok
+
+
+def flux_unpack_latents(tok, lat, stream=None):
+    import torch
+    _check(lib().flux_unpack_latents(_ptr(tok, torch.float32, "tok"), _ptr(lat, torch.float32, "lat"),
+                                     lat.shape[1], lat.shape[2], _stream(stream)))
+    return lat
+
+
+def flux_joint_attention(q, k, v, o, scale=None, stream=None):
+    n, heads, hd = q.shape
+    scale = hd ** -0.5 if scale is None else scale
+    _check(lib().flux_joint_attention(_bits(q, "q"), _bits(k, "k"), _bits(v, "v"), _bits(o, "o"), n, heads, hd,
+                                      float(scale), _stream(stream)))
+    return o
+
+
+def flux_linear(a, w, bias, mode, out, gate=None, stream=None):
+    import torch
+    m, k = a.shape
+    n = w.shape[0]
+    lda = a.stride(0)
+    if a.stride(1) != 1:
+        raise ValueError("a must have unit column stride")
+    _check(lib().flux_linear(ctypes.c_void_p(a.data_ptr()), m, k, lda, _bits(w, "w"), n, _bits(bias, "bias"), mode,
+                             ctypes.c_void_p(out.data_ptr()), out.stride(0),
+                             _ptr(gate, torch.float32, "gate"), _stream(stream)))
+    return out
+
+
+def flux_layernorm_modulate(x, y, shift, scale, eps=1e-6, stream=None):
+    import torch
+    rows, dim = x.shape
+    _check(lib().flux_layernorm_modulate(_ptr(x, torch.float32, "x"), _bits(y, "y"), rows, dim,
+                                         _ptr(shift, torch.float32, "shift"), _ptr(scale, torch.float32, "scale"),
+                                         float(eps), _stream(stream)))
+    return y
+
+
+def flux_rope_table(table, n_txt, grid_hw, ref_hw=(0, 0), theta=1e4, stream=None):
+    import torch
+    _check(lib().flux_rope_table(_ptr(table, torch.float32, "table"), n_txt, grid_hw[0], grid_hw[1], ref_hw[0],
+                                 ref_hw[1], float(theta), _stream(stream)))
+    return table
+
+
+def flux_qk_rmsnorm_rope(qkv, k_col, heads, q_gain, k_gain, table, eps=1e-6, stream=None):
+    import torch
+    rows, ld = qkv.shape
+    _check(lib().flux_qk_rmsnorm_rope(_bits(qkv, "qkv"), rows, ld, k_col, heads, _bits(q_gain, "q_gain"),
+                                      _bits(k_gain, "k_gain"), _ptr(table, torch.float32, "table"), float(eps),
+                                      _stream(stream)))
+    return qkv
+
+
+def flux_device_error(stream=None) -> int:
+    return lib().flux_device_error(_stream(stream))
+
+
+def flux_sample(model: FluxDiT, latent, txt, n_steps, ref_latent=None, on_step=None, stream=None):
+    """Euler sampling on the device: pack -> S x (forward, Euler) -> unpack.
+
+    latent fp32 [32, h8, w8] (device), txt fp32 [n_txt, txt_dim] (device),
+    ref_latent fp32 [32, r8, r8] or None.  Returns the final latent (new tensor).
+    ``on_step(i, v)`` sees each velocity (device tensor, reused between steps).
+    """
+    import torch
+    c, h8, w8 = latent.shape
+    gh, gw = h8 // 2, w8 // 2
+    tok = torch.empty(gh * gw, 4 * c, device=latent.device, dtype=torch.float32)
+    flux_pack_latents(latent, tok, stream)
+    ref_tok, ref_hw = None, (0, 0)
+    if ref_latent is not None:
+        rh, rw = ref_latent.shape[1] // 2, ref_latent.shape[2] // 2
+        ref_tok = torch.empty(rh * rw, 4 * c, device=latent.device, dtype=torch.float32)
+        flux_pack_latents(ref_latent, ref_tok, stream)
+        ref_hw = (rh, rw)
+    v = torch.empty_like(tok)
+    ts = euler_schedule(n_steps)
+    for i in range(n_steps):
+        model.forward(tok, (gh, gw), txt, ts[i], v, ref_tok, ref_hw, stream)
+        if on_step is not None:
+            on_step(i, v)
+        flux_euler_step(tok, v, ts[i + 1] - ts[i], stream)
+    out = torch.empty_like(latent)
+    flux_unpack_latents(tok, out, stream)
+    return out

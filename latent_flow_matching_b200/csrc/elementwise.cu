@@ -1,0 +1,355 @@
+// HBM-bound kernels of the transformer forward and the sampler:
+//   2x2 latent pack / unpack, Euler update, fp32 -> bf16 casts, LayerNorm + adaLN
+//   modulation, QK-RMSNorm + RoPE, the RoPE (cos, sin) table, the sinusoidal
+//   timestep embedding and the GEMV used for the time MLP and the modulation vectors.
+//
+// Sources: FLUX.3 Image Klein in Diffusers write-up (mindverse): "Zweistufiger
+// Transformer und Tokenisierung" (2x2 packing to 128 channels), "Entkoppelte
+// Vorverarbeitung und gemeinsame Attention-Blöcke" (QK-RMSNorm, SwiGLU),
+// "Modulation pro Token-Typ, Flow-Map-Destillation und 4D-RoPE" (LayerNorm
+// without affine, shift/scale/gate from the timestep embedding, 4-axis RoPE).
+// The Euler step x += dt * v follows the 4-step sampler of the FLUX.2-klein
+// pages ("Modellarchitektur und Leistung").
+#include <math.h>
+
+#include "common.cuh"
+#include "fluxdit_internal.h"
+
+namespace fdit {
+namespace {
+
+inline int blocks_for(size_t n, int per_block) {
+  size_t b = (n + per_block - 1) / per_block;
+  return static_cast<int>(b < 1 ? 1 : (b > 1048576 ? 1048576 : b));
+}
+
+// ------------------------------------------------------------------ pack / unpack
+// token (i, j) channel c*4 + py*2 + px  <->  lat[c, 2i+py, 2j+px]
+__global__ void pack_kernel(const float* __restrict__ lat, float* __restrict__ tok, int C, int h8, int w8) {
+  const int gw = w8 / 2;
+  const size_t total = static_cast<size_t>(h8 / 2) * gw * C;
+  for (size_t idx = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(idx % C);
+    const size_t t = idx / C;
+    const int i = static_cast<int>(t / gw), j = static_cast<int>(t % gw);
+    const float* src = lat + (static_cast<size_t>(c) * h8 + 2 * i) * w8 + 2 * j;
+    const float2 top = *reinterpret_cast<const float2*>(src);
+    const float2 bot = *reinterpret_cast<const float2*>(src + w8);
+    reinterpret_cast<float4*>(tok)[idx] = make_float4(top.x, top.y, bot.x, bot.y);
+  }
+}
+
+__global__ void unpack_kernel(const float* __restrict__ tok, float* __restrict__ lat, int C, int h8, int w8) {
+  const int gw = w8 / 2;
+  const size_t total = static_cast<size_t>(h8 / 2) * gw * C;
+  for (size_t idx = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(idx % C);
+    const size_t t = idx / C;
+    const int i = static_cast<int>(t / gw), j = static_cast<int>(t % gw);
+    const float4 v = reinterpret_cast<const float4*>(tok)[idx];
+    float* dst = lat + (static_cast<size_t>(c) * h8 + 2 * i) * w8 + 2 * j;
+    *reinterpret_cast<float2*>(dst) = make_float2(v.x, v.y);
+    *reinterpret_cast<float2*>(dst + w8) = make_float2(v.z, v.w);
+  }
+}
+
+// ------------------------------------------------------------------ Euler, casts
+__global__ void euler_kernel(float* __restrict__ x, const float* __restrict__ v, size_t n, float dt) {
+  const size_t n4 = n / 4;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4; i += stride) {
+    float4 a = reinterpret_cast<float4*>(x)[i];
+    const float4 b = reinterpret_cast<const float4*>(v)[i];
+    a.x = fmaf(dt, b.x, a.x);
+    a.y = fmaf(dt, b.y, a.y);
+    a.z = fmaf(dt, b.z, a.z);
+    a.w = fmaf(dt, b.w, a.w);
+    reinterpret_cast<float4*>(x)[i] = a;
+  }
+  for (size_t i = n4 * 4 + blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n; i += stride)
+    x[i] = fmaf(dt, v[i], x[i]);
+}
+
+__global__ void cast_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y, size_t n) {
+  const size_t n4 = n / 4;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4; i += stride) {
+    const float4 a = reinterpret_cast<const float4*>(x)[i];
+    reinterpret_cast<uint2*>(y)[i] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+  }
+  for (size_t i = n4 * 4 + blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n; i += stride)
+    y[i] = __float2bfloat16_rn(x[i]);
+}
+
+// ------------------------------------------------------------------ LayerNorm + adaLN modulation
+// One warp per row; the row stays in registers (V float4 per lane, dim = 128 V).
+template <int V>
+__global__ void __launch_bounds__(256) ln_mod_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y,
+                                                     int rows, int split, const float* __restrict__ sh0,
+                                                     const float* __restrict__ sc0, const float* __restrict__ sh1,
+                                                     const float* __restrict__ sc1, float eps) {
+  constexpr int dim = 128 * V;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(warp) * dim);
+  float4 v[V];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    v[i] = __ldcs(xr + i * 32 + lane);
+    s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float mean = s * (1.0f / dim);
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const float a = v[i].x - mean, b = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
+    q += (a * a + b * b) + (c * c + d * d);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+  const float rstd = rsqrtf(q * (1.0f / dim) + eps);
+  const float4* shp = reinterpret_cast<const float4*>(warp < split ? sh0 : sh1);
+  const float4* scp = reinterpret_cast<const float4*>(warp < split ? sc0 : sc1);
+  uint2* yr = reinterpret_cast<uint2*>(y + static_cast<size_t>(warp) * dim);
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const float4 sh = __ldg(shp + i * 32 + lane), sc = __ldg(scp + i * 32 + lane);
+    const float a = (v[i].x - mean) * rstd * (1.f + sc.x) + sh.x;
+    const float b = (v[i].y - mean) * rstd * (1.f + sc.y) + sh.y;
+    const float c = (v[i].z - mean) * rstd * (1.f + sc.z) + sh.z;
+    const float d = (v[i].w - mean) * rstd * (1.f + sc.w) + sh.w;
+    yr[i * 32 + lane] = make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
+  }
+}
+
+// Any dim that is a multiple of 4: three passes over the row in global memory.
+__global__ void ln_mod_generic_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y, int rows, int dim,
+                                      int split, const float* __restrict__ sh0, const float* __restrict__ sc0,
+                                      const float* __restrict__ sh1, const float* __restrict__ sc1, float eps) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const float* xr = x + static_cast<size_t>(warp) * dim;
+  float s = 0.f;
+  for (int i = lane; i < dim; i += 32) s += xr[i];
+  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float mean = s / dim;
+  float q = 0.f;
+  for (int i = lane; i < dim; i += 32) q += (xr[i] - mean) * (xr[i] - mean);
+  for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+  const float rstd = rsqrtf(q / dim + eps);
+  const float* sh = warp < split ? sh0 : sh1;
+  const float* sc = warp < split ? sc0 : sc1;
+  for (int i = lane; i < dim; i += 32)
+    y[static_cast<size_t>(warp) * dim + i] = __float2bfloat16_rn((xr[i] - mean) * rstd * (1.f + sc[i]) + sh[i]);
+}
+
+// ------------------------------------------------------------------ QK-RMSNorm + RoPE (head_dim 128)
+// One warp per (row, q or k); a half-warp per head, 8 dims (4 rotation pairs) per lane.
+__global__ void __launch_bounds__(256) qk_norm_rope_kernel(__nv_bfloat16* __restrict__ qkv, int rows, int ld, int kcol,
+                                                           int heads, int split, const __nv_bfloat16* __restrict__ gq0,
+                                                           const __nv_bfloat16* __restrict__ gk0,
+                                                           const __nv_bfloat16* __restrict__ gq1,
+                                                           const __nv_bfloat16* __restrict__ gk1,
+                                                           const float2* __restrict__ rope, float eps) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int row = gw >> 1;
+  const int which = gw & 1;                       // 0: q, 1: k
+  if (row >= rows) return;
+  const int hl = lane & 15;                       // dims [8 hl, 8 hl + 8)
+  const int hsub = lane >> 4;                     // which head of the pair
+  const __nv_bfloat16* gain = which == 0 ? (row < split ? gq0 : gq1) : (row < split ? gk0 : gk1);
+  const uint4 g4 = __ldg(reinterpret_cast<const uint4*>(gain) + hl);
+  const float g[8] = {bf16lo(g4.x), bf16hi(g4.x), bf16lo(g4.y), bf16hi(g4.y),
+                      bf16lo(g4.z), bf16hi(g4.z), bf16lo(g4.w), bf16hi(g4.w)};
+  const float4* rp = reinterpret_cast<const float4*>(rope + static_cast<size_t>(row) * 64 + 4 * hl);
+  const float4 r01 = __ldg(rp), r23 = __ldg(rp + 1);
+  const float cs[4] = {r01.x, r01.z, r23.x, r23.z};
+  const float sn[4] = {r01.y, r01.w, r23.y, r23.w};
+  __nv_bfloat16* base = qkv + static_cast<size_t>(row) * ld + (which ? kcol : 0);
+  for (int h = hsub; h < heads; h += 2) {
+    uint4* p = reinterpret_cast<uint4*>(base + h * 128) + hl;
+    const uint4 w = *p;
+    float x[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
+                  bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
+#pragma unroll
+    for (int o = 8; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float r = rsqrtf(ss * (1.0f / 128.0f) + eps);
+    uint32_t out[4];
+#pragma unroll
+    for (int pr = 0; pr < 4; ++pr) {
+      const float a = x[2 * pr] * r * g[2 * pr];
+      const float b = x[2 * pr + 1] * r * g[2 * pr + 1];
+      out[pr] = pack_bf16x2(a * cs[pr] - b * sn[pr], a * sn[pr] + b * cs[pr]);
+    }
+    *p = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+// (cos, sin) of pos_axis * theta^(-2m/32) for the 64 pairs of a 128-dim head, axes (t, h, w, l).
+// text i: (0,0,0,i); image (r,c): (0,r,c,0); reference (r,c): (0,r,c,-1).
+__global__ void rope_table_kernel(float2* __restrict__ table, int n_txt, int gh, int gw, int rh, int rw,
+                                  float theta) {
+  const int n = n_txt + gh * gw + rh * rw;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n * 64) return;
+  const int row = idx >> 6, pr = idx & 63;
+  const int axis = pr >> 4, m = pr & 15;
+  double pos[4] = {0.0, 0.0, 0.0, 0.0};
+  if (row < n_txt) {
+    pos[3] = row;
+  } else if (row < n_txt + gh * gw) {
+    const int t = row - n_txt;
+    pos[1] = t / gw;
+    pos[2] = t % gw;
+  } else {
+    const int t = row - n_txt - gh * gw;
+    pos[1] = t / rw;
+    pos[2] = t % rw;
+    pos[3] = -1.0;
+  }
+  const double ang = pos[axis] * pow(static_cast<double>(theta), -2.0 * m / 32.0);
+  double s, c;
+  sincos(ang, &s, &c);
+  table[idx] = make_float2(static_cast<float>(c), static_cast<float>(s));
+}
+
+// ------------------------------------------------------------------ timestep embedding, GEMV
+__global__ void timestep_embed_kernel(float* __restrict__ out, float t, int dim) {
+  const int half = dim / 2;
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= half) return;
+  const double f = exp(-log(10000.0) * j / half);
+  const double a = static_cast<double>(t) * 1000.0 * f;
+  double s, c;
+  sincos(a, &s, &c);
+  out[j] = static_cast<float>(c);
+  out[half + j] = static_cast<float>(s);
+}
+
+constexpr int kGemvRowsPerWarp = 4;
+constexpr int kGemvWarps = 8;
+
+__global__ void __launch_bounds__(256) gemv_kernel(const __nv_bfloat16* __restrict__ W,
+                                                   const __nv_bfloat16* __restrict__ b, const float* __restrict__ x,
+                                                   float* __restrict__ y, int rows, int k, int silu_in,
+                                                   int silu_out) {
+  extern __shared__ float xs[];
+  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+    const float v = x[i];
+    xs[i] = silu_in ? silu_f(v) : v;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunks = k / 8;
+  for (int r0 = (blockIdx.x * kGemvWarps + warp) * kGemvRowsPerWarp; r0 < rows;
+       r0 += gridDim.x * kGemvWarps * kGemvRowsPerWarp) {
+    float acc[kGemvRowsPerWarp] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int c = lane; c < chunks; c += 32) {
+      const float4 x0 = reinterpret_cast<const float4*>(xs)[2 * c];
+      const float4 x1 = reinterpret_cast<const float4*>(xs)[2 * c + 1];
+#pragma unroll
+      for (int rr = 0; rr < kGemvRowsPerWarp; ++rr) {
+        if (r0 + rr < rows) {
+          const uint4 w = __ldcs(reinterpret_cast<const uint4*>(W + static_cast<size_t>(r0 + rr) * k) + c);
+          acc[rr] += bf16lo(w.x) * x0.x + bf16hi(w.x) * x0.y + bf16lo(w.y) * x0.z + bf16hi(w.y) * x0.w +
+                     bf16lo(w.z) * x1.x + bf16hi(w.z) * x1.y + bf16lo(w.w) * x1.z + bf16hi(w.w) * x1.w;
+        }
+      }
+    }
+#pragma unroll
+    for (int rr = 0; rr < kGemvRowsPerWarp; ++rr) {
+      float a = acc[rr];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (lane == 0 && r0 + rr < rows) {
+        a += __bfloat162float(b[r0 + rr]);
+        y[r0 + rr] = silu_out ? silu_f(a) : a;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t pack_latents_launch(const float* lat, float* tok, int c, int h8, int w8, cudaStream_t s) {
+  const size_t total = static_cast<size_t>(h8 / 2) * (w8 / 2) * c;
+  pack_kernel<<<blocks_for(total, 256), 256, 0, s>>>(lat, tok, c, h8, w8);
+  return cudaGetLastError();
+}
+
+cudaError_t unpack_latents_launch(const float* tok, float* lat, int c, int h8, int w8, cudaStream_t s) {
+  const size_t total = static_cast<size_t>(h8 / 2) * (w8 / 2) * c;
+  unpack_kernel<<<blocks_for(total, 256), 256, 0, s>>>(tok, lat, c, h8, w8);
+  return cudaGetLastError();
+}
+
+cudaError_t euler_launch(float* x, const float* v, size_t n, float dt, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  euler_kernel<<<blocks_for((n + 3) / 4, 256), 256, 0, s>>>(x, v, n, dt);
+  return cudaGetLastError();
+}
+
+cudaError_t cast_bf16_launch(const float* x, __nv_bfloat16* y, size_t n, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  cast_bf16_kernel<<<blocks_for((n + 3) / 4, 256), 256, 0, s>>>(x, y, n);
+  return cudaGetLastError();
+}
+
+cudaError_t ln_modulate_launch(const float* x, __nv_bfloat16* y, int rows, int dim, int split, const float* shift0,
+                               const float* scale0, const float* shift1, const float* scale1, float eps,
+                               cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  const int grid = (rows + 7) / 8;
+  if (dim == 3072)
+    ln_mod_kernel<24><<<grid, 256, 0, s>>>(x, y, rows, split, shift0, scale0, shift1, scale1, eps);
+  else
+    ln_mod_generic_kernel<<<grid, 256, 0, s>>>(x, y, rows, dim, split, shift0, scale0, shift1, scale1, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t qk_norm_rope_launch(__nv_bfloat16* qkv, int rows, int ld, int kcol, int heads, int split,
+                                const __nv_bfloat16* gq0, const __nv_bfloat16* gk0, const __nv_bfloat16* gq1,
+                                const __nv_bfloat16* gk1, const float2* rope, float eps, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  const int warps = rows * 2;
+  qk_norm_rope_kernel<<<(warps + 7) / 8, 256, 0, s>>>(qkv, rows, ld, kcol, heads, split, gq0, gk0, gq1, gk1, rope,
+                                                      eps);
+  return cudaGetLastError();
+}
+
+cudaError_t rope_table_launch(float2* table, int n_txt, int gh, int gw, int rh, int rw, float theta, cudaStream_t s) {
+  const int n = n_txt + gh * gw + rh * rw;
+  if (n <= 0) return cudaSuccess;
+  rope_table_kernel<<<(n * 64 + 255) / 256, 256, 0, s>>>(table, n_txt, gh, gw, rh, rw, theta);
+  return cudaGetLastError();
+}
+
+cudaError_t timestep_embed_launch(float* temb, float t, int dim, cudaStream_t s) {
+  timestep_embed_kernel<<<(dim / 2 + 127) / 128, 128, 0, s>>>(temb, t, dim);
+  return cudaGetLastError();
+}
+
+cudaError_t gemv_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, const float* x, float* y, int rows, int k,
+                        int silu_in, int silu_out, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  const int per_block = kGemvWarps * kGemvRowsPerWarp;
+  int grid = (rows + per_block - 1) / per_block;
+  const int cap = num_sms_current() * 8;
+  if (grid > cap) grid = cap;
+  gemv_kernel<<<grid, 256, k * sizeof(float), s>>>(W, b, x, y, rows, k, silu_in, silu_out);
+  return cudaGetLastError();
+}
+
+}  // namespace fdit

@@ -1,0 +1,696 @@
+// C ABI of the FLUX.2-klein denoising transformer on B200 and the host-side
+// runner that enqueues one forward as a sequence of sm_100a kernels.
+//
+// Forward (one CUDA stream, no host synchronisation):
+//   timestep embedding -> time MLP -> every block's modulation (one GEMV)
+//   img_in / txt_in projections (grouped tcgen05 GEMM) into the fp32 residual X
+//   5 x double block: LN+mod -> qkv GEMM (text | image problems) -> QK-RMSNorm+RoPE
+//                     -> joint attention -> proj GEMM + gate*residual -> LN+mod
+//                     -> SwiGLU GEMM -> out GEMM + gate*residual
+//   20 x single block: LN+mod -> fused linear1 GEMM (qkv | SwiGLU problems)
+//                     -> QK-RMSNorm+RoPE -> joint attention -> linear2 GEMM + gate*residual
+//   final LN+mod on the image rows -> output GEMM -> velocity (fp32)
+// Block structure: "Flux 2 Klein: Reine C-basierte Inferenz" ("Modellarchitektur
+// und Leistung") and the FLUX.3 Image Klein in Diffusers write-up ("Entkoppelte
+// Vorverarbeitung und gemeinsame Attention-Blöcke", "Modulation pro Token-Typ,
+// Flow-Map-Destillation und 4D-RoPE").
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/fluxdit.h"
+#include "fluxdit_internal.h"
+
+using bf16 = __nv_bfloat16;
+
+namespace fdit {
+
+// ------------------------------------------------------------------ errors
+static thread_local std::string g_error;
+
+static int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_error = buf;
+  return code;
+}
+
+#define FD_CUDA(expr)                                                                          \
+  do {                                                                                         \
+    cudaError_t e_ = (expr);                                                                   \
+    if (e_ != cudaSuccess) return fail(FLUX_EIO, "%s: %s", #expr, cudaGetErrorString(e_));     \
+  } while (0)
+
+// ------------------------------------------------------------------ tensor maps
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+static std::once_flag g_encode_once;
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
+                    uint32_t box_rows) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode || rows == 0 || cols == 0) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms_current() {
+  int dev = 0, n = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+// ------------------------------------------------------------------ blob layout
+struct BlobTensor {
+  std::string name;
+  size_t rows, cols;        // cols = 1 for vectors
+  size_t blob_off;          // byte offset in the blob
+};
+
+static bool valid_cfg(const flux_dit_config& c) {
+  return c.n_double >= 0 && c.n_single >= 0 && c.n_double + c.n_single >= 1 && c.head_dim == 128 &&
+         c.heads >= 1 && c.hidden == c.heads * c.head_dim && c.mlp_hidden > 0 && c.mlp_hidden % 128 == 0 &&
+         c.in_ch == 128 && c.txt_dim > 0 && c.txt_dim % 64 == 0 && c.t_freq_dim > 0 && c.t_freq_dim % 64 == 0 &&
+         c.rope_theta > 0 && c.eps_ln > 0 && c.eps_rms > 0;
+}
+
+// Tensor order of the blob (documented in fluxdit.h).
+static std::vector<BlobTensor> blob_tensors(const flux_dit_config& c, size_t* total) {
+  const size_t D = c.hidden, F = c.mlp_hidden, hd = c.head_dim;
+  std::vector<BlobTensor> t;
+  auto add = [&](const std::string& n, size_t r, size_t k) { t.push_back({n, r, k, 0}); };
+  add("time_in.w1", D, c.t_freq_dim); add("time_in.b1", D, 1);
+  add("time_in.w2", D, D); add("time_in.b2", D, 1);
+  add("img_in.w", D, c.in_ch); add("img_in.b", D, 1);
+  add("txt_in.w", D, c.txt_dim); add("txt_in.b", D, 1);
+  for (int i = 0; i < c.n_double; ++i)
+    for (const char* s : {"img", "txt"}) {
+      const std::string p = "double." + std::to_string(i) + "." + s + ".";
+      add(p + "mod.w", 6 * D, D); add(p + "mod.b", 6 * D, 1);
+      add(p + "qkv.w", 3 * D, D); add(p + "qkv.b", 3 * D, 1);
+      add(p + "q_gain", hd, 1); add(p + "k_gain", hd, 1);
+      add(p + "proj.w", D, D); add(p + "proj.b", D, 1);
+      add(p + "mlp_in.w", 2 * F, D); add(p + "mlp_in.b", 2 * F, 1);
+      add(p + "mlp_out.w", D, F); add(p + "mlp_out.b", D, 1);
+    }
+  for (int i = 0; i < c.n_single; ++i) {
+    const std::string p = "single." + std::to_string(i) + ".";
+    add(p + "mod.w", 3 * D, D); add(p + "mod.b", 3 * D, 1);
+    add(p + "lin1.w", 3 * D + 2 * F, D); add(p + "lin1.b", 3 * D + 2 * F, 1);
+    add(p + "q_gain", hd, 1); add(p + "k_gain", hd, 1);
+    add(p + "lin2.w", D, D + F); add(p + "lin2.b", D, 1);
+  }
+  add("final.mod.w", 2 * D, D); add("final.mod.b", 2 * D, 1);
+  add("final.out.w", c.in_ch, D); add("final.out.b", c.in_ch, 1);
+  size_t off = 256;
+  for (auto& x : t) {
+    x.blob_off = off;
+    off = (off + x.rows * x.cols * 2 + 255) / 256 * 256;
+  }
+  *total = off;
+  return t;
+}
+
+struct BlobHeader {
+  char magic[8];
+  uint32_t version, n_tensors;
+  int32_t n_double, n_single, hidden, heads, head_dim, mlp_hidden, in_ch, txt_dim, t_freq_dim;
+  float rope_theta, eps_ln, eps_rms;
+  uint64_t data_offset, data_bytes;
+};
+static_assert(sizeof(BlobHeader) == 80, "blob header layout");
+
+// ------------------------------------------------------------------ model
+struct StreamW {                       // one stream of a double block
+  const bf16 *qkv_b, *q_gain, *k_gain, *proj_b, *mlp_in_b, *mlp_out_b;
+  size_t mod_off;                      // into the modulation vector (floats)
+  CUtensorMap m_qkv, m_proj, m_mlp_in, m_mlp_out;
+};
+struct SingleW {
+  const bf16 *qkv_b, *mlp_b, *q_gain, *k_gain, *lin2_b;
+  size_t mod_off;
+  CUtensorMap m_qkv, m_mlp, m_lin2;
+};
+
+struct Workspace {
+  size_t cap_n = 0, cap_tok = 0, cap_txt = 0;
+  float* X = nullptr;
+  bf16 *Y = nullptr, *QKV = nullptr, *CC = nullptr, *tokb = nullptr, *txtb = nullptr;
+  float2* rope = nullptr;
+  int nt = -1, gh = -1, gw = -1, rh = -1, rw = -1;     // shape the maps and the RoPE table were built for
+  CUtensorMap a_txtb, a_tokb, a_Ytxt, a_Yimg, a_Yall, a_Yout, a_Otxt, a_Oimg, a_Htxt, a_Himg, a_CC, qkv;
+};
+
+}  // namespace fdit
+
+struct flux_dit {
+  flux_dit_config cfg;
+  int device = 0, num_sms = 148;
+  void* wbuf = nullptr;                // every tensor except the modulation linears
+  bf16* mods_w = nullptr;              // all modulation weights, rows concatenated
+  bf16* mods_b = nullptr;
+  size_t mods_rows = 0;
+  float *temb = nullptr, *th = nullptr, *vec = nullptr, *mods = nullptr;
+  const bf16 *t_w1, *t_b1, *t_w2, *t_b2, *img_b, *txt_b, *fin_b;
+  size_t fin_mod_off = 0;
+  CUtensorMap m_img_in, m_txt_in, m_fin;
+  std::vector<fdit::StreamW> dbl;      // [2 * i + 0] image stream, [2 * i + 1] text stream of block i
+  std::vector<fdit::SingleW> sgl;
+  int act_double = 0, act_single = 0;
+  fdit::Workspace ws;
+};
+
+namespace fdit {
+
+static void free_ws(Workspace& w) {
+  cudaFree(w.X); cudaFree(w.Y); cudaFree(w.QKV); cudaFree(w.CC); cudaFree(w.tokb); cudaFree(w.txtb);
+  cudaFree(w.rope);
+  w = Workspace();
+}
+
+static void destroy(flux_dit* m) {
+  if (!m) return;
+  free_ws(m->ws);
+  cudaFree(m->wbuf); cudaFree(m->mods_w); cudaFree(m->mods_b);
+  cudaFree(m->temb); cudaFree(m->th); cudaFree(m->vec); cudaFree(m->mods);
+  delete m;
+}
+
+// Host -> device copy of SwiGLU rows [a (F rows); b (F rows)] of width `row_bytes`
+// into the GEMM order: for each group of 128 output columns, its 128 a-rows then its 128 b-rows.
+static cudaError_t copy_swiglu(void* dst, const uint8_t* src, size_t F, size_t row_bytes, cudaStream_t s) {
+  const size_t chunk = 128 * row_bytes;
+  const size_t groups = F / 128;
+  cudaError_t e = cudaMemcpy2DAsync(dst, 2 * chunk, src, chunk, chunk, groups, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return e;
+  return cudaMemcpy2DAsync(static_cast<uint8_t*>(dst) + chunk, 2 * chunk, src + F * row_bytes, chunk, chunk, groups,
+                           cudaMemcpyHostToDevice, s);
+}
+
+static int create_impl(const void* blob, size_t blob_bytes, const flux_dit_config* cfg_in, cudaStream_t s,
+                       flux_dit** out) {
+  *out = nullptr;
+  if (!blob || blob_bytes < sizeof(BlobHeader)) return fail(FLUX_EINVAL, "blob is NULL or too small");
+  BlobHeader h;
+  memcpy(&h, blob, sizeof(h));
+  if (memcmp(h.magic, "FLUXDIT\0", 8) != 0 || h.version != 1 || h.data_offset != 256)
+    return fail(FLUX_EINVAL, "not a FLUXDIT v1 blob");
+  flux_dit_config c = {h.n_double, h.n_single, h.hidden, h.heads, h.head_dim, h.mlp_hidden,
+                       h.in_ch, h.txt_dim, h.t_freq_dim, h.rope_theta, h.eps_ln, h.eps_rms};
+  if (cfg_in && memcmp(cfg_in, &c, sizeof(c)) != 0) return fail(FLUX_EINVAL, "config differs from the blob header");
+  if (!valid_cfg(c)) return fail(FLUX_EINVAL, "unsupported model config in blob header");
+  size_t total = 0;
+  const std::vector<BlobTensor> ts = blob_tensors(c, &total);
+  if (h.n_tensors != ts.size() || h.data_bytes + 256 != total || blob_bytes < total)
+    return fail(FLUX_EINVAL, "blob size / tensor count mismatch (expected %zu bytes, %zu tensors)", total, ts.size());
+
+  flux_dit* m = new flux_dit();
+  m->cfg = c;
+  cudaGetDevice(&m->device);
+  m->num_sms = num_sms_current();
+  const size_t D = c.hidden, F = c.mlp_hidden;
+  const uint8_t* b8 = static_cast<const uint8_t*>(blob);
+
+  // device layout: non-modulation tensors packed in blob order; modulation rows concatenated
+  std::vector<size_t> dev_off(ts.size(), SIZE_MAX);
+  size_t wbytes = 0, mrows = 0;
+  for (size_t i = 0; i < ts.size(); ++i) {
+    const std::string& n = ts[i].name;
+    const bool is_mod = n.size() > 5 && (n.compare(n.size() - 5, 5, "mod.w") == 0 || n.compare(n.size() - 5, 5, "mod.b") == 0);
+    if (is_mod) {
+      if (n.back() == 'w') mrows += ts[i].rows;
+      continue;
+    }
+    dev_off[i] = wbytes;
+    wbytes = (wbytes + ts[i].rows * ts[i].cols * 2 + 255) / 256 * 256;
+  }
+  m->mods_rows = mrows;
+  auto cleanup = [&](int code, const char* what) {
+    destroy(m);
+    return fail(code, "%s", what);
+  };
+  if (cudaMalloc(&m->wbuf, wbytes) != cudaSuccess || cudaMalloc(&m->mods_w, mrows * D * 2) != cudaSuccess ||
+      cudaMalloc(&m->mods_b, mrows * 2) != cudaSuccess || cudaMalloc(&m->temb, c.t_freq_dim * 4) != cudaSuccess ||
+      cudaMalloc(&m->th, D * 4) != cudaSuccess || cudaMalloc(&m->vec, D * 4) != cudaSuccess ||
+      cudaMalloc(&m->mods, mrows * 4) != cudaSuccess)
+    return cleanup(FLUX_ENOMEM, "cudaMalloc of model weights failed");
+
+  uint8_t* wb = static_cast<uint8_t*>(m->wbuf);
+  size_t mrow = 0;
+  std::vector<size_t> mod_row(ts.size(), 0);
+  for (size_t i = 0; i < ts.size(); ++i) {
+    const BlobTensor& t = ts[i];
+    const uint8_t* src = b8 + t.blob_off;
+    const size_t bytes = t.rows * t.cols * 2;
+    cudaError_t e = cudaSuccess;
+    if (dev_off[i] == SIZE_MAX) {
+      if (t.name.back() == 'w') {
+        mod_row[i] = mrow;
+        e = cudaMemcpyAsync(m->mods_w + mrow * D, src, bytes, cudaMemcpyHostToDevice, s);
+      } else {
+        mod_row[i] = mrow;                                   // bias follows its weight
+        e = cudaMemcpyAsync(m->mods_b + mrow, src, bytes, cudaMemcpyHostToDevice, s);
+        mrow += t.rows;
+      }
+    } else {
+      uint8_t* dst = wb + dev_off[i];
+      const std::string& n = t.name;
+      const bool mlp_in = n.find("mlp_in.") != std::string::npos;
+      const bool lin1 = n.find("lin1.") != std::string::npos;
+      if (mlp_in) {
+        e = copy_swiglu(dst, src, F, t.cols * 2, s);
+      } else if (lin1) {
+        const size_t qkv_bytes = 3 * D * t.cols * 2;
+        e = cudaMemcpyAsync(dst, src, qkv_bytes, cudaMemcpyHostToDevice, s);
+        if (e == cudaSuccess) e = copy_swiglu(dst + qkv_bytes, src + qkv_bytes, F, t.cols * 2, s);
+      } else {
+        e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, s);
+      }
+    }
+    if (e != cudaSuccess) return cleanup(FLUX_EIO, "weight upload failed");
+  }
+
+  auto find = [&](const std::string& n) -> size_t {
+    for (size_t i = 0; i < ts.size(); ++i)
+      if (ts[i].name == n) return i;
+    return SIZE_MAX;
+  };
+  auto W = [&](const std::string& n) { return reinterpret_cast<const bf16*>(wb + dev_off[find(n)]); };
+  auto MOD = [&](const std::string& n) { return mod_row[find(n)]; };
+  bool maps_ok = true;
+  auto wmap = [&](CUtensorMap* map, const bf16* base, size_t rows, size_t cols, uint32_t box) {
+    maps_ok &= make_tmap_bf16(map, base, rows, cols, cols * 2, box);
+  };
+
+  m->t_w1 = W("time_in.w1"); m->t_b1 = W("time_in.b1");
+  m->t_w2 = W("time_in.w2"); m->t_b2 = W("time_in.b2");
+  m->img_b = W("img_in.b"); m->txt_b = W("txt_in.b"); m->fin_b = W("final.out.b");
+  wmap(&m->m_img_in, W("img_in.w"), D, c.in_ch, 256);
+  wmap(&m->m_txt_in, W("txt_in.w"), D, c.txt_dim, 256);
+  wmap(&m->m_fin, W("final.out.w"), c.in_ch, D, 128);
+  m->fin_mod_off = MOD("final.mod.w");
+  m->dbl.resize(2 * c.n_double);
+  for (int i = 0; i < c.n_double; ++i)
+    for (int sidx = 0; sidx < 2; ++sidx) {
+      const std::string p = "double." + std::to_string(i) + (sidx == 0 ? ".img." : ".txt.");
+      StreamW& sw = m->dbl[2 * i + sidx];
+      sw.qkv_b = W(p + "qkv.b"); sw.q_gain = W(p + "q_gain"); sw.k_gain = W(p + "k_gain");
+      sw.proj_b = W(p + "proj.b"); sw.mlp_in_b = W(p + "mlp_in.b"); sw.mlp_out_b = W(p + "mlp_out.b");
+      sw.mod_off = MOD(p + "mod.w");
+      wmap(&sw.m_qkv, W(p + "qkv.w"), 3 * D, D, 256);
+      wmap(&sw.m_proj, W(p + "proj.w"), D, D, 256);
+      wmap(&sw.m_mlp_in, W(p + "mlp_in.w"), 2 * F, D, 256);
+      wmap(&sw.m_mlp_out, W(p + "mlp_out.w"), D, F, 256);
+    }
+  m->sgl.resize(c.n_single);
+  for (int i = 0; i < c.n_single; ++i) {
+    const std::string p = "single." + std::to_string(i) + ".";
+    SingleW& sw = m->sgl[i];
+    const bf16* l1 = W(p + "lin1.w");
+    const bf16* l1b = W(p + "lin1.b");
+    sw.qkv_b = l1b; sw.mlp_b = l1b + 3 * D;
+    sw.q_gain = W(p + "q_gain"); sw.k_gain = W(p + "k_gain"); sw.lin2_b = W(p + "lin2.b");
+    sw.mod_off = MOD(p + "mod.w");
+    wmap(&sw.m_qkv, l1, 3 * D, D, 256);
+    wmap(&sw.m_mlp, l1 + 3 * D * D, 2 * F, D, 256);
+    wmap(&sw.m_lin2, W(p + "lin2.w"), D, D + F, 256);
+  }
+  if (!maps_ok) return cleanup(FLUX_EIO, "cuTensorMapEncodeTiled failed for a weight tensor");
+  m->act_double = c.n_double;
+  m->act_single = c.n_single;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return cleanup(FLUX_EIO, "weight upload failed (sync)");
+  *out = m;
+  return FLUX_OK;
+}
+
+template <typename T>
+static cudaError_t grow(T** p, size_t* cap, size_t need) {
+  if (need <= *cap) return cudaSuccess;
+  cudaFree(*p);
+  *p = nullptr;
+  *cap = 0;
+  cudaError_t e = cudaMalloc(p, need * sizeof(T));
+  if (e == cudaSuccess) *cap = need;
+  return e;
+}
+
+static int prepare_shape(flux_dit* m, int nt, int gh, int gw, int rh, int rw, cudaStream_t s) {
+  Workspace& w = m->ws;
+  const flux_dit_config& c = m->cfg;
+  const size_t D = c.hidden, F = c.mlp_hidden;
+  const size_t ni = static_cast<size_t>(gh) * gw, nr = static_cast<size_t>(rh) * rw;
+  const size_t n = nt + ni + nr;
+  if (n > w.cap_n) {
+    size_t cap = 0;
+    float* X = nullptr;
+    free_ws(w);
+    const size_t need = n;
+    bool ok = cudaMalloc(&X, need * D * 4) == cudaSuccess;
+    w.X = X;
+    ok = ok && cudaMalloc(&w.Y, need * D * 2) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.QKV, need * 3 * D * 2) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.CC, need * (D + F) * 2) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.rope, need * 64 * sizeof(float2)) == cudaSuccess;
+    if (!ok) {
+      free_ws(w);
+      return fail(FLUX_ENOMEM, "workspace allocation for %zu tokens failed", need);
+    }
+    (void)cap;
+    w.cap_n = need;
+  }
+  if (grow(&w.tokb, &w.cap_tok, (ni + nr) * c.in_ch) != cudaSuccess ||
+      grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt, 1) * c.txt_dim) != cudaSuccess)
+    return fail(FLUX_ENOMEM, "workspace allocation failed");
+  if (w.nt == nt && w.gh == gh && w.gw == gw && w.rh == rh && w.rw == rw) return FLUX_OK;
+
+  const size_t nimg = ni + nr;
+  const uint64_t ldD = D * 2, ldC = (D + F) * 2;
+  bool ok = true;
+  auto amap = [&](CUtensorMap* map, const void* base, size_t rows, size_t cols, uint64_t stride, uint32_t box) {
+    if (rows == 0) {
+      memset(map, 0, sizeof(*map));
+      return;
+    }
+    ok &= make_tmap_bf16(map, base, rows, cols, stride, box);
+  };
+  amap(&w.a_txtb, w.txtb, nt, c.txt_dim, c.txt_dim * 2, 128);
+  amap(&w.a_tokb, w.tokb, nimg, c.in_ch, c.in_ch * 2, 128);
+  amap(&w.a_Ytxt, w.Y, nt, D, ldD, 128);
+  amap(&w.a_Yimg, w.Y + nt * D, nimg, D, ldD, 128);
+  amap(&w.a_Yall, w.Y, n, D, ldD, 128);
+  amap(&w.a_Yout, w.Y, ni, D, ldD, 128);
+  amap(&w.a_Otxt, w.CC, nt, D, ldC, 128);
+  amap(&w.a_Oimg, w.CC + nt * (D + F), nimg, D, ldC, 128);
+  amap(&w.a_Htxt, w.CC + D, nt, F, ldC, 128);
+  amap(&w.a_Himg, w.CC + nt * (D + F) + D, nimg, F, ldC, 128);
+  amap(&w.a_CC, w.CC, n, D + F, ldC, 128);
+  amap(&w.qkv, w.QKV, n, 3 * D, 3 * D * 2, 128);
+  if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an activation buffer");
+  if (rope_table_launch(w.rope, nt, gh, gw, rh, rw, c.rope_theta, s) != cudaSuccess)
+    return fail(FLUX_EIO, "rope table launch failed");
+  w.nt = nt; w.gh = gh; w.gw = gw; w.rh = rh; w.rw = rw;
+  return FLUX_OK;
+}
+
+static void problem(GemmParams& P, int i, const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, int mode,
+                    void* out, int ldo, const bf16* bias, const float* gate) {
+  P.mapA[i] = a;
+  P.mapB[i] = b;
+  GemmProblem& pr = P.prob[i];
+  pr = GemmProblem();
+  pr.M = M; pr.N = N; pr.K = K; pr.mode = mode; pr.out = out; pr.ldo = ldo; pr.bias = bias; pr.gate = gate;
+}
+
+static int run_modulation(flux_dit* m, float t, cudaStream_t s) {
+  const flux_dit_config& c = m->cfg;
+  const int D = c.hidden;
+  FD_CUDA(timestep_embed_launch(m->temb, t, c.t_freq_dim, s));
+  FD_CUDA(gemv_launch(m->t_w1, m->t_b1, m->temb, m->th, D, c.t_freq_dim, 0, 1, s));
+  FD_CUDA(gemv_launch(m->t_w2, m->t_b2, m->th, m->vec, D, D, 0, 0, s));
+  FD_CUDA(gemv_launch(m->mods_w, m->mods_b, m->vec, m->mods, static_cast<int>(m->mods_rows), D, 1, 0, s));
+  return FLUX_OK;
+}
+
+static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const float* txt, int nt,
+                        const float* ref_tok, int rh, int rw, float t, float* v_out, cudaStream_t s) {
+  const flux_dit_config& c = m->cfg;
+  const int D = c.hidden, F = c.mlp_hidden, H = c.heads;
+  if (!img_tok || !v_out) return fail(FLUX_EINVAL, "img_tok and v_out must be device pointers");
+  if (gh < 4 || gh > 64 || gw < 4 || gw > 64) return fail(FLUX_EINVAL, "image grid %dx%d outside 4..64", gh, gw);
+  if (nt < 0 || nt > 4096 || (nt > 0 && !txt)) return fail(FLUX_EINVAL, "bad text (n_txt=%d)", nt);
+  if (!((rh == 0 && rw == 0) || (rh >= 4 && rh <= 64 && rw >= 4 && rw <= 64)))
+    return fail(FLUX_EINVAL, "reference grid %dx%d outside 4..64", rh, rw);
+  if (rh > 0 && !ref_tok) return fail(FLUX_EINVAL, "ref_tok is NULL for a %dx%d reference", rh, rw);
+  if (!std::isfinite(t)) return fail(FLUX_EINVAL, "t is not finite");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != m->device) return fail(FLUX_EINVAL, "model lives on device %d, current device is %d", m->device, dev);
+
+  int rc = prepare_shape(m, nt, gh, gw, rh, rw, s);
+  if (rc) return rc;
+  Workspace& w = m->ws;
+  const int ni = gh * gw, nr = rh * rw, nimg = ni + nr, n = nt + nimg;
+  const float eps_ln = c.eps_ln, eps_rms = c.eps_rms;
+  const float* mods = m->mods;
+
+  rc = run_modulation(m, t, s);
+  if (rc) return rc;
+  FD_CUDA(cast_bf16_launch(img_tok, w.tokb, static_cast<size_t>(ni) * c.in_ch, s));
+  if (nr) FD_CUDA(cast_bf16_launch(ref_tok, w.tokb + static_cast<size_t>(ni) * c.in_ch, static_cast<size_t>(nr) * c.in_ch, s));
+  if (nt) FD_CUDA(cast_bf16_launch(txt, w.txtb, static_cast<size_t>(nt) * c.txt_dim, s));
+
+  GemmParams P;
+  P.num_problems = 2;
+  problem(P, 0, w.a_txtb, m->m_txt_in, nt, D, c.txt_dim, kEpiF32Bias, w.X, D, m->txt_b, nullptr);
+  problem(P, 1, w.a_tokb, m->m_img_in, nimg, D, c.in_ch, kEpiF32Bias, w.X + static_cast<size_t>(nt) * D, D, m->img_b,
+          nullptr);
+  FD_CUDA(gemm_launch(P, 256, m->num_sms, s));
+
+  float* Ximg = w.X + static_cast<size_t>(nt) * D;
+  bf16* Otxt = w.CC;
+  bf16* Oimg = w.CC + static_cast<size_t>(nt) * (D + F);
+  AttnParams A;
+  A.mapQ = w.qkv; A.mapK = w.qkv; A.mapV = w.qkv;
+  A.out = w.CC; A.ldo = D + F; A.n = n; A.heads = H;
+  A.q_col0 = 0; A.k_col0 = D; A.v_col0 = 2 * D;
+  A.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
+
+  for (int i = 0; i < m->act_double; ++i) {
+    const StreamW& si = m->dbl[2 * i];
+    const StreamW& st = m->dbl[2 * i + 1];
+    const float* mi = mods + si.mod_off;          // shift1, scale1, gate1, shift2, scale2, gate2
+    const float* mt = mods + st.mod_off;
+    FD_CUDA(ln_modulate_launch(w.X, w.Y, n, D, nt, mt, mt + D, mi, mi + D, eps_ln, s));
+    P.num_problems = 2;
+    problem(P, 0, w.a_Ytxt, st.m_qkv, nt, 3 * D, D, kEpiBf16Bias, w.QKV, 3 * D, st.qkv_b, nullptr);
+    problem(P, 1, w.a_Yimg, si.m_qkv, nimg, 3 * D, D, kEpiBf16Bias, w.QKV + static_cast<size_t>(nt) * 3 * D, 3 * D,
+            si.qkv_b, nullptr);
+    FD_CUDA(gemm_launch(P, 256, m->num_sms, s));
+    FD_CUDA(qk_norm_rope_launch(w.QKV, n, 3 * D, D, H, nt, st.q_gain, st.k_gain, si.q_gain, si.k_gain, w.rope,
+                                eps_rms, s));
+    FD_CUDA(attention_launch(A, s));
+    P.num_problems = 2;
+    problem(P, 0, w.a_Otxt, st.m_proj, nt, D, D, kEpiResidGate, w.X, D, st.proj_b, mt + 2 * D);
+    problem(P, 1, w.a_Oimg, si.m_proj, nimg, D, D, kEpiResidGate, Ximg, D, si.proj_b, mi + 2 * D);
+    FD_CUDA(gemm_launch(P, 256, m->num_sms, s));
+    FD_CUDA(ln_modulate_launch(w.X, w.Y, n, D, nt, mt + 3 * D, mt + 4 * D, mi + 3 * D, mi + 4 * D, eps_ln, s));
+    P.num_problems = 2;
+    problem(P, 0, w.a_Ytxt, st.m_mlp_in, nt, 2 * F, D, kEpiSwiGLU, Otxt + D, D + F, st.mlp_in_b, nullptr);
+    problem(P, 1, w.a_Yimg, si.m_mlp_in, nimg, 2 * F, D, kEpiSwiGLU, Oimg + D, D + F, si.mlp_in_b, nullptr);
+    FD_CUDA(gemm_launch(P, 256, m->num_sms, s));
+    P.num_problems = 2;
+    problem(P, 0, w.a_Htxt, st.m_mlp_out, nt, D, F, kEpiResidGate, w.X, D, st.mlp_out_b, mt + 5 * D);
+    problem(P, 1, w.a_Himg, si.m_mlp_out, nimg, D, F, kEpiResidGate, Ximg, D, si.mlp_out_b, mi + 5 * D);
+    FD_CUDA(gemm_launch(P, 256, m->num_sms, s));
+  }
+  for (int i = 0; i < m->act_single; ++i) {
+    const SingleW& sw = m->sgl[i];
+    const float* ms = mods + sw.mod_off;          // shift, scale, gate
+    FD_CUDA(ln_modulate_launch(w.X, w.Y, n, D, n, ms, ms + D, ms, ms + D, eps_ln, s));
+    P.num_problems = 2;
+    problem(P, 0, w.a_Yall, sw.m_qkv, n, 3 * D, D, kEpiBf16Bias, w.QKV, 3 * D, sw.qkv_b, nullptr);
+    problem(P, 1, w.a_Yall, sw.m_mlp, n, 2 * F, D, kEpiSwiGLU, w.CC + D, D + F, sw.mlp_b, nullptr);
+    FD_CUDA(gemm_launch(P, 256, m->num_sms, s));
+    FD_CUDA(qk_norm_rope_launch(w.QKV, n, 3 * D, D, H, n, sw.q_gain, sw.k_gain, sw.q_gain, sw.k_gain, w.rope, eps_rms,
+                                s));
+    FD_CUDA(attention_launch(A, s));
+    P.num_problems = 1;
+    problem(P, 0, w.a_CC, sw.m_lin2, n, D, D + F, kEpiResidGate, w.X, D, sw.lin2_b, ms + 2 * D);
+    FD_CUDA(gemm_launch(P, 256, m->num_sms, s));
+  }
+  const float* mf = mods + m->fin_mod_off;         // shift, scale
+  FD_CUDA(ln_modulate_launch(Ximg, w.Y, ni, D, ni, mf, mf + D, mf, mf + D, eps_ln, s));
+  P.num_problems = 1;
+  problem(P, 0, w.a_Yout, m->m_fin, ni, c.in_ch, D, kEpiF32Bias, v_out, c.in_ch, m->fin_b, nullptr);
+  FD_CUDA(gemm_launch(P, 128, m->num_sms, s));
+  return FLUX_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace fdit
+
+using namespace fdit;
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* flux_get_error(void) { return g_error.c_str(); }
+
+size_t flux_blob_expected_bytes(const flux_dit_config* cfg) {
+  if (!cfg || !valid_cfg(*cfg)) return 0;
+  size_t total = 0;
+  blob_tensors(*cfg, &total);
+  return total;
+}
+
+flux_dit* flux_dit_create(const void* blob, size_t blob_bytes, const flux_dit_config* cfg, void* stream) {
+  flux_dit* m = nullptr;
+  create_impl(blob, blob_bytes, cfg, static_cast<cudaStream_t>(stream), &m);
+  return m;
+}
+
+void flux_dit_destroy(flux_dit* m) { destroy(m); }
+
+int flux_dit_forward(flux_dit* m, const float* img_tok, int grid_h, int grid_w, const float* txt, int n_txt,
+                     const float* ref_tok, int ref_h, int ref_w, float t, float* v_out, void* stream) {
+  if (!m) return fail(FLUX_EINVAL, "model is NULL");
+  return forward_impl(m, img_tok, grid_h, grid_w, txt, n_txt, ref_tok, ref_h, ref_w, t, v_out,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int flux_dit_set_active_blocks(flux_dit* m, int n_double, int n_single) {
+  if (!m) return fail(FLUX_EINVAL, "model is NULL");
+  m->act_double = n_double < 0 ? m->cfg.n_double : std::min(n_double, m->cfg.n_double);
+  m->act_single = n_single < 0 ? m->cfg.n_single : std::min(n_single, m->cfg.n_single);
+  return FLUX_OK;
+}
+
+size_t flux_dit_modulation_size(const flux_dit* m) { return m ? m->mods_rows : 0; }
+
+int flux_dit_modulation(flux_dit* m, float t, float* mods_out, void* stream) {
+  if (!m || !mods_out) return fail(FLUX_EINVAL, "NULL argument");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int rc = run_modulation(m, t, s);
+  if (rc) return rc;
+  FD_CUDA(cudaMemcpyAsync(mods_out, m->mods, m->mods_rows * sizeof(float), cudaMemcpyDeviceToDevice, s));
+  return FLUX_OK;
+}
+
+int flux_euler_step(float* x, const float* v, size_t n, float dt, void* stream) {
+  if (n && (!x || !v)) return fail(FLUX_EINVAL, "NULL argument");
+  if (!aligned16(x) || !aligned16(v)) return fail(FLUX_EINVAL, "x and v must be 16-byte aligned");
+  FD_CUDA(euler_launch(x, v, n, dt, static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_pack_latents(const float* lat, float* tok, int h8, int w8, void* stream) {
+  if (!lat || !tok) return fail(FLUX_EINVAL, "NULL argument");
+  if (h8 < 2 || w8 < 2 || h8 % 2 || w8 % 2) return fail(FLUX_EINVAL, "latent %dx%d must be even and >= 2", h8, w8);
+  if (!aligned16(lat) || !aligned16(tok)) return fail(FLUX_EINVAL, "lat and tok must be 16-byte aligned");
+  FD_CUDA(pack_latents_launch(lat, tok, 32, h8, w8, static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_unpack_latents(const float* tok, float* lat, int h8, int w8, void* stream) {
+  if (!lat || !tok) return fail(FLUX_EINVAL, "NULL argument");
+  if (h8 < 2 || w8 < 2 || h8 % 2 || w8 % 2) return fail(FLUX_EINVAL, "latent %dx%d must be even and >= 2", h8, w8);
+  if (!aligned16(lat) || !aligned16(tok)) return fail(FLUX_EINVAL, "lat and tok must be 16-byte aligned");
+  FD_CUDA(unpack_latents_launch(tok, lat, 32, h8, w8, static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_joint_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o, int n, int heads,
+                         int head_dim, float scale, void* stream) {
+  if (!q || !k || !v || !o) return fail(FLUX_EINVAL, "NULL argument");
+  if (head_dim != 128) return fail(FLUX_EINVAL, "head_dim must be 128 (got %d)", head_dim);
+  if (n < 1 || heads < 1 || heads > 1024) return fail(FLUX_EINVAL, "bad n=%d heads=%d", n, heads);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(FLUX_EINVAL, "q, k, v, o must be 16-byte aligned");
+  if (!(scale > 0) || !std::isfinite(scale)) return fail(FLUX_EINVAL, "scale must be positive");
+  AttnParams A;
+  const uint64_t ld = static_cast<uint64_t>(heads) * 128;
+  if (!make_tmap_bf16(&A.mapQ, q, n, ld, ld * 2, 128) || !make_tmap_bf16(&A.mapK, k, n, ld, ld * 2, 128) ||
+      !make_tmap_bf16(&A.mapV, v, n, ld, ld * 2, 128))
+    return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed");
+  A.out = reinterpret_cast<bf16*>(o);
+  A.ldo = static_cast<int>(ld);
+  A.n = n;
+  A.heads = heads;
+  A.q_col0 = A.k_col0 = A.v_col0 = 0;
+  A.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
+  FD_CUDA(attention_launch(A, static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_linear(const uint16_t* a, int m, int k, int lda, const uint16_t* w, int n, const uint16_t* bias, int mode,
+                void* out, int ldo, const float* gate, void* stream) {
+  if (!a || !w || !bias || !out) return fail(FLUX_EINVAL, "NULL argument");
+  if (m < 1 || k < 64 || k % 64 || n < 32 || n % 32 || lda < k || lda % 8)
+    return fail(FLUX_EINVAL, "bad shape m=%d k=%d n=%d lda=%d", m, k, n, lda);
+  if (mode < 0 || mode > 3) return fail(FLUX_EINVAL, "bad mode %d", mode);
+  if (mode == kEpiSwiGLU && n % 256) return fail(FLUX_EINVAL, "SwiGLU mode needs n %% 256 == 0");
+  if (mode == kEpiResidGate && !gate) return fail(FLUX_EINVAL, "gate is NULL");
+  const int out_cols = mode == kEpiSwiGLU ? n / 2 : n;
+  if (ldo < out_cols || ldo % 8) return fail(FLUX_EINVAL, "bad ldo=%d", ldo);
+  if (!aligned16(a) || !aligned16(w) || !aligned16(bias) || !aligned16(out) || (gate && !aligned16(gate)))
+    return fail(FLUX_EINVAL, "pointers must be 16-byte aligned");
+  const int bn = mode == kEpiSwiGLU ? 256 : gemm_bn_for(n);
+  GemmParams P;
+  P.num_problems = 1;
+  if (!make_tmap_bf16(&P.mapA[0], a, m, k, static_cast<uint64_t>(lda) * 2, 128) ||
+      !make_tmap_bf16(&P.mapB[0], w, n, k, static_cast<uint64_t>(k) * 2, bn))
+    return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed");
+  GemmProblem& pr = P.prob[0];
+  pr = GemmProblem();
+  pr.M = m; pr.N = n; pr.K = k; pr.mode = mode; pr.out = out; pr.ldo = ldo;
+  pr.bias = reinterpret_cast<const bf16*>(bias);
+  pr.gate = gate;
+  FD_CUDA(gemm_launch(P, bn, num_sms_current(), static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_layernorm_modulate(const float* x, uint16_t* y, int rows, int dim, const float* shift, const float* scale,
+                            float eps, void* stream) {
+  if (!x || !y || !shift || !scale) return fail(FLUX_EINVAL, "NULL argument");
+  if (rows < 0 || dim < 4 || dim % 4) return fail(FLUX_EINVAL, "bad shape rows=%d dim=%d", rows, dim);
+  if (!aligned16(x) || !aligned16(y) || !aligned16(shift) || !aligned16(scale))
+    return fail(FLUX_EINVAL, "pointers must be 16-byte aligned");
+  FD_CUDA(ln_modulate_launch(x, reinterpret_cast<bf16*>(y), rows, dim, rows, shift, scale, shift, scale, eps,
+                             static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_rope_table(float* table, int n_txt, int gh, int gw, int rh, int rw, float theta, void* stream) {
+  if (!table) return fail(FLUX_EINVAL, "NULL argument");
+  if (n_txt < 0 || gh < 0 || gw < 0 || rh < 0 || rw < 0 || !(theta > 0))
+    return fail(FLUX_EINVAL, "bad arguments");
+  FD_CUDA(rope_table_launch(reinterpret_cast<float2*>(table), n_txt, gh, gw, rh, rw, theta,
+                            static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_qk_rmsnorm_rope(uint16_t* qkv, int rows, int ld, int k_col, int heads, const uint16_t* q_gain,
+                         const uint16_t* k_gain, const float* table, float eps, void* stream) {
+  if (!qkv || !q_gain || !k_gain || !table) return fail(FLUX_EINVAL, "NULL argument");
+  if (rows < 0 || heads < 1 || ld % 8 || k_col % 8 || ld < heads * 128 || k_col + heads * 128 > ld)
+    return fail(FLUX_EINVAL, "bad shape rows=%d ld=%d k_col=%d heads=%d", rows, ld, k_col, heads);
+  if (!aligned16(qkv) || !aligned16(q_gain) || !aligned16(k_gain) || !aligned16(table))
+    return fail(FLUX_EINVAL, "pointers must be 16-byte aligned");
+  const bf16* gq = reinterpret_cast<const bf16*>(q_gain);
+  const bf16* gk = reinterpret_cast<const bf16*>(k_gain);
+  FD_CUDA(qk_norm_rope_launch(reinterpret_cast<bf16*>(qkv), rows, ld, k_col, heads, rows, gq, gk, gq, gk,
+                              reinterpret_cast<const float2*>(table), eps, static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_device_error(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FD_CUDA(cudaStreamSynchronize(s));
+  const int g = gemm_read_device_error(s);
+  const int a = attention_read_device_error(s);
+  return g ? g : a;
+}
+
+}  // extern "C"

@@ -1,0 +1,86 @@
+// Internal interfaces between the kernel files and the C-ABI layer (not exported).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace fdit {
+
+// ------------------------------------------------------------------ GEMM
+enum EpiMode : int { kEpiBf16Bias = 0, kEpiF32Bias = 1, kEpiSwiGLU = 2, kEpiResidGate = 3 };
+constexpr int kMaxProblems = 4;
+
+struct GemmProblem {
+  int M, N, K;                    // out rows, W rows, reduction (K % 64 == 0, N % 32 == 0)
+  int mode;                       // EpiMode
+  int ldo;                        // leading dimension of out, elements
+  int tiles_m, tiles_n, tile_begin;   // filled by gemm_launch
+  void* out;                      // bf16 or f32 (see mode); kEpiResidGate: the f32 residual
+  const __nv_bfloat16* bias;      // [N]
+  const float* gate;              // [N], kEpiResidGate only
+};
+
+struct GemmParams {
+  CUtensorMap mapA[kMaxProblems];     // activations [M, K], box {64, 128}
+  CUtensorMap mapB[kMaxProblems];     // weights [N, K], box {64, BN}
+  GemmProblem prob[kMaxProblems];
+  int num_problems;
+  int total_tiles;
+};
+
+int gemm_bn_for(int n);
+cudaError_t gemm_launch(GemmParams& P, int bn, int num_sms, cudaStream_t stream);
+int gemm_read_device_error(cudaStream_t stream);
+
+// ------------------------------------------------------------------ attention
+struct AttnParams {
+  CUtensorMap mapQ, mapK, mapV;   // 2D bf16 [rows = n, cols], box {64, 128}, 128B swizzle
+  __nv_bfloat16* out;             // O row i, head h at out + i*ldo + h*128
+  int ldo;
+  int n, heads;
+  int q_col0, k_col0, v_col0;     // column of head 0's first element in each map
+  float scale_log2;               // softmax scale * log2(e)
+};
+cudaError_t attention_launch(const AttnParams& P, cudaStream_t stream);
+int attention_read_device_error(cudaStream_t stream);
+
+// ------------------------------------------------------------------ HBM-bound kernels
+cudaError_t pack_latents_launch(const float* lat, float* tok, int c, int h8, int w8, cudaStream_t s);
+cudaError_t unpack_latents_launch(const float* tok, float* lat, int c, int h8, int w8, cudaStream_t s);
+cudaError_t euler_launch(float* x, const float* v, size_t n, float dt, cudaStream_t s);
+cudaError_t cast_bf16_launch(const float* x, __nv_bfloat16* y, size_t n, cudaStream_t s);
+
+// y[r, :] = LN(x[r, :]) * (1 + scale) + shift; rows r < split use (shift0, scale0), others (shift1, scale1)
+cudaError_t ln_modulate_launch(const float* x, __nv_bfloat16* y, int rows, int dim, int split,
+                               const float* shift0, const float* scale0, const float* shift1,
+                               const float* scale1, float eps, cudaStream_t s);
+
+// In place on q (columns [0, heads*hd)) and k (columns [kcol, kcol + heads*hd)) of a [rows, ld] bf16 buffer:
+// RMSNorm over each head's hd values with gain (rows < split: gq0/gk0, else gq1/gk1), then RoPE from
+// the [rows, hd/2] float2 (cos, sin) table.
+cudaError_t qk_norm_rope_launch(__nv_bfloat16* qkv, int rows, int ld, int kcol, int heads, int split,
+                                const __nv_bfloat16* gq0, const __nv_bfloat16* gk0,
+                                const __nv_bfloat16* gq1, const __nv_bfloat16* gk1,
+                                const float2* rope, float eps, cudaStream_t s);
+
+// (cos, sin) table for the joint sequence [text; image grid; reference grid], head_dim 128, 4 axes.
+cudaError_t rope_table_launch(float2* table, int n_txt, int gh, int gw, int rh, int rw, float theta,
+                              cudaStream_t s);
+
+// temb[j] = cos(t*1000*f_j), temb[128+j] = sin(...), f_j = 1e4^(-j/128)
+cudaError_t timestep_embed_launch(float* temb, float t, int dim, cudaStream_t s);
+
+// y[r] = act_out(sum_k W[r,k] * act_in(x[k]) + b[r]); W bf16 [rows, k], b bf16 [rows]
+cudaError_t gemv_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, const float* x, float* y, int rows,
+                        int k, int silu_in, int silu_out, cudaStream_t s);
+
+// ------------------------------------------------------------------ host helpers
+// 2D bf16 tensor map: rows x cols, row stride in bytes, box {64 cols, box_rows}, 128B swizzle.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
+                    uint32_t box_rows);
+int num_sms_current();
+
+}  // namespace fdit

@@ -1,0 +1,135 @@
+"""Host-side checks of the C ABI: the library loads, exports what the header declares,
+agrees with the blob generator on sizes, and rejects bad arguments with error codes.
+None of these tests launches a kernel, so they run without a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import latent_flow_matching_b200 as F
+from latent_flow_matching_b200 import build as fbuild
+from synthetic import FluxDims, FULL_DIMS, TINY_DIMS, blob_layout
+from synthetic.flux_inputs import HEADER_BYTES
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fluxdit.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    fbuild.build()
+    return F.lib()
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"FLUX_API\s+[\w\s\*]*?\b(flux_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for required in ("flux_dit_create", "flux_dit_destroy", "flux_dit_forward", "flux_euler_step",
+                     "flux_pack_latents", "flux_unpack_latents", "flux_joint_attention", "flux_get_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", F.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (flux_\w+)", out))
+    assert set(declared_symbols()) <= exported
+    assert set(F.EXPORTED) == set(declared_symbols())
+
+
+@pytest.mark.parametrize("dims", [FULL_DIMS, TINY_DIMS,
+                                  FluxDims(n_double=2, n_single=3, hidden=256, heads=2, mlp_hidden=512,
+                                           txt_dim=192, t_freq_dim=256)])
+def test_blob_size_matches_generator(L, dims):
+    _, total = blob_layout(dims)
+    assert F.flux_blob_expected_bytes(dims) == total
+
+
+def test_full_model_parameter_count():
+    layout, total = blob_layout(FULL_DIMS)
+    n = sum(e[4] for e in layout)
+    assert 4.8e9 < n < 4.9e9           # 5 double + 20 single blocks at width 3072
+    assert total - HEADER_BYTES >= 2 * n
+
+
+def test_invalid_config_gives_zero(L):
+    bad = FluxDims(head_dim=64, hidden=64 * 24)
+    assert F.flux_blob_expected_bytes(bad) == 0
+
+
+def _tiny_blob():
+    dims = FluxDims(n_double=1, n_single=1, hidden=256, heads=2, mlp_hidden=256, txt_dim=128)
+    _, total = blob_layout(dims)
+    from synthetic.flux_inputs import _header
+    from synthetic import tensor_specs
+    blob = np.zeros(total, np.uint8)
+    blob[:HEADER_BYTES] = np.frombuffer(_header(dims, len(tensor_specs(dims)), total), np.uint8)
+    return dims, blob
+
+
+def test_create_rejects_corrupt_blob(L):
+    dims, blob = _tiny_blob()
+    bad = blob.copy()
+    bad[0] = ord("X")
+    h = L.flux_dit_create(ctypes.c_void_p(bad.ctypes.data), bad.nbytes, None, None)
+    assert not h
+    assert "FLUXDIT" in F.get_error()
+    h = L.flux_dit_create(ctypes.c_void_p(blob.ctypes.data), blob.nbytes - 256, None, None)
+    assert not h
+    assert "size" in F.get_error()
+    h = L.flux_dit_create(None, 0, None, None)
+    assert not h
+
+
+def test_create_rejects_config_mismatch(L):
+    dims, blob = _tiny_blob()
+    other = F.FluxConfig.from_dims(FluxDims(n_double=2, n_single=1, hidden=256, heads=2, mlp_hidden=256,
+                                            txt_dim=128))
+    h = L.flux_dit_create(ctypes.c_void_p(blob.ctypes.data), blob.nbytes, ctypes.byref(other), None)
+    assert not h
+    assert "config" in F.get_error()
+
+
+def test_entry_points_reject_bad_arguments(L):
+    p = ctypes.c_void_p(16)            # never dereferenced: validation fails first
+    assert L.flux_pack_latents(None, p, 8, 8, None) == F.FLUX_EINVAL
+    assert L.flux_pack_latents(p, p, 7, 8, None) == F.FLUX_EINVAL
+    assert "even" in F.get_error()
+    assert L.flux_unpack_latents(p, p, 8, 0, None) == F.FLUX_EINVAL
+    assert L.flux_joint_attention(p, p, p, p, 10, 2, 64, 0.1, None) == F.FLUX_EINVAL
+    assert "head_dim" in F.get_error()
+    assert L.flux_joint_attention(p, p, p, p, 0, 2, 128, 0.1, None) == F.FLUX_EINVAL
+    assert L.flux_linear(p, 10, 100, 100, p, 64, p, 0, p, 64, None, None) == F.FLUX_EINVAL   # k % 64
+    assert L.flux_linear(p, 10, 128, 128, p, 128, p, 2, p, 64, None, None) == F.FLUX_EINVAL  # swiglu n % 256
+    assert L.flux_linear(p, 10, 128, 128, p, 128, p, 3, p, 128, None, None) == F.FLUX_EINVAL  # gate missing
+    assert L.flux_linear(p, 10, 128, 128, p, 128, p, 9, p, 128, None, None) == F.FLUX_EINVAL
+    assert L.flux_layernorm_modulate(p, p, 4, 3, p, p, 1e-6, None) == F.FLUX_EINVAL
+    assert L.flux_qk_rmsnorm_rope(p, 4, 100, 0, 1, p, p, p, 1e-6, None) == F.FLUX_EINVAL
+    assert L.flux_dit_forward(None, p, 8, 8, p, 4, None, 0, 0, 1.0, p, None) == F.FLUX_EINVAL
+    assert L.flux_dit_set_active_blocks(None, 1, 1) == F.FLUX_EINVAL
+    assert L.flux_dit_modulation_size(None) == 0
+    L.flux_dit_destroy(None)
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(4, 4)
+    with pytest.raises(ValueError):
+        F._ptr(x, torch.float32, "x")
+
+
+def test_product_path_does_not_reference_the_oracle():
+    pkg = os.path.join(ROOT, "latent_flow_matching_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert "oracle" not in src, f
