@@ -1,0 +1,390 @@
+#!/usr/bin/env python
+"""Benchmark of the FLUX.2-klein denoising-transformer step on B200.
+
+One step = one sampling step of the 1024x1024 text-to-image workload (4096
+image + 512 text tokens, 5 double + 20 single blocks, width 3072, 24 heads):
+pack the latent -> transformer forward -> Euler update -> unpack, all through
+the library's C ABI on one CUDA stream.  Prints one JSON line (rank 0):
+
+  value     ms per DiT forward (whole job: max-over-ranks time / forwards of all ranks)
+  e2e       the same through host buffers (H2D of latent + text, D2H of the latent, per step)
+  roofline  the tcgen05 GEMM (most of the FLOPs) from CUDA events around its launches
+  cpu_baseline   the CPU oracle on a bounded sample (rank 0, one GPU only)
+
+``--impl reference`` times the CPU oracle instead (rank 0 only).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: torchrun --nproc-per-node N bench.py --gpus N  (independent replicas, no data-path collective)
+"""
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synthetic import WORKLOADS, make_weights, make_inputs  # noqa: E402
+
+METRIC = "ms per DiT forward & TFLOP/s at 1024^2 (4096+512 tok), % of BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_BF16_TFLOPS = 2250.0
+
+
+def forward_flops(w):
+    """Algorithmic FLOPs of one forward: dense linears + non-causal attention (QK^T and PV)."""
+    d = w.dims
+    D, F_, C = d.hidden, d.mlp_hidden, d.in_ch
+    n = w.n_tokens
+    per_block = n * 2.0 * D * (4 * D + 3 * F_) + 4.0 * n * n * D
+    total = (d.n_double + d.n_single) * per_block
+    total += 2.0 * (w.n_img + w.n_ref) * C * D + 2.0 * w.n_txt * d.txt_dim * D + 2.0 * w.n_img * D * C
+    return total
+
+
+def single_block_flops(w):
+    d, n = w.dims, w.n_tokens
+    return n * 2.0 * d.hidden * (4 * d.hidden + 3 * d.mlp_hidden) + 4.0 * n * n * d.hidden
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return {k: float(j[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"fluxdit_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- helpers
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def profile_traffic(kernel_file):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel source."""
+    src = os.path.join(ROOT, "latent_flow_matching_b200", "csrc", kernel_file)
+    prof = os.path.join(ROOT, "profiles", "gemm_tc_t2i1024.md")
+    if not (os.path.exists(src) and os.path.exists(prof)):
+        return None, None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    text = open(prof).read()
+    m_sha = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"dram_bytes_per_gflop:\s*([0-9.eE+]+)", text)
+    if not (m_sha and m_tr) or m_sha.group(1) != sha:
+        return None, sha
+    return float(m_tr.group(1)), sha
+
+
+def cpu_oracle_sample(w, params, lat, txt, ref):
+    """Oracle time of one double and one single block at full size (fp32, host cores), scaled to a forward."""
+    from oracle import flux_oracle as O
+    torch.set_grad_enabled(False)
+    hp = O.hyper(w.dims)
+    D = w.dims.hidden
+    g = torch.Generator().manual_seed(0)
+    x_txt = torch.randn(w.n_txt, D, generator=g)
+    x_img = torch.randn(w.n_img + w.n_ref, D, generator=g)
+    s = torch.randn(D, generator=g)
+    ang = O.rope_angles(O.token_positions(w.n_txt, w.grid, w.grid, w.ref_grid, w.ref_grid), 128, 1e4).float()
+    t0 = time.perf_counter()
+    O.double_block(params, 0, x_txt, x_img, s, ang, hp, torch.float32)
+    t1 = time.perf_counter()
+    O.single_block(params, 0, torch.cat([x_txt, x_img]), s, ang, hp, torch.float32)
+    t2 = time.perf_counter()
+    ms = 1e3 * (w.dims.n_double * (t1 - t0) + w.dims.n_single * (t2 - t1))
+    return ms, t2 - t0
+
+
+# ---------------------------------------------------------------------------- reference arm (CPU oracle)
+def run_reference(args, w):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    from oracle import flux_oracle as O
+    torch.set_grad_enabled(False)
+    _, params = make_weights(w.dims, w.seed)
+    hp = O.hyper(w.dims)
+    D = w.dims.hidden
+    g = torch.Generator().manual_seed(0)
+    x = torch.randn(w.n_tokens, D, generator=g)
+    s = torch.randn(D, generator=g)
+    ang = O.rope_angles(O.token_positions(w.n_txt, w.grid, w.grid, w.ref_grid, w.ref_grid), 128, 1e4).float()
+    scale = forward_flops(w) / single_block_flops(w)
+    for _ in range(args.warmup):
+        O.single_block(params, 0, x, s, ang, hp, torch.float32)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        O.single_block(params, 0, x, s, ang, hp, torch.float32)
+        times.append(time.perf_counter() - t0)
+    ms_block = 1e3 * sum(times) / len(times)
+    value = ms_block * scale
+    sample = (f"one single-stream block at the full {w.name} size ({w.n_tokens} tokens) per step, fp32 oracle; "
+              f"value scaled by forward FLOPs / block FLOPs = {scale:.2f}")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "ms/forward",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_block, 3),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded N(0,1) bf16-rounded weights and inputs)",
+        "config": {"workload": f"{w.name}: {w.image}x{w.image} text-to-image, {w.n_img} image + {w.n_txt} text "
+                               f"tokens, 5 double + 20 single blocks, width 3072", "seq_len": w.n_tokens,
+                   "global_batch": 1, "parallelism": "CPU oracle on rank 0"},
+        "tflops": round(forward_flops(w) / (value / 1e3) / 1e12, 4),
+        "cpu_baseline": {"value": round(value, 3), "unit": "ms/forward", "cores": torch.get_num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "ms/forward", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------- our arm
+def run_ours(args, w):
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    import latent_flow_matching_b200 as F
+    F.lib()                                         # fails loudly if the library is missing
+    torch.set_grad_enabled(False)
+
+    blob, params = make_weights(w.dims, w.seed)
+    lat_h, txt_h, ref_h = make_inputs(w)
+    model = F.FluxDiT(blob, w.dims)
+    stream = torch.cuda.current_stream()
+    dev = torch.device("cuda", local)
+    lat0 = torch.from_numpy(lat_h).to(dev)
+    lat = lat0.clone()
+    txt = torch.from_numpy(txt_h).to(dev)
+    gh = w.grid
+    tok = torch.empty(w.n_img, 128, device=dev)
+    v = torch.empty_like(tok)
+    ref_tok, ref_hw = None, (0, 0)
+    if ref_h is not None:
+        ref_tok = torch.empty(w.n_ref, 128, device=dev)
+        F.flux_pack_latents(torch.from_numpy(ref_h).to(dev), ref_tok)
+        ref_hw = (w.ref_grid, w.ref_grid)
+    ts = F.euler_schedule(w.n_steps)
+
+    def step(i, lat_buf):
+        k = i % w.n_steps
+        if k == 0:
+            lat_buf.copy_(lat0)                     # every sampling run starts from the same noise
+        F.flux_pack_latents(lat_buf, tok)
+        model.forward(tok, (gh, gh), txt, ts[k], v, ref_tok, ref_hw)
+        F.flux_euler_step(tok, v, ts[k + 1] - ts[k])
+        F.flux_unpack_latents(tok, lat_buf)
+
+    for i in range(args.warmup):
+        step(i, lat)
+    torch.cuda.synchronize()
+    assert F.flux_device_error() == 0
+
+    # ---- timed region: K steps, device time, max over ranks
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    launches0 = F.flux_kernel_launches()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i, lat)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_total = ev0.elapsed_time(ev1)
+    launches = F.flux_kernel_launches() - launches0
+    clk = clocks.stop()
+    ms_total = max_over_ranks(ms_total, world)
+    ms_step = ms_total / args.steps
+    value = ms_total / (args.steps * world)
+
+    # ---- per-kernel device time (CUDA events around every launch of the forward)
+    model.profile(True)
+    for i in range(args.steps):
+        step(i, lat)
+    prof = model.profile_read()
+    model.profile(False)
+    assert F.flux_device_error() == 0
+
+    # ---- end to end through host buffers (pinned), H2D inputs and D2H latent every step
+    lat_pin = torch.from_numpy(lat_h).pin_memory()
+    txt_pin = torch.from_numpy(txt_h).pin_memory()
+    out_pin = torch.empty_like(lat_pin).pin_memory()
+    lat_d = torch.empty_like(lat0)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(args.steps):
+        k = i % w.n_steps
+        lat_d.copy_(lat_pin if k == 0 else out_pin, non_blocking=True)
+        txt.copy_(txt_pin, non_blocking=True)
+        F.flux_pack_latents(lat_d, tok)
+        model.forward(tok, (gh, gh), txt, ts[k], v, ref_tok, ref_hw)
+        F.flux_euler_step(tok, v, ts[k + 1] - ts[k])
+        F.flux_unpack_latents(tok, lat_d)
+        out_pin.copy_(lat_d, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / (args.steps * world)
+    assert torch.isfinite(out_pin).all()
+    h2d = lat_pin.numel() * 4 + txt_pin.numel() * 4
+    d2h = out_pin.numel() * 4
+
+    peaks, peak_src = load_peaks()
+    flops = forward_flops(w)
+    tflops = flops / (ms_step / 1e3) / 1e12
+    g_ms, g_fl, g_by, g_n = prof["gemm"]
+    a_ms, a_fl, a_by, a_n = prof["attention"]
+    gemm_tflops = g_fl / (g_ms / 1e3) / 1e12
+    attn_tflops = a_fl / (a_ms / 1e3) / 1e12
+    traffic_per_gflop, src_sha = profile_traffic("gemm_tc.cu")
+    traffic = None if traffic_per_gflop is None else traffic_per_gflop * (g_fl / g_n) / 1e9
+    kinds = {k: {"ms_per_forward": round(v_[0] / args.steps, 4), "launches_per_forward": v_[3] // args.steps,
+                 "achieved": round((v_[1] / (v_[0] / 1e3) / 1e12) if v_[1] else (v_[2] / (v_[0] / 1e3) / 1e9), 1),
+                 "unit": "TFLOP/s" if v_[1] else "GB/s"} for k, v_ in prof.items() if v_[3]}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 4), "unit": "ms/forward", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) weights scaled 1/sqrt(fan_in), bf16; N(0,1) latent and text)",
+            "config": {"workload": f"{w.name}: {w.image}x{w.image} text-to-image, {w.n_img} image + {w.n_txt} text "
+                                   f"tokens, 5 double + 20 single blocks, width 3072, 24x128 heads, "
+                                   f"one Euler step (pack, forward, Euler, unpack)",
+                       "global_batch": world, "seq_len": w.n_tokens,
+                       "parallelism": f"replicas x{world}, no data-path collective",
+                       "l2": "inputs larger than L2: 9.7 GB of bf16 weights streamed every forward"},
+            "tflops": round(tflops, 1),
+            "frac_bf16_peak": {"measured_burst": round(tflops / peaks["bf16_tflops"], 4),
+                               "measured_sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
+                               "spec_2250": round(tflops / SPEC_BF16_TFLOPS, 4), "peaks": peak_src},
+            "forwards_per_s": round(1e3 / value, 3),
+            "roofline": {"kernel": "gemm_bf16_tc (tcgen05 GEMM, all linear layers)", "bound": "tensor",
+                         "achieved": round(gemm_tflops, 1), "peak": peaks["bf16_tflops_sustained"],
+                         "unit": "TFLOP/s", "frac": round(gemm_tflops / peaks["bf16_tflops_sustained"], 4),
+                         "peak_kind": f"bf16 sustained, {peak_src}", "traffic": traffic,
+                         "launches_per_forward": g_n // args.steps,
+                         "share_of_step": round(g_ms / args.steps / ms_step, 3)},
+            "attention": {"achieved": round(attn_tflops, 1), "unit": "TFLOP/s",
+                          "frac": round(attn_tflops / peaks["bf16_tflops_sustained"], 4),
+                          "share_of_step": round(a_ms / args.steps / ms_step, 3)},
+            "kernels": kinds,
+            "e2e": {"value": round(e2e_ms, 4), "unit": "ms/forward", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            ms_cpu, secs = cpu_oracle_sample(w, params, lat_h, txt_h, ref_h)
+            line["cpu_baseline"] = {"value": round(ms_cpu, 1), "unit": "ms/forward", "cores": torch.get_num_threads(),
+                                    "kind": "oracle",
+                                    "sample": f"one double + one single block at full {w.name} size, fp32 oracle "
+                                              f"({secs:.1f} s), scaled x5 and x20 to a forward"}
+        print(json.dumps(line), flush=True)
+    model.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=4)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="t2i1024", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

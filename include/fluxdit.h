@@ -170,6 +170,19 @@ FLUX_API int flux_rope_table(float *table, int n_txt, int gh, int gw, int rh, in
 FLUX_API int flux_qk_rmsnorm_rope(uint16_t *qkv, int rows, int ld, int k_col, int heads, const uint16_t *q_gain,
                          const uint16_t *k_gain, const float *table, float eps, void *stream);
 
+/* Measurement hooks (used by the benchmark).
+ * flux_dit_profile(m, 1) starts bracketing every kernel launch of later
+ * forwards with CUDA events on the launch's stream (0 stops); both reset the
+ * totals.  flux_dit_profile_read synchronises the device and returns, for one
+ * kernel kind (0 GEMM, 1 attention, 2 LayerNorm+modulation, 3 QK-RMSNorm+RoPE,
+ * 4 GEMV, 5 other), the summed device time in ms, the algorithmic FLOPs and
+ * HBM bytes of those launches, and their number.  Any pointer may be NULL. */
+FLUX_API int flux_dit_profile(flux_dit *m, int enable);
+FLUX_API int flux_dit_profile_read(flux_dit *m, int kind, double *ms, double *flops, double *bytes, long long *launches);
+
+/* Number of kernel launches the library has enqueued since it was loaded. */
+FLUX_API unsigned long long flux_kernel_launches(void);
+
 /* Synchronise `stream`, then read and clear the kernels' device error words:
  * 0 when no kernel gave up waiting, else the first nonzero code. */
 FLUX_API int flux_device_error(void *stream);

@@ -55,6 +55,10 @@ _SIGS = {
     "flux_layernorm_modulate": (_I, [_P, _P, _I, _I, _P, _P, _F, _P]),
     "flux_rope_table": (_I, [_P, _I, _I, _I, _I, _I, _F, _P]),
     "flux_qk_rmsnorm_rope": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _F, _P]),
+    "flux_dit_profile": (_I, [_P, _I]),
+    "flux_dit_profile_read": (_I, [_P, _I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
+                                   ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]),
+    "flux_kernel_launches": (ctypes.c_ulonglong, []),
     "flux_device_error": (_I, [_P]),
 }
 EXPORTED = tuple(_SIGS)
@@ -153,6 +157,21 @@ class FluxDiT:
     def set_active_blocks(self, n_double=-1, n_single=-1):
         _check(lib().flux_dit_set_active_blocks(self._h, n_double, n_single))
 
+    PROFILE_KINDS = ("gemm", "attention", "ln_mod", "qk_norm_rope", "gemv", "other")
+
+    def profile(self, enable: bool):
+        _check(lib().flux_dit_profile(self._h, 1 if enable else 0))
+
+    def profile_read(self):
+        """{kind: (ms, flops, bytes, launches)} accumulated since profile(True)."""
+        out = {}
+        for i, name in enumerate(self.PROFILE_KINDS):
+            ms, fl, by, n = ctypes.c_double(), ctypes.c_double(), ctypes.c_double(), ctypes.c_longlong()
+            _check(lib().flux_dit_profile_read(self._h, i, ctypes.byref(ms), ctypes.byref(fl), ctypes.byref(by),
+                                               ctypes.byref(n)))
+            out[name] = (ms.value, fl.value, by.value, n.value)
+        return out
+
     def modulation_size(self) -> int:
         return lib().flux_dit_modulation_size(self._h)
 
@@ -232,6 +251,10 @@ def flux_qk_rmsnorm_rope(qkv, k_col, heads, q_gain, k_gain, table, eps=1e-6, str
                                       _bits(k_gain, "k_gain"), _ptr(table, torch.float32, "table"), float(eps),
                                       _stream(stream)))
     return qkv
+
+
+def flux_kernel_launches() -> int:
+    return lib().flux_kernel_launches()
 
 
 def flux_device_error(stream=None) -> int:

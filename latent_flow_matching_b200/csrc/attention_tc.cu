@@ -306,6 +306,7 @@ cudaError_t attention_launch(const AttnParams& P, cudaStream_t stream) {
   }
   if (P.n <= 0 || P.heads <= 0) return cudaSuccess;
   dim3 grid((P.n + kTile - 1) / kTile, P.heads);
+  count_launch();
   attention_tc_kernel<<<grid, 192, kSmemBytes, stream>>>(P);
   return cudaGetLastError();
 }

@@ -285,24 +285,28 @@ __global__ void __launch_bounds__(256) gemv_kernel(const __nv_bfloat16* __restri
 
 cudaError_t pack_latents_launch(const float* lat, float* tok, int c, int h8, int w8, cudaStream_t s) {
   const size_t total = static_cast<size_t>(h8 / 2) * (w8 / 2) * c;
+  count_launch();
   pack_kernel<<<blocks_for(total, 256), 256, 0, s>>>(lat, tok, c, h8, w8);
   return cudaGetLastError();
 }
 
 cudaError_t unpack_latents_launch(const float* tok, float* lat, int c, int h8, int w8, cudaStream_t s) {
   const size_t total = static_cast<size_t>(h8 / 2) * (w8 / 2) * c;
+  count_launch();
   unpack_kernel<<<blocks_for(total, 256), 256, 0, s>>>(tok, lat, c, h8, w8);
   return cudaGetLastError();
 }
 
 cudaError_t euler_launch(float* x, const float* v, size_t n, float dt, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
+  count_launch();
   euler_kernel<<<blocks_for((n + 3) / 4, 256), 256, 0, s>>>(x, v, n, dt);
   return cudaGetLastError();
 }
 
 cudaError_t cast_bf16_launch(const float* x, __nv_bfloat16* y, size_t n, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
+  count_launch();
   cast_bf16_kernel<<<blocks_for((n + 3) / 4, 256), 256, 0, s>>>(x, y, n);
   return cudaGetLastError();
 }
@@ -312,6 +316,7 @@ cudaError_t ln_modulate_launch(const float* x, __nv_bfloat16* y, int rows, int d
                                cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   const int grid = (rows + 7) / 8;
+  count_launch();
   if (dim == 3072)
     ln_mod_kernel<24><<<grid, 256, 0, s>>>(x, y, rows, split, shift0, scale0, shift1, scale1, eps);
   else
@@ -324,6 +329,7 @@ cudaError_t qk_norm_rope_launch(__nv_bfloat16* qkv, int rows, int ld, int kcol, 
                                 const __nv_bfloat16* gk1, const float2* rope, float eps, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   const int warps = rows * 2;
+  count_launch();
   qk_norm_rope_kernel<<<(warps + 7) / 8, 256, 0, s>>>(qkv, rows, ld, kcol, heads, split, gq0, gk0, gq1, gk1, rope,
                                                       eps);
   return cudaGetLastError();
@@ -332,11 +338,13 @@ cudaError_t qk_norm_rope_launch(__nv_bfloat16* qkv, int rows, int ld, int kcol, 
 cudaError_t rope_table_launch(float2* table, int n_txt, int gh, int gw, int rh, int rw, float theta, cudaStream_t s) {
   const int n = n_txt + gh * gw + rh * rw;
   if (n <= 0) return cudaSuccess;
+  count_launch();
   rope_table_kernel<<<(n * 64 + 255) / 256, 256, 0, s>>>(table, n_txt, gh, gw, rh, rw, theta);
   return cudaGetLastError();
 }
 
 cudaError_t timestep_embed_launch(float* temb, float t, int dim, cudaStream_t s) {
+  count_launch();
   timestep_embed_kernel<<<(dim / 2 + 127) / 128, 128, 0, s>>>(temb, t, dim);
   return cudaGetLastError();
 }
@@ -348,6 +356,7 @@ cudaError_t gemv_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, const fl
   int grid = (rows + per_block - 1) / per_block;
   const int cap = num_sms_current() * 8;
   if (grid > cap) grid = cap;
+  count_launch();
   gemv_kernel<<<grid, 256, k * sizeof(float), s>>>(W, b, x, y, rows, k, silu_in, silu_out);
   return cudaGetLastError();
 }

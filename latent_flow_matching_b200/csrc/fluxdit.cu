@@ -17,6 +17,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -79,6 +80,77 @@ int num_sms_current() {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n;
+}
+
+// ------------------------------------------------------------------ launch counter
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+// ------------------------------------------------------------------ per-kernel profiling
+// When enabled, every launch of a forward is bracketed by two CUDA events on its
+// stream; flux_dit_profile_read() synchronises and accumulates the elapsed time
+// per kernel kind together with the launch's algorithmic FLOPs and HBM bytes.
+enum ProfKind { kProfGemm = 0, kProfAttention, kProfLnMod, kProfQkNormRope, kProfGemv, kProfOther, kProfKinds };
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+  double flops, bytes;
+};
+struct Profiler {
+  bool on = false;
+  std::vector<cudaEvent_t> pool;
+  std::vector<ProfRec> pending;
+  double ms[kProfKinds] = {}, flops[kProfKinds] = {}, bytes[kProfKinds] = {};
+  long long launches[kProfKinds] = {};
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+  void settle() {
+    for (const ProfRec& r : pending) {
+      float t = 0.f;
+      if (cudaEventElapsedTime(&t, r.a, r.b) == cudaSuccess) {
+        ms[r.kind] += t;
+        flops[r.kind] += r.flops;
+        bytes[r.kind] += r.bytes;
+        launches[r.kind] += 1;
+      }
+      pool.push_back(r.a);
+      pool.push_back(r.b);
+    }
+    pending.clear();
+  }
+  void reset() {
+    settle();
+    for (int k = 0; k < kProfKinds; ++k) ms[k] = flops[k] = bytes[k] = 0, launches[k] = 0;
+  }
+  ~Profiler() {
+    settle();
+    for (cudaEvent_t e : pool) cudaEventDestroy(e);
+  }
+};
+
+static double gemm_flops(const GemmParams& P) {
+  double f = 0;
+  for (int i = 0; i < P.num_problems; ++i)
+    if (P.prob[i].M > 0) f += 2.0 * P.prob[i].M * static_cast<double>(P.prob[i].N) * P.prob[i].K;
+  return f;
+}
+static double gemm_bytes(const GemmParams& P) {
+  double b = 0;
+  for (int i = 0; i < P.num_problems; ++i) {
+    const GemmProblem& pr = P.prob[i];
+    if (pr.M <= 0) continue;
+    const double out_elt = pr.mode == kEpiBf16Bias ? 2 : pr.mode == kEpiSwiGLU ? 1 : pr.mode == kEpiF32Bias ? 4 : 8;
+    b += 2.0 * pr.M * pr.K + 2.0 * pr.N * pr.K + out_elt * pr.M * pr.N;
+  }
+  return b;
 }
 
 // ------------------------------------------------------------------ blob layout
@@ -179,6 +251,7 @@ struct flux_dit {
   std::vector<fdit::SingleW> sgl;
   int act_double = 0, act_single = 0;
   fdit::Workspace ws;
+  fdit::Profiler prof;
 };
 
 namespace fdit {
@@ -362,7 +435,6 @@ static int prepare_shape(flux_dit* m, int nt, int gh, int gw, int rh, int rw, cu
   const size_t ni = static_cast<size_t>(gh) * gw, nr = static_cast<size_t>(rh) * rw;
   const size_t n = nt + ni + nr;
   if (n > w.cap_n) {
-    size_t cap = 0;
     float* X = nullptr;
     free_ws(w);
     const size_t need = n;
@@ -376,7 +448,6 @@ static int prepare_shape(flux_dit* m, int nt, int gh, int gw, int rh, int rw, cu
       free_ws(w);
       return fail(FLUX_ENOMEM, "workspace allocation for %zu tokens failed", need);
     }
-    (void)cap;
     w.cap_n = need;
   }
   if (grow(&w.tokb, &w.cap_tok, (ni + nr) * c.in_ch) != cudaSuccess ||
@@ -413,6 +484,22 @@ static int prepare_shape(flux_dit* m, int nt, int gh, int gw, int rh, int rw, cu
   return FLUX_OK;
 }
 
+// Enqueue `expr` (a launch returning cudaError_t); bracket it with profiling events when enabled.
+#define FD_LAUNCH(m, kind, fl, by, expr)                                                   \
+  do {                                                                                     \
+    cudaEvent_t ea_ = nullptr, eb_ = nullptr;                                              \
+    if ((m)->prof.on) {                                                                    \
+      ea_ = (m)->prof.get();                                                               \
+      eb_ = (m)->prof.get();                                                               \
+      cudaEventRecord(ea_, s);                                                             \
+    }                                                                                      \
+    FD_CUDA(expr);                                                                         \
+    if ((m)->prof.on) {                                                                    \
+      cudaEventRecord(eb_, s);                                                             \
+      (m)->prof.pending.push_back({(kind), ea_, eb_, (fl), (by)});                         \
+    }                                                                                      \
+  } while (0)
+
 static void problem(GemmParams& P, int i, const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, int mode,
                     void* out, int ldo, const bf16* bias, const float* gate) {
   P.mapA[i] = a;
@@ -425,10 +512,13 @@ static void problem(GemmParams& P, int i, const CUtensorMap& a, const CUtensorMa
 static int run_modulation(flux_dit* m, float t, cudaStream_t s) {
   const flux_dit_config& c = m->cfg;
   const int D = c.hidden;
-  FD_CUDA(timestep_embed_launch(m->temb, t, c.t_freq_dim, s));
-  FD_CUDA(gemv_launch(m->t_w1, m->t_b1, m->temb, m->th, D, c.t_freq_dim, 0, 1, s));
-  FD_CUDA(gemv_launch(m->t_w2, m->t_b2, m->th, m->vec, D, D, 0, 0, s));
-  FD_CUDA(gemv_launch(m->mods_w, m->mods_b, m->vec, m->mods, static_cast<int>(m->mods_rows), D, 1, 0, s));
+  auto gv = [](double rows, double k) { return rows * k * 2 + rows * 6 + k * 4; };
+  FD_LAUNCH(m, kProfOther, 0, c.t_freq_dim * 4.0, timestep_embed_launch(m->temb, t, c.t_freq_dim, s));
+  FD_LAUNCH(m, kProfGemv, 2.0 * D * c.t_freq_dim, gv(D, c.t_freq_dim),
+            gemv_launch(m->t_w1, m->t_b1, m->temb, m->th, D, c.t_freq_dim, 0, 1, s));
+  FD_LAUNCH(m, kProfGemv, 2.0 * D * D, gv(D, D), gemv_launch(m->t_w2, m->t_b2, m->th, m->vec, D, D, 0, 0, s));
+  FD_LAUNCH(m, kProfGemv, 2.0 * m->mods_rows * D, gv(static_cast<double>(m->mods_rows), D),
+            gemv_launch(m->mods_w, m->mods_b, m->vec, m->mods, static_cast<int>(m->mods_rows), D, 1, 0, s));
   return FLUX_OK;
 }
 
@@ -456,16 +546,25 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
 
   rc = run_modulation(m, t, s);
   if (rc) return rc;
-  FD_CUDA(cast_bf16_launch(img_tok, w.tokb, static_cast<size_t>(ni) * c.in_ch, s));
-  if (nr) FD_CUDA(cast_bf16_launch(ref_tok, w.tokb + static_cast<size_t>(ni) * c.in_ch, static_cast<size_t>(nr) * c.in_ch, s));
-  if (nt) FD_CUDA(cast_bf16_launch(txt, w.txtb, static_cast<size_t>(nt) * c.txt_dim, s));
+  FD_LAUNCH(m, kProfOther, 0, 6.0 * ni * c.in_ch,
+            cast_bf16_launch(img_tok, w.tokb, static_cast<size_t>(ni) * c.in_ch, s));
+  if (nr)
+    FD_LAUNCH(m, kProfOther, 0, 6.0 * nr * c.in_ch,
+              cast_bf16_launch(ref_tok, w.tokb + static_cast<size_t>(ni) * c.in_ch,
+                               static_cast<size_t>(nr) * c.in_ch, s));
+  if (nt)
+    FD_LAUNCH(m, kProfOther, 0, 6.0 * nt * c.txt_dim,
+              cast_bf16_launch(txt, w.txtb, static_cast<size_t>(nt) * c.txt_dim, s));
+  const double ln_bytes = 6.0 * n * D + 16.0 * D, ln_bytes_img = 6.0 * ni * D + 8.0 * D;
+  const double qk_bytes = 8.0 * n * D + 512.0 * n;
+  const double at_flops = 4.0 * n * static_cast<double>(n) * D, at_bytes = 8.0 * n * D;
 
   GemmParams P;
   P.num_problems = 2;
   problem(P, 0, w.a_txtb, m->m_txt_in, nt, D, c.txt_dim, kEpiF32Bias, w.X, D, m->txt_b, nullptr);
   problem(P, 1, w.a_tokb, m->m_img_in, nimg, D, c.in_ch, kEpiF32Bias, w.X + static_cast<size_t>(nt) * D, D, m->img_b,
           nullptr);
-  FD_CUDA(gemm_launch(P, 256, m->num_sms, s));
+  FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 256, m->num_sms, s));
 
   float* Ximg = w.X + static_cast<size_t>(nt) * D;
   bf16* Otxt = w.CC;
@@ -481,49 +580,49 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
     const StreamW& st = m->dbl[2 * i + 1];
     const float* mi = mods + si.mod_off;          // shift1, scale1, gate1, shift2, scale2, gate2
     const float* mt = mods + st.mod_off;
-    FD_CUDA(ln_modulate_launch(w.X, w.Y, n, D, nt, mt, mt + D, mi, mi + D, eps_ln, s));
+    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes, ln_modulate_launch(w.X, w.Y, n, D, nt, mt, mt + D, mi, mi + D, eps_ln, s));
     P.num_problems = 2;
     problem(P, 0, w.a_Ytxt, st.m_qkv, nt, 3 * D, D, kEpiBf16Bias, w.QKV, 3 * D, st.qkv_b, nullptr);
     problem(P, 1, w.a_Yimg, si.m_qkv, nimg, 3 * D, D, kEpiBf16Bias, w.QKV + static_cast<size_t>(nt) * 3 * D, 3 * D,
             si.qkv_b, nullptr);
-    FD_CUDA(gemm_launch(P, 256, m->num_sms, s));
-    FD_CUDA(qk_norm_rope_launch(w.QKV, n, 3 * D, D, H, nt, st.q_gain, st.k_gain, si.q_gain, si.k_gain, w.rope,
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 256, m->num_sms, s));
+    FD_LAUNCH(m, kProfQkNormRope, 0, qk_bytes, qk_norm_rope_launch(w.QKV, n, 3 * D, D, H, nt, st.q_gain, st.k_gain, si.q_gain, si.k_gain, w.rope,
                                 eps_rms, s));
-    FD_CUDA(attention_launch(A, s));
+    FD_LAUNCH(m, kProfAttention, at_flops, at_bytes, attention_launch(A, s));
     P.num_problems = 2;
     problem(P, 0, w.a_Otxt, st.m_proj, nt, D, D, kEpiResidGate, w.X, D, st.proj_b, mt + 2 * D);
     problem(P, 1, w.a_Oimg, si.m_proj, nimg, D, D, kEpiResidGate, Ximg, D, si.proj_b, mi + 2 * D);
-    FD_CUDA(gemm_launch(P, 256, m->num_sms, s));
-    FD_CUDA(ln_modulate_launch(w.X, w.Y, n, D, nt, mt + 3 * D, mt + 4 * D, mi + 3 * D, mi + 4 * D, eps_ln, s));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 256, m->num_sms, s));
+    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes, ln_modulate_launch(w.X, w.Y, n, D, nt, mt + 3 * D, mt + 4 * D, mi + 3 * D, mi + 4 * D, eps_ln, s));
     P.num_problems = 2;
     problem(P, 0, w.a_Ytxt, st.m_mlp_in, nt, 2 * F, D, kEpiSwiGLU, Otxt + D, D + F, st.mlp_in_b, nullptr);
     problem(P, 1, w.a_Yimg, si.m_mlp_in, nimg, 2 * F, D, kEpiSwiGLU, Oimg + D, D + F, si.mlp_in_b, nullptr);
-    FD_CUDA(gemm_launch(P, 256, m->num_sms, s));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 256, m->num_sms, s));
     P.num_problems = 2;
     problem(P, 0, w.a_Htxt, st.m_mlp_out, nt, D, F, kEpiResidGate, w.X, D, st.mlp_out_b, mt + 5 * D);
     problem(P, 1, w.a_Himg, si.m_mlp_out, nimg, D, F, kEpiResidGate, Ximg, D, si.mlp_out_b, mi + 5 * D);
-    FD_CUDA(gemm_launch(P, 256, m->num_sms, s));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 256, m->num_sms, s));
   }
   for (int i = 0; i < m->act_single; ++i) {
     const SingleW& sw = m->sgl[i];
     const float* ms = mods + sw.mod_off;          // shift, scale, gate
-    FD_CUDA(ln_modulate_launch(w.X, w.Y, n, D, n, ms, ms + D, ms, ms + D, eps_ln, s));
+    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes, ln_modulate_launch(w.X, w.Y, n, D, n, ms, ms + D, ms, ms + D, eps_ln, s));
     P.num_problems = 2;
     problem(P, 0, w.a_Yall, sw.m_qkv, n, 3 * D, D, kEpiBf16Bias, w.QKV, 3 * D, sw.qkv_b, nullptr);
     problem(P, 1, w.a_Yall, sw.m_mlp, n, 2 * F, D, kEpiSwiGLU, w.CC + D, D + F, sw.mlp_b, nullptr);
-    FD_CUDA(gemm_launch(P, 256, m->num_sms, s));
-    FD_CUDA(qk_norm_rope_launch(w.QKV, n, 3 * D, D, H, n, sw.q_gain, sw.k_gain, sw.q_gain, sw.k_gain, w.rope, eps_rms,
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 256, m->num_sms, s));
+    FD_LAUNCH(m, kProfQkNormRope, 0, qk_bytes, qk_norm_rope_launch(w.QKV, n, 3 * D, D, H, n, sw.q_gain, sw.k_gain, sw.q_gain, sw.k_gain, w.rope, eps_rms,
                                 s));
-    FD_CUDA(attention_launch(A, s));
+    FD_LAUNCH(m, kProfAttention, at_flops, at_bytes, attention_launch(A, s));
     P.num_problems = 1;
     problem(P, 0, w.a_CC, sw.m_lin2, n, D, D + F, kEpiResidGate, w.X, D, sw.lin2_b, ms + 2 * D);
-    FD_CUDA(gemm_launch(P, 256, m->num_sms, s));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 256, m->num_sms, s));
   }
   const float* mf = mods + m->fin_mod_off;         // shift, scale
-  FD_CUDA(ln_modulate_launch(Ximg, w.Y, ni, D, ni, mf, mf + D, mf, mf + D, eps_ln, s));
+  FD_LAUNCH(m, kProfLnMod, 0, ln_bytes_img, ln_modulate_launch(Ximg, w.Y, ni, D, ni, mf, mf + D, mf, mf + D, eps_ln, s));
   P.num_problems = 1;
   problem(P, 0, w.a_Yout, m->m_fin, ni, c.in_ch, D, kEpiF32Bias, v_out, c.in_ch, m->fin_b, nullptr);
-  FD_CUDA(gemm_launch(P, 128, m->num_sms, s));
+  FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 128, m->num_sms, s));
   return FLUX_OK;
 }
 
@@ -684,6 +783,27 @@ int flux_qk_rmsnorm_rope(uint16_t* qkv, int rows, int ld, int k_col, int heads, 
                               reinterpret_cast<const float2*>(table), eps, static_cast<cudaStream_t>(stream)));
   return FLUX_OK;
 }
+
+int flux_dit_profile(flux_dit* m, int enable) {
+  if (!m) return fail(FLUX_EINVAL, "model is NULL");
+  FD_CUDA(cudaDeviceSynchronize());
+  m->prof.reset();
+  m->prof.on = enable != 0;
+  return FLUX_OK;
+}
+
+int flux_dit_profile_read(flux_dit* m, int kind, double* ms, double* flops, double* bytes, long long* launches) {
+  if (!m || kind < 0 || kind >= kProfKinds) return fail(FLUX_EINVAL, "bad model or kernel kind");
+  FD_CUDA(cudaDeviceSynchronize());
+  m->prof.settle();
+  if (ms) *ms = m->prof.ms[kind];
+  if (flops) *flops = m->prof.flops[kind];
+  if (bytes) *bytes = m->prof.bytes[kind];
+  if (launches) *launches = m->prof.launches[kind];
+  return FLUX_OK;
+}
+
+unsigned long long flux_kernel_launches(void) { return g_launches.load(); }
 
 int flux_device_error(void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);

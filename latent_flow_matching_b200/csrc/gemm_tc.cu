@@ -308,6 +308,7 @@ cudaError_t launch_bn(GemmParams& P, int num_sms, cudaStream_t stream) {
     attr_set = true;
   }
   const int grid = P.total_tiles < num_sms ? P.total_tiles : num_sms;
+  count_launch();
   gemm_bf16_tc_kernel<BN><<<grid, 192, C::SMEM_BYTES, stream>>>(P);
   return cudaGetLastError();
 }

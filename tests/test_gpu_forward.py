@@ -1,0 +1,163 @@
+"""Forward and sampler parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Bars: velocity relative L2 <= 2e-2 at every step, final latent relative L2 <=
+3e-2 after all steps, modulation vector normalised max error <= 1e-2.
+* tiny 64^2 workload (1 double + 1 single block): the oracle runs live in float64.
+* 256^2 .. 1024^2(+reference) workloads: the oracle's sampled rows, written by
+  tests/golden/make_goldens.py (oracle only), are compared row by row.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import latent_flow_matching_b200 as F
+from oracle import flux_oracle as O
+from synthetic import WORKLOADS, FluxDims, Workload, make_weights, make_inputs
+
+pytestmark = pytest.mark.gpu
+torch.set_grad_enabled(False)
+DEV = "cuda"
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+V_TOL, X_TOL, K_TOL = 2e-2, 3e-2, 1e-2
+
+
+def rel_l2(a, b):
+    a = torch.as_tensor(a).double().cpu()
+    b = torch.as_tensor(b).double().cpu()
+    return ((a - b).norm() / b.norm()).item()
+
+
+def gpu_sample(model, w, lat, txt, ref):
+    vs = []
+    final = F.flux_sample(model, torch.from_numpy(lat).to(DEV), torch.from_numpy(txt).to(DEV), w.n_steps,
+                          None if ref is None else torch.from_numpy(ref).to(DEV),
+                          on_step=lambda i, v: vs.append(v.cpu().clone()))
+    return final.cpu(), vs
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    w = WORKLOADS["tiny64"]
+    blob, p = make_weights(w.dims, w.seed)
+    model = F.FluxDiT(blob, w.dims)
+    yield w, p, model
+    model.close()
+
+
+def test_tiny_modulation_vector(tiny):
+    w, p, model = tiny
+    for t in (1.0, 0.25):
+        out = torch.empty(model.modulation_size(), device=DEV)
+        model.modulation(t, out)
+        temb = O.timestep_embedding(t)
+        h = O.silu(O.linear(temb, O.weight(p, "time_in.w1", torch.float64), O.weight(p, "time_in.b1", torch.float64)))
+        s = O.silu(O.linear(h, O.weight(p, "time_in.w2", torch.float64), O.weight(p, "time_in.b2", torch.float64)))
+        names = [k for k in p if k.endswith("mod.w")]
+        ref = torch.cat([O.linear(s, O.weight(p, n, torch.float64), O.weight(p, n[:-1] + "b", torch.float64))
+                         for n in names])
+        err = ((out.cpu().double() - ref).abs().max() / ref.abs().max()).item()
+        assert err <= K_TOL, err
+
+
+@pytest.mark.parametrize("n_double,n_single", [(0, 0), (1, 0), (1, 1)])
+def test_tiny_forward_block_by_block(tiny, n_double, n_single):
+    w, p, model = tiny
+    lat, txt, _ = make_inputs(w)
+    keep = {k: v for k, v in p.items()
+            if not ((k.startswith("double.") and int(k.split(".")[1]) >= n_double) or
+                    (k.startswith("single.") and int(k.split(".")[1]) >= n_single))}
+    tok = O.pack_latents(torch.from_numpy(lat))
+    ref = O.forward(keep, O.hyper(w.dims), tok, torch.from_numpy(txt), 0.75, (w.grid, w.grid))
+    model.set_active_blocks(n_double, n_single)
+    try:
+        v = torch.empty(w.n_img, 128, device=DEV)
+        model.forward(tok.float().to(DEV), (w.grid, w.grid), torch.from_numpy(txt).to(DEV), 0.75, v)
+    finally:
+        model.set_active_blocks(-1, -1)
+    assert rel_l2(v, ref) <= V_TOL
+    assert F.flux_device_error() == 0
+
+
+def test_tiny_sampler_matches_oracle(tiny):
+    w, p, model = tiny
+    lat, txt, _ = make_inputs(w)
+    ref_final, ref_vs = O.sample(p, O.hyper(w.dims), torch.from_numpy(lat), torch.from_numpy(txt), w.n_steps)
+    final, vs = gpu_sample(model, w, lat, txt, None)
+    for i in range(w.n_steps):
+        assert rel_l2(vs[i], ref_vs[i]) <= V_TOL
+    assert rel_l2(final, ref_final) <= X_TOL
+    assert F.flux_device_error() == 0
+
+
+def test_forward_is_deterministic(tiny):
+    w, p, model = tiny
+    lat, txt, _ = make_inputs(w)
+    a, _ = gpu_sample(model, w, lat, txt, None)
+    b, _ = gpu_sample(model, w, lat, txt, None)
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("n_txt,grid,ref_grid", [(0, (4, 6), (0, 0)), (5, (6, 4), (4, 4)), (131, (8, 8), (4, 8))])
+def test_tiny_forward_ragged_and_degenerate_shapes(tiny, n_txt, grid, ref_grid):
+    """No text, non-square grids, a reference of another size, sequence lengths off the 128-row tiles."""
+    w, p, model = tiny
+    g = torch.Generator().manual_seed(n_txt)
+    tok = torch.randn(grid[0] * grid[1], 128, generator=g).to(torch.bfloat16).float()
+    txt = torch.randn(n_txt, 3072, generator=g).to(torch.bfloat16).float()
+    ref = None
+    if ref_grid[0]:
+        ref = torch.randn(ref_grid[0] * ref_grid[1], 128, generator=g).to(torch.bfloat16).float()
+    want = O.forward(p, O.hyper(w.dims), tok, txt, 0.5, grid, ref, ref_grid)
+    v = torch.empty(grid[0] * grid[1], 128, device=DEV)
+    model.forward(tok.to(DEV), grid, txt.to(DEV) if n_txt else None, 0.5, v,
+                  None if ref is None else ref.to(DEV), ref_grid)
+    assert rel_l2(v, want) <= V_TOL
+
+
+def test_forward_rejects_bad_shapes(tiny):
+    w, p, model = tiny
+    v = torch.empty(16, 128, device=DEV)
+    tok = torch.zeros(16, 128, device=DEV)
+    txt = torch.zeros(4, 3072, device=DEV)
+    for grid in ((2, 8), (65, 4)):
+        with pytest.raises(F.FluxError):
+            model.forward(tok, grid, txt, 1.0, v)
+    with pytest.raises(F.FluxError):
+        model.forward(tok, (4, 4), txt, 1.0, v, None, (4, 4))       # reference grid without tokens
+    with pytest.raises(F.FluxError):
+        model.forward(tok, (4, 4), txt, float("nan"), v)
+
+
+# ---------------------------------------------------------------------------- full-size workloads vs goldens
+def _golden(name):
+    path = os.path.join(GOLDEN, f"{name}.npz")
+    if not os.path.exists(path):
+        pytest.skip(f"golden {path} not generated")
+    return np.load(path)
+
+
+@pytest.mark.parametrize("name", ["t2i256", "t2i512", "t2i1024", "i2i1024"])
+def test_full_workload_against_oracle_goldens(name):
+    gd = _golden(name)
+    w = WORKLOADS[name]
+    meta = json.loads(str(gd["meta"]))
+    assert meta["workload"] == name and meta["seed"] == w.seed
+    blob, _ = make_weights(w.dims, w.seed)
+    lat, txt, ref = make_inputs(w)
+    model = F.FluxDiT(blob, w.dims)
+    del blob
+    try:
+        final, vs = gpu_sample(model, w, lat, txt, ref)
+    finally:
+        model.close()
+    rows = torch.from_numpy(gd["rows"]).long()
+    for i in range(w.n_steps):
+        err = rel_l2(vs[i][rows], gd["v"][i])
+        assert err <= V_TOL, (i, err)
+    tok = O.pack_latents(final)
+    err = rel_l2(tok[rows], gd["final"])
+    assert err <= X_TOL, err
+    assert F.flux_device_error() == 0
