@@ -183,6 +183,30 @@ FLUX_API int flux_dit_profile_read(flux_dit *m, int kind, double *ms, double *fl
 /* Number of kernel launches the library has enqueued since it was loaded. */
 FLUX_API unsigned long long flux_kernel_launches(void);
 
+/* Timestep conditioning that allocates no device memory (the pages have no
+ * counterpart; this is a deployment convenience).  For callers that may not
+ * call cudaMalloc once running -- runtimes that hand all device memory to a
+ * pre-sized pool at start-up, or latency-critical loops that cannot take the
+ * stall of cudaMalloc/cudaFree (cudaFree can synchronise the whole device).
+ * Computes what flux_dit_modulation computes, from caller-owned weights:
+ *   temb = [cos(t*1000*f_j), sin(t*1000*f_j)], vec = w2 silu(w1 temb + b1) + b2,
+ *   mods_out = wmod silu(vec) + bmod
+ * w1 bf16 [hidden, t_freq_dim], w2 bf16 [hidden, hidden], wmod bf16 [mod_rows,
+ * hidden] (every modulation linear stacked in blob order), biases bf16,
+ * mods_out fp32 [mod_rows]; weight and output pointers 16-byte aligned.
+ * Limits: hidden <= 8192 and t_freq_dim <= 1024, both multiples of 8; larger
+ * sizes return FLUX_EINVAL.  The intermediates live in one 68 KiB device array
+ * inside the library, which every GPU that loads the library holds until the
+ * process exits.  The first call on a device looks up that array's address
+ * (cudaGetSymbolAddress) with the device current; make that first call before
+ * any stream capture.  All calls on a device share the array: calls whose
+ * kernels overlap on the GPU (different streams without ordering) race.  Each
+ * call writes every scratch element before reading it, so nothing is cleared. */
+FLUX_API int flux_timestep_modulation_noalloc(const uint16_t *w1, const uint16_t *b1, const uint16_t *w2,
+                                              const uint16_t *b2, const uint16_t *wmod, const uint16_t *bmod,
+                                              int hidden, int t_freq_dim, int mod_rows, float t, float *mods_out,
+                                              void *stream);
+
 /* Synchronise `stream`, then read and clear the kernels' device error words:
  * 0 when no kernel gave up waiting, else the first nonzero code. */
 FLUX_API int flux_device_error(void *stream);

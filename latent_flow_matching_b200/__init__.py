@@ -59,6 +59,7 @@ _SIGS = {
     "flux_dit_profile_read": (_I, [_P, _I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
                                    ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]),
     "flux_kernel_launches": (ctypes.c_ulonglong, []),
+    "flux_timestep_modulation_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _F, _P, _P]),
     "flux_device_error": (_I, [_P]),
 }
 EXPORTED = tuple(_SIGS)
@@ -251,6 +252,17 @@ def flux_qk_rmsnorm_rope(qkv, k_col, heads, q_gain, k_gain, table, eps=1e-6, str
                                       _bits(k_gain, "k_gain"), _ptr(table, torch.float32, "table"), float(eps),
                                       _stream(stream)))
     return qkv
+
+
+def flux_timestep_modulation_noalloc(w1, b1, w2, b2, wmod, bmod, t, mods_out, stream=None):
+    """Timestep conditioning with no device allocation (see fluxdit.h); weights bf16, mods_out fp32."""
+    import torch
+    hidden, t_freq_dim = w1.shape
+    _check(lib().flux_timestep_modulation_noalloc(_bits(w1, "w1"), _bits(b1, "b1"), _bits(w2, "w2"), _bits(b2, "b2"),
+                                                  _bits(wmod, "wmod"), _bits(bmod, "bmod"), hidden, t_freq_dim,
+                                                  wmod.shape[0], float(t), _ptr(mods_out, torch.float32, "mods_out"),
+                                                  _stream(stream)))
+    return mods_out
 
 
 def flux_kernel_launches() -> int:

@@ -46,6 +46,8 @@ static int fail(int code, const char* fmt, ...) {
   return code;
 }
 
+int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
 #define FD_CUDA(expr)                                                                          \
   do {                                                                                         \
     cudaError_t e_ = (expr);                                                                   \

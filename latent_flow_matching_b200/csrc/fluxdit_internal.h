@@ -78,6 +78,8 @@ cudaError_t gemv_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, const fl
                         int k, int silu_in, int silu_out, cudaStream_t s);
 
 // ------------------------------------------------------------------ host helpers
+// Record `msg` as the calling thread's flux_get_error() message and return `code`.
+int record_error(int code, const char* msg);
 // Counts kernel launches enqueued by the library (reported by flux_kernel_launches).
 void count_launch();
 // 2D bf16 tensor map: rows x cols, row stride in bytes, box {64 cols, box_rows}, 128B swizzle.
