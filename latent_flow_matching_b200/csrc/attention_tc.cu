@@ -4,18 +4,24 @@
 // Klein in Diffusers write-up, "Entkoppelte Vorverarbeitung und gemeinsame
 // Attention-Blöcke" and "Verarbeitung einzelner Prompts und Batching-Architektur".
 //
-// CTA = one 128-row query tile of one head, 6 warps:
-//   warp 0      TMA: Q once, then K_j / V_j tiles into a 2-deep ring
-//   warp 1      one thread issues tcgen05.mma: S_j = Q K_j^T into TMEM buffer j&1,
-//               then O += P_{j-1} V_{j-1} with P read from TMEM (A operand in TMEM)
-//   warps 2..5  one thread per query row: read S_j from TMEM, online softmax in
-//               the exp2 domain, write P_j as packed bf16 over the S_j columns,
-//               rescale the O row in TMEM when the running max moved, and at
-//               the end write O / l as bf16.
-// The running max is only moved when it grows by more than 8 (log2 units), so
-// most iterations skip the O rescale; P stays below 2^8, safe in bf16/fp32.
+// CTA = two 128-row query tiles (A, B) of one head that share every K/V tile and
+// take turns on the tensor core, 12 warps in three warpgroups:
+//   warps 0..3   softmax of tile A   (one thread per query row)
+//   warps 4..7   softmax of tile B
+//   warp 8       TMA: Q_A, Q_B once, then K_j / V_j into a 2-deep ring
+//   warp 9       one thread issues tcgen05.mma in the order
+//                  S_A(0) S_B(0) | PV_A(0) S_A(1) PV_B(0) S_B(1) | PV_A(1) S_A(2) ...
+//                so the tensor core works on one tile while the other tile's
+//                softmax runs, and S_X(j) is issued after PV_X(j-1): when a
+//                softmax warpgroup sees S_X(j), O_X already holds every earlier
+//                P V and can be rescaled in place without another wait.
+// Softmax: read S from TMEM, online softmax in the exp2 domain, write P as packed
+// bf16 over the S columns (the PV MMA reads its A operand from TMEM), rescale the
+// O row only when the running max grows by more than 8 (log2 units; P stays below
+// 2^8), and at the end write O / l as bf16.  setmaxnreg moves registers from the
+// control warpgroup to the two softmax warpgroups.
 //
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,384) of a 512-column allocation.
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
 #include "common.cuh"
 #include "fluxdit_internal.h"
 
@@ -27,14 +33,19 @@ namespace {
 
 constexpr int kTile = 128;          // query rows and key rows per tile
 constexpr int kHeadDim = 128;
+constexpr int kQTiles = 2;          // query tiles per CTA
 constexpr int kBox = 64;            // 64 bf16 = 128 bytes: one swizzle row
 constexpr int kBoxBytes = kTile * kBox * 2;          // 16 KB
 constexpr int kTileBytes = 2 * kBoxBytes;            // 32 KB: 128 rows x 128 dims
 constexpr int kStages = 2;
-constexpr int kSmemBytes = kTileBytes * (1 + 2 * kStages) + 1024 + 256;
+constexpr int kThreads = 384;
+constexpr int kSmemBytes = kTileBytes * (kQTiles + 2 * kStages) + 1024 + 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOCol = 256;
 constexpr float kRescaleThreshold = 8.0f;
+// 384 threads x 168 registers at launch = 256 x 224 (softmax) + 128 x 56 (control)
+constexpr int kSoftmaxRegs = 224;
+constexpr int kControlRegs = 56;
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -42,27 +53,48 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-__global__ void __launch_bounds__(192, 1) attention_tc_kernel(const __grid_constant__ AttnParams P) {
+// 2^x on the FMA pipe, to take part of the exponentials off the MUFU unit: split
+// x = j + f with j the nearest integer (|f| <= 1/2) by the 1.5 * 2^23 rounding
+// trick, evaluate 2^f with a cubic minimax polynomial (coefficients from a Remez
+// exchange fit of 2^f on [-1/2, 1/2]; max relative error 7.5e-5, well below the
+// 2^-9 of the bf16 P it feeds), and add j to the exponent field.  Inputs below
+// -126 are clamped (their weight is < 2^-126).
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// one score pair in kPolyEvery goes through ex2_poly, the rest through MUFU ex2 (0: none)
+#ifndef FDIT_POLY_EVERY
+#define FDIT_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = FDIT_POLY_EVERY;
+
+__global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_constant__ AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + kTileBytes;                       // kStages tiles
+  uint8_t* sQ = smem;                                    // kQTiles tiles
+  uint8_t* sK = sQ + kQTiles * kTileBytes;               // kStages tiles
   uint8_t* sV = sK + kStages * kTileBytes;               // kStages tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kStages * kTileBytes);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;                           // [2]
-  uint64_t* v_full = bars + 3;                           // [2]
-  uint64_t* kv_empty = bars + 5;                         // [2]
-  uint64_t* s_full = bars + 7;                           // [2]
-  uint64_t* p_full = bars + 9;                           // [2]
-  uint64_t* o_done = bars + 11;                          // [2]: PV_i completes o_done[i & 1]
-  uint64_t* drain = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* k_full = bars + 1;                           // [stage]
+  uint64_t* v_full = bars + 3;                           // [stage]
+  uint64_t* k_empty = bars + 5;                          // [stage]
+  uint64_t* s_full = bars + 7;                           // [query tile]
+  uint64_t* p_full = bars + 9;                           // [query tile], 4 arrivals
+  uint64_t* o_final = bars + 11;                         // [query tile]
+  uint64_t* v_empty = bars + 13;                         // [stage]
+  uint64_t* drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * kTile;
+  const int q0 = blockIdx.x * (kQTiles * kTile);
   const int head = blockIdx.y;
   const int n_kv = (P.n + kTile - 1) / kTile;
 
@@ -71,21 +103,22 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(const __grid_const
     for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);
-      mbar_init(&o_done[i], 1);
+      mbar_init(&o_final[i], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch_map(&P.mapQ);
     tma_prefetch_map(&P.mapK);
     tma_prefetch_map(&P.mapV);
   }
-  if (warp == 1) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -94,88 +127,114 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
+    if (warp == 8 && lane == 0) {
       // ------------------------------------------------------------ TMA producer
       const int qc = P.q_col0 + head * kHeadDim;
       const int kc = P.k_col0 + head * kHeadDim;
       const int vc = P.v_col0 + head * kHeadDim;
-      mbar_arrive_expect_tx(q_full, kTileBytes);
-      tma_load_2d(sQ, &P.mapQ, q_full, qc, q0);
-      tma_load_2d(sQ + kBoxBytes, &P.mapQ, q_full, qc + kBox, q0);
-      uint32_t armed_k = 0, armed_v = 0, parity = 0;
+      mbar_arrive_expect_tx(q_full, kQTiles * kTileBytes);
+      for (int t = 0; t < kQTiles; ++t) {
+        tma_load_2d(sQ + t * kTileBytes, &P.mapQ, q_full, qc, q0 + t * kTile);
+        tma_load_2d(sQ + t * kTileBytes + kBoxBytes, &P.mapQ, q_full, qc + kBox, q0 + t * kTile);
+      }
+      uint32_t armed = 0, parity = 0;
       bool ok = true;
       for (int j = 0; j < n_kv; ++j) {
         const int st = j & 1;
         const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(&kv_empty[st], ph ^ 1u, abort_flag)) {
+        const int r0 = j * kTile;
+        if (!mbar_wait(&k_empty[st], ph ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
-        const int r0 = j * kTile;
         mbar_arrive_expect_tx(&k_full[st], kTileBytes);
         tma_load_2d(sK + st * kTileBytes, &P.mapK, &k_full[st], kc, r0);
         tma_load_2d(sK + st * kTileBytes + kBoxBytes, &P.mapK, &k_full[st], kc + kBox, r0);
+        armed |= 1u << st;
+        parity = (parity & ~(1u << st)) | (ph << st);
+        if (!mbar_wait(&v_empty[st], ph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
         mbar_arrive_expect_tx(&v_full[st], kTileBytes);
         tma_load_2d(sV + st * kTileBytes, &P.mapV, &v_full[st], vc, r0);
         tma_load_2d(sV + st * kTileBytes + kBoxBytes, &P.mapV, &v_full[st], vc + kBox, r0);
-        armed_k |= 1u << st;
-        armed_v |= 1u << st;
-        parity = (parity & ~(1u << st)) | (ph << st);
+        armed |= 1u << (st + 2);
       }
       mbar_drain(q_full, 0);
       if (!ok) {
         atomicExch(&g_attn_error, kErrTimeoutProducer);
         for (int s = 0; s < 2; ++s) {
-          if (armed_k & (1u << s)) mbar_drain(&k_full[s], (parity >> s) & 1u);
-          if (armed_v & (1u << s)) mbar_drain(&v_full[s], (parity >> s) & 1u);
+          if (armed & (1u << s)) mbar_drain(&k_full[s], (parity >> s) & 1u);
+          if (armed & (1u << (s + 2))) mbar_drain(&v_full[s], (parity >> s) & 1u);
         }
       }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
+    } else if (warp == 9 && lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       const uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, 0, 0);      // Q, K both K-major
       const uint32_t idesc_o = idesc_bf16_f32(kTile, kHeadDim, 0, 1);   // P K-major (TMEM), V MN-major
-      bool ok = mbar_wait(q_full, 0, abort_flag);
       const uint32_t q_addr = smem_u32(sQ);
-      for (int j = 0; ok && j <= n_kv; ++j) {
-        if (j < n_kv) {
-          const int st = j & 1;
-          if (!mbar_wait(&k_full[st], (j >> 1) & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(sK + st * kTileBytes);
-          const uint32_t s_tmem = tmem_base + static_cast<uint32_t>(st * kTile);
+      auto issue_s = [&](int t, int j) {        // S_t(j) = Q_t K_j^T
+        const uint32_t k_addr = smem_u32(sK + (j & 1) * kTileBytes);
+        const uint32_t qa = q_addr + t * kTileBytes;
+        const uint32_t s_tmem = tmem_base + static_cast<uint32_t>(t * kTile);
 #pragma unroll
-          for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-            mma_ss(s_tmem, sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024), idesc_s,
-                   kk != 0 ? 1u : 0u);
-          }
-          mma_commit(&s_full[st]);
+        for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+          mma_ss(s_tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024), idesc_s,
+                 kk != 0 ? 1u : 0u);
         }
-        if (j >= 1) {
-          const int jp = j - 1;
-          const int st = jp & 1;
-          if (!mbar_wait(&p_full[st], (jp >> 1) & 1, abort_flag) ||
-              !mbar_wait(&v_full[st], (jp >> 1) & 1, abort_flag)) {
+        mma_commit(&s_full[t]);
+      };
+      auto issue_pv = [&](int t, int j) {       // O_t += P_t(j) V_j, P from TMEM
+        const uint32_t v_addr = smem_u32(sV + (j & 1) * kTileBytes);
+        const uint32_t p_tmem = tmem_base + static_cast<uint32_t>(t * kTile);
+        const uint32_t o_tmem = tmem_base + kOCol + static_cast<uint32_t>(t * kTile);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(o_tmem, p_tmem + kk * 8, sw128_desc(v_addr + kk * 2048, kBoxBytes, 1024), idesc_o,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&k_full[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        mma_commit(&k_empty[0]);                 // K_0 is no longer read
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int st = j & 1;
+        const uint32_t ph = j & 1;
+        if (!mbar_wait(&p_full[0], ph, abort_flag) || !mbar_wait(&v_full[st], (j >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv(0, j);
+        if (j + 1 < n_kv) {
+          if (!mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t v_addr = smem_u32(sV + st * kTileBytes);
-          const uint32_t p_tmem = tmem_base + static_cast<uint32_t>(st * kTile);
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            // A: 16 keys of P = 8 packed columns; B: 16 rows of V (2 x 8-row groups) per step
-            mma_ts(tmem_base + kOCol, p_tmem + kk * 8, sw128_desc(v_addr + kk * 2048, kBoxBytes, 1024),
-                   idesc_o, (jp > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(&o_done[jp & 1]);
-          mma_commit(&kv_empty[st]);
+          issue_s(0, j + 1);
+        } else {
+          mma_commit(&o_final[0]);
+        }
+        if (!mbar_wait(&p_full[1], ph, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv(1, j);
+        mma_commit(&v_empty[st]);                // V_j is no longer read
+        if (j + 1 < n_kv) {
+          issue_s(1, j + 1);
+          mma_commit(&k_empty[(j + 1) & 1]);     // K_{j+1} is no longer read
+        } else {
+          mma_commit(&o_final[1]);
         }
       }
       if (!ok) atomicExch(&g_attn_error, kErrTimeoutMma);
@@ -183,22 +242,24 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(const __grid_const
       mbar_drain(drain, 0);
     }
   } else {
-    // -------------------------------------------------------------- softmax warps 2..5
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    // -------------------------------------------------------------- softmax, warpgroup t = query tile t
+    const int t = warp >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t s_addr = tmem_base + lane_addr + static_cast<uint32_t>(t * kTile);
+    const uint32_t o_addr = tmem_base + lane_addr + kOCol + static_cast<uint32_t>(t * kTile);
     const float sl2 = P.scale_log2;
-    float m_run = -INFINITY;      // running max, log2 domain (scaled)
+    float m_run = -INFINITY;      // running max of the scaled scores, log2 domain
     float l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(&s_full[st], (j >> 1) & 1, abort_flag)) {
+      if (!mbar_wait(&s_full[t], j & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t s_addr = tmem_base + lane_addr + static_cast<uint32_t>(st * kTile);
       uint32_t s[kTile];
       tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
       tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
@@ -206,42 +267,40 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(const __grid_const
       tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tmem_ld_wait();
       const int valid = P.n - j * kTile;          // keys of this tile inside the sequence
-      float mx = -INFINITY;
+      if (valid < kTile) {
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) {
-        float x = __uint_as_float(s[c]) * sl2;
-        if (c >= valid) x = -INFINITY;
-        s[c] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+        for (int c = 0; c < kTile; ++c)
+          if (c >= valid) s[c] = __float_as_uint(-INFINITY);
       }
-      const bool grow = mx > m_run + kRescaleThreshold;
-      const bool warp_grow = __any_sync(0xffffffffu, grow);
-      float m_use = m_run;
-      if (warp_grow) m_use = fmaxf(m_run, mx);
-      const float alpha = ex2(m_run - m_use);   // 0 on the first tile, 1 when not moved
+      float mx = __uint_as_float(s[0]);
+#pragma unroll
+      for (int c = 1; c < kTile; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+      const float mxs = mx * sl2;
+      const bool warp_grow = __any_sync(0xffffffffu, mxs > m_run + kRescaleThreshold);
+      const float m_use = warp_grow ? fmaxf(m_run, mxs) : m_run;
+      const float alpha = ex2(m_run - m_use);     // 0 on the first tile, 1 when not moved
+      const float neg_m = -m_use;
       float sum = 0.0f;
-      uint32_t pk[kTile / 2];
 #pragma unroll
-      for (int c = 0; c < kTile; c += 2) {
-        const float p0 = ex2(__uint_as_float(s[c]) - m_use);
-        const float p1 = ex2(__uint_as_float(s[c + 1]) - m_use);
+      for (int c = 0; c < kTile; c += 2) {        // P packed in place over the first half of s
+        const float x0 = fmaf(__uint_as_float(s[c]), sl2, neg_m);
+        const float x1 = fmaf(__uint_as_float(s[c + 1]), sl2, neg_m);
+        float p0, p1;
+        if (kPolyEvery > 0 && (c / 2) % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+          p0 = ex2_poly(x0);
+          p1 = ex2_poly(x1);
+        } else {
+          p0 = ex2(x0);
+          p1 = ex2(x1);
+        }
         sum += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
+        s[c / 2] = pack_bf16x2(p0, p1);
       }
-      tmem_st32(s_addr + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(s_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+      tmem_st32(s_addr + 0, *reinterpret_cast<const uint32_t(*)[32]>(&s[0]));
+      tmem_st32(s_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(&s[32]));
       l_run = l_run * alpha + sum;
       if (warp_grow && j > 0) {
-        // O holds sum_{i<j} P_i V_i once PV_{j-1} retired; rescale it by alpha
-        // Softmax warps may skip these waits, so PV completions are split over two
-        // barriers by parity of the PV index: the wanted phase is then never more
-        // than one phase behind the barrier, which a parity wait requires.
-        if (!mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t o_addr = tmem_base + lane_addr + kOCol;
+        // S_t(j) was issued after PV_t(j-1), so O_t is complete up to tile j-1 here
 #pragma unroll 1
         for (int c = 0; c < kHeadDim; c += 32) {
           uint32_t o[32];
@@ -256,13 +315,12 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(const __grid_const
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[st]);
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
-    if (ok && mbar_wait(&o_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag)) {
+    if (ok && mbar_wait(&o_final[t], 0, abort_flag)) {
       tc_fence_after();
       const float inv_l = 1.0f / l_run;
-      const int qrow = q0 + row;
-      const uint32_t o_addr = tmem_base + lane_addr + kOCol;
+      const int qrow = q0 + t * kTile + row;
 #pragma unroll 1
       for (int c = 0; c < kHeadDim; c += 32) {
         uint32_t o[32];
@@ -288,7 +346,7 @@ __global__ void __launch_bounds__(192, 1) attention_tc_kernel(const __grid_const
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
@@ -305,9 +363,9 @@ cudaError_t attention_launch(const AttnParams& P, cudaStream_t stream) {
     attr_set = true;
   }
   if (P.n <= 0 || P.heads <= 0) return cudaSuccess;
-  dim3 grid((P.n + kTile - 1) / kTile, P.heads);
+  dim3 grid((P.n + kQTiles * kTile - 1) / (kQTiles * kTile), P.heads);
   count_launch();
-  attention_tc_kernel<<<grid, 192, kSmemBytes, stream>>>(P);
+  attention_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(P);
   return cudaGetLastError();
 }
 
