@@ -153,6 +153,16 @@ FLUX_API int flux_joint_attention(const uint16_t *q, const uint16_t *k, const ui
 FLUX_API int flux_linear(const uint16_t *a, int m, int k, int lda, const uint16_t *w, int n, const uint16_t *bias, int mode,
                 void *out, int ldo, const float *gate, void *stream);
 
+/* Fused qkv projection on the tensor cores: qkv = A W^T + bias, bf16 [m, 3*heads*128] in
+ * q | k | v order (W bf16 [3*heads*128, k], bias bf16), then each 128-value head of q and k
+ * is RMS-normalised (eps), scaled by q_gain / k_gain (bf16 [128]) and rotated by rows
+ * table_row0 .. table_row0+m-1 of a flux_rope_table table ("Entkoppelte Vorverarbeitung und
+ * gemeinsame Attention-Blöcke": QK-RMSNorm before attention; "Modulation pro Token-Typ,
+ * Flow-Map-Destillation und 4D-RoPE": 4-axis RoPE).  k % 64 == 0, heads even. */
+FLUX_API int flux_qkv_projection(const uint16_t *a, int m, int k, int lda, const uint16_t *w, const uint16_t *bias,
+                                 int heads, const uint16_t *q_gain, const uint16_t *k_gain, const float *table,
+                                 int table_row0, float eps, uint16_t *qkv, void *stream);
+
 /* y = LayerNorm(x) * (1 + scale) + shift per row (no learned affine; eps):
  * x fp32 [rows, dim], shift/scale fp32 [dim], y bf16 [rows, dim]
  * ("Modulation pro Token-Typ, Flow-Map-Destillation und 4D-RoPE"). */

@@ -52,6 +52,7 @@ _SIGS = {
     "flux_unpack_latents": (_I, [_P, _P, _I, _I, _P]),
     "flux_joint_attention": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P]),
     "flux_linear": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _P]),
+    "flux_qkv_projection": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _I, _F, _P, _P]),
     "flux_layernorm_modulate": (_I, [_P, _P, _I, _I, _P, _P, _F, _P]),
     "flux_rope_table": (_I, [_P, _I, _I, _I, _I, _I, _F, _P]),
     "flux_qk_rmsnorm_rope": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _F, _P]),
@@ -227,6 +228,19 @@ def flux_linear(a, w, bias, mode, out, gate=None, stream=None):
                              ctypes.c_void_p(out.data_ptr()), out.stride(0),
                              _ptr(gate, torch.float32, "gate"), _stream(stream)))
     return out
+
+
+def flux_qkv_projection(a, w, bias, heads, q_gain, k_gain, table, qkv, table_row0=0, eps=1e-6, stream=None):
+    """qkv = a w^T + bias with QK-RMSNorm + RoPE fused on the q and k heads (see fluxdit.h)."""
+    import torch
+    m, k = a.shape
+    if a.stride(1) != 1:
+        raise ValueError("a must have unit column stride")
+    _check(lib().flux_qkv_projection(ctypes.c_void_p(a.data_ptr()), m, k, a.stride(0), _bits(w, "w"),
+                                     _bits(bias, "bias"), heads, _bits(q_gain, "q_gain"), _bits(k_gain, "k_gain"),
+                                     _ptr(table, torch.float32, "table"), table_row0, float(eps), _bits(qkv, "qkv"),
+                                     _stream(stream)))
+    return qkv
 
 
 def flux_layernorm_modulate(x, y, shift, scale, eps=1e-6, stream=None):

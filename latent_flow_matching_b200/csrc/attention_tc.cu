@@ -8,7 +8,7 @@
 // take turns on the tensor core, 12 warps in three warpgroups:
 //   warps 0..3   softmax of tile A   (one thread per query row)
 //   warps 4..7   softmax of tile B
-//   warp 8       TMA: Q_A, Q_B once, then K_j / V_j into a 2-deep ring
+//   warp 8       TMA: Q_A, Q_B once, then K_j / V_j into 2- and 3-deep rings
 //   warp 9       one thread issues tcgen05.mma in the order
 //                  S_A(0) S_B(0) | PV_A(0) S_A(1) PV_B(0) S_B(1) | PV_A(1) S_A(2) ...
 //                so the tensor core works on one tile while the other tile's
@@ -37,9 +37,10 @@ constexpr int kQTiles = 2;          // query tiles per CTA
 constexpr int kBox = 64;            // 64 bf16 = 128 bytes: one swizzle row
 constexpr int kBoxBytes = kTile * kBox * 2;          // 16 KB
 constexpr int kTileBytes = 2 * kBoxBytes;            // 32 KB: 128 rows x 128 dims
-constexpr int kStages = 2;
+constexpr int kStagesK = 2;        // K is released right after its second QK^T, so 2 slots suffice
+constexpr int kStagesV = 3;        // V is held until the second PV; a third slot hides the L2 round trip
 constexpr int kThreads = 384;
-constexpr int kSmemBytes = kTileBytes * (kQTiles + 2 * kStages) + 1024 + 256;
+constexpr int kSmemBytes = kTileBytes * (kQTiles + kStagesK + kStagesV) + 1024 + 256;   // 225 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOCol = 256;
 constexpr float kRescaleThreshold = 8.0f;
@@ -77,19 +78,19 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                                    // kQTiles tiles
-  uint8_t* sK = sQ + kQTiles * kTileBytes;               // kStages tiles
-  uint8_t* sV = sK + kStages * kTileBytes;               // kStages tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kStages * kTileBytes);
+  uint8_t* sK = sQ + kQTiles * kTileBytes;               // kStagesK tiles
+  uint8_t* sV = sK + kStagesK * kTileBytes;              // kStagesV tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kStagesV * kTileBytes);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;                           // [stage]
-  uint64_t* v_full = bars + 3;                           // [stage]
-  uint64_t* k_empty = bars + 5;                          // [stage]
-  uint64_t* s_full = bars + 7;                           // [query tile]
-  uint64_t* p_full = bars + 9;                           // [query tile], 4 arrivals
-  uint64_t* o_final = bars + 11;                         // [query tile]
-  uint64_t* v_empty = bars + 13;                         // [stage]
-  uint64_t* drain = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* k_full = q_full + 1;                         // [kStagesK]
+  uint64_t* k_empty = k_full + kStagesK;                 // [kStagesK]
+  uint64_t* v_full = k_empty + kStagesK;                 // [kStagesV]
+  uint64_t* v_empty = v_full + kStagesV;                 // [kStagesV]
+  uint64_t* s_full = v_empty + kStagesV;                 // [query tile]
+  uint64_t* p_full = s_full + 2;                         // [query tile], 4 arrivals
+  uint64_t* o_final = p_full + 2;                        // [query tile]
+  uint64_t* drain = o_final + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -100,11 +101,15 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kStagesK; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&v_full[i], 1);
       mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kStagesV; ++i) {
+      mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);
       mbar_init(&o_final[i], 1);
@@ -139,37 +144,38 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
         tma_load_2d(sQ + t * kTileBytes, &P.mapQ, q_full, qc, q0 + t * kTile);
         tma_load_2d(sQ + t * kTileBytes + kBoxBytes, &P.mapQ, q_full, qc + kBox, q0 + t * kTile);
       }
-      uint32_t armed = 0, parity = 0;
+      uint32_t armed_k = 0, armed_v = 0, par_k = 0, par_v = 0;   // per slot: armed once / parity of last arming
       bool ok = true;
       for (int j = 0; j < n_kv; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
         const int r0 = j * kTile;
-        if (!mbar_wait(&k_empty[st], ph ^ 1u, abort_flag)) {
+        const int sk = j % kStagesK, sv = j % kStagesV;
+        const uint32_t pk = (j / kStagesK) & 1, pv = (j / kStagesV) & 1;
+        if (!mbar_wait(&k_empty[sk], pk ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&k_full[st], kTileBytes);
-        tma_load_2d(sK + st * kTileBytes, &P.mapK, &k_full[st], kc, r0);
-        tma_load_2d(sK + st * kTileBytes + kBoxBytes, &P.mapK, &k_full[st], kc + kBox, r0);
-        armed |= 1u << st;
-        parity = (parity & ~(1u << st)) | (ph << st);
-        if (!mbar_wait(&v_empty[st], ph ^ 1u, abort_flag)) {
+        mbar_arrive_expect_tx(&k_full[sk], kTileBytes);
+        tma_load_2d(sK + sk * kTileBytes, &P.mapK, &k_full[sk], kc, r0);
+        tma_load_2d(sK + sk * kTileBytes + kBoxBytes, &P.mapK, &k_full[sk], kc + kBox, r0);
+        armed_k |= 1u << sk;
+        par_k = (par_k & ~(1u << sk)) | (pk << sk);
+        if (!mbar_wait(&v_empty[sv], pv ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&v_full[st], kTileBytes);
-        tma_load_2d(sV + st * kTileBytes, &P.mapV, &v_full[st], vc, r0);
-        tma_load_2d(sV + st * kTileBytes + kBoxBytes, &P.mapV, &v_full[st], vc + kBox, r0);
-        armed |= 1u << (st + 2);
+        mbar_arrive_expect_tx(&v_full[sv], kTileBytes);
+        tma_load_2d(sV + sv * kTileBytes, &P.mapV, &v_full[sv], vc, r0);
+        tma_load_2d(sV + sv * kTileBytes + kBoxBytes, &P.mapV, &v_full[sv], vc + kBox, r0);
+        armed_v |= 1u << sv;
+        par_v = (par_v & ~(1u << sv)) | (pv << sv);
       }
       mbar_drain(q_full, 0);
       if (!ok) {
         atomicExch(&g_attn_error, kErrTimeoutProducer);
-        for (int s = 0; s < 2; ++s) {
-          if (armed & (1u << s)) mbar_drain(&k_full[s], (parity >> s) & 1u);
-          if (armed & (1u << (s + 2))) mbar_drain(&v_full[s], (parity >> s) & 1u);
-        }
+        for (int i = 0; i < kStagesK; ++i)
+          if (armed_k & (1u << i)) mbar_drain(&k_full[i], (par_k >> i) & 1u);
+        for (int i = 0; i < kStagesV; ++i)
+          if (armed_v & (1u << i)) mbar_drain(&v_full[i], (par_v >> i) & 1u);
       }
     } else if (warp == 9 && lane == 0) {
       // ------------------------------------------------------------ MMA issuer
@@ -177,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
       const uint32_t idesc_o = idesc_bf16_f32(kTile, kHeadDim, 0, 1);   // P K-major (TMEM), V MN-major
       const uint32_t q_addr = smem_u32(sQ);
       auto issue_s = [&](int t, int j) {        // S_t(j) = Q_t K_j^T
-        const uint32_t k_addr = smem_u32(sK + (j & 1) * kTileBytes);
+        const uint32_t k_addr = smem_u32(sK + (j % kStagesK) * kTileBytes);
         const uint32_t qa = q_addr + t * kTileBytes;
         const uint32_t s_tmem = tmem_base + static_cast<uint32_t>(t * kTile);
 #pragma unroll
@@ -189,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
         mma_commit(&s_full[t]);
       };
       auto issue_pv = [&](int t, int j) {       // O_t += P_t(j) V_j, P from TMEM
-        const uint32_t v_addr = smem_u32(sV + (j & 1) * kTileBytes);
+        const uint32_t v_addr = smem_u32(sV + (j % kStagesV) * kTileBytes);
         const uint32_t p_tmem = tmem_base + static_cast<uint32_t>(t * kTile);
         const uint32_t o_tmem = tmem_base + kOCol + static_cast<uint32_t>(t * kTile);
 #pragma unroll
@@ -205,16 +211,16 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
         mma_commit(&k_empty[0]);                 // K_0 is no longer read
       }
       for (int j = 0; ok && j < n_kv; ++j) {
-        const int st = j & 1;
         const uint32_t ph = j & 1;
-        if (!mbar_wait(&p_full[0], ph, abort_flag) || !mbar_wait(&v_full[st], (j >> 1) & 1, abort_flag)) {
+        if (!mbar_wait(&p_full[0], ph, abort_flag) ||
+            !mbar_wait(&v_full[j % kStagesV], (j / kStagesV) & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         issue_pv(0, j);
         if (j + 1 < n_kv) {
-          if (!mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag)) {
+          if (!mbar_wait(&k_full[(j + 1) % kStagesK], ((j + 1) / kStagesK) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -229,10 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
         }
         tc_fence_after();
         issue_pv(1, j);
-        mma_commit(&v_empty[st]);                // V_j is no longer read
+        mma_commit(&v_empty[j % kStagesV]);      // V_j is no longer read
         if (j + 1 < n_kv) {
           issue_s(1, j + 1);
-          mma_commit(&k_empty[(j + 1) & 1]);     // K_{j+1} is no longer read
+          mma_commit(&k_empty[(j + 1) % kStagesK]);   // K_{j+1} is no longer read
         } else {
           mma_commit(&o_final[1]);
         }
@@ -272,15 +278,20 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
         for (int c = 0; c < kTile; ++c)
           if (c >= valid) s[c] = __float_as_uint(-INFINITY);
       }
-      float mx = __uint_as_float(s[0]);
+      // row max as 8 independent partial maxima (a single chain would serialise 128 dependent ops)
+      float mp[8];
 #pragma unroll
-      for (int c = 1; c < kTile; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+      for (int i = 0; i < 8; ++i) mp[i] = __uint_as_float(s[i]);
+#pragma unroll
+      for (int c = 8; c < kTile; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(s[c]));
+      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
       const float mxs = mx * sl2;
       const bool warp_grow = __any_sync(0xffffffffu, mxs > m_run + kRescaleThreshold);
       const float m_use = warp_grow ? fmaxf(m_run, mxs) : m_run;
       const float alpha = ex2(m_run - m_use);     // 0 on the first tile, 1 when not moved
       const float neg_m = -m_use;
-      float sum = 0.0f;
+      float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};     // 8 independent partial sums
 #pragma unroll
       for (int c = 0; c < kTile; c += 2) {        // P packed in place over the first half of s
         const float x0 = fmaf(__uint_as_float(s[c]), sl2, neg_m);
@@ -293,9 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
           p0 = ex2(x0);
           p1 = ex2(x1);
         }
-        sum += p0 + p1;
+        sp[(c / 2) & 7] += p0 + p1;
         s[c / 2] = pack_bf16x2(p0, p1);
       }
+      const float sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
       tmem_st32(s_addr + 0, *reinterpret_cast<const uint32_t(*)[32]>(&s[0]));
       tmem_st32(s_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(&s[32]));
       l_run = l_run * alpha + sum;

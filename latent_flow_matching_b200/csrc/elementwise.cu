@@ -84,47 +84,58 @@ __global__ void cast_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __r
 }
 
 // ------------------------------------------------------------------ LayerNorm + adaLN modulation
-// One warp per row; the row stays in registers (V float4 per lane, dim = 128 V).
-template <int V>
+// One 256-thread CTA per row: each thread keeps VPT float4 of the row in registers (dim = 1024 VPT),
+// mean and variance come from two block reductions, so many CTAs stay resident per SM.
+template <int VPT>
 __global__ void __launch_bounds__(256) ln_mod_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y,
                                                      int rows, int split, const float* __restrict__ sh0,
                                                      const float* __restrict__ sc0, const float* __restrict__ sh1,
                                                      const float* __restrict__ sc1, float eps) {
-  constexpr int dim = 128 * V;
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= rows) return;
-  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(warp) * dim);
-  float4 v[V];
+  constexpr int dim = 1024 * VPT;
+  __shared__ float red[2][8];
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(row) * dim);
+  float4 v[VPT];
   float s = 0.f;
 #pragma unroll
-  for (int i = 0; i < V; ++i) {
-    v[i] = __ldcs(xr + i * 32 + lane);
+  for (int i = 0; i < VPT; ++i) {
+    v[i] = __ldcs(xr + i * 256 + tid);
     s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) red[0][warp] = s;
+  __syncthreads();
+  s = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) s += red[0][w];
   const float mean = s * (1.0f / dim);
   float q = 0.f;
 #pragma unroll
-  for (int i = 0; i < V; ++i) {
+  for (int i = 0; i < VPT; ++i) {
     const float a = v[i].x - mean, b = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
     q += (a * a + b * b) + (c * c + d * d);
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-  const float rstd = rsqrtf(q * (1.0f / dim) + eps);
-  const float4* shp = reinterpret_cast<const float4*>(warp < split ? sh0 : sh1);
-  const float4* scp = reinterpret_cast<const float4*>(warp < split ? sc0 : sc1);
-  uint2* yr = reinterpret_cast<uint2*>(y + static_cast<size_t>(warp) * dim);
+  if (lane == 0) red[1][warp] = q;
+  __syncthreads();
+  q = 0.f;
 #pragma unroll
-  for (int i = 0; i < V; ++i) {
-    const float4 sh = __ldg(shp + i * 32 + lane), sc = __ldg(scp + i * 32 + lane);
+  for (int w = 0; w < 8; ++w) q += red[1][w];
+  const float rstd = rsqrtf(q * (1.0f / dim) + eps);
+  const float4* shp = reinterpret_cast<const float4*>(row < split ? sh0 : sh1);
+  const float4* scp = reinterpret_cast<const float4*>(row < split ? sc0 : sc1);
+  uint2* yr = reinterpret_cast<uint2*>(y + static_cast<size_t>(row) * dim);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const float4 sh = __ldg(shp + i * 256 + tid), sc = __ldg(scp + i * 256 + tid);
     const float a = (v[i].x - mean) * rstd * (1.f + sc.x) + sh.x;
     const float b = (v[i].y - mean) * rstd * (1.f + sc.y) + sh.y;
     const float c = (v[i].z - mean) * rstd * (1.f + sc.z) + sh.z;
     const float d = (v[i].w - mean) * rstd * (1.f + sc.w) + sh.w;
-    yr[i * 32 + lane] = make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
+    yr[i * 256 + tid] = make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
   }
 }
 
@@ -315,12 +326,12 @@ cudaError_t ln_modulate_launch(const float* x, __nv_bfloat16* y, int rows, int d
                                const float* scale0, const float* shift1, const float* scale1, float eps,
                                cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  const int grid = (rows + 7) / 8;
   count_launch();
   if (dim == 3072)
-    ln_mod_kernel<24><<<grid, 256, 0, s>>>(x, y, rows, split, shift0, scale0, shift1, scale1, eps);
+    ln_mod_kernel<3><<<rows, 256, 0, s>>>(x, y, rows, split, shift0, scale0, shift1, scale1, eps);
   else
-    ln_mod_generic_kernel<<<grid, 256, 0, s>>>(x, y, rows, dim, split, shift0, scale0, shift1, scale1, eps);
+    ln_mod_generic_kernel<<<(rows + 7) / 8, 256, 0, s>>>(x, y, rows, dim, split, shift0, scale0, shift1, scale1,
+                                                          eps);
   return cudaGetLastError();
 }
 

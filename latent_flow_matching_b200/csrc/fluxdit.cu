@@ -381,8 +381,8 @@ static int create_impl(const void* blob, size_t blob_bytes, const flux_dit_confi
   m->t_w1 = W("time_in.w1"); m->t_b1 = W("time_in.b1");
   m->t_w2 = W("time_in.w2"); m->t_b2 = W("time_in.b2");
   m->img_b = W("img_in.b"); m->txt_b = W("txt_in.b"); m->fin_b = W("final.out.b");
-  wmap(&m->m_img_in, W("img_in.w"), D, c.in_ch, 256);
-  wmap(&m->m_txt_in, W("txt_in.w"), D, c.txt_dim, 256);
+  wmap(&m->m_img_in, W("img_in.w"), D, c.in_ch, 128);
+  wmap(&m->m_txt_in, W("txt_in.w"), D, c.txt_dim, 128);
   wmap(&m->m_fin, W("final.out.w"), c.in_ch, D, 128);
   m->fin_mod_off = MOD("final.mod.w");
   m->dbl.resize(2 * c.n_double);
@@ -393,10 +393,10 @@ static int create_impl(const void* blob, size_t blob_bytes, const flux_dit_confi
       sw.qkv_b = W(p + "qkv.b"); sw.q_gain = W(p + "q_gain"); sw.k_gain = W(p + "k_gain");
       sw.proj_b = W(p + "proj.b"); sw.mlp_in_b = W(p + "mlp_in.b"); sw.mlp_out_b = W(p + "mlp_out.b");
       sw.mod_off = MOD(p + "mod.w");
-      wmap(&sw.m_qkv, W(p + "qkv.w"), 3 * D, D, 256);
-      wmap(&sw.m_proj, W(p + "proj.w"), D, D, 256);
-      wmap(&sw.m_mlp_in, W(p + "mlp_in.w"), 2 * F, D, 256);
-      wmap(&sw.m_mlp_out, W(p + "mlp_out.w"), D, F, 256);
+      wmap(&sw.m_qkv, W(p + "qkv.w"), 3 * D, D, 128);
+      wmap(&sw.m_proj, W(p + "proj.w"), D, D, 128);
+      wmap(&sw.m_mlp_in, W(p + "mlp_in.w"), 2 * F, D, 128);
+      wmap(&sw.m_mlp_out, W(p + "mlp_out.w"), D, F, 128);
     }
   m->sgl.resize(c.n_single);
   for (int i = 0; i < c.n_single; ++i) {
@@ -407,9 +407,9 @@ static int create_impl(const void* blob, size_t blob_bytes, const flux_dit_confi
     sw.qkv_b = l1b; sw.mlp_b = l1b + 3 * D;
     sw.q_gain = W(p + "q_gain"); sw.k_gain = W(p + "k_gain"); sw.lin2_b = W(p + "lin2.b");
     sw.mod_off = MOD(p + "mod.w");
-    wmap(&sw.m_qkv, l1, 3 * D, D, 256);
-    wmap(&sw.m_mlp, l1 + 3 * D * D, 2 * F, D, 256);
-    wmap(&sw.m_lin2, W(p + "lin2.w"), D, D + F, 256);
+    wmap(&sw.m_qkv, l1, 3 * D, D, 128);
+    wmap(&sw.m_mlp, l1 + 3 * D * D, 2 * F, D, 128);
+    wmap(&sw.m_lin2, W(p + "lin2.w"), D, D + F, 128);
   }
   if (!maps_ok) return cleanup(FLUX_EIO, "cuTensorMapEncodeTiled failed for a weight tensor");
   m->act_double = c.n_double;
@@ -511,6 +511,18 @@ static void problem(GemmParams& P, int i, const CUtensorMap& a, const CUtensorMa
   pr.M = M; pr.N = N; pr.K = K; pr.mode = mode; pr.out = out; pr.ldo = ldo; pr.bias = bias; pr.gate = gate;
 }
 
+// Make problem i a fused qkv + QK-RMSNorm + RoPE projection (rows start at token rope_row0).
+static void qk_fuse(GemmParams& P, int i, const bf16* gq, const bf16* gk, const float2* rope, int rope_row0,
+                    float eps) {
+  GemmProblem& pr = P.prob[i];
+  pr.mode = kEpiQKNormRope;
+  pr.gain_q = gq;
+  pr.gain_k = gk;
+  pr.rope = rope;
+  pr.rope_row0 = rope_row0;
+  pr.eps = eps;
+}
+
 static int run_modulation(flux_dit* m, float t, cudaStream_t s) {
   const flux_dit_config& c = m->cfg;
   const int D = c.hidden;
@@ -558,7 +570,6 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
     FD_LAUNCH(m, kProfOther, 0, 6.0 * nt * c.txt_dim,
               cast_bf16_launch(txt, w.txtb, static_cast<size_t>(nt) * c.txt_dim, s));
   const double ln_bytes = 6.0 * n * D + 16.0 * D, ln_bytes_img = 6.0 * ni * D + 8.0 * D;
-  const double qk_bytes = 8.0 * n * D + 512.0 * n;
   const double at_flops = 4.0 * n * static_cast<double>(n) * D, at_bytes = 8.0 * n * D;
 
   GemmParams P;
@@ -566,7 +577,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
   problem(P, 0, w.a_txtb, m->m_txt_in, nt, D, c.txt_dim, kEpiF32Bias, w.X, D, m->txt_b, nullptr);
   problem(P, 1, w.a_tokb, m->m_img_in, nimg, D, c.in_ch, kEpiF32Bias, w.X + static_cast<size_t>(nt) * D, D, m->img_b,
           nullptr);
-  FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 256, m->num_sms, s));
+  FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
 
   float* Ximg = w.X + static_cast<size_t>(nt) * D;
   bf16* Otxt = w.CC;
@@ -587,23 +598,23 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
     problem(P, 0, w.a_Ytxt, st.m_qkv, nt, 3 * D, D, kEpiBf16Bias, w.QKV, 3 * D, st.qkv_b, nullptr);
     problem(P, 1, w.a_Yimg, si.m_qkv, nimg, 3 * D, D, kEpiBf16Bias, w.QKV + static_cast<size_t>(nt) * 3 * D, 3 * D,
             si.qkv_b, nullptr);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 256, m->num_sms, s));
-    FD_LAUNCH(m, kProfQkNormRope, 0, qk_bytes, qk_norm_rope_launch(w.QKV, n, 3 * D, D, H, nt, st.q_gain, st.k_gain, si.q_gain, si.k_gain, w.rope,
-                                eps_rms, s));
+    qk_fuse(P, 0, st.q_gain, st.k_gain, w.rope, 0, eps_rms);
+    qk_fuse(P, 1, si.q_gain, si.k_gain, w.rope, nt, eps_rms);
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
     FD_LAUNCH(m, kProfAttention, at_flops, at_bytes, attention_launch(A, s));
     P.num_problems = 2;
     problem(P, 0, w.a_Otxt, st.m_proj, nt, D, D, kEpiResidGate, w.X, D, st.proj_b, mt + 2 * D);
     problem(P, 1, w.a_Oimg, si.m_proj, nimg, D, D, kEpiResidGate, Ximg, D, si.proj_b, mi + 2 * D);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 256, m->num_sms, s));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
     FD_LAUNCH(m, kProfLnMod, 0, ln_bytes, ln_modulate_launch(w.X, w.Y, n, D, nt, mt + 3 * D, mt + 4 * D, mi + 3 * D, mi + 4 * D, eps_ln, s));
     P.num_problems = 2;
     problem(P, 0, w.a_Ytxt, st.m_mlp_in, nt, 2 * F, D, kEpiSwiGLU, Otxt + D, D + F, st.mlp_in_b, nullptr);
     problem(P, 1, w.a_Yimg, si.m_mlp_in, nimg, 2 * F, D, kEpiSwiGLU, Oimg + D, D + F, si.mlp_in_b, nullptr);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 256, m->num_sms, s));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
     P.num_problems = 2;
     problem(P, 0, w.a_Htxt, st.m_mlp_out, nt, D, F, kEpiResidGate, w.X, D, st.mlp_out_b, mt + 5 * D);
     problem(P, 1, w.a_Himg, si.m_mlp_out, nimg, D, F, kEpiResidGate, Ximg, D, si.mlp_out_b, mi + 5 * D);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 256, m->num_sms, s));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
   }
   for (int i = 0; i < m->act_single; ++i) {
     const SingleW& sw = m->sgl[i];
@@ -612,13 +623,12 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
     P.num_problems = 2;
     problem(P, 0, w.a_Yall, sw.m_qkv, n, 3 * D, D, kEpiBf16Bias, w.QKV, 3 * D, sw.qkv_b, nullptr);
     problem(P, 1, w.a_Yall, sw.m_mlp, n, 2 * F, D, kEpiSwiGLU, w.CC + D, D + F, sw.mlp_b, nullptr);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 256, m->num_sms, s));
-    FD_LAUNCH(m, kProfQkNormRope, 0, qk_bytes, qk_norm_rope_launch(w.QKV, n, 3 * D, D, H, n, sw.q_gain, sw.k_gain, sw.q_gain, sw.k_gain, w.rope, eps_rms,
-                                s));
+    qk_fuse(P, 0, sw.q_gain, sw.k_gain, w.rope, 0, eps_rms);
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
     FD_LAUNCH(m, kProfAttention, at_flops, at_bytes, attention_launch(A, s));
     P.num_problems = 1;
     problem(P, 0, w.a_CC, sw.m_lin2, n, D, D + F, kEpiResidGate, w.X, D, sw.lin2_b, ms + 2 * D);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 256, m->num_sms, s));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
   }
   const float* mf = mods + m->fin_mod_off;         // shift, scale
   FD_LAUNCH(m, kProfLnMod, 0, ln_bytes_img, ln_modulate_launch(Ximg, w.Y, ni, D, ni, mf, mf + D, mf, mf + D, eps_ln, s));
@@ -741,14 +751,39 @@ int flux_linear(const uint16_t* a, int m, int k, int lda, const uint16_t* w, int
   GemmParams P;
   P.num_problems = 1;
   if (!make_tmap_bf16(&P.mapA[0], a, m, k, static_cast<uint64_t>(lda) * 2, 128) ||
-      !make_tmap_bf16(&P.mapB[0], w, n, k, static_cast<uint64_t>(k) * 2, bn))
+      !make_tmap_bf16(&P.mapB[0], w, n, k, static_cast<uint64_t>(k) * 2, 128))
     return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed");
   GemmProblem& pr = P.prob[0];
   pr = GemmProblem();
   pr.M = m; pr.N = n; pr.K = k; pr.mode = mode; pr.out = out; pr.ldo = ldo;
   pr.bias = reinterpret_cast<const bf16*>(bias);
   pr.gate = gate;
-  FD_CUDA(gemm_launch(P, bn, num_sms_current(), static_cast<cudaStream_t>(stream)));
+  if (bn == 256)
+    FD_CUDA(gemm2_launch(P, num_sms_current(), static_cast<cudaStream_t>(stream)));
+  else
+    FD_CUDA(gemm_launch(P, bn, num_sms_current(), static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_qkv_projection(const uint16_t* a, int m, int k, int lda, const uint16_t* w, const uint16_t* bias, int heads,
+                        const uint16_t* q_gain, const uint16_t* k_gain, const float* table, int table_row0, float eps,
+                        uint16_t* qkv, void* stream) {
+  if (!a || !w || !bias || !q_gain || !k_gain || !table || !qkv) return fail(FLUX_EINVAL, "NULL argument");
+  if (m < 1 || k < 64 || k % 64 || lda < k || lda % 8 || heads < 1 || heads % 2 || table_row0 < 0)
+    return fail(FLUX_EINVAL, "bad shape m=%d k=%d lda=%d heads=%d (heads must be even)", m, k, lda, heads);
+  if (!aligned16(a) || !aligned16(w) || !aligned16(bias) || !aligned16(q_gain) || !aligned16(k_gain) ||
+      !aligned16(table) || !aligned16(qkv))
+    return fail(FLUX_EINVAL, "pointers must be 16-byte aligned");
+  const int n = 3 * heads * 128;
+  GemmParams P;
+  P.num_problems = 1;
+  if (!make_tmap_bf16(&P.mapA[0], a, m, k, static_cast<uint64_t>(lda) * 2, 128) ||
+      !make_tmap_bf16(&P.mapB[0], w, n, k, static_cast<uint64_t>(k) * 2, 128))
+    return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed");
+  problem(P, 0, P.mapA[0], P.mapB[0], m, n, k, kEpiBf16Bias, qkv, n, reinterpret_cast<const bf16*>(bias), nullptr);
+  qk_fuse(P, 0, reinterpret_cast<const bf16*>(q_gain), reinterpret_cast<const bf16*>(k_gain),
+          reinterpret_cast<const float2*>(table), table_row0, eps);
+  FD_CUDA(gemm2_launch(P, num_sms_current(), static_cast<cudaStream_t>(stream)));
   return FLUX_OK;
 }
 
@@ -811,8 +846,9 @@ int flux_device_error(void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   FD_CUDA(cudaStreamSynchronize(s));
   const int g = gemm_read_device_error(s);
+  const int g2 = gemm2_read_device_error(s);
   const int a = attention_read_device_error(s);
-  return g ? g : a;
+  return g ? g : (g2 ? g2 : a);
 }
 
 }  // extern "C"

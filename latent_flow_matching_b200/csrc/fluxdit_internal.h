@@ -10,7 +10,7 @@
 namespace fdit {
 
 // ------------------------------------------------------------------ GEMM
-enum EpiMode : int { kEpiBf16Bias = 0, kEpiF32Bias = 1, kEpiSwiGLU = 2, kEpiResidGate = 3 };
+enum EpiMode : int { kEpiBf16Bias = 0, kEpiF32Bias = 1, kEpiSwiGLU = 2, kEpiResidGate = 3, kEpiQKNormRope = 4 };
 constexpr int kMaxProblems = 4;
 
 struct GemmProblem {
@@ -21,6 +21,14 @@ struct GemmProblem {
   void* out;                      // bf16 or f32 (see mode); kEpiResidGate: the f32 residual
   const __nv_bfloat16* bias;      // [N]
   const float* gate;              // [N], kEpiResidGate only
+  // kEpiQKNormRope (bf16 out, N = 3 * heads * 128 in q | k | v order, BN = 256): each 128-column
+  // head of q and k is RMS-normalised (eps), scaled by its gain and rotated by the RoPE table row
+  // rope_row0 + m; v columns get the plain bias epilogue.
+  const __nv_bfloat16* gain_q;    // [128]
+  const __nv_bfloat16* gain_k;    // [128]
+  const float2* rope;             // (cos, sin) [tokens, 64]
+  int rope_row0;
+  float eps;
 };
 
 struct GemmParams {
@@ -34,6 +42,9 @@ struct GemmParams {
 int gemm_bn_for(int n);
 cudaError_t gemm_launch(GemmParams& P, int bn, int num_sms, cudaStream_t stream);
 int gemm_read_device_error(cudaStream_t stream);
+// CTA-pair variant (cta_group::2, 256 x 256 tiles, W maps with a 128-row box): same problems and epilogues
+cudaError_t gemm2_launch(GemmParams& P, int num_sms, cudaStream_t stream);
+int gemm2_read_device_error(cudaStream_t stream);
 
 // ------------------------------------------------------------------ attention
 struct AttnParams {

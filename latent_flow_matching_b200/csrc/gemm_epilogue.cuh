@@ -1,0 +1,154 @@
+// Fused epilogue shared by the one-CTA (gemm_tc.cu) and CTA-pair (gemm_tc2.cu) tcgen05 GEMMs.
+//
+// Called by one epilogue warp for one accumulator tile; thread i of the warp owns accumulator
+// row m (global row of this problem) whose BN fp32 columns start at TMEM address `tbase`.
+// Every tcgen05.ld is warp-collective, so rows outside the problem still load and only skip
+// their global stores.
+#pragma once
+
+#include "common.cuh"
+#include "fluxdit_internal.h"
+
+namespace fdit {
+
+template <int BN>
+__device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32_t tbase, int m, int n0) {
+  const bool row_ok = m < pr.M;
+  if (pr.mode == kEpiSwiGLU) {
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(pr.out);
+    const int on0 = n0 / 2;                // output column of this tile's first pair
+#pragma unroll 1
+    for (int c = 0; c < BN / 2; c += 32) {
+      uint32_t ra[32], rb[32];
+      tmem_ld32(tbase + c, ra);
+      tmem_ld32(tbase + BN / 2 + c, rb);
+      tmem_ld_wait();
+      if (row_ok && n0 + c < pr.N) {
+        const uint4* ba = reinterpret_cast<const uint4*>(pr.bias + n0 + c);
+        const uint4* bb = reinterpret_cast<const uint4*>(pr.bias + n0 + BN / 2 + c);
+        uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(m) * pr.ldo + on0 + c);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 wa = __ldg(ba + v), wb = __ldg(bb + v);
+          const uint32_t xa[4] = {wa.x, wa.y, wa.z, wa.w}, xb[4] = {wb.x, wb.y, wb.z, wb.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = v * 8 + e * 2;
+            const float a0 = __uint_as_float(ra[j]) + bf16lo(xa[e]);
+            const float a1 = __uint_as_float(ra[j + 1]) + bf16hi(xa[e]);
+            const float b0 = __uint_as_float(rb[j]) + bf16lo(xb[e]);
+            const float b1 = __uint_as_float(rb[j + 1]) + bf16hi(xb[e]);
+            o[e] = pack_bf16x2(silu_f(a0) * b0, silu_f(a1) * b1);
+          }
+          dst[v] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+    }
+  } else if (pr.mode == kEpiQKNormRope && n0 < 2 * (pr.N / 3)) {
+    const bool is_k = n0 >= pr.N / 3;
+    const __nv_bfloat16* gain = is_k ? pr.gain_k : pr.gain_q;
+    const float4* rrow = reinterpret_cast<const float4*>(pr.rope + static_cast<size_t>(pr.rope_row0 + (row_ok ? m : 0)) * 64);
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(pr.out);
+#pragma unroll 1
+    for (int hh = 0; hh < BN / 128; ++hh) {
+      const uint32_t hb = tbase + hh * 128;
+      const __nv_bfloat16* bh = pr.bias + n0 + hh * 128;
+      float ss = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 128; c += 32) {           // pass 1: sum of squares of the head
+        uint32_t r[32];
+        tmem_ld32(hb + c, r);
+        tmem_ld_wait();
+        const uint4* bsrc = reinterpret_cast<const uint4*>(bh + c);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 w = __ldg(bsrc + v);
+          const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float a0 = __uint_as_float(r[v * 8 + e * 2]) + bf16lo(x[e]);
+            const float a1 = __uint_as_float(r[v * 8 + e * 2 + 1]) + bf16hi(x[e]);
+            ss = fmaf(a0, a0, fmaf(a1, a1, ss));
+          }
+        }
+      }
+      const float rstd = rsqrtf(ss * (1.0f / 128.0f) + pr.eps);
+#pragma unroll 1
+      for (int c = 0; c < 128; c += 32) {           // pass 2: normalise, gain, rotate, store
+        uint32_t r[32];
+        tmem_ld32(hb + c, r);
+        tmem_ld_wait();
+        if (!row_ok) continue;
+        const uint4* bsrc = reinterpret_cast<const uint4*>(bh + c);
+        const uint4* gsrc = reinterpret_cast<const uint4*>(gain + c);
+        uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(m) * pr.ldo + n0 + hh * 128 + c);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 w = __ldg(bsrc + v), g = __ldg(gsrc + v);
+          const uint32_t x[4] = {w.x, w.y, w.z, w.w}, gg[4] = {g.x, g.y, g.z, g.w};
+          const float4 cs01 = __ldg(rrow + (c + v * 8) / 4);       // (cos, sin) of pairs p, p+1
+          const float4 cs23 = __ldg(rrow + (c + v * 8) / 4 + 1);   // pairs p+2, p+3
+          const float cs[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
+          const float sn[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float a0 = (__uint_as_float(r[v * 8 + e * 2]) + bf16lo(x[e])) * rstd * bf16lo(gg[e]);
+            const float a1 = (__uint_as_float(r[v * 8 + e * 2 + 1]) + bf16hi(x[e])) * rstd * bf16hi(gg[e]);
+            o[e] = pack_bf16x2(a0 * cs[e] - a1 * sn[e], a0 * sn[e] + a1 * cs[e]);
+          }
+          dst[v] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t r[32];
+      tmem_ld32(tbase + c, r);
+      tmem_ld_wait();
+      const int n = n0 + c;
+      if (!row_ok || n >= pr.N) continue;
+      const uint4* bsrc = reinterpret_cast<const uint4*>(pr.bias + n);
+      float f[32];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 w = __ldg(bsrc + v);
+        const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          f[v * 8 + e * 2] = __uint_as_float(r[v * 8 + e * 2]) + bf16lo(x[e]);
+          f[v * 8 + e * 2 + 1] = __uint_as_float(r[v * 8 + e * 2 + 1]) + bf16hi(x[e]);
+        }
+      }
+      if (pr.mode == kEpiBf16Bias || pr.mode == kEpiQKNormRope) {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(pr.out) +
+                                              static_cast<size_t>(m) * pr.ldo + n);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          dst[v] = make_uint4(pack_bf16x2(f[v * 8 + 0], f[v * 8 + 1]), pack_bf16x2(f[v * 8 + 2], f[v * 8 + 3]),
+                              pack_bf16x2(f[v * 8 + 4], f[v * 8 + 5]), pack_bf16x2(f[v * 8 + 6], f[v * 8 + 7]));
+      } else if (pr.mode == kEpiF32Bias) {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(pr.out) + static_cast<size_t>(m) * pr.ldo + n);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) dst[v] = make_float4(f[v * 4], f[v * 4 + 1], f[v * 4 + 2], f[v * 4 + 3]);
+      } else {                              // kEpiResidGate
+        float4* x = reinterpret_cast<float4*>(static_cast<float*>(pr.out) + static_cast<size_t>(m) * pr.ldo + n);
+        const float4* g = reinterpret_cast<const float4*>(pr.gate + n);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          float4 xv = x[v];
+          const float4 gv = __ldg(g + v);
+          xv.x += gv.x * f[v * 4];
+          xv.y += gv.y * f[v * 4 + 1];
+          xv.z += gv.z * f[v * 4 + 2];
+          xv.w += gv.w * f[v * 4 + 3];
+          x[v] = xv;
+        }
+      }
+    }
+  }
+}
+
+}  // namespace fdit

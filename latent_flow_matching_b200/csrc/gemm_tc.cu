@@ -1,4 +1,6 @@
-// Persistent tcgen05 GEMM for the transformer's linear layers, C = A W^T (+ fused epilogue).
+// Persistent one-CTA tcgen05 GEMM, C = A W^T (+ fused epilogue), 128 x 128 tiles: used for the
+// 128-wide output projection and small standalone calls.  The wide linear layers of the forward
+// run on the CTA-pair kernel (gemm_tc2.cu), which shares this file's epilogue (gemm_epilogue.cuh).
 //
 //   A [M, K] bf16 row-major (activations), W [N, K] bf16 row-major (nn.Linear
 //   [out, in] layout), fp32 accumulation in tensor memory.
@@ -21,10 +23,14 @@
 //                                                          so a tile holds BN/2 a-rows then
 //                                                          the matching BN/2 b-rows)
 //   kEpiResidGate   X_f32   += gate * (acc + bias)         (gated residual add)
+//   kEpiQKNormRope  out_bf16 = rope(rms(acc + bias) * gain) on the q and k heads, acc + bias on v
+//                                                          (fused qkv projection + QK-RMSNorm + RoPE;
+//                                                          a 256-column tile is two whole heads)
 #include <cstdio>
 
 #include "common.cuh"
 #include "fluxdit_internal.h"
+#include "gemm_epilogue.cuh"
 
 namespace fdit {
 
@@ -37,7 +43,7 @@ constexpr int BK = 64;
 
 template <int BN>
 struct GemmCfg {
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int STAGES = 6;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -203,85 +209,7 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(acc * BN);
-      const bool row_ok = m < pr.M;
-      if (pr.mode == kEpiSwiGLU) {
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(pr.out);
-        const int on0 = n0 / 2;                // output column of this tile's first pair
-#pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
-          uint32_t ra[32], rb[32];
-          tmem_ld32(tbase + c, ra);
-          tmem_ld32(tbase + BN / 2 + c, rb);
-          tmem_ld_wait();
-          if (row_ok && n0 + c < pr.N) {
-            const uint4* ba = reinterpret_cast<const uint4*>(pr.bias + n0 + c);
-            const uint4* bb = reinterpret_cast<const uint4*>(pr.bias + n0 + BN / 2 + c);
-            uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(m) * pr.ldo + on0 + c);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const uint4 wa = __ldg(ba + v), wb = __ldg(bb + v);
-              const uint32_t xa[4] = {wa.x, wa.y, wa.z, wa.w}, xb[4] = {wb.x, wb.y, wb.z, wb.w};
-              uint32_t o[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int j = v * 8 + e * 2;
-                const float a0 = __uint_as_float(ra[j]) + bf16lo(xa[e]);
-                const float a1 = __uint_as_float(ra[j + 1]) + bf16hi(xa[e]);
-                const float b0 = __uint_as_float(rb[j]) + bf16lo(xb[e]);
-                const float b1 = __uint_as_float(rb[j + 1]) + bf16hi(xb[e]);
-                o[e] = pack_bf16x2(silu_f(a0) * b0, silu_f(a1) * b1);
-              }
-              dst[v] = make_uint4(o[0], o[1], o[2], o[3]);
-            }
-          }
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          tmem_ld32(tbase + c, r);
-          tmem_ld_wait();
-          const int n = n0 + c;
-          if (!row_ok || n >= pr.N) continue;
-          const uint4* bsrc = reinterpret_cast<const uint4*>(pr.bias + n);
-          float f[32];
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint4 w = __ldg(bsrc + v);
-            const uint32_t x[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              f[v * 8 + e * 2] = __uint_as_float(r[v * 8 + e * 2]) + bf16lo(x[e]);
-              f[v * 8 + e * 2 + 1] = __uint_as_float(r[v * 8 + e * 2 + 1]) + bf16hi(x[e]);
-            }
-          }
-          if (pr.mode == kEpiBf16Bias) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(pr.out) +
-                                                  static_cast<size_t>(m) * pr.ldo + n);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pack_bf16x2(f[v * 8 + 0], f[v * 8 + 1]), pack_bf16x2(f[v * 8 + 2], f[v * 8 + 3]),
-                                  pack_bf16x2(f[v * 8 + 4], f[v * 8 + 5]), pack_bf16x2(f[v * 8 + 6], f[v * 8 + 7]));
-          } else if (pr.mode == kEpiF32Bias) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(pr.out) + static_cast<size_t>(m) * pr.ldo + n);
-#pragma unroll
-            for (int v = 0; v < 8; ++v) dst[v] = make_float4(f[v * 4], f[v * 4 + 1], f[v * 4 + 2], f[v * 4 + 3]);
-          } else {                              // kEpiResidGate
-            float4* x = reinterpret_cast<float4*>(static_cast<float*>(pr.out) + static_cast<size_t>(m) * pr.ldo + n);
-            const float4* g = reinterpret_cast<const float4*>(pr.gate + n);
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              float4 xv = x[v];
-              const float4 gv = __ldg(g + v);
-              xv.x += gv.x * f[v * 4];
-              xv.y += gv.y * f[v * 4 + 1];
-              xv.z += gv.z * f[v * 4 + 2];
-              xv.w += gv.w * f[v * 4 + 3];
-              x[v] = xv;
-            }
-          }
-        }
-      }
+      gemm_epilogue_tile<BN>(pr, tbase, m, n0);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
@@ -336,7 +264,8 @@ cudaError_t gemm_launch(GemmParams& P, int bn, int num_sms, cudaStream_t stream)
   P.num_problems = w;
   P.total_tiles = total;
   if (total == 0) return cudaSuccess;
-  return bn == 128 ? launch_bn<128>(P, num_sms, stream) : launch_bn<256>(P, num_sms, stream);
+  if (bn != 128) return cudaErrorInvalidValue;      // 256-wide tiles run on the CTA-pair kernel
+  return launch_bn<128>(P, num_sms, stream);
 }
 
 int gemm_read_device_error(cudaStream_t stream) {

@@ -110,6 +110,31 @@ def test_qk_rmsnorm_rope(nt, gh, gw, rh, rw):
     assert torch.equal(out[:, 2 * D:], qkv[:, 2 * D:])           # v untouched
 
 
+@pytest.mark.parametrize("m,row0", [(300, 7), (4608, 0)])
+def test_qkv_projection_fused_norm_rope(m, row0):
+    """GEMM with the fused QK-RMSNorm + RoPE epilogue vs linear -> rms_norm -> rope in float64."""
+    heads, k = 24, 3072
+    D = heads * 128
+    nt, gh, gw = 512, 64, 64                       # table for the 1024^2 joint sequence (4608 rows)
+    a = bf(rand((m, k), 60))
+    w = bf(rand((3 * D, k), 61, k ** -0.5))
+    b = bf(rand((3 * D,), 62, 0.5))
+    gq, gk = bf(rand((128,), 63)), bf(rand((128,), 64))
+    table = torch.empty(nt + gh * gw, 64, 2, device=DEV)
+    F.flux_rope_table(table, nt, (gh, gw), (0, 0), 1e4)
+    out = torch.empty(m, 3 * D, device=DEV, dtype=torch.bfloat16)
+    F.flux_qkv_projection(a.to(DEV), w.to(DEV), b.to(DEV), heads, gq.to(DEV), gk.to(DEV), table, out, row0, 1e-6)
+    rows = torch.arange(0, m, max(1, m // 64))
+    y = O.linear(a[rows].double(), w.double(), b.double())
+    ang = O.rope_angles(O.token_positions(nt, gh, gw), 128, 1e4)[row0 + rows]
+    got = out.cpu()[rows]
+    for col, g in ((0, gq), (D, gk)):
+        h = y[:, col:col + D].reshape(len(rows), heads, 128)
+        ref = O.apply_rope(O.rms_norm(h, g.double(), 1e-6), ang).reshape(len(rows), D)
+        assert nmax(got[:, col:col + D], ref) <= TOL
+    assert nmax(got[:, 2 * D:], y[:, 2 * D:]) <= TOL
+
+
 # ---------------------------------------------------------------------------- tcgen05 GEMM
 def interleave_swiglu(w):
     """[a; b] rows -> per 128 output columns: 128 a-rows then 128 b-rows (GEMM order)."""
