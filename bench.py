@@ -120,12 +120,19 @@ def dist_env():
 
 
 def max_over_ranks(x, world):
+    """Max of a host scalar over all ranks (NCCL on the GPU machine; gloo in the CPU tests)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_ms_per_forward(ms_total_max, steps, world):
+    """Whole-job time per forward: every rank runs `steps` independent forwards (replicas)."""
+    return ms_total_max / (steps * world)
 
 
 def barrier(world):
@@ -278,7 +285,7 @@ def run_ours(args, w):
     clk = clocks.stop()
     ms_total = max_over_ranks(ms_total, world)
     ms_step = ms_total / args.steps
-    value = ms_total / (args.steps * world)
+    value = aggregate_ms_per_forward(ms_total, args.steps, world)
 
     # ---- per-kernel device time (CUDA events around every launch of the forward)
     model.profile(True)
@@ -308,7 +315,7 @@ def run_ours(args, w):
         out_pin.copy_(lat_d, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / (args.steps * world)
+    e2e_ms = aggregate_ms_per_forward(max_over_ranks(e0.elapsed_time(e1), world), args.steps, world)
     assert torch.isfinite(out_pin).all()
     h2d = lat_pin.numel() * 4 + txt_pin.numel() * 4
     d2h = out_pin.numel() * 4
