@@ -42,6 +42,9 @@ Readings where the pages are silent (each is listed in the design doc):
 * SwiGLU: [a; b] = W_in y + bias, output W_out (silu(a) * b) + bias.
 * LN and RMS eps 1e-6; RMSNorm gain of 128 values per stream, shared by heads.
 * Euler: t_i = linspace(1, 0, S+1); x <- x + (t_{i+1} - t_i) v(x, t_i).
+* img2img strength s: run the last floor(S s) steps, starting from
+  (1 - t) x_in + t noise at the first kept t.  Several references: reference k at
+  RoPE l = -(k+1), tokens appended in order after the image tokens.
 """
 from __future__ import annotations
 
@@ -53,7 +56,7 @@ __all__ = [
     "pack_latents", "unpack_latents", "token_positions", "rope_angles", "apply_rope",
     "layer_norm", "rms_norm", "modulate", "silu", "linear", "attention_probs",
     "attention", "timestep_embedding", "double_block", "single_block", "forward",
-    "schedule", "euler_update", "sample", "weight",
+    "schedule", "euler_update", "img2img_start", "blend_latents", "sample", "weight",
 ]
 
 CPU = torch.device("cpu")
@@ -94,17 +97,24 @@ def unpack_latents(tok: torch.Tensor, h8: int, w8: int) -> torch.Tensor:
 # ----------------------------------------------------------------------------
 # [P5 "Modulation pro Token-Typ, Flow-Map-Destillation und 4D-RoPE"] positions
 # ----------------------------------------------------------------------------
-def token_positions(n_txt, grid_h, grid_w, ref_h=0, ref_w=0, dtype=torch.float64):
-    """(t, h, w, l) coordinates of the joint sequence [text; image; reference]."""
+def token_positions(n_txt, grid_h, grid_w, ref_h=0, ref_w=0, dtype=torch.float64, ref_grids=None):
+    """(t, h, w, l) coordinates of the joint sequence [text; image; reference 0; reference 1; ...].
+
+    Reference k's token (r, c) sits at (0, r, c, -(k+1)).  ``ref_grids`` lists the (h, w) of
+    every reference; without it, (ref_h, ref_w) describes a single reference (0 = none).
+    """
+    if ref_grids is None:
+        ref_grids = [(ref_h, ref_w)] if ref_h > 0 else []
     rows = []
     for i in range(n_txt):
         rows.append((0.0, 0.0, 0.0, float(i)))
     for r in range(grid_h):
         for c in range(grid_w):
             rows.append((0.0, float(r), float(c), 0.0))
-    for r in range(ref_h):
-        for c in range(ref_w):
-            rows.append((0.0, float(r), float(c), -1.0))
+    for k, (rh, rw) in enumerate(ref_grids):
+        for r in range(rh):
+            for c in range(rw):
+                rows.append((0.0, float(r), float(c), -float(k + 1)))
     return torch.tensor(rows, dtype=dtype).reshape(-1, 4)
 
 
@@ -270,12 +280,19 @@ def forward(p, hp, img_tok, txt, t, grid_hw, ref_tok=None, ref_hw=(0, 0),
             dtype=torch.float64, positions=None):
     """Velocity v [Ni, 128] of the image tokens at time t.
 
-    img_tok [Ni, 128], txt [Nt, txt_dim], ref_tok [Nr, 128] or None.  The joint
-    sequence is ordered text | image | reference [P5]; reference tokens go
-    through the image-stream weights and the same t (one timestep for every
-    token in FLUX.2 [P5]).  ``positions`` overrides the RoPE coordinates (all
-    zeros switches RoPE off).
+    img_tok [Ni, 128], txt [Nt, txt_dim].  References: ref_tok [Nr, 128] with
+    ref_hw = (h, w) for one, or a list of token tensors with a list of (h, w)
+    for several (reference k at RoPE l = -(k+1) [P5]).  The joint sequence is
+    ordered text | image | references [P5]; reference tokens go through the
+    image-stream weights and the same t (one timestep for every token in
+    FLUX.2 [P5]).  ``positions`` overrides the RoPE coordinates (all zeros
+    switches RoPE off).
     """
+    if isinstance(ref_tok, (list, tuple)):
+        ref_grids = list(ref_hw)
+        ref_tok = torch.cat([torch.as_tensor(r) for r in ref_tok]) if ref_tok else None
+    else:
+        ref_grids = [tuple(ref_hw)] if ref_tok is not None else []
     img_tok = torch.as_tensor(img_tok).to(dtype)
     txt = torch.as_tensor(txt).to(dtype)
     ni, nt = img_tok.shape[0], txt.shape[0]
@@ -291,7 +308,7 @@ def forward(p, hp, img_tok, txt, t, grid_hw, ref_tok=None, ref_hw=(0, 0),
     x_txt = linear(txt, weight(p, "txt_in.w", dtype), weight(p, "txt_in.b", dtype))
 
     if positions is None:
-        positions = token_positions(nt, grid_hw[0], grid_hw[1], ref_hw[0], ref_hw[1], dtype)
+        positions = token_positions(nt, grid_hw[0], grid_hw[1], dtype=dtype, ref_grids=ref_grids)
     ang = rope_angles(positions.to(dtype), hp["head_dim"], hp["rope_theta"])
 
     for i in range(_count(p, "double")):
@@ -319,24 +336,52 @@ def euler_update(x: torch.Tensor, v: torch.Tensor, dt: float) -> torch.Tensor:
     return x + dt * v
 
 
-def sample(p, hp, latent, txt, n_steps, ref_latent=None, dtype=torch.float64, on_step=None):
+# ----------------------------------------------------------------------------
+# img2img strength ["Flux 2 Klein: Reine C-basierte Inferenz", "Nutzungsbeispiele":
+# -t 0.0 keeps the input, 1.0 regenerates it; hakusoku "コマンドラインオプション": default 0.75]
+# ----------------------------------------------------------------------------
+def img2img_start(n_steps: int, strength: float) -> int:
+    """Index of the first schedule step run for a given strength.
+
+    Reading (the pages give only the two end points): run the last floor(S * strength)
+    steps of the S-step schedule; strength 1 runs them all, 0 runs none.
+    """
+    k = min(int(n_steps * strength), n_steps)
+    return n_steps - k
+
+
+def blend_latents(x: torch.Tensor, noise: torch.Tensor, t: float) -> torch.Tensor:
+    """The flow-matching state at time t between data x (t = 0) and noise (t = 1)."""
+    return (1.0 - t) * x + t * noise
+
+
+def sample(p, hp, latent, txt, n_steps, ref_latent=None, dtype=torch.float64, on_step=None,
+           init_latent=None, strength=1.0):
     """Run the sampler; returns (final latent [32, h8, w8], list of velocities [Ni, 128]).
 
-    The state is the packed image tokens; reference tokens are context only and
-    never updated.  ``on_step(i, v)`` is called after every forward if given.
+    ``latent`` is the noise.  ``ref_latent`` is one reference latent or a list of them
+    (context tokens, never updated).  With ``init_latent`` (the latent of an image to
+    edit) and ``strength`` < 1 the run starts at schedule step img2img_start(S, strength)
+    from blend_latents(init_latent, latent, t_start).  ``on_step(i, v)`` is called after
+    every forward if given.
     """
     latent = torch.as_tensor(latent).to(dtype)
     c, h8, w8 = latent.shape
-    tok = pack_latents(latent)
-    ref_tok, ref_hw = None, (0, 0)
-    if ref_latent is not None:
-        ref_latent = torch.as_tensor(ref_latent).to(dtype)
-        ref_tok = pack_latents(ref_latent)
-        ref_hw = (ref_latent.shape[1] // 2, ref_latent.shape[2] // 2)
     ts = schedule(n_steps)
+    start = 0
+    if init_latent is not None:
+        start = img2img_start(n_steps, strength)
+        latent = blend_latents(torch.as_tensor(init_latent).to(dtype), latent, ts[start])
+    tok = pack_latents(latent)
+    refs = [] if ref_latent is None else (list(ref_latent) if isinstance(ref_latent, (list, tuple)) else [ref_latent])
+    ref_toks, ref_grids = [], []
+    for r in refs:
+        r = torch.as_tensor(r).to(dtype)
+        ref_toks.append(pack_latents(r))
+        ref_grids.append((r.shape[1] // 2, r.shape[2] // 2))
     vs = []
-    for i in range(n_steps):
-        v = forward(p, hp, tok, txt, ts[i], (h8 // 2, w8 // 2), ref_tok, ref_hw, dtype)
+    for i in range(start, n_steps):
+        v = forward(p, hp, tok, txt, ts[i], (h8 // 2, w8 // 2), ref_toks, ref_grids, dtype)
         vs.append(v)
         if on_step is not None:
             on_step(i, v)

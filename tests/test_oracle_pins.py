@@ -162,16 +162,22 @@ def test_silu_closed_form():
 def test_rope_coordinate_table_from_pages():
     g = json.load(open(os.path.join(GOLDEN, "rope_coordinates.json")))
     n_txt, gh, gw, rh, rw = 6, 3, 4, 2, 3
-    pos = O.token_positions(n_txt, gh, gw, rh, rw)
-    assert pos.shape == (n_txt + gh * gw + rh * rw, 4)
+    pos = O.token_positions(n_txt, gh, gw, ref_grids=[(rh, rw), (rh, rw)])
+    assert pos.shape == (n_txt + gh * gw + 2 * rh * rw, 4)
+    assert torch.equal(O.token_positions(n_txt, gh, gw, rh, rw), pos[:n_txt + gh * gw + rh * rw])
     for c in g["cases"]:
         if c["kind"] == "text":
             row = c["index"]
         elif c["kind"] == "image":
             row = n_txt + c["row"] * gw + c["col"]
         else:
-            row = n_txt + gh * gw + c["row"] * rw + c["col"]
+            row = n_txt + gh * gw + c["k"] * rh * rw + c["row"] * rw + c["col"]
         assert pos[row].tolist() == [float(v) for v in c["coord"]]
+    # several references of different sizes follow one another, reference k at l = -(k+1)
+    pos2 = O.token_positions(n_txt, gh, gw, ref_grids=[(rh, rw), (rh, rw), (1, 2)])
+    assert pos2.shape[0] == n_txt + gh * gw + 2 * rh * rw + 2
+    assert pos2[-1].tolist() == [0.0, 0.0, 1.0, -3.0]
+    assert torch.equal(pos2[:pos.shape[0]], pos)
 
 
 def test_rope_unit_vector_closed_form():
@@ -448,6 +454,56 @@ def test_sampler_uses_schedule_times():
     v1 = O.forward(p, hp_of(MICRO), tok1, txt, 0.5, (2, 2))
     assert torch.allclose(vs[1], v1, atol=1e-12, rtol=0)
     assert torch.allclose(final, O.unpack_latents(tok1 - 0.5 * v1, 4, 4), atol=1e-12, rtol=0)
+
+
+def test_img2img_strength_end_points_from_pages():
+    """strength 0 keeps the input latent unchanged; strength 1 equals sampling from pure noise."""
+    g = json.load(open(os.path.join(GOLDEN, "img2img_and_references.json")))
+    p = micro_params(9)
+    gen = torch.Generator().manual_seed(11)
+    noise = torch.randn(32, 4, 4, generator=gen, dtype=F64)
+    init = torch.randn(32, 4, 4, generator=gen, dtype=F64)
+    txt = torch.randn(3, MICRO.txt_dim, generator=gen, dtype=F64)
+    kept, vs = O.sample(p, hp_of(MICRO), noise, txt, 4, init_latent=init, strength=g["strength_keeps_original"])
+    assert vs == [] and torch.equal(kept, init)
+    full, _ = O.sample(p, hp_of(MICRO), noise, txt, 4, init_latent=init, strength=g["strength_regenerates"])
+    plain, _ = O.sample(p, hp_of(MICRO), noise, txt, 4)
+    assert torch.equal(full, plain)
+    # the default strength runs the last 3 of 4 steps, from t = 0.75
+    assert O.img2img_start(4, g["strength_default"]) == 1 and O.schedule(4)[1] == 0.75
+    part, vs = O.sample(p, hp_of(MICRO), noise, txt, 4, init_latent=init, strength=0.75)
+    assert len(vs) == 3
+
+
+def test_blend_latents_closed_forms():
+    x = torch.randn(5, dtype=F64)
+    n = torch.randn(5, dtype=F64)
+    assert torch.equal(O.blend_latents(x, n, 0.0), x)
+    assert torch.equal(O.blend_latents(x, n, 1.0), n)
+    assert torch.allclose(O.blend_latents(x, n, 0.5), (x + n) / 2, atol=1e-15, rtol=0)
+
+
+def test_multiple_references_are_ordered_and_distinguished():
+    """Reference order matters (l = -1 vs -2); a one-element list equals the single-reference call."""
+    g = json.load(open(os.path.join(GOLDEN, "img2img_and_references.json")))
+    p = micro_params(10)
+    img, txt = _micro_inputs(4, gh=2, gw=2)
+    gen = torch.Generator().manual_seed(12)
+    r0 = torch.randn(4, MICRO.in_ch, generator=gen, dtype=F64)
+    r1 = torch.randn(4, MICRO.in_ch, generator=gen, dtype=F64)
+    one = O.forward(p, hp_of(MICRO), img, txt, 0.5, (2, 2), r0, (2, 2))
+    one_list = O.forward(p, hp_of(MICRO), img, txt, 0.5, (2, 2), [r0], [(2, 2)])
+    assert torch.equal(one, one_list)
+    a = O.forward(p, hp_of(MICRO), img, txt, 0.5, (2, 2), [r0, r1], [(2, 2), (2, 2)])
+    b = O.forward(p, hp_of(MICRO), img, txt, 0.5, (2, 2), [r1, r0], [(2, 2), (2, 2)])
+    assert (a - b).abs().max() > 1e-6
+    # with RoPE off the two references are interchangeable context
+    n = 5 + 4 + 8
+    z = torch.zeros(n, 4, dtype=F64)
+    az = O.forward(p, hp_of(MICRO), img, txt, 0.5, (2, 2), [r0, r1], [(2, 2), (2, 2)], positions=z)
+    bz = O.forward(p, hp_of(MICRO), img, txt, 0.5, (2, 2), [r1, r0], [(2, 2), (2, 2)], positions=z)
+    assert torch.allclose(az, bz, atol=1e-10, rtol=0)
+    assert g["max_reference_images"] == 10
 
 
 @pytest.mark.slow
