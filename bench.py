@@ -169,7 +169,7 @@ def cpu_oracle_sample(w, params, lat, txt, ref):
     x_txt = torch.randn(w.n_txt, D, generator=g)
     x_img = torch.randn(w.n_img + w.n_ref, D, generator=g)
     s = torch.randn(D, generator=g)
-    ang = O.rope_angles(O.token_positions(w.n_txt, w.grid, w.grid, w.ref_grid, w.ref_grid), 128, 1e4).float()
+    ang = O.rope_angles(O.token_positions(w.n_txt, w.grid, w.grid, ref_grids=w.ref_grids), 128, 1e4).float()
     t0 = time.perf_counter()
     O.double_block(params, 0, x_txt, x_img, s, ang, hp, torch.float32)
     t1 = time.perf_counter()
@@ -192,7 +192,7 @@ def run_reference(args, w):
     g = torch.Generator().manual_seed(0)
     x = torch.randn(w.n_tokens, D, generator=g)
     s = torch.randn(D, generator=g)
-    ang = O.rope_angles(O.token_positions(w.n_txt, w.grid, w.grid, w.ref_grid, w.ref_grid), 128, 1e4).float()
+    ang = O.rope_angles(O.token_positions(w.n_txt, w.grid, w.grid, ref_grids=w.ref_grids), 128, 1e4).float()
     scale = forward_flops(w) / single_block_flops(w)
     for _ in range(args.warmup):
         O.single_block(params, 0, x, s, ang, hp, torch.float32)
@@ -210,8 +210,8 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_block, 3),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded N(0,1) bf16-rounded weights and inputs)",
-        "config": {"workload": f"{w.name}: {w.image}x{w.image} text-to-image, {w.n_img} image + {w.n_txt} text "
-                               f"tokens, 5 double + 20 single blocks, width 3072", "seq_len": w.n_tokens,
+        "config": {"workload": f"{w.name}: {w.image}x{w.image}, {w.n_img} image + {w.n_txt} text + {w.n_ref} "
+                               f"reference tokens, 5 double + 20 single blocks, width 3072", "seq_len": w.n_tokens,
                    "global_batch": 1, "parallelism": "CPU oracle on rank 0"},
         "tflops": round(forward_flops(w) / (value / 1e3) / 1e12, 4),
         "cpu_baseline": {"value": round(value, 3), "unit": "ms/forward", "cores": torch.get_num_threads(),
@@ -248,8 +248,11 @@ def run_ours(args, w):
     ref_tok, ref_hw = None, (0, 0)
     if ref_h is not None:
         ref_tok = torch.empty(w.n_ref, 128, device=dev)
-        F.flux_pack_latents(torch.from_numpy(ref_h).to(dev), ref_tok)
-        ref_hw = (w.ref_grid, w.ref_grid)
+        row = 0
+        for r, (h, w_) in zip(ref_h if isinstance(ref_h, list) else [ref_h], w.ref_grids):
+            F.flux_pack_latents(torch.from_numpy(r).to(dev), ref_tok[row:row + h * w_])
+            row += h * w_
+        ref_hw = w.ref_grids if isinstance(ref_h, list) else w.ref_grids[0]
     ts = F.euler_schedule(w.n_steps)
 
     def step(i, lat_buf):
@@ -339,9 +342,9 @@ def run_ours(args, w):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) weights scaled 1/sqrt(fan_in), bf16; N(0,1) latent and text)",
-            "config": {"workload": f"{w.name}: {w.image}x{w.image} text-to-image, {w.n_img} image + {w.n_txt} text "
-                                   f"tokens, 5 double + 20 single blocks, width 3072, 24x128 heads, "
-                                   f"one Euler step (pack, forward, Euler, unpack)",
+            "config": {"workload": f"{w.name}: {w.image}x{w.image}, {w.n_img} image + {w.n_txt} text + {w.n_ref} "
+                                   f"reference tokens ({len(w.ref_grids)} reference images), 5 double + 20 single "
+                                   f"blocks, width 3072, 24x128 heads, one Euler step (pack, forward, Euler, unpack)",
                        "global_batch": world, "seq_len": w.n_tokens,
                        "parallelism": f"replicas x{world}, no data-path collective",
                        "l2": "inputs larger than L2: 9.7 GB of bf16 weights streamed every forward"},

@@ -111,6 +111,16 @@ FLUX_API void flux_dit_destroy(flux_dit *m);
 FLUX_API int flux_dit_forward(flux_dit *m, const float *img_tok, int grid_h, int grid_w, const float *txt, int n_txt,
                      const float *ref_tok, int ref_h, int ref_w, float t, float *v_out, void *stream);
 
+/* One forward with several reference images (at most 10): their packed tokens are
+ * concatenated in order in ref_tok (fp32 [sum_k h_k*w_k, 128]); ref_grids is a HOST
+ * array of n_refs (h, w) pairs, each in 4..64.  Reference k sits at RoPE coordinate
+ * l = -(k+1) ("FLUX.3 Image Klein in Diffusers: ...", section "Modulation pro Token-Typ,
+ * Flow-Map-Destillation und 4D-RoPE"; up to ten reference images: we0.ai FLUX.3 Image
+ * Klein article).  n_refs = 0 is a text-to-image forward.  Otherwise as flux_dit_forward. */
+FLUX_API int flux_dit_forward_refs(flux_dit *m, const float *img_tok, int grid_h, int grid_w, const float *txt,
+                                   int n_txt, const float *ref_tok, int n_refs, const int *ref_grids, float t,
+                                   float *v_out, void *stream);
+
 /* Diagnostic: run only the first n_double double blocks and n_single single
  * blocks in later forwards (-1 = all).  Used to bisect parity; not a model change. */
 FLUX_API int flux_dit_set_active_blocks(flux_dit *m, int n_double, int n_single);
@@ -125,6 +135,13 @@ FLUX_API int flux_dit_modulation(flux_dit *m, float t, float *mods_out, void *st
  * ("Flux 2 Klein: Reine C-basierte Inferenz", "Modellarchitektur und Leistung":
  * 4 sampling steps; t_i = linspace(1, 0, S+1), dt = t_{i+1} - t_i). */
 FLUX_API int flux_euler_step(float *x, const float *v, size_t n, float dt, void *stream);
+
+/* img2img start state: out = (1 - t) x + t noise over n fp32 values (x the latent of the
+ * image to edit, noise N(0,1)): the flow-matching state at time t.  With strength s the
+ * sampler starts at the first of the last floor(S*s) schedule times; s = 0 keeps the image
+ * and s = 1 regenerates it ("Flux 2 Klein: Reine C-basierte Inferenz", "Nutzungsbeispiele";
+ * hakusoku.com story 4662, "コマンドラインオプション": -t/--strength, default 0.75). */
+FLUX_API int flux_blend_latents(const float *x, const float *noise, float t, float *out, size_t n, void *stream);
 
 /* 2x2 latent packing ("Zweistufiger Transformer und Tokenisierung"):
  *   lat fp32 [32, h8, w8]  <->  tok fp32 [(h8/2)*(w8/2), 128],

@@ -44,6 +44,8 @@ _SIGS = {
     "flux_dit_create": (_P, [_P, _Z, ctypes.POINTER(FluxConfig), _P]),
     "flux_dit_destroy": (None, [_P]),
     "flux_dit_forward": (_I, [_P, _P, _I, _I, _P, _I, _P, _I, _I, _F, _P, _P]),
+    "flux_dit_forward_refs": (_I, [_P, _P, _I, _I, _P, _I, _P, _I, ctypes.POINTER(ctypes.c_int), _F, _P, _P]),
+    "flux_blend_latents": (_I, [_P, _P, _F, _P, _Z, _P]),
     "flux_dit_set_active_blocks": (_I, [_P, _I, _I]),
     "flux_dit_modulation_size": (_Z, [_P]),
     "flux_dit_modulation": (_I, [_P, _F, _P, _P]),
@@ -148,8 +150,17 @@ class FluxDiT:
             pass
 
     def forward(self, img_tok, grid_hw, txt, t, v_out, ref_tok=None, ref_hw=(0, 0), stream=None):
+        """One forward.  ref_hw is one (h, w) or a list of them (then ref_tok holds every
+        reference's packed tokens, concatenated in order)."""
         import torch
         n_txt = 0 if txt is None else txt.shape[0]
+        if ref_hw and isinstance(ref_hw[0], (tuple, list)):
+            grids = (ctypes.c_int * (2 * len(ref_hw)))(*[v for hw in ref_hw for v in hw])
+            _check(lib().flux_dit_forward_refs(self._h, _ptr(img_tok, torch.float32, "img_tok"), grid_hw[0],
+                                               grid_hw[1], _ptr(txt, torch.float32, "txt"), n_txt,
+                                               _ptr(ref_tok, torch.float32, "ref_tok"), len(ref_hw), grids,
+                                               float(t), _ptr(v_out, torch.float32, "v_out"), _stream(stream)))
+            return v_out
         _check(lib().flux_dit_forward(self._h, _ptr(img_tok, torch.float32, "img_tok"), grid_hw[0], grid_hw[1],
                                       _ptr(txt, torch.float32, "txt"), n_txt,
                                       _ptr(ref_tok, torch.float32, "ref_tok"), ref_hw[0], ref_hw[1],
@@ -186,6 +197,19 @@ class FluxDiT:
 def euler_schedule(n_steps: int):
     """t_0 = 1 > ... > t_S = 0 evenly spaced (float32 values)."""
     return [float(np.float32(1.0 - i / n_steps)) for i in range(n_steps + 1)]
+
+
+def img2img_first_step(n_steps: int, strength: float) -> int:
+    """First schedule index run at img2img strength s: the last floor(S * s) steps are run."""
+    return n_steps - min(int(n_steps * strength), n_steps)
+
+
+def flux_blend_latents(x, noise, t, out, stream=None):
+    """out = (1 - t) x + t noise (img2img start state)."""
+    import torch
+    _check(lib().flux_blend_latents(_ptr(x, torch.float32, "x"), _ptr(noise, torch.float32, "noise"), float(t),
+                                    _ptr(out, torch.float32, "out"), x.numel(), _stream(stream)))
+    return out
 
 
 def flux_euler_step(x, v, dt, stream=None):
@@ -287,27 +311,38 @@ def flux_device_error(stream=None) -> int:
     return lib().flux_device_error(_stream(stream))
 
 
-def flux_sample(model: FluxDiT, latent, txt, n_steps, ref_latent=None, on_step=None, stream=None):
+def flux_sample(model: FluxDiT, latent, txt, n_steps, ref_latent=None, on_step=None, stream=None,
+                init_latent=None, strength=1.0):
     """Euler sampling on the device: pack -> S x (forward, Euler) -> unpack.
 
-    latent fp32 [32, h8, w8] (device), txt fp32 [n_txt, txt_dim] (device),
-    ref_latent fp32 [32, r8, r8] or None.  Returns the final latent (new tensor).
-    ``on_step(i, v)`` sees each velocity (device tensor, reused between steps).
+    latent fp32 [32, h8, w8] (device): the noise.  txt fp32 [n_txt, txt_dim] (device).
+    ref_latent: one fp32 [32, r8, r8] latent, a list of them (context images), or None.
+    init_latent (the latent of an image to edit) with strength s < 1: start from
+    flux_blend_latents(init_latent, latent, t) at schedule step img2img_first_step(S, s).
+    Returns the final latent (new tensor).  ``on_step(i, v)`` sees each velocity.
     """
     import torch
     c, h8, w8 = latent.shape
     gh, gw = h8 // 2, w8 // 2
+    ts = euler_schedule(n_steps)
+    start = 0
+    if init_latent is not None:
+        start = img2img_first_step(n_steps, strength)
+        latent = flux_blend_latents(init_latent, latent, ts[start], torch.empty_like(latent), stream)
     tok = torch.empty(gh * gw, 4 * c, device=latent.device, dtype=torch.float32)
     flux_pack_latents(latent, tok, stream)
     ref_tok, ref_hw = None, (0, 0)
     if ref_latent is not None:
-        rh, rw = ref_latent.shape[1] // 2, ref_latent.shape[2] // 2
-        ref_tok = torch.empty(rh * rw, 4 * c, device=latent.device, dtype=torch.float32)
-        flux_pack_latents(ref_latent, ref_tok, stream)
-        ref_hw = (rh, rw)
+        refs = list(ref_latent) if isinstance(ref_latent, (list, tuple)) else [ref_latent]
+        grids = [(r.shape[1] // 2, r.shape[2] // 2) for r in refs]
+        ref_tok = torch.empty(sum(h * w for h, w in grids), 4 * c, device=latent.device, dtype=torch.float32)
+        row = 0
+        for r, (h, w) in zip(refs, grids):
+            flux_pack_latents(r, ref_tok[row:row + h * w], stream)
+            row += h * w
+        ref_hw = grids if isinstance(ref_latent, (list, tuple)) else grids[0]
     v = torch.empty_like(tok)
-    ts = euler_schedule(n_steps)
-    for i in range(n_steps):
+    for i in range(start, n_steps):
         model.forward(tok, (gh, gw), txt, ts[i], v, ref_tok, ref_hw, stream)
         if on_step is not None:
             on_step(i, v)

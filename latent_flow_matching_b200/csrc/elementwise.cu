@@ -208,10 +208,11 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(__nv_bfloat16* __rest
 }
 
 // (cos, sin) of pos_axis * theta^(-2m/32) for the 64 pairs of a 128-dim head, axes (t, h, w, l).
-// text i: (0,0,0,i); image (r,c): (0,r,c,0); reference (r,c): (0,r,c,-1).
-__global__ void rope_table_kernel(float2* __restrict__ table, int n_txt, int gh, int gw, int rh, int rw,
+// text i: (0,0,0,i); image (r,c): (0,r,c,0); reference k (r,c): (0,r,c,-(k+1)).
+__global__ void rope_table_kernel(float2* __restrict__ table, int n_txt, int gh, int gw, RefGrids refs,
                                   float theta) {
-  const int n = n_txt + gh * gw + rh * rw;
+  int n = n_txt + gh * gw;
+  for (int k = 0; k < refs.count; ++k) n += refs.h[k] * refs.w[k];
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= n * 64) return;
   const int row = idx >> 6, pr = idx & 63;
@@ -224,15 +225,28 @@ __global__ void rope_table_kernel(float2* __restrict__ table, int n_txt, int gh,
     pos[1] = t / gw;
     pos[2] = t % gw;
   } else {
-    const int t = row - n_txt - gh * gw;
-    pos[1] = t / rw;
-    pos[2] = t % rw;
-    pos[3] = -1.0;
+    int t = row - n_txt - gh * gw;
+    int k = 0;
+    while (k + 1 < refs.count && t >= refs.h[k] * refs.w[k]) {
+      t -= refs.h[k] * refs.w[k];
+      ++k;
+    }
+    pos[1] = t / refs.w[k];
+    pos[2] = t % refs.w[k];
+    pos[3] = -(k + 1.0);
   }
   const double ang = pos[axis] * pow(static_cast<double>(theta), -2.0 * m / 32.0);
   double s, c;
   sincos(ang, &s, &c);
   table[idx] = make_float2(static_cast<float>(c), static_cast<float>(s));
+}
+
+// (1 - t) x + t noise: the flow-matching state at time t between data (t = 0) and noise (t = 1)
+__global__ void blend_kernel(const float* __restrict__ x, const float* __restrict__ noise, float t,
+                             float* __restrict__ out, size_t n) {
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n; i += stride)
+    out[i] = (1.0f - t) * x[i] + t * noise[i];
 }
 
 // ------------------------------------------------------------------ timestep embedding, GEMV
@@ -346,11 +360,20 @@ cudaError_t qk_norm_rope_launch(__nv_bfloat16* qkv, int rows, int ld, int kcol, 
   return cudaGetLastError();
 }
 
-cudaError_t rope_table_launch(float2* table, int n_txt, int gh, int gw, int rh, int rw, float theta, cudaStream_t s) {
-  const int n = n_txt + gh * gw + rh * rw;
+cudaError_t rope_table_launch(float2* table, int n_txt, int gh, int gw, const RefGrids& refs, float theta,
+                              cudaStream_t s) {
+  int n = n_txt + gh * gw;
+  for (int k = 0; k < refs.count; ++k) n += refs.h[k] * refs.w[k];
   if (n <= 0) return cudaSuccess;
   count_launch();
-  rope_table_kernel<<<(n * 64 + 255) / 256, 256, 0, s>>>(table, n_txt, gh, gw, rh, rw, theta);
+  rope_table_kernel<<<(n * 64 + 255) / 256, 256, 0, s>>>(table, n_txt, gh, gw, refs, theta);
+  return cudaGetLastError();
+}
+
+cudaError_t blend_launch(const float* x, const float* noise, float t, float* out, size_t n, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  count_launch();
+  blend_kernel<<<blocks_for(n, 256), 256, 0, s>>>(x, noise, t, out, n);
   return cudaGetLastError();
 }
 

@@ -232,7 +232,8 @@ struct Workspace {
   float* X = nullptr;
   bf16 *Y = nullptr, *QKV = nullptr, *CC = nullptr, *tokb = nullptr, *txtb = nullptr;
   float2* rope = nullptr;
-  int nt = -1, gh = -1, gw = -1, rh = -1, rw = -1;     // shape the maps and the RoPE table were built for
+  int nt = -1, gh = -1, gw = -1;                        // shape the maps and the RoPE table were built for
+  RefGrids refs = {-1, {}, {}};
   CUtensorMap a_txtb, a_tokb, a_Ytxt, a_Yimg, a_Yall, a_Yout, a_Otxt, a_Oimg, a_Htxt, a_Himg, a_CC, qkv;
 };
 
@@ -430,11 +431,24 @@ static cudaError_t grow(T** p, size_t* cap, size_t need) {
   return e;
 }
 
-static int prepare_shape(flux_dit* m, int nt, int gh, int gw, int rh, int rw, cudaStream_t s) {
+static size_t ref_tokens(const RefGrids& r) {
+  size_t n = 0;
+  for (int k = 0; k < r.count; ++k) n += static_cast<size_t>(r.h[k]) * r.w[k];
+  return n;
+}
+
+static bool same_refs(const RefGrids& a, const RefGrids& b) {
+  if (a.count != b.count) return false;
+  for (int k = 0; k < a.count; ++k)
+    if (a.h[k] != b.h[k] || a.w[k] != b.w[k]) return false;
+  return true;
+}
+
+static int prepare_shape(flux_dit* m, int nt, int gh, int gw, const RefGrids& refs, cudaStream_t s) {
   Workspace& w = m->ws;
   const flux_dit_config& c = m->cfg;
   const size_t D = c.hidden, F = c.mlp_hidden;
-  const size_t ni = static_cast<size_t>(gh) * gw, nr = static_cast<size_t>(rh) * rw;
+  const size_t ni = static_cast<size_t>(gh) * gw, nr = ref_tokens(refs);
   const size_t n = nt + ni + nr;
   if (n > w.cap_n) {
     float* X = nullptr;
@@ -455,7 +469,7 @@ static int prepare_shape(flux_dit* m, int nt, int gh, int gw, int rh, int rw, cu
   if (grow(&w.tokb, &w.cap_tok, (ni + nr) * c.in_ch) != cudaSuccess ||
       grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt, 1) * c.txt_dim) != cudaSuccess)
     return fail(FLUX_ENOMEM, "workspace allocation failed");
-  if (w.nt == nt && w.gh == gh && w.gw == gw && w.rh == rh && w.rw == rw) return FLUX_OK;
+  if (w.nt == nt && w.gh == gh && w.gw == gw && same_refs(w.refs, refs)) return FLUX_OK;
 
   const size_t nimg = ni + nr;
   const uint64_t ldD = D * 2, ldC = (D + F) * 2;
@@ -480,9 +494,9 @@ static int prepare_shape(flux_dit* m, int nt, int gh, int gw, int rh, int rw, cu
   amap(&w.a_CC, w.CC, n, D + F, ldC, 128);
   amap(&w.qkv, w.QKV, n, 3 * D, 3 * D * 2, 128);
   if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an activation buffer");
-  if (rope_table_launch(w.rope, nt, gh, gw, rh, rw, c.rope_theta, s) != cudaSuccess)
+  if (rope_table_launch(w.rope, nt, gh, gw, refs, c.rope_theta, s) != cudaSuccess)
     return fail(FLUX_EIO, "rope table launch failed");
-  w.nt = nt; w.gh = gh; w.gw = gw; w.rh = rh; w.rw = rw;
+  w.nt = nt; w.gh = gh; w.gw = gw; w.refs = refs;
   return FLUX_OK;
 }
 
@@ -537,24 +551,27 @@ static int run_modulation(flux_dit* m, float t, cudaStream_t s) {
 }
 
 static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const float* txt, int nt,
-                        const float* ref_tok, int rh, int rw, float t, float* v_out, cudaStream_t s) {
+                        const float* ref_tok, const RefGrids& refs, float t, float* v_out, cudaStream_t s) {
   const flux_dit_config& c = m->cfg;
   const int D = c.hidden, F = c.mlp_hidden, H = c.heads;
   if (!img_tok || !v_out) return fail(FLUX_EINVAL, "img_tok and v_out must be device pointers");
   if (gh < 4 || gh > 64 || gw < 4 || gw > 64) return fail(FLUX_EINVAL, "image grid %dx%d outside 4..64", gh, gw);
   if (nt < 0 || nt > 4096 || (nt > 0 && !txt)) return fail(FLUX_EINVAL, "bad text (n_txt=%d)", nt);
-  if (!((rh == 0 && rw == 0) || (rh >= 4 && rh <= 64 && rw >= 4 && rw <= 64)))
-    return fail(FLUX_EINVAL, "reference grid %dx%d outside 4..64", rh, rw);
-  if (rh > 0 && !ref_tok) return fail(FLUX_EINVAL, "ref_tok is NULL for a %dx%d reference", rh, rw);
+  if (refs.count < 0 || refs.count > kMaxRefs)
+    return fail(FLUX_EINVAL, "%d reference images (at most %d)", refs.count, kMaxRefs);
+  for (int k = 0; k < refs.count; ++k)
+    if (refs.h[k] < 4 || refs.h[k] > 64 || refs.w[k] < 4 || refs.w[k] > 64)
+      return fail(FLUX_EINVAL, "reference %d grid %dx%d outside 4..64", k, refs.h[k], refs.w[k]);
+  if (refs.count > 0 && !ref_tok) return fail(FLUX_EINVAL, "ref_tok is NULL for %d reference(s)", refs.count);
   if (!std::isfinite(t)) return fail(FLUX_EINVAL, "t is not finite");
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev != m->device) return fail(FLUX_EINVAL, "model lives on device %d, current device is %d", m->device, dev);
 
-  int rc = prepare_shape(m, nt, gh, gw, rh, rw, s);
+  int rc = prepare_shape(m, nt, gh, gw, refs, s);
   if (rc) return rc;
   Workspace& w = m->ws;
-  const int ni = gh * gw, nr = rh * rw, nimg = ni + nr, n = nt + nimg;
+  const int ni = gh * gw, nr = static_cast<int>(ref_tokens(refs)), nimg = ni + nr, n = nt + nimg;
   const float eps_ln = c.eps_ln, eps_rms = c.eps_rms;
   const float* mods = m->mods;
 
@@ -667,8 +684,33 @@ void flux_dit_destroy(flux_dit* m) { destroy(m); }
 int flux_dit_forward(flux_dit* m, const float* img_tok, int grid_h, int grid_w, const float* txt, int n_txt,
                      const float* ref_tok, int ref_h, int ref_w, float t, float* v_out, void* stream) {
   if (!m) return fail(FLUX_EINVAL, "model is NULL");
-  return forward_impl(m, img_tok, grid_h, grid_w, txt, n_txt, ref_tok, ref_h, ref_w, t, v_out,
+  if (!((ref_h == 0 && ref_w == 0) || (ref_h > 0 && ref_w > 0)))
+    return fail(FLUX_EINVAL, "reference grid %dx%d", ref_h, ref_w);
+  RefGrids refs = {ref_h > 0 ? 1 : 0, {ref_h}, {ref_w}};
+  return forward_impl(m, img_tok, grid_h, grid_w, txt, n_txt, ref_tok, refs, t, v_out,
                       static_cast<cudaStream_t>(stream));
+}
+
+int flux_dit_forward_refs(flux_dit* m, const float* img_tok, int grid_h, int grid_w, const float* txt, int n_txt,
+                          const float* ref_tok, int n_refs, const int* ref_grids, float t, float* v_out,
+                          void* stream) {
+  if (!m) return fail(FLUX_EINVAL, "model is NULL");
+  if (n_refs < 0 || n_refs > kMaxRefs) return fail(FLUX_EINVAL, "%d reference images (at most %d)", n_refs, kMaxRefs);
+  if (n_refs > 0 && !ref_grids) return fail(FLUX_EINVAL, "ref_grids is NULL");
+  RefGrids refs = {n_refs, {}, {}};
+  for (int k = 0; k < n_refs; ++k) {
+    refs.h[k] = ref_grids[2 * k];
+    refs.w[k] = ref_grids[2 * k + 1];
+  }
+  return forward_impl(m, img_tok, grid_h, grid_w, txt, n_txt, ref_tok, refs, t, v_out,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int flux_blend_latents(const float* x, const float* noise, float t, float* out, size_t n, void* stream) {
+  if (n && (!x || !noise || !out)) return fail(FLUX_EINVAL, "NULL argument");
+  if (!std::isfinite(t)) return fail(FLUX_EINVAL, "t is not finite");
+  FD_CUDA(blend_launch(x, noise, t, out, n, static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
 }
 
 int flux_dit_set_active_blocks(flux_dit* m, int n_double, int n_single) {
@@ -802,7 +844,8 @@ int flux_rope_table(float* table, int n_txt, int gh, int gw, int rh, int rw, flo
   if (!table) return fail(FLUX_EINVAL, "NULL argument");
   if (n_txt < 0 || gh < 0 || gw < 0 || rh < 0 || rw < 0 || !(theta > 0))
     return fail(FLUX_EINVAL, "bad arguments");
-  FD_CUDA(rope_table_launch(reinterpret_cast<float2*>(table), n_txt, gh, gw, rh, rw, theta,
+  const RefGrids refs = {rh > 0 && rw > 0 ? 1 : 0, {rh}, {rw}};
+  FD_CUDA(rope_table_launch(reinterpret_cast<float2*>(table), n_txt, gh, gw, refs, theta,
                             static_cast<cudaStream_t>(stream)));
   return FLUX_OK;
 }

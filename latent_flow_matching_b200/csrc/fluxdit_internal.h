@@ -77,9 +77,19 @@ cudaError_t qk_norm_rope_launch(__nv_bfloat16* qkv, int rows, int ld, int kcol, 
                                 const __nv_bfloat16* gq1, const __nv_bfloat16* gk1,
                                 const float2* rope, float eps, cudaStream_t s);
 
-// (cos, sin) table for the joint sequence [text; image grid; reference grid], head_dim 128, 4 axes.
-cudaError_t rope_table_launch(float2* table, int n_txt, int gh, int gw, int rh, int rw, float theta,
+// Token grids of the reference images, in sequence order.
+constexpr int kMaxRefs = 10;
+struct RefGrids {
+  int count;
+  int h[kMaxRefs], w[kMaxRefs];
+};
+
+// (cos, sin) table for the joint sequence [text; image grid; reference grids], head_dim 128, 4 axes.
+cudaError_t rope_table_launch(float2* table, int n_txt, int gh, int gw, const RefGrids& refs, float theta,
                               cudaStream_t s);
+
+// out = (1 - t) x + t noise over n floats
+cudaError_t blend_launch(const float* x, const float* noise, float t, float* out, size_t n, cudaStream_t s);
 
 // temb[j] = cos(t*1000*f_j), temb[128+j] = sin(...), f_j = 1e4^(-j/128)
 cudaError_t timestep_embed_launch(float* temb, float t, int dim, cudaStream_t s);

@@ -65,6 +65,7 @@ class Workload:
     ref_image: int        # 0 = no reference image
     n_steps: int
     dims: FluxDims
+    extra_refs: tuple = ()  # sides of further reference images, after ref_image
 
     @property
     def grid(self) -> int:       # image tokens per side (16 px per token)
@@ -75,12 +76,20 @@ class Workload:
         return self.ref_image // 16
 
     @property
+    def ref_images(self) -> tuple:
+        return ((self.ref_image,) if self.ref_image else ()) + tuple(self.extra_refs)
+
+    @property
+    def ref_grids(self) -> list:
+        return [(r // 16, r // 16) for r in self.ref_images]
+
+    @property
     def n_img(self) -> int:
         return self.grid * self.grid
 
     @property
     def n_ref(self) -> int:
-        return self.ref_grid * self.ref_grid
+        return sum(h * w for h, w in self.ref_grids)
 
     @property
     def n_tokens(self) -> int:
@@ -96,6 +105,7 @@ WORKLOADS = {
     "t2i512": Workload("t2i512", 2, 512, 512, 0, 4, FULL_DIMS),
     "t2i1024": Workload("t2i1024", 3, 1024, 512, 0, 4, FULL_DIMS),
     "i2i1024": Workload("i2i1024", 4, 1024, 512, 1024, 4, FULL_DIMS),
+    "mref1024": Workload("mref1024", 5, 1024, 512, 512, 4, FULL_DIMS, extra_refs=(512,)),
 }
 
 
@@ -199,7 +209,11 @@ def make_weights(d: FluxDims, seed: int, threads: int | None = None):
 
 
 def make_inputs(w: Workload):
-    """Latent, text and reference latent as float32 arrays holding bf16 values."""
+    """Latent, text and reference latent(s) as float32 arrays holding bf16 values.
+
+    The reference is None, one array, or (several references) a list of arrays drawn
+    with keys INPUT_KEY + 2, + 3, ...
+    """
     def draw(k, shape):
         g = np.random.default_rng([w.seed, INPUT_KEY + k])
         x = g.standard_normal(int(np.prod(shape)), dtype=np.float32)
@@ -208,9 +222,7 @@ def make_inputs(w: Workload):
     h8 = w.image // 8
     latent = draw(0, (32, h8, h8))
     txt = draw(1, (w.n_txt, w.dims.txt_dim))
-    ref = None
-    if w.ref_image:
-        r8 = w.ref_image // 8
-        ref = draw(2, (32, r8, r8))
+    refs = [draw(2 + k, (32, r // 8, r // 8)) for k, r in enumerate(w.ref_images)]
+    ref = None if not refs else (refs[0] if len(refs) == 1 else refs)
     return latent, txt, ref
 

@@ -25,7 +25,7 @@ sys.path.insert(0, os.path.dirname(os.path.dirname(HERE)))
 from synthetic import WORKLOADS, make_weights, make_inputs  # noqa: E402
 from oracle import flux_oracle as O  # noqa: E402
 
-ROW_STRIDE = {"t2i256": 1, "t2i512": 2, "t2i1024": 8, "i2i1024": 8}
+ROW_STRIDE = {"t2i256": 1, "t2i512": 2, "t2i1024": 8, "i2i1024": 8, "mref1024": 8}
 
 
 def rows_for(name):
@@ -46,9 +46,12 @@ def make(name):
         print(f"  {name} step {i} done at {time.time() - t0:.0f}s", flush=True)
 
     with torch.no_grad():
+        if isinstance(ref, list):
+            ref = [torch.from_numpy(r) for r in ref]
+        elif ref is not None:
+            ref = torch.from_numpy(ref)
         final, _ = O.sample(p, O.hyper(w.dims), torch.from_numpy(lat), torch.from_numpy(txt),
-                            w.n_steps, None if ref is None else torch.from_numpy(ref),
-                            dtype=torch.float32, on_step=on_step)
+                            w.n_steps, ref, dtype=torch.float32, on_step=on_step)
     final_tok = O.pack_latents(final)[rows].float().numpy()
     meta = {"workload": name, "seed": w.seed, "oracle_dtype": "float32", "n_steps": w.n_steps,
             "row_stride": ROW_STRIDE[name], "seconds": round(time.time() - t0, 1)}

@@ -32,8 +32,11 @@ def rel_l2(a, b):
 
 def gpu_sample(model, w, lat, txt, ref):
     vs = []
-    final = F.flux_sample(model, torch.from_numpy(lat).to(DEV), torch.from_numpy(txt).to(DEV), w.n_steps,
-                          None if ref is None else torch.from_numpy(ref).to(DEV),
+    if isinstance(ref, list):
+        ref = [torch.from_numpy(r).to(DEV) for r in ref]
+    elif ref is not None:
+        ref = torch.from_numpy(ref).to(DEV)
+    final = F.flux_sample(model, torch.from_numpy(lat).to(DEV), torch.from_numpy(txt).to(DEV), w.n_steps, ref,
                           on_step=lambda i, v: vs.append(v.cpu().clone()))
     return final.cpu(), vs
 
@@ -139,7 +142,7 @@ def _golden(name):
     return np.load(path)
 
 
-@pytest.mark.parametrize("name", ["t2i256", "t2i512", "t2i1024", "i2i1024"])
+@pytest.mark.parametrize("name", ["t2i256", "t2i512", "t2i1024", "i2i1024", "mref1024"])
 def test_full_workload_against_oracle_goldens(name):
     gd = _golden(name)
     w = WORKLOADS[name]
@@ -161,3 +164,51 @@ def test_full_workload_against_oracle_goldens(name):
     err = rel_l2(tok[rows], gd["final"])
     assert err <= X_TOL, err
     assert F.flux_device_error() == 0
+
+
+# ---------------------------------------------------------------------------- several references, img2img
+def test_tiny_forward_with_several_references(tiny):
+    """Two references of different sizes (RoPE l = -1, -2) against the oracle."""
+    w, p, model = tiny
+    g = torch.Generator().manual_seed(21)
+    tok = torch.randn(16, 128, generator=g).to(torch.bfloat16).float()
+    txt = torch.randn(7, 3072, generator=g).to(torch.bfloat16).float()
+    grids = [(4, 4), (6, 4)]
+    refs = [torch.randn(h * w_, 128, generator=g).to(torch.bfloat16).float() for h, w_ in grids]
+    want = O.forward(p, O.hyper(w.dims), tok, txt, 0.5, (4, 4), refs, grids)
+    v = torch.empty(16, 128, device=DEV)
+    model.forward(tok.to(DEV), (4, 4), txt.to(DEV), 0.5, v, torch.cat(refs).to(DEV), grids)
+    assert rel_l2(v, want) <= V_TOL
+    # swapping the references changes the result (their RoPE offsets differ)
+    v2 = torch.empty(16, 128, device=DEV)
+    model.forward(tok.to(DEV), (4, 4), txt.to(DEV), 0.5, v2, torch.cat(refs[::-1]).to(DEV), grids[::-1])
+    assert rel_l2(v2, v) > 1e-3
+    assert F.flux_device_error() == 0
+
+
+def test_tiny_img2img_sampler_matches_oracle(tiny):
+    """strength 0.75 with 4 steps: the last 3 steps from the blended start state."""
+    w, p, model = tiny
+    lat, txt, _ = make_inputs(w)
+    init = torch.randn(32, 8, 8, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16).float()
+    ref_final, ref_vs = O.sample(p, O.hyper(w.dims), torch.from_numpy(lat), torch.from_numpy(txt), 4,
+                                 init_latent=init, strength=0.75)
+    vs = []
+    final = F.flux_sample(model, torch.from_numpy(lat).to(DEV), torch.from_numpy(txt).to(DEV), 4,
+                          init_latent=init.to(DEV), strength=0.75, on_step=lambda i, v: vs.append(v.cpu().clone()))
+    assert len(vs) == len(ref_vs) == 3
+    for a, b in zip(vs, ref_vs):
+        assert rel_l2(a, b) <= V_TOL
+    assert rel_l2(final.cpu(), ref_final) <= X_TOL
+    kept = F.flux_sample(model, torch.from_numpy(lat).to(DEV), torch.from_numpy(txt).to(DEV), 4,
+                         init_latent=init.to(DEV), strength=0.0)
+    assert torch.equal(kept.cpu(), init)                      # strength 0 keeps the image
+
+
+def test_forward_rejects_too_many_references(tiny):
+    w, p, model = tiny
+    v = torch.empty(16, 128, device=DEV)
+    tok = torch.zeros(16, 128, device=DEV)
+    refs = torch.zeros(11 * 16, 128, device=DEV)
+    with pytest.raises(F.FluxError):
+        model.forward(tok, (4, 4), None, 1.0, v, refs, [(4, 4)] * 11)

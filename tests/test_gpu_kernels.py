@@ -232,3 +232,15 @@ def test_attention_zero_query_is_mean_of_values():
     F.flux_joint_attention(q.to(DEV), k.to(DEV), v.to(DEV), o)
     ref = v.double().mean(0, keepdim=True).expand(n, heads, 128)
     assert nmax(o, ref) <= TOL
+
+
+@pytest.mark.parametrize("t", [0.0, 0.25, 0.75, 1.0])
+def test_blend_latents(t):
+    x = rand((32, 64, 64), 70)
+    noise = rand((32, 64, 64), 71)
+    out = torch.empty(32, 64, 64, device=DEV)
+    F.flux_blend_latents(x.to(DEV), noise.to(DEV), t, out)
+    ref = O.blend_latents(x.double(), noise.double(), t)
+    assert (out.cpu().double() - ref).abs().max() <= 1e-6
+    if t in (0.0, 1.0):
+        assert torch.equal(out.cpu(), x if t == 0.0 else noise)
