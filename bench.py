@@ -141,6 +141,10 @@ def barrier(world):
         dist.barrier()
 
 
+# the sources whose change invalidates the committed DRAM-traffic figure of the pair GEMM
+GEMM_TRAFFIC_SOURCES = ("gemm_tc2.cu", "gemm_epilogue.cuh", "pair.cuh", "common.cuh")
+
+
 def profile_traffic(kernel_files, profile):
     """DRAM bytes per GFLOP from a committed ncu summary, if it matches the current kernel sources."""
     srcs = [os.path.join(ROOT, "latent_flow_matching_b200", "csrc", f) for f in kernel_files]
@@ -330,7 +334,7 @@ def run_ours(args, w):
     a_ms, a_fl, a_by, a_n = prof["attention"]
     gemm_tflops = g_fl / (g_ms / 1e3) / 1e12
     attn_tflops = a_fl / (a_ms / 1e3) / 1e12
-    traffic_per_gflop, src_sha = profile_traffic(("gemm_tc2.cu", "gemm_epilogue.cuh"), "gemm_tc2_t2i1024.md")
+    traffic_per_gflop, src_sha = profile_traffic(GEMM_TRAFFIC_SOURCES, "gemm_tc2_t2i1024.md")
     traffic = None if traffic_per_gflop is None else traffic_per_gflop * (g_fl / g_n) / 1e9
     kinds = {k: {"ms_per_forward": round(v_[0] / args.steps, 4), "launches_per_forward": v_[3] // args.steps,
                  "achieved": round((v_[1] / (v_[0] / 1e3) / 1e12) if v_[1] else (v_[2] / (v_[0] / 1e3) / 1e9), 1),

@@ -9,16 +9,19 @@
 //   warps 0..3   softmax of tile A   (one thread per query row)
 //   warps 4..7   softmax of tile B
 //   warp 8       TMA: Q_A, Q_B once, then K_j / V_j into 2- and 3-deep rings
-//   warp 9       one thread issues tcgen05.mma in the order
+//   warp 9       issues tcgen05.mma (warp-convergent code, one elected lane) in the order
 //                  S_A(0) S_B(0) | PV_A(0) S_A(1) PV_B(0) S_B(1) | PV_A(1) S_A(2) ...
 //                so the tensor core works on one tile while the other tile's
 //                softmax runs, and S_X(j) is issued after PV_X(j-1): when a
 //                softmax warpgroup sees S_X(j), O_X already holds every earlier
 //                P V and can be rescaled in place without another wait.
-// Softmax: read S from TMEM, online softmax in the exp2 domain, write P as packed
-// bf16 over the S columns (the PV MMA reads its A operand from TMEM), rescale the
-// O row only when the running max grows by more than 8 (log2 units; P stays below
-// 2^8), and at the end write O / l as bf16.  setmaxnreg moves registers from the
+// Softmax: read S from TMEM, online softmax in the exp2 domain, rescale the O row
+// only when the running max grows by more than 8 (log2 units; P stays below 2^8),
+// write P as packed bf16 over the S columns (the PV MMA reads its A operand from
+// TMEM), and at the end write O / l as bf16.  Packed f32x2 arithmetic and 3-input
+// maxima halve the FMA/ADD/MAX issue slots, and one exponential pair in three is
+// evaluated on the FMA pipe so the MUFU unit, which otherwise runs at the tensor
+// core's pace, is off the critical path.  setmaxnreg moves registers from the
 // control warpgroup to the two softmax warpgroups.
 //
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
@@ -44,9 +47,10 @@ constexpr int kSmemBytes = kTileBytes * (kQTiles + kStagesK + kStagesV) + 1024 +
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOCol = 256;
 constexpr float kRescaleThreshold = 8.0f;
-// 384 threads x 168 registers at launch = 256 x 224 (softmax) + 128 x 56 (control)
-constexpr int kSoftmaxRegs = 224;
-constexpr int kControlRegs = 56;
+// 384 threads x 168 registers at launch >= 256 x 200 (softmax) + 128 x 96 (control); the control
+// warps (TMA producer, MMA issuer) need 96 to run without spilling
+constexpr int kSoftmaxRegs = 200;
+constexpr int kControlRegs = 96;
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -54,25 +58,34 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, to take part of the exponentials off the MUFU unit: split
-// x = j + f with j the nearest integer (|f| <= 1/2) by the 1.5 * 2^23 rounding
-// trick, evaluate 2^f with a cubic minimax polynomial (coefficients from a Remez
-// exchange fit of 2^f on [-1/2, 1/2]; max relative error 7.5e-5, well below the
-// 2^-9 of the bf16 P it feeds), and add j to the exponent field.  Inputs below
-// -126 are clamped (their weight is < 2^-126).
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(0.0551716685f, f, 0.2426111251f), f, 0.6932609677f), f, 0.9999280572f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+// 2^x on the FMA pipe for two lanes at once (packed f32x2 arithmetic), to take part of the
+// exponentials off the MUFU unit: split x = j + f with j the nearest integer (|f| <= 1/2) by
+// the 1.5 * 2^23 rounding trick, evaluate 2^f with a cubic minimax polynomial (coefficients
+// from a Remez exchange fit of 2^f on [-1/2, 1/2]; max relative error 7.5e-5, well below the
+// 2^-9 of the bf16 P it feeds), and add j to the exponent field.  Inputs below -126 are
+// clamped (their weight is < 2^-126).
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);
+  const float2 t = __fadd2_rn(x, magic);
+  const float2 r = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __ffma2_rn(r, make_float2(-1.0f, -1.0f), x);
+  float2 p = __ffma2_rn(make_float2(0.0551716685f, 0.0551716685f), f, make_float2(0.2426111251f, 0.2426111251f));
+  p = __ffma2_rn(p, f, make_float2(0.6932609677f, 0.6932609677f));
+  p = __ffma2_rn(p, f, make_float2(0.9999280572f, 0.9999280572f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
-// one score pair in kPolyEvery goes through ex2_poly, the rest through MUFU ex2 (0: none)
-#ifndef FDIT_POLY_EVERY
-#define FDIT_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = FDIT_POLY_EVERY;
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// one score pair in kPolyEvery goes through ex2_poly2, the rest through MUFU ex2
+constexpr int kPolyEvery = 3;
 
 __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_constant__ AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
@@ -177,74 +190,77 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
         for (int i = 0; i < kStagesV; ++i)
           if (armed_v & (1u << i)) mbar_drain(&v_full[i], (par_v >> i) & 1u);
       }
-    } else if (warp == 9 && lane == 0) {
+    } else if (warp == 9) {
       // ------------------------------------------------------------ MMA issuer
       const uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, 0, 0);      // Q, K both K-major
       const uint32_t idesc_o = idesc_bf16_f32(kTile, kHeadDim, 0, 1);   // P K-major (TMEM), V MN-major
-      const uint32_t q_addr = smem_u32(sQ);
+      // Base descriptors are built once; each MMA adds a compile-time offset (one 64-bit add),
+      // which keeps this single issuing thread ahead of the tensor core.
+      const uint64_t q_desc0 = sw128_desc(smem_u32(sQ), 16, 1024);
+      const uint64_t k_desc0 = sw128_desc(smem_u32(sK), 16, 1024);
+      const uint64_t v_desc0 = sw128_desc(smem_u32(sV), kBoxBytes, 1024);
       auto issue_s = [&](int t, int j) {        // S_t(j) = Q_t K_j^T
-        const uint32_t k_addr = smem_u32(sK + (j % kStagesK) * kTileBytes);
-        const uint32_t qa = q_addr + t * kTileBytes;
+        const uint64_t qd = desc_advance(q_desc0, t * kTileBytes);
+        const uint64_t kd = desc_advance(k_desc0, (j % kStagesK) * kTileBytes);
         const uint32_t s_tmem = tmem_base + static_cast<uint32_t>(t * kTile);
 #pragma unroll
         for (int kk = 0; kk < kHeadDim / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          mma_ss(s_tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024), idesc_s,
-                 kk != 0 ? 1u : 0u);
+          mma_ss_warp(s_tmem, desc_advance(qd, off), desc_advance(kd, off), idesc_s, kk != 0 ? 1u : 0u);
         }
-        mma_commit(&s_full[t]);
+        mma_commit_warp(&s_full[t]);
       };
       auto issue_pv = [&](int t, int j) {       // O_t += P_t(j) V_j, P from TMEM
-        const uint32_t v_addr = smem_u32(sV + (j % kStagesV) * kTileBytes);
+        const uint64_t vd = desc_advance(v_desc0, (j % kStagesV) * kTileBytes);
         const uint32_t p_tmem = tmem_base + static_cast<uint32_t>(t * kTile);
         const uint32_t o_tmem = tmem_base + kOCol + static_cast<uint32_t>(t * kTile);
+        const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(o_tmem, p_tmem + kk * 8, sw128_desc(v_addr + kk * 2048, kBoxBytes, 1024), idesc_o,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+          mma_ts_warp(o_tmem, p_tmem + kk * 8, desc_advance(vd, kk * 2048), idesc_o, kk > 0 ? 1u : acc0);
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&k_full[0], 0, abort_flag);
+      auto wait_issue_pv = [&](int t, int j) -> bool {
+        if (!mbar_wait_warp(&p_full[t], j & 1, abort_flag)) return false;
+        tc_fence_after();
+        issue_pv(t, j);
+        return true;
+      };
+      bool ok = mbar_wait_warp(q_full, 0, abort_flag) && mbar_wait_warp(&k_full[0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
         issue_s(1, 0);
-        mma_commit(&k_empty[0]);                 // K_0 is no longer read
+        mma_commit_warp(&k_empty[0]);                 // K_0 is no longer read
       }
       for (int j = 0; ok && j < n_kv; ++j) {
-        const uint32_t ph = j & 1;
-        if (!mbar_wait(&p_full[0], ph, abort_flag) ||
-            !mbar_wait(&v_full[j % kStagesV], (j / kStagesV) & 1, abort_flag)) {
+        if (!mbar_wait_warp(&v_full[j % kStagesV], (j / kStagesV) & 1, abort_flag) || !wait_issue_pv(0, j)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        issue_pv(0, j);
         if (j + 1 < n_kv) {
-          if (!mbar_wait(&k_full[(j + 1) % kStagesK], ((j + 1) / kStagesK) & 1, abort_flag)) {
+          if (!mbar_wait_warp(&k_full[(j + 1) % kStagesK], ((j + 1) / kStagesK) & 1, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           issue_s(0, j + 1);
         } else {
-          mma_commit(&o_final[0]);
+          mma_commit_warp(&o_final[0]);
         }
-        if (!mbar_wait(&p_full[1], ph, abort_flag)) {
+        if (!wait_issue_pv(1, j)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        issue_pv(1, j);
-        mma_commit(&v_empty[j % kStagesV]);      // V_j is no longer read
+        mma_commit_warp(&v_empty[j % kStagesV]);      // V_j is no longer read
         if (j + 1 < n_kv) {
           issue_s(1, j + 1);
-          mma_commit(&k_empty[(j + 1) % kStagesK]);   // K_{j+1} is no longer read
+          mma_commit_warp(&k_empty[(j + 1) % kStagesK]);   // K_{j+1} is no longer read
         } else {
-          mma_commit(&o_final[1]);
+          mma_commit_warp(&o_final[1]);
         }
       }
-      if (!ok) atomicExch(&g_attn_error, kErrTimeoutMma);
-      mma_commit(drain);
+      if (!ok && lane == 0) atomicExch(&g_attn_error, kErrTimeoutMma);
+      mma_commit_warp(drain);
       mbar_drain(drain, 0);
     }
   } else {
@@ -278,56 +294,60 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
         for (int c = 0; c < kTile; ++c)
           if (c >= valid) s[c] = __float_as_uint(-INFINITY);
       }
-      // row max as 8 independent partial maxima (a single chain would serialise 128 dependent ops)
-      float mp[8];
+      // row max: 4 independent chains of 3-input maxima (one chain would serialise 64 dependent ops)
+      float mp[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mp[i] = __uint_as_float(s[i]);
+      for (int i = 0; i < 4; ++i) mp[i] = fmaxf(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]));
 #pragma unroll
-      for (int c = 8; c < kTile; ++c) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(s[c]));
-      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+      for (int c = 8; c < kTile; c += 2)
+        mp[(c >> 1) & 3] = max3f(mp[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+      const float mx = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
       const float mxs = mx * sl2;
       const bool warp_grow = __any_sync(0xffffffffu, mxs > m_run + kRescaleThreshold);
       const float m_use = warp_grow ? fmaxf(m_run, mxs) : m_run;
       const float alpha = ex2(m_run - m_use);     // 0 on the first tile, 1 when not moved
-      const float neg_m = -m_use;
-      float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};     // 8 independent partial sums
-#pragma unroll
-      for (int c = 0; c < kTile; c += 2) {        // P packed in place over the first half of s
-        const float x0 = fmaf(__uint_as_float(s[c]), sl2, neg_m);
-        const float x1 = fmaf(__uint_as_float(s[c + 1]), sl2, neg_m);
-        float p0, p1;
-        if (kPolyEvery > 0 && (c / 2) % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
-          p0 = ex2_poly(x0);
-          p1 = ex2_poly(x1);
-        } else {
-          p0 = ex2(x0);
-          p1 = ex2(x1);
-        }
-        sp[(c / 2) & 7] += p0 + p1;
-        s[c / 2] = pack_bf16x2(p0, p1);
-      }
-      const float sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
-      tmem_st32(s_addr + 0, *reinterpret_cast<const uint32_t(*)[32]>(&s[0]));
-      tmem_st32(s_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(&s[32]));
-      l_run = l_run * alpha + sum;
       if (warp_grow && j > 0) {
-        // S_t(j) was issued after PV_t(j-1), so O_t is complete up to tile j-1 here
+        // S_t(j) was issued after PV_t(j-1), so O_t is complete up to tile j-1 here and is
+        // rescaled before P_t(j) lets PV_t(j) start
 #pragma unroll 1
         for (int c = 0; c < kHeadDim; c += 32) {
           uint32_t o[32];
           tmem_ld32(o_addr + c, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          for (int e = 0; e < 32; e += 2) {
+            const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])),
+                                        make_float2(alpha, alpha));
+            o[e] = __float_as_uint(v.x);
+            o[e + 1] = __float_as_uint(v.y);
+          }
           tmem_st32(o_addr + c, o);
         }
       }
-      m_run = m_use;
+      const float2 sl2_2 = make_float2(sl2, sl2);
+      const float2 neg_m2 = make_float2(-m_use, -m_use);
+      float2 sp[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int c = 0; c < kTile; c += 2) {        // P packed in place over the first half of s
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2_2, neg_m2);
+        float2 p;
+        if ((c / 2) % kPolyEvery == kPolyEvery - 1) {
+          p = ex2_poly2(x);
+        } else {
+          p = make_float2(ex2(x.x), ex2(x.y));
+        }
+        sp[(c >> 1) & 3] = __fadd2_rn(sp[(c >> 1) & 3], p);
+        s[c / 2] = pack_bf16x2(p.x, p.y);
+      }
+      tmem_st32(s_addr + 0, *reinterpret_cast<const uint32_t(*)[32]>(&s[0]));
+      tmem_st32(s_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(&s[32]));
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[t]);
+      const float2 s01 = __fadd2_rn(__fadd2_rn(sp[0], sp[1]), __fadd2_rn(sp[2], sp[3]));
+      l_run = l_run * alpha + (s01.x + s01.y);
+      m_run = m_use;
     }
     if (ok && mbar_wait(&o_final[t], 0, abort_flag)) {
       tc_fence_after();

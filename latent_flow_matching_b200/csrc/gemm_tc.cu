@@ -143,51 +143,50 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
+    {
+      // ------------------------------------------------------------ MMA issuer (whole warp, one elected lane issues)
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
+      const uint64_t a_desc0 = sw128_desc(smem_u32(sA), 16, 1024);
+      const uint64_t b_desc0 = sw128_desc(smem_u32(sB), 16, 1024);
       for (int tile = blockIdx.x; ok && tile < P.total_tiles; tile += gridDim.x) {
         const int p = find_problem(P, tile);
         const GemmProblem& pr = P.prob[p];
         const int nk = pr.K / BK;
         const uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
-        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
+        if (!mbar_wait_warp(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+          if (!mbar_wait_warp(&full[stage], phase, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * C::A_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * C::B_BYTES);
+          const uint64_t ad = desc_advance(a_desc0, stage * C::A_BYTES);
+          const uint64_t bd = desc_advance(b_desc0, stage * C::B_BYTES);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t ad = sw128_desc(a_addr + k * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(b_addr + k * 32, 16, 1024);
-            mma_ss(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
-          }
-          mma_commit(&empty[stage]);           // frees the smem stage once these MMAs retire
+          for (int k = 0; k < BK / 16; ++k)
+            mma_ss_warp(d_tmem, desc_advance(ad, k * 32), desc_advance(bd, k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+          mma_commit_warp(&empty[stage]);           // frees the smem stage once these MMAs retire
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit(&acc_full[acc]);            // accumulator ready for the epilogue
+        mma_commit_warp(&acc_full[acc]);            // accumulator ready for the epilogue
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
-      if (!ok) atomicExch(&g_gemm_error, kErrTimeoutMma);
-      mma_commit(drain);                       // every MMA issued by this thread has retired ...
+      if (!ok && lane == 0) atomicExch(&g_gemm_error, kErrTimeoutMma);
+      mma_commit_warp(drain);                       // every MMA issued by the elected lane has retired ...
       mbar_drain(drain, 0);                    // ... before TMEM is released
     }
   } else {

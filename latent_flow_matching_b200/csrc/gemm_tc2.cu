@@ -9,7 +9,7 @@
 // instruction does twice the work and each SM stages half as many W bytes per FLOP.
 //
 // Roles per CTA (6 warps, same as the one-CTA kernel): warp 0 TMA producer, warp 1 MMA issuer
-// (leader CTA only) and TMEM allocator, warps 2..5 epilogue of this CTA's 128 accumulator rows.
+// (leader CTA only, one elected lane of a convergent warp) and TMEM allocator, warps 2..5 epilogue of this CTA's 128 accumulator rows.
 // Barrier protocol:
 //   full[s]      leader only: 2 arrivals (one expect_tx from each CTA's producer) + the bytes
 //   empty[s]     both CTAs: the leader's MMA commit multicasts one arrival to each
@@ -130,48 +130,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
-      // ------------------------------------------------------------ MMA issuer (leader only)
+    if (rank == 0) {
+      // ------------------------------------------------------------ MMA issuer (leader only; whole warp, one elected lane issues)
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       const uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
+      const uint64_t a_desc0 = sw128_desc(smem_u32(sA), 16, 1024);
+      const uint64_t b_desc0 = sw128_desc(smem_u32(sB), 16, 1024);
       for (int tile = pair; ok && tile < P.total_tiles; tile += num_pairs) {
         const int p = find_problem(P, tile);
         const int nk = P.prob[p].K / BK;
-        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
+        if (!mbar_wait_warp(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+          if (!mbar_wait_warp(&full[stage], phase, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
+          const uint64_t ad = desc_advance(a_desc0, stage * A_BYTES);
+          const uint64_t bd = desc_advance(b_desc0, stage * B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            mma_pair(d_tmem, sw128_desc(a_addr + k * 32, 16, 1024), sw128_desc(b_addr + k * 32, 16, 1024), idesc,
-                     (kb | k) != 0 ? 1u : 0u);
-          mma_commit_pair(&empty[stage]);            // frees this stage in both CTAs
+            mma_pair_warp(d_tmem, desc_advance(ad, k * 32), desc_advance(bd, k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+          mma_commit_pair_warp(&empty[stage]);            // frees this stage in both CTAs
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        mma_commit_pair(&acc_full[acc]);             // accumulator halves ready in both CTAs
+        mma_commit_pair_warp(&acc_full[acc]);             // accumulator halves ready in both CTAs
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
-      if (!ok) atomicExch(&g_gemm2_error, kErrTimeoutMma);
-      mma_commit_pair_local(drain);
+      if (!ok && lane == 0) atomicExch(&g_gemm2_error, kErrTimeoutMma);
+      mma_commit_pair_local_warp(drain);
       mbar_drain(drain, 0);
     }
   } else {

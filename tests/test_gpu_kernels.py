@@ -198,8 +198,8 @@ def test_linear_full_size_sampled_rows():
 
 
 # ---------------------------------------------------------------------------- attention
-@pytest.mark.parametrize("n,heads,qscale", [(1, 2, 1.0), (77, 3, 1.0), (128, 1, 1.0), (300, 2, 1.0),
-                                            (1030, 2, 1.0), (700, 2, 6.0)])
+@pytest.mark.parametrize("n,heads,qscale", [(1, 2, 1.0), (77, 3, 1.0), (128, 1, 1.0), (200, 2, 1.0), (300, 2, 1.0),
+                                            (1030, 2, 1.0), (700, 2, 6.0), (2500, 1, 4.0)])
 def test_attention(n, heads, qscale):
     q = bf(rand((n, heads, 128), 30, qscale))
     k = bf(rand((n, heads, 128), 31))
