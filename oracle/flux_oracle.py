@@ -45,6 +45,9 @@ Readings where the pages are silent (each is listed in the design doc):
 * img2img strength s: run the last floor(S s) steps, starting from
   (1 - t) x_in + t noise at the first kept t.  Several references: reference k at
   RoPE l = -(k+1), tokens appended in order after the image tokens.
+* guidance g: v = v_u + g (v_c - v_u) with v_u the velocity for an unconditional text
+  of the same token count (prompts are padded and the padding is attended, so both
+  passes see sequences of one length).
 """
 from __future__ import annotations
 
@@ -56,7 +59,7 @@ __all__ = [
     "pack_latents", "unpack_latents", "token_positions", "rope_angles", "apply_rope",
     "layer_norm", "rms_norm", "modulate", "silu", "linear", "attention_probs",
     "attention", "timestep_embedding", "double_block", "single_block", "forward",
-    "schedule", "euler_update", "img2img_start", "blend_latents", "sample", "weight",
+    "schedule", "euler_update", "img2img_start", "blend_latents", "guided_velocity", "sample", "weight",
 ]
 
 CPU = torch.device("cpu")
@@ -355,15 +358,30 @@ def blend_latents(x: torch.Tensor, noise: torch.Tensor, t: float) -> torch.Tenso
     return (1.0 - t) * x + t * noise
 
 
+# ----------------------------------------------------------------------------
+# Classifier-free guidance [hakusoku.com story 4662, "CライブラリAPI": the parameter
+# struct carries guidance_scale, the CFG scale; "FLUX.3 Image Klein: offene Gewichte
+# ..." (kimiseek), opening section: the base checkpoint samples 50 steps with guidance,
+# the distilled one 16 steps without; we0.ai article on FLUX 3 Image Klein, checkpoint
+# table: Klein Base, 50 steps, guidance 3.5]
+# ----------------------------------------------------------------------------
+def guided_velocity(v_cond: torch.Tensor, v_uncond: torch.Tensor, g: float) -> torch.Tensor:
+    """Reading (the pages name the scale, not the formula): extrapolate from the velocity of
+    the unconditional text towards that of the prompt, v_u + g (v_c - v_u)."""
+    return v_uncond + g * (v_cond - v_uncond)
+
+
 def sample(p, hp, latent, txt, n_steps, ref_latent=None, dtype=torch.float64, on_step=None,
-           init_latent=None, strength=1.0):
+           init_latent=None, strength=1.0, txt_uncond=None, guidance=None):
     """Run the sampler; returns (final latent [32, h8, w8], list of velocities [Ni, 128]).
 
     ``latent`` is the noise.  ``ref_latent`` is one reference latent or a list of them
     (context tokens, never updated).  With ``init_latent`` (the latent of an image to
     edit) and ``strength`` < 1 the run starts at schedule step img2img_start(S, strength)
-    from blend_latents(init_latent, latent, t_start).  ``on_step(i, v)`` is called after
-    every forward if given.
+    from blend_latents(init_latent, latent, t_start).  With ``guidance`` g, every step
+    runs the forward once with ``txt`` and once with ``txt_uncond`` (same image and
+    references) and moves along guided_velocity; the returned velocities are the guided
+    ones.  ``on_step(i, v)`` is called after every step if given.
     """
     latent = torch.as_tensor(latent).to(dtype)
     c, h8, w8 = latent.shape
@@ -382,6 +400,9 @@ def sample(p, hp, latent, txt, n_steps, ref_latent=None, dtype=torch.float64, on
     vs = []
     for i in range(start, n_steps):
         v = forward(p, hp, tok, txt, ts[i], (h8 // 2, w8 // 2), ref_toks, ref_grids, dtype)
+        if guidance is not None:
+            v_u = forward(p, hp, tok, txt_uncond, ts[i], (h8 // 2, w8 // 2), ref_toks, ref_grids, dtype)
+            v = guided_velocity(v, v_u, guidance)
         vs.append(v)
         if on_step is not None:
             on_step(i, v)

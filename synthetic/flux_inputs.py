@@ -66,6 +66,7 @@ class Workload:
     n_steps: int
     dims: FluxDims
     extra_refs: tuple = ()  # sides of further reference images, after ref_image
+    guidance: float | None = None   # classifier-free guidance scale (None: unguided)
 
     @property
     def grid(self) -> int:       # image tokens per side (16 px per token)
@@ -106,6 +107,10 @@ WORKLOADS = {
     "t2i1024": Workload("t2i1024", 3, 1024, 512, 0, 4, FULL_DIMS),
     "i2i1024": Workload("i2i1024", 4, 1024, 512, 1024, 4, FULL_DIMS),
     "mref1024": Workload("mref1024", 5, 1024, 512, 512, 4, FULL_DIMS, extra_refs=(512,)),
+    # guided sampling: the base checkpoint's 3.5 (its 50 steps on the 1024^2 workload; the
+    # 256^2 golden case keeps 4 steps so the oracle finishes in minutes)
+    "cfg256": Workload("cfg256", 6, 256, 512, 0, 4, FULL_DIMS, guidance=3.5),
+    "cfg1024": Workload("cfg1024", 7, 1024, 512, 0, 50, FULL_DIMS, guidance=3.5),
 }
 
 
@@ -225,4 +230,15 @@ def make_inputs(w: Workload):
     refs = [draw(2 + k, (32, r // 8, r // 8)) for k, r in enumerate(w.ref_images)]
     ref = None if not refs else (refs[0] if len(refs) == 1 else refs)
     return latent, txt, ref
+
+
+UNCOND_KEY = 100
+
+
+def make_uncond_text(w: Workload):
+    """The unconditional text of a guided workload: same token count as the prompt (prompts
+    are padded to one length), N(0,1) features rounded to bf16, its own generator stream."""
+    g = np.random.default_rng([w.seed, INPUT_KEY + UNCOND_KEY])
+    x = g.standard_normal(w.n_txt * w.dims.txt_dim, dtype=np.float32)
+    return bf16_bits_to_f32(round_to_bf16_bits(x)).reshape(w.n_txt, w.dims.txt_dim)
 

@@ -7,7 +7,8 @@ step's velocity and the final packed latent:
 
     <workload>.npz: rows int32 [R], v float32 [S, R, 128], final float32 [R, 128]
 
-Row sets: all rows at 256^2, every 2nd at 512^2, every 8th at 1024^2.
+Row sets: all rows at 256^2, every 2nd at 512^2, every 8th at 1024^2.  For a guided workload
+the stored velocities are the guided ones.
 
 Usage: python tests/golden/make_goldens.py [workload ...]   (about an hour on 8 cores)
 """
@@ -22,10 +23,10 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, os.path.dirname(os.path.dirname(HERE)))
 
-from synthetic import WORKLOADS, make_weights, make_inputs  # noqa: E402
+from synthetic import WORKLOADS, make_weights, make_inputs, make_uncond_text  # noqa: E402
 from oracle import flux_oracle as O  # noqa: E402
 
-ROW_STRIDE = {"t2i256": 1, "t2i512": 2, "t2i1024": 8, "i2i1024": 8, "mref1024": 8}
+ROW_STRIDE = {"t2i256": 1, "t2i512": 2, "t2i1024": 8, "i2i1024": 8, "mref1024": 8, "cfg256": 1}
 
 
 def rows_for(name):
@@ -50,10 +51,13 @@ def make(name):
             ref = [torch.from_numpy(r) for r in ref]
         elif ref is not None:
             ref = torch.from_numpy(ref)
+        guided = {}
+        if w.guidance is not None:
+            guided = {"txt_uncond": torch.from_numpy(make_uncond_text(w)), "guidance": w.guidance}
         final, _ = O.sample(p, O.hyper(w.dims), torch.from_numpy(lat), torch.from_numpy(txt),
-                            w.n_steps, ref, dtype=torch.float32, on_step=on_step)
+                            w.n_steps, ref, dtype=torch.float32, on_step=on_step, **guided)
     final_tok = O.pack_latents(final)[rows].float().numpy()
-    meta = {"workload": name, "seed": w.seed, "oracle_dtype": "float32", "n_steps": w.n_steps,
+    meta = {"workload": name, "seed": w.seed, "oracle_dtype": "float32", "n_steps": w.n_steps, "guidance": w.guidance,
             "row_stride": ROW_STRIDE[name], "seconds": round(time.time() - t0, 1)}
     np.savez(os.path.join(HERE, f"{name}.npz"), rows=rows, v=np.stack(vs), final=final_tok,
              meta=np.array(json.dumps(meta)))

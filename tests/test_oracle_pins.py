@@ -524,3 +524,55 @@ def test_weight_widening_is_exact():
     w = O.weight({"w": bits}, "w", F64)
     ref = [1.0, -1.0, 0.0, 3.140625, 3.3895313892515355e38, 9.183549615799121e-41]
     assert w.tolist() == ref
+
+
+# ---------------------------------------------------------------------------- classifier-free guidance
+def _guidance_case(seed):
+    p = micro_params(seed)
+    gen = torch.Generator().manual_seed(100 + seed)
+    noise = torch.randn(32, 4, 6, generator=gen, dtype=F64)
+    txt_c = torch.randn(5, MICRO.txt_dim, generator=gen, dtype=F64)
+    txt_u = torch.randn(5, MICRO.txt_dim, generator=gen, dtype=F64)
+    return p, noise, txt_c, txt_u
+
+
+def test_guidance_one_and_zero_select_one_text():
+    """g = 1 follows the prompt alone, g = 0 the unconditional text alone (which side is which)."""
+    p, noise, txt_c, txt_u = _guidance_case(13)
+    cond, vc = O.sample(p, hp_of(MICRO), noise, txt_c, 3)
+    uncond, vu = O.sample(p, hp_of(MICRO), noise, txt_u, 3)
+    g1, v1 = O.sample(p, hp_of(MICRO), noise, txt_c, 3, txt_uncond=txt_u, guidance=1.0)
+    g0, v0 = O.sample(p, hp_of(MICRO), noise, txt_c, 3, txt_uncond=txt_u, guidance=0.0)
+    assert torch.allclose(g1, cond, atol=1e-12, rtol=0) and torch.allclose(g0, uncond, atol=1e-12, rtol=0)
+    for a, b in zip(v1, vc):
+        assert torch.allclose(a, b, atol=1e-12, rtol=0)
+    assert (cond - uncond).abs().max() > 1e-3          # the two texts do steer differently
+
+
+def test_guidance_with_identical_texts_is_unguided():
+    p, noise, txt_c, _ = _guidance_case(14)
+    g = json.load(open(os.path.join(GOLDEN, "guidance.json")))
+    plain, _ = O.sample(p, hp_of(MICRO), noise, txt_c, 2)
+    guided, _ = O.sample(p, hp_of(MICRO), noise, txt_c, 2, txt_uncond=txt_c.clone(), guidance=g["base_guidance"])
+    assert torch.allclose(guided, plain, atol=1e-12, rtol=0)
+
+
+def test_guided_velocity_is_affine_in_the_scale():
+    """One step from the same state: v(g) = (1 - g) v(0) + g v(1) also outside [0, 1] (no clamping)."""
+    p, noise, txt_c, txt_u = _guidance_case(15)
+    g = json.load(open(os.path.join(GOLDEN, "guidance.json")))["base_guidance"]
+    vs = {}
+    for s in (0.0, 1.0, g):
+        _, v = O.sample(p, hp_of(MICRO), noise, txt_c, 1, txt_uncond=txt_u, guidance=s)
+        vs[s] = v[0]
+    assert torch.allclose(vs[g], (1 - g) * vs[0.0] + g * vs[1.0], atol=1e-12, rtol=0)
+    assert (vs[g] - vs[1.0]).abs().max() > 1e-3
+
+
+def test_guidance_settings_from_pages():
+    g = json.load(open(os.path.join(GOLDEN, "guidance.json")))
+    assert g["base_steps"] == 50 and g["base_guidance"] == 3.5
+    assert g["distilled_steps"] == 16 and g["distilled_guidance"] is None
+    # the base schedule: 51 evenly spaced times from 1 to 0
+    ts = O.schedule(g["base_steps"])
+    assert len(ts) == 51 and ts[0] == 1.0 and ts[-1] == 0.0 and abs(ts[25] - 0.5) < 1e-7
