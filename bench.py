@@ -32,7 +32,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synthetic import WORKLOADS, make_weights, make_inputs  # noqa: E402
+from synthetic import WORKLOADS, make_weights, make_inputs, make_uncond_text  # noqa: E402
 
 METRIC = "ms per DiT forward & TFLOP/s at 1024^2 (4096+512 tok), % of BF16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -48,6 +48,15 @@ def forward_flops(w):
     total = (d.n_double + d.n_single) * per_block
     total += 2.0 * (w.n_img + w.n_ref) * C * D + 2.0 * w.n_txt * d.txt_dim * D + 2.0 * w.n_img * D * C
     return total
+
+
+def n_sequences(w):
+    """Sequences per forward: 2 for a guided workload (prompt and unconditional text in one batch)."""
+    return 1 if w.guidance is None else 2
+
+
+def step_unit(w):
+    return "ms/forward" if w.guidance is None else "ms/guided step (batch-2 forward)"
 
 
 def single_block_flops(w):
@@ -197,7 +206,7 @@ def run_reference(args, w):
     x = torch.randn(w.n_tokens, D, generator=g)
     s = torch.randn(D, generator=g)
     ang = O.rope_angles(O.token_positions(w.n_txt, w.grid, w.grid, ref_grids=w.ref_grids), 128, 1e4).float()
-    scale = forward_flops(w) / single_block_flops(w)
+    scale = n_sequences(w) * forward_flops(w) / single_block_flops(w)
     for _ in range(args.warmup):
         O.single_block(params, 0, x, s, ang, hp, torch.float32)
     times = []
@@ -208,19 +217,19 @@ def run_reference(args, w):
     ms_block = 1e3 * sum(times) / len(times)
     value = ms_block * scale
     sample = (f"one single-stream block at the full {w.name} size ({w.n_tokens} tokens) per step, fp32 oracle; "
-              f"value scaled by forward FLOPs / block FLOPs = {scale:.2f}")
+              f"value scaled by (sequences x forward FLOPs) / block FLOPs = {scale:.2f}")
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "ms/forward",
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": step_unit(w),
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_block, 3),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded N(0,1) bf16-rounded weights and inputs)",
         "config": {"workload": f"{w.name}: {w.image}x{w.image}, {w.n_img} image + {w.n_txt} text + {w.n_ref} "
                                f"reference tokens, 5 double + 20 single blocks, width 3072", "seq_len": w.n_tokens,
                    "global_batch": 1, "parallelism": "CPU oracle on rank 0"},
-        "tflops": round(forward_flops(w) / (value / 1e3) / 1e12, 4),
-        "cpu_baseline": {"value": round(value, 3), "unit": "ms/forward", "cores": torch.get_num_threads(),
+        "tflops": round(n_sequences(w) * forward_flops(w) / (value / 1e3) / 1e12, 4),
+        "cpu_baseline": {"value": round(value, 3), "unit": step_unit(w), "cores": torch.get_num_threads(),
                          "kind": "oracle", "sample": sample},
-        "e2e": {"value": round(value, 3), "unit": "ms/forward", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": round(value, 3), "unit": step_unit(w), "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -258,14 +267,27 @@ def run_ours(args, w):
             row += h * w_
         ref_hw = w.ref_grids if isinstance(ref_h, list) else w.ref_grids[0]
     ts = F.euler_schedule(w.n_steps)
+    guided = w.guidance is not None
+    txt_u_h = make_uncond_text(w) if guided else None
+    txt_u = torch.from_numpy(txt_u_h).to(dev) if guided else None
+    v_u = torch.empty_like(tok)
+    hw_list = list(w.ref_grids)
+
+    def forward_update(k):
+        """The forward(s) of one sampling step and its Euler update."""
+        if guided:
+            model.forward_cfg(tok, (gh, gh), txt, txt_u, ts[k], v, v_u, ref_tok, hw_list)
+            F.flux_cfg_euler_step(tok, v, v_u, w.guidance, ts[k + 1] - ts[k])
+        else:
+            model.forward(tok, (gh, gh), txt, ts[k], v, ref_tok, ref_hw)
+            F.flux_euler_step(tok, v, ts[k + 1] - ts[k])
 
     def step(i, lat_buf):
         k = i % w.n_steps
         if k == 0:
             lat_buf.copy_(lat0)                     # every sampling run starts from the same noise
         F.flux_pack_latents(lat_buf, tok)
-        model.forward(tok, (gh, gh), txt, ts[k], v, ref_tok, ref_hw)
-        F.flux_euler_step(tok, v, ts[k + 1] - ts[k])
+        forward_update(k)
         F.flux_unpack_latents(tok, lat_buf)
 
     for i in range(args.warmup):
@@ -305,6 +327,7 @@ def run_ours(args, w):
     # ---- end to end through host buffers (pinned), H2D inputs and D2H latent every step
     lat_pin = torch.from_numpy(lat_h).pin_memory()
     txt_pin = torch.from_numpy(txt_h).pin_memory()
+    txt_u_pin = torch.from_numpy(txt_u_h).pin_memory() if guided else None
     out_pin = torch.empty_like(lat_pin).pin_memory()
     lat_d = torch.empty_like(lat0)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -315,20 +338,21 @@ def run_ours(args, w):
         k = i % w.n_steps
         lat_d.copy_(lat_pin if k == 0 else out_pin, non_blocking=True)
         txt.copy_(txt_pin, non_blocking=True)
+        if guided:
+            txt_u.copy_(txt_u_pin, non_blocking=True)
         F.flux_pack_latents(lat_d, tok)
-        model.forward(tok, (gh, gh), txt, ts[k], v, ref_tok, ref_hw)
-        F.flux_euler_step(tok, v, ts[k + 1] - ts[k])
+        forward_update(k)
         F.flux_unpack_latents(tok, lat_d)
         out_pin.copy_(lat_d, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = aggregate_ms_per_forward(max_over_ranks(e0.elapsed_time(e1), world), args.steps, world)
     assert torch.isfinite(out_pin).all()
-    h2d = lat_pin.numel() * 4 + txt_pin.numel() * 4
+    h2d = lat_pin.numel() * 4 + txt_pin.numel() * 4 * n_sequences(w)
     d2h = out_pin.numel() * 4
 
     peaks, peak_src = load_peaks()
-    flops = forward_flops(w)
+    flops = n_sequences(w) * forward_flops(w)
     tflops = flops / (ms_step / 1e3) / 1e12
     g_ms, g_fl, g_by, g_n = prof["gemm"]
     a_ms, a_fl, a_by, a_n = prof["attention"]
@@ -342,13 +366,15 @@ def run_ours(args, w):
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": round(value, 4), "unit": "ms/forward", "n_gpus": world,
+            "metric": METRIC, "value": round(value, 4), "unit": step_unit(w), "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) weights scaled 1/sqrt(fan_in), bf16; N(0,1) latent and text)",
             "config": {"workload": f"{w.name}: {w.image}x{w.image}, {w.n_img} image + {w.n_txt} text + {w.n_ref} "
                                    f"reference tokens ({len(w.ref_grids)} reference images), 5 double + 20 single "
-                                   f"blocks, width 3072, 24x128 heads, one Euler step (pack, forward, Euler, unpack)",
+                                   f"blocks, width 3072, 24x128 heads, one Euler step (pack, forward, Euler, unpack)"
+                                   + ("" if not guided else f"; guidance {w.guidance}: prompt and unconditional "
+                                      f"text as one batch-2 forward, fused guided Euler update"),
                        "global_batch": world, "seq_len": w.n_tokens,
                        "parallelism": f"replicas x{world}, no data-path collective",
                        "l2": "inputs larger than L2: 9.7 GB of bf16 weights streamed every forward"},
@@ -367,17 +393,18 @@ def run_ours(args, w):
                           "frac": round(attn_tflops / peaks["bf16_tflops_sustained"], 4),
                           "share_of_step": round(a_ms / args.steps / ms_step, 3)},
             "kernels": kinds,
-            "e2e": {"value": round(e2e_ms, 4), "unit": "ms/forward", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": round(e2e_ms, 4), "unit": step_unit(w), "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:
             ms_cpu, secs = cpu_oracle_sample(w, params, lat_h, txt_h, ref_h)
-            line["cpu_baseline"] = {"value": round(ms_cpu, 1), "unit": "ms/forward", "cores": torch.get_num_threads(),
-                                    "kind": "oracle",
+            line["cpu_baseline"] = {"value": round(ms_cpu * n_sequences(w), 1), "unit": step_unit(w),
+                                    "cores": torch.get_num_threads(), "kind": "oracle",
                                     "sample": f"one double + one single block at full {w.name} size, fp32 oracle "
-                                              f"({secs:.1f} s), scaled x5 and x20 to a forward"}
+                                              f"({secs:.1f} s), scaled x5 and x20 to a forward"
+                                              + ("" if not guided else ", x2 for the two guided sequences")}
         print(json.dumps(line), flush=True)
     model.close()
     if world > 1:

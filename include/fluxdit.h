@@ -121,6 +121,22 @@ FLUX_API int flux_dit_forward_refs(flux_dit *m, const float *img_tok, int grid_h
                                    int n_txt, const float *ref_tok, int n_refs, const int *ref_grids, float t,
                                    float *v_out, void *stream);
 
+/* Classifier-free guidance forward: the velocities of the prompt and of the unconditional
+ * text for the same image, references and t, as ONE batch of two sequences (every GEMM
+ * and attention launch covers both).  txt_cond and txt_uncond are fp32 [n_txt, 3072]
+ * device buffers with the same token count (prompts are padded to one length and the
+ * padding is attended: "FLUX.3 Image Klein in Diffusers: ...", section "Verarbeitung
+ * einzelner Prompts und Batching-Architektur"); v_cond and v_uncond are distinct fp32
+ * [grid_h*grid_w, 128] outputs.  The guidance scale is a sampler parameter (hakusoku.com
+ * story 4662, "CライブラリAPI": guidance_scale; base checkpoint: 50 steps at guidance 3.5,
+ * we0.ai FLUX 3 Image Klein article, checkpoint table); combine the two velocities with
+ * flux_cfg_euler_step.  The workspace holds both sequences (twice the rows of a
+ * single-text forward).  Otherwise as flux_dit_forward_refs; each velocity equals, bit for
+ * bit, what flux_dit_forward_refs returns for that text alone. */
+FLUX_API int flux_dit_forward_cfg(flux_dit *m, const float *img_tok, int grid_h, int grid_w, const float *txt_cond,
+                                  const float *txt_uncond, int n_txt, const float *ref_tok, int n_refs,
+                                  const int *ref_grids, float t, float *v_cond, float *v_uncond, void *stream);
+
 /* Diagnostic: run only the first n_double double blocks and n_single single
  * blocks in later forwards (-1 = all).  Used to bisect parity; not a model change. */
 FLUX_API int flux_dit_set_active_blocks(flux_dit *m, int n_double, int n_single);
@@ -135,6 +151,13 @@ FLUX_API int flux_dit_modulation(flux_dit *m, float t, float *mods_out, void *st
  * ("Flux 2 Klein: Reine C-basierte Inferenz", "Modellarchitektur und Leistung":
  * 4 sampling steps; t_i = linspace(1, 0, S+1), dt = t_{i+1} - t_i). */
 FLUX_API int flux_euler_step(float *x, const float *v, size_t n, float dt, void *stream);
+
+/* Guided Euler update in one pass: x += dt * (v_uncond + guidance * (v_cond - v_uncond)) over
+ * n fp32 values, in place.  The combination is the usual classifier-free guidance
+ * extrapolation; the pages name the scale but not the formula (see flux_dit_forward_cfg).
+ * x, v_cond, v_uncond 16-byte aligned device buffers; guidance and dt finite. */
+FLUX_API int flux_cfg_euler_step(float *x, const float *v_cond, const float *v_uncond, size_t n, float guidance,
+                                 float dt, void *stream);
 
 /* img2img start state: out = (1 - t) x + t noise over n fp32 values (x the latent of the
  * image to edit, noise N(0,1)): the flow-matching state at time t.  With strength s the
@@ -155,6 +178,12 @@ FLUX_API int flux_unpack_latents(const float *tok, float *lat, int h8, int w8, v
  * head_dim == 128, n >= 1.  fp32 softmax statistics, bf16 P, fp32 accumulation. */
 FLUX_API int flux_joint_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, uint16_t *o, int n, int heads,
                          int head_dim, float scale, void *stream);
+
+/* The same over a batch of independent sequences of n tokens each, stored one after
+ * another: q, k, v, o bf16 [batch * n, heads, 128]; sequence b attends only to its own
+ * rows [b n, (b + 1) n).  1 <= batch <= 65535. */
+FLUX_API int flux_joint_attention_batch(const uint16_t *q, const uint16_t *k, const uint16_t *v, uint16_t *o, int batch,
+                                        int n, int heads, int head_dim, float scale, void *stream);
 
 /* Kernel-level entry points of the forward's steps (for parity tests and reuse). */
 

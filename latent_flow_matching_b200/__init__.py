@@ -45,6 +45,9 @@ _SIGS = {
     "flux_dit_destroy": (None, [_P]),
     "flux_dit_forward": (_I, [_P, _P, _I, _I, _P, _I, _P, _I, _I, _F, _P, _P]),
     "flux_dit_forward_refs": (_I, [_P, _P, _I, _I, _P, _I, _P, _I, ctypes.POINTER(ctypes.c_int), _F, _P, _P]),
+    "flux_dit_forward_cfg": (_I, [_P, _P, _I, _I, _P, _P, _I, _P, _I, ctypes.POINTER(ctypes.c_int), _F, _P, _P,
+                                  _P]),
+    "flux_cfg_euler_step": (_I, [_P, _P, _P, _Z, _F, _F, _P]),
     "flux_blend_latents": (_I, [_P, _P, _F, _P, _Z, _P]),
     "flux_dit_set_active_blocks": (_I, [_P, _I, _I]),
     "flux_dit_modulation_size": (_Z, [_P]),
@@ -53,6 +56,7 @@ _SIGS = {
     "flux_pack_latents": (_I, [_P, _P, _I, _I, _P]),
     "flux_unpack_latents": (_I, [_P, _P, _I, _I, _P]),
     "flux_joint_attention": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P]),
+    "flux_joint_attention_batch": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P]),
     "flux_linear": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _I, _P, _P]),
     "flux_qkv_projection": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _I, _F, _P, _P]),
     "flux_layernorm_modulate": (_I, [_P, _P, _I, _I, _P, _P, _F, _P]),
@@ -167,6 +171,25 @@ class FluxDiT:
                                       float(t), _ptr(v_out, torch.float32, "v_out"), _stream(stream)))
         return v_out
 
+    def forward_cfg(self, img_tok, grid_hw, txt_cond, txt_uncond, t, v_cond, v_uncond, ref_tok=None, ref_hw=(),
+                    stream=None):
+        """Velocities for the prompt and the unconditional text in one batch-2 forward.
+        ref_hw: a list of (h, w) (ref_tok holds every reference's packed tokens), or ()."""
+        import torch
+        n_txt = 0 if txt_cond is None else txt_cond.shape[0]
+        if (0 if txt_uncond is None else txt_uncond.shape[0]) != n_txt:
+            raise ValueError("txt_cond and txt_uncond must have the same token count")
+        if ref_hw and not isinstance(ref_hw[0], (tuple, list)):
+            ref_hw = [tuple(ref_hw)] if ref_hw[0] else []
+        grids = (ctypes.c_int * max(1, 2 * len(ref_hw)))(*[v for hw in ref_hw for v in hw])
+        _check(lib().flux_dit_forward_cfg(self._h, _ptr(img_tok, torch.float32, "img_tok"), grid_hw[0], grid_hw[1],
+                                          _ptr(txt_cond, torch.float32, "txt_cond"),
+                                          _ptr(txt_uncond, torch.float32, "txt_uncond"), n_txt,
+                                          _ptr(ref_tok, torch.float32, "ref_tok"), len(ref_hw), grids, float(t),
+                                          _ptr(v_cond, torch.float32, "v_cond"),
+                                          _ptr(v_uncond, torch.float32, "v_uncond"), _stream(stream)))
+        return v_cond, v_uncond
+
     def set_active_blocks(self, n_double=-1, n_single=-1):
         _check(lib().flux_dit_set_active_blocks(self._h, n_double, n_single))
 
@@ -219,6 +242,15 @@ def flux_euler_step(x, v, dt, stream=None):
     return x
 
 
+def flux_cfg_euler_step(x, v_cond, v_uncond, guidance, dt, stream=None):
+    """x += dt * (v_uncond + guidance * (v_cond - v_uncond)), in place."""
+    import torch
+    _check(lib().flux_cfg_euler_step(_ptr(x, torch.float32, "x"), _ptr(v_cond, torch.float32, "v_cond"),
+                                     _ptr(v_uncond, torch.float32, "v_uncond"), x.numel(), float(guidance),
+                                     float(dt), _stream(stream)))
+    return x
+
+
 def flux_pack_latents(lat, tok, stream=None):
     import torch
     _check(lib().flux_pack_latents(_ptr(lat, torch.float32, "lat"), _ptr(tok, torch.float32, "tok"),
@@ -238,6 +270,17 @@ def flux_joint_attention(q, k, v, o, scale=None, stream=None):
     scale = hd ** -0.5 if scale is None else scale
     _check(lib().flux_joint_attention(_bits(q, "q"), _bits(k, "k"), _bits(v, "v"), _bits(o, "o"), n, heads, hd,
                                       float(scale), _stream(stream)))
+    return o
+
+
+def flux_joint_attention_batch(q, k, v, o, batch, scale=None, stream=None):
+    """q, k, v, o bf16 [batch * n, heads, 128]; sequence b attends within rows [b n, (b + 1) n)."""
+    rows, heads, hd = q.shape
+    if rows % batch:
+        raise ValueError("rows must be a multiple of batch")
+    scale = hd ** -0.5 if scale is None else scale
+    _check(lib().flux_joint_attention_batch(_bits(q, "q"), _bits(k, "k"), _bits(v, "v"), _bits(o, "o"), batch,
+                                            rows // batch, heads, hd, float(scale), _stream(stream)))
     return o
 
 
@@ -312,13 +355,16 @@ def flux_device_error(stream=None) -> int:
 
 
 def flux_sample(model: FluxDiT, latent, txt, n_steps, ref_latent=None, on_step=None, stream=None,
-                init_latent=None, strength=1.0):
+                init_latent=None, strength=1.0, txt_uncond=None, guidance=None):
     """Euler sampling on the device: pack -> S x (forward, Euler) -> unpack.
 
     latent fp32 [32, h8, w8] (device): the noise.  txt fp32 [n_txt, txt_dim] (device).
     ref_latent: one fp32 [32, r8, r8] latent, a list of them (context images), or None.
     init_latent (the latent of an image to edit) with strength s < 1: start from
     flux_blend_latents(init_latent, latent, t) at schedule step img2img_first_step(S, s).
+    With ``guidance`` g (and ``txt_uncond``, the unconditional text of the same length) each
+    step is one batch-2 forward and the fused guided Euler update; ``on_step(i, v)`` then sees
+    the guided velocity (computed for it only when a callback is given).
     Returns the final latent (new tensor).  ``on_step(i, v)`` sees each velocity.
     """
     import torch
@@ -342,6 +388,19 @@ def flux_sample(model: FluxDiT, latent, txt, n_steps, ref_latent=None, on_step=N
             row += h * w
         ref_hw = grids if isinstance(ref_latent, (list, tuple)) else grids[0]
     v = torch.empty_like(tok)
+    if guidance is not None:
+        if txt_uncond is None:
+            raise ValueError("guidance needs txt_uncond")
+        v_u = torch.empty_like(tok)
+        hw_list = ref_hw if (ref_hw and isinstance(ref_hw[0], (tuple, list))) else ([ref_hw] if ref_hw[0] else [])
+        for i in range(start, n_steps):
+            model.forward_cfg(tok, (gh, gw), txt, txt_uncond, ts[i], v, v_u, ref_tok, hw_list, stream)
+            if on_step is not None:
+                on_step(i, v_u + guidance * (v - v_u))
+            flux_cfg_euler_step(tok, v, v_u, guidance, ts[i + 1] - ts[i], stream)
+        out = torch.empty_like(latent)
+        flux_unpack_latents(tok, out, stream)
+        return out
     for i in range(start, n_steps):
         model.forward(tok, (gh, gw), txt, ts[i], v, ref_tok, ref_hw, stream)
         if on_step is not None:

@@ -4,6 +4,11 @@
 // Klein in Diffusers write-up, "Entkoppelte Vorverarbeitung und gemeinsame
 // Attention-Blöcke" and "Verarbeitung einzelner Prompts und Batching-Architektur".
 //
+// A batch of sequences of equal length n sits row after row in q, k, v and out; grid.z picks
+// the sequence and every row coordinate is offset by z * n.  Key tiles that run past a
+// sequence's end read the next sequence's rows (or the tensor map's zero fill) and are
+// masked like the ragged tail.
+//
 // CTA = two 128-row query tiles (A, B) of one head that share every K/V tile and
 // take turns on the tensor core, 12 warps in three warpgroups:
 //   warps 0..3   softmax of tile A   (one thread per query row)
@@ -108,8 +113,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * (kQTiles * kTile);
+  const int q0 = blockIdx.x * (kQTiles * kTile);      // first query row inside this sequence
   const int head = blockIdx.y;
+  const int row_base = blockIdx.z * P.n;               // first row of this sequence in q, k, v and out
   const int n_kv = (P.n + kTile - 1) / kTile;
 
   if (threadIdx.x == 0) {
@@ -154,13 +160,13 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
       const int vc = P.v_col0 + head * kHeadDim;
       mbar_arrive_expect_tx(q_full, kQTiles * kTileBytes);
       for (int t = 0; t < kQTiles; ++t) {
-        tma_load_2d(sQ + t * kTileBytes, &P.mapQ, q_full, qc, q0 + t * kTile);
-        tma_load_2d(sQ + t * kTileBytes + kBoxBytes, &P.mapQ, q_full, qc + kBox, q0 + t * kTile);
+        tma_load_2d(sQ + t * kTileBytes, &P.mapQ, q_full, qc, row_base + q0 + t * kTile);
+        tma_load_2d(sQ + t * kTileBytes + kBoxBytes, &P.mapQ, q_full, qc + kBox, row_base + q0 + t * kTile);
       }
       uint32_t armed_k = 0, armed_v = 0, par_k = 0, par_v = 0;   // per slot: armed once / parity of last arming
       bool ok = true;
       for (int j = 0; j < n_kv; ++j) {
-        const int r0 = j * kTile;
+        const int r0 = row_base + j * kTile;   // a tile past the sequence end reads masked rows
         const int sk = j % kStagesK, sv = j % kStagesV;
         const uint32_t pk = (j / kStagesK) & 1, pv = (j / kStagesV) & 1;
         if (!mbar_wait(&k_empty[sk], pk ^ 1u, abort_flag)) {
@@ -359,7 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
         tmem_ld32(o_addr + c, o);
         tmem_ld_wait();
         if (qrow < P.n) {
-          uint4* dst = reinterpret_cast<uint4*>(P.out + static_cast<size_t>(qrow) * P.ldo + head * kHeadDim + c);
+          uint4* dst = reinterpret_cast<uint4*>(P.out + static_cast<size_t>(row_base + qrow) * P.ldo +
+                                                head * kHeadDim + c);
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint32_t w[4];
@@ -394,8 +401,8 @@ cudaError_t attention_launch(const AttnParams& P, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  if (P.n <= 0 || P.heads <= 0) return cudaSuccess;
-  dim3 grid((P.n + kQTiles * kTile - 1) / (kQTiles * kTile), P.heads);
+  if (P.n <= 0 || P.heads <= 0 || P.batch <= 0) return cudaSuccess;
+  dim3 grid((P.n + kQTiles * kTile - 1) / (kQTiles * kTile), P.heads, P.batch);
   count_launch();
   attention_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(P);
   return cudaGetLastError();

@@ -88,7 +88,7 @@ __global__ void cast_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __r
 // mean and variance come from two block reductions, so many CTAs stay resident per SM.
 template <int VPT>
 __global__ void __launch_bounds__(256) ln_mod_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y,
-                                                     int rows, int split, const float* __restrict__ sh0,
+                                                     int rows, int split, int period, const float* __restrict__ sh0,
                                                      const float* __restrict__ sc0, const float* __restrict__ sh1,
                                                      const float* __restrict__ sc1, float eps) {
   constexpr int dim = 1024 * VPT;
@@ -125,8 +125,9 @@ __global__ void __launch_bounds__(256) ln_mod_kernel(const float* __restrict__ x
 #pragma unroll
   for (int w = 0; w < 8; ++w) q += red[1][w];
   const float rstd = rsqrtf(q * (1.0f / dim) + eps);
-  const float4* shp = reinterpret_cast<const float4*>(row < split ? sh0 : sh1);
-  const float4* scp = reinterpret_cast<const float4*>(row < split ? sc0 : sc1);
+  const bool first = row % period < split;
+  const float4* shp = reinterpret_cast<const float4*>(first ? sh0 : sh1);
+  const float4* scp = reinterpret_cast<const float4*>(first ? sc0 : sc1);
   uint2* yr = reinterpret_cast<uint2*>(y + static_cast<size_t>(row) * dim);
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(256) ln_mod_kernel(const float* __restrict__ x
 
 // Any dim that is a multiple of 4: three passes over the row in global memory.
 __global__ void ln_mod_generic_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y, int rows, int dim,
-                                      int split, const float* __restrict__ sh0, const float* __restrict__ sc0,
+                                      int split, int period, const float* __restrict__ sh0, const float* __restrict__ sc0,
                                       const float* __restrict__ sh1, const float* __restrict__ sc1, float eps) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -155,8 +156,8 @@ __global__ void ln_mod_generic_kernel(const float* __restrict__ x, __nv_bfloat16
   for (int i = lane; i < dim; i += 32) q += (xr[i] - mean) * (xr[i] - mean);
   for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
   const float rstd = rsqrtf(q / dim + eps);
-  const float* sh = warp < split ? sh0 : sh1;
-  const float* sc = warp < split ? sc0 : sc1;
+  const float* sh = warp % period < split ? sh0 : sh1;
+  const float* sc = warp % period < split ? sc0 : sc1;
   for (int i = lane; i < dim; i += 32)
     y[static_cast<size_t>(warp) * dim + i] = __float2bfloat16_rn((xr[i] - mean) * rstd * (1.f + sc[i]) + sh[i]);
 }
@@ -242,6 +243,25 @@ __global__ void rope_table_kernel(float2* __restrict__ table, int n_txt, int gh,
 }
 
 // (1 - t) x + t noise: the flow-matching state at time t between data (t = 0) and noise (t = 1)
+// x += dt * (v_u + g (v_c - v_u)): the guided velocity and the Euler step in one pass.
+__global__ void cfg_euler_kernel(float* __restrict__ x, const float* __restrict__ vc, const float* __restrict__ vu,
+                                 size_t n, float g, float dt) {
+  const size_t n4 = n / 4;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4; i += stride) {
+    float4 a = reinterpret_cast<float4*>(x)[i];
+    const float4 c = reinterpret_cast<const float4*>(vc)[i];
+    const float4 u = reinterpret_cast<const float4*>(vu)[i];
+    a.x = fmaf(dt, fmaf(g, c.x - u.x, u.x), a.x);
+    a.y = fmaf(dt, fmaf(g, c.y - u.y, u.y), a.y);
+    a.z = fmaf(dt, fmaf(g, c.z - u.z, u.z), a.z);
+    a.w = fmaf(dt, fmaf(g, c.w - u.w, u.w), a.w);
+    reinterpret_cast<float4*>(x)[i] = a;
+  }
+  for (size_t i = n4 * 4 + blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n; i += stride)
+    x[i] = fmaf(dt, fmaf(g, vc[i] - vu[i], vu[i]), x[i]);
+}
+
 __global__ void blend_kernel(const float* __restrict__ x, const float* __restrict__ noise, float t,
                              float* __restrict__ out, size_t n) {
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
@@ -329,6 +349,14 @@ cudaError_t euler_launch(float* x, const float* v, size_t n, float dt, cudaStrea
   return cudaGetLastError();
 }
 
+cudaError_t cfg_euler_launch(float* x, const float* vc, const float* vu, size_t n, float g, float dt,
+                             cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  count_launch();
+  cfg_euler_kernel<<<blocks_for((n + 3) / 4, 256), 256, 0, s>>>(x, vc, vu, n, g, dt);
+  return cudaGetLastError();
+}
+
 cudaError_t cast_bf16_launch(const float* x, __nv_bfloat16* y, size_t n, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   count_launch();
@@ -336,16 +364,17 @@ cudaError_t cast_bf16_launch(const float* x, __nv_bfloat16* y, size_t n, cudaStr
   return cudaGetLastError();
 }
 
-cudaError_t ln_modulate_launch(const float* x, __nv_bfloat16* y, int rows, int dim, int split, const float* shift0,
-                               const float* scale0, const float* shift1, const float* scale1, float eps,
-                               cudaStream_t s) {
+cudaError_t ln_modulate_launch(const float* x, __nv_bfloat16* y, int rows, int dim, int split, int period,
+                               const float* shift0, const float* scale0, const float* shift1, const float* scale1,
+                               float eps, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
+  if (period <= 0) return cudaErrorInvalidValue;
   count_launch();
   if (dim == 3072)
-    ln_mod_kernel<3><<<rows, 256, 0, s>>>(x, y, rows, split, shift0, scale0, shift1, scale1, eps);
+    ln_mod_kernel<3><<<rows, 256, 0, s>>>(x, y, rows, split, period, shift0, scale0, shift1, scale1, eps);
   else
-    ln_mod_generic_kernel<<<(rows + 7) / 8, 256, 0, s>>>(x, y, rows, dim, split, shift0, scale0, shift1, scale1,
-                                                          eps);
+    ln_mod_generic_kernel<<<(rows + 7) / 8, 256, 0, s>>>(x, y, rows, dim, split, period, shift0, scale0, shift1,
+                                                          scale1, eps);
   return cudaGetLastError();
 }
 

@@ -227,14 +227,21 @@ struct SingleW {
   CUtensorMap m_qkv, m_mlp, m_lin2;
 };
 
+constexpr int kMaxBatch = 2;            // sequences of one shape per forward (prompt and unconditional text)
+
+// Activations of a batch of nb sequences of one shape (nt text + ni image + nr reference rows
+// each), stored sequence after sequence: rows [b n, (b + 1) n) of X, Y, QKV, CC and the RoPE table
+// belong to sequence b.
 struct Workspace {
   size_t cap_n = 0, cap_tok = 0, cap_txt = 0;
   float* X = nullptr;
   bf16 *Y = nullptr, *QKV = nullptr, *CC = nullptr, *tokb = nullptr, *txtb = nullptr;
   float2* rope = nullptr;
-  int nt = -1, gh = -1, gw = -1;                        // shape the maps and the RoPE table were built for
+  int nt = -1, gh = -1, gw = -1, nb = -1;               // shape the maps and the RoPE table were built for
   RefGrids refs = {-1, {}, {}};
-  CUtensorMap a_txtb, a_tokb, a_Ytxt, a_Yimg, a_Yall, a_Yout, a_Otxt, a_Oimg, a_Htxt, a_Himg, a_CC, qkv;
+  CUtensorMap a_tokb, a_Yall, a_CC, qkv;                // shared image input; whole-batch views
+  CUtensorMap a_txtb[kMaxBatch], a_Ytxt[kMaxBatch], a_Yimg[kMaxBatch], a_Yout[kMaxBatch], a_Otxt[kMaxBatch],
+      a_Oimg[kMaxBatch], a_Htxt[kMaxBatch], a_Himg[kMaxBatch];   // per-sequence views
 };
 
 }  // namespace fdit
@@ -444,59 +451,65 @@ static bool same_refs(const RefGrids& a, const RefGrids& b) {
   return true;
 }
 
-static int prepare_shape(flux_dit* m, int nt, int gh, int gw, const RefGrids& refs, cudaStream_t s) {
+static int prepare_shape(flux_dit* m, int nt, int gh, int gw, const RefGrids& refs, int nb, cudaStream_t s) {
   Workspace& w = m->ws;
   const flux_dit_config& c = m->cfg;
   const size_t D = c.hidden, F = c.mlp_hidden;
   const size_t ni = static_cast<size_t>(gh) * gw, nr = ref_tokens(refs);
-  const size_t n = nt + ni + nr;
-  if (n > w.cap_n) {
+  const size_t n = nt + ni + nr, rows = n * nb;
+  if (rows > w.cap_n) {
     float* X = nullptr;
     free_ws(w);
-    const size_t need = n;
-    bool ok = cudaMalloc(&X, need * D * 4) == cudaSuccess;
+    bool ok = cudaMalloc(&X, rows * D * 4) == cudaSuccess;
     w.X = X;
-    ok = ok && cudaMalloc(&w.Y, need * D * 2) == cudaSuccess;
-    ok = ok && cudaMalloc(&w.QKV, need * 3 * D * 2) == cudaSuccess;
-    ok = ok && cudaMalloc(&w.CC, need * (D + F) * 2) == cudaSuccess;
-    ok = ok && cudaMalloc(&w.rope, need * 64 * sizeof(float2)) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.Y, rows * D * 2) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.QKV, rows * 3 * D * 2) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.CC, rows * (D + F) * 2) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.rope, rows * 64 * sizeof(float2)) == cudaSuccess;
     if (!ok) {
       free_ws(w);
-      return fail(FLUX_ENOMEM, "workspace allocation for %zu tokens failed", need);
+      return fail(FLUX_ENOMEM, "workspace allocation for %zu tokens failed", rows);
     }
-    w.cap_n = need;
+    w.cap_n = rows;
   }
   if (grow(&w.tokb, &w.cap_tok, (ni + nr) * c.in_ch) != cudaSuccess ||
-      grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt, 1) * c.txt_dim) != cudaSuccess)
+      grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt * nb, 1) * c.txt_dim) != cudaSuccess)
     return fail(FLUX_ENOMEM, "workspace allocation failed");
-  if (w.nt == nt && w.gh == gh && w.gw == gw && same_refs(w.refs, refs)) return FLUX_OK;
+  if (w.nt == nt && w.gh == gh && w.gw == gw && w.nb == nb && same_refs(w.refs, refs)) return FLUX_OK;
 
   const size_t nimg = ni + nr;
   const uint64_t ldD = D * 2, ldC = (D + F) * 2;
   bool ok = true;
-  auto amap = [&](CUtensorMap* map, const void* base, size_t rows, size_t cols, uint64_t stride, uint32_t box) {
-    if (rows == 0) {
+  auto amap = [&](CUtensorMap* map, const void* base, size_t nrows, size_t cols, uint64_t stride, uint32_t box) {
+    if (nrows == 0) {
       memset(map, 0, sizeof(*map));
       return;
     }
-    ok &= make_tmap_bf16(map, base, rows, cols, stride, box);
+    ok &= make_tmap_bf16(map, base, nrows, cols, stride, box);
   };
-  amap(&w.a_txtb, w.txtb, nt, c.txt_dim, c.txt_dim * 2, 128);
   amap(&w.a_tokb, w.tokb, nimg, c.in_ch, c.in_ch * 2, 128);
-  amap(&w.a_Ytxt, w.Y, nt, D, ldD, 128);
-  amap(&w.a_Yimg, w.Y + nt * D, nimg, D, ldD, 128);
-  amap(&w.a_Yall, w.Y, n, D, ldD, 128);
-  amap(&w.a_Yout, w.Y, ni, D, ldD, 128);
-  amap(&w.a_Otxt, w.CC, nt, D, ldC, 128);
-  amap(&w.a_Oimg, w.CC + nt * (D + F), nimg, D, ldC, 128);
-  amap(&w.a_Htxt, w.CC + D, nt, F, ldC, 128);
-  amap(&w.a_Himg, w.CC + nt * (D + F) + D, nimg, F, ldC, 128);
-  amap(&w.a_CC, w.CC, n, D + F, ldC, 128);
-  amap(&w.qkv, w.QKV, n, 3 * D, 3 * D * 2, 128);
+  amap(&w.a_Yall, w.Y, rows, D, ldD, 128);
+  amap(&w.a_CC, w.CC, rows, D + F, ldC, 128);
+  amap(&w.qkv, w.QKV, rows, 3 * D, 3 * D * 2, 128);
+  for (int b = 0; b < nb; ++b) {
+    const size_t r0 = b * n;                           // first row of sequence b
+    amap(&w.a_txtb[b], w.txtb + b * nt * c.txt_dim, nt, c.txt_dim, c.txt_dim * 2, 128);
+    amap(&w.a_Ytxt[b], w.Y + r0 * D, nt, D, ldD, 128);
+    amap(&w.a_Yimg[b], w.Y + (r0 + nt) * D, nimg, D, ldD, 128);
+    amap(&w.a_Yout[b], w.Y + b * ni * D, ni, D, ldD, 128);   // output layer input: image rows only
+    amap(&w.a_Otxt[b], w.CC + r0 * (D + F), nt, D, ldC, 128);
+    amap(&w.a_Oimg[b], w.CC + (r0 + nt) * (D + F), nimg, D, ldC, 128);
+    amap(&w.a_Htxt[b], w.CC + r0 * (D + F) + D, nt, F, ldC, 128);
+    amap(&w.a_Himg[b], w.CC + (r0 + nt) * (D + F) + D, nimg, F, ldC, 128);
+  }
   if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an activation buffer");
   if (rope_table_launch(w.rope, nt, gh, gw, refs, c.rope_theta, s) != cudaSuccess)
     return fail(FLUX_EIO, "rope table launch failed");
-  w.nt = nt; w.gh = gh; w.gw = gw; w.refs = refs;
+  for (int b = 1; b < nb; ++b)                         // every sequence has the same positions
+    if (cudaMemcpyAsync(w.rope + b * n * 64, w.rope, n * 64 * sizeof(float2), cudaMemcpyDeviceToDevice, s) !=
+        cudaSuccess)
+      return fail(FLUX_EIO, "rope table copy failed");
+  w.nt = nt; w.gh = gh; w.gw = gw; w.nb = nb; w.refs = refs;
   return FLUX_OK;
 }
 
@@ -550,13 +563,22 @@ static int run_modulation(flux_dit* m, float t, cudaStream_t s) {
   return FLUX_OK;
 }
 
-static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const float* txt, int nt,
-                        const float* ref_tok, const RefGrids& refs, float t, float* v_out, cudaStream_t s) {
+// One forward of nb sequences that share the image tokens, the references and t and differ in
+// their text (nb = 2: the prompt and the unconditional text of classifier-free guidance).
+// txt[b] and v_out[b] are the text rows and the velocity output of sequence b.
+static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const float* const* txt, int nt,
+                        const float* ref_tok, const RefGrids& refs, float t, float* const* v_out, int nb,
+                        cudaStream_t s) {
   const flux_dit_config& c = m->cfg;
   const int D = c.hidden, F = c.mlp_hidden, H = c.heads;
-  if (!img_tok || !v_out) return fail(FLUX_EINVAL, "img_tok and v_out must be device pointers");
+  if (nb < 1 || nb > kMaxBatch) return fail(FLUX_EINVAL, "batch of %d sequences (1..%d)", nb, kMaxBatch);
+  if (!img_tok) return fail(FLUX_EINVAL, "img_tok must be a device pointer");
+  for (int b = 0; b < nb; ++b) {
+    if (!v_out[b]) return fail(FLUX_EINVAL, "velocity output %d is NULL", b);
+    if (nt > 0 && !txt[b]) return fail(FLUX_EINVAL, "text %d is NULL", b);
+  }
   if (gh < 4 || gh > 64 || gw < 4 || gw > 64) return fail(FLUX_EINVAL, "image grid %dx%d outside 4..64", gh, gw);
-  if (nt < 0 || nt > 4096 || (nt > 0 && !txt)) return fail(FLUX_EINVAL, "bad text (n_txt=%d)", nt);
+  if (nt < 0 || nt > 4096) return fail(FLUX_EINVAL, "bad text (n_txt=%d)", nt);
   if (refs.count < 0 || refs.count > kMaxRefs)
     return fail(FLUX_EINVAL, "%d reference images (at most %d)", refs.count, kMaxRefs);
   for (int k = 0; k < refs.count; ++k)
@@ -568,14 +590,16 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
   cudaGetDevice(&dev);
   if (dev != m->device) return fail(FLUX_EINVAL, "model lives on device %d, current device is %d", m->device, dev);
 
-  int rc = prepare_shape(m, nt, gh, gw, refs, s);
+  int rc = prepare_shape(m, nt, gh, gw, refs, nb, s);
   if (rc) return rc;
   Workspace& w = m->ws;
   const int ni = gh * gw, nr = static_cast<int>(ref_tokens(refs)), nimg = ni + nr, n = nt + nimg;
+  const int rows = n * nb;
   const float eps_ln = c.eps_ln, eps_rms = c.eps_rms;
   const float* mods = m->mods;
+  auto seq_row = [&](int b, int r) { return static_cast<size_t>(b) * n + r; };   // row r of sequence b
 
-  rc = run_modulation(m, t, s);
+  rc = run_modulation(m, t, s);                   // one t, so one modulation vector for every sequence
   if (rc) return rc;
   FD_LAUNCH(m, kProfOther, 0, 6.0 * ni * c.in_ch,
             cast_bf16_launch(img_tok, w.tokb, static_cast<size_t>(ni) * c.in_ch, s));
@@ -583,25 +607,27 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
     FD_LAUNCH(m, kProfOther, 0, 6.0 * nr * c.in_ch,
               cast_bf16_launch(ref_tok, w.tokb + static_cast<size_t>(ni) * c.in_ch,
                                static_cast<size_t>(nr) * c.in_ch, s));
-  if (nt)
+  for (int b = 0; b < nb && nt; ++b)
     FD_LAUNCH(m, kProfOther, 0, 6.0 * nt * c.txt_dim,
-              cast_bf16_launch(txt, w.txtb, static_cast<size_t>(nt) * c.txt_dim, s));
-  const double ln_bytes = 6.0 * n * D + 16.0 * D, ln_bytes_img = 6.0 * ni * D + 8.0 * D;
-  const double at_flops = 4.0 * n * static_cast<double>(n) * D, at_bytes = 8.0 * n * D;
+              cast_bf16_launch(txt[b], w.txtb + static_cast<size_t>(b) * nt * c.txt_dim,
+                               static_cast<size_t>(nt) * c.txt_dim, s));
+  const double ln_bytes = 6.0 * rows * D + 16.0 * D, ln_bytes_img = 6.0 * ni * D + 8.0 * D;
+  const double at_flops = 4.0 * nb * n * static_cast<double>(n) * D, at_bytes = 8.0 * rows * D;
 
+  // input projections: text rows with txt_in, image + reference rows with img_in, per sequence
   GemmParams P;
-  P.num_problems = 2;
-  problem(P, 0, w.a_txtb, m->m_txt_in, nt, D, c.txt_dim, kEpiF32Bias, w.X, D, m->txt_b, nullptr);
-  problem(P, 1, w.a_tokb, m->m_img_in, nimg, D, c.in_ch, kEpiF32Bias, w.X + static_cast<size_t>(nt) * D, D, m->img_b,
-          nullptr);
+  P.num_problems = 2 * nb;
+  for (int b = 0; b < nb; ++b) {
+    problem(P, 2 * b, w.a_txtb[b], m->m_txt_in, nt, D, c.txt_dim, kEpiF32Bias, w.X + seq_row(b, 0) * D, D,
+            m->txt_b, nullptr);
+    problem(P, 2 * b + 1, w.a_tokb, m->m_img_in, nimg, D, c.in_ch, kEpiF32Bias, w.X + seq_row(b, nt) * D, D,
+            m->img_b, nullptr);
+  }
   FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
 
-  float* Ximg = w.X + static_cast<size_t>(nt) * D;
-  bf16* Otxt = w.CC;
-  bf16* Oimg = w.CC + static_cast<size_t>(nt) * (D + F);
   AttnParams A;
   A.mapQ = w.qkv; A.mapK = w.qkv; A.mapV = w.qkv;
-  A.out = w.CC; A.ldo = D + F; A.n = n; A.heads = H;
+  A.out = w.CC; A.ldo = D + F; A.n = n; A.heads = H; A.batch = nb;
   A.q_col0 = 0; A.k_col0 = D; A.v_col0 = 2 * D;
   A.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
 
@@ -610,47 +636,72 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
     const StreamW& st = m->dbl[2 * i + 1];
     const float* mi = mods + si.mod_off;          // shift1, scale1, gate1, shift2, scale2, gate2
     const float* mt = mods + st.mod_off;
-    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes, ln_modulate_launch(w.X, w.Y, n, D, nt, mt, mt + D, mi, mi + D, eps_ln, s));
-    P.num_problems = 2;
-    problem(P, 0, w.a_Ytxt, st.m_qkv, nt, 3 * D, D, kEpiBf16Bias, w.QKV, 3 * D, st.qkv_b, nullptr);
-    problem(P, 1, w.a_Yimg, si.m_qkv, nimg, 3 * D, D, kEpiBf16Bias, w.QKV + static_cast<size_t>(nt) * 3 * D, 3 * D,
-            si.qkv_b, nullptr);
-    qk_fuse(P, 0, st.q_gain, st.k_gain, w.rope, 0, eps_rms);
-    qk_fuse(P, 1, si.q_gain, si.k_gain, w.rope, nt, eps_rms);
+    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes,
+              ln_modulate_launch(w.X, w.Y, rows, D, nt, n, mt, mt + D, mi, mi + D, eps_ln, s));
+    P.num_problems = 2 * nb;
+    for (int b = 0; b < nb; ++b) {
+      problem(P, 2 * b, w.a_Ytxt[b], st.m_qkv, nt, 3 * D, D, kEpiBf16Bias, w.QKV + seq_row(b, 0) * 3 * D, 3 * D,
+              st.qkv_b, nullptr);
+      problem(P, 2 * b + 1, w.a_Yimg[b], si.m_qkv, nimg, 3 * D, D, kEpiBf16Bias, w.QKV + seq_row(b, nt) * 3 * D,
+              3 * D, si.qkv_b, nullptr);
+      qk_fuse(P, 2 * b, st.q_gain, st.k_gain, w.rope, static_cast<int>(seq_row(b, 0)), eps_rms);
+      qk_fuse(P, 2 * b + 1, si.q_gain, si.k_gain, w.rope, static_cast<int>(seq_row(b, nt)), eps_rms);
+    }
     FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
     FD_LAUNCH(m, kProfAttention, at_flops, at_bytes, attention_launch(A, s));
-    P.num_problems = 2;
-    problem(P, 0, w.a_Otxt, st.m_proj, nt, D, D, kEpiResidGate, w.X, D, st.proj_b, mt + 2 * D);
-    problem(P, 1, w.a_Oimg, si.m_proj, nimg, D, D, kEpiResidGate, Ximg, D, si.proj_b, mi + 2 * D);
+    P.num_problems = 2 * nb;
+    for (int b = 0; b < nb; ++b) {
+      problem(P, 2 * b, w.a_Otxt[b], st.m_proj, nt, D, D, kEpiResidGate, w.X + seq_row(b, 0) * D, D, st.proj_b,
+              mt + 2 * D);
+      problem(P, 2 * b + 1, w.a_Oimg[b], si.m_proj, nimg, D, D, kEpiResidGate, w.X + seq_row(b, nt) * D, D,
+              si.proj_b, mi + 2 * D);
+    }
     FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
-    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes, ln_modulate_launch(w.X, w.Y, n, D, nt, mt + 3 * D, mt + 4 * D, mi + 3 * D, mi + 4 * D, eps_ln, s));
-    P.num_problems = 2;
-    problem(P, 0, w.a_Ytxt, st.m_mlp_in, nt, 2 * F, D, kEpiSwiGLU, Otxt + D, D + F, st.mlp_in_b, nullptr);
-    problem(P, 1, w.a_Yimg, si.m_mlp_in, nimg, 2 * F, D, kEpiSwiGLU, Oimg + D, D + F, si.mlp_in_b, nullptr);
+    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes,
+              ln_modulate_launch(w.X, w.Y, rows, D, nt, n, mt + 3 * D, mt + 4 * D, mi + 3 * D, mi + 4 * D, eps_ln,
+                                 s));
+    P.num_problems = 2 * nb;
+    for (int b = 0; b < nb; ++b) {
+      problem(P, 2 * b, w.a_Ytxt[b], st.m_mlp_in, nt, 2 * F, D, kEpiSwiGLU, w.CC + seq_row(b, 0) * (D + F) + D,
+              D + F, st.mlp_in_b, nullptr);
+      problem(P, 2 * b + 1, w.a_Yimg[b], si.m_mlp_in, nimg, 2 * F, D, kEpiSwiGLU,
+              w.CC + seq_row(b, nt) * (D + F) + D, D + F, si.mlp_in_b, nullptr);
+    }
     FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
-    P.num_problems = 2;
-    problem(P, 0, w.a_Htxt, st.m_mlp_out, nt, D, F, kEpiResidGate, w.X, D, st.mlp_out_b, mt + 5 * D);
-    problem(P, 1, w.a_Himg, si.m_mlp_out, nimg, D, F, kEpiResidGate, Ximg, D, si.mlp_out_b, mi + 5 * D);
+    P.num_problems = 2 * nb;
+    for (int b = 0; b < nb; ++b) {
+      problem(P, 2 * b, w.a_Htxt[b], st.m_mlp_out, nt, D, F, kEpiResidGate, w.X + seq_row(b, 0) * D, D,
+              st.mlp_out_b, mt + 5 * D);
+      problem(P, 2 * b + 1, w.a_Himg[b], si.m_mlp_out, nimg, D, F, kEpiResidGate, w.X + seq_row(b, nt) * D, D,
+              si.mlp_out_b, mi + 5 * D);
+    }
     FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
   }
+  // single blocks: one set of weights for every row, so the whole batch is one problem
   for (int i = 0; i < m->act_single; ++i) {
     const SingleW& sw = m->sgl[i];
     const float* ms = mods + sw.mod_off;          // shift, scale, gate
-    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes, ln_modulate_launch(w.X, w.Y, n, D, n, ms, ms + D, ms, ms + D, eps_ln, s));
+    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes,
+              ln_modulate_launch(w.X, w.Y, rows, D, n, n, ms, ms + D, ms, ms + D, eps_ln, s));
     P.num_problems = 2;
-    problem(P, 0, w.a_Yall, sw.m_qkv, n, 3 * D, D, kEpiBf16Bias, w.QKV, 3 * D, sw.qkv_b, nullptr);
-    problem(P, 1, w.a_Yall, sw.m_mlp, n, 2 * F, D, kEpiSwiGLU, w.CC + D, D + F, sw.mlp_b, nullptr);
+    problem(P, 0, w.a_Yall, sw.m_qkv, rows, 3 * D, D, kEpiBf16Bias, w.QKV, 3 * D, sw.qkv_b, nullptr);
+    problem(P, 1, w.a_Yall, sw.m_mlp, rows, 2 * F, D, kEpiSwiGLU, w.CC + D, D + F, sw.mlp_b, nullptr);
     qk_fuse(P, 0, sw.q_gain, sw.k_gain, w.rope, 0, eps_rms);
     FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
     FD_LAUNCH(m, kProfAttention, at_flops, at_bytes, attention_launch(A, s));
     P.num_problems = 1;
-    problem(P, 0, w.a_CC, sw.m_lin2, n, D, D + F, kEpiResidGate, w.X, D, sw.lin2_b, ms + 2 * D);
+    problem(P, 0, w.a_CC, sw.m_lin2, rows, D, D + F, kEpiResidGate, w.X, D, sw.lin2_b, ms + 2 * D);
     FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
   }
+  // output layer on the image rows of each sequence
   const float* mf = mods + m->fin_mod_off;         // shift, scale
-  FD_LAUNCH(m, kProfLnMod, 0, ln_bytes_img, ln_modulate_launch(Ximg, w.Y, ni, D, ni, mf, mf + D, mf, mf + D, eps_ln, s));
-  P.num_problems = 1;
-  problem(P, 0, w.a_Yout, m->m_fin, ni, c.in_ch, D, kEpiF32Bias, v_out, c.in_ch, m->fin_b, nullptr);
+  for (int b = 0; b < nb; ++b)
+    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes_img,
+              ln_modulate_launch(w.X + seq_row(b, nt) * D, w.Y + static_cast<size_t>(b) * ni * D, ni, D, ni, ni, mf,
+                                 mf + D, mf, mf + D, eps_ln, s));
+  P.num_problems = nb;
+  for (int b = 0; b < nb; ++b)
+    problem(P, b, w.a_Yout[b], m->m_fin, ni, c.in_ch, D, kEpiF32Bias, v_out[b], c.in_ch, m->fin_b, nullptr);
   FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 128, m->num_sms, s));
   return FLUX_OK;
 }
@@ -687,7 +738,7 @@ int flux_dit_forward(flux_dit* m, const float* img_tok, int grid_h, int grid_w, 
   if (!((ref_h == 0 && ref_w == 0) || (ref_h > 0 && ref_w > 0)))
     return fail(FLUX_EINVAL, "reference grid %dx%d", ref_h, ref_w);
   RefGrids refs = {ref_h > 0 ? 1 : 0, {ref_h}, {ref_w}};
-  return forward_impl(m, img_tok, grid_h, grid_w, txt, n_txt, ref_tok, refs, t, v_out,
+  return forward_impl(m, img_tok, grid_h, grid_w, &txt, n_txt, ref_tok, refs, t, &v_out, 1,
                       static_cast<cudaStream_t>(stream));
 }
 
@@ -702,8 +753,36 @@ int flux_dit_forward_refs(flux_dit* m, const float* img_tok, int grid_h, int gri
     refs.h[k] = ref_grids[2 * k];
     refs.w[k] = ref_grids[2 * k + 1];
   }
-  return forward_impl(m, img_tok, grid_h, grid_w, txt, n_txt, ref_tok, refs, t, v_out,
+  return forward_impl(m, img_tok, grid_h, grid_w, &txt, n_txt, ref_tok, refs, t, &v_out, 1,
                       static_cast<cudaStream_t>(stream));
+}
+
+int flux_dit_forward_cfg(flux_dit* m, const float* img_tok, int grid_h, int grid_w, const float* txt_cond,
+                         const float* txt_uncond, int n_txt, const float* ref_tok, int n_refs, const int* ref_grids,
+                         float t, float* v_cond, float* v_uncond, void* stream) {
+  if (!m) return fail(FLUX_EINVAL, "model is NULL");
+  if (n_refs < 0 || n_refs > kMaxRefs) return fail(FLUX_EINVAL, "%d reference images (at most %d)", n_refs, kMaxRefs);
+  if (n_refs > 0 && !ref_grids) return fail(FLUX_EINVAL, "ref_grids is NULL");
+  if (v_cond && v_cond == v_uncond) return fail(FLUX_EINVAL, "v_cond and v_uncond must be different buffers");
+  RefGrids refs = {n_refs, {}, {}};
+  for (int k = 0; k < n_refs; ++k) {
+    refs.h[k] = ref_grids[2 * k];
+    refs.w[k] = ref_grids[2 * k + 1];
+  }
+  const float* txt[2] = {txt_cond, txt_uncond};
+  float* v[2] = {v_cond, v_uncond};
+  return forward_impl(m, img_tok, grid_h, grid_w, txt, n_txt, ref_tok, refs, t, v, 2,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int flux_cfg_euler_step(float* x, const float* v_cond, const float* v_uncond, size_t n, float guidance, float dt,
+                        void* stream) {
+  if (n && (!x || !v_cond || !v_uncond)) return fail(FLUX_EINVAL, "NULL argument");
+  if (!aligned16(x) || !aligned16(v_cond) || !aligned16(v_uncond))
+    return fail(FLUX_EINVAL, "x, v_cond and v_uncond must be 16-byte aligned");
+  if (!std::isfinite(guidance) || !std::isfinite(dt)) return fail(FLUX_EINVAL, "guidance and dt must be finite");
+  FD_CUDA(cfg_euler_launch(x, v_cond, v_uncond, n, guidance, dt, static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
 }
 
 int flux_blend_latents(const float* x, const float* noise, float t, float* out, size_t n, void* stream) {
@@ -756,21 +835,30 @@ int flux_unpack_latents(const float* tok, float* lat, int h8, int w8, void* stre
 
 int flux_joint_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o, int n, int heads,
                          int head_dim, float scale, void* stream) {
+  return flux_joint_attention_batch(q, k, v, o, 1, n, heads, head_dim, scale, stream);
+}
+
+int flux_joint_attention_batch(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o, int batch,
+                               int n, int heads, int head_dim, float scale, void* stream) {
   if (!q || !k || !v || !o) return fail(FLUX_EINVAL, "NULL argument");
   if (head_dim != 128) return fail(FLUX_EINVAL, "head_dim must be 128 (got %d)", head_dim);
+  if (batch < 1 || batch > 65535) return fail(FLUX_EINVAL, "bad batch=%d", batch);
   if (n < 1 || heads < 1 || heads > 1024) return fail(FLUX_EINVAL, "bad n=%d heads=%d", n, heads);
+  if (static_cast<long long>(batch) * n > (1ll << 31) - 1) return fail(FLUX_EINVAL, "batch * n too large");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return fail(FLUX_EINVAL, "q, k, v, o must be 16-byte aligned");
   if (!(scale > 0) || !std::isfinite(scale)) return fail(FLUX_EINVAL, "scale must be positive");
   AttnParams A;
   const uint64_t ld = static_cast<uint64_t>(heads) * 128;
-  if (!make_tmap_bf16(&A.mapQ, q, n, ld, ld * 2, 128) || !make_tmap_bf16(&A.mapK, k, n, ld, ld * 2, 128) ||
-      !make_tmap_bf16(&A.mapV, v, n, ld, ld * 2, 128))
+  const size_t rows = static_cast<size_t>(batch) * n;
+  if (!make_tmap_bf16(&A.mapQ, q, rows, ld, ld * 2, 128) || !make_tmap_bf16(&A.mapK, k, rows, ld, ld * 2, 128) ||
+      !make_tmap_bf16(&A.mapV, v, rows, ld, ld * 2, 128))
     return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed");
   A.out = reinterpret_cast<bf16*>(o);
   A.ldo = static_cast<int>(ld);
   A.n = n;
   A.heads = heads;
+  A.batch = batch;
   A.q_col0 = A.k_col0 = A.v_col0 = 0;
   A.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
   FD_CUDA(attention_launch(A, static_cast<cudaStream_t>(stream)));
@@ -835,7 +923,7 @@ int flux_layernorm_modulate(const float* x, uint16_t* y, int rows, int dim, cons
   if (rows < 0 || dim < 4 || dim % 4) return fail(FLUX_EINVAL, "bad shape rows=%d dim=%d", rows, dim);
   if (!aligned16(x) || !aligned16(y) || !aligned16(shift) || !aligned16(scale))
     return fail(FLUX_EINVAL, "pointers must be 16-byte aligned");
-  FD_CUDA(ln_modulate_launch(x, reinterpret_cast<bf16*>(y), rows, dim, rows, shift, scale, shift, scale, eps,
+  FD_CUDA(ln_modulate_launch(x, reinterpret_cast<bf16*>(y), rows, dim, rows, rows, shift, scale, shift, scale, eps,
                              static_cast<cudaStream_t>(stream)));
   return FLUX_OK;
 }

@@ -51,7 +51,8 @@ struct AttnParams {
   CUtensorMap mapQ, mapK, mapV;   // 2D bf16 [rows = n, cols], box {64, 128}, 128B swizzle
   __nv_bfloat16* out;             // O row i, head h at out + i*ldo + h*128
   int ldo;
-  int n, heads;
+  int n, heads;                   // tokens per sequence, heads
+  int batch;                      // sequences of n rows each, one after another (grid.z)
   int q_col0, k_col0, v_col0;     // column of head 0's first element in each map
   float scale_log2;               // softmax scale * log2(e)
 };
@@ -62,10 +63,14 @@ int attention_read_device_error(cudaStream_t stream);
 cudaError_t pack_latents_launch(const float* lat, float* tok, int c, int h8, int w8, cudaStream_t s);
 cudaError_t unpack_latents_launch(const float* tok, float* lat, int c, int h8, int w8, cudaStream_t s);
 cudaError_t euler_launch(float* x, const float* v, size_t n, float dt, cudaStream_t s);
+// x += dt * (vu + g * (vc - vu)), element-wise
+cudaError_t cfg_euler_launch(float* x, const float* vc, const float* vu, size_t n, float g, float dt,
+                             cudaStream_t s);
 cudaError_t cast_bf16_launch(const float* x, __nv_bfloat16* y, size_t n, cudaStream_t s);
 
-// y[r, :] = LN(x[r, :]) * (1 + scale) + shift; rows r < split use (shift0, scale0), others (shift1, scale1)
-cudaError_t ln_modulate_launch(const float* x, __nv_bfloat16* y, int rows, int dim, int split,
+// y[r, :] = LN(x[r, :]) * (1 + scale) + shift; rows with r % period < split use (shift0, scale0), the
+// others (shift1, scale1) (period: rows per sequence of a batch, the row count for one sequence)
+cudaError_t ln_modulate_launch(const float* x, __nv_bfloat16* y, int rows, int dim, int split, int period,
                                const float* shift0, const float* scale0, const float* shift1,
                                const float* scale1, float eps, cudaStream_t s);
 

@@ -15,7 +15,7 @@ import torch
 
 import latent_flow_matching_b200 as F
 from oracle import flux_oracle as O
-from synthetic import WORKLOADS, FluxDims, Workload, make_weights, make_inputs
+from synthetic import WORKLOADS, FluxDims, Workload, make_weights, make_inputs, make_uncond_text
 
 pytestmark = pytest.mark.gpu
 torch.set_grad_enabled(False)
@@ -36,8 +36,11 @@ def gpu_sample(model, w, lat, txt, ref):
         ref = [torch.from_numpy(r).to(DEV) for r in ref]
     elif ref is not None:
         ref = torch.from_numpy(ref).to(DEV)
+    guided = {}
+    if w.guidance is not None:
+        guided = {"txt_uncond": torch.from_numpy(make_uncond_text(w)).to(DEV), "guidance": w.guidance}
     final = F.flux_sample(model, torch.from_numpy(lat).to(DEV), torch.from_numpy(txt).to(DEV), w.n_steps, ref,
-                          on_step=lambda i, v: vs.append(v.cpu().clone()))
+                          on_step=lambda i, v: vs.append(v.cpu().clone()), **guided)
     return final.cpu(), vs
 
 
@@ -142,7 +145,7 @@ def _golden(name):
     return np.load(path)
 
 
-@pytest.mark.parametrize("name", ["t2i256", "t2i512", "t2i1024", "i2i1024", "mref1024"])
+@pytest.mark.parametrize("name", ["t2i256", "t2i512", "t2i1024", "i2i1024", "mref1024", "cfg256"])
 def test_full_workload_against_oracle_goldens(name):
     gd = _golden(name)
     w = WORKLOADS[name]
@@ -212,3 +215,90 @@ def test_forward_rejects_too_many_references(tiny):
     refs = torch.zeros(11 * 16, 128, device=DEV)
     with pytest.raises(F.FluxError):
         model.forward(tok, (4, 4), None, 1.0, v, refs, [(4, 4)] * 11)
+
+
+# ---------------------------------------------------------------------------- classifier-free guidance
+@pytest.mark.parametrize("n_txt,grid,refs", [(7, (4, 4), []), (5, (6, 4), [(4, 4), (4, 6)]), (0, (4, 5), []),
+                                             (131, (8, 8), [(4, 8)])])
+def test_tiny_cfg_batch_equals_two_single_forwards(tiny, n_txt, grid, refs):
+    """The batch-2 forward returns, bit for bit, the two single-text forwards (no row depends on
+    another sequence); sequence lengths off the 128-row tiles put the batch boundary inside a tile."""
+    w, p, model = tiny
+    g = torch.Generator().manual_seed(40 + n_txt)
+    tok = torch.randn(grid[0] * grid[1], 128, generator=g).to(torch.bfloat16).float().to(DEV)
+    tc = torch.randn(n_txt, 3072, generator=g).to(torch.bfloat16).float().to(DEV)
+    tu = torch.randn(n_txt, 3072, generator=g).to(torch.bfloat16).float().to(DEV)
+    ref = None
+    if refs:
+        ref = torch.randn(sum(h * w_ for h, w_ in refs), 128, generator=g).to(torch.bfloat16).float().to(DEV)
+    ni = grid[0] * grid[1]
+    vc, vu, a, b = (torch.empty(ni, 128, device=DEV) for _ in range(4))
+    model.forward_cfg(tok, grid, tc if n_txt else None, tu if n_txt else None, 0.6, vc, vu, ref, refs)
+    hw = refs if refs else (0, 0)
+    model.forward(tok, grid, tc if n_txt else None, 0.6, a, ref, hw)
+    model.forward(tok, grid, tu if n_txt else None, 0.6, b, ref, hw)
+    assert torch.equal(vc, a) and torch.equal(vu, b)
+    if n_txt:
+        assert not torch.equal(vc, vu)
+    assert F.flux_device_error() == 0
+
+
+def test_tiny_cfg_sampler_matches_oracle(tiny):
+    """Guidance 3.5 with an unconditional text: every guided velocity and the final latent
+    against the live float64 oracle."""
+    w, p, model = tiny
+    lat, txt, _ = make_inputs(w)
+    txt_u = np.random.default_rng(77).standard_normal(txt.shape).astype(np.float32)
+    txt_u = torch.from_numpy(txt_u).to(torch.bfloat16).float()
+    ref_final, ref_vs = O.sample(p, O.hyper(w.dims), torch.from_numpy(lat), torch.from_numpy(txt), 3,
+                                 txt_uncond=txt_u, guidance=3.5)
+    vs = []
+    final = F.flux_sample(model, torch.from_numpy(lat).to(DEV), torch.from_numpy(txt).to(DEV), 3,
+                          txt_uncond=txt_u.to(DEV), guidance=3.5, on_step=lambda i, v: vs.append(v.cpu().clone()))
+    assert len(vs) == len(ref_vs) == 3
+    for a, b in zip(vs, ref_vs):
+        assert rel_l2(a, b) <= V_TOL
+    assert rel_l2(final.cpu(), ref_final) <= X_TOL
+    # guidance 1 is the prompt-only sampler, bit for bit
+    one = F.flux_sample(model, torch.from_numpy(lat).to(DEV), torch.from_numpy(txt).to(DEV), 3,
+                        txt_uncond=txt_u.to(DEV), guidance=1.0)
+    plain = F.flux_sample(model, torch.from_numpy(lat).to(DEV), torch.from_numpy(txt).to(DEV), 3)
+    assert rel_l2(one.cpu(), plain.cpu()) <= 1e-6
+    assert F.flux_device_error() == 0
+
+
+def test_cfg_rejects_bad_arguments(tiny):
+    w, p, model = tiny
+    tok = torch.zeros(16, 128, device=DEV)
+    v = torch.empty(16, 128, device=DEV)
+    tc, tu = torch.zeros(4, 3072, device=DEV), torch.zeros(5, 3072, device=DEV)
+    with pytest.raises(ValueError):
+        model.forward_cfg(tok, (4, 4), tc, tu, 1.0, v, torch.empty_like(v))
+    with pytest.raises(F.FluxError):                         # one buffer for both velocities
+        model.forward_cfg(tok, (4, 4), tc, tc, 1.0, v, v)
+    with pytest.raises(F.FluxError):
+        F.flux_cfg_euler_step(v, v, v, float("nan"), 0.1)
+
+
+def test_cfg_batch_bit_exact_at_full_size():
+    """1024^2 workload (4608 tokens per sequence, full model): the batch-2 forward equals the two
+    single-text forwards bit for bit, so the single-text goldens pin both velocities."""
+    w = WORKLOADS["t2i1024"]
+    blob, _ = make_weights(w.dims, w.seed)
+    lat, txt, _ = make_inputs(w)
+    model = F.FluxDiT(blob, w.dims)
+    del blob
+    try:
+        tok = O.pack_latents(torch.from_numpy(lat)).float().to(DEV)
+        tc = torch.from_numpy(txt).to(DEV)
+        tu = torch.from_numpy(make_uncond_text(WORKLOADS["cfg1024"])).to(DEV)
+        vc, vu, a, b = (torch.empty(w.n_img, 128, device=DEV) for _ in range(4))
+        model.forward_cfg(tok, (w.grid, w.grid), tc, tu, 0.75, vc, vu)
+        model.forward(tok, (w.grid, w.grid), tc, 0.75, a)
+        model.forward(tok, (w.grid, w.grid), tu, 0.75, b)
+        torch.cuda.synchronize()
+        assert torch.equal(vc, a) and torch.equal(vu, b)
+        assert rel_l2(vc, vu) > 1e-3
+    finally:
+        model.close()
+    assert F.flux_device_error() == 0

@@ -244,3 +244,35 @@ def test_blend_latents(t):
     assert (out.cpu().double() - ref).abs().max() <= 1e-6
     if t in (0.0, 1.0):
         assert torch.equal(out.cpu(), x if t == 0.0 else noise)
+
+
+# ---------------------------------------------------------------------------- guidance, batched attention
+@pytest.mark.parametrize("n", [1, 7, 4096 * 128 + 3])
+def test_cfg_euler_step(n):
+    g = torch.Generator().manual_seed(n % 1000)
+    x = torch.randn(n, generator=g)
+    vc = torch.randn(n, generator=g)
+    vu = torch.randn(n, generator=g)
+    xd = x.to(DEV)
+    F.flux_cfg_euler_step(xd, vc.to(DEV), vu.to(DEV), 3.5, -0.25)
+    ref = O.euler_update(x.double(), O.guided_velocity(vc.double(), vu.double(), 3.5), -0.25)
+    assert (xd.cpu().double() - ref).abs().max().item() <= 1e-5
+
+
+@pytest.mark.parametrize("batch,n", [(2, 77), (2, 300), (3, 129), (2, 4608)])
+def test_attention_batch_sequences_are_independent(batch, n):
+    """Each sequence of the batch attends only to itself; rows equal the one-sequence call bit for bit."""
+    heads = 2
+    q = bf(rand((batch * n, heads, 128), 60))
+    k = bf(rand((batch * n, heads, 128), 61))
+    v = bf(rand((batch * n, heads, 128), 62))
+    o = torch.empty(batch * n, heads, 128, device=DEV, dtype=torch.bfloat16)
+    F.flux_joint_attention_batch(q.to(DEV), k.to(DEV), v.to(DEV), o, batch)
+    for b in range(batch):
+        sl = slice(b * n, (b + 1) * n)
+        one = torch.empty(n, heads, 128, device=DEV, dtype=torch.bfloat16)
+        F.flux_joint_attention(q[sl].to(DEV), k[sl].to(DEV), v[sl].to(DEV), one)
+        assert torch.equal(o[sl], one)
+        rows = torch.arange(0, n, max(1, n // 40))
+        ref = O.attention(q[sl][rows].double(), k[sl].double(), v[sl].double())
+        assert nmax(o[sl].cpu()[rows].reshape(len(rows), -1), ref) <= TOL
