@@ -34,6 +34,7 @@ import numpy as np
 CHUNK = 1 << 22           # elements per independently seeded chunk
 INPUT_KEY = 1_000_000     # seed-key offset of the latent / text / reference draws
 BLOB_MAGIC = b"FLUXDIT\0"
+BLOB3_MAGIC = b"FLUX3DT\0"
 BLOB_VERSION = 1
 HEADER_BYTES = 256
 ALIGN = 256
@@ -53,6 +54,31 @@ class FluxDims:
     rope_theta: float = 10000.0
     eps_ln: float = 1e-6
     eps_rms: float = 1e-6
+
+
+@dataclasses.dataclass(frozen=True)
+class Flux3Dims:
+    """FLUX.3 Image Klein ("FLUX.3 Image Klein in Diffusers: ..." (mindverse), sections
+    "Zweistufiger Transformer und Tokenisierung" and "Entkoppelte Vorverarbeitung und
+    gemeinsame Attention-Blöcke"): 5 per-mode blocks (own weights for the text, image and
+    reference streams, attention within a stream) then 28 joint blocks (one weight set,
+    attention over text | image | reference), every block in the parallel attention + SwiGLU
+    form; text features are 8 stacked encoder layers of 2560 (20480) projected to 3072.
+    ``flow_map``: the time-distilled checkpoint's extra embedding of the target time
+    (section "Modulation pro Token-Typ, Flow-Map-Destillation und 4D-RoPE")."""
+    n_mode: int = 5
+    n_joint: int = 28
+    hidden: int = 3072
+    heads: int = 24
+    head_dim: int = 128
+    mlp_hidden: int = 9216
+    in_ch: int = 128
+    txt_dim: int = 20480
+    t_freq_dim: int = 256
+    rope_theta: float = 10000.0
+    eps_ln: float = 1e-6
+    eps_rms: float = 1e-6
+    flow_map: bool = True
 
 
 @dataclasses.dataclass(frozen=True)
@@ -99,6 +125,8 @@ class Workload:
 
 TINY_DIMS = FluxDims(n_double=1, n_single=1)
 FULL_DIMS = FluxDims()
+F3_TINY_DIMS = Flux3Dims(n_mode=1, n_joint=1)
+F3_FULL_DIMS = Flux3Dims()
 
 WORKLOADS = {
     "tiny64": Workload("tiny64", 0, 64, 16, 0, 1, TINY_DIMS),
@@ -111,11 +139,61 @@ WORKLOADS = {
     # 256^2 golden case keeps 4 steps so the oracle finishes in minutes)
     "cfg256": Workload("cfg256", 6, 256, 512, 0, 4, FULL_DIMS, guidance=3.5),
     "cfg1024": Workload("cfg1024", 7, 1024, 512, 0, 50, FULL_DIMS, guidance=3.5),
+    # FLUX.3 Image Klein, time-distilled checkpoint (16 steps, flow-map target time).  Text token
+    # counts from the pages' per-call totals: 4256 = 4096 + 160 at 1024^2, 8272 = 4096 + 4096 + 80
+    # with one 1024^2 reference (mindverse, "Einfluss von Referenzbildern auf die Sequenzlänge").
+    "f3tiny64": Workload("f3tiny64", 20, 64, 16, 64, 1, F3_TINY_DIMS),
+    "f3t2i256": Workload("f3t2i256", 21, 256, 160, 0, 4, F3_FULL_DIMS),
+    "f3i2i256": Workload("f3i2i256", 22, 256, 80, 256, 4, F3_FULL_DIMS),
+    "f3t2i1024": Workload("f3t2i1024", 23, 1024, 160, 0, 16, F3_FULL_DIMS),
+    "f3i2i1024": Workload("f3i2i1024", 24, 1024, 80, 1024, 16, F3_FULL_DIMS),
 }
 
 
-def tensor_specs(d: FluxDims):
+def _parallel_block_specs(p, D, F, hd):
+    return [
+        (p + "lin1.w", (3 * D + 2 * F, D), D), (p + "lin1.b", (3 * D + 2 * F,), D),
+        (p + "q_gain", (hd,), 1), (p + "k_gain", (hd,), 1),
+        (p + "lin2.w", (D, D + F), D + F), (p + "lin2.b", (D,), D + F),
+    ]
+
+
+def tensor_specs3(d: Flux3Dims):
+    """FLUX.3 blob order: list of (name, shape, fan_in).  Modulation linears are shared by the
+    blocks of a phase: one per stream for the per-mode blocks, one for the joint blocks."""
+    D, F, hd = d.hidden, d.mlp_hidden, d.head_dim
+    specs = [
+        ("time_in.w1", (D, d.t_freq_dim), d.t_freq_dim), ("time_in.b1", (D,), d.t_freq_dim),
+        ("time_in.w2", (D, D), D), ("time_in.b2", (D,), D),
+    ]
+    if d.flow_map:
+        specs += [
+            ("target_in.w1", (D, d.t_freq_dim), d.t_freq_dim), ("target_in.b1", (D,), d.t_freq_dim),
+            ("target_in.w2", (D, D), D), ("target_in.b2", (D,), D),
+        ]
+    specs += [
+        ("img_in.w", (D, d.in_ch), d.in_ch), ("img_in.b", (D,), d.in_ch),
+        ("txt_in.w", (D, d.txt_dim), d.txt_dim), ("txt_in.b", (D,), d.txt_dim),
+    ]
+    for s in ("txt", "img", "ref"):
+        specs += [(f"mode_mod.{s}.w", (3 * D, D), D), (f"mode_mod.{s}.b", (3 * D,), D)]
+    for i in range(d.n_mode):
+        for s in ("txt", "img", "ref"):
+            specs += _parallel_block_specs(f"mode.{i}.{s}.", D, F, hd)
+    specs += [("joint_mod.w", (3 * D, D), D), ("joint_mod.b", (3 * D,), D)]
+    for i in range(d.n_joint):
+        specs += _parallel_block_specs(f"joint.{i}.", D, F, hd)
+    specs += [
+        ("final.mod.w", (2 * D, D), D), ("final.mod.b", (2 * D,), D),
+        ("final.out.w", (d.in_ch, D), D), ("final.out.b", (d.in_ch,), D),
+    ]
+    return specs
+
+
+def tensor_specs(d):
     """Blob order: list of (name, shape, fan_in)."""
+    if isinstance(d, Flux3Dims):
+        return tensor_specs3(d)
     D, F, hd = d.hidden, d.mlp_hidden, d.head_dim
     specs = [
         ("time_in.w1", (D, d.t_freq_dim), d.t_freq_dim), ("time_in.b1", (D,), d.t_freq_dim),
@@ -153,7 +231,7 @@ def _align(x: int) -> int:
     return (x + ALIGN - 1) // ALIGN * ALIGN
 
 
-def blob_layout(d: FluxDims):
+def blob_layout(d):
     """Byte offset (from the start of the blob) of every tensor, and total size."""
     off = HEADER_BYTES
     layout = []
@@ -175,7 +253,14 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
-def _header(d: FluxDims, n_tensors: int, total: int) -> bytes:
+def _header(d, n_tensors: int, total: int) -> bytes:
+    if isinstance(d, Flux3Dims):
+        h = BLOB3_MAGIC + struct.pack(
+            "<II10i3fQQ", BLOB_VERSION, n_tensors,
+            d.n_mode, d.n_joint, d.hidden, d.heads, d.head_dim, d.mlp_hidden,
+            d.in_ch, d.txt_dim, d.t_freq_dim, 1 if d.flow_map else 0, d.rope_theta, d.eps_ln, d.eps_rms,
+            HEADER_BYTES, total - HEADER_BYTES)
+        return h + b"\0" * (HEADER_BYTES - len(h))
     h = BLOB_MAGIC + struct.pack(
         "<II9i3fQQ", BLOB_VERSION, n_tensors,
         d.n_double, d.n_single, d.hidden, d.heads, d.head_dim, d.mlp_hidden,
@@ -194,7 +279,7 @@ def _fill(dst_u16: np.ndarray, seed: int, idx: int, chunk: int, scale: np.float3
     dst_u16[lo:hi] = round_to_bf16_bits(x)
 
 
-def make_weights(d: FluxDims, seed: int, threads: int | None = None):
+def make_weights(d, seed: int, threads: int | None = None):
     """Return (blob: uint8 array, params: dict name -> uint16 view of bf16 bits)."""
     layout, total = blob_layout(d)
     blob = np.zeros(total, dtype=np.uint8)
