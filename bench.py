@@ -32,20 +32,44 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synthetic import WORKLOADS, make_weights, make_inputs, make_uncond_text  # noqa: E402
+from synthetic import WORKLOADS, Flux3Dims, make_weights, make_inputs, make_uncond_text  # noqa: E402
 
 METRIC = "ms per DiT forward & TFLOP/s at 1024^2 (4096+512 tok), % of BF16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_BF16_TFLOPS = 2250.0
 
 
+def is_flux3(w):
+    return isinstance(w.dims, Flux3Dims)
+
+
+def n_blocks(w):
+    d = w.dims
+    return d.n_mode + d.n_joint if is_flux3(w) else d.n_double + d.n_single
+
+
+def blocks_text(w):
+    d = w.dims
+    if is_flux3(w):
+        return f"FLUX.3 Image Klein: {d.n_mode} per-mode + {d.n_joint} joint blocks"
+    return f"{d.n_double} double + {d.n_single} single blocks"
+
+
 def forward_flops(w):
-    """Algorithmic FLOPs of one forward: dense linears + non-causal attention (QK^T and PV)."""
+    """Algorithmic FLOPs of one forward: dense linears + non-causal attention (QK^T and PV).
+
+    Every block's linears cost N 2D(4D + 3F) over its rows.  FLUX.2 blocks and FLUX.3 joint blocks
+    attend over the whole sequence (4 N^2 D); FLUX.3 per-mode blocks attend within each stream
+    (4 D (Nt^2 + Ni^2 + Nr^2))."""
     d = w.dims
     D, F_, C = d.hidden, d.mlp_hidden, d.in_ch
     n = w.n_tokens
-    per_block = n * 2.0 * D * (4 * D + 3 * F_) + 4.0 * n * n * D
-    total = (d.n_double + d.n_single) * per_block
+    lin = n * 2.0 * D * (4 * D + 3 * F_)
+    if is_flux3(w):
+        total = (d.n_mode + d.n_joint) * lin + d.n_joint * 4.0 * n * n * D
+        total += d.n_mode * 4.0 * D * (w.n_txt ** 2 + w.n_img ** 2 + w.n_ref ** 2)
+    else:
+        total = (d.n_double + d.n_single) * (lin + 4.0 * n * n * D)
     total += 2.0 * (w.n_img + w.n_ref) * C * D + 2.0 * w.n_txt * d.txt_dim * D + 2.0 * w.n_img * D * C
     return total
 
@@ -62,6 +86,11 @@ def step_unit(w):
 def single_block_flops(w):
     d, n = w.dims, w.n_tokens
     return n * 2.0 * d.hidden * (4 * d.hidden + 3 * d.mlp_hidden) + 4.0 * n * n * d.hidden
+
+
+def weight_gb(w):
+    from synthetic import blob_layout
+    return blob_layout(w.dims)[1] / 1e9
 
 
 def load_peaks():
@@ -173,9 +202,13 @@ def profile_traffic(kernel_files, profile):
 
 
 def cpu_oracle_sample(w, params, lat, txt, ref):
-    """Oracle time of one double and one single block at full size (fp32, host cores), scaled to a forward."""
+    """Oracle time of one double and one single block at full size (fp32, host cores), scaled to a forward
+    (FLUX.3: one joint block, scaled by forward FLOPs / block FLOPs)."""
     from oracle import flux_oracle as O
     torch.set_grad_enabled(False)
+    if is_flux3(w):
+        ms_block, secs = oracle_joint_block_ms(w, params)
+        return ms_block * forward_flops(w) / single_block_flops(w), secs
     hp = O.hyper(w.dims)
     D = w.dims.hidden
     g = torch.Generator().manual_seed(0)
@@ -192,6 +225,24 @@ def cpu_oracle_sample(w, params, lat, txt, ref):
     return ms, t2 - t0
 
 
+def oracle_joint_block_ms(w, params, repeats=1):
+    """fp32 oracle time of one FLUX.3 joint block at the workload's full size (host cores)."""
+    from oracle import flux_oracle as O
+    from oracle import flux3_oracle as O3
+    torch.set_grad_enabled(False)
+    hp = O.hyper(w.dims)
+    D = w.dims.hidden
+    g = torch.Generator().manual_seed(0)
+    x = torch.randn(w.n_tokens, D, generator=g)
+    sh, sc, gt = (torch.randn(D, generator=g) for _ in range(3))
+    ang = O.rope_angles(O.token_positions(w.n_txt, w.grid, w.grid, ref_grids=w.ref_grids), 128, 1e4).float()
+    t0 = time.perf_counter()
+    for _ in range(repeats):
+        O3.parallel_block(params, "joint.0.", x, sh, sc, gt, ang, hp, torch.float32)
+    secs = time.perf_counter() - t0
+    return 1e3 * secs / repeats, secs
+
+
 # ---------------------------------------------------------------------------- reference arm (CPU oracle)
 def run_reference(args, w):
     world, rank, _ = dist_env()
@@ -200,6 +251,8 @@ def run_reference(args, w):
     from oracle import flux_oracle as O
     torch.set_grad_enabled(False)
     _, params = make_weights(w.dims, w.seed)
+    if is_flux3(w):
+        return run_reference3(args, w, params)
     hp = O.hyper(w.dims)
     D = w.dims.hidden
     g = torch.Generator().manual_seed(0)
@@ -224,9 +277,36 @@ def run_reference(args, w):
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded N(0,1) bf16-rounded weights and inputs)",
         "config": {"workload": f"{w.name}: {w.image}x{w.image}, {w.n_img} image + {w.n_txt} text + {w.n_ref} "
-                               f"reference tokens, 5 double + 20 single blocks, width 3072", "seq_len": w.n_tokens,
+                               f"reference tokens, {blocks_text(w)}, width 3072", "seq_len": w.n_tokens,
                    "global_batch": 1, "parallelism": "CPU oracle on rank 0"},
         "tflops": round(n_sequences(w) * forward_flops(w) / (value / 1e3) / 1e12, 4),
+        "cpu_baseline": {"value": round(value, 3), "unit": step_unit(w), "cores": torch.get_num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": step_unit(w), "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_reference3(args, w, params):
+    """Reference arm for a FLUX.3 workload: the fp32 oracle's joint block, scaled to a forward."""
+    for _ in range(args.warmup):
+        oracle_joint_block_ms(w, params)
+    times = [oracle_joint_block_ms(w, params)[0] for _ in range(args.steps)]
+    ms_block = sum(times) / len(times)
+    scale = forward_flops(w) / single_block_flops(w)
+    value = ms_block * scale
+    sample = (f"one joint block at the full {w.name} size ({w.n_tokens} tokens) per step, fp32 oracle; "
+              f"value scaled by forward FLOPs / block FLOPs = {scale:.2f}")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": step_unit(w),
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_block, 3),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded N(0,1) bf16-rounded weights and inputs)",
+        "config": {"workload": f"{w.name}: {w.image}x{w.image}, {w.n_img} image + {w.n_txt} text + {w.n_ref} "
+                               f"reference tokens, {blocks_text(w)}, width 3072", "seq_len": w.n_tokens,
+                   "global_batch": 1, "parallelism": "CPU oracle on rank 0"},
+        "tflops": round(forward_flops(w) / (value / 1e3) / 1e12, 4),
         "cpu_baseline": {"value": round(value, 3), "unit": step_unit(w), "cores": torch.get_num_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 3), "unit": step_unit(w), "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -249,7 +329,9 @@ def run_ours(args, w):
 
     blob, params = make_weights(w.dims, w.seed)
     lat_h, txt_h, ref_h = make_inputs(w)
-    model = F.FluxDiT(blob, w.dims)
+    flux3 = is_flux3(w)
+    model = (F.Flux3DiT if flux3 else F.FluxDiT)(blob, w.dims)
+    del blob
     stream = torch.cuda.current_stream()
     dev = torch.device("cuda", local)
     lat0 = torch.from_numpy(lat_h).to(dev)
@@ -278,6 +360,9 @@ def run_ours(args, w):
         if guided:
             model.forward_cfg(tok, (gh, gh), txt, txt_u, ts[k], v, v_u, ref_tok, hw_list)
             F.flux_cfg_euler_step(tok, v, v_u, w.guidance, ts[k + 1] - ts[k])
+        elif flux3:                                 # flow-map checkpoint: target time t_{k+1}
+            model.forward(tok, (gh, gh), txt, ts[k], v, ref_tok, hw_list, t_target=ts[k + 1])
+            F.flux_euler_step(tok, v, ts[k + 1] - ts[k])
         else:
             model.forward(tok, (gh, gh), txt, ts[k], v, ref_tok, ref_hw)
             F.flux_euler_step(tok, v, ts[k + 1] - ts[k])
@@ -371,13 +456,13 @@ def run_ours(args, w):
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) weights scaled 1/sqrt(fan_in), bf16; N(0,1) latent and text)",
             "config": {"workload": f"{w.name}: {w.image}x{w.image}, {w.n_img} image + {w.n_txt} text + {w.n_ref} "
-                                   f"reference tokens ({len(w.ref_grids)} reference images), 5 double + 20 single "
-                                   f"blocks, width 3072, 24x128 heads, one Euler step (pack, forward, Euler, unpack)"
+                                   f"reference tokens ({len(w.ref_grids)} reference images), {blocks_text(w)}, "
+                                   f"width 3072, 24x128 heads, one Euler step (pack, forward, Euler, unpack)"
                                    + ("" if not guided else f"; guidance {w.guidance}: prompt and unconditional "
                                       f"text as one batch-2 forward, fused guided Euler update"),
                        "global_batch": world, "seq_len": w.n_tokens,
                        "parallelism": f"replicas x{world}, no data-path collective",
-                       "l2": "inputs larger than L2: 9.7 GB of bf16 weights streamed every forward"},
+                       "l2": f"inputs larger than L2: {weight_gb(w):.1f} GB of bf16 weights streamed every forward"},
             "tflops": round(tflops, 1),
             "frac_bf16_peak": {"measured_burst": round(tflops / peaks["bf16_tflops"], 4),
                                "measured_sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
@@ -402,8 +487,10 @@ def run_ours(args, w):
             ms_cpu, secs = cpu_oracle_sample(w, params, lat_h, txt_h, ref_h)
             line["cpu_baseline"] = {"value": round(ms_cpu * n_sequences(w), 1), "unit": step_unit(w),
                                     "cores": torch.get_num_threads(), "kind": "oracle",
-                                    "sample": f"one double + one single block at full {w.name} size, fp32 oracle "
-                                              f"({secs:.1f} s), scaled x5 and x20 to a forward"
+                                    "sample": (f"one joint block at full {w.name} size, fp32 oracle ({secs:.1f} s), "
+                                               f"scaled by forward FLOPs / block FLOPs" if flux3 else
+                                               f"one double + one single block at full {w.name} size, fp32 oracle "
+                                               f"({secs:.1f} s), scaled x5 and x20 to a forward")
                                               + ("" if not guided else ", x2 for the two guided sequences")}
         print(json.dumps(line), flush=True)
     model.close()

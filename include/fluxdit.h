@@ -263,6 +263,88 @@ FLUX_API int flux_timestep_modulation_noalloc(const uint16_t *w1, const uint16_t
                                               int hidden, int t_freq_dim, int mod_rows, float t, float *mods_out,
                                               void *stream);
 
+/* ======================================================================
+ * FLUX.3 Image Klein ("FLUX.3 Image Klein in Diffusers: Architektur, Layout-Steuerung und
+ * Systemanforderungen im Überblick", mindverse).  The same kernels in the FLUX.3 block
+ * structure:
+ *   - "Zweistufiger Transformer und Tokenisierung": text features are the hidden states of 8
+ *     encoder layers (8 x 2560 = 20480 values per token) projected to the width by one linear;
+ *   - "Entkoppelte Vorverarbeitung und gemeinsame Attention-Blöcke": n_mode (5) per-mode blocks
+ *     in which the text, image and reference streams have their own weights and attend only to
+ *     themselves, then n_joint (28) joint blocks with one weight set over text | image |
+ *     reference; in every block attention and the SwiGLU MLP run in parallel on one
+ *     normalised input (the FLUX.2 single-stream block);
+ *   - "Modulation pro Token-Typ, Flow-Map-Destillation und 4D-RoPE": image tokens are modulated
+ *     with the current t, text and reference tokens with t = 0; the time-distilled checkpoint
+ *     (flow_map = 1) embeds the step's target time with its own MLP and adds it to the time
+ *     vector of every token.
+ * Readings where the page is silent: the modulation linears are shared by the blocks of a phase
+ * (one per stream for the per-mode phase, one for the joint phase: 5.49 B parameters against the
+ * page's 5.6 B; per-block linears would give 6.7 B); the target embedding has the time MLP's
+ * shape and is added before SiLU; the reference stream of the per-mode phase is every reference
+ * image together; block arithmetic as in the FLUX.2 single-stream block. */
+typedef struct flux3_dit flux3_dit;
+
+/* Defaults (FLUX.3 Image Klein): 5, 28, 3072, 24, 128, 9216, 128, 20480, 256, 1, 1e4, 1e-6, 1e-6.
+ * hidden == heads * head_dim, head_dim == 128, heads even, hidden and t_freq_dim <= 6144. */
+typedef struct {
+  int n_mode, n_joint, hidden, heads, head_dim, mlp_hidden, in_ch, txt_dim, t_freq_dim, flow_map;
+  float rope_theta, eps_ln, eps_rms;
+} flux3_dit_config;
+
+/* Bytes of a FLUX.3 weight blob for `cfg`, or 0 if cfg is invalid.
+ * Blob format (little endian, fields packed without padding): a 256-byte header
+ *   char magic[8] = "FLUX3DT\0"; uint32 version = 1; uint32 n_tensors;
+ *   int32 n_mode, n_joint, hidden, heads, head_dim, mlp_hidden, in_ch, txt_dim, t_freq_dim, flow_map;
+ *   float32 rope_theta, eps_ln, eps_rms; uint64 data_offset (= 256, at byte 68); uint64 data_bytes;
+ * then every tensor as bf16, row-major, each starting on a 256-byte boundary, in this order:
+ *   time_in.{w1 [D,256], b1, w2 [D,D], b2}, (flow_map only) target_in.{w1, b1, w2, b2},
+ *   img_in.{w [D,128], b}, txt_in.{w [D,txt_dim], b},
+ *   mode_mod.{txt, img, ref}.{w [3D,D], b [3D]}      rows: shift, scale, gate
+ *   for each per-mode block i, for stream s in (txt, img, ref):
+ *     lin1.{w [3D+2F,D], b}  q_gain [128]  k_gain [128]  lin2.{w [D,D+F], b [D]}
+ *   joint_mod.{w [3D,D], b [3D]}
+ *   for each joint block i: lin1, q_gain, k_gain, lin2 as above
+ *   final.mod.{w [2D,D], b [2D]} (shift, scale), final.out.{w [128,D], b [128]}. */
+FLUX_API size_t flux3_blob_expected_bytes(const flux3_dit_config *cfg);
+
+/* Create a FLUX.3 model from a weight blob in HOST memory (format above); as flux_dit_create. */
+FLUX_API flux3_dit *flux3_dit_create(const void *blob, size_t blob_bytes, const flux3_dit_config *cfg, void *stream);
+FLUX_API void flux3_dit_destroy(flux3_dit *m);
+
+/* One FLUX.3 forward: the velocity of the image tokens at time t.
+ *   img_tok fp32 [grid_h*grid_w, 128], txt fp32 [n_txt, txt_dim], ref_tok fp32 [sum_k h_k*w_k, 128]
+ *   (n_refs <= 10 references, ref_grids a HOST array of (h, w) pairs, RoPE l = -(k+1)),
+ *   v_out fp32 [grid_h*grid_w, 128].
+ * t_target: the step's target time (the sampler's next schedule point), read only by the
+ * flow-map model.  Shapes and workspace growth as flux_dit_forward_refs. */
+FLUX_API int flux3_dit_forward(flux3_dit *m, const float *img_tok, int grid_h, int grid_w, const float *txt,
+                               int n_txt, const float *ref_tok, int n_refs, const int *ref_grids, float t,
+                               float t_target, float *v_out, void *stream);
+
+/* Diagnostic: run only the first n_mode per-mode and n_joint joint blocks (-1 = all). */
+FLUX_API int flux3_dit_set_active_blocks(flux3_dit *m, int n_mode, int n_joint);
+
+/* Every modulation vector of a forward at (t, t_target), fp32 [17 * hidden]:
+ * per-mode text (shift, scale, gate; from the t = 0 time vector) | per-mode image (from t) |
+ * per-mode reference (t = 0) | joint image (t) | joint text and reference (t = 0) |
+ * output layer (shift, scale; from t). */
+FLUX_API size_t flux3_dit_modulation_size(const flux3_dit *m);
+FLUX_API int flux3_dit_modulation(flux3_dit *m, float t, float t_target, float *mods_out, void *stream);
+
+/* Per-kernel timing of later forwards; as flux_dit_profile / flux_dit_profile_read. */
+FLUX_API int flux3_dit_profile(flux3_dit *m, int enable);
+FLUX_API int flux3_dit_profile_read(flux3_dit *m, int kind, double *ms, double *flops, double *bytes,
+                                    long long *launches);
+
+/* Attention over n_seg (1..4) independent segments stored one after another: segment z is
+ * the seg_len[z] rows that follow segment z-1 and attends only to itself (the per-mode blocks'
+ * stream-local attention).  q, k, v, o bf16 [sum seg_len, heads, 128]; seg_len a HOST array,
+ * entries >= 0 (0 = empty segment).  Otherwise as flux_joint_attention. */
+FLUX_API int flux_joint_attention_segments(const uint16_t *q, const uint16_t *k, const uint16_t *v, uint16_t *o,
+                                           int n_seg, const int *seg_len, int heads, int head_dim, float scale,
+                                           void *stream);
+
 /* Synchronise `stream`, then read and clear the kernels' device error words:
  * 0 when no kernel gave up waiting, else the first nonzero code. */
 FLUX_API int flux_device_error(void *stream);

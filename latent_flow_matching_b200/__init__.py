@@ -1,4 +1,4 @@
-"""Python binding of libfluxdit.so, the sm_100a FLUX.2-klein transformer library.
+"""Python binding of libfluxdit.so, the sm_100a FLUX.2-klein / FLUX.3 Image Klein transformer library.
 
 Argument marshalling only: every function forwards device pointers of torch
 tensors (PyTorch owns the memory and the stream) to the C ABI declared in
@@ -29,6 +29,16 @@ class FluxConfig(ctypes.Structure):
     @classmethod
     def from_dims(cls, d):
         return cls(*(getattr(d, f) for f, _ in cls._fields_))
+
+
+class Flux3Config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("n_mode", "n_joint", "hidden", "heads", "head_dim", "mlp_hidden",
+                                            "in_ch", "txt_dim", "t_freq_dim", "flow_map")] + \
+               [(n, ctypes.c_float) for n in ("rope_theta", "eps_ln", "eps_rms")]
+
+    @classmethod
+    def from_dims(cls, d):
+        return cls(*(int(getattr(d, f)) if t is ctypes.c_int else getattr(d, f) for f, t in cls._fields_))
 
 
 class FluxError(RuntimeError):
@@ -68,6 +78,17 @@ _SIGS = {
     "flux_kernel_launches": (ctypes.c_ulonglong, []),
     "flux_timestep_modulation_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _F, _P, _P]),
     "flux_device_error": (_I, [_P]),
+    "flux3_blob_expected_bytes": (_Z, [ctypes.POINTER(Flux3Config)]),
+    "flux3_dit_create": (_P, [_P, _Z, ctypes.POINTER(Flux3Config), _P]),
+    "flux3_dit_destroy": (None, [_P]),
+    "flux3_dit_forward": (_I, [_P, _P, _I, _I, _P, _I, _P, _I, ctypes.POINTER(ctypes.c_int), _F, _F, _P, _P]),
+    "flux3_dit_set_active_blocks": (_I, [_P, _I, _I]),
+    "flux3_dit_modulation_size": (_Z, [_P]),
+    "flux3_dit_modulation": (_I, [_P, _F, _F, _P, _P]),
+    "flux3_dit_profile": (_I, [_P, _I]),
+    "flux3_dit_profile_read": (_I, [_P, _I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
+                                    ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]),
+    "flux_joint_attention_segments": (_I, [_P, _P, _P, _P, _I, ctypes.POINTER(ctypes.c_int), _I, _I, _F, _P]),
 }
 EXPORTED = tuple(_SIGS)
 
@@ -217,6 +238,83 @@ class FluxDiT:
         return out
 
 
+def flux3_blob_expected_bytes(dims) -> int:
+    cfg = Flux3Config.from_dims(dims)
+    return lib().flux3_blob_expected_bytes(ctypes.byref(cfg))
+
+
+def _grids(ref_hw):
+    """ref_hw: (), one (h, w), or a list of (h, w) -> (count, ctypes int array)."""
+    if ref_hw and not isinstance(ref_hw[0], (tuple, list)):
+        ref_hw = [tuple(ref_hw)] if ref_hw[0] else []
+    ref_hw = list(ref_hw or [])
+    return len(ref_hw), (ctypes.c_int * max(1, 2 * len(ref_hw)))(*[v for hw in ref_hw for v in hw])
+
+
+class Flux3DiT:
+    """A FLUX.3 Image Klein model created from a FLUX3DT weight blob (host bytes); see flux3_dit_create."""
+
+    PROFILE_KINDS = FluxDiT.PROFILE_KINDS
+
+    def __init__(self, blob: np.ndarray, dims=None, stream=None):
+        blob = np.ascontiguousarray(blob)
+        cfg = ctypes.byref(Flux3Config.from_dims(dims)) if dims is not None else None
+        h = lib().flux3_dit_create(ctypes.c_void_p(blob.ctypes.data), blob.nbytes, cfg, _stream(stream))
+        if not h:
+            raise FluxError(FLUX_EINVAL, get_error())
+        self._h = ctypes.c_void_p(h)
+        self.dims = dims
+        self.flow_map = bool(dims.flow_map) if dims is not None else True
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().flux3_dit_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def forward(self, img_tok, grid_hw, txt, t, v_out, ref_tok=None, ref_hw=(), t_target=0.0, stream=None):
+        """One forward.  ref_hw: (), one (h, w) or a list of them (ref_tok then holds every
+        reference's packed tokens in order).  t_target: the step's target time (flow-map model)."""
+        import torch
+        n_txt = 0 if txt is None else txt.shape[0]
+        n_refs, grids = _grids(ref_hw)
+        _check(lib().flux3_dit_forward(self._h, _ptr(img_tok, torch.float32, "img_tok"), grid_hw[0], grid_hw[1],
+                                       _ptr(txt, torch.float32, "txt"), n_txt,
+                                       _ptr(ref_tok, torch.float32, "ref_tok"), n_refs, grids, float(t),
+                                       float(t_target), _ptr(v_out, torch.float32, "v_out"), _stream(stream)))
+        return v_out
+
+    def set_active_blocks(self, n_mode=-1, n_joint=-1):
+        _check(lib().flux3_dit_set_active_blocks(self._h, n_mode, n_joint))
+
+    def modulation_size(self) -> int:
+        return lib().flux3_dit_modulation_size(self._h)
+
+    def modulation(self, t, t_target, out, stream=None):
+        import torch
+        _check(lib().flux3_dit_modulation(self._h, float(t), float(t_target), _ptr(out, torch.float32, "mods"),
+                                          _stream(stream)))
+        return out
+
+    def profile(self, enable: bool):
+        _check(lib().flux3_dit_profile(self._h, 1 if enable else 0))
+
+    def profile_read(self):
+        """{kind: (ms, flops, bytes, launches)} accumulated since profile(True)."""
+        out = {}
+        for i, name in enumerate(self.PROFILE_KINDS):
+            ms, fl, by, n = ctypes.c_double(), ctypes.c_double(), ctypes.c_double(), ctypes.c_longlong()
+            _check(lib().flux3_dit_profile_read(self._h, i, ctypes.byref(ms), ctypes.byref(fl), ctypes.byref(by),
+                                                ctypes.byref(n)))
+            out[name] = (ms.value, fl.value, by.value, n.value)
+        return out
+
+
 def euler_schedule(n_steps: int):
     """t_0 = 1 > ... > t_S = 0 evenly spaced (float32 values)."""
     return [float(np.float32(1.0 - i / n_steps)) for i in range(n_steps + 1)]
@@ -281,6 +379,18 @@ def flux_joint_attention_batch(q, k, v, o, batch, scale=None, stream=None):
     scale = hd ** -0.5 if scale is None else scale
     _check(lib().flux_joint_attention_batch(_bits(q, "q"), _bits(k, "k"), _bits(v, "v"), _bits(o, "o"), batch,
                                             rows // batch, heads, hd, float(scale), _stream(stream)))
+    return o
+
+
+def flux_joint_attention_segments(q, k, v, o, seg_len, scale=None, stream=None):
+    """q, k, v, o bf16 [sum(seg_len), heads, 128]; each segment attends only within itself."""
+    rows, heads, hd = q.shape
+    if sum(seg_len) != rows:
+        raise ValueError("segment lengths must add up to the row count")
+    scale = hd ** -0.5 if scale is None else scale
+    lens = (ctypes.c_int * len(seg_len))(*seg_len)
+    _check(lib().flux_joint_attention_segments(_bits(q, "q"), _bits(k, "k"), _bits(v, "v"), _bits(o, "o"),
+                                               len(seg_len), lens, heads, hd, float(scale), _stream(stream)))
     return o
 
 
@@ -403,6 +513,39 @@ def flux_sample(model: FluxDiT, latent, txt, n_steps, ref_latent=None, on_step=N
         return out
     for i in range(start, n_steps):
         model.forward(tok, (gh, gw), txt, ts[i], v, ref_tok, ref_hw, stream)
+        if on_step is not None:
+            on_step(i, v)
+        flux_euler_step(tok, v, ts[i + 1] - ts[i], stream)
+    out = torch.empty_like(latent)
+    flux_unpack_latents(tok, out, stream)
+    return out
+
+
+def flux3_sample(model: Flux3DiT, latent, txt, n_steps, ref_latent=None, on_step=None, stream=None):
+    """Euler sampling with a FLUX.3 model on the device: pack -> S x (forward, Euler) -> unpack.
+
+    The flow-map model receives t_{i+1} as the target time of step i.  latent fp32 [32, h8, w8]
+    (device): the noise; txt fp32 [n_txt, txt_dim]; ref_latent: None, one latent or a list.
+    Returns the final latent (new tensor); ``on_step(i, v)`` sees each velocity.
+    """
+    import torch
+    c, h8, w8 = latent.shape
+    gh, gw = h8 // 2, w8 // 2
+    ts = euler_schedule(n_steps)
+    tok = torch.empty(gh * gw, 4 * c, device=latent.device, dtype=torch.float32)
+    flux_pack_latents(latent, tok, stream)
+    ref_tok, grids = None, []
+    if ref_latent is not None:
+        refs = list(ref_latent) if isinstance(ref_latent, (list, tuple)) else [ref_latent]
+        grids = [(r.shape[1] // 2, r.shape[2] // 2) for r in refs]
+        ref_tok = torch.empty(sum(h * w for h, w in grids), 4 * c, device=latent.device, dtype=torch.float32)
+        row = 0
+        for r, (h, w) in zip(refs, grids):
+            flux_pack_latents(r, ref_tok[row:row + h * w], stream)
+            row += h * w
+    v = torch.empty_like(tok)
+    for i in range(n_steps):
+        model.forward(tok, (gh, gw), txt, ts[i], v, ref_tok, grids, t_target=ts[i + 1], stream=stream)
         if on_step is not None:
             on_step(i, v)
         flux_euler_step(tok, v, ts[i + 1] - ts[i], stream)

@@ -86,11 +86,16 @@ __global__ void cast_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __r
 // ------------------------------------------------------------------ LayerNorm + adaLN modulation
 // One 256-thread CTA per row: each thread keeps VPT float4 of the row in registers (dim = 1024 VPT),
 // mean and variance come from two block reductions, so many CTAs stay resident per SM.
+// Row r uses modulation set 0 when r % period < split, set 1 when it is < split2, else set 2.
+struct LnModSets {
+  int split, split2, period;
+  const float* sh[3];
+  const float* sc[3];
+};
+
 template <int VPT>
 __global__ void __launch_bounds__(256) ln_mod_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y,
-                                                     int rows, int split, int period, const float* __restrict__ sh0,
-                                                     const float* __restrict__ sc0, const float* __restrict__ sh1,
-                                                     const float* __restrict__ sc1, float eps) {
+                                                     int rows, const LnModSets m, float eps) {
   constexpr int dim = 1024 * VPT;
   __shared__ float red[2][8];
   const int row = blockIdx.x;
@@ -125,9 +130,10 @@ __global__ void __launch_bounds__(256) ln_mod_kernel(const float* __restrict__ x
 #pragma unroll
   for (int w = 0; w < 8; ++w) q += red[1][w];
   const float rstd = rsqrtf(q * (1.0f / dim) + eps);
-  const bool first = row % period < split;
-  const float4* shp = reinterpret_cast<const float4*>(first ? sh0 : sh1);
-  const float4* scp = reinterpret_cast<const float4*>(first ? sc0 : sc1);
+  const int r = row % m.period;
+  const int set = r < m.split ? 0 : (r < m.split2 ? 1 : 2);
+  const float4* shp = reinterpret_cast<const float4*>(m.sh[set]);
+  const float4* scp = reinterpret_cast<const float4*>(m.sc[set]);
   uint2* yr = reinterpret_cast<uint2*>(y + static_cast<size_t>(row) * dim);
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
@@ -142,8 +148,7 @@ __global__ void __launch_bounds__(256) ln_mod_kernel(const float* __restrict__ x
 
 // Any dim that is a multiple of 4: three passes over the row in global memory.
 __global__ void ln_mod_generic_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y, int rows, int dim,
-                                      int split, int period, const float* __restrict__ sh0, const float* __restrict__ sc0,
-                                      const float* __restrict__ sh1, const float* __restrict__ sc1, float eps) {
+                                      const LnModSets m, float eps) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= rows) return;
@@ -156,8 +161,10 @@ __global__ void ln_mod_generic_kernel(const float* __restrict__ x, __nv_bfloat16
   for (int i = lane; i < dim; i += 32) q += (xr[i] - mean) * (xr[i] - mean);
   for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
   const float rstd = rsqrtf(q / dim + eps);
-  const float* sh = warp % period < split ? sh0 : sh1;
-  const float* sc = warp % period < split ? sc0 : sc1;
+  const int r = warp % m.period;
+  const int set = r < m.split ? 0 : (r < m.split2 ? 1 : 2);
+  const float* sh = m.sh[set];
+  const float* sc = m.sc[set];
   for (int i = lane; i < dim; i += 32)
     y[static_cast<size_t>(warp) * dim + i] = __float2bfloat16_rn((xr[i] - mean) * rstd * (1.f + sc[i]) + sh[i]);
 }
@@ -285,12 +292,15 @@ __global__ void timestep_embed_kernel(float* __restrict__ out, float t, int dim)
 constexpr int kGemvRowsPerWarp = 4;
 constexpr int kGemvWarps = 8;
 
+// NV input vectors x[v] (k floats each, one after another) against one read of W:
+// y[v * rows + r] = act_out(W[r] . act_in(x[v]) + b[r] + add[r]) (add may be NULL).
+template <int NV>
 __global__ void __launch_bounds__(256) gemv_kernel(const __nv_bfloat16* __restrict__ W,
                                                    const __nv_bfloat16* __restrict__ b, const float* __restrict__ x,
-                                                   float* __restrict__ y, int rows, int k, int silu_in,
-                                                   int silu_out) {
+                                                   float* __restrict__ y, const float* __restrict__ add, int rows,
+                                                   int k, int silu_in, int silu_out) {
   extern __shared__ float xs[];
-  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+  for (int i = threadIdx.x; i < NV * k; i += blockDim.x) {
     const float v = x[i];
     xs[i] = silu_in ? silu_f(v) : v;
   }
@@ -299,30 +309,38 @@ __global__ void __launch_bounds__(256) gemv_kernel(const __nv_bfloat16* __restri
   const int chunks = k / 8;
   for (int r0 = (blockIdx.x * kGemvWarps + warp) * kGemvRowsPerWarp; r0 < rows;
        r0 += gridDim.x * kGemvWarps * kGemvRowsPerWarp) {
-    float acc[kGemvRowsPerWarp] = {0.f, 0.f, 0.f, 0.f};
+    float acc[NV][kGemvRowsPerWarp] = {};
 #pragma unroll 4
     for (int c = lane; c < chunks; c += 32) {
-      const float4 x0 = reinterpret_cast<const float4*>(xs)[2 * c];
-      const float4 x1 = reinterpret_cast<const float4*>(xs)[2 * c + 1];
+      uint4 w[kGemvRowsPerWarp];
+#pragma unroll
+      for (int rr = 0; rr < kGemvRowsPerWarp; ++rr)
+        w[rr] = r0 + rr < rows ? __ldcs(reinterpret_cast<const uint4*>(W + static_cast<size_t>(r0 + rr) * k) + c)
+                               : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        const float4 x0 = reinterpret_cast<const float4*>(xs + v * k)[2 * c];
+        const float4 x1 = reinterpret_cast<const float4*>(xs + v * k)[2 * c + 1];
+#pragma unroll
+        for (int rr = 0; rr < kGemvRowsPerWarp; ++rr)
+          acc[v][rr] += bf16lo(w[rr].x) * x0.x + bf16hi(w[rr].x) * x0.y + bf16lo(w[rr].y) * x0.z +
+                        bf16hi(w[rr].y) * x0.w + bf16lo(w[rr].z) * x1.x + bf16hi(w[rr].z) * x1.y +
+                        bf16lo(w[rr].w) * x1.z + bf16hi(w[rr].w) * x1.w;
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < NV; ++v)
 #pragma unroll
       for (int rr = 0; rr < kGemvRowsPerWarp; ++rr) {
-        if (r0 + rr < rows) {
-          const uint4 w = __ldcs(reinterpret_cast<const uint4*>(W + static_cast<size_t>(r0 + rr) * k) + c);
-          acc[rr] += bf16lo(w.x) * x0.x + bf16hi(w.x) * x0.y + bf16lo(w.y) * x0.z + bf16hi(w.y) * x0.w +
-                     bf16lo(w.z) * x1.x + bf16hi(w.z) * x1.y + bf16lo(w.w) * x1.z + bf16hi(w.w) * x1.w;
+        float a = acc[v][rr];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0 && r0 + rr < rows) {
+          a += __bfloat162float(b[r0 + rr]);
+          if (add) a += add[r0 + rr];
+          y[static_cast<size_t>(v) * rows + r0 + rr] = silu_out ? silu_f(a) : a;
         }
       }
-    }
-#pragma unroll
-    for (int rr = 0; rr < kGemvRowsPerWarp; ++rr) {
-      float a = acc[rr];
-#pragma unroll
-      for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-      if (lane == 0 && r0 + rr < rows) {
-        a += __bfloat162float(b[r0 + rr]);
-        y[r0 + rr] = silu_out ? silu_f(a) : a;
-      }
-    }
   }
 }
 
@@ -364,18 +382,26 @@ cudaError_t cast_bf16_launch(const float* x, __nv_bfloat16* y, size_t n, cudaStr
   return cudaGetLastError();
 }
 
+cudaError_t ln_modulate3_launch(const float* x, __nv_bfloat16* y, int rows, int dim, int split, int split2,
+                                int period, const float* shift0, const float* scale0, const float* shift1,
+                                const float* scale1, const float* shift2, const float* scale2, float eps,
+                                cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if (period <= 0) return cudaErrorInvalidValue;
+  const LnModSets m = {split, split2, period, {shift0, shift1, shift2}, {scale0, scale1, scale2}};
+  count_launch();
+  if (dim == 3072)
+    ln_mod_kernel<3><<<rows, 256, 0, s>>>(x, y, rows, m, eps);
+  else
+    ln_mod_generic_kernel<<<(rows + 7) / 8, 256, 0, s>>>(x, y, rows, dim, m, eps);
+  return cudaGetLastError();
+}
+
 cudaError_t ln_modulate_launch(const float* x, __nv_bfloat16* y, int rows, int dim, int split, int period,
                                const float* shift0, const float* scale0, const float* shift1, const float* scale1,
                                float eps, cudaStream_t s) {
-  if (rows <= 0) return cudaSuccess;
-  if (period <= 0) return cudaErrorInvalidValue;
-  count_launch();
-  if (dim == 3072)
-    ln_mod_kernel<3><<<rows, 256, 0, s>>>(x, y, rows, split, period, shift0, scale0, shift1, scale1, eps);
-  else
-    ln_mod_generic_kernel<<<(rows + 7) / 8, 256, 0, s>>>(x, y, rows, dim, split, period, shift0, scale0, shift1,
-                                                          scale1, eps);
-  return cudaGetLastError();
+  return ln_modulate3_launch(x, y, rows, dim, split, period, period, shift0, scale0, shift1, scale1, shift1, scale1,
+                             eps, s);
 }
 
 cudaError_t qk_norm_rope_launch(__nv_bfloat16* qkv, int rows, int ld, int kcol, int heads, int split,
@@ -412,16 +438,27 @@ cudaError_t timestep_embed_launch(float* temb, float t, int dim, cudaStream_t s)
   return cudaGetLastError();
 }
 
-cudaError_t gemv_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, const float* x, float* y, int rows, int k,
-                        int silu_in, int silu_out, cudaStream_t s) {
+cudaError_t gemv_multi_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, const float* x, int nvec, float* y,
+                              const float* add, int rows, int k, int silu_in, int silu_out, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
+  if (nvec < 1 || nvec > 2 || k % 8) return cudaErrorInvalidValue;
   const int per_block = kGemvWarps * kGemvRowsPerWarp;
   int grid = (rows + per_block - 1) / per_block;
   const int cap = num_sms_current() * 8;
   if (grid > cap) grid = cap;
+  const size_t smem = static_cast<size_t>(nvec) * k * sizeof(float);
+  if (smem > 48 * 1024) return cudaErrorInvalidValue;
   count_launch();
-  gemv_kernel<<<grid, 256, k * sizeof(float), s>>>(W, b, x, y, rows, k, silu_in, silu_out);
+  if (nvec == 1)
+    gemv_kernel<1><<<grid, 256, smem, s>>>(W, b, x, y, add, rows, k, silu_in, silu_out);
+  else
+    gemv_kernel<2><<<grid, 256, smem, s>>>(W, b, x, y, add, rows, k, silu_in, silu_out);
   return cudaGetLastError();
+}
+
+cudaError_t gemv_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, const float* x, float* y, int rows, int k,
+                        int silu_in, int silu_out, cudaStream_t s) {
+  return gemv_multi_launch(W, b, x, 1, y, nullptr, rows, k, silu_in, silu_out, s);
 }
 
 }  // namespace fdit

@@ -28,6 +28,7 @@
 
 #include "../../include/fluxdit.h"
 #include "fluxdit_internal.h"
+#include "runner.h"
 
 using bf16 = __nv_bfloat16;
 
@@ -36,7 +37,7 @@ namespace fdit {
 // ------------------------------------------------------------------ errors
 static thread_local std::string g_error;
 
-static int fail(int code, const char* fmt, ...) {
+int fail(int code, const char* fmt, ...) {
   char buf[512];
   va_list ap;
   va_start(ap, fmt);
@@ -48,11 +49,7 @@ static int fail(int code, const char* fmt, ...) {
 
 int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
 
-#define FD_CUDA(expr)                                                                          \
-  do {                                                                                         \
-    cudaError_t e_ = (expr);                                                                   \
-    if (e_ != cudaSuccess) return fail(FLUX_EIO, "%s: %s", #expr, cudaGetErrorString(e_));     \
-  } while (0)
+const char* last_error() { return g_error.c_str(); }
 
 // ------------------------------------------------------------------ tensor maps
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -88,79 +85,19 @@ int num_sms_current() {
 static std::atomic<unsigned long long> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
-// ------------------------------------------------------------------ per-kernel profiling
-// When enabled, every launch of a forward is bracketed by two CUDA events on its
-// stream; flux_dit_profile_read() synchronises and accumulates the elapsed time
-// per kernel kind together with the launch's algorithmic FLOPs and HBM bytes.
-enum ProfKind { kProfGemm = 0, kProfAttention, kProfLnMod, kProfQkNormRope, kProfGemv, kProfOther, kProfKinds };
-struct ProfRec {
-  int kind;
-  cudaEvent_t a, b;
-  double flops, bytes;
-};
-struct Profiler {
-  bool on = false;
-  std::vector<cudaEvent_t> pool;
-  std::vector<ProfRec> pending;
-  double ms[kProfKinds] = {}, flops[kProfKinds] = {}, bytes[kProfKinds] = {};
-  long long launches[kProfKinds] = {};
-  cudaEvent_t get() {
-    if (!pool.empty()) {
-      cudaEvent_t e = pool.back();
-      pool.pop_back();
-      return e;
-    }
-    cudaEvent_t e = nullptr;
-    cudaEventCreate(&e);
-    return e;
-  }
-  void settle() {
-    for (const ProfRec& r : pending) {
-      float t = 0.f;
-      if (cudaEventElapsedTime(&t, r.a, r.b) == cudaSuccess) {
-        ms[r.kind] += t;
-        flops[r.kind] += r.flops;
-        bytes[r.kind] += r.bytes;
-        launches[r.kind] += 1;
-      }
-      pool.push_back(r.a);
-      pool.push_back(r.b);
-    }
-    pending.clear();
-  }
-  void reset() {
-    settle();
-    for (int k = 0; k < kProfKinds; ++k) ms[k] = flops[k] = bytes[k] = 0, launches[k] = 0;
-  }
-  ~Profiler() {
-    settle();
-    for (cudaEvent_t e : pool) cudaEventDestroy(e);
-  }
-};
-
-static double gemm_flops(const GemmParams& P) {
-  double f = 0;
-  for (int i = 0; i < P.num_problems; ++i)
-    if (P.prob[i].M > 0) f += 2.0 * P.prob[i].M * static_cast<double>(P.prob[i].N) * P.prob[i].K;
-  return f;
-}
-static double gemm_bytes(const GemmParams& P) {
-  double b = 0;
-  for (int i = 0; i < P.num_problems; ++i) {
-    const GemmProblem& pr = P.prob[i];
-    if (pr.M <= 0) continue;
-    const double out_elt = pr.mode == kEpiBf16Bias ? 2 : pr.mode == kEpiSwiGLU ? 1 : pr.mode == kEpiF32Bias ? 4 : 8;
-    b += 2.0 * pr.M * pr.K + 2.0 * pr.N * pr.K + out_elt * pr.M * pr.N;
-  }
-  return b;
-}
-
 // ------------------------------------------------------------------ blob layout
 struct BlobTensor {
   std::string name;
   size_t rows, cols;        // cols = 1 for vectors
   size_t blob_off;          // byte offset in the blob
 };
+
+int device_error_words(cudaStream_t s) {
+  const int g = gemm_read_device_error(s);
+  const int g2 = gemm2_read_device_error(s);
+  const int a = attention_read_device_error(s);
+  return g ? g : (g2 ? g2 : a);
+}
 
 static bool valid_cfg(const flux_dit_config& c) {
   return c.n_double >= 0 && c.n_single >= 0 && c.n_double + c.n_single >= 1 && c.head_dim == 128 &&
@@ -280,9 +217,7 @@ static void destroy(flux_dit* m) {
   delete m;
 }
 
-// Host -> device copy of SwiGLU rows [a (F rows); b (F rows)] of width `row_bytes`
-// into the GEMM order: for each group of 128 output columns, its 128 a-rows then its 128 b-rows.
-static cudaError_t copy_swiglu(void* dst, const uint8_t* src, size_t F, size_t row_bytes, cudaStream_t s) {
+cudaError_t copy_swiglu(void* dst, const uint8_t* src, size_t F, size_t row_bytes, cudaStream_t s) {
   const size_t chunk = 128 * row_bytes;
   const size_t groups = F / 128;
   cudaError_t e = cudaMemcpy2DAsync(dst, 2 * chunk, src, chunk, chunk, groups, cudaMemcpyHostToDevice, s);
@@ -427,30 +362,6 @@ static int create_impl(const void* blob, size_t blob_bytes, const flux_dit_confi
   return FLUX_OK;
 }
 
-template <typename T>
-static cudaError_t grow(T** p, size_t* cap, size_t need) {
-  if (need <= *cap) return cudaSuccess;
-  cudaFree(*p);
-  *p = nullptr;
-  *cap = 0;
-  cudaError_t e = cudaMalloc(p, need * sizeof(T));
-  if (e == cudaSuccess) *cap = need;
-  return e;
-}
-
-static size_t ref_tokens(const RefGrids& r) {
-  size_t n = 0;
-  for (int k = 0; k < r.count; ++k) n += static_cast<size_t>(r.h[k]) * r.w[k];
-  return n;
-}
-
-static bool same_refs(const RefGrids& a, const RefGrids& b) {
-  if (a.count != b.count) return false;
-  for (int k = 0; k < a.count; ++k)
-    if (a.h[k] != b.h[k] || a.w[k] != b.w[k]) return false;
-  return true;
-}
-
 static int prepare_shape(flux_dit* m, int nt, int gh, int gw, const RefGrids& refs, int nb, cudaStream_t s) {
   Workspace& w = m->ws;
   const flux_dit_config& c = m->cfg;
@@ -511,43 +422,6 @@ static int prepare_shape(flux_dit* m, int nt, int gh, int gw, const RefGrids& re
       return fail(FLUX_EIO, "rope table copy failed");
   w.nt = nt; w.gh = gh; w.gw = gw; w.nb = nb; w.refs = refs;
   return FLUX_OK;
-}
-
-// Enqueue `expr` (a launch returning cudaError_t); bracket it with profiling events when enabled.
-#define FD_LAUNCH(m, kind, fl, by, expr)                                                   \
-  do {                                                                                     \
-    cudaEvent_t ea_ = nullptr, eb_ = nullptr;                                              \
-    if ((m)->prof.on) {                                                                    \
-      ea_ = (m)->prof.get();                                                               \
-      eb_ = (m)->prof.get();                                                               \
-      cudaEventRecord(ea_, s);                                                             \
-    }                                                                                      \
-    FD_CUDA(expr);                                                                         \
-    if ((m)->prof.on) {                                                                    \
-      cudaEventRecord(eb_, s);                                                             \
-      (m)->prof.pending.push_back({(kind), ea_, eb_, (fl), (by)});                         \
-    }                                                                                      \
-  } while (0)
-
-static void problem(GemmParams& P, int i, const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, int mode,
-                    void* out, int ldo, const bf16* bias, const float* gate) {
-  P.mapA[i] = a;
-  P.mapB[i] = b;
-  GemmProblem& pr = P.prob[i];
-  pr = GemmProblem();
-  pr.M = M; pr.N = N; pr.K = K; pr.mode = mode; pr.out = out; pr.ldo = ldo; pr.bias = bias; pr.gate = gate;
-}
-
-// Make problem i a fused qkv + QK-RMSNorm + RoPE projection (rows start at token rope_row0).
-static void qk_fuse(GemmParams& P, int i, const bf16* gq, const bf16* gk, const float2* rope, int rope_row0,
-                    float eps) {
-  GemmProblem& pr = P.prob[i];
-  pr.mode = kEpiQKNormRope;
-  pr.gain_q = gq;
-  pr.gain_k = gk;
-  pr.rope = rope;
-  pr.rope_row0 = rope_row0;
-  pr.eps = eps;
 }
 
 static int run_modulation(flux_dit* m, float t, cudaStream_t s) {
@@ -706,8 +580,6 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
   return FLUX_OK;
 }
 
-static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
-
 }  // namespace fdit
 
 using namespace fdit;
@@ -715,7 +587,7 @@ using namespace fdit;
 // ====================================================================== C ABI
 extern "C" {
 
-const char* flux_get_error(void) { return g_error.c_str(); }
+const char* flux_get_error(void) { return last_error(); }
 
 size_t flux_blob_expected_bytes(const flux_dit_config* cfg) {
   if (!cfg || !valid_cfg(*cfg)) return 0;
@@ -976,10 +848,7 @@ unsigned long long flux_kernel_launches(void) { return g_launches.load(); }
 int flux_device_error(void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   FD_CUDA(cudaStreamSynchronize(s));
-  const int g = gemm_read_device_error(s);
-  const int g2 = gemm2_read_device_error(s);
-  const int a = attention_read_device_error(s);
-  return g ? g : (g2 ? g2 : a);
+  return device_error_words(s);
 }
 
 }  // extern "C"

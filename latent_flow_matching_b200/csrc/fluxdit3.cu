@@ -1,0 +1,620 @@
+// FLUX.3 Image Klein denoising transformer on B200: host runner and C ABI.
+//
+// The same sm_100a kernels as the FLUX.2-klein runner, arranged into the FLUX.3 block
+// structure ("FLUX.3 Image Klein in Diffusers: Architektur, Layout-Steuerung und
+// Systemanforderungen im Überblick", mindverse):
+//   * "Zweistufiger Transformer und Tokenisierung": text features are 8 encoder layers of
+//     2560 values (20480 per token) projected to the width 3072 by one linear layer;
+//   * "Entkoppelte Vorverarbeitung und gemeinsame Attention-Blöcke": 5 per-mode blocks in which
+//     the text, noisy-image and reference streams have their own weights and attend only to
+//     themselves, then 28 joint blocks with one weight set over text | image | reference; every
+//     block runs attention and the SwiGLU MLP in parallel on one normalised input;
+//   * "Modulation pro Token-Typ, Flow-Map-Destillation und 4D-RoPE": image tokens are
+//     modulated with the current t, text and reference tokens with t = 0; the time-distilled
+//     checkpoint adds an embedding of the step's target time to every token's conditioning.
+//
+// Forward (one CUDA stream, no host synchronisation):
+//   time vectors: vec_img = MLP_time(emb(t)) (+ MLP_target(emb(t_target))),
+//                 vec_ctx = MLP_time(emb(0)) (+ the same target term)
+//   modulation GEMVs: per-mode linears (text and reference from vec_ctx, image from vec_img),
+//                 the joint linear on both vectors at once, the output layer's from vec_img
+//   txt_in (K = 20480) / img_in projections (one grouped GEMM) into the fp32 residual X
+//   5 x per-mode block: LN+mod (three row ranges, three modulation sets)
+//        -> linear1 GEMM, 6 problems (qkv with fused QK-RMSNorm + RoPE, SwiGLU; per stream)
+//        -> attention over three independent segments (one launch)
+//        -> linear2 GEMM, 3 problems (per-stream weights and gates) + gate * residual
+//   28 x joint block: LN+mod (image rows: the t set; text and reference rows: the t = 0 set)
+//        -> linear1 GEMM (qkv | SwiGLU over all rows) -> joint attention
+//        -> linear2 GEMM, 3 row-range problems sharing W, each with its token type's gate
+//   final LN+mod on the image rows -> output GEMM -> velocity (fp32)
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/fluxdit.h"
+#include "fluxdit_internal.h"
+#include "runner.h"
+
+namespace fdit {
+namespace {
+
+constexpr size_t kHeaderBytes = 256;
+
+struct BlobTensor3 {
+  std::string name;
+  size_t rows, cols;     // cols = 1 for vectors
+  size_t off;            // byte offset in the blob
+};
+
+bool valid_cfg3(const flux3_dit_config& c) {
+  return c.n_mode >= 0 && c.n_joint >= 0 && c.n_mode + c.n_joint >= 1 && c.head_dim == 128 && c.heads >= 2 &&
+         c.heads % 2 == 0 && c.hidden == c.heads * c.head_dim && c.mlp_hidden > 0 && c.mlp_hidden % 128 == 0 &&
+         c.in_ch == 128 && c.txt_dim > 0 && c.txt_dim % 64 == 0 && c.t_freq_dim > 0 && c.t_freq_dim % 64 == 0 &&
+         c.t_freq_dim <= 6144 && c.hidden <= 6144 && (c.flow_map == 0 || c.flow_map == 1) && c.rope_theta > 0 &&
+         c.eps_ln > 0 && c.eps_rms > 0;
+}
+
+const char* kStreams[3] = {"txt", "img", "ref"};
+
+// Tensor order of the FLUX.3 blob (documented in fluxdit.h).
+std::vector<BlobTensor3> blob_tensors3(const flux3_dit_config& c, size_t* total) {
+  const size_t D = c.hidden, F = c.mlp_hidden, hd = c.head_dim;
+  std::vector<BlobTensor3> t;
+  auto add = [&](const std::string& n, size_t r, size_t k) { t.push_back({n, r, k, 0}); };
+  auto block = [&](const std::string& p) {
+    add(p + "lin1.w", 3 * D + 2 * F, D); add(p + "lin1.b", 3 * D + 2 * F, 1);
+    add(p + "q_gain", hd, 1); add(p + "k_gain", hd, 1);
+    add(p + "lin2.w", D, D + F); add(p + "lin2.b", D, 1);
+  };
+  add("time_in.w1", D, c.t_freq_dim); add("time_in.b1", D, 1);
+  add("time_in.w2", D, D); add("time_in.b2", D, 1);
+  if (c.flow_map) {
+    add("target_in.w1", D, c.t_freq_dim); add("target_in.b1", D, 1);
+    add("target_in.w2", D, D); add("target_in.b2", D, 1);
+  }
+  add("img_in.w", D, c.in_ch); add("img_in.b", D, 1);
+  add("txt_in.w", D, c.txt_dim); add("txt_in.b", D, 1);
+  for (const char* s : kStreams) {
+    add(std::string("mode_mod.") + s + ".w", 3 * D, D);
+    add(std::string("mode_mod.") + s + ".b", 3 * D, 1);
+  }
+  for (int i = 0; i < c.n_mode; ++i)
+    for (const char* s : kStreams) block("mode." + std::to_string(i) + "." + s + ".");
+  add("joint_mod.w", 3 * D, D); add("joint_mod.b", 3 * D, 1);
+  for (int i = 0; i < c.n_joint; ++i) block("joint." + std::to_string(i) + ".");
+  add("final.mod.w", 2 * D, D); add("final.mod.b", 2 * D, 1);
+  add("final.out.w", c.in_ch, D); add("final.out.b", c.in_ch, 1);
+  size_t off = kHeaderBytes;
+  for (auto& x : t) {
+    x.off = off;
+    off = (off + x.rows * x.cols * 2 + 255) / 256 * 256;
+  }
+  *total = off;
+  return t;
+}
+
+// Header fields at their byte offsets (little endian, no padding):
+// magic[8] | u32 version | u32 n_tensors | i32 x 10 | f32 x 3 | u64 data_offset | u64 data_bytes
+struct Header3 {
+  uint32_t version, n_tensors;
+  flux3_dit_config cfg;
+  uint64_t data_offset, data_bytes;
+};
+
+bool read_header3(const void* blob, size_t bytes, Header3* h) {
+  if (!blob || bytes < kHeaderBytes) return false;
+  const uint8_t* b = static_cast<const uint8_t*>(blob);
+  if (memcmp(b, "FLUX3DT\0", 8) != 0) return false;
+  int32_t iv[10];
+  float fv[3];
+  memcpy(&h->version, b + 8, 4);
+  memcpy(&h->n_tensors, b + 12, 4);
+  memcpy(iv, b + 16, 40);
+  memcpy(fv, b + 56, 12);
+  memcpy(&h->data_offset, b + 68, 8);
+  memcpy(&h->data_bytes, b + 76, 8);
+  h->cfg = {iv[0], iv[1], iv[2], iv[3], iv[4], iv[5], iv[6], iv[7], iv[8], iv[9], fv[0], fv[1], fv[2]};
+  return true;
+}
+
+// One parallel block's weights (per-mode stream or joint block).
+struct BlockW3 {
+  const bf16 *qkv_b, *mlp_b, *q_gain, *k_gain, *lin2_b;
+  CUtensorMap m_qkv, m_mlp, m_lin2;
+};
+
+// Row ranges of the joint sequence: text | image | reference (all references together).
+enum Seg { kSegTxt = 0, kSegImg = 1, kSegRef = 2 };
+
+struct Workspace3 {
+  size_t cap_n = 0, cap_tok = 0, cap_txt = 0;
+  float* X = nullptr;
+  bf16 *Y = nullptr, *QKV = nullptr, *CC = nullptr, *tokb = nullptr, *txtb = nullptr;
+  float2* rope = nullptr;
+  int nt = -1, gh = -1, gw = -1;
+  RefGrids refs = {-1, {}, {}};
+  CUtensorMap a_tokb, a_txtb, a_Yall, a_Yout, qkv;
+  CUtensorMap a_Yseg[3], a_CCseg[3];
+};
+
+// Offsets (in units of D floats) of the modulation vectors in the model's mods buffer.
+constexpr int kModTxt = 0, kModImg = 3, kModRef = 6, kModJointImg = 9, kModJointCtx = 12, kModFinal = 15,
+              kModRowsD = 17;
+
+}  // namespace
+}  // namespace fdit
+
+using fdit::bf16;
+
+struct flux3_dit {
+  flux3_dit_config cfg;
+  int device = 0, num_sms = 148;
+  void* wbuf = nullptr;
+  float* scratch = nullptr;      // temb [3][t_freq] | th [3][D] | tt [D] | vec [2][D] | mods [17 D]
+  float *temb = nullptr, *th = nullptr, *tt = nullptr, *vec = nullptr, *mods = nullptr;
+  const bf16 *t_w1, *t_b1, *t_w2, *t_b2, *g_w1 = nullptr, *g_b1 = nullptr, *g_w2 = nullptr, *g_b2 = nullptr;
+  const bf16 *img_b, *txt_b, *fin_b;
+  const bf16 *mode_mod_w[3], *mode_mod_b[3], *joint_mod_w, *joint_mod_b, *fin_mod_w, *fin_mod_b;
+  CUtensorMap m_img_in, m_txt_in, m_fin;
+  std::vector<fdit::BlockW3> mode;    // [3 i + stream], stream 0 text, 1 image, 2 reference
+  std::vector<fdit::BlockW3> joint;
+  int act_mode = 0, act_joint = 0;
+  fdit::Workspace3 ws;
+  fdit::Profiler prof;
+};
+
+namespace fdit {
+namespace {
+
+void free_ws3(Workspace3& w) {
+  cudaFree(w.X); cudaFree(w.Y); cudaFree(w.QKV); cudaFree(w.CC); cudaFree(w.tokb); cudaFree(w.txtb);
+  cudaFree(w.rope);
+  w = Workspace3();
+}
+
+void destroy3(flux3_dit* m) {
+  if (!m) return;
+  free_ws3(m->ws);
+  cudaFree(m->wbuf);
+  cudaFree(m->scratch);
+  delete m;
+}
+
+int create3_impl(const void* blob, size_t blob_bytes, const flux3_dit_config* cfg_in, cudaStream_t s,
+                 flux3_dit** out) {
+  *out = nullptr;
+  Header3 h;
+  if (!read_header3(blob, blob_bytes, &h) || h.version != 1 || h.data_offset != kHeaderBytes)
+    return fail(FLUX_EINVAL, "not a FLUX3DT v1 blob");
+  const flux3_dit_config c = h.cfg;
+  if (cfg_in && memcmp(cfg_in, &c, sizeof(c)) != 0) return fail(FLUX_EINVAL, "config differs from the blob header");
+  if (!valid_cfg3(c)) return fail(FLUX_EINVAL, "unsupported FLUX.3 model config in blob header");
+  size_t total = 0;
+  const std::vector<BlobTensor3> ts = blob_tensors3(c, &total);
+  if (h.n_tensors != ts.size() || h.data_bytes + kHeaderBytes != total || blob_bytes < total)
+    return fail(FLUX_EINVAL, "blob size / tensor count mismatch (expected %zu bytes, %zu tensors)", total, ts.size());
+
+  flux3_dit* m = new flux3_dit();
+  m->cfg = c;
+  cudaGetDevice(&m->device);
+  m->num_sms = num_sms_current();
+  const size_t D = c.hidden, F = c.mlp_hidden;
+  auto cleanup = [&](int code, const char* what) {
+    destroy3(m);
+    return fail(code, "%s", what);
+  };
+  // device copy: the blob's tensor area as is (same offsets), SwiGLU rows of linear1 re-interleaved
+  const size_t scratch_floats = 3 * c.t_freq_dim + 3 * D + D + 2 * D + kModRowsD * D;
+  if (cudaMalloc(&m->wbuf, total - kHeaderBytes) != cudaSuccess ||
+      cudaMalloc(&m->scratch, scratch_floats * sizeof(float)) != cudaSuccess)
+    return cleanup(FLUX_ENOMEM, "cudaMalloc of model weights failed");
+  m->temb = m->scratch;
+  m->th = m->temb + 3 * c.t_freq_dim;
+  m->tt = m->th + 3 * D;
+  m->vec = m->tt + D;
+  m->mods = m->vec + 2 * D;
+  uint8_t* wb = static_cast<uint8_t*>(m->wbuf);
+  const uint8_t* b8 = static_cast<const uint8_t*>(blob);
+  for (const BlobTensor3& t : ts) {
+    uint8_t* dst = wb + (t.off - kHeaderBytes);
+    const uint8_t* src = b8 + t.off;
+    cudaError_t e;
+    if (t.name.find("lin1.") != std::string::npos) {
+      const size_t qkv_bytes = 3 * D * t.cols * 2;
+      e = cudaMemcpyAsync(dst, src, qkv_bytes, cudaMemcpyHostToDevice, s);
+      if (e == cudaSuccess) e = copy_swiglu(dst + qkv_bytes, src + qkv_bytes, F, t.cols * 2, s);
+    } else {
+      e = cudaMemcpyAsync(dst, src, t.rows * t.cols * 2, cudaMemcpyHostToDevice, s);
+    }
+    if (e != cudaSuccess) return cleanup(FLUX_EIO, "weight upload failed");
+  }
+
+  auto W = [&](const std::string& n) -> const bf16* {
+    for (const BlobTensor3& t : ts)
+      if (t.name == n) return reinterpret_cast<const bf16*>(wb + (t.off - kHeaderBytes));
+    return nullptr;
+  };
+  bool maps_ok = true;
+  auto wmap = [&](CUtensorMap* map, const bf16* base, size_t rows, size_t cols) {
+    maps_ok &= make_tmap_bf16(map, base, rows, cols, cols * 2, 128);
+  };
+  m->t_w1 = W("time_in.w1"); m->t_b1 = W("time_in.b1"); m->t_w2 = W("time_in.w2"); m->t_b2 = W("time_in.b2");
+  if (c.flow_map) {
+    m->g_w1 = W("target_in.w1"); m->g_b1 = W("target_in.b1");
+    m->g_w2 = W("target_in.w2"); m->g_b2 = W("target_in.b2");
+  }
+  m->img_b = W("img_in.b"); m->txt_b = W("txt_in.b"); m->fin_b = W("final.out.b");
+  wmap(&m->m_img_in, W("img_in.w"), D, c.in_ch);
+  wmap(&m->m_txt_in, W("txt_in.w"), D, c.txt_dim);
+  wmap(&m->m_fin, W("final.out.w"), c.in_ch, D);
+  for (int sidx = 0; sidx < 3; ++sidx) {
+    m->mode_mod_w[sidx] = W(std::string("mode_mod.") + kStreams[sidx] + ".w");
+    m->mode_mod_b[sidx] = W(std::string("mode_mod.") + kStreams[sidx] + ".b");
+  }
+  m->joint_mod_w = W("joint_mod.w"); m->joint_mod_b = W("joint_mod.b");
+  m->fin_mod_w = W("final.mod.w"); m->fin_mod_b = W("final.mod.b");
+  auto block = [&](BlockW3& bw, const std::string& p) {
+    const bf16* l1 = W(p + "lin1.w");
+    const bf16* l1b = W(p + "lin1.b");
+    bw.qkv_b = l1b; bw.mlp_b = l1b + 3 * D;
+    bw.q_gain = W(p + "q_gain"); bw.k_gain = W(p + "k_gain"); bw.lin2_b = W(p + "lin2.b");
+    wmap(&bw.m_qkv, l1, 3 * D, D);
+    wmap(&bw.m_mlp, l1 + 3 * D * D, 2 * F, D);
+    wmap(&bw.m_lin2, W(p + "lin2.w"), D, D + F);
+  };
+  m->mode.resize(3 * c.n_mode);
+  for (int i = 0; i < c.n_mode; ++i)
+    for (int sidx = 0; sidx < 3; ++sidx)
+      block(m->mode[3 * i + sidx], "mode." + std::to_string(i) + "." + kStreams[sidx] + ".");
+  m->joint.resize(c.n_joint);
+  for (int i = 0; i < c.n_joint; ++i) block(m->joint[i], "joint." + std::to_string(i) + ".");
+  if (!maps_ok) return cleanup(FLUX_EIO, "cuTensorMapEncodeTiled failed for a weight tensor");
+  m->act_mode = c.n_mode;
+  m->act_joint = c.n_joint;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return cleanup(FLUX_EIO, "weight upload failed (sync)");
+  *out = m;
+  return FLUX_OK;
+}
+
+int prepare_shape3(flux3_dit* m, int nt, int gh, int gw, const RefGrids& refs, cudaStream_t s) {
+  Workspace3& w = m->ws;
+  const flux3_dit_config& c = m->cfg;
+  const size_t D = c.hidden, F = c.mlp_hidden;
+  const size_t ni = static_cast<size_t>(gh) * gw, nr = ref_tokens(refs);
+  const size_t n = nt + ni + nr;
+  if (n > w.cap_n) {
+    free_ws3(w);
+    bool ok = cudaMalloc(&w.X, n * D * 4) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.Y, n * D * 2) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.QKV, n * 3 * D * 2) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.CC, n * (D + F) * 2) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.rope, n * 64 * sizeof(float2)) == cudaSuccess;
+    if (!ok) {
+      free_ws3(w);
+      return fail(FLUX_ENOMEM, "workspace allocation for %zu tokens failed", n);
+    }
+    w.cap_n = n;
+  }
+  if (grow(&w.tokb, &w.cap_tok, (ni + nr) * c.in_ch) != cudaSuccess ||
+      grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt, 1) * c.txt_dim) != cudaSuccess)
+    return fail(FLUX_ENOMEM, "workspace allocation failed");
+  if (w.nt == nt && w.gh == gh && w.gw == gw && same_refs(w.refs, refs)) return FLUX_OK;
+
+  const uint64_t ldD = D * 2, ldC = (D + F) * 2;
+  bool ok = true;
+  auto amap = [&](CUtensorMap* map, const void* base, size_t rows, size_t cols, uint64_t stride) {
+    if (rows == 0) {
+      memset(map, 0, sizeof(*map));
+      return;
+    }
+    ok &= make_tmap_bf16(map, base, rows, cols, stride, 128);
+  };
+  const size_t row0[3] = {0, static_cast<size_t>(nt), nt + ni};
+  const size_t rows[3] = {static_cast<size_t>(nt), ni, nr};
+  amap(&w.a_tokb, w.tokb, ni + nr, c.in_ch, c.in_ch * 2);
+  amap(&w.a_txtb, w.txtb, nt, c.txt_dim, static_cast<uint64_t>(c.txt_dim) * 2);
+  amap(&w.a_Yall, w.Y, n, D, ldD);
+  amap(&w.a_Yout, w.Y, ni, D, ldD);                // output layer input: LN of the image rows
+  amap(&w.qkv, w.QKV, n, 3 * D, 3 * D * 2);
+  for (int sg = 0; sg < 3; ++sg) {
+    amap(&w.a_Yseg[sg], w.Y + row0[sg] * D, rows[sg], D, ldD);
+    amap(&w.a_CCseg[sg], w.CC + row0[sg] * (D + F), rows[sg], D + F, ldC);
+  }
+  if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an activation buffer");
+  if (rope_table_launch(w.rope, nt, gh, gw, refs, c.rope_theta, s) != cudaSuccess)
+    return fail(FLUX_EIO, "rope table launch failed");
+  w.nt = nt; w.gh = gh; w.gw = gw; w.refs = refs;
+  return FLUX_OK;
+}
+
+// Every modulation vector of one forward into m->mods (layout: kMod* offsets).
+int run_modulation3(flux3_dit* m, float t, float t_target, cudaStream_t s) {
+  const flux3_dit_config& c = m->cfg;
+  const int D = c.hidden, tf = c.t_freq_dim;
+  auto gv = [](double rows, double k, double nvec) { return rows * k * 2 + nvec * (rows * 6 + k * 4); };
+  float* mods = m->mods;
+  // embeddings of t (image tokens) and 0 (text and reference tokens), and of the target time
+  FD_LAUNCH(m, kProfOther, 0, tf * 4.0, timestep_embed_launch(m->temb, t, tf, s));
+  FD_LAUNCH(m, kProfOther, 0, tf * 4.0, timestep_embed_launch(m->temb + tf, 0.0f, tf, s));
+  FD_LAUNCH(m, kProfGemv, 4.0 * D * tf, gv(D, tf, 2),
+            gemv_multi_launch(m->t_w1, m->t_b1, m->temb, 2, m->th, nullptr, D, tf, 0, 1, s));
+  const float* add = nullptr;
+  if (c.flow_map) {
+    FD_LAUNCH(m, kProfOther, 0, tf * 4.0, timestep_embed_launch(m->temb + 2 * tf, t_target, tf, s));
+    FD_LAUNCH(m, kProfGemv, 2.0 * D * tf, gv(D, tf, 1),
+              gemv_multi_launch(m->g_w1, m->g_b1, m->temb + 2 * tf, 1, m->th + 2 * D, nullptr, D, tf, 0, 1, s));
+    FD_LAUNCH(m, kProfGemv, 2.0 * D * D, gv(D, D, 1),
+              gemv_multi_launch(m->g_w2, m->g_b2, m->th + 2 * D, 1, m->tt, nullptr, D, D, 0, 0, s));
+    add = m->tt;
+  }
+  // vec[0] = vec_img, vec[1] = vec_ctx
+  FD_LAUNCH(m, kProfGemv, 4.0 * D * D, gv(D, D, 2),
+            gemv_multi_launch(m->t_w2, m->t_b2, m->th, 2, m->vec, add, D, D, 0, 0, s));
+  const float* v_img = m->vec;
+  const float* v_ctx = m->vec + D;
+  const float* src[3] = {v_ctx, v_img, v_ctx};
+  const int dst[3] = {kModTxt, kModImg, kModRef};
+  for (int sidx = 0; sidx < 3; ++sidx)
+    FD_LAUNCH(m, kProfGemv, 6.0 * D * D, gv(3.0 * D, D, 1),
+              gemv_multi_launch(m->mode_mod_w[sidx], m->mode_mod_b[sidx], src[sidx], 1,
+                                mods + static_cast<size_t>(dst[sidx]) * D, nullptr, 3 * D, D, 1, 0, s));
+  // joint modulation on both vectors with one weight read: image set at kModJointImg, context set right after
+  FD_LAUNCH(m, kProfGemv, 12.0 * D * D, gv(3.0 * D, D, 2),
+            gemv_multi_launch(m->joint_mod_w, m->joint_mod_b, m->vec, 2,
+                              mods + static_cast<size_t>(kModJointImg) * D, nullptr, 3 * D, D, 1, 0, s));
+  FD_LAUNCH(m, kProfGemv, 4.0 * D * D, gv(2.0 * D, D, 1),
+            gemv_multi_launch(m->fin_mod_w, m->fin_mod_b, v_img, 1, mods + static_cast<size_t>(kModFinal) * D,
+                              nullptr, 2 * D, D, 1, 0, s));
+  return FLUX_OK;
+}
+
+int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const float* txt, int nt,
+                  const float* ref_tok, const RefGrids& refs, float t, float t_target, float* v_out, cudaStream_t s) {
+  const flux3_dit_config& c = m->cfg;
+  const int D = c.hidden, F = c.mlp_hidden, H = c.heads;
+  if (!img_tok || !v_out) return fail(FLUX_EINVAL, "img_tok and v_out must be device pointers");
+  if (nt > 0 && !txt) return fail(FLUX_EINVAL, "txt is NULL for %d text tokens", nt);
+  if (gh < 4 || gh > 64 || gw < 4 || gw > 64) return fail(FLUX_EINVAL, "image grid %dx%d outside 4..64", gh, gw);
+  if (nt < 0 || nt > 4096) return fail(FLUX_EINVAL, "bad text (n_txt=%d)", nt);
+  if (refs.count < 0 || refs.count > kMaxRefs)
+    return fail(FLUX_EINVAL, "%d reference images (at most %d)", refs.count, kMaxRefs);
+  for (int k = 0; k < refs.count; ++k)
+    if (refs.h[k] < 4 || refs.h[k] > 64 || refs.w[k] < 4 || refs.w[k] > 64)
+      return fail(FLUX_EINVAL, "reference %d grid %dx%d outside 4..64", k, refs.h[k], refs.w[k]);
+  if (refs.count > 0 && !ref_tok) return fail(FLUX_EINVAL, "ref_tok is NULL for %d reference(s)", refs.count);
+  if (!std::isfinite(t) || (c.flow_map && !std::isfinite(t_target)))
+    return fail(FLUX_EINVAL, "t (and, for the flow-map model, t_target) must be finite");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != m->device) return fail(FLUX_EINVAL, "model lives on device %d, current device is %d", m->device, dev);
+
+  int rc = prepare_shape3(m, nt, gh, gw, refs, s);
+  if (rc) return rc;
+  Workspace3& w = m->ws;
+  const int ni = gh * gw, nr = static_cast<int>(ref_tokens(refs)), n = nt + ni + nr;
+  const int row0[3] = {0, nt, nt + ni};
+  const int rows[3] = {nt, ni, nr};
+  const float eps_ln = c.eps_ln, eps_rms = c.eps_rms;
+  const float* mods = m->mods;
+  auto md = [&](int off) { return mods + static_cast<size_t>(off) * D; };
+
+  rc = run_modulation3(m, t, t_target, s);
+  if (rc) return rc;
+  FD_LAUNCH(m, kProfOther, 0, 6.0 * ni * c.in_ch,
+            cast_bf16_launch(img_tok, w.tokb, static_cast<size_t>(ni) * c.in_ch, s));
+  if (nr)
+    FD_LAUNCH(m, kProfOther, 0, 6.0 * nr * c.in_ch,
+              cast_bf16_launch(ref_tok, w.tokb + static_cast<size_t>(ni) * c.in_ch,
+                               static_cast<size_t>(nr) * c.in_ch, s));
+  if (nt)
+    FD_LAUNCH(m, kProfOther, 0, 6.0 * nt * c.txt_dim,
+              cast_bf16_launch(txt, w.txtb, static_cast<size_t>(nt) * c.txt_dim, s));
+  const double ln_bytes = 6.0 * n * D + 16.0 * D;
+
+  GemmParams P;
+  P.num_problems = 2;
+  problem(P, 0, w.a_txtb, m->m_txt_in, nt, D, c.txt_dim, kEpiF32Bias, w.X, D, m->txt_b, nullptr);
+  problem(P, 1, w.a_tokb, m->m_img_in, ni + nr, D, c.in_ch, kEpiF32Bias, w.X + static_cast<size_t>(nt) * D, D,
+          m->img_b, nullptr);
+  FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+
+  AttnParams A;
+  A.mapQ = w.qkv; A.mapK = w.qkv; A.mapV = w.qkv;
+  A.out = w.CC; A.ldo = D + F; A.heads = H; A.batch = 1;
+  A.q_col0 = 0; A.k_col0 = D; A.v_col0 = 2 * D;
+  A.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
+
+  // ---------------- per-mode blocks: each stream with its own weights, attention within the stream
+  AttnParams As = A;
+  As.nseg = 3;
+  double seg_flops = 0;
+  for (int sg = 0; sg < 3; ++sg) {
+    As.seg_row0[sg] = row0[sg];
+    As.seg_n[sg] = rows[sg];
+    seg_flops += 4.0 * rows[sg] * static_cast<double>(rows[sg]) * D;
+  }
+  const int mode_set[3] = {kModTxt, kModImg, kModRef};
+  for (int i = 0; i < m->act_mode; ++i) {
+    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes,
+              ln_modulate3_launch(w.X, w.Y, n, D, nt, nt + ni, n, md(kModTxt), md(kModTxt + 1), md(kModImg),
+                                  md(kModImg + 1), md(kModRef), md(kModRef + 1), eps_ln, s));
+    P.num_problems = 6;
+    for (int sg = 0; sg < 3; ++sg) {
+      const BlockW3& bw = m->mode[3 * i + sg];
+      problem(P, 2 * sg, w.a_Yseg[sg], bw.m_qkv, rows[sg], 3 * D, D, kEpiBf16Bias,
+              w.QKV + static_cast<size_t>(row0[sg]) * 3 * D, 3 * D, bw.qkv_b, nullptr);
+      qk_fuse(P, 2 * sg, bw.q_gain, bw.k_gain, w.rope, row0[sg], eps_rms);
+      problem(P, 2 * sg + 1, w.a_Yseg[sg], bw.m_mlp, rows[sg], 2 * F, D, kEpiSwiGLU,
+              w.CC + static_cast<size_t>(row0[sg]) * (D + F) + D, D + F, bw.mlp_b, nullptr);
+    }
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+    FD_LAUNCH(m, kProfAttention, seg_flops, 8.0 * n * D, attention_launch(As, s));
+    P.num_problems = 3;
+    for (int sg = 0; sg < 3; ++sg) {
+      const BlockW3& bw = m->mode[3 * i + sg];
+      problem(P, sg, w.a_CCseg[sg], bw.m_lin2, rows[sg], D, D + F, kEpiResidGate,
+              w.X + static_cast<size_t>(row0[sg]) * D, D, bw.lin2_b, md(mode_set[sg] + 2));
+    }
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+  }
+
+  // ---------------- joint blocks: one weight set, attention over the whole sequence, modulation per token type
+  const int joint_set[3] = {kModJointCtx, kModJointImg, kModJointCtx};
+  const double at_flops = 4.0 * n * static_cast<double>(n) * D;
+  for (int i = 0; i < m->act_joint; ++i) {
+    const BlockW3& bw = m->joint[i];
+    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes,
+              ln_modulate3_launch(w.X, w.Y, n, D, nt, nt + ni, n, md(kModJointCtx), md(kModJointCtx + 1),
+                                  md(kModJointImg), md(kModJointImg + 1), md(kModJointCtx), md(kModJointCtx + 1),
+                                  eps_ln, s));
+    P.num_problems = 2;
+    problem(P, 0, w.a_Yall, bw.m_qkv, n, 3 * D, D, kEpiBf16Bias, w.QKV, 3 * D, bw.qkv_b, nullptr);
+    qk_fuse(P, 0, bw.q_gain, bw.k_gain, w.rope, 0, eps_rms);
+    problem(P, 1, w.a_Yall, bw.m_mlp, n, 2 * F, D, kEpiSwiGLU, w.CC + D, D + F, bw.mlp_b, nullptr);
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+    A.n = n;
+    FD_LAUNCH(m, kProfAttention, at_flops, 8.0 * n * D, attention_launch(A, s));
+    P.num_problems = 3;
+    for (int sg = 0; sg < 3; ++sg)
+      problem(P, sg, w.a_CCseg[sg], bw.m_lin2, rows[sg], D, D + F, kEpiResidGate,
+              w.X + static_cast<size_t>(row0[sg]) * D, D, bw.lin2_b, md(joint_set[sg] + 2));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+  }
+
+  // ---------------- output layer on the image rows (text and reference tokens are dropped)
+  FD_LAUNCH(m, kProfLnMod, 0, 6.0 * ni * D + 8.0 * D,
+            ln_modulate_launch(w.X + static_cast<size_t>(nt) * D, w.Y, ni, D, ni, ni, md(kModFinal),
+                               md(kModFinal + 1), md(kModFinal), md(kModFinal + 1), eps_ln, s));
+  P.num_problems = 1;
+  problem(P, 0, w.a_Yout, m->m_fin, ni, c.in_ch, D, kEpiF32Bias, v_out, c.in_ch, m->fin_b, nullptr);
+  FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 128, m->num_sms, s));
+  return FLUX_OK;
+}
+
+int read_ref_grids(int n_refs, const int* ref_grids, RefGrids* refs) {
+  if (n_refs < 0 || n_refs > kMaxRefs) return fail(FLUX_EINVAL, "%d reference images (at most %d)", n_refs, kMaxRefs);
+  if (n_refs > 0 && !ref_grids) return fail(FLUX_EINVAL, "ref_grids is NULL");
+  refs->count = n_refs;
+  for (int k = 0; k < n_refs; ++k) {
+    refs->h[k] = ref_grids[2 * k];
+    refs->w[k] = ref_grids[2 * k + 1];
+  }
+  return FLUX_OK;
+}
+
+}  // namespace
+}  // namespace fdit
+
+using namespace fdit;
+
+// ====================================================================== C ABI
+extern "C" {
+
+size_t flux3_blob_expected_bytes(const flux3_dit_config* cfg) {
+  if (!cfg || !valid_cfg3(*cfg)) return 0;
+  size_t total = 0;
+  blob_tensors3(*cfg, &total);
+  return total;
+}
+
+flux3_dit* flux3_dit_create(const void* blob, size_t blob_bytes, const flux3_dit_config* cfg, void* stream) {
+  flux3_dit* m = nullptr;
+  create3_impl(blob, blob_bytes, cfg, static_cast<cudaStream_t>(stream), &m);
+  return m;
+}
+
+void flux3_dit_destroy(flux3_dit* m) { destroy3(m); }
+
+int flux3_dit_forward(flux3_dit* m, const float* img_tok, int grid_h, int grid_w, const float* txt, int n_txt,
+                      const float* ref_tok, int n_refs, const int* ref_grids, float t, float t_target, float* v_out,
+                      void* stream) {
+  if (!m) return fail(FLUX_EINVAL, "model is NULL");
+  RefGrids refs;
+  const int rc = read_ref_grids(n_refs, ref_grids, &refs);
+  if (rc) return rc;
+  return forward3_impl(m, img_tok, grid_h, grid_w, txt, n_txt, ref_tok, refs, t, t_target, v_out,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int flux3_dit_set_active_blocks(flux3_dit* m, int n_mode, int n_joint) {
+  if (!m) return fail(FLUX_EINVAL, "model is NULL");
+  m->act_mode = n_mode < 0 ? m->cfg.n_mode : std::min(n_mode, m->cfg.n_mode);
+  m->act_joint = n_joint < 0 ? m->cfg.n_joint : std::min(n_joint, m->cfg.n_joint);
+  return FLUX_OK;
+}
+
+size_t flux3_dit_modulation_size(const flux3_dit* m) {
+  return m ? static_cast<size_t>(kModRowsD) * m->cfg.hidden : 0;
+}
+
+int flux3_dit_modulation(flux3_dit* m, float t, float t_target, float* mods_out, void* stream) {
+  if (!m || !mods_out) return fail(FLUX_EINVAL, "NULL argument");
+  if (!std::isfinite(t) || (m->cfg.flow_map && !std::isfinite(t_target)))
+    return fail(FLUX_EINVAL, "t (and, for the flow-map model, t_target) must be finite");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int rc = run_modulation3(m, t, t_target, s);
+  if (rc) return rc;
+  FD_CUDA(cudaMemcpyAsync(mods_out, m->mods, flux3_dit_modulation_size(m) * sizeof(float),
+                          cudaMemcpyDeviceToDevice, s));
+  return FLUX_OK;
+}
+
+int flux3_dit_profile(flux3_dit* m, int enable) {
+  if (!m) return fail(FLUX_EINVAL, "model is NULL");
+  FD_CUDA(cudaDeviceSynchronize());
+  m->prof.reset();
+  m->prof.on = enable != 0;
+  return FLUX_OK;
+}
+
+int flux3_dit_profile_read(flux3_dit* m, int kind, double* ms, double* flops, double* bytes, long long* launches) {
+  if (!m || kind < 0 || kind >= kProfKinds) return fail(FLUX_EINVAL, "bad model or kernel kind");
+  FD_CUDA(cudaDeviceSynchronize());
+  m->prof.settle();
+  if (ms) *ms = m->prof.ms[kind];
+  if (flops) *flops = m->prof.flops[kind];
+  if (bytes) *bytes = m->prof.bytes[kind];
+  if (launches) *launches = m->prof.launches[kind];
+  return FLUX_OK;
+}
+
+int flux_joint_attention_segments(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o, int n_seg,
+                                  const int* seg_len, int heads, int head_dim, float scale, void* stream) {
+  if (!q || !k || !v || !o || !seg_len) return fail(FLUX_EINVAL, "NULL argument");
+  if (head_dim != 128) return fail(FLUX_EINVAL, "head_dim must be 128 (got %d)", head_dim);
+  if (n_seg < 1 || n_seg > kMaxSegs) return fail(FLUX_EINVAL, "n_seg=%d outside 1..%d", n_seg, kMaxSegs);
+  if (heads < 1 || heads > 1024) return fail(FLUX_EINVAL, "bad heads=%d", heads);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(FLUX_EINVAL, "q, k, v, o must be 16-byte aligned");
+  if (!(scale > 0) || !std::isfinite(scale)) return fail(FLUX_EINVAL, "scale must be positive");
+  AttnParams A;
+  A.nseg = n_seg;
+  long long rows = 0;
+  for (int z = 0; z < n_seg; ++z) {
+    if (seg_len[z] < 0) return fail(FLUX_EINVAL, "segment %d has negative length", z);
+    A.seg_row0[z] = static_cast<int>(rows);
+    A.seg_n[z] = seg_len[z];
+    rows += seg_len[z];
+    if (rows > (1ll << 31) - 1) return fail(FLUX_EINVAL, "segments too long");
+  }
+  if (rows == 0) return FLUX_OK;
+  const uint64_t ld = static_cast<uint64_t>(heads) * 128;
+  if (!make_tmap_bf16(&A.mapQ, q, rows, ld, ld * 2, 128) || !make_tmap_bf16(&A.mapK, k, rows, ld, ld * 2, 128) ||
+      !make_tmap_bf16(&A.mapV, v, rows, ld, ld * 2, 128))
+    return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed");
+  A.out = reinterpret_cast<bf16*>(o);
+  A.ldo = static_cast<int>(ld);
+  A.n = 0;
+  A.heads = heads;
+  A.batch = 1;
+  A.q_col0 = A.k_col0 = A.v_col0 = 0;
+  A.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
+  FD_CUDA(attention_launch(A, static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+}  // extern "C"

@@ -11,7 +11,7 @@ namespace fdit {
 
 // ------------------------------------------------------------------ GEMM
 enum EpiMode : int { kEpiBf16Bias = 0, kEpiF32Bias = 1, kEpiSwiGLU = 2, kEpiResidGate = 3, kEpiQKNormRope = 4 };
-constexpr int kMaxProblems = 4;
+constexpr int kMaxProblems = 6;
 
 struct GemmProblem {
   int M, N, K;                    // out rows, W rows, reduction (K % 64 == 0, N % 32 == 0)
@@ -47,6 +47,7 @@ cudaError_t gemm2_launch(GemmParams& P, int num_sms, cudaStream_t stream);
 int gemm2_read_device_error(cudaStream_t stream);
 
 // ------------------------------------------------------------------ attention
+constexpr int kMaxSegs = 4;       // independent segments of one attention launch
 struct AttnParams {
   CUtensorMap mapQ, mapK, mapV;   // 2D bf16 [rows = n, cols], box {64, 128}, 128B swizzle
   __nv_bfloat16* out;             // O row i, head h at out + i*ldo + h*128
@@ -55,6 +56,10 @@ struct AttnParams {
   int batch;                      // sequences of n rows each, one after another (grid.z)
   int q_col0, k_col0, v_col0;     // column of head 0's first element in each map
   float scale_log2;               // softmax scale * log2(e)
+  // nseg > 0 replaces the batch: grid.z = segment, segment z is rows [seg_row0[z], +seg_n[z]) and
+  // attends only to itself (n and batch are then ignored)
+  int nseg = 0;
+  int seg_row0[kMaxSegs], seg_n[kMaxSegs];
 };
 cudaError_t attention_launch(const AttnParams& P, cudaStream_t stream);
 int attention_read_device_error(cudaStream_t stream);
@@ -73,6 +78,12 @@ cudaError_t cast_bf16_launch(const float* x, __nv_bfloat16* y, size_t n, cudaStr
 cudaError_t ln_modulate_launch(const float* x, __nv_bfloat16* y, int rows, int dim, int split, int period,
                                const float* shift0, const float* scale0, const float* shift1,
                                const float* scale1, float eps, cudaStream_t s);
+// Three row regions: r % period in [0, split) set 0, [split, split2) set 1, [split2, period) set 2
+// (FLUX.3 per-token-type modulation: text | image | reference).
+cudaError_t ln_modulate3_launch(const float* x, __nv_bfloat16* y, int rows, int dim, int split, int split2,
+                                int period, const float* shift0, const float* scale0, const float* shift1,
+                                const float* scale1, const float* shift2, const float* scale2, float eps,
+                                cudaStream_t s);
 
 // In place on q (columns [0, heads*hd)) and k (columns [kcol, kcol + heads*hd)) of a [rows, ld] bf16 buffer:
 // RMSNorm over each head's hd values with gain (rows < split: gq0/gk0, else gq1/gk1), then RoPE from
@@ -102,6 +113,10 @@ cudaError_t timestep_embed_launch(float* temb, float t, int dim, cudaStream_t s)
 // y[r] = act_out(sum_k W[r,k] * act_in(x[k]) + b[r]); W bf16 [rows, k], b bf16 [rows]
 cudaError_t gemv_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, const float* x, float* y, int rows,
                         int k, int silu_in, int silu_out, cudaStream_t s);
+// nvec (1 or 2) input vectors of k floats, one after another, against one read of W: output v is
+// y[v * rows .. v * rows + rows); add (NULL or [rows]) is added before act_out.  nvec * k <= 12288.
+cudaError_t gemv_multi_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, const float* x, int nvec, float* y,
+                              const float* add, int rows, int k, int silu_in, int silu_out, cudaStream_t s);
 
 // ------------------------------------------------------------------ host helpers
 // Record `msg` as the calling thread's flux_get_error() message and return `code`.

@@ -1,0 +1,168 @@
+// Host-side pieces shared by the model runners (fluxdit.cu: FLUX.2-klein, fluxdit3.cu: FLUX.3
+// Image Klein): error recording, the per-launch profiler, the launch macro and grouped-GEMM
+// problem set-up.  Internal; not exported.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/fluxdit.h"
+#include "fluxdit_internal.h"
+
+namespace fdit {
+
+using bf16 = __nv_bfloat16;
+
+// printf-style flux_get_error() message for the calling thread; returns `code`.
+int fail(int code, const char* fmt, ...);
+const char* last_error();
+
+#define FD_CUDA(expr)                                                                          \
+  do {                                                                                         \
+    cudaError_t e_ = (expr);                                                                   \
+    if (e_ != cudaSuccess) return fail(FLUX_EIO, "%s: %s", #expr, cudaGetErrorString(e_));     \
+  } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// ------------------------------------------------------------------ per-kernel profiling
+// When enabled, every launch of a forward is bracketed by two CUDA events on its
+// stream; settle() (after a device synchronisation) accumulates the elapsed time
+// per kernel kind together with the launch's algorithmic FLOPs and HBM bytes.
+enum ProfKind { kProfGemm = 0, kProfAttention, kProfLnMod, kProfQkNormRope, kProfGemv, kProfOther, kProfKinds };
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+  double flops, bytes;
+};
+struct Profiler {
+  bool on = false;
+  std::vector<cudaEvent_t> pool;
+  std::vector<ProfRec> pending;
+  double ms[kProfKinds] = {}, flops[kProfKinds] = {}, bytes[kProfKinds] = {};
+  long long launches[kProfKinds] = {};
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+  void settle() {
+    for (const ProfRec& r : pending) {
+      float t = 0.f;
+      if (cudaEventElapsedTime(&t, r.a, r.b) == cudaSuccess) {
+        ms[r.kind] += t;
+        flops[r.kind] += r.flops;
+        bytes[r.kind] += r.bytes;
+        launches[r.kind] += 1;
+      }
+      pool.push_back(r.a);
+      pool.push_back(r.b);
+    }
+    pending.clear();
+  }
+  void reset() {
+    settle();
+    for (int k = 0; k < kProfKinds; ++k) ms[k] = flops[k] = bytes[k] = 0, launches[k] = 0;
+  }
+  ~Profiler() {
+    settle();
+    for (cudaEvent_t e : pool) cudaEventDestroy(e);
+  }
+};
+
+inline double gemm_flops(const GemmParams& P) {
+  double f = 0;
+  for (int i = 0; i < P.num_problems; ++i)
+    if (P.prob[i].M > 0) f += 2.0 * P.prob[i].M * static_cast<double>(P.prob[i].N) * P.prob[i].K;
+  return f;
+}
+inline double gemm_bytes(const GemmParams& P) {
+  double b = 0;
+  for (int i = 0; i < P.num_problems; ++i) {
+    const GemmProblem& pr = P.prob[i];
+    if (pr.M <= 0) continue;
+    const double out_elt = pr.mode == kEpiBf16Bias ? 2 : pr.mode == kEpiSwiGLU ? 1 : pr.mode == kEpiF32Bias ? 4 : 8;
+    b += 2.0 * pr.M * pr.K + 2.0 * pr.N * pr.K + out_elt * pr.M * pr.N;
+  }
+  return b;
+}
+
+// Enqueue `expr` (a launch returning cudaError_t) on stream `s`; bracket it with profiling events
+// when (m)->prof is enabled.
+#define FD_LAUNCH(m, kind, fl, by, expr)                                                   \
+  do {                                                                                     \
+    cudaEvent_t ea_ = nullptr, eb_ = nullptr;                                              \
+    if ((m)->prof.on) {                                                                    \
+      ea_ = (m)->prof.get();                                                               \
+      eb_ = (m)->prof.get();                                                               \
+      cudaEventRecord(ea_, s);                                                             \
+    }                                                                                      \
+    FD_CUDA(expr);                                                                         \
+    if ((m)->prof.on) {                                                                    \
+      cudaEventRecord(eb_, s);                                                             \
+      (m)->prof.pending.push_back({(kind), ea_, eb_, (fl), (by)});                         \
+    }                                                                                      \
+  } while (0)
+
+inline void problem(GemmParams& P, int i, const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, int mode,
+                    void* out, int ldo, const bf16* bias, const float* gate) {
+  P.mapA[i] = a;
+  P.mapB[i] = b;
+  GemmProblem& pr = P.prob[i];
+  pr = GemmProblem();
+  pr.M = M; pr.N = N; pr.K = K; pr.mode = mode; pr.out = out; pr.ldo = ldo; pr.bias = bias; pr.gate = gate;
+}
+
+// Make problem i a fused qkv + QK-RMSNorm + RoPE projection (rows start at token rope_row0).
+inline void qk_fuse(GemmParams& P, int i, const bf16* gq, const bf16* gk, const float2* rope, int rope_row0,
+                    float eps) {
+  GemmProblem& pr = P.prob[i];
+  pr.mode = kEpiQKNormRope;
+  pr.gain_q = gq;
+  pr.gain_k = gk;
+  pr.rope = rope;
+  pr.rope_row0 = rope_row0;
+  pr.eps = eps;
+}
+
+// Grow a device buffer to `need` elements (contents are not kept).
+template <typename T>
+cudaError_t grow(T** p, size_t* cap, size_t need) {
+  if (need <= *cap) return cudaSuccess;
+  cudaFree(*p);
+  *p = nullptr;
+  *cap = 0;
+  cudaError_t e = cudaMalloc(p, need * sizeof(T));
+  if (e == cudaSuccess) *cap = need;
+  return e;
+}
+
+inline size_t ref_tokens(const RefGrids& r) {
+  size_t n = 0;
+  for (int k = 0; k < r.count; ++k) n += static_cast<size_t>(r.h[k]) * r.w[k];
+  return n;
+}
+
+inline bool same_refs(const RefGrids& a, const RefGrids& b) {
+  if (a.count != b.count) return false;
+  for (int k = 0; k < a.count; ++k)
+    if (a.h[k] != b.h[k] || a.w[k] != b.w[k]) return false;
+  return true;
+}
+
+// Host -> device copy of SwiGLU rows [a (F rows); b (F rows)] of width `row_bytes` into the GEMM
+// order: for each group of 128 output columns, its 128 a-rows then its 128 b-rows.
+cudaError_t copy_swiglu(void* dst, const uint8_t* src, size_t F, size_t row_bytes, cudaStream_t s);
+
+// Device error words of the tcgen05 kernels (synchronises `s`): 0, or the first nonzero code.
+int device_error_words(cudaStream_t s);
+
+}  // namespace fdit

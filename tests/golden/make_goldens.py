@@ -10,6 +10,10 @@ step's velocity and the final packed latent:
 Row sets: all rows at 256^2, every 2nd at 512^2, every 8th at 1024^2.  For a guided workload
 the stored velocities are the guided ones.
 
+FLUX.3 workloads (``f3*``) use the FLUX.3 oracle with the flow-map target time t_{i+1}; the
+8272-token image-to-image case runs the first STEPS_RUN steps of its 16-step schedule (``v`` then
+holds those steps and ``final`` the packed state after them, ``meta.steps_run`` says how many).
+
 Usage: python tests/golden/make_goldens.py [workload ...]   (about an hour on 8 cores)
 """
 import json
@@ -25,8 +29,11 @@ sys.path.insert(0, os.path.dirname(os.path.dirname(HERE)))
 
 from synthetic import WORKLOADS, make_weights, make_inputs, make_uncond_text  # noqa: E402
 from oracle import flux_oracle as O  # noqa: E402
+from oracle import flux3_oracle as O3  # noqa: E402
 
-ROW_STRIDE = {"t2i256": 1, "t2i512": 2, "t2i1024": 8, "i2i1024": 8, "mref1024": 8, "cfg256": 1}
+ROW_STRIDE = {"t2i256": 1, "t2i512": 2, "t2i1024": 8, "i2i1024": 8, "mref1024": 8, "cfg256": 1,
+              "f3t2i256": 1, "f3i2i256": 1, "f3t2i1024": 8, "f3i2i1024": 8}
+STEPS_RUN = {"f3i2i1024": 4}
 
 
 def rows_for(name):
@@ -34,7 +41,38 @@ def rows_for(name):
     return np.arange(0, w.n_img, ROW_STRIDE[name], dtype=np.int32)
 
 
+def make3(name):
+    """FLUX.3 sampler: forward3 with target time t_{i+1}, Euler update, for the first k steps."""
+    w = WORKLOADS[name]
+    t0 = time.time()
+    _, p = make_weights(w.dims, w.seed)
+    lat, txt, ref = make_inputs(w)
+    rows = rows_for(name)
+    k = STEPS_RUN.get(name, w.n_steps)
+    hp = O.hyper(w.dims)
+    ts = O.schedule(w.n_steps)
+    tok = O.pack_latents(torch.from_numpy(lat)).float()
+    refs = [] if ref is None else (ref if isinstance(ref, list) else [ref])
+    ref_toks = [O.pack_latents(torch.from_numpy(r)).float() for r in refs]
+    ref_grids = [(r.shape[1] // 2, r.shape[2] // 2) for r in refs]
+    vs = []
+    for i in range(k):
+        v = O3.forward3(p, hp, tok, torch.from_numpy(txt), ts[i], (w.grid, w.grid), ref_toks, ref_grids,
+                        t_target=ts[i + 1] if w.dims.flow_map else None, dtype=torch.float32)
+        vs.append(v[rows].float().numpy())
+        tok = O.euler_update(tok, v, ts[i + 1] - ts[i])
+        print(f"  {name} step {i} done at {time.time() - t0:.0f}s", flush=True)
+    meta = {"workload": name, "seed": w.seed, "oracle_dtype": "float32", "n_steps": w.n_steps, "steps_run": k,
+            "flow_map": bool(w.dims.flow_map), "row_stride": ROW_STRIDE[name],
+            "seconds": round(time.time() - t0, 1)}
+    np.savez(os.path.join(HERE, f"{name}.npz"), rows=rows, v=np.stack(vs), final=tok[rows].float().numpy(),
+             meta=np.array(json.dumps(meta)))
+    print(f"{name}: wrote {len(rows)} rows x {k} steps in {time.time() - t0:.0f}s", flush=True)
+
+
 def make(name):
+    if name.startswith("f3"):
+        return make3(name)
     w = WORKLOADS[name]
     t0 = time.time()
     _, p = make_weights(w.dims, w.seed)

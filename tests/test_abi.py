@@ -11,7 +11,7 @@ import pytest
 
 import latent_flow_matching_b200 as F
 from latent_flow_matching_b200 import build as fbuild
-from synthetic import FluxDims, FULL_DIMS, TINY_DIMS, blob_layout
+from synthetic import FluxDims, Flux3Dims, FULL_DIMS, TINY_DIMS, F3_FULL_DIMS, F3_TINY_DIMS, blob_layout
 from synthetic.flux_inputs import HEADER_BYTES
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -26,7 +26,7 @@ def L():
 
 def declared_symbols():
     src = open(HEADER).read()
-    return sorted(set(re.findall(r"FLUX_API\s+[\w\s\*]*?\b(flux_\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"FLUX_API\s+[\w\s\*]*?\b(flux3?_\w+)\s*\(", src)))
 
 
 def test_header_declares_the_boundary():
@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol(L):
     for name in declared_symbols():
         assert hasattr(L, name), name
     out = subprocess.run(["nm", "-D", "--defined-only", F.LIB_PATH], capture_output=True, text=True).stdout
-    exported = set(re.findall(r"\bT (flux_\w+)", out))
+    exported = set(re.findall(r"\bT (flux3?_\w+)", out))
     assert set(declared_symbols()) <= exported
     assert set(F.EXPORTED) == set(declared_symbols())
 
@@ -133,3 +133,60 @@ def test_product_path_does_not_reference_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert "oracle" not in src, f
+
+
+# ---------------------------------------------------------------------------- FLUX.3 entry points
+MICRO3 = Flux3Dims(n_mode=1, n_joint=2, hidden=256, heads=2, mlp_hidden=256, txt_dim=192, t_freq_dim=256,
+                   flow_map=False)
+
+
+@pytest.mark.parametrize("dims", [F3_FULL_DIMS, F3_TINY_DIMS, MICRO3])
+def test_flux3_blob_size_matches_generator(L, dims):
+    _, total = blob_layout(dims)
+    assert F.flux3_blob_expected_bytes(dims) == total
+
+
+def test_flux3_invalid_config_gives_zero(L):
+    assert F.flux3_blob_expected_bytes(Flux3Dims(heads=3, hidden=384)) == 0          # odd head count
+    assert F.flux3_blob_expected_bytes(Flux3Dims(flow_map=2)) == 0
+
+
+def _micro3_blob():
+    from synthetic.flux_inputs import _header
+    from synthetic import tensor_specs
+    _, total = blob_layout(MICRO3)
+    blob = np.zeros(total, np.uint8)
+    blob[:HEADER_BYTES] = np.frombuffer(_header(MICRO3, len(tensor_specs(MICRO3)), total), np.uint8)
+    return blob
+
+
+def test_flux3_create_rejects_corrupt_blob_and_mismatch(L):
+    blob = _micro3_blob()
+    bad = blob.copy()
+    bad[3] = ord("Z")
+    assert not L.flux3_dit_create(ctypes.c_void_p(bad.ctypes.data), bad.nbytes, None, None)
+    assert "FLUX3DT" in F.get_error()
+    assert not L.flux3_dit_create(ctypes.c_void_p(blob.ctypes.data), blob.nbytes - 512, None, None)
+    assert "size" in F.get_error()
+    other = F.Flux3Config.from_dims(Flux3Dims(n_mode=2, n_joint=2, hidden=256, heads=2, mlp_hidden=256,
+                                              txt_dim=192, flow_map=False))
+    assert not L.flux3_dit_create(ctypes.c_void_p(blob.ctypes.data), blob.nbytes, ctypes.byref(other), None)
+    assert "config" in F.get_error()
+    # a FLUX.2 blob is not a FLUX.3 blob and the other way round
+    assert not L.flux_dit_create(ctypes.c_void_p(blob.ctypes.data), blob.nbytes, None, None)
+
+
+def test_flux3_entry_points_reject_bad_arguments(L):
+    p = ctypes.c_void_p(16)            # never dereferenced: validation fails first
+    lens = (ctypes.c_int * 3)(4, 5, 6)
+    assert L.flux_joint_attention_segments(p, p, p, p, 0, lens, 2, 128, 0.1, None) == F.FLUX_EINVAL
+    assert L.flux_joint_attention_segments(p, p, p, p, 5, lens, 2, 128, 0.1, None) == F.FLUX_EINVAL
+    assert L.flux_joint_attention_segments(p, p, p, p, 3, lens, 2, 64, 0.1, None) == F.FLUX_EINVAL
+    assert "head_dim" in F.get_error()
+    neg = (ctypes.c_int * 2)(4, -1)
+    assert L.flux_joint_attention_segments(p, p, p, p, 2, neg, 2, 128, 0.1, None) == F.FLUX_EINVAL
+    assert L.flux_joint_attention_segments(p, p, p, p, 2, None, 2, 128, 0.1, None) == F.FLUX_EINVAL
+    assert L.flux3_dit_forward(None, p, 8, 8, p, 4, None, 0, None, 1.0, 0.5, p, None) == F.FLUX_EINVAL
+    assert L.flux3_dit_set_active_blocks(None, 1, 1) == F.FLUX_EINVAL
+    assert L.flux3_dit_modulation_size(None) == 0
+    L.flux3_dit_destroy(None)

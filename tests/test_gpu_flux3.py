@@ -1,0 +1,238 @@
+"""FLUX.3 Image Klein on the GPU (through the C ABI) against the FLUX.3 CPU oracle.
+
+Bars as for FLUX.2: velocity relative L2 <= 2e-2 per step, final latent <= 3e-2, modulation
+and attention normalised max error <= 1e-2.
+* segmented attention (the per-mode blocks' stream-local attention): bit-identical to one call
+  per segment, and against the oracle's attention per segment;
+* the tiny model (1 per-mode + 1 joint block, full width): live float64 oracle, block by block,
+  ragged and degenerate shapes, several references, the flow-map sampler;
+* 256^2 and 1024^2 workloads (+ a reference): the oracle's sampled rows, written by
+  tests/golden/make_goldens.py (oracle only).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import latent_flow_matching_b200 as F
+from oracle import flux_oracle as O
+from oracle import flux3_oracle as O3
+from synthetic import WORKLOADS, make_weights, make_inputs
+
+pytestmark = pytest.mark.gpu
+torch.set_grad_enabled(False)
+DEV = "cuda"
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+V_TOL, X_TOL, K_TOL = 2e-2, 3e-2, 1e-2
+
+
+def rel_l2(a, b):
+    a = torch.as_tensor(a).double().cpu()
+    b = torch.as_tensor(b).double().cpu()
+    return ((a - b).norm() / b.norm()).item()
+
+
+def nmax(a, b):
+    a = torch.as_tensor(a).double().cpu()
+    b = torch.as_tensor(b).double().cpu()
+    return ((a - b).abs().max() / b.abs().max()).item()
+
+
+def bf16r(x):
+    return x.to(torch.bfloat16).float()
+
+
+# ---------------------------------------------------------------------------- segmented attention
+@pytest.mark.parametrize("seg_len", [[37, 300, 0, 129], [160, 256], [1, 1, 1], [513]])
+def test_segment_attention_matches_per_segment_calls_and_oracle(seg_len):
+    g = torch.Generator().manual_seed(sum(seg_len))
+    heads = 4
+    rows = sum(seg_len)
+    q, k, v = (torch.randn(rows, heads, 128, generator=g).to(torch.bfloat16) for _ in range(3))
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    o = torch.empty_like(qd)
+    F.flux_joint_attention_segments(qd, kd, vd, o, seg_len)
+    r0 = 0
+    for n in seg_len:
+        if n:
+            sl = slice(r0, r0 + n)
+            one = torch.empty(n, heads, 128, dtype=torch.bfloat16, device=DEV)
+            F.flux_joint_attention(qd[sl].contiguous(), kd[sl].contiguous(), vd[sl].contiguous(), one)
+            assert torch.equal(one, o[sl]), (n, r0)
+            want = O.attention(q[sl].double(), k[sl].double(), v[sl].double())
+            assert nmax(o[sl].float(), want) <= K_TOL
+        r0 += n
+    assert F.flux_device_error() == 0
+
+
+# ---------------------------------------------------------------------------- tiny model, live oracle
+@pytest.fixture(scope="module")
+def tiny3():
+    w = WORKLOADS["f3tiny64"]
+    blob, p = make_weights(w.dims, w.seed)
+    model = F.Flux3DiT(blob, w.dims)
+    yield w, p, model
+    model.close()
+
+
+def _mods_ref(p, t, t_target):
+    D = p["time_in.w2"].shape[0]
+    f64 = torch.float64
+    s_img = O.silu(O3.time_vector(p, t, t_target, f64))
+    s_ctx = O.silu(O3.time_vector(p, 0.0, t_target, f64))
+
+    def lin(name, s):
+        return O.linear(s, O.weight(p, name + ".w", f64), O.weight(p, name + ".b", f64))
+    return torch.cat([lin("mode_mod.txt", s_ctx), lin("mode_mod.img", s_img), lin("mode_mod.ref", s_ctx),
+                      lin("joint_mod", s_img), lin("joint_mod", s_ctx), lin("final.mod", s_img)]), D
+
+
+@pytest.mark.parametrize("t,t_target", [(1.0, 0.75), (0.25, 0.0)])
+def test_tiny3_modulation_vectors(tiny3, t, t_target):
+    w, p, model = tiny3
+    out = torch.empty(model.modulation_size(), device=DEV)
+    model.modulation(t, t_target, out)
+    ref, D = _mods_ref(p, t, t_target)
+    assert out.numel() == ref.numel() == 17 * D
+    assert nmax(out, ref) <= K_TOL
+    # the context sets do not depend on t, the image sets do
+    out2 = torch.empty_like(out)
+    model.modulation(0.5 * t + 0.1, t_target, out2)
+    ctx = torch.cat([torch.arange(0, 3 * D), torch.arange(6 * D, 9 * D), torch.arange(12 * D, 15 * D)])
+    assert torch.equal(out[ctx], out2[ctx])
+    assert not torch.equal(out[3 * D:6 * D], out2[3 * D:6 * D])
+
+
+def _tiny_inputs(seed, nt, grid, ref_grids):
+    g = torch.Generator().manual_seed(seed)
+    tok = bf16r(torch.randn(grid[0] * grid[1], 128, generator=g))
+    txt = bf16r(torch.randn(nt, 20480, generator=g))
+    refs = [bf16r(torch.randn(h * w_, 128, generator=g)) for h, w_ in ref_grids]
+    return tok, txt, refs
+
+
+def _gpu_forward(model, tok, grid, txt, t, refs, ref_grids, t_target):
+    v = torch.empty(grid[0] * grid[1], 128, device=DEV)
+    ref_tok = torch.cat(refs).to(DEV) if refs else None
+    model.forward(tok.to(DEV), grid, txt.to(DEV) if txt.shape[0] else None, t, v, ref_tok, ref_grids,
+                  t_target=t_target)
+    return v
+
+
+@pytest.mark.parametrize("n_mode,n_joint", [(0, 0), (1, 0), (0, 1), (1, 1)])
+def test_tiny3_forward_block_by_block(tiny3, n_mode, n_joint):
+    w, p, model = tiny3
+    keep = {k: v for k, v in p.items()
+            if not ((k.startswith("mode.") and int(k.split(".")[1]) >= n_mode) or
+                    (k.startswith("joint.") and int(k.split(".")[1]) >= n_joint))}
+    tok, txt, refs = _tiny_inputs(3, 16, (4, 4), [(4, 4)])
+    want = O3.forward3(keep, O.hyper(w.dims), tok, txt, 0.75, (4, 4), refs, [(4, 4)], t_target=0.5)
+    model.set_active_blocks(n_mode, n_joint)
+    try:
+        v = _gpu_forward(model, tok, (4, 4), txt, 0.75, refs, [(4, 4)], 0.5)
+    finally:
+        model.set_active_blocks(-1, -1)
+    assert rel_l2(v, want) <= V_TOL
+    assert F.flux_device_error() == 0
+
+
+@pytest.mark.parametrize("nt,grid,ref_grids", [(0, (4, 6), []), (5, (6, 4), [(4, 4)]), (16, (4, 4), []),
+                                               (131, (8, 8), [(4, 8), (4, 4)]), (200, (12, 12), [(12, 12)])])
+def test_tiny3_forward_ragged_and_degenerate_shapes(tiny3, nt, grid, ref_grids):
+    """No text, no reference, several references, segments off the 128-row tiles and longer than one."""
+    w, p, model = tiny3
+    tok, txt, refs = _tiny_inputs(100 + nt, nt, grid, ref_grids)
+    want = O3.forward3(p, O.hyper(w.dims), tok, txt, 0.6, grid, refs, ref_grids, t_target=0.35)
+    v = _gpu_forward(model, tok, grid, txt, 0.6, refs, ref_grids, 0.35)
+    assert rel_l2(v, want) <= V_TOL
+    assert F.flux_device_error() == 0
+
+
+def test_tiny3_target_time_and_reference_order_matter(tiny3):
+    w, p, model = tiny3
+    tok, txt, refs = _tiny_inputs(9, 7, (4, 4), [(4, 4), (6, 4)])
+    grids = [(4, 4), (6, 4)]
+    a = _gpu_forward(model, tok, (4, 4), txt, 0.5, refs, grids, 0.25)
+    b = _gpu_forward(model, tok, (4, 4), txt, 0.5, refs, grids, 0.0)
+    c = _gpu_forward(model, tok, (4, 4), txt, 0.5, refs[::-1], grids[::-1], 0.25)
+    assert rel_l2(a, b) > 1e-3 and rel_l2(a, c) > 1e-3
+    want = O3.forward3(p, O.hyper(w.dims), tok, txt, 0.5, (4, 4), refs[::-1], grids[::-1], t_target=0.25)
+    assert rel_l2(c, want) <= V_TOL
+
+
+def test_tiny3_sampler_matches_oracle(tiny3):
+    """4 flow-map steps (target t_{i+1}) with a 64^2 reference: every velocity and the final latent."""
+    w, p, model = tiny3
+    lat, txt, ref = make_inputs(w)
+    ref_final, ref_vs = O3.sample3(p, O.hyper(w.dims), torch.from_numpy(lat), torch.from_numpy(txt), 4,
+                                   ref_latent=torch.from_numpy(ref))
+    vs = []
+    final = F.flux3_sample(model, torch.from_numpy(lat).to(DEV), torch.from_numpy(txt).to(DEV), 4,
+                           ref_latent=torch.from_numpy(ref).to(DEV), on_step=lambda i, v: vs.append(v.cpu().clone()))
+    assert len(vs) == 4
+    for i in range(4):
+        assert rel_l2(vs[i], ref_vs[i]) <= V_TOL, i
+    assert rel_l2(final.cpu(), ref_final) <= X_TOL
+    again = F.flux3_sample(model, torch.from_numpy(lat).to(DEV), torch.from_numpy(txt).to(DEV), 4,
+                           ref_latent=torch.from_numpy(ref).to(DEV))
+    assert torch.equal(final, again)                       # deterministic
+    assert F.flux_device_error() == 0
+
+
+def test_flux3_rejects_bad_arguments(tiny3):
+    w, p, model = tiny3
+    tok = torch.zeros(16, 128, device=DEV)
+    v = torch.empty(16, 128, device=DEV)
+    txt = torch.zeros(4, 20480, device=DEV)
+    with pytest.raises(F.FluxError):
+        model.forward(tok, (2, 8), txt, 1.0, v, t_target=0.5)
+    with pytest.raises(F.FluxError):
+        model.forward(tok, (4, 4), txt, 1.0, v, None, [(4, 4)], t_target=0.5)   # reference grid, no tokens
+    with pytest.raises(F.FluxError):
+        model.forward(tok, (4, 4), txt, 1.0, v, t_target=float("nan"))          # flow-map model needs t_target
+    with pytest.raises(F.FluxError):
+        model.forward(tok, (4, 4), txt, 1.0, v, torch.zeros(11 * 16, 128, device=DEV), [(4, 4)] * 11, t_target=0.5)
+
+
+# ---------------------------------------------------------------------------- full-size workloads vs goldens
+def _golden(name):
+    path = os.path.join(GOLDEN, f"{name}.npz")
+    if not os.path.exists(path):
+        pytest.skip(f"golden {path} not generated")
+    return np.load(path)
+
+
+@pytest.mark.parametrize("name", ["f3t2i256", "f3i2i256", "f3t2i1024", "f3i2i1024"])
+def test_flux3_workload_against_oracle_goldens(name):
+    gd = _golden(name)
+    w = WORKLOADS[name]
+    meta = json.loads(str(gd["meta"]))
+    assert meta["workload"] == name and meta["seed"] == w.seed
+    k = meta["steps_run"]
+    blob, _ = make_weights(w.dims, w.seed)
+    lat, txt, ref = make_inputs(w)
+    model = F.Flux3DiT(blob, w.dims)
+    del blob
+    try:
+        ts = F.euler_schedule(w.n_steps)
+        tok = torch.empty(w.n_img, 128, device=DEV)
+        F.flux_pack_latents(torch.from_numpy(lat).to(DEV), tok)
+        ref_tok, grids = None, []
+        if ref is not None:
+            ref_tok = O.pack_latents(torch.from_numpy(ref)).float().to(DEV)
+            grids = [(w.ref_grid, w.ref_grid)]
+        txt_d = torch.from_numpy(txt).to(DEV)
+        v = torch.empty_like(tok)
+        rows = torch.from_numpy(gd["rows"]).long()
+        for i in range(k):
+            model.forward(tok, (w.grid, w.grid), txt_d, ts[i], v, ref_tok, grids, t_target=ts[i + 1])
+            err = rel_l2(v.cpu()[rows], gd["v"][i])
+            assert err <= V_TOL, (i, err)
+            F.flux_euler_step(tok, v, ts[i + 1] - ts[i])
+        err = rel_l2(tok.cpu()[rows], gd["final"])
+        assert err <= X_TOL, err
+    finally:
+        model.close()
+    assert F.flux_device_error() == 0
