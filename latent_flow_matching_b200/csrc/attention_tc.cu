@@ -95,6 +95,9 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 // one score pair in kPolyEvery goes through ex2_poly2, the rest through MUFU ex2
 constexpr int kPolyEvery = 3;
 
+// kSegs: grid.z indexes P's segments (lengths read once from the parameter arrays); otherwise
+// grid.z is a batch index and the sequence length stays a constant-bank operand.
+template <bool kSegs>
 __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_constant__ AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -118,9 +121,9 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
   const int lane = threadIdx.x & 31;
   const int q0 = blockIdx.x * (kQTiles * kTile);      // first query row inside this sequence
   const int head = blockIdx.y;
-  const int n = P.nseg ? P.seg_n[blockIdx.z] : P.n;   // rows of this sequence
-  const int row_base = P.nseg ? P.seg_row0[blockIdx.z] : static_cast<int>(blockIdx.z) * P.n;
-  if (q0 >= n) return;                                 // whole CTA: nothing initialised yet
+  const int n = kSegs ? P.seg_n[blockIdx.z] : P.n;   // rows of this sequence
+  const int row_base = kSegs ? P.seg_row0[blockIdx.z] : static_cast<int>(blockIdx.z) * P.n;
+  if (kSegs && q0 >= n) return;                        // whole CTA: nothing initialised yet
   const int n_kv = (n + kTile - 1) / kTile;
 
   if (threadIdx.x == 0) {
@@ -402,7 +405,9 @@ cudaError_t attention_launch(const AttnParams& P, cudaStream_t stream) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e =
-        cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        cudaFuncSetAttribute(attention_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attention_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -419,7 +424,10 @@ cudaError_t attention_launch(const AttnParams& P, cudaStream_t stream) {
   if (n_max <= 0 || P.heads <= 0 || nz <= 0) return cudaSuccess;
   dim3 grid((n_max + kQTiles * kTile - 1) / (kQTiles * kTile), P.heads, nz);
   count_launch();
-  attention_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(P);
+  if (P.nseg)
+    attention_tc_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(P);
+  else
+    attention_tc_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(P);
   return cudaGetLastError();
 }
 

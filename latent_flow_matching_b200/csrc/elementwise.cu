@@ -87,10 +87,19 @@ __global__ void cast_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __r
 // One 256-thread CTA per row: each thread keeps VPT float4 of the row in registers (dim = 1024 VPT),
 // mean and variance come from two block reductions, so many CTAs stay resident per SM.
 // Row r uses modulation set 0 when r % period < split, set 1 when it is < split2, else set 2.
+// (Scalar members: a runtime index into a kernel-parameter array would copy it to the stack.)
 struct LnModSets {
   int split, split2, period;
-  const float* sh[3];
-  const float* sc[3];
+  const float *sh0, *sh1, *sh2;
+  const float *sc0, *sc1, *sc2;
+  __device__ __forceinline__ const float* shift(int row) const {
+    const int r = row % period;
+    return r < split ? sh0 : (r < split2 ? sh1 : sh2);
+  }
+  __device__ __forceinline__ const float* scale(int row) const {
+    const int r = row % period;
+    return r < split ? sc0 : (r < split2 ? sc1 : sc2);
+  }
 };
 
 template <int VPT>
@@ -130,10 +139,8 @@ __global__ void __launch_bounds__(256) ln_mod_kernel(const float* __restrict__ x
 #pragma unroll
   for (int w = 0; w < 8; ++w) q += red[1][w];
   const float rstd = rsqrtf(q * (1.0f / dim) + eps);
-  const int r = row % m.period;
-  const int set = r < m.split ? 0 : (r < m.split2 ? 1 : 2);
-  const float4* shp = reinterpret_cast<const float4*>(m.sh[set]);
-  const float4* scp = reinterpret_cast<const float4*>(m.sc[set]);
+  const float4* shp = reinterpret_cast<const float4*>(m.shift(row));
+  const float4* scp = reinterpret_cast<const float4*>(m.scale(row));
   uint2* yr = reinterpret_cast<uint2*>(y + static_cast<size_t>(row) * dim);
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
@@ -161,10 +168,8 @@ __global__ void ln_mod_generic_kernel(const float* __restrict__ x, __nv_bfloat16
   for (int i = lane; i < dim; i += 32) q += (xr[i] - mean) * (xr[i] - mean);
   for (int o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
   const float rstd = rsqrtf(q / dim + eps);
-  const int r = warp % m.period;
-  const int set = r < m.split ? 0 : (r < m.split2 ? 1 : 2);
-  const float* sh = m.sh[set];
-  const float* sc = m.sc[set];
+  const float* sh = m.shift(warp);
+  const float* sc = m.scale(warp);
   for (int i = lane; i < dim; i += 32)
     y[static_cast<size_t>(warp) * dim + i] = __float2bfloat16_rn((xr[i] - mean) * rstd * (1.f + sc[i]) + sh[i]);
 }
@@ -388,7 +393,7 @@ cudaError_t ln_modulate3_launch(const float* x, __nv_bfloat16* y, int rows, int 
                                 cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   if (period <= 0) return cudaErrorInvalidValue;
-  const LnModSets m = {split, split2, period, {shift0, shift1, shift2}, {scale0, scale1, scale2}};
+  const LnModSets m = {split, split2, period, shift0, shift1, shift2, scale0, scale1, scale2};
   count_launch();
   if (dim == 3072)
     ln_mod_kernel<3><<<rows, 256, 0, s>>>(x, y, rows, m, eps);
