@@ -60,6 +60,7 @@ __all__ = [
     "layer_norm", "rms_norm", "modulate", "silu", "linear", "attention_probs",
     "attention", "timestep_embedding", "double_block", "single_block", "forward",
     "schedule", "euler_update", "img2img_start", "blend_latents", "guided_velocity", "sample", "weight",
+    "block_linear",
 ]
 
 CPU = torch.device("cpu")
@@ -214,6 +215,15 @@ def timestep_embedding(t: float, dim: int = 256, max_period: float = 10000.0,
     return torch.cat([torch.cos(a), torch.sin(a)])
 
 
+def block_linear(hp):
+    """The linear layer used inside the transformer blocks: the plain definition, or the
+    row-wise FP8 one (``oracle/fp8_oracle.py``) when ``hp["fp8"]`` is set."""
+    if hp.get("fp8"):
+        from .fp8_oracle import linear_fp8
+        return linear_fp8
+    return linear
+
+
 def _heads(x, heads, head_dim):
     return x.reshape(x.shape[0], heads, head_dim)
 
@@ -224,18 +234,18 @@ def _pre_attention(p, prefix, x, s, hp, dtype):
     m = linear(s, weight(p, prefix + "mod.w", dtype), weight(p, prefix + "mod.b", dtype))
     sh1, sc1, g1, sh2, sc2, g2 = m.split(D)
     y = modulate(layer_norm(x, hp["eps_ln"]), sh1, sc1)
-    qkv = linear(y, weight(p, prefix + "qkv.w", dtype), weight(p, prefix + "qkv.b", dtype))
+    qkv = block_linear(hp)(y, weight(p, prefix + "qkv.w", dtype), weight(p, prefix + "qkv.b", dtype))
     q, k, v = (_heads(z, hp["heads"], hp["head_dim"]) for z in qkv.split(D, dim=1))
     q = rms_norm(q, weight(p, prefix + "q_gain", dtype), hp["eps_rms"])
     k = rms_norm(k, weight(p, prefix + "k_gain", dtype), hp["eps_rms"])
     return q, k, v, (g1, sh2, sc2, g2)
 
 
-def _mlp(p, prefix, y, dtype, lin_in="mlp_in", lin_out="mlp_out"):
-    h = linear(y, weight(p, prefix + lin_in + ".w", dtype), weight(p, prefix + lin_in + ".b", dtype))
+def _mlp(p, prefix, y, dtype, lin_in="mlp_in", lin_out="mlp_out", hp=None):
+    lin = block_linear(hp or {})
+    h = lin(y, weight(p, prefix + lin_in + ".w", dtype), weight(p, prefix + lin_in + ".b", dtype))
     a, b = h.chunk(2, dim=1)
-    return linear(silu(a) * b, weight(p, prefix + lin_out + ".w", dtype),
-                  weight(p, prefix + lin_out + ".b", dtype))
+    return lin(silu(a) * b, weight(p, prefix + lin_out + ".w", dtype), weight(p, prefix + lin_out + ".b", dtype))
 
 
 def double_block(p, i, x_txt, x_img, s, ang, hp, dtype=torch.float64):
@@ -250,9 +260,9 @@ def double_block(p, i, x_txt, x_img, s, ang, hp, dtype=torch.float64):
     nt = x_txt.shape[0]
     outs = []
     for x, o_s, (g1, sh2, sc2, g2), pre in ((x_txt, o[:nt], mt, pt), (x_img, o[nt:], mi, pi)):
-        x = x + g1 * linear(o_s, weight(p, pre + "proj.w", dtype), weight(p, pre + "proj.b", dtype))
+        x = x + g1 * block_linear(hp)(o_s, weight(p, pre + "proj.w", dtype), weight(p, pre + "proj.b", dtype))
         y = modulate(layer_norm(x, hp["eps_ln"]), sh2, sc2)
-        x = x + g2 * _mlp(p, pre, y, dtype)
+        x = x + g2 * _mlp(p, pre, y, dtype, hp=hp)
         outs.append(x)
     return outs[0], outs[1]
 
@@ -264,14 +274,14 @@ def single_block(p, i, x, s, ang, hp, dtype=torch.float64):
     F = (p[pre + "lin1.w"].shape[0] - 3 * D) // 2
     sh, sc, g = linear(s, weight(p, pre + "mod.w", dtype), weight(p, pre + "mod.b", dtype)).split(D)
     y = modulate(layer_norm(x, hp["eps_ln"]), sh, sc)
-    h = linear(y, weight(p, pre + "lin1.w", dtype), weight(p, pre + "lin1.b", dtype))
+    h = block_linear(hp)(y, weight(p, pre + "lin1.w", dtype), weight(p, pre + "lin1.b", dtype))
     q, k, v, a, b = h.split([D, D, D, F, F], dim=1)
     q = rms_norm(_heads(q, hp["heads"], hp["head_dim"]), weight(p, pre + "q_gain", dtype), hp["eps_rms"])
     k = rms_norm(_heads(k, hp["heads"], hp["head_dim"]), weight(p, pre + "k_gain", dtype), hp["eps_rms"])
     v = _heads(v, hp["heads"], hp["head_dim"])
     o = attention(apply_rope(q, ang), apply_rope(k, ang), v)
-    return x + g * linear(torch.cat([o, silu(a) * b], dim=1),
-                          weight(p, pre + "lin2.w", dtype), weight(p, pre + "lin2.b", dtype))
+    return x + g * block_linear(hp)(torch.cat([o, silu(a) * b], dim=1),
+                                    weight(p, pre + "lin2.w", dtype), weight(p, pre + "lin2.b", dtype))
 
 
 def _count(p, kind):
