@@ -332,6 +332,11 @@ def run_ours(args, w):
     flux3 = is_flux3(w)
     model = (F.Flux3DiT if flux3 else F.FluxDiT)(blob, w.dims)
     del blob
+    fp8 = args.precision == "fp8"
+    if fp8:
+        if flux3:
+            raise SystemExit("--precision fp8 is implemented for the FLUX.2 workloads")
+        model.set_precision(F.PRECISION_FP8)
     stream = torch.cuda.current_stream()
     dev = torch.device("cuda", local)
     lat0 = torch.from_numpy(lat_h).to(dev)
@@ -437,6 +442,9 @@ def run_ours(args, w):
     d2h = out_pin.numel() * 4
 
     peaks, peak_src = load_peaks()
+    # FP8 tensor peak: the measured bf16 figure times the nominal dense ratio 4.5 / 2.25 PFLOP/s
+    gemm_peak = peaks["bf16_tflops_sustained"] * (2.0 if fp8 else 1.0)
+    gemm_peak_kind = ("fp8 = 2 x bf16 sustained (nominal dense ratio), " if fp8 else "bf16 sustained, ") + peak_src
     flops = n_sequences(w) * forward_flops(w)
     tflops = flops / (ms_step / 1e3) / 1e12
     g_ms, g_fl, g_by, g_n = prof["gemm"]
@@ -453,7 +461,8 @@ def run_ours(args, w):
         line = {
             "metric": METRIC, "value": round(value, 4), "unit": step_unit(w), "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8-e4m3 row-wise block linears, bf16 attention" if fp8 else "bf16",
             "data": "synthetic (seeded N(0,1) weights scaled 1/sqrt(fan_in), bf16; N(0,1) latent and text)",
             "config": {"workload": f"{w.name}: {w.image}x{w.image}, {w.n_img} image + {w.n_txt} text + {w.n_ref} "
                                    f"reference tokens ({len(w.ref_grids)} reference images), {blocks_text(w)}, "
@@ -468,10 +477,13 @@ def run_ours(args, w):
                                "measured_sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
                                "spec_2250": round(tflops / SPEC_BF16_TFLOPS, 4), "peaks": peak_src},
             "forwards_per_s": round(1e3 / value, 3),
-            "roofline": {"kernel": "gemm_bf16_tc2 (CTA-pair tcgen05 GEMM) + the 128-wide output GEMM, all linear layers", "bound": "tensor",
-                         "achieved": round(gemm_tflops, 1), "peak": peaks["bf16_tflops_sustained"],
-                         "unit": "TFLOP/s", "frac": round(gemm_tflops / peaks["bf16_tflops_sustained"], 4),
-                         "peak_kind": f"bf16 sustained, {peak_src}", "traffic": traffic,
+            "roofline": {"kernel": ("gemm_bf16_tc2<fp8> (CTA-pair tcgen05 kind::f8f6f4) for the block linears, "
+                                    "bf16 for the input / output projections" if fp8 else
+                                    "gemm_bf16_tc2 (CTA-pair tcgen05 GEMM) + the 128-wide output GEMM, all linear layers"),
+                         "bound": "tensor",
+                         "achieved": round(gemm_tflops, 1), "peak": round(gemm_peak, 1),
+                         "unit": "TFLOP/s", "frac": round(gemm_tflops / gemm_peak, 4),
+                         "peak_kind": gemm_peak_kind, "traffic": None if fp8 else traffic,
                          "launches_per_forward": g_n // args.steps,
                          "share_of_step": round(g_ms / args.steps / ms_step, 3)},
             "attention": {"achieved": round(attn_tflops, 1), "unit": "TFLOP/s",
@@ -508,6 +520,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="t2i1024", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--precision", choices=("bf16", "fp8"), default="bf16",
+                    help="block linears in bf16, or row-wise FP8 (e4m3 codes with per-row scales)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -137,6 +137,20 @@ FLUX_API int flux_dit_forward_cfg(flux_dit *m, const float *img_tok, int grid_h,
                                   const float *txt_uncond, int n_txt, const float *ref_tok, int n_refs,
                                   const int *ref_grids, float t, float *v_cond, float *v_uncond, void *stream);
 
+/* Precision of the block linears (qkv, projection, MLP in / out; linear1 / linear2) of later
+ * forwards.  FLUX_PRECISION_BF16 (the default): bf16 operands.  FLUX_PRECISION_FP8: row-wise FP8,
+ * the "fp8r" format of the FLUX.3 Image Klein in Diffusers write-up, section "Hardwareanforderungen,
+ * Quantisierung und Inferenzlatenz": every weight row and every activation row is quantised to
+ * e4m3 with its own fp32 scale (amax / 448; codes e4m3(x * 448 / amax), round to nearest even,
+ * saturating), the products are accumulated in fp32 and scaled by both rows' scales.  The first
+ * switch to FP8 quantises the block weights once (a device allocation of one byte per weight, and
+ * a host synchronisation); the input / output projections, the modulation, attention and the
+ * residual stream keep their precision.  Needs hidden in {1024, 2048, 3072, 4096} and
+ * hidden + mlp_hidden <= 16384. */
+#define FLUX_PRECISION_BF16 0
+#define FLUX_PRECISION_FP8 1
+FLUX_API int flux_dit_set_precision(flux_dit *m, int precision);
+
 /* Diagnostic: run only the first n_double double blocks and n_single single
  * blocks in later forwards (-1 = all).  Used to bisect parity; not a model change. */
 FLUX_API int flux_dit_set_active_blocks(flux_dit *m, int n_double, int n_single);
@@ -225,6 +239,28 @@ FLUX_API int flux_rope_table(float *table, int n_txt, int gh, int gw, int rh, in
  * scaled by the gain (bf16 [128]), then rotated by the table (flux_rope_table). */
 FLUX_API int flux_qk_rmsnorm_rope(uint16_t *qkv, int rows, int ld, int k_col, int heads, const uint16_t *q_gain,
                          const uint16_t *k_gain, const float *table, float eps, void *stream);
+
+/* Row-wise e4m3 quantisation (see flux_dit_set_precision): for each of `rows` rows of x (bf16,
+ * row stride ldx elements) q[r, j] = e4m3(x[r, j] * inv_r) (uint8 codes, row stride ldq bytes) and
+ * scale[r] = amax_r / 448 with amax_r = max_j |x[r, j]| and inv_r = 448 / amax_r (0 for a zero row),
+ * the division and the product rounded to float32.  cols % 8 == 0, cols <= 16384; x 16-byte, q
+ * 8-byte aligned. */
+FLUX_API int flux_quantize_rows_e4m3(const uint16_t *x, int rows, int cols, int ldx, uint8_t *q, int ldq,
+                                     float *scale, void *stream);
+
+/* flux_layernorm_modulate with its output quantised row-wise to e4m3 in the same pass: q uint8
+ * [rows, dim] codes and q_scale fp32 [rows] as in flux_quantize_rows_e4m3 (the modulated values
+ * are quantised from float32).  dim in {1024, 2048, 3072, 4096}. */
+FLUX_API int flux_layernorm_modulate_fp8(const float *x, uint8_t *q, float *q_scale, int rows, int dim,
+                                         const float *shift, const float *scale, float eps, void *stream);
+
+/* FP8 linear layer on the tensor cores (tcgen05 kind::f8f6f4, CTA pairs): acc = (A W^T) with A e4m3
+ * codes [m, k] (row stride lda bytes) and W e4m3 codes [n, k], then acc[i][j] * a_scale[i] *
+ * w_scale[j] goes through the epilogue `mode` of flux_linear (0 bf16 + bias, 1 fp32 + bias,
+ * 2 SwiGLU, 3 gated residual).  k % 128 == 0, n % 32 == 0, lda % 16 == 0; pointers 16-byte aligned. */
+FLUX_API int flux_linear_fp8(const uint8_t *a, const float *a_scale, int m, int k, int lda, const uint8_t *w,
+                             const float *w_scale, int n, const uint16_t *bias, int mode, void *out, int ldo,
+                             const float *gate, void *stream);
 
 /* Measurement hooks (used by the benchmark).
  * flux_dit_profile(m, 1) starts bracketing every kernel launch of later

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libfluxdit.so")
 FLUX_OK, FLUX_EIO, FLUX_ENOMEM, FLUX_EINVAL = 0, -5, -12, -22
 
 EPI_BF16_BIAS, EPI_F32_BIAS, EPI_SWIGLU, EPI_RESID_GATE = 0, 1, 2, 3
+PRECISION_BF16, PRECISION_FP8 = 0, 1
 
 
 class FluxConfig(ctypes.Structure):
@@ -89,6 +90,10 @@ _SIGS = {
     "flux3_dit_profile_read": (_I, [_P, _I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
                                     ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]),
     "flux_joint_attention_segments": (_I, [_P, _P, _P, _P, _I, ctypes.POINTER(ctypes.c_int), _I, _I, _F, _P]),
+    "flux_dit_set_precision": (_I, [_P, _I]),
+    "flux_quantize_rows_e4m3": (_I, [_P, _I, _I, _I, _P, _I, _P, _P]),
+    "flux_layernorm_modulate_fp8": (_I, [_P, _P, _P, _I, _I, _P, _P, _F, _P]),
+    "flux_linear_fp8": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _P, _I, _P, _I, _P, _P]),
 }
 EXPORTED = tuple(_SIGS)
 
@@ -213,6 +218,10 @@ class FluxDiT:
 
     def set_active_blocks(self, n_double=-1, n_single=-1):
         _check(lib().flux_dit_set_active_blocks(self._h, n_double, n_single))
+
+    def set_precision(self, precision):
+        """PRECISION_BF16 or PRECISION_FP8 (row-wise e4m3 block linears); see flux_dit_set_precision."""
+        _check(lib().flux_dit_set_precision(self._h, int(precision)))
 
     PROFILE_KINDS = ("gemm", "attention", "ln_mod", "qk_norm_rope", "gemv", "other")
 
@@ -404,6 +413,49 @@ def flux_linear(a, w, bias, mode, out, gate=None, stream=None):
     _check(lib().flux_linear(ctypes.c_void_p(a.data_ptr()), m, k, lda, _bits(w, "w"), n, _bits(bias, "bias"), mode,
                              ctypes.c_void_p(out.data_ptr()), out.stride(0),
                              _ptr(gate, torch.float32, "gate"), _stream(stream)))
+    return out
+
+
+def _u8(t, what):
+    import torch
+    if t.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise ValueError(f"{what} must be uint8 e4m3 codes")
+    return _ptr(t, None, what)
+
+
+def flux_quantize_rows_e4m3(x, q, scale, stream=None):
+    """Row-wise e4m3 codes q (uint8 [rows, cols]) and scales (fp32 [rows]) of bf16 x [rows, cols]."""
+    import torch
+    rows, cols = x.shape
+    if x.stride(1) != 1 or q.stride(1) != 1:
+        raise ValueError("x and q must have unit column stride")
+    _check(lib().flux_quantize_rows_e4m3(ctypes.c_void_p(x.data_ptr()), rows, cols, x.stride(0),
+                                         ctypes.c_void_p(q.data_ptr()), q.stride(0),
+                                         _ptr(scale, torch.float32, "scale"), _stream(stream)))
+    return q, scale
+
+
+def flux_layernorm_modulate_fp8(x, q, q_scale, shift, scale, eps=1e-6, stream=None):
+    import torch
+    rows, dim = x.shape
+    _check(lib().flux_layernorm_modulate_fp8(_ptr(x, torch.float32, "x"), _u8(q, "q"),
+                                             _ptr(q_scale, torch.float32, "q_scale"), rows, dim,
+                                             _ptr(shift, torch.float32, "shift"), _ptr(scale, torch.float32, "scale"),
+                                             float(eps), _stream(stream)))
+    return q, q_scale
+
+
+def flux_linear_fp8(a, a_scale, w, w_scale, bias, mode, out, gate=None, stream=None):
+    """FP8 linear: a, w uint8 e4m3 codes [m, k] / [n, k] with row scales; epilogue modes as flux_linear."""
+    import torch
+    m, k = a.shape
+    n = w.shape[0]
+    if a.stride(1) != 1:
+        raise ValueError("a must have unit column stride")
+    _check(lib().flux_linear_fp8(ctypes.c_void_p(a.data_ptr()), _ptr(a_scale, torch.float32, "a_scale"), m, k,
+                                 a.stride(0), _u8(w, "w"), _ptr(w_scale, torch.float32, "w_scale"), n,
+                                 _bits(bias, "bias"), mode, ctypes.c_void_p(out.data_ptr()), out.stride(0),
+                                 _ptr(gate, torch.float32, "gate"), _stream(stream)))
     return out
 
 

@@ -55,8 +55,7 @@ const char* last_error() { return g_error.c_str(); }
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 static std::once_flag g_encode_once;
 
-bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
-                    uint32_t box_rows) {
+static bool encoder_ready() {
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -64,14 +63,30 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
         q == cudaDriverEntryPointSuccess)
       g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   });
-  if (!g_encode || rows == 0 || cols == 0) return false;
+  return g_encode != nullptr;
+}
+
+// 2D map with a box of 128 bytes along the row (one 128-byte swizzle row) and box_rows rows.
+static bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType type, uint32_t box_cols, const void* base,
+                         uint64_t rows, uint64_t cols, uint64_t row_stride_bytes, uint32_t box_rows) {
+  if (!encoder_ready() || rows == 0 || cols == 0) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {row_stride_bytes};
-  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return g_encode(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
+                    uint32_t box_rows) {
+  return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, base, rows, cols, row_stride_bytes, box_rows);
+}
+
+bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
+                  uint32_t box_rows) {
+  return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, base, rows, cols, row_stride_bytes, box_rows);
 }
 
 int num_sms_current() {
@@ -155,13 +170,20 @@ static_assert(sizeof(BlobHeader) == 80, "blob header layout");
 // ------------------------------------------------------------------ model
 struct StreamW {                       // one stream of a double block
   const bf16 *qkv_b, *q_gain, *k_gain, *proj_b, *mlp_in_b, *mlp_out_b;
+  const bf16 *w_qkv, *w_proj, *w_mlp_in, *w_mlp_out;
   size_t mod_off;                      // into the modulation vector (floats)
   CUtensorMap m_qkv, m_proj, m_mlp_in, m_mlp_out;
+  // FP8 precision: e4m3 codes of the same matrices (same row order) and their row scales
+  CUtensorMap m8_qkv, m8_proj, m8_mlp_in, m8_mlp_out;
+  const float *s_qkv, *s_proj, *s_mlp_in, *s_mlp_out;
 };
 struct SingleW {
   const bf16 *qkv_b, *mlp_b, *q_gain, *k_gain, *lin2_b;
+  const bf16 *w_lin1, *w_lin2;
   size_t mod_off;
   CUtensorMap m_qkv, m_mlp, m_lin2;
+  CUtensorMap m8_qkv, m8_mlp, m8_lin2;
+  const float *s_qkv, *s_mlp, *s_lin2;
 };
 
 constexpr int kMaxBatch = 2;            // sequences of one shape per forward (prompt and unconditional text)
@@ -179,6 +201,14 @@ struct Workspace {
   CUtensorMap a_tokb, a_Yall, a_CC, qkv;                // shared image input; whole-batch views
   CUtensorMap a_txtb[kMaxBatch], a_Ytxt[kMaxBatch], a_Yimg[kMaxBatch], a_Yout[kMaxBatch], a_Otxt[kMaxBatch],
       a_Oimg[kMaxBatch], a_Htxt[kMaxBatch], a_Himg[kMaxBatch];   // per-sequence views
+  // FP8 precision: e4m3 copies of the GEMM A operands (Y8 = LN-mod output, C8 = [O | H]) with one
+  // scale per row (sY; sC over [O | H] for linear2, sO and sH over O and H for the double blocks)
+  size_t cap8 = 0;
+  uint8_t *Y8 = nullptr, *C8 = nullptr;
+  float *sY = nullptr, *sC = nullptr, *sO = nullptr, *sH = nullptr;
+  bool maps8 = false;
+  CUtensorMap a8_Yall, a8_CC, a8_Ytxt[kMaxBatch], a8_Yimg[kMaxBatch], a8_Otxt[kMaxBatch], a8_Oimg[kMaxBatch],
+      a8_Htxt[kMaxBatch], a8_Himg[kMaxBatch];
 };
 
 }  // namespace fdit
@@ -197,13 +227,25 @@ struct flux_dit {
   std::vector<fdit::StreamW> dbl;      // [2 * i + 0] image stream, [2 * i + 1] text stream of block i
   std::vector<fdit::SingleW> sgl;
   int act_double = 0, act_single = 0;
+  int precision = FLUX_PRECISION_BF16;
+  uint8_t* w8 = nullptr;               // e4m3 block linears (allocated on the first switch to FP8)
+  float* w8_scale = nullptr;
   fdit::Workspace ws;
   fdit::Profiler prof;
 };
 
 namespace fdit {
 
+static void free_ws8(Workspace& w) {
+  cudaFree(w.Y8); cudaFree(w.C8); cudaFree(w.sY); cudaFree(w.sC); cudaFree(w.sO); cudaFree(w.sH);
+  w.Y8 = w.C8 = nullptr;
+  w.sY = w.sC = w.sO = w.sH = nullptr;
+  w.cap8 = 0;
+  w.maps8 = false;
+}
+
 static void free_ws(Workspace& w) {
+  free_ws8(w);
   cudaFree(w.X); cudaFree(w.Y); cudaFree(w.QKV); cudaFree(w.CC); cudaFree(w.tokb); cudaFree(w.txtb);
   cudaFree(w.rope);
   w = Workspace();
@@ -213,6 +255,7 @@ static void destroy(flux_dit* m) {
   if (!m) return;
   free_ws(m->ws);
   cudaFree(m->wbuf); cudaFree(m->mods_w); cudaFree(m->mods_b);
+  cudaFree(m->w8); cudaFree(m->w8_scale);
   cudaFree(m->temb); cudaFree(m->th); cudaFree(m->vec); cudaFree(m->mods);
   delete m;
 }
@@ -336,6 +379,8 @@ static int create_impl(const void* blob, size_t blob_bytes, const flux_dit_confi
       sw.qkv_b = W(p + "qkv.b"); sw.q_gain = W(p + "q_gain"); sw.k_gain = W(p + "k_gain");
       sw.proj_b = W(p + "proj.b"); sw.mlp_in_b = W(p + "mlp_in.b"); sw.mlp_out_b = W(p + "mlp_out.b");
       sw.mod_off = MOD(p + "mod.w");
+      sw.w_qkv = W(p + "qkv.w"); sw.w_proj = W(p + "proj.w");
+      sw.w_mlp_in = W(p + "mlp_in.w"); sw.w_mlp_out = W(p + "mlp_out.w");
       wmap(&sw.m_qkv, W(p + "qkv.w"), 3 * D, D, 128);
       wmap(&sw.m_proj, W(p + "proj.w"), D, D, 128);
       wmap(&sw.m_mlp_in, W(p + "mlp_in.w"), 2 * F, D, 128);
@@ -350,6 +395,7 @@ static int create_impl(const void* blob, size_t blob_bytes, const flux_dit_confi
     sw.qkv_b = l1b; sw.mlp_b = l1b + 3 * D;
     sw.q_gain = W(p + "q_gain"); sw.k_gain = W(p + "k_gain"); sw.lin2_b = W(p + "lin2.b");
     sw.mod_off = MOD(p + "mod.w");
+    sw.w_lin1 = l1; sw.w_lin2 = W(p + "lin2.w");
     wmap(&sw.m_qkv, l1, 3 * D, D, 128);
     wmap(&sw.m_mlp, l1 + 3 * D * D, 2 * F, D, 128);
     wmap(&sw.m_lin2, W(p + "lin2.w"), D, D + F, 128);
@@ -359,6 +405,48 @@ static int create_impl(const void* blob, size_t blob_bytes, const flux_dit_confi
   m->act_single = c.n_single;
   if (cudaStreamSynchronize(s) != cudaSuccess) return cleanup(FLUX_EIO, "weight upload failed (sync)");
   *out = m;
+  return FLUX_OK;
+}
+
+// FP8 copies of the GEMM A operands for a batch of nb sequences of n = nt + nimg rows, and their maps.
+static int prepare_fp8(flux_dit* m, int nt, int nimg, int nb) {
+  Workspace& w = m->ws;
+  const flux_dit_config& c = m->cfg;
+  const size_t D = c.hidden, F = c.mlp_hidden;
+  const size_t n = nt + nimg, rows = n * nb;
+  if (rows > w.cap8) {
+    free_ws8(w);
+    bool ok = cudaMalloc(&w.Y8, rows * D) == cudaSuccess && cudaMalloc(&w.C8, rows * (D + F)) == cudaSuccess &&
+              cudaMalloc(&w.sY, rows * 4) == cudaSuccess && cudaMalloc(&w.sC, rows * 4) == cudaSuccess &&
+              cudaMalloc(&w.sO, rows * 4) == cudaSuccess && cudaMalloc(&w.sH, rows * 4) == cudaSuccess;
+    if (!ok) {
+      free_ws8(w);
+      return fail(FLUX_ENOMEM, "FP8 workspace allocation for %zu tokens failed", rows);
+    }
+    w.cap8 = rows;
+  }
+  if (w.maps8) return FLUX_OK;
+  bool ok = true;
+  auto amap = [&](CUtensorMap* map, const uint8_t* base, size_t nrows, size_t cols, uint64_t stride) {
+    if (nrows == 0) {
+      memset(map, 0, sizeof(*map));
+      return;
+    }
+    ok &= make_tmap_u8(map, base, nrows, cols, stride, 128);
+  };
+  amap(&w.a8_Yall, w.Y8, rows, D, D);
+  amap(&w.a8_CC, w.C8, rows, D + F, D + F);
+  for (int b = 0; b < nb; ++b) {
+    const size_t r0 = b * n;
+    amap(&w.a8_Ytxt[b], w.Y8 + r0 * D, nt, D, D);
+    amap(&w.a8_Yimg[b], w.Y8 + (r0 + nt) * D, nimg, D, D);
+    amap(&w.a8_Otxt[b], w.C8 + r0 * (D + F), nt, D, D + F);
+    amap(&w.a8_Oimg[b], w.C8 + (r0 + nt) * (D + F), nimg, D, D + F);
+    amap(&w.a8_Htxt[b], w.C8 + r0 * (D + F) + D, nt, F, D + F);
+    amap(&w.a8_Himg[b], w.C8 + (r0 + nt) * (D + F) + D, nimg, F, D + F);
+  }
+  if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an FP8 activation buffer");
+  w.maps8 = true;
   return FLUX_OK;
 }
 
@@ -386,7 +474,10 @@ static int prepare_shape(flux_dit* m, int nt, int gh, int gw, const RefGrids& re
   if (grow(&w.tokb, &w.cap_tok, (ni + nr) * c.in_ch) != cudaSuccess ||
       grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt * nb, 1) * c.txt_dim) != cudaSuccess)
     return fail(FLUX_ENOMEM, "workspace allocation failed");
-  if (w.nt == nt && w.gh == gh && w.gw == gw && w.nb == nb && same_refs(w.refs, refs)) return FLUX_OK;
+  const bool fp8 = m->precision == FLUX_PRECISION_FP8;
+  if (w.nt == nt && w.gh == gh && w.gw == gw && w.nb == nb && same_refs(w.refs, refs))
+    return fp8 ? prepare_fp8(m, nt, static_cast<int>(ni + nr), nb) : FLUX_OK;
+  w.maps8 = false;
 
   const size_t nimg = ni + nr;
   const uint64_t ldD = D * 2, ldC = (D + F) * 2;
@@ -421,6 +512,75 @@ static int prepare_shape(flux_dit* m, int nt, int gh, int gw, const RefGrids& re
         cudaSuccess)
       return fail(FLUX_EIO, "rope table copy failed");
   w.nt = nt; w.gh = gh; w.gw = gw; w.nb = nb; w.refs = refs;
+  return fp8 ? prepare_fp8(m, nt, static_cast<int>(nimg), nb) : FLUX_OK;
+}
+
+// Quantise every block linear to e4m3 with one scale per output row (done once per model).
+static int quantize_block_weights(flux_dit* m, cudaStream_t s) {
+  const flux_dit_config& c = m->cfg;
+  const size_t D = c.hidden, F = c.mlp_hidden;
+  struct Mat {
+    const bf16* w;
+    size_t rows, cols;
+  };
+  std::vector<Mat> mats;
+  for (const StreamW& sw : m->dbl) {
+    mats.push_back({sw.w_qkv, 3 * D, D});
+    mats.push_back({sw.w_proj, D, D});
+    mats.push_back({sw.w_mlp_in, 2 * F, D});
+    mats.push_back({sw.w_mlp_out, D, F});
+  }
+  for (const SingleW& sw : m->sgl) {
+    mats.push_back({sw.w_lin1, 3 * D + 2 * F, D});
+    mats.push_back({sw.w_lin2, D, D + F});
+  }
+  size_t bytes = 0, rows = 0;
+  for (const Mat& x : mats) {
+    bytes += (x.rows * x.cols + 255) / 256 * 256;
+    rows += (x.rows + 63) / 64 * 64;
+  }
+  if (cudaMalloc(&m->w8, bytes) != cudaSuccess || cudaMalloc(&m->w8_scale, rows * 4) != cudaSuccess) {
+    cudaFree(m->w8);
+    cudaFree(m->w8_scale);
+    m->w8 = nullptr;
+    m->w8_scale = nullptr;
+    return fail(FLUX_ENOMEM, "cudaMalloc of the FP8 weights (%zu bytes) failed", bytes);
+  }
+  std::vector<const uint8_t*> q(mats.size());
+  std::vector<const float*> sc(mats.size());
+  size_t boff = 0, roff = 0;
+  for (size_t i = 0; i < mats.size(); ++i) {
+    const Mat& x = mats[i];
+    uint8_t* qd = m->w8 + boff;
+    float* sd = m->w8_scale + roff;
+    FD_CUDA(quantize_rows_launch(x.w, static_cast<int>(x.cols), static_cast<int>(x.rows), static_cast<int>(x.cols),
+                                 qd, static_cast<int>(x.cols), sd, s));
+    q[i] = qd;
+    sc[i] = sd;
+    boff += (x.rows * x.cols + 255) / 256 * 256;
+    roff += (x.rows + 63) / 64 * 64;
+  }
+  bool ok = true;
+  auto wmap = [&](CUtensorMap* map, const uint8_t* base, size_t r, size_t cols) {
+    ok &= make_tmap_u8(map, base, r, cols, cols, 128);
+  };
+  size_t i = 0;
+  for (StreamW& sw : m->dbl) {
+    wmap(&sw.m8_qkv, q[i], 3 * D, D); sw.s_qkv = sc[i++];
+    wmap(&sw.m8_proj, q[i], D, D); sw.s_proj = sc[i++];
+    wmap(&sw.m8_mlp_in, q[i], 2 * F, D); sw.s_mlp_in = sc[i++];
+    wmap(&sw.m8_mlp_out, q[i], D, F); sw.s_mlp_out = sc[i++];
+  }
+  for (SingleW& sw : m->sgl) {
+    wmap(&sw.m8_qkv, q[i], 3 * D, D);
+    wmap(&sw.m8_mlp, q[i] + 3 * D * D, 2 * F, D);
+    sw.s_qkv = sc[i];
+    sw.s_mlp = sc[i] + 3 * D;
+    ++i;
+    wmap(&sw.m8_lin2, q[i], D, D + F); sw.s_lin2 = sc[i++];
+  }
+  if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an FP8 weight tensor");
+  FD_CUDA(cudaStreamSynchronize(s));
   return FLUX_OK;
 }
 
@@ -505,13 +665,40 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
   A.q_col0 = 0; A.k_col0 = D; A.v_col0 = 2 * D;
   A.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
 
+  // FP8 precision: block linears on e4m3 codes (row-wise scales); LN-mod quantises its output,
+  // the attention output and the SwiGLU hidden are quantised before the linears that read them
+  const bool fp8 = m->precision == FLUX_PRECISION_FP8;
+  auto f8 = [&](int i, const CUtensorMap& a8, const CUtensorMap& w8, const float* sa, const float* sb) {
+    P.mapA[i] = a8;
+    P.mapB[i] = w8;
+    P.prob[i].scale_a = sa;
+    P.prob[i].scale_b = sb;
+  };
+  // LN-mod of every row: rows r % n < split use (sh0, sc0), the others (sh1, sc1)
+  auto ln_mod = [&](int split, const float* sh0, const float* sc0, const float* sh1, const float* sc1) -> int {
+    if (fp8)
+      FD_LAUNCH(m, kProfLnMod, 0, 5.0 * rows * D + 4.0 * rows,
+                ln_modulate_fp8_launch(w.X, w.Y8, w.sY, rows, D, split, n, n, sh0, sc0, sh1, sc1, sh1, sc1, eps_ln,
+                                       s));
+    else
+      FD_LAUNCH(m, kProfLnMod, 0, ln_bytes, ln_modulate_launch(w.X, w.Y, rows, D, split, n, sh0, sc0, sh1, sc1,
+                                                               eps_ln, s));
+    return FLUX_OK;
+  };
+  // e4m3 codes of CC columns [col0, col0 + cols) into C8, one scale per row
+  auto quant_cc = [&](int col0, int cols, float* scale) -> int {
+    FD_LAUNCH(m, kProfOther, 0, 3.0 * rows * cols + 4.0 * rows,
+              quantize_rows_launch(w.CC + col0, D + F, rows, cols, w.C8 + col0, D + F, scale, s));
+    return FLUX_OK;
+  };
+
   for (int i = 0; i < m->act_double; ++i) {
     const StreamW& si = m->dbl[2 * i];
     const StreamW& st = m->dbl[2 * i + 1];
     const float* mi = mods + si.mod_off;          // shift1, scale1, gate1, shift2, scale2, gate2
     const float* mt = mods + st.mod_off;
-    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes,
-              ln_modulate_launch(w.X, w.Y, rows, D, nt, n, mt, mt + D, mi, mi + D, eps_ln, s));
+    rc = ln_mod(nt, mt, mt + D, mi, mi + D);
+    if (rc) return rc;
     P.num_problems = 2 * nb;
     for (int b = 0; b < nb; ++b) {
       problem(P, 2 * b, w.a_Ytxt[b], st.m_qkv, nt, 3 * D, D, kEpiBf16Bias, w.QKV + seq_row(b, 0) * 3 * D, 3 * D,
@@ -520,52 +707,75 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
               3 * D, si.qkv_b, nullptr);
       qk_fuse(P, 2 * b, st.q_gain, st.k_gain, w.rope, static_cast<int>(seq_row(b, 0)), eps_rms);
       qk_fuse(P, 2 * b + 1, si.q_gain, si.k_gain, w.rope, static_cast<int>(seq_row(b, nt)), eps_rms);
+      if (fp8) {
+        f8(2 * b, w.a8_Ytxt[b], st.m8_qkv, w.sY + seq_row(b, 0), st.s_qkv);
+        f8(2 * b + 1, w.a8_Yimg[b], si.m8_qkv, w.sY + seq_row(b, nt), si.s_qkv);
+      }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
     FD_LAUNCH(m, kProfAttention, at_flops, at_bytes, attention_launch(A, s));
+    if (fp8 && (rc = quant_cc(0, D, w.sO))) return rc;
     P.num_problems = 2 * nb;
     for (int b = 0; b < nb; ++b) {
       problem(P, 2 * b, w.a_Otxt[b], st.m_proj, nt, D, D, kEpiResidGate, w.X + seq_row(b, 0) * D, D, st.proj_b,
               mt + 2 * D);
       problem(P, 2 * b + 1, w.a_Oimg[b], si.m_proj, nimg, D, D, kEpiResidGate, w.X + seq_row(b, nt) * D, D,
               si.proj_b, mi + 2 * D);
+      if (fp8) {
+        f8(2 * b, w.a8_Otxt[b], st.m8_proj, w.sO + seq_row(b, 0), st.s_proj);
+        f8(2 * b + 1, w.a8_Oimg[b], si.m8_proj, w.sO + seq_row(b, nt), si.s_proj);
+      }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
-    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes,
-              ln_modulate_launch(w.X, w.Y, rows, D, nt, n, mt + 3 * D, mt + 4 * D, mi + 3 * D, mi + 4 * D, eps_ln,
-                                 s));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
+    rc = ln_mod(nt, mt + 3 * D, mt + 4 * D, mi + 3 * D, mi + 4 * D);
+    if (rc) return rc;
     P.num_problems = 2 * nb;
     for (int b = 0; b < nb; ++b) {
       problem(P, 2 * b, w.a_Ytxt[b], st.m_mlp_in, nt, 2 * F, D, kEpiSwiGLU, w.CC + seq_row(b, 0) * (D + F) + D,
               D + F, st.mlp_in_b, nullptr);
       problem(P, 2 * b + 1, w.a_Yimg[b], si.m_mlp_in, nimg, 2 * F, D, kEpiSwiGLU,
               w.CC + seq_row(b, nt) * (D + F) + D, D + F, si.mlp_in_b, nullptr);
+      if (fp8) {
+        f8(2 * b, w.a8_Ytxt[b], st.m8_mlp_in, w.sY + seq_row(b, 0), st.s_mlp_in);
+        f8(2 * b + 1, w.a8_Yimg[b], si.m8_mlp_in, w.sY + seq_row(b, nt), si.s_mlp_in);
+      }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
+    if (fp8 && (rc = quant_cc(D, F, w.sH))) return rc;
     P.num_problems = 2 * nb;
     for (int b = 0; b < nb; ++b) {
       problem(P, 2 * b, w.a_Htxt[b], st.m_mlp_out, nt, D, F, kEpiResidGate, w.X + seq_row(b, 0) * D, D,
               st.mlp_out_b, mt + 5 * D);
       problem(P, 2 * b + 1, w.a_Himg[b], si.m_mlp_out, nimg, D, F, kEpiResidGate, w.X + seq_row(b, nt) * D, D,
               si.mlp_out_b, mi + 5 * D);
+      if (fp8) {
+        f8(2 * b, w.a8_Htxt[b], st.m8_mlp_out, w.sH + seq_row(b, 0), st.s_mlp_out);
+        f8(2 * b + 1, w.a8_Himg[b], si.m8_mlp_out, w.sH + seq_row(b, nt), si.s_mlp_out);
+      }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
   }
   // single blocks: one set of weights for every row, so the whole batch is one problem
   for (int i = 0; i < m->act_single; ++i) {
     const SingleW& sw = m->sgl[i];
     const float* ms = mods + sw.mod_off;          // shift, scale, gate
-    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes,
-              ln_modulate_launch(w.X, w.Y, rows, D, n, n, ms, ms + D, ms, ms + D, eps_ln, s));
+    rc = ln_mod(n, ms, ms + D, ms, ms + D);
+    if (rc) return rc;
     P.num_problems = 2;
     problem(P, 0, w.a_Yall, sw.m_qkv, rows, 3 * D, D, kEpiBf16Bias, w.QKV, 3 * D, sw.qkv_b, nullptr);
     problem(P, 1, w.a_Yall, sw.m_mlp, rows, 2 * F, D, kEpiSwiGLU, w.CC + D, D + F, sw.mlp_b, nullptr);
     qk_fuse(P, 0, sw.q_gain, sw.k_gain, w.rope, 0, eps_rms);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+    if (fp8) {
+      f8(0, w.a8_Yall, sw.m8_qkv, w.sY, sw.s_qkv);
+      f8(1, w.a8_Yall, sw.m8_mlp, w.sY, sw.s_mlp);
+    }
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
     FD_LAUNCH(m, kProfAttention, at_flops, at_bytes, attention_launch(A, s));
+    if (fp8 && (rc = quant_cc(0, D + F, w.sC))) return rc;
     P.num_problems = 1;
     problem(P, 0, w.a_CC, sw.m_lin2, rows, D, D + F, kEpiResidGate, w.X, D, sw.lin2_b, ms + 2 * D);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+    if (fp8) f8(0, w.a8_CC, sw.m8_lin2, w.sC, sw.s_lin2);
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
   }
   // output layer on the image rows of each sequence
   const float* mf = mods + m->fin_mod_off;         // shift, scale
@@ -661,6 +871,28 @@ int flux_blend_latents(const float* x, const float* noise, float t, float* out, 
   if (n && (!x || !noise || !out)) return fail(FLUX_EINVAL, "NULL argument");
   if (!std::isfinite(t)) return fail(FLUX_EINVAL, "t is not finite");
   FD_CUDA(blend_launch(x, noise, t, out, n, static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_dit_set_precision(flux_dit* m, int precision) {
+  if (!m) return fail(FLUX_EINVAL, "model is NULL");
+  if (precision == FLUX_PRECISION_BF16) {
+    m->precision = precision;
+    return FLUX_OK;
+  }
+  if (precision != FLUX_PRECISION_FP8) return fail(FLUX_EINVAL, "unknown precision %d", precision);
+  const flux_dit_config& c = m->cfg;
+  if (c.hidden % 128 || c.mlp_hidden % 128 || (c.hidden != 1024 && c.hidden != 2048 && c.hidden != 3072 &&
+                                                c.hidden != 4096) || c.hidden + c.mlp_hidden > 16384)
+    return fail(FLUX_EINVAL, "FP8 needs hidden in {1024, 2048, 3072, 4096} and hidden + mlp_hidden <= 16384");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != m->device) return fail(FLUX_EINVAL, "model lives on device %d, current device is %d", m->device, dev);
+  if (!m->w8) {
+    const int rc = quantize_block_weights(m, nullptr);
+    if (rc) return rc;
+  }
+  m->precision = precision;
   return FLUX_OK;
 }
 
@@ -764,6 +996,56 @@ int flux_linear(const uint16_t* a, int m, int k, int lda, const uint16_t* w, int
     FD_CUDA(gemm2_launch(P, num_sms_current(), static_cast<cudaStream_t>(stream)));
   else
     FD_CUDA(gemm_launch(P, bn, num_sms_current(), static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_quantize_rows_e4m3(const uint16_t* x, int rows, int cols, int ldx, uint8_t* q, int ldq, float* scale,
+                            void* stream) {
+  if (!x || !q || !scale) return fail(FLUX_EINVAL, "NULL argument");
+  if (rows < 0 || cols < 8 || cols % 8 || cols > 16384 || ldx < cols || ldx % 8 || ldq < cols || ldq % 8)
+    return fail(FLUX_EINVAL, "bad shape rows=%d cols=%d ldx=%d ldq=%d", rows, cols, ldx, ldq);
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(q) & 7) || (reinterpret_cast<uintptr_t>(scale) & 3))
+    return fail(FLUX_EINVAL, "x must be 16-byte and q 8-byte aligned");
+  FD_CUDA(quantize_rows_launch(reinterpret_cast<const bf16*>(x), ldx, rows, cols, q, ldq, scale,
+                               static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_layernorm_modulate_fp8(const float* x, uint8_t* q, float* q_scale, int rows, int dim, const float* shift,
+                                const float* scale, float eps, void* stream) {
+  if (!x || !q || !q_scale || !shift || !scale) return fail(FLUX_EINVAL, "NULL argument");
+  if (rows < 0 || (dim != 1024 && dim != 2048 && dim != 3072 && dim != 4096))
+    return fail(FLUX_EINVAL, "bad shape rows=%d dim=%d (dim in 1024, 2048, 3072, 4096)", rows, dim);
+  if (!aligned16(x) || !aligned16(q) || !aligned16(shift) || !aligned16(scale))
+    return fail(FLUX_EINVAL, "pointers must be 16-byte aligned");
+  FD_CUDA(ln_modulate_fp8_launch(x, q, q_scale, rows, dim, rows, rows, rows, shift, scale, shift, scale, shift, scale,
+                                 eps, static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_linear_fp8(const uint8_t* a, const float* a_scale, int m, int k, int lda, const uint8_t* w,
+                    const float* w_scale, int n, const uint16_t* bias, int mode, void* out, int ldo, const float* gate,
+                    void* stream) {
+  if (!a || !a_scale || !w || !w_scale || !bias || !out) return fail(FLUX_EINVAL, "NULL argument");
+  if (m < 1 || k < 128 || k % 128 || n < 32 || n % 32 || lda < k || lda % 16)
+    return fail(FLUX_EINVAL, "bad shape m=%d k=%d n=%d lda=%d (k %% 128, n %% 32, lda %% 16)", m, k, n, lda);
+  if (mode < 0 || mode > 3) return fail(FLUX_EINVAL, "bad mode %d", mode);
+  if (mode == kEpiSwiGLU && n % 256) return fail(FLUX_EINVAL, "SwiGLU mode needs n %% 256 == 0");
+  if (mode == kEpiResidGate && !gate) return fail(FLUX_EINVAL, "gate is NULL");
+  const int out_cols = mode == kEpiSwiGLU ? n / 2 : n;
+  if (ldo < out_cols || ldo % 8) return fail(FLUX_EINVAL, "bad ldo=%d", ldo);
+  if (!aligned16(a) || !aligned16(w) || !aligned16(bias) || !aligned16(out) || !aligned16(a_scale) ||
+      !aligned16(w_scale) || (gate && !aligned16(gate)))
+    return fail(FLUX_EINVAL, "pointers must be 16-byte aligned");
+  GemmParams P;
+  P.num_problems = 1;
+  if (!make_tmap_u8(&P.mapA[0], a, m, k, static_cast<uint64_t>(lda), 128) ||
+      !make_tmap_u8(&P.mapB[0], w, n, k, static_cast<uint64_t>(k), 128))
+    return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed");
+  problem(P, 0, P.mapA[0], P.mapB[0], m, n, k, mode, out, ldo, reinterpret_cast<const bf16*>(bias), gate);
+  P.prob[0].scale_a = a_scale;
+  P.prob[0].scale_b = w_scale;
+  FD_CUDA(gemm2_launch(P, num_sms_current(), static_cast<cudaStream_t>(stream), true));
   return FLUX_OK;
 }
 

@@ -29,6 +29,10 @@ struct GemmProblem {
   const float2* rope;             // (cos, sin) [tokens, 64]
   int rope_row0;
   float eps;
+  // 8-bit operands (gemm2 launched with fp8): the accumulator is scaled by scale_a[m] (per row of
+  // A, [M]) and scale_b[n] (per row of W, [N]) before the epilogue above
+  const float* scale_a;
+  const float* scale_b;
 };
 
 struct GemmParams {
@@ -42,8 +46,9 @@ struct GemmParams {
 int gemm_bn_for(int n);
 cudaError_t gemm_launch(GemmParams& P, int bn, int num_sms, cudaStream_t stream);
 int gemm_read_device_error(cudaStream_t stream);
-// CTA-pair variant (cta_group::2, 256 x 256 tiles, W maps with a 128-row box): same problems and epilogues
-cudaError_t gemm2_launch(GemmParams& P, int num_sms, cudaStream_t stream);
+// CTA-pair variant (cta_group::2, 256 x 256 tiles, W maps with a 128-row box): same problems and epilogues.
+// fp8: A and W are e4m3 codes (u8 maps with a 128-byte box, K % 128 == 0) with per-row scales.
+cudaError_t gemm2_launch(GemmParams& P, int num_sms, cudaStream_t stream, bool fp8 = false);
 int gemm2_read_device_error(cudaStream_t stream);
 
 // ------------------------------------------------------------------ attention
@@ -118,6 +123,18 @@ cudaError_t gemv_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, const fl
 cudaError_t gemv_multi_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, const float* x, int nvec, float* y,
                               const float* add, int rows, int k, int silu_in, int silu_out, cudaStream_t s);
 
+// ------------------------------------------------------------------ row-wise e4m3 (fp8.cu)
+// codes[r, 0..cols) = e4m3(x[r, j] * 448 / amax_r), scale[r] = amax_r / 448; x bf16 rows of stride
+// ldx, codes of stride ldq (bytes); cols % 8 == 0, cols <= 16384.
+cudaError_t quantize_rows_launch(const __nv_bfloat16* x, int ldx, int rows, int cols, uint8_t* q, int ldq,
+                                 float* scale, cudaStream_t s);
+// ln_modulate3_launch whose modulated rows are quantised to e4m3 codes [rows, dim] + scales [rows];
+// dim in {1024, 2048, 3072, 4096}.
+cudaError_t ln_modulate_fp8_launch(const float* x, uint8_t* q, float* qscale, int rows, int dim, int split,
+                                   int split2, int period, const float* shift0, const float* scale0,
+                                   const float* shift1, const float* scale1, const float* shift2,
+                                   const float* scale2, float eps, cudaStream_t s);
+
 // ------------------------------------------------------------------ host helpers
 // Record `msg` as the calling thread's flux_get_error() message and return `code`.
 int record_error(int code, const char* msg);
@@ -126,6 +143,9 @@ void count_launch();
 // 2D bf16 tensor map: rows x cols, row stride in bytes, box {64 cols, box_rows}, 128B swizzle.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
                     uint32_t box_rows);
+// 2D u8 tensor map (e4m3 codes): rows x cols bytes, box {128 bytes, box_rows}, 128B swizzle.
+bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
+                  uint32_t box_rows);
 int num_sms_current();
 
 }  // namespace fdit

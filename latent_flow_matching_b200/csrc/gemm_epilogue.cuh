@@ -11,9 +11,27 @@
 
 namespace fdit {
 
-template <int BN>
+// kScale (8-bit operands): acc[m][n] *= scale_a[m] * scale_b[n] as each 32-column chunk is read.
+template <bool kScale>
+__device__ __forceinline__ void scale_chunk(uint32_t (&r)[32], float sa, const float* sb) {
+  if constexpr (kScale) {
+    const float4* s4 = reinterpret_cast<const float4*>(sb);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const float4 w = __ldg(s4 + v);
+      r[4 * v + 0] = __float_as_uint(__uint_as_float(r[4 * v + 0]) * sa * w.x);
+      r[4 * v + 1] = __float_as_uint(__uint_as_float(r[4 * v + 1]) * sa * w.y);
+      r[4 * v + 2] = __float_as_uint(__uint_as_float(r[4 * v + 2]) * sa * w.z);
+      r[4 * v + 3] = __float_as_uint(__uint_as_float(r[4 * v + 3]) * sa * w.w);
+    }
+  }
+}
+
+template <int BN, bool kScale = false>
 __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32_t tbase, int m, int n0) {
   const bool row_ok = m < pr.M;
+  float sa = 0.f;                          // row scale (kScale only; rows outside the problem read none)
+  if constexpr (kScale) sa = row_ok ? __ldg(pr.scale_a + m) : 0.f;
   if (pr.mode == kEpiSwiGLU) {
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(pr.out);
     const int on0 = n0 / 2;                // output column of this tile's first pair
@@ -24,6 +42,8 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
       tmem_ld32(tbase + BN / 2 + c, rb);
       tmem_ld_wait();
       if (row_ok && n0 + c < pr.N) {
+        scale_chunk<kScale>(ra, sa, pr.scale_b + n0 + c);
+        scale_chunk<kScale>(rb, sa, pr.scale_b + n0 + BN / 2 + c);
         const uint4* ba = reinterpret_cast<const uint4*>(pr.bias + n0 + c);
         const uint4* bb = reinterpret_cast<const uint4*>(pr.bias + n0 + BN / 2 + c);
         uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(m) * pr.ldo + on0 + c);
@@ -60,6 +80,7 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
         uint32_t r[32];
         tmem_ld32(hb + c, r);
         tmem_ld_wait();
+        if (row_ok) scale_chunk<kScale>(r, sa, pr.scale_b + n0 + hh * 128 + c);
         const uint4* bsrc = reinterpret_cast<const uint4*>(bh + c);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
@@ -80,6 +101,7 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
         tmem_ld32(hb + c, r);
         tmem_ld_wait();
         if (!row_ok) continue;
+        scale_chunk<kScale>(r, sa, pr.scale_b + n0 + hh * 128 + c);
         const uint4* bsrc = reinterpret_cast<const uint4*>(bh + c);
         const uint4* gsrc = reinterpret_cast<const uint4*>(gain + c);
         uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(m) * pr.ldo + n0 + hh * 128 + c);
@@ -110,6 +132,7 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
       tmem_ld_wait();
       const int n = n0 + c;
       if (!row_ok || n >= pr.N) continue;
+      scale_chunk<kScale>(r, sa, pr.scale_b + n);
       const uint4* bsrc = reinterpret_cast<const uint4*>(pr.bias + n);
       float f[32];
 #pragma unroll

@@ -45,8 +45,12 @@ __device__ __forceinline__ int find_problem(const GemmParams& P, int tile) {
   return p;
 }
 
+// kFp8: e4m3 operands, 128 per 128-byte swizzle row (BK = 128 elements per stage, the same bytes
+// as 64 bf16), kind::f8f6f4 MMAs with K = 32, and the epilogue applies the row / column scales.
+template <bool kFp8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     gemm_bf16_tc2_kernel(const __grid_constant__ GemmParams P) {
+  constexpr int BKE = kFp8 ? 2 * BK : BK;           // K elements per stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -105,7 +109,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         const int lt = tile - pr.tile_begin;
         const int m0 = (lt % pr.tiles_m) * BM + 128 * static_cast<int>(rank);
         const int n0 = (lt / pr.tiles_m) * BN + 128 * static_cast<int>(rank);
-        const int nk = pr.K / BK;
+        const int nk = pr.K / BKE;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -113,8 +117,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           }
           const uint32_t fb = map_to_rank(&full[stage], 0);
           mbar_arrive_expect_tx_cluster(fb, STAGE_BYTES);
-          tma_load_2d_pair(sA + stage * A_BYTES, &P.mapA[p], fb, kb * BK, m0);
-          tma_load_2d_pair(sB + stage * B_BYTES, &P.mapB[p], fb, kb * BK, n0);
+          tma_load_2d_pair(sA + stage * A_BYTES, &P.mapA[p], fb, kb * BKE, m0);
+          tma_load_2d_pair(sB + stage * B_BYTES, &P.mapB[p], fb, kb * BKE, n0);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -137,12 +141,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      const uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
+      const uint32_t idesc = kFp8 ? idesc_e4m3_f32(BM, BN) : idesc_bf16_f32(BM, BN, 0, 0);
       const uint64_t a_desc0 = sw128_desc(smem_u32(sA), 16, 1024);
       const uint64_t b_desc0 = sw128_desc(smem_u32(sB), 16, 1024);
       for (int tile = pair; ok && tile < P.total_tiles; tile += num_pairs) {
         const int p = find_problem(P, tile);
-        const int nk = P.prob[p].K / BK;
+        const int nk = P.prob[p].K / BKE;
         if (!mbar_wait_warp(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -158,8 +162,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           const uint64_t ad = desc_advance(a_desc0, stage * A_BYTES);
           const uint64_t bd = desc_advance(b_desc0, stage * B_BYTES);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            mma_pair_warp(d_tmem, desc_advance(ad, k * 32), desc_advance(bd, k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {                  // 32 bytes of K per MMA: 16 bf16 or 32 e4m3
+            if constexpr (kFp8)
+              mma_pair_f8_warp(d_tmem, desc_advance(ad, k * 32), desc_advance(bd, k * 32), idesc,
+                               (kb | k) != 0 ? 1u : 0u);
+            else
+              mma_pair_warp(d_tmem, desc_advance(ad, k * 32), desc_advance(bd, k * 32), idesc,
+                            (kb | k) != 0 ? 1u : 0u);
+          }
           mma_commit_pair_warp(&empty[stage]);            // frees this stage in both CTAs
           if (++stage == STAGES) {
             stage = 0;
@@ -195,7 +205,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(acc * BN);
-      gemm_epilogue_tile<BN>(pr, tbase, m, n0);
+      gemm_epilogue_tile<BN, kFp8>(pr, tbase, m, n0);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader[acc]);
@@ -214,13 +224,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 
 }  // namespace
 
-cudaError_t gemm2_launch(GemmParams& P, int num_sms, cudaStream_t stream) {
+cudaError_t gemm2_launch(GemmParams& P, int num_sms, cudaStream_t stream, bool fp8) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e =
-        cudaFuncSetAttribute(gemm_bf16_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        cudaFuncSetAttribute(gemm_bf16_tc2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm_bf16_tc2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
+  }
+  for (int i = 0; i < P.num_problems; ++i) {        // 8-bit problems: K in whole stages, scales present
+    const GemmProblem& pr = P.prob[i];
+    if (pr.M > 0 && (pr.K % (fp8 ? 2 * BK : BK) != 0 || (fp8 && (!pr.scale_a || !pr.scale_b))))
+      return cudaErrorInvalidValue;
   }
   int w = 0, total = 0;
   for (int i = 0; i < P.num_problems; ++i) {
@@ -242,7 +259,10 @@ cudaError_t gemm2_launch(GemmParams& P, int num_sms, cudaStream_t stream) {
   int pairs = num_sms / 2;
   if (pairs > total) pairs = total;
   count_launch();
-  gemm_bf16_tc2_kernel<<<2 * pairs, 192, SMEM_BYTES, stream>>>(P);
+  if (fp8)
+    gemm_bf16_tc2_kernel<true><<<2 * pairs, 192, SMEM_BYTES, stream>>>(P);
+  else
+    gemm_bf16_tc2_kernel<false><<<2 * pairs, 192, SMEM_BYTES, stream>>>(P);
   return cudaGetLastError();
 }
 

@@ -69,6 +69,16 @@ __device__ __forceinline__ void mma_pair_warp(uint32_t d_tmem, uint64_t a_desc, 
       "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
+// The same for 8-bit operands (kind::f8f6f4: e4m3 / e5m2 A and B, K = 32 per instruction).
+__device__ __forceinline__ void mma_pair_f8_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
 __device__ __forceinline__ void mma_commit_pair_warp(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
