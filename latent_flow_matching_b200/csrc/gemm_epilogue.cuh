@@ -1,7 +1,10 @@
 // Fused epilogue shared by the one-CTA (gemm_tc.cu) and CTA-pair (gemm_tc2.cu) tcgen05 GEMMs.
 //
 // Called by one epilogue warp for one accumulator tile; thread i of the warp owns accumulator
-// row m (global row of this problem) whose BN fp32 columns start at TMEM address `tbase`.
+// row m (global row of this problem) whose BN fp32 columns start at TMEM address `tbase`.  With
+// kParts > 1 the tile's columns are shared by kParts warps of the same lane quarter and this call
+// handles part `part`: a contiguous 1/kParts of the columns (of the a/b pairs for SwiGLU, of the
+// 128-wide heads for the fused QK-RMSNorm).
 // Every tcgen05.ld is warp-collective, so rows outside the problem still load and only skip
 // their global stores.
 #pragma once
@@ -27,23 +30,25 @@ __device__ __forceinline__ void scale_chunk(uint32_t (&r)[32], float sa, const f
   }
 }
 
-template <int BN, bool kScale = false>
-__device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32_t tbase, int m, int n0) {
+template <int BN, bool kScale = false, int kParts = 1>
+__device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32_t tbase, int m, int n0,
+                                                   int part = 0) {
+  static_assert(BN % (128 * kParts) == 0, "each part must hold whole 128-wide heads");
   const bool row_ok = m < pr.M;
+  // fp32 outputs whose rows start on 32-byte boundaries take 256-bit loads / stores
+  const bool v8_ok = ((reinterpret_cast<uintptr_t>(pr.out) | (static_cast<uintptr_t>(pr.ldo) * 4)) & 31) == 0;
   float sa = 0.f;                          // row scale (kScale only; rows outside the problem read none)
   if constexpr (kScale) sa = row_ok ? __ldg(pr.scale_a + m) : 0.f;
   if (pr.mode == kEpiSwiGLU) {
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(pr.out);
     const int on0 = n0 / 2;                // output column of this tile's first pair
 #pragma unroll 1
-    for (int c = 0; c < BN / 2; c += 32) {
+    for (int c = part * (BN / 2 / kParts); c < (part + 1) * (BN / 2 / kParts); c += 32) {
       uint32_t ra[32], rb[32];
       tmem_ld32(tbase + c, ra);
       tmem_ld32(tbase + BN / 2 + c, rb);
       tmem_ld_wait();
       if (row_ok && n0 + c < pr.N) {
-        scale_chunk<kScale>(ra, sa, pr.scale_b + n0 + c);
-        scale_chunk<kScale>(rb, sa, pr.scale_b + n0 + BN / 2 + c);
         const uint4* ba = reinterpret_cast<const uint4*>(pr.bias + n0 + c);
         const uint4* bb = reinterpret_cast<const uint4*>(pr.bias + n0 + BN / 2 + c);
         uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(m) * pr.ldo + on0 + c);
@@ -51,14 +56,29 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
         for (int v = 0; v < 4; ++v) {
           const uint4 wa = __ldg(ba + v), wb = __ldg(bb + v);
           const uint32_t xa[4] = {wa.x, wa.y, wa.z, wa.w}, xb[4] = {wb.x, wb.y, wb.z, wb.w};
+          float fa[8], fb[8];                        // accumulators of these 8 columns, scaled (kScale)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            fa[e] = __uint_as_float(ra[v * 8 + e]);
+            fb[e] = __uint_as_float(rb[v * 8 + e]);
+          }
+          if constexpr (kScale) {
+            const float4* sa4 = reinterpret_cast<const float4*>(pr.scale_b + n0 + c + v * 8);
+            const float4* sb4 = reinterpret_cast<const float4*>(pr.scale_b + n0 + BN / 2 + c + v * 8);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float4 ka = __ldg(sa4 + h), kb = __ldg(sb4 + h);
+              fa[4 * h] *= sa * ka.x; fa[4 * h + 1] *= sa * ka.y; fa[4 * h + 2] *= sa * ka.z; fa[4 * h + 3] *= sa * ka.w;
+              fb[4 * h] *= sa * kb.x; fb[4 * h + 1] *= sa * kb.y; fb[4 * h + 2] *= sa * kb.z; fb[4 * h + 3] *= sa * kb.w;
+            }
+          }
           uint32_t o[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int j = v * 8 + e * 2;
-            const float a0 = __uint_as_float(ra[j]) + bf16lo(xa[e]);
-            const float a1 = __uint_as_float(ra[j + 1]) + bf16hi(xa[e]);
-            const float b0 = __uint_as_float(rb[j]) + bf16lo(xb[e]);
-            const float b1 = __uint_as_float(rb[j + 1]) + bf16hi(xb[e]);
+            const float a0 = fa[2 * e] + bf16lo(xa[e]);
+            const float a1 = fa[2 * e + 1] + bf16hi(xa[e]);
+            const float b0 = fb[2 * e] + bf16lo(xb[e]);
+            const float b1 = fb[2 * e + 1] + bf16hi(xb[e]);
             o[e] = pack_bf16x2(silu_f(a0) * b0, silu_f(a1) * b1);
           }
           dst[v] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -71,7 +91,7 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
     const float4* rrow = reinterpret_cast<const float4*>(pr.rope + static_cast<size_t>(pr.rope_row0 + (row_ok ? m : 0)) * 64);
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(pr.out);
 #pragma unroll 1
-    for (int hh = 0; hh < BN / 128; ++hh) {
+    for (int hh = part * (BN / 128 / kParts); hh < (part + 1) * (BN / 128 / kParts); ++hh) {
       const uint32_t hb = tbase + hh * 128;
       const __nv_bfloat16* bh = pr.bias + n0 + hh * 128;
       float ss = 0.f;
@@ -126,7 +146,7 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
     }
   } else {
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = part * (BN / kParts); c < (part + 1) * (BN / kParts); c += 32) {
       uint32_t r[32];
       tmem_ld32(tbase + c, r);
       tmem_ld_wait();
@@ -153,9 +173,34 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
           dst[v] = make_uint4(pack_bf16x2(f[v * 8 + 0], f[v * 8 + 1]), pack_bf16x2(f[v * 8 + 2], f[v * 8 + 3]),
                               pack_bf16x2(f[v * 8 + 4], f[v * 8 + 5]), pack_bf16x2(f[v * 8 + 6], f[v * 8 + 7]));
       } else if (pr.mode == kEpiF32Bias) {
-        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(pr.out) + static_cast<size_t>(m) * pr.ldo + n);
+        float* dstp = static_cast<float*>(pr.out) + static_cast<size_t>(m) * pr.ldo + n;
+        if (v8_ok) {                        // one 32-byte access per 8 values: half the L1 wavefronts
 #pragma unroll
-        for (int v = 0; v < 8; ++v) dst[v] = make_float4(f[v * 4], f[v * 4 + 1], f[v * 4 + 2], f[v * 4 + 3]);
+          for (int v = 0; v < 4; ++v) st_global_v8(dstp + 8 * v, f + 8 * v);
+        } else {
+          float4* dst = reinterpret_cast<float4*>(dstp);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) dst[v] = make_float4(f[v * 4], f[v * 4 + 1], f[v * 4 + 2], f[v * 4 + 3]);
+        }
+      } else if (v8_ok) {                   // kEpiResidGate, 32-byte accesses
+        float* xp = static_cast<float*>(pr.out) + static_cast<size_t>(m) * pr.ldo + n;
+        const float4* g = reinterpret_cast<const float4*>(pr.gate + n);
+        float xv[4][8];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) ld_global_v8(xp + 8 * v, xv[v]);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const float4 g0 = __ldg(g + 2 * v), g1 = __ldg(g + 2 * v + 1);
+          xv[v][0] = fmaf(g0.x, f[8 * v + 0], xv[v][0]);
+          xv[v][1] = fmaf(g0.y, f[8 * v + 1], xv[v][1]);
+          xv[v][2] = fmaf(g0.z, f[8 * v + 2], xv[v][2]);
+          xv[v][3] = fmaf(g0.w, f[8 * v + 3], xv[v][3]);
+          xv[v][4] = fmaf(g1.x, f[8 * v + 4], xv[v][4]);
+          xv[v][5] = fmaf(g1.y, f[8 * v + 5], xv[v][5]);
+          xv[v][6] = fmaf(g1.z, f[8 * v + 6], xv[v][6]);
+          xv[v][7] = fmaf(g1.w, f[8 * v + 7], xv[v][7]);
+          st_global_v8(xp + 8 * v, xv[v]);
+        }
       } else {                              // kEpiResidGate
         float4* x = reinterpret_cast<float4*>(static_cast<float*>(pr.out) + static_cast<size_t>(m) * pr.ldo + n);
         const float4* g = reinterpret_cast<const float4*>(pr.gate + n);

@@ -8,13 +8,17 @@
 // the accumulator into CTA r's tensor memory.  Compared with one CTA per 128 x 256 tile, every
 // instruction does twice the work and each SM stages half as many W bytes per FLOP.
 //
-// Roles per CTA (6 warps, same as the one-CTA kernel): warp 0 TMA producer, warp 1 MMA issuer
-// (leader CTA only, one elected lane of a convergent warp) and TMEM allocator, warps 2..5 epilogue of this CTA's 128 accumulator rows.
+// Roles per CTA (10 warps): warp 0 TMA producer, warp 1 MMA issuer (leader CTA only, one elected
+// lane of a convergent warp) and TMEM allocator, warps 2..9 epilogue of this CTA's 128 accumulator
+// rows: two warps per TMEM lane quarter, each draining half of the tile's 256 columns (one 128-wide
+// head for the fused QK-RMSNorm, half of the a/b pairs for SwiGLU).  With 8-bit operands a tile's
+// MMAs take half as long, and four epilogue warps could not empty an accumulator before the other
+// one was full.
 // Barrier protocol:
 //   full[s]      leader only: 2 arrivals (one expect_tx from each CTA's producer) + the bytes
 //   empty[s]     both CTAs: the leader's MMA commit multicasts one arrival to each
 //   acc_full[a]  both CTAs: multicast commit after a tile's last MMA
-//   acc_empty[a] leader only: 8 arrivals (4 epilogue warps of each CTA)
+//   acc_empty[a] leader only: 16 arrivals (8 epilogue warps of each CTA)
 // The epilogue modes are those of the one-CTA kernel (gemm_tc.cu).
 #include "common.cuh"
 #include "fluxdit_internal.h"
@@ -35,6 +39,8 @@ constexpr int A_BYTES = 128 * BK * 2;          // 16 KB
 constexpr int B_BYTES = 128 * BK * 2;          // 16 KB (this CTA's half of W)
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * BN;              // double-buffered 128 x 256 fp32 accumulator per CTA
+constexpr int kEpiWarps = 8;                   // two per TMEM lane quarter
+constexpr int kThreads2 = 32 * (2 + kEpiWarps);
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512;
 
 __device__ __forceinline__ int find_problem(const GemmParams& P, int tile) {
@@ -48,7 +54,7 @@ __device__ __forceinline__ int find_problem(const GemmParams& P, int tile) {
 // kFp8: e4m3 operands, 128 per 128-byte swizzle row (BK = 128 elements per stage, the same bytes
 // as 64 bf16), kind::f8f6f4 MMAs with K = 32, and the epilogue applies the row / column scales.
 template <bool kFp8>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     gemm_bf16_tc2_kernel(const __grid_constant__ GemmParams P) {
   constexpr int BKE = kFp8 ? 2 * BK : BK;           // K elements per stage
   extern __shared__ uint8_t smem_raw[];
@@ -76,7 +82,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 8);
+      mbar_init(&acc_empty[a], 2 * kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -186,8 +192,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       mbar_drain(drain, 0);
     }
   } else {
-    // -------------------------------------------------------------- epilogue warps 2..5 (both CTAs)
-    const int quarter = warp & 3;
+    // -------------------------------------------------------------- epilogue warps 2..9 (both CTAs)
+    const int quarter = warp & 3;                   // the TMEM lane quarter this warp may read
+    const int part = (warp - 2) / 4;                // which half of the tile's columns
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t acc_empty_leader[2] = {map_to_rank(&acc_empty[0], 0), map_to_rank(&acc_empty[1], 0)};
@@ -205,7 +212,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(acc * BN);
-      gemm_epilogue_tile<BN, kFp8>(pr, tbase, m, n0);
+      gemm_epilogue_tile<BN, kFp8, 2>(pr, tbase, m, n0, part);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader[acc]);
@@ -260,9 +267,9 @@ cudaError_t gemm2_launch(GemmParams& P, int num_sms, cudaStream_t stream, bool f
   if (pairs > total) pairs = total;
   count_launch();
   if (fp8)
-    gemm_bf16_tc2_kernel<true><<<2 * pairs, 192, SMEM_BYTES, stream>>>(P);
+    gemm_bf16_tc2_kernel<true><<<2 * pairs, kThreads2, SMEM_BYTES, stream>>>(P);
   else
-    gemm_bf16_tc2_kernel<false><<<2 * pairs, 192, SMEM_BYTES, stream>>>(P);
+    gemm_bf16_tc2_kernel<false><<<2 * pairs, kThreads2, SMEM_BYTES, stream>>>(P);
   return cudaGetLastError();
 }
 
