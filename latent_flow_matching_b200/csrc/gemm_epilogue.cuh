@@ -30,6 +30,18 @@ __device__ __forceinline__ void scale_chunk(uint32_t (&r)[32], float sa, const f
   }
 }
 
+// 32 bf16 values (16 packed words) of one row: two 32-byte stores when aligned, else four 16-byte ones.
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t (&w)[16], bool v8) {
+  if (v8) {
+    st_global_v8(reinterpret_cast<uint32_t*>(dst), w);
+    st_global_v8(reinterpret_cast<uint32_t*>(dst) + 8, w + 8);
+  } else {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) d[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+  }
+}
+
 template <int BN, bool kScale = false, int kParts = 1>
 __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32_t tbase, int m, int n0,
                                                    int part = 0) {
@@ -37,6 +49,7 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
   const bool row_ok = m < pr.M;
   // fp32 outputs whose rows start on 32-byte boundaries take 256-bit loads / stores
   const bool v8_ok = ((reinterpret_cast<uintptr_t>(pr.out) | (static_cast<uintptr_t>(pr.ldo) * 4)) & 31) == 0;
+  const bool v8b_ok = ((reinterpret_cast<uintptr_t>(pr.out) | (static_cast<uintptr_t>(pr.ldo) * 2)) & 31) == 0;
   float sa = 0.f;                          // row scale (kScale only; rows outside the problem read none)
   if constexpr (kScale) sa = row_ok ? __ldg(pr.scale_a + m) : 0.f;
   if (pr.mode == kEpiSwiGLU) {
@@ -51,7 +64,8 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
       if (row_ok && n0 + c < pr.N) {
         const uint4* ba = reinterpret_cast<const uint4*>(pr.bias + n0 + c);
         const uint4* bb = reinterpret_cast<const uint4*>(pr.bias + n0 + BN / 2 + c);
-        uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(m) * pr.ldo + on0 + c);
+        __nv_bfloat16* dstp = out + static_cast<size_t>(m) * pr.ldo + on0 + c;
+        uint32_t ob[16];                             // this chunk's 32 outputs, packed
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const uint4 wa = __ldg(ba + v), wb = __ldg(bb + v);
@@ -81,8 +95,10 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
             const float b1 = fb[2 * e + 1] + bf16hi(xb[e]);
             o[e] = pack_bf16x2(silu_f(a0) * b0, silu_f(a1) * b1);
           }
-          dst[v] = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) ob[4 * v + e] = o[e];
         }
+        store_bf16x32(dstp, ob, v8b_ok);
       }
     }
   } else if (pr.mode == kEpiQKNormRope && n0 < 2 * (pr.N / 3)) {
@@ -124,7 +140,8 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
         scale_chunk<kScale>(r, sa, pr.scale_b + n0 + hh * 128 + c);
         const uint4* bsrc = reinterpret_cast<const uint4*>(bh + c);
         const uint4* gsrc = reinterpret_cast<const uint4*>(gain + c);
-        uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(m) * pr.ldo + n0 + hh * 128 + c);
+        __nv_bfloat16* dstp = out + static_cast<size_t>(m) * pr.ldo + n0 + hh * 128 + c;
+        uint32_t ob[16];
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const uint4 w = __ldg(bsrc + v), g = __ldg(gsrc + v);
@@ -140,8 +157,10 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
             const float a1 = (__uint_as_float(r[v * 8 + e * 2 + 1]) + bf16hi(x[e])) * rstd * bf16hi(gg[e]);
             o[e] = pack_bf16x2(a0 * cs[e] - a1 * sn[e], a0 * sn[e] + a1 * cs[e]);
           }
-          dst[v] = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) ob[4 * v + e] = o[e];
         }
+        store_bf16x32(dstp, ob, v8b_ok);
       }
     }
   } else {
@@ -166,12 +185,10 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
         }
       }
       if (pr.mode == kEpiBf16Bias || pr.mode == kEpiQKNormRope) {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(pr.out) +
-                                              static_cast<size_t>(m) * pr.ldo + n);
+        uint32_t ob[16];
 #pragma unroll
-        for (int v = 0; v < 4; ++v)
-          dst[v] = make_uint4(pack_bf16x2(f[v * 8 + 0], f[v * 8 + 1]), pack_bf16x2(f[v * 8 + 2], f[v * 8 + 3]),
-                              pack_bf16x2(f[v * 8 + 4], f[v * 8 + 5]), pack_bf16x2(f[v * 8 + 6], f[v * 8 + 7]));
+        for (int e = 0; e < 16; ++e) ob[e] = pack_bf16x2(f[2 * e], f[2 * e + 1]);
+        store_bf16x32(static_cast<__nv_bfloat16*>(pr.out) + static_cast<size_t>(m) * pr.ldo + n, ob, v8b_ok);
       } else if (pr.mode == kEpiF32Bias) {
         float* dstp = static_cast<float*>(pr.out) + static_cast<size_t>(m) * pr.ldo + n;
         if (v8_ok) {                        // one 32-byte access per 8 values: half the L1 wavefronts
