@@ -451,7 +451,8 @@ def run_ours(args, w):
     a_ms, a_fl, a_by, a_n = prof["attention"]
     gemm_tflops = g_fl / (g_ms / 1e3) / 1e12
     attn_tflops = a_fl / (a_ms / 1e3) / 1e12
-    traffic_per_gflop, src_sha = profile_traffic(GEMM_TRAFFIC_SOURCES, "gemm_tc2_t2i1024.md")
+    traffic_per_gflop, src_sha = profile_traffic(GEMM_TRAFFIC_SOURCES,
+                                                 "gemm_tc2_fp8_t2i1024.md" if fp8 else "gemm_tc2_t2i1024.md")
     traffic = None if traffic_per_gflop is None else traffic_per_gflop * (g_fl / g_n) / 1e9
     kinds = {k: {"ms_per_forward": round(v_[0] / args.steps, 4), "launches_per_forward": v_[3] // args.steps,
                  "achieved": round((v_[1] / (v_[0] / 1e3) / 1e12) if v_[1] else (v_[2] / (v_[0] / 1e3) / 1e9), 1),
@@ -483,7 +484,7 @@ def run_ours(args, w):
                          "bound": "tensor",
                          "achieved": round(gemm_tflops, 1), "peak": round(gemm_peak, 1),
                          "unit": "TFLOP/s", "frac": round(gemm_tflops / gemm_peak, 4),
-                         "peak_kind": gemm_peak_kind, "traffic": None if fp8 else traffic,
+                         "peak_kind": gemm_peak_kind, "traffic": traffic,
                          "launches_per_forward": g_n // args.steps,
                          "share_of_step": round(g_ms / args.steps / ms_step, 3)},
             "attention": {"achieved": round(attn_tflops, 1), "unit": "TFLOP/s",
