@@ -37,7 +37,8 @@ Readings where the page is silent (each is listed in the design doc):
 * reference tokens use the image input projection; the reference stream of the per-mode
   blocks is all reference images together (they attend to one another);
 * block arithmetic (QK-RMSNorm gain per stream, biases, SwiGLU silu(a) * b, eps 1e-6) as in
-  the FLUX.2 single-stream block.
+  the FLUX.2 single-stream block; with ``hp["fp8"]`` its two linears are the row-wise FP8 ones
+  (the fp8r format of section "Hardwareanforderungen, Quantisierung und Inferenzlatenz").
 """
 from __future__ import annotations
 
@@ -75,14 +76,15 @@ def parallel_block(p, pre, x, shift, scale, gate, ang, hp, dtype=torch.float64):
     D = x.shape[1]
     F = (p[pre + "lin1.w"].shape[0] - 3 * D) // 2
     y = O.modulate(O.layer_norm(x, hp["eps_ln"]), shift, scale)
-    h = O.linear(y, O.weight(p, pre + "lin1.w", dtype), O.weight(p, pre + "lin1.b", dtype))
+    lin = O.block_linear(hp)                    # row-wise FP8 when hp["fp8"] (oracle/fp8_oracle.py)
+    h = lin(y, O.weight(p, pre + "lin1.w", dtype), O.weight(p, pre + "lin1.b", dtype))
     q, k, v, a, b = h.split([D, D, D, F, F], dim=1)
     q = O.rms_norm(O._heads(q, hp["heads"], hp["head_dim"]), O.weight(p, pre + "q_gain", dtype), hp["eps_rms"])
     k = O.rms_norm(O._heads(k, hp["heads"], hp["head_dim"]), O.weight(p, pre + "k_gain", dtype), hp["eps_rms"])
     v = O._heads(v, hp["heads"], hp["head_dim"])
     o = O.attention(O.apply_rope(q, ang), O.apply_rope(k, ang), v)
-    return x + gate * O.linear(torch.cat([o, O.silu(a) * b], dim=1),
-                               O.weight(p, pre + "lin2.w", dtype), O.weight(p, pre + "lin2.b", dtype))
+    return x + gate * lin(torch.cat([o, O.silu(a) * b], dim=1),
+                          O.weight(p, pre + "lin2.w", dtype), O.weight(p, pre + "lin2.b", dtype))
 
 
 def forward3(p, hp, img_tok, txt, t, grid_hw, ref_tok=None, ref_hw=(), t_target=None,
