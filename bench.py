@@ -334,8 +334,6 @@ def run_ours(args, w):
     del blob
     fp8 = args.precision == "fp8"
     if fp8:
-        if flux3:
-            raise SystemExit("--precision fp8 is implemented for the FLUX.2 workloads")
         model.set_precision(F.PRECISION_FP8)
     stream = torch.cuda.current_stream()
     dev = torch.device("cuda", local)

@@ -358,6 +358,10 @@ FLUX_API int flux3_dit_forward(flux3_dit *m, const float *img_tok, int grid_h, i
                                int n_txt, const float *ref_tok, int n_refs, const int *ref_grids, float t,
                                float t_target, float *v_out, void *stream);
 
+/* Precision of the block linears of later FLUX.3 forwards (linear1 / linear2 of the per-mode and
+ * joint blocks): FLUX_PRECISION_BF16 or FLUX_PRECISION_FP8, as flux_dit_set_precision. */
+FLUX_API int flux3_dit_set_precision(flux3_dit *m, int precision);
+
 /* Diagnostic: run only the first n_mode per-mode and n_joint joint blocks (-1 = all). */
 FLUX_API int flux3_dit_set_active_blocks(flux3_dit *m, int n_mode, int n_joint);
 

@@ -84,6 +84,7 @@ _SIGS = {
     "flux3_dit_destroy": (None, [_P]),
     "flux3_dit_forward": (_I, [_P, _P, _I, _I, _P, _I, _P, _I, ctypes.POINTER(ctypes.c_int), _F, _F, _P, _P]),
     "flux3_dit_set_active_blocks": (_I, [_P, _I, _I]),
+    "flux3_dit_set_precision": (_I, [_P, _I]),
     "flux3_dit_modulation_size": (_Z, [_P]),
     "flux3_dit_modulation": (_I, [_P, _F, _F, _P, _P]),
     "flux3_dit_profile": (_I, [_P, _I]),
@@ -300,6 +301,10 @@ class Flux3DiT:
 
     def set_active_blocks(self, n_mode=-1, n_joint=-1):
         _check(lib().flux3_dit_set_active_blocks(self._h, n_mode, n_joint))
+
+    def set_precision(self, precision):
+        """PRECISION_BF16 or PRECISION_FP8 (row-wise e4m3 block linears); see flux3_dit_set_precision."""
+        _check(lib().flux3_dit_set_precision(self._h, int(precision)))
 
     def modulation_size(self) -> int:
         return lib().flux3_dit_modulation_size(self._h)

@@ -124,7 +124,11 @@ bool read_header3(const void* blob, size_t bytes, Header3* h) {
 // One parallel block's weights (per-mode stream or joint block).
 struct BlockW3 {
   const bf16 *qkv_b, *mlp_b, *q_gain, *k_gain, *lin2_b;
+  const bf16 *w_lin1, *w_lin2;
   CUtensorMap m_qkv, m_mlp, m_lin2;
+  // FP8 precision: e4m3 codes of linear1 (qkv rows, SwiGLU rows) and linear2, row scales
+  CUtensorMap m8_qkv, m8_mlp, m8_lin2;
+  const float *s_qkv, *s_mlp, *s_lin2;
 };
 
 // Row ranges of the joint sequence: text | image | reference (all references together).
@@ -139,6 +143,12 @@ struct Workspace3 {
   RefGrids refs = {-1, {}, {}};
   CUtensorMap a_tokb, a_txtb, a_Yall, a_Yout, qkv;
   CUtensorMap a_Yseg[3], a_CCseg[3];
+  // FP8 precision: e4m3 LN-mod output (Y8, scale sY) and [O | H] (C8, scale sC per row)
+  size_t cap8 = 0;
+  uint8_t *Y8 = nullptr, *C8 = nullptr;
+  float *sY = nullptr, *sC = nullptr;
+  bool maps8 = false;
+  CUtensorMap a8_Yall, a8_Yseg[3], a8_CCseg[3];
 };
 
 // Offsets (in units of D floats) of the modulation vectors in the model's mods buffer.
@@ -163,6 +173,9 @@ struct flux3_dit {
   std::vector<fdit::BlockW3> mode;    // [3 i + stream], stream 0 text, 1 image, 2 reference
   std::vector<fdit::BlockW3> joint;
   int act_mode = 0, act_joint = 0;
+  int precision = FLUX_PRECISION_BF16;
+  uint8_t* w8 = nullptr;               // e4m3 block linears (allocated on the first switch to FP8)
+  float* w8_scale = nullptr;
   fdit::Workspace3 ws;
   fdit::Profiler prof;
 };
@@ -170,7 +183,16 @@ struct flux3_dit {
 namespace fdit {
 namespace {
 
+void free_ws3_fp8(Workspace3& w) {
+  cudaFree(w.Y8); cudaFree(w.C8); cudaFree(w.sY); cudaFree(w.sC);
+  w.Y8 = w.C8 = nullptr;
+  w.sY = w.sC = nullptr;
+  w.cap8 = 0;
+  w.maps8 = false;
+}
+
 void free_ws3(Workspace3& w) {
+  free_ws3_fp8(w);
   cudaFree(w.X); cudaFree(w.Y); cudaFree(w.QKV); cudaFree(w.CC); cudaFree(w.tokb); cudaFree(w.txtb);
   cudaFree(w.rope);
   w = Workspace3();
@@ -179,6 +201,8 @@ void free_ws3(Workspace3& w) {
 void destroy3(flux3_dit* m) {
   if (!m) return;
   free_ws3(m->ws);
+  cudaFree(m->w8);
+  cudaFree(m->w8_scale);
   cudaFree(m->wbuf);
   cudaFree(m->scratch);
   delete m;
@@ -260,6 +284,7 @@ int create3_impl(const void* blob, size_t blob_bytes, const flux3_dit_config* cf
   auto block = [&](BlockW3& bw, const std::string& p) {
     const bf16* l1 = W(p + "lin1.w");
     const bf16* l1b = W(p + "lin1.b");
+    bw.w_lin1 = l1; bw.w_lin2 = W(p + "lin2.w");
     bw.qkv_b = l1b; bw.mlp_b = l1b + 3 * D;
     bw.q_gain = W(p + "q_gain"); bw.k_gain = W(p + "k_gain"); bw.lin2_b = W(p + "lin2.b");
     wmap(&bw.m_qkv, l1, 3 * D, D);
@@ -277,6 +302,43 @@ int create3_impl(const void* blob, size_t blob_bytes, const flux3_dit_config* cf
   m->act_joint = c.n_joint;
   if (cudaStreamSynchronize(s) != cudaSuccess) return cleanup(FLUX_EIO, "weight upload failed (sync)");
   *out = m;
+  return FLUX_OK;
+}
+
+// FP8 copies of the GEMM A operands (LN-mod output and [O | H]) and their maps.
+int prepare3_fp8(flux3_dit* m, int nt, int ni, int nr) {
+  Workspace3& w = m->ws;
+  const flux3_dit_config& c = m->cfg;
+  const size_t D = c.hidden, F = c.mlp_hidden;
+  const size_t n = static_cast<size_t>(nt) + ni + nr;
+  if (n > w.cap8) {
+    free_ws3_fp8(w);
+    const bool ok = cudaMalloc(&w.Y8, n * D) == cudaSuccess && cudaMalloc(&w.C8, n * (D + F)) == cudaSuccess &&
+                    cudaMalloc(&w.sY, n * 4) == cudaSuccess && cudaMalloc(&w.sC, n * 4) == cudaSuccess;
+    if (!ok) {
+      free_ws3_fp8(w);
+      return fail(FLUX_ENOMEM, "FP8 workspace allocation for %zu tokens failed", n);
+    }
+    w.cap8 = n;
+  }
+  if (w.maps8) return FLUX_OK;
+  bool ok = true;
+  auto amap = [&](CUtensorMap* map, const uint8_t* base, size_t rows, size_t cols, uint64_t stride) {
+    if (rows == 0) {
+      memset(map, 0, sizeof(*map));
+      return;
+    }
+    ok &= make_tmap_u8(map, base, rows, cols, stride, 128);
+  };
+  const size_t row0[3] = {0, static_cast<size_t>(nt), static_cast<size_t>(nt) + ni};
+  const size_t rows[3] = {static_cast<size_t>(nt), static_cast<size_t>(ni), static_cast<size_t>(nr)};
+  amap(&w.a8_Yall, w.Y8, n, D, D);
+  for (int sg = 0; sg < 3; ++sg) {
+    amap(&w.a8_Yseg[sg], w.Y8 + row0[sg] * D, rows[sg], D, D);
+    amap(&w.a8_CCseg[sg], w.C8 + row0[sg] * (D + F), rows[sg], D + F, D + F);
+  }
+  if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an FP8 activation buffer");
+  w.maps8 = true;
   return FLUX_OK;
 }
 
@@ -302,7 +364,10 @@ int prepare_shape3(flux3_dit* m, int nt, int gh, int gw, const RefGrids& refs, c
   if (grow(&w.tokb, &w.cap_tok, (ni + nr) * c.in_ch) != cudaSuccess ||
       grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt, 1) * c.txt_dim) != cudaSuccess)
     return fail(FLUX_ENOMEM, "workspace allocation failed");
-  if (w.nt == nt && w.gh == gh && w.gw == gw && same_refs(w.refs, refs)) return FLUX_OK;
+  const bool fp8 = m->precision == FLUX_PRECISION_FP8;
+  if (w.nt == nt && w.gh == gh && w.gw == gw && same_refs(w.refs, refs))
+    return fp8 ? prepare3_fp8(m, nt, static_cast<int>(ni), static_cast<int>(nr)) : FLUX_OK;
+  w.maps8 = false;
 
   const uint64_t ldD = D * 2, ldC = (D + F) * 2;
   bool ok = true;
@@ -328,6 +393,47 @@ int prepare_shape3(flux3_dit* m, int nt, int gh, int gw, const RefGrids& refs, c
   if (rope_table_launch(w.rope, nt, gh, gw, refs, c.rope_theta, s) != cudaSuccess)
     return fail(FLUX_EIO, "rope table launch failed");
   w.nt = nt; w.gh = gh; w.gw = gw; w.refs = refs;
+  return fp8 ? prepare3_fp8(m, nt, static_cast<int>(ni), static_cast<int>(nr)) : FLUX_OK;
+}
+
+// Quantise every block linear (per-mode streams and joint blocks) to e4m3, one scale per row.
+int quantize3_block_weights(flux3_dit* m, cudaStream_t s) {
+  const flux3_dit_config& c = m->cfg;
+  const size_t D = c.hidden, F = c.mlp_hidden;
+  std::vector<BlockW3*> blocks;
+  for (BlockW3& b : m->mode) blocks.push_back(&b);
+  for (BlockW3& b : m->joint) blocks.push_back(&b);
+  const size_t r1 = 3 * D + 2 * F, r2 = D;
+  const size_t b1 = (r1 * D + 255) / 256 * 256, b2 = (r2 * (D + F) + 255) / 256 * 256;
+  const size_t s1 = (r1 + 63) / 64 * 64, s2 = (r2 + 63) / 64 * 64;
+  const size_t nb = blocks.size();
+  if (cudaMalloc(&m->w8, nb * (b1 + b2)) != cudaSuccess || cudaMalloc(&m->w8_scale, nb * (s1 + s2) * 4) != cudaSuccess) {
+    cudaFree(m->w8);
+    cudaFree(m->w8_scale);
+    m->w8 = nullptr;
+    m->w8_scale = nullptr;
+    return fail(FLUX_ENOMEM, "cudaMalloc of the FP8 weights failed");
+  }
+  bool ok = true;
+  for (size_t i = 0; i < nb; ++i) {
+    BlockW3& bw = *blocks[i];
+    uint8_t* q1 = m->w8 + i * (b1 + b2);
+    uint8_t* q2 = q1 + b1;
+    float* sc1 = m->w8_scale + i * (s1 + s2);
+    float* sc2 = sc1 + s1;
+    FD_CUDA(quantize_rows_launch(bw.w_lin1, static_cast<int>(D), static_cast<int>(r1), static_cast<int>(D), q1,
+                                 static_cast<int>(D), sc1, s));
+    FD_CUDA(quantize_rows_launch(bw.w_lin2, static_cast<int>(D + F), static_cast<int>(r2), static_cast<int>(D + F),
+                                 q2, static_cast<int>(D + F), sc2, s));
+    ok &= make_tmap_u8(&bw.m8_qkv, q1, 3 * D, D, D, 128);
+    ok &= make_tmap_u8(&bw.m8_mlp, q1 + 3 * D * D, 2 * F, D, D, 128);
+    ok &= make_tmap_u8(&bw.m8_lin2, q2, D, D + F, D + F, 128);
+    bw.s_qkv = sc1;
+    bw.s_mlp = sc1 + 3 * D;
+    bw.s_lin2 = sc2;
+  }
+  if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an FP8 weight tensor");
+  FD_CUDA(cudaStreamSynchronize(s));
   return FLUX_OK;
 }
 
@@ -437,11 +543,35 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
     As.seg_n[sg] = rows[sg];
     seg_flops += 4.0 * rows[sg] * static_cast<double>(rows[sg]) * D;
   }
+  // FP8 precision: block linears on e4m3 codes; LN-mod quantises its output, [O | H] is quantised
+  // (one scale per row) before linear2
+  const bool fp8 = m->precision == FLUX_PRECISION_FP8;
+  auto f8 = [&](int i, const CUtensorMap& a8, const CUtensorMap& w8, const float* sa, const float* sb) {
+    P.mapA[i] = a8;
+    P.mapB[i] = w8;
+    P.prob[i].scale_a = sa;
+    P.prob[i].scale_b = sb;
+  };
+  auto ln3 = [&](const float* sh0, const float* sc0, const float* sh1, const float* sc1, const float* sh2,
+                 const float* sc2) -> int {
+    if (fp8)
+      FD_LAUNCH(m, kProfLnMod, 0, 5.0 * n * D + 4.0 * n,
+                ln_modulate_fp8_launch(w.X, w.Y8, w.sY, n, D, nt, nt + ni, n, sh0, sc0, sh1, sc1, sh2, sc2, eps_ln,
+                                       s));
+    else
+      FD_LAUNCH(m, kProfLnMod, 0, ln_bytes,
+                ln_modulate3_launch(w.X, w.Y, n, D, nt, nt + ni, n, sh0, sc0, sh1, sc1, sh2, sc2, eps_ln, s));
+    return FLUX_OK;
+  };
+  auto quant_cc = [&]() -> int {
+    FD_LAUNCH(m, kProfOther, 0, 3.0 * n * (D + F) + 4.0 * n,
+              quantize_rows_launch(w.CC, D + F, n, D + F, w.C8, D + F, w.sC, s));
+    return FLUX_OK;
+  };
   const int mode_set[3] = {kModTxt, kModImg, kModRef};
   for (int i = 0; i < m->act_mode; ++i) {
-    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes,
-              ln_modulate3_launch(w.X, w.Y, n, D, nt, nt + ni, n, md(kModTxt), md(kModTxt + 1), md(kModImg),
-                                  md(kModImg + 1), md(kModRef), md(kModRef + 1), eps_ln, s));
+    rc = ln3(md(kModTxt), md(kModTxt + 1), md(kModImg), md(kModImg + 1), md(kModRef), md(kModRef + 1));
+    if (rc) return rc;
     P.num_problems = 6;
     for (int sg = 0; sg < 3; ++sg) {
       const BlockW3& bw = m->mode[3 * i + sg];
@@ -450,16 +580,22 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
       qk_fuse(P, 2 * sg, bw.q_gain, bw.k_gain, w.rope, row0[sg], eps_rms);
       problem(P, 2 * sg + 1, w.a_Yseg[sg], bw.m_mlp, rows[sg], 2 * F, D, kEpiSwiGLU,
               w.CC + static_cast<size_t>(row0[sg]) * (D + F) + D, D + F, bw.mlp_b, nullptr);
+      if (fp8) {
+        f8(2 * sg, w.a8_Yseg[sg], bw.m8_qkv, w.sY + row0[sg], bw.s_qkv);
+        f8(2 * sg + 1, w.a8_Yseg[sg], bw.m8_mlp, w.sY + row0[sg], bw.s_mlp);
+      }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
     FD_LAUNCH(m, kProfAttention, seg_flops, 8.0 * n * D, attention_launch(As, s));
+    if (fp8 && (rc = quant_cc())) return rc;
     P.num_problems = 3;
     for (int sg = 0; sg < 3; ++sg) {
       const BlockW3& bw = m->mode[3 * i + sg];
       problem(P, sg, w.a_CCseg[sg], bw.m_lin2, rows[sg], D, D + F, kEpiResidGate,
               w.X + static_cast<size_t>(row0[sg]) * D, D, bw.lin2_b, md(mode_set[sg] + 2));
+      if (fp8) f8(sg, w.a8_CCseg[sg], bw.m8_lin2, w.sC + row0[sg], bw.s_lin2);
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
   }
 
   // ---------------- joint blocks: one weight set, attention over the whole sequence, modulation per token type
@@ -467,22 +603,28 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
   const double at_flops = 4.0 * n * static_cast<double>(n) * D;
   for (int i = 0; i < m->act_joint; ++i) {
     const BlockW3& bw = m->joint[i];
-    FD_LAUNCH(m, kProfLnMod, 0, ln_bytes,
-              ln_modulate3_launch(w.X, w.Y, n, D, nt, nt + ni, n, md(kModJointCtx), md(kModJointCtx + 1),
-                                  md(kModJointImg), md(kModJointImg + 1), md(kModJointCtx), md(kModJointCtx + 1),
-                                  eps_ln, s));
+    rc = ln3(md(kModJointCtx), md(kModJointCtx + 1), md(kModJointImg), md(kModJointImg + 1), md(kModJointCtx),
+             md(kModJointCtx + 1));
+    if (rc) return rc;
     P.num_problems = 2;
     problem(P, 0, w.a_Yall, bw.m_qkv, n, 3 * D, D, kEpiBf16Bias, w.QKV, 3 * D, bw.qkv_b, nullptr);
     qk_fuse(P, 0, bw.q_gain, bw.k_gain, w.rope, 0, eps_rms);
     problem(P, 1, w.a_Yall, bw.m_mlp, n, 2 * F, D, kEpiSwiGLU, w.CC + D, D + F, bw.mlp_b, nullptr);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+    if (fp8) {
+      f8(0, w.a8_Yall, bw.m8_qkv, w.sY, bw.s_qkv);
+      f8(1, w.a8_Yall, bw.m8_mlp, w.sY, bw.s_mlp);
+    }
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
     A.n = n;
     FD_LAUNCH(m, kProfAttention, at_flops, 8.0 * n * D, attention_launch(A, s));
+    if (fp8 && (rc = quant_cc())) return rc;
     P.num_problems = 3;
-    for (int sg = 0; sg < 3; ++sg)
+    for (int sg = 0; sg < 3; ++sg) {
       problem(P, sg, w.a_CCseg[sg], bw.m_lin2, rows[sg], D, D + F, kEpiResidGate,
               w.X + static_cast<size_t>(row0[sg]) * D, D, bw.lin2_b, md(joint_set[sg] + 2));
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+      if (fp8) f8(sg, w.a8_CCseg[sg], bw.m8_lin2, w.sC + row0[sg], bw.s_lin2);
+    }
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
   }
 
   // ---------------- output layer on the image rows (text and reference tokens are dropped)
@@ -538,6 +680,28 @@ int flux3_dit_forward(flux3_dit* m, const float* img_tok, int grid_h, int grid_w
   if (rc) return rc;
   return forward3_impl(m, img_tok, grid_h, grid_w, txt, n_txt, ref_tok, refs, t, t_target, v_out,
                        static_cast<cudaStream_t>(stream));
+}
+
+int flux3_dit_set_precision(flux3_dit* m, int precision) {
+  if (!m) return fail(FLUX_EINVAL, "model is NULL");
+  if (precision == FLUX_PRECISION_BF16) {
+    m->precision = precision;
+    return FLUX_OK;
+  }
+  if (precision != FLUX_PRECISION_FP8) return fail(FLUX_EINVAL, "unknown precision %d", precision);
+  const flux3_dit_config& c = m->cfg;
+  if ((c.hidden != 1024 && c.hidden != 2048 && c.hidden != 3072 && c.hidden != 4096) ||
+      c.hidden + c.mlp_hidden > 16384)
+    return fail(FLUX_EINVAL, "FP8 needs hidden in {1024, 2048, 3072, 4096} and hidden + mlp_hidden <= 16384");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != m->device) return fail(FLUX_EINVAL, "model lives on device %d, current device is %d", m->device, dev);
+  if (!m->w8) {
+    const int rc = quantize3_block_weights(m, nullptr);
+    if (rc) return rc;
+  }
+  m->precision = precision;
+  return FLUX_OK;
 }
 
 int flux3_dit_set_active_blocks(flux3_dit* m, int n_mode, int n_joint) {

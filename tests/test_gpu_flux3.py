@@ -236,3 +236,47 @@ def test_flux3_workload_against_oracle_goldens(name):
     finally:
         model.close()
     assert F.flux_device_error() == 0
+
+
+# ---------------------------------------------------------------------------- row-wise FP8 block linears
+@pytest.mark.parametrize("nt,grid,ref_grids", [(16, (4, 4), [(4, 4)]), (131, (8, 8), [(4, 8), (4, 4)]),
+                                               (0, (4, 6), [])])
+def test_tiny3_fp8_forward_against_fp8_oracle(tiny3, nt, grid, ref_grids):
+    """FP8 per-mode and joint linears against the oracle's FP8 forward (bar 2e-2, as for FLUX.2);
+    switching back to bf16 gives the bf16 result bit for bit."""
+    w, p, model = tiny3
+    tok, txt, refs = _tiny_inputs(300 + nt, nt, grid, ref_grids)
+    hq = dict(O.hyper(w.dims), fp8=True)
+    want = O3.forward3(p, hq, tok, txt, 0.6, grid, refs, ref_grids, t_target=0.35)
+    v16 = _gpu_forward(model, tok, grid, txt, 0.6, refs, ref_grids, 0.35)
+    model.set_precision(F.PRECISION_FP8)
+    try:
+        v8 = _gpu_forward(model, tok, grid, txt, 0.6, refs, ref_grids, 0.35)
+    finally:
+        model.set_precision(F.PRECISION_BF16)
+    assert rel_l2(v8, want) <= V_TOL, rel_l2(v8, want)
+    again = _gpu_forward(model, tok, grid, txt, 0.6, refs, ref_grids, 0.35)
+    assert torch.equal(again, v16)
+    assert F.flux_device_error() == 0
+
+
+def test_flux3_fp8_full_size_against_bf16():
+    """FLUX.3 1024^2 workload, full model: the FP8 forward stays within a few percent of the bf16 one."""
+    w = WORKLOADS["f3t2i1024"]
+    blob, _ = make_weights(w.dims, w.seed)
+    lat, txt, _ = make_inputs(w)
+    model = F.Flux3DiT(blob, w.dims)
+    del blob
+    try:
+        tok = O.pack_latents(torch.from_numpy(lat)).float().to(DEV)
+        tx = torch.from_numpy(txt).to(DEV)
+        v16, v8 = torch.empty(w.n_img, 128, device=DEV), torch.empty(w.n_img, 128, device=DEV)
+        model.forward(tok, (w.grid, w.grid), tx, 1.0, v16, t_target=15 / 16)
+        model.set_precision(F.PRECISION_FP8)
+        model.forward(tok, (w.grid, w.grid), tx, 1.0, v8, t_target=15 / 16)
+        torch.cuda.synchronize()
+        err = rel_l2(v8, v16)
+        assert 1e-3 < err < 0.1, err
+    finally:
+        model.close()
+    assert F.flux_device_error() == 0
