@@ -657,7 +657,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
     problem(P, 2 * b + 1, w.a_tokb, m->m_img_in, nimg, D, c.in_ch, kEpiF32Bias, w.X + seq_row(b, nt) * D, D,
             m->img_b, nullptr);
   }
-  FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+  FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, false, nb));
 
   AttnParams A;
   A.mapQ = w.qkv; A.mapK = w.qkv; A.mapV = w.qkv;
@@ -712,7 +712,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
         f8(2 * b + 1, w.a8_Yimg[b], si.m8_qkv, w.sY + seq_row(b, nt), si.s_qkv);
       }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
     FD_LAUNCH(m, kProfAttention, at_flops, at_bytes, attention_launch(A, s));
     if (fp8 && (rc = quant_cc(0, D, w.sO))) return rc;
     P.num_problems = 2 * nb;
@@ -726,7 +726,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
         f8(2 * b + 1, w.a8_Oimg[b], si.m8_proj, w.sO + seq_row(b, nt), si.s_proj);
       }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
     rc = ln_mod(nt, mt + 3 * D, mt + 4 * D, mi + 3 * D, mi + 4 * D);
     if (rc) return rc;
     P.num_problems = 2 * nb;
@@ -740,7 +740,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
         f8(2 * b + 1, w.a8_Yimg[b], si.m8_mlp_in, w.sY + seq_row(b, nt), si.s_mlp_in);
       }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
     if (fp8 && (rc = quant_cc(D, F, w.sH))) return rc;
     P.num_problems = 2 * nb;
     for (int b = 0; b < nb; ++b) {
@@ -753,7 +753,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
         f8(2 * b + 1, w.a8_Himg[b], si.m8_mlp_out, w.sH + seq_row(b, nt), si.s_mlp_out);
       }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
   }
   // single blocks: one set of weights for every row, so the whole batch is one problem
   for (int i = 0; i < m->act_single; ++i) {
@@ -769,13 +769,13 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
       f8(0, w.a8_Yall, sw.m8_qkv, w.sY, sw.s_qkv);
       f8(1, w.a8_Yall, sw.m8_mlp, w.sY, sw.s_mlp);
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
     FD_LAUNCH(m, kProfAttention, at_flops, at_bytes, attention_launch(A, s));
     if (fp8 && (rc = quant_cc(0, D + F, w.sC))) return rc;
     P.num_problems = 1;
     problem(P, 0, w.a_CC, sw.m_lin2, rows, D, D + F, kEpiResidGate, w.X, D, sw.lin2_b, ms + 2 * D);
     if (fp8) f8(0, w.a8_CC, sw.m8_lin2, w.sC, sw.s_lin2);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
   }
   // output layer on the image rows of each sequence
   const float* mf = mods + m->fin_mod_off;         // shift, scale

@@ -526,7 +526,7 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
   problem(P, 0, w.a_txtb, m->m_txt_in, nt, D, c.txt_dim, kEpiF32Bias, w.X, D, m->txt_b, nullptr);
   problem(P, 1, w.a_tokb, m->m_img_in, ni + nr, D, c.in_ch, kEpiF32Bias, w.X + static_cast<size_t>(nt) * D, D,
           m->img_b, nullptr);
-  FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s));
+  FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, false));
 
   AttnParams A;
   A.mapQ = w.qkv; A.mapK = w.qkv; A.mapV = w.qkv;
@@ -585,7 +585,7 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
         f8(2 * sg + 1, w.a8_Yseg[sg], bw.m8_mlp, w.sY + row0[sg], bw.s_mlp);
       }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8));
     FD_LAUNCH(m, kProfAttention, seg_flops, 8.0 * n * D, attention_launch(As, s));
     if (fp8 && (rc = quant_cc())) return rc;
     P.num_problems = 3;
@@ -595,7 +595,7 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
               w.X + static_cast<size_t>(row0[sg]) * D, D, bw.lin2_b, md(mode_set[sg] + 2));
       if (fp8) f8(sg, w.a8_CCseg[sg], bw.m8_lin2, w.sC + row0[sg], bw.s_lin2);
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8));
   }
 
   // ---------------- joint blocks: one weight set, attention over the whole sequence, modulation per token type
@@ -614,7 +614,7 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
       f8(0, w.a8_Yall, bw.m8_qkv, w.sY, bw.s_qkv);
       f8(1, w.a8_Yall, bw.m8_mlp, w.sY, bw.s_mlp);
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8));
     A.n = n;
     FD_LAUNCH(m, kProfAttention, at_flops, 8.0 * n * D, attention_launch(A, s));
     if (fp8 && (rc = quant_cc())) return rc;
@@ -624,7 +624,7 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
               w.X + static_cast<size_t>(row0[sg]) * D, D, bw.lin2_b, md(joint_set[sg] + 2));
       if (fp8) f8(sg, w.a8_CCseg[sg], bw.m8_lin2, w.sC + row0[sg], bw.s_lin2);
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8));
   }
 
   // ---------------- output layer on the image rows (text and reference tokens are dropped)
