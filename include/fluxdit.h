@@ -1,5 +1,6 @@
 /*
- * fluxdit.h -- C ABI of the B200 (sm_100a) FLUX.2-klein denoising transformer.
+ * fluxdit.h -- C ABI of the B200 (sm_100a) FLUX.2-klein denoising transformer
+ * (and of its FLUX.3 Image Klein variant, flux3_dit_*, further below).
  *
  * The library evaluates the velocity field of the FLUX.2-klein image generator
  * once per Euler flow-matching step: 5 double-stream blocks (separate text and
