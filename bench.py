@@ -374,6 +374,8 @@ def run_ours(args, w):
         k = i % w.n_steps
         if k == 0:
             lat_buf.copy_(lat0)                     # every sampling run starts from the same noise
+            if not flux3:                           # the run's modulation vectors, one weight pass per 4 steps
+                model.prepare_timesteps(ts[:-1])
         F.flux_pack_latents(lat_buf, tok)
         forward_update(k)
         F.flux_unpack_latents(tok, lat_buf)
@@ -424,6 +426,8 @@ def run_ours(args, w):
     e0.record(stream)
     for i in range(args.steps):
         k = i % w.n_steps
+        if k == 0 and not flux3:
+            model.prepare_timesteps(ts[:-1])
         lat_d.copy_(lat_pin if k == 0 else out_pin, non_blocking=True)
         txt.copy_(txt_pin, non_blocking=True)
         if guided:

@@ -162,6 +162,15 @@ FLUX_API int flux_dit_set_active_blocks(flux_dit *m, int n_double, int n_single)
 FLUX_API size_t flux_dit_modulation_size(const flux_dit *m);
 FLUX_API int flux_dit_modulation(flux_dit *m, float t, float *mods_out, void *stream);
 
+/* Compute the modulation vectors of n timesteps (a sampler's schedule, n <= 64, HOST array) in
+ * passes of up to four that read the time-MLP and modulation weights once per pass, and keep them:
+ * a later forward (or flux_dit_modulation) whose t equals one of them exactly uses the kept vector
+ * instead of computing it (the modulation linears read 2.3 GB of weights per forward at the
+ * default size; "Modulation pro Token-Typ, Flow-Map-Destillation und 4D-RoPE": shift, scale and
+ * gate depend on the timestep only).  A new call replaces the kept set; n = 0 clears it.  Uses a
+ * stream-ordered temporary allocation; the first call allocates the cache (64 vectors). */
+FLUX_API int flux_dit_prepare_timesteps(flux_dit *m, const float *ts, int n, void *stream);
+
 /* Euler flow-matching update x += dt * v over n fp32 values, in place
  * ("Flux 2 Klein: Reine C-basierte Inferenz", "Modellarchitektur und Leistung":
  * 4 sampling steps; t_i = linspace(1, 0, S+1), dt = t_{i+1} - t_i). */

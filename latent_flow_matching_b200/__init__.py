@@ -92,6 +92,7 @@ _SIGS = {
                                     ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]),
     "flux_joint_attention_segments": (_I, [_P, _P, _P, _P, _I, ctypes.POINTER(ctypes.c_int), _I, _I, _F, _P]),
     "flux_dit_set_precision": (_I, [_P, _I]),
+    "flux_dit_prepare_timesteps": (_I, [_P, ctypes.POINTER(ctypes.c_float), _I, _P]),
     "flux_quantize_rows_e4m3": (_I, [_P, _I, _I, _I, _P, _I, _P, _P]),
     "flux_layernorm_modulate_fp8": (_I, [_P, _P, _P, _I, _I, _P, _P, _F, _P]),
     "flux_linear_fp8": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _P, _I, _P, _I, _P, _P]),
@@ -223,6 +224,11 @@ class FluxDiT:
     def set_precision(self, precision):
         """PRECISION_BF16 or PRECISION_FP8 (row-wise e4m3 block linears); see flux_dit_set_precision."""
         _check(lib().flux_dit_set_precision(self._h, int(precision)))
+
+    def prepare_timesteps(self, ts, stream=None):
+        """Compute and keep the modulation vectors of these timesteps (see flux_dit_prepare_timesteps)."""
+        arr = (ctypes.c_float * max(1, len(ts)))(*[float(t) for t in ts])
+        _check(lib().flux_dit_prepare_timesteps(self._h, arr, len(ts), _stream(stream)))
 
     PROFILE_KINDS = ("gemm", "attention", "ln_mod", "qk_norm_rope", "gemv", "other")
 
@@ -555,6 +561,7 @@ def flux_sample(model: FluxDiT, latent, txt, n_steps, ref_latent=None, on_step=N
             row += h * w
         ref_hw = grids if isinstance(ref_latent, (list, tuple)) else grids[0]
     v = torch.empty_like(tok)
+    model.prepare_timesteps(ts[start:n_steps], stream)      # every step's modulation in one pass
     if guidance is not None:
         if txt_uncond is None:
             raise ValueError("guidance needs txt_uncond")

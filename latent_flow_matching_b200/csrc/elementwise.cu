@@ -446,7 +446,7 @@ cudaError_t timestep_embed_launch(float* temb, float t, int dim, cudaStream_t s)
 cudaError_t gemv_multi_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, const float* x, int nvec, float* y,
                               const float* add, int rows, int k, int silu_in, int silu_out, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  if (nvec < 1 || nvec > 2 || k % 8) return cudaErrorInvalidValue;
+  if (nvec < 1 || nvec > 4 || k % 8) return cudaErrorInvalidValue;
   const int per_block = kGemvWarps * kGemvRowsPerWarp;
   int grid = (rows + per_block - 1) / per_block;
   const int cap = num_sms_current() * 8;
@@ -456,8 +456,12 @@ cudaError_t gemv_multi_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, co
   count_launch();
   if (nvec == 1)
     gemv_kernel<1><<<grid, 256, smem, s>>>(W, b, x, y, add, rows, k, silu_in, silu_out);
-  else
+  else if (nvec == 2)
     gemv_kernel<2><<<grid, 256, smem, s>>>(W, b, x, y, add, rows, k, silu_in, silu_out);
+  else if (nvec == 3)
+    gemv_kernel<3><<<grid, 256, smem, s>>>(W, b, x, y, add, rows, k, silu_in, silu_out);
+  else
+    gemv_kernel<4><<<grid, 256, smem, s>>>(W, b, x, y, add, rows, k, silu_in, silu_out);
   return cudaGetLastError();
 }
 

@@ -221,6 +221,12 @@ struct flux_dit {
   bf16* mods_b = nullptr;
   size_t mods_rows = 0;
   float *temb = nullptr, *th = nullptr, *vec = nullptr, *mods = nullptr;
+  // modulation vectors of a sampler's timesteps, computed together by flux_dit_prepare_timesteps
+  static constexpr int kMaxCachedT = 64;
+  float* mods_cache = nullptr;          // [cache_n][mods_rows]
+  float cache_t[kMaxCachedT] = {};
+  int cache_n = 0;
+  const float* mods_cur = nullptr;      // the vector the current forward uses
   const bf16 *t_w1, *t_b1, *t_w2, *t_b2, *img_b, *txt_b, *fin_b;
   size_t fin_mod_off = 0;
   CUtensorMap m_img_in, m_txt_in, m_fin;
@@ -256,7 +262,7 @@ static void destroy(flux_dit* m) {
   free_ws(m->ws);
   cudaFree(m->wbuf); cudaFree(m->mods_w); cudaFree(m->mods_b);
   cudaFree(m->w8); cudaFree(m->w8_scale);
-  cudaFree(m->temb); cudaFree(m->th); cudaFree(m->vec); cudaFree(m->mods);
+  cudaFree(m->temb); cudaFree(m->th); cudaFree(m->vec); cudaFree(m->mods); cudaFree(m->mods_cache);
   delete m;
 }
 
@@ -587,6 +593,12 @@ static int quantize_block_weights(flux_dit* m, cudaStream_t s) {
 static int run_modulation(flux_dit* m, float t, cudaStream_t s) {
   const flux_dit_config& c = m->cfg;
   const int D = c.hidden;
+  for (int i = 0; i < m->cache_n; ++i)
+    if (m->cache_t[i] == t) {                 // prepared with the other timesteps of the sampler
+      m->mods_cur = m->mods_cache + static_cast<size_t>(i) * m->mods_rows;
+      return FLUX_OK;
+    }
+  m->mods_cur = m->mods;
   auto gv = [](double rows, double k) { return rows * k * 2 + rows * 6 + k * 4; };
   FD_LAUNCH(m, kProfOther, 0, c.t_freq_dim * 4.0, timestep_embed_launch(m->temb, t, c.t_freq_dim, s));
   FD_LAUNCH(m, kProfGemv, 2.0 * D * c.t_freq_dim, gv(D, c.t_freq_dim),
@@ -630,11 +642,11 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
   const int ni = gh * gw, nr = static_cast<int>(ref_tokens(refs)), nimg = ni + nr, n = nt + nimg;
   const int rows = n * nb;
   const float eps_ln = c.eps_ln, eps_rms = c.eps_rms;
-  const float* mods = m->mods;
   auto seq_row = [&](int b, int r) { return static_cast<size_t>(b) * n + r; };   // row r of sequence b
 
   rc = run_modulation(m, t, s);                   // one t, so one modulation vector for every sequence
   if (rc) return rc;
+  const float* mods = m->mods_cur;
   FD_LAUNCH(m, kProfOther, 0, 6.0 * ni * c.in_ch,
             cast_bf16_launch(img_tok, w.tokb, static_cast<size_t>(ni) * c.in_ch, s));
   if (nr)
@@ -903,6 +915,52 @@ int flux_dit_set_active_blocks(flux_dit* m, int n_double, int n_single) {
   return FLUX_OK;
 }
 
+int flux_dit_prepare_timesteps(flux_dit* m, const float* ts, int n, void* stream) {
+  if (!m) return fail(FLUX_EINVAL, "model is NULL");
+  if (n < 0 || n > flux_dit::kMaxCachedT || (n > 0 && !ts))
+    return fail(FLUX_EINVAL, "%d timesteps (0..%d, host array)", n, flux_dit::kMaxCachedT);
+  for (int i = 0; i < n; ++i)
+    if (!std::isfinite(ts[i])) return fail(FLUX_EINVAL, "timestep %d is not finite", i);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const flux_dit_config& c = m->cfg;
+  const int D = c.hidden, tf = c.t_freq_dim;
+  m->cache_n = 0;
+  if (n == 0) return FLUX_OK;
+  if (!m->mods_cache &&
+      cudaMalloc(&m->mods_cache, static_cast<size_t>(flux_dit::kMaxCachedT) * m->mods_rows * 4) != cudaSuccess)
+    return fail(FLUX_ENOMEM, "cudaMalloc of the modulation cache failed");
+  // up to four timesteps per pass: the embeddings, the time MLP and every modulation linear read
+  // their weights once for the group (the GEMV takes the group's vectors together)
+  float* temb = nullptr;
+  float* th = nullptr;
+  float* vec = nullptr;
+  const size_t scratch = 4 * (static_cast<size_t>(tf) + 2 * D);
+  if (cudaMallocAsync(&temb, scratch * sizeof(float), s) != cudaSuccess)
+    return fail(FLUX_ENOMEM, "cudaMallocAsync of the timestep scratch failed");
+  th = temb + 4 * tf;
+  vec = th + 4 * D;
+  auto gv = [](double rows, double k, double nvec) { return rows * k * 2 + nvec * (rows * 6 + k * 4); };
+  auto group = [&](int g, int k) -> int {
+    for (int i = 0; i < k; ++i)
+      FD_LAUNCH(m, kProfOther, 0, tf * 4.0, timestep_embed_launch(temb + i * tf, ts[g + i], tf, s));
+    FD_LAUNCH(m, kProfGemv, 2.0 * k * D * tf, gv(D, tf, k),
+              gemv_multi_launch(m->t_w1, m->t_b1, temb, k, th, nullptr, D, tf, 0, 1, s));
+    FD_LAUNCH(m, kProfGemv, 2.0 * k * D * D, gv(D, D, k),
+              gemv_multi_launch(m->t_w2, m->t_b2, th, k, vec, nullptr, D, D, 0, 0, s));
+    FD_LAUNCH(m, kProfGemv, 2.0 * k * m->mods_rows * D, gv(static_cast<double>(m->mods_rows), D, k),
+              gemv_multi_launch(m->mods_w, m->mods_b, vec, k, m->mods_cache + static_cast<size_t>(g) * m->mods_rows,
+                                nullptr, static_cast<int>(m->mods_rows), D, 1, 0, s));
+    return FLUX_OK;
+  };
+  int rc = FLUX_OK;
+  for (int g = 0; g < n && rc == FLUX_OK; g += 4) rc = group(g, std::min(4, n - g));
+  cudaFreeAsync(temb, s);
+  if (rc) return rc;
+  for (int i = 0; i < n; ++i) m->cache_t[i] = ts[i];
+  m->cache_n = n;
+  return FLUX_OK;
+}
+
 size_t flux_dit_modulation_size(const flux_dit* m) { return m ? m->mods_rows : 0; }
 
 int flux_dit_modulation(flux_dit* m, float t, float* mods_out, void* stream) {
@@ -910,7 +968,7 @@ int flux_dit_modulation(flux_dit* m, float t, float* mods_out, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int rc = run_modulation(m, t, s);
   if (rc) return rc;
-  FD_CUDA(cudaMemcpyAsync(mods_out, m->mods, m->mods_rows * sizeof(float), cudaMemcpyDeviceToDevice, s));
+  FD_CUDA(cudaMemcpyAsync(mods_out, m->mods_cur, m->mods_rows * sizeof(float), cudaMemcpyDeviceToDevice, s));
   return FLUX_OK;
 }
 

@@ -118,7 +118,7 @@ cudaError_t timestep_embed_launch(float* temb, float t, int dim, cudaStream_t s)
 // y[r] = act_out(sum_k W[r,k] * act_in(x[k]) + b[r]); W bf16 [rows, k], b bf16 [rows]
 cudaError_t gemv_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, const float* x, float* y, int rows,
                         int k, int silu_in, int silu_out, cudaStream_t s);
-// nvec (1 or 2) input vectors of k floats, one after another, against one read of W: output v is
+// nvec (1 to 4) input vectors of k floats, one after another, against one read of W: output v is
 // y[v * rows .. v * rows + rows); add (NULL or [rows]) is added before act_out.  nvec * k <= 12288.
 cudaError_t gemv_multi_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, const float* x, int nvec, float* y,
                               const float* add, int rows, int k, int silu_in, int silu_out, cudaStream_t s);

@@ -68,6 +68,37 @@ def test_tiny_modulation_vector(tiny):
         assert err <= K_TOL, err
 
 
+@pytest.mark.parametrize("n", [1, 3, 5])
+def test_prepared_timesteps_match_per_forward_modulation(tiny, n):
+    """Vectors computed together (up to four per weight read) equal, bit for bit, the ones a
+    forward computes alone; a forward at a prepared t gives the same velocity."""
+    w, p, model = tiny
+    ts = [float(np.float32(1.0 - i / 7)) for i in range(n)]
+    size = model.modulation_size()
+    alone = []
+    model.prepare_timesteps([])
+    for t in ts:
+        out = torch.empty(size, device=DEV)
+        model.modulation(t, out)
+        alone.append(out)
+    lat, txt, _ = make_inputs(w)
+    tok = O.pack_latents(torch.from_numpy(lat)).float().to(DEV)
+    v0 = torch.empty(w.n_img, 128, device=DEV)
+    model.forward(tok, (w.grid, w.grid), torch.from_numpy(txt).to(DEV), ts[-1], v0)
+    model.prepare_timesteps(ts)
+    try:
+        for t, ref in zip(ts, alone):
+            out = torch.empty(size, device=DEV)
+            model.modulation(t, out)
+            assert torch.equal(out, ref)
+        v1 = torch.empty_like(v0)
+        model.forward(tok, (w.grid, w.grid), torch.from_numpy(txt).to(DEV), ts[-1], v1)
+        assert torch.equal(v0, v1)
+    finally:
+        model.prepare_timesteps([])
+    assert F.flux_device_error() == 0
+
+
 @pytest.mark.parametrize("n_double,n_single", [(0, 0), (1, 0), (1, 1)])
 def test_tiny_forward_block_by_block(tiny, n_double, n_single):
     w, p, model = tiny
