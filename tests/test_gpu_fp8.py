@@ -234,3 +234,23 @@ def test_fp8_forward_full_size_against_bf16():
         assert 1e-3 < err < 0.1, err
     finally:
         model.close()
+
+
+def test_fp8_guided_batch_equals_two_single_forwards(tiny):
+    """The batch-2 guided forward in FP8 returns, bit for bit, the two single-text FP8 forwards:
+    every quantisation scale belongs to one row and the GEMM choice is made per sequence."""
+    w, p, model = tiny
+    g = torch.Generator().manual_seed(90)
+    grid = (6, 4)
+    tok = torch.randn(24, 128, generator=g).to(torch.bfloat16).float().to(DEV)
+    tc = torch.randn(131, 3072, generator=g).to(torch.bfloat16).float().to(DEV)
+    tu = torch.randn(131, 3072, generator=g).to(torch.bfloat16).float().to(DEV)
+    vc, vu, a, b = (torch.empty(24, 128, device=DEV) for _ in range(4))
+    model.set_precision(F.PRECISION_FP8)
+    try:
+        model.forward_cfg(tok, grid, tc, tu, 0.6, vc, vu)
+        model.forward(tok, grid, tc, 0.6, a)
+        model.forward(tok, grid, tu, 0.6, b)
+    finally:
+        model.set_precision(F.PRECISION_BF16)
+    assert torch.equal(vc, a) and torch.equal(vu, b)
