@@ -154,20 +154,36 @@ def forward3(p, hp, img_tok, txt, t, grid_hw, ref_tok=None, ref_hw=(), t_target=
     return O.linear(y, O.weight(p, "final.out.w", dtype), O.weight(p, "final.out.b", dtype))
 
 
-def sample3(p, hp, latent, txt, n_steps, ref_latent=None, dtype=torch.float64, on_step=None):
+def sample3(p, hp, latent, txt, n_steps, ref_latent=None, dtype=torch.float64, on_step=None,
+            init_latent=None, strength=1.0, txt_uncond=None, guidance=None):
     """Euler sampling with the FLUX.3 model; the flow-map checkpoint gets t_{i+1} as the target
-    time of step i.  Returns (final latent [32, h8, w8], list of velocities)."""
+    time of step i.  Returns (final latent [32, h8, w8], list of velocities).
+
+    ``init_latent`` / ``strength`` (image editing) and ``guidance`` / ``txt_uncond``
+    (classifier-free guidance, the base checkpoint's 50 steps at guidance 3.5 in the we0.ai
+    FLUX 3 Image Klein article's checkpoint table) follow the FLUX.2 sampler's readings:
+    start at schedule step img2img_start(S, strength) from blend_latents(init, noise, t_start);
+    every guided step evaluates the prompt and the unconditional text on the same image and
+    moves along guided_velocity (the returned velocities are the guided ones)."""
     latent = torch.as_tensor(latent).to(dtype)
     c, h8, w8 = latent.shape
     ts = O.schedule(n_steps)
+    start = 0
+    if init_latent is not None:
+        start = O.img2img_start(n_steps, strength)
+        latent = O.blend_latents(torch.as_tensor(init_latent).to(dtype), latent, ts[start])
     tok = O.pack_latents(latent)
     refs = [] if ref_latent is None else (list(ref_latent) if isinstance(ref_latent, (list, tuple)) else [ref_latent])
     ref_toks = [O.pack_latents(torch.as_tensor(r).to(dtype)) for r in refs]
     ref_grids = [(r.shape[1] // 2, r.shape[2] // 2) for r in refs]
     vs = []
-    for i in range(n_steps):
-        v = forward3(p, hp, tok, txt, ts[i], (h8 // 2, w8 // 2), ref_toks, ref_grids,
-                     t_target=ts[i + 1] if "target_in.w1" in p else None, dtype=dtype)
+    for i in range(start, n_steps):
+        tt = ts[i + 1] if "target_in.w1" in p else None
+        v = forward3(p, hp, tok, txt, ts[i], (h8 // 2, w8 // 2), ref_toks, ref_grids, t_target=tt, dtype=dtype)
+        if guidance is not None:
+            v_u = forward3(p, hp, tok, txt_uncond, ts[i], (h8 // 2, w8 // 2), ref_toks, ref_grids, t_target=tt,
+                           dtype=dtype)
+            v = O.guided_velocity(v, v_u, guidance)
         vs.append(v)
         if on_step is not None:
             on_step(i, v)

@@ -185,3 +185,75 @@ def test_text_and_reference_streams_are_at_time_zero_throughout():
     tc = {}
     O3.forward3(p3, hp(d), img, txt, 0.2, (3, 4), refs, grids, trace=tc, ctx_time=0.5)
     assert (tc["x_txt"] - ta["x_txt"]).abs().max() > 1e-4
+
+
+# ---------------------------------------------------------------- guidance and image editing (sampler)
+def _sampler_case(seed, flow_map=False):
+    d = Flux3Dims(**{**MICRO3.__dict__, "flow_map": flow_map})
+    p3 = params(d, seed)
+    g = torch.Generator().manual_seed(seed + 100)
+    noise = torch.randn(32, 6, 8, generator=g, dtype=F64)
+    txt_c = torch.randn(5, 40, generator=g, dtype=F64)
+    txt_u = torch.randn(5, 40, generator=g, dtype=F64)
+    return d, p3, noise, txt_c, txt_u
+
+
+def test_guidance_one_and_zero_select_one_text():
+    """v_u + g (v_c - v_u): g = 1 is the prompt's sampler, g = 0 the unconditional text's."""
+    d, p3, noise, txt_c, txt_u = _sampler_case(21)
+    plain_c, _ = O3.sample3(p3, hp(d), noise, txt_c, 3)
+    plain_u, _ = O3.sample3(p3, hp(d), noise, txt_u, 3)
+    g1, _ = O3.sample3(p3, hp(d), noise, txt_c, 3, txt_uncond=txt_u, guidance=1.0)
+    g0, _ = O3.sample3(p3, hp(d), noise, txt_c, 3, txt_uncond=txt_u, guidance=0.0)
+    assert torch.allclose(g1, plain_c, atol=1e-12, rtol=0)
+    assert torch.allclose(g0, plain_u, atol=1e-12, rtol=0)
+    g3, _ = O3.sample3(p3, hp(d), noise, txt_c, 3, txt_uncond=txt_u, guidance=3.5)
+    assert (g3 - plain_c).abs().max() > 1e-3      # a real extrapolation moves the result
+
+
+def test_guidance_with_one_text_is_the_plain_sampler():
+    d, p3, noise, txt_c, _ = _sampler_case(22, flow_map=True)
+    plain, _ = O3.sample3(p3, hp(d), noise, txt_c, 3)
+    guided, _ = O3.sample3(p3, hp(d), noise, txt_c, 3, txt_uncond=txt_c, guidance=3.5)
+    assert torch.allclose(guided, plain, atol=1e-12, rtol=0)
+
+
+def test_image_and_reference_streams_leave_the_per_mode_phase_independent_of_the_text():
+    """In the per-mode blocks each stream attends only to itself, so the image and reference
+    streams that enter the joint blocks are the same for the prompt and the unconditional text
+    (a guided batch may compute them once)."""
+    d = Flux3Dims(**{**MICRO3.__dict__, "n_mode": 2})
+    p3 = params(d, 23)
+    img, txt, refs, grids = inputs(24)
+    txt2 = torch.randn_like(txt)
+    a, b = {}, {}
+    va = O3.forward3(p3, hp(d), img, txt, 0.6, (3, 4), refs, grids, trace=a)
+    vb = O3.forward3(p3, hp(d), img, txt2, 0.6, (3, 4), refs, grids, trace=b)
+    assert torch.equal(a["x_img"], b["x_img"]) and torch.equal(a["x_ref"], b["x_ref"])
+    assert (a["x_txt"] - b["x_txt"]).abs().max() > 1e-3
+    assert (va - vb).abs().max() > 1e-4        # the joint blocks bring the text in
+
+
+def test_image_editing_starts_late_on_the_blended_latent():
+    """strength 1 is text-to-image; strength s < 1 starts at schedule step img2img_start(S, s)
+    from (1 - t) init + t noise, and the flow-map target times follow the same schedule."""
+    d, p3, noise, txt_c, _ = _sampler_case(25, flow_map=True)
+    init = torch.randn(32, 6, 8, generator=torch.Generator().manual_seed(26), dtype=F64)
+    plain, _ = O3.sample3(p3, hp(d), noise, txt_c, 4)
+    full, _ = O3.sample3(p3, hp(d), noise, txt_c, 4, init_latent=init, strength=1.0)
+    assert torch.allclose(full, plain, atol=1e-12, rtol=0)
+    seen = []
+    orig = O3.forward3
+
+    def spy(*args, **kw):
+        seen.append((args[2].clone(), args[4], kw.get("t_target")))
+        return orig(*args, **kw)
+
+    O3.forward3 = spy
+    try:
+        O3.sample3(p3, hp(d), noise, txt_c, 4, init_latent=init, strength=0.5)
+    finally:
+        O3.forward3 = orig
+    assert [(t, tt) for _, t, tt in seen] == [(0.5, 0.25), (0.25, 0.0)]
+    first = O.unpack_latents(seen[0][0], 6, 8)
+    assert torch.allclose(first, 0.5 * init + 0.5 * noise, atol=1e-12, rtol=0)
