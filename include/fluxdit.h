@@ -368,6 +368,23 @@ FLUX_API int flux3_dit_forward(flux3_dit *m, const float *img_tok, int grid_h, i
                                int n_txt, const float *ref_tok, int n_refs, const int *ref_grids, float t,
                                float t_target, float *v_out, void *stream);
 
+/* Classifier-free guidance forward of a FLUX.3 model: the velocities of the prompt and of the
+ * unconditional text for the same image, references, t and t_target as ONE batch of two
+ * sequences.  The base checkpoint samples 50 steps at guidance 3.5 (we0.ai FLUX 3 Image Klein
+ * article, checkpoint table); combine the two velocities with flux_cfg_euler_step.  In the
+ * per-mode blocks the image and reference streams attend only to themselves ("FLUX.3 Image Klein
+ * in Diffusers: ...", section "Entkoppelte Vorverarbeitung und gemeinsame Attention-Blöcke"), so
+ * they do not depend on the text: they are computed once for both sequences; the text streams
+ * and every joint block run per sequence.  txt_cond and txt_uncond are fp32 [n_txt, txt_dim]
+ * device buffers with the same token count; v_cond and v_uncond are distinct fp32
+ * [grid_h*grid_w, 128] outputs.  The workspace holds both sequences.  Otherwise as
+ * flux3_dit_forward; each velocity equals, bit for bit, what flux3_dit_forward returns for that
+ * text alone. */
+FLUX_API int flux3_dit_forward_cfg(flux3_dit *m, const float *img_tok, int grid_h, int grid_w, const float *txt_cond,
+                                   const float *txt_uncond, int n_txt, const float *ref_tok, int n_refs,
+                                   const int *ref_grids, float t, float t_target, float *v_cond, float *v_uncond,
+                                   void *stream);
+
 /* Precision of the block linears of later FLUX.3 forwards (linear1 / linear2 of the per-mode and
  * joint blocks): FLUX_PRECISION_BF16 or FLUX_PRECISION_FP8, as flux_dit_set_precision. */
 FLUX_API int flux3_dit_set_precision(flux3_dit *m, int precision);

@@ -83,6 +83,8 @@ _SIGS = {
     "flux3_dit_create": (_P, [_P, _Z, ctypes.POINTER(Flux3Config), _P]),
     "flux3_dit_destroy": (None, [_P]),
     "flux3_dit_forward": (_I, [_P, _P, _I, _I, _P, _I, _P, _I, ctypes.POINTER(ctypes.c_int), _F, _F, _P, _P]),
+    "flux3_dit_forward_cfg": (_I, [_P, _P, _I, _I, _P, _P, _I, _P, _I, ctypes.POINTER(ctypes.c_int), _F, _F, _P,
+                                   _P, _P]),
     "flux3_dit_set_active_blocks": (_I, [_P, _I, _I]),
     "flux3_dit_set_precision": (_I, [_P, _I]),
     "flux3_dit_modulation_size": (_Z, [_P]),
@@ -304,6 +306,23 @@ class Flux3DiT:
                                        _ptr(ref_tok, torch.float32, "ref_tok"), n_refs, grids, float(t),
                                        float(t_target), _ptr(v_out, torch.float32, "v_out"), _stream(stream)))
         return v_out
+
+    def forward_cfg(self, img_tok, grid_hw, txt_cond, txt_uncond, t, v_cond, v_uncond, ref_tok=None, ref_hw=(),
+                    t_target=0.0, stream=None):
+        """Velocities for the prompt and the unconditional text in one batch-2 forward (the
+        per-mode image and reference streams are computed once); see flux3_dit_forward_cfg."""
+        import torch
+        n_txt = 0 if txt_cond is None else txt_cond.shape[0]
+        if (0 if txt_uncond is None else txt_uncond.shape[0]) != n_txt:
+            raise ValueError("txt_cond and txt_uncond must have the same token count")
+        n_refs, grids = _grids(ref_hw)
+        _check(lib().flux3_dit_forward_cfg(self._h, _ptr(img_tok, torch.float32, "img_tok"), grid_hw[0], grid_hw[1],
+                                           _ptr(txt_cond, torch.float32, "txt_cond"),
+                                           _ptr(txt_uncond, torch.float32, "txt_uncond"), n_txt,
+                                           _ptr(ref_tok, torch.float32, "ref_tok"), n_refs, grids, float(t),
+                                           float(t_target), _ptr(v_cond, torch.float32, "v_cond"),
+                                           _ptr(v_uncond, torch.float32, "v_uncond"), _stream(stream)))
+        return v_cond, v_uncond
 
     def set_active_blocks(self, n_mode=-1, n_joint=-1):
         _check(lib().flux3_dit_set_active_blocks(self._h, n_mode, n_joint))
@@ -585,17 +604,25 @@ def flux_sample(model: FluxDiT, latent, txt, n_steps, ref_latent=None, on_step=N
     return out
 
 
-def flux3_sample(model: Flux3DiT, latent, txt, n_steps, ref_latent=None, on_step=None, stream=None):
+def flux3_sample(model: Flux3DiT, latent, txt, n_steps, ref_latent=None, on_step=None, stream=None,
+                 init_latent=None, strength=1.0, txt_uncond=None, guidance=None):
     """Euler sampling with a FLUX.3 model on the device: pack -> S x (forward, Euler) -> unpack.
 
     The flow-map model receives t_{i+1} as the target time of step i.  latent fp32 [32, h8, w8]
     (device): the noise; txt fp32 [n_txt, txt_dim]; ref_latent: None, one latent or a list.
+    init_latent / strength: image editing as in flux_sample.  With ``guidance`` g (and
+    ``txt_uncond`` of the same length) each step is one batch-2 forward (flux3_dit_forward_cfg)
+    and the fused guided Euler update; ``on_step(i, v)`` then sees the guided velocity.
     Returns the final latent (new tensor); ``on_step(i, v)`` sees each velocity.
     """
     import torch
     c, h8, w8 = latent.shape
     gh, gw = h8 // 2, w8 // 2
     ts = euler_schedule(n_steps)
+    start = 0
+    if init_latent is not None:
+        start = img2img_first_step(n_steps, strength)
+        latent = flux_blend_latents(init_latent, latent, ts[start], torch.empty_like(latent), stream)
     tok = torch.empty(gh * gw, 4 * c, device=latent.device, dtype=torch.float32)
     flux_pack_latents(latent, tok, stream)
     ref_tok, grids = None, []
@@ -608,11 +635,22 @@ def flux3_sample(model: Flux3DiT, latent, txt, n_steps, ref_latent=None, on_step
             flux_pack_latents(r, ref_tok[row:row + h * w], stream)
             row += h * w
     v = torch.empty_like(tok)
-    for i in range(n_steps):
-        model.forward(tok, (gh, gw), txt, ts[i], v, ref_tok, grids, t_target=ts[i + 1], stream=stream)
-        if on_step is not None:
-            on_step(i, v)
-        flux_euler_step(tok, v, ts[i + 1] - ts[i], stream)
+    if guidance is not None:
+        if txt_uncond is None:
+            raise ValueError("guidance needs txt_uncond")
+        v_u = torch.empty_like(tok)
+        for i in range(start, n_steps):
+            model.forward_cfg(tok, (gh, gw), txt, txt_uncond, ts[i], v, v_u, ref_tok, grids, t_target=ts[i + 1],
+                              stream=stream)
+            if on_step is not None:
+                on_step(i, v_u + guidance * (v - v_u))
+            flux_cfg_euler_step(tok, v, v_u, guidance, ts[i + 1] - ts[i], stream)
+    else:
+        for i in range(start, n_steps):
+            model.forward(tok, (gh, gw), txt, ts[i], v, ref_tok, grids, t_target=ts[i + 1], stream=stream)
+            if on_step is not None:
+                on_step(i, v)
+            flux_euler_step(tok, v, ts[i + 1] - ts[i], stream)
     out = torch.empty_like(latent)
     flux_unpack_latents(tok, out, stream)
     return out

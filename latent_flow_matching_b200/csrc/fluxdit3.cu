@@ -134,21 +134,26 @@ struct BlockW3 {
 // Row ranges of the joint sequence: text | image | reference (all references together).
 enum Seg { kSegTxt = 0, kSegImg = 1, kSegRef = 2 };
 
+// A forward evaluates up to two sequences that share the image, the references and t and differ
+// in their text (classifier-free guidance); sequence b occupies rows [b n, (b + 1) n).
+constexpr int kMaxBatch3 = 2;
+
 struct Workspace3 {
   size_t cap_n = 0, cap_tok = 0, cap_txt = 0;
   float* X = nullptr;
   bf16 *Y = nullptr, *QKV = nullptr, *CC = nullptr, *tokb = nullptr, *txtb = nullptr;
-  float2* rope = nullptr;
-  int nt = -1, gh = -1, gw = -1;
+  float2* rope = nullptr;        // one sequence's positions (every sequence has the same)
+  int nt = -1, gh = -1, gw = -1, nb = -1;
   RefGrids refs = {-1, {}, {}};
-  CUtensorMap a_tokb, a_txtb, a_Yall, a_Yout, qkv;
-  CUtensorMap a_Yseg[3], a_CCseg[3];
+  CUtensorMap a_tokb, qkv;
+  CUtensorMap a_txtb[kMaxBatch3], a_Yall[kMaxBatch3], a_Yout[kMaxBatch3];
+  CUtensorMap a_Yseg[kMaxBatch3][3], a_CCseg[kMaxBatch3][3];
   // FP8 precision: e4m3 LN-mod output (Y8, scale sY) and [O | H] (C8, scale sC per row)
   size_t cap8 = 0;
   uint8_t *Y8 = nullptr, *C8 = nullptr;
   float *sY = nullptr, *sC = nullptr;
   bool maps8 = false;
-  CUtensorMap a8_Yall, a8_Yseg[3], a8_CCseg[3];
+  CUtensorMap a8_Yall[kMaxBatch3], a8_Yseg[kMaxBatch3][3], a8_CCseg[kMaxBatch3][3];
 };
 
 // Offsets (in units of D floats) of the modulation vectors in the model's mods buffer.
@@ -306,94 +311,102 @@ int create3_impl(const void* blob, size_t blob_bytes, const flux3_dit_config* cf
 }
 
 // FP8 copies of the GEMM A operands (LN-mod output and [O | H]) and their maps.
-int prepare3_fp8(flux3_dit* m, int nt, int ni, int nr) {
+int prepare3_fp8(flux3_dit* m, int nt, int ni, int nr, int nb) {
   Workspace3& w = m->ws;
   const flux3_dit_config& c = m->cfg;
   const size_t D = c.hidden, F = c.mlp_hidden;
-  const size_t n = static_cast<size_t>(nt) + ni + nr;
-  if (n > w.cap8) {
+  const size_t n = static_cast<size_t>(nt) + ni + nr, rows = n * nb;
+  if (rows > w.cap8) {
     free_ws3_fp8(w);
-    const bool ok = cudaMalloc(&w.Y8, n * D) == cudaSuccess && cudaMalloc(&w.C8, n * (D + F)) == cudaSuccess &&
-                    cudaMalloc(&w.sY, n * 4) == cudaSuccess && cudaMalloc(&w.sC, n * 4) == cudaSuccess;
+    const bool ok = cudaMalloc(&w.Y8, rows * D) == cudaSuccess &&
+                    cudaMalloc(&w.C8, rows * (D + F)) == cudaSuccess && cudaMalloc(&w.sY, rows * 4) == cudaSuccess &&
+                    cudaMalloc(&w.sC, rows * 4) == cudaSuccess;
     if (!ok) {
       free_ws3_fp8(w);
-      return fail(FLUX_ENOMEM, "FP8 workspace allocation for %zu tokens failed", n);
+      return fail(FLUX_ENOMEM, "FP8 workspace allocation for %zu tokens failed", rows);
     }
-    w.cap8 = n;
+    w.cap8 = rows;
   }
   if (w.maps8) return FLUX_OK;
   bool ok = true;
-  auto amap = [&](CUtensorMap* map, const uint8_t* base, size_t rows, size_t cols, uint64_t stride) {
-    if (rows == 0) {
+  auto amap = [&](CUtensorMap* map, const uint8_t* base, size_t r, size_t cols, uint64_t stride) {
+    if (r == 0) {
       memset(map, 0, sizeof(*map));
       return;
     }
-    ok &= make_tmap_u8(map, base, rows, cols, stride, 128);
+    ok &= make_tmap_u8(map, base, r, cols, stride, 128);
   };
   const size_t row0[3] = {0, static_cast<size_t>(nt), static_cast<size_t>(nt) + ni};
-  const size_t rows[3] = {static_cast<size_t>(nt), static_cast<size_t>(ni), static_cast<size_t>(nr)};
-  amap(&w.a8_Yall, w.Y8, n, D, D);
-  for (int sg = 0; sg < 3; ++sg) {
-    amap(&w.a8_Yseg[sg], w.Y8 + row0[sg] * D, rows[sg], D, D);
-    amap(&w.a8_CCseg[sg], w.C8 + row0[sg] * (D + F), rows[sg], D + F, D + F);
+  const size_t seg[3] = {static_cast<size_t>(nt), static_cast<size_t>(ni), static_cast<size_t>(nr)};
+  for (int bb = 0; bb < nb; ++bb) {
+    const size_t r0 = bb * n;
+    amap(&w.a8_Yall[bb], w.Y8 + r0 * D, n, D, D);
+    for (int sg = 0; sg < 3; ++sg) {
+      amap(&w.a8_Yseg[bb][sg], w.Y8 + (r0 + row0[sg]) * D, seg[sg], D, D);
+      amap(&w.a8_CCseg[bb][sg], w.C8 + (r0 + row0[sg]) * (D + F), seg[sg], D + F, D + F);
+    }
   }
   if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an FP8 activation buffer");
   w.maps8 = true;
   return FLUX_OK;
 }
 
-int prepare_shape3(flux3_dit* m, int nt, int gh, int gw, const RefGrids& refs, cudaStream_t s) {
+int prepare_shape3(flux3_dit* m, int nt, int gh, int gw, const RefGrids& refs, int nb, cudaStream_t s) {
   Workspace3& w = m->ws;
   const flux3_dit_config& c = m->cfg;
   const size_t D = c.hidden, F = c.mlp_hidden;
   const size_t ni = static_cast<size_t>(gh) * gw, nr = ref_tokens(refs);
-  const size_t n = nt + ni + nr;
-  if (n > w.cap_n) {
+  const size_t n = nt + ni + nr, rows = n * nb;
+  if (rows > w.cap_n) {
     free_ws3(w);
-    bool ok = cudaMalloc(&w.X, n * D * 4) == cudaSuccess;
-    ok = ok && cudaMalloc(&w.Y, n * D * 2) == cudaSuccess;
-    ok = ok && cudaMalloc(&w.QKV, n * 3 * D * 2) == cudaSuccess;
-    ok = ok && cudaMalloc(&w.CC, n * (D + F) * 2) == cudaSuccess;
-    ok = ok && cudaMalloc(&w.rope, n * 64 * sizeof(float2)) == cudaSuccess;
+    bool ok = cudaMalloc(&w.X, rows * D * 4) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.Y, rows * D * 2) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.QKV, rows * 3 * D * 2) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.CC, rows * (D + F) * 2) == cudaSuccess;
+    ok = ok && cudaMalloc(&w.rope, rows * 64 * sizeof(float2)) == cudaSuccess;
     if (!ok) {
       free_ws3(w);
-      return fail(FLUX_ENOMEM, "workspace allocation for %zu tokens failed", n);
+      return fail(FLUX_ENOMEM, "workspace allocation for %zu tokens failed", rows);
     }
-    w.cap_n = n;
+    w.cap_n = rows;
   }
   if (grow(&w.tokb, &w.cap_tok, (ni + nr) * c.in_ch) != cudaSuccess ||
-      grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt, 1) * c.txt_dim) != cudaSuccess)
+      grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt * nb, 1) * c.txt_dim) != cudaSuccess)
     return fail(FLUX_ENOMEM, "workspace allocation failed");
   const bool fp8 = m->precision == FLUX_PRECISION_FP8;
-  if (w.nt == nt && w.gh == gh && w.gw == gw && same_refs(w.refs, refs))
-    return fp8 ? prepare3_fp8(m, nt, static_cast<int>(ni), static_cast<int>(nr)) : FLUX_OK;
+  if (w.nt == nt && w.gh == gh && w.gw == gw && w.nb == nb && same_refs(w.refs, refs))
+    return fp8 ? prepare3_fp8(m, nt, static_cast<int>(ni), static_cast<int>(nr), nb) : FLUX_OK;
   w.maps8 = false;
 
   const uint64_t ldD = D * 2, ldC = (D + F) * 2;
   bool ok = true;
-  auto amap = [&](CUtensorMap* map, const void* base, size_t rows, size_t cols, uint64_t stride) {
-    if (rows == 0) {
+  auto amap = [&](CUtensorMap* map, const void* base, size_t r, size_t cols, uint64_t stride) {
+    if (r == 0) {
       memset(map, 0, sizeof(*map));
       return;
     }
-    ok &= make_tmap_bf16(map, base, rows, cols, stride, 128);
+    ok &= make_tmap_bf16(map, base, r, cols, stride, 128);
   };
   const size_t row0[3] = {0, static_cast<size_t>(nt), nt + ni};
-  const size_t rows[3] = {static_cast<size_t>(nt), ni, nr};
+  const size_t seg[3] = {static_cast<size_t>(nt), ni, nr};
   amap(&w.a_tokb, w.tokb, ni + nr, c.in_ch, c.in_ch * 2);
-  amap(&w.a_txtb, w.txtb, nt, c.txt_dim, static_cast<uint64_t>(c.txt_dim) * 2);
-  amap(&w.a_Yall, w.Y, n, D, ldD);
-  amap(&w.a_Yout, w.Y, ni, D, ldD);                // output layer input: LN of the image rows
-  amap(&w.qkv, w.QKV, n, 3 * D, 3 * D * 2);
-  for (int sg = 0; sg < 3; ++sg) {
-    amap(&w.a_Yseg[sg], w.Y + row0[sg] * D, rows[sg], D, ldD);
-    amap(&w.a_CCseg[sg], w.CC + row0[sg] * (D + F), rows[sg], D + F, ldC);
+  amap(&w.qkv, w.QKV, rows, 3 * D, 3 * D * 2);
+  for (int bb = 0; bb < nb; ++bb) {
+    const size_t r0 = bb * n;
+    amap(&w.a_txtb[bb], w.txtb + bb * nt * static_cast<size_t>(c.txt_dim), nt, c.txt_dim,
+         static_cast<uint64_t>(c.txt_dim) * 2);
+    amap(&w.a_Yall[bb], w.Y + r0 * D, n, D, ldD);
+    amap(&w.a_Yout[bb], w.Y + bb * ni * D, ni, D, ldD);        // output layer input: LN of sequence bb's image rows
+    for (int sg = 0; sg < 3; ++sg) {
+      amap(&w.a_Yseg[bb][sg], w.Y + (r0 + row0[sg]) * D, seg[sg], D, ldD);
+      amap(&w.a_CCseg[bb][sg], w.CC + (r0 + row0[sg]) * (D + F), seg[sg], D + F, ldC);
+    }
   }
   if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an activation buffer");
   if (rope_table_launch(w.rope, nt, gh, gw, refs, c.rope_theta, s) != cudaSuccess)
     return fail(FLUX_EIO, "rope table launch failed");
-  w.nt = nt; w.gh = gh; w.gw = gw; w.refs = refs;
-  return fp8 ? prepare3_fp8(m, nt, static_cast<int>(ni), static_cast<int>(nr)) : FLUX_OK;
+  w.nt = nt; w.gh = gh; w.gw = gw; w.nb = nb; w.refs = refs;
+  return fp8 ? prepare3_fp8(m, nt, static_cast<int>(ni), static_cast<int>(nr), nb) : FLUX_OK;
 }
 
 // Quantise every block linear (per-mode streams and joint blocks) to e4m3, one scale per row.
@@ -478,12 +491,26 @@ int run_modulation3(flux3_dit* m, float t, float t_target, cudaStream_t s) {
   return FLUX_OK;
 }
 
-int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const float* txt, int nt,
-                  const float* ref_tok, const RefGrids& refs, float t, float t_target, float* v_out, cudaStream_t s) {
+// One forward of nb sequences that share the image tokens, the references, t and t_target and
+// differ in their text (nb = 2: the prompt and the unconditional text of classifier-free
+// guidance).  In the per-mode blocks the image and reference streams attend only to themselves
+// and are modulated from t and t = 0 alone, so they are the same for every sequence: they run
+// once (in sequence 0's rows) and are copied to the other sequences before the joint blocks.
+// Every GEMM takes the kernel a one-sequence forward would take, so each velocity equals, bit
+// for bit, that of a forward with its text alone.
+int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const float* const* txt, int nt,
+                  const float* ref_tok, const RefGrids& refs, float t, float t_target, float* const* v_out, int nb,
+                  cudaStream_t s) {
   const flux3_dit_config& c = m->cfg;
   const int D = c.hidden, F = c.mlp_hidden, H = c.heads;
-  if (!img_tok || !v_out) return fail(FLUX_EINVAL, "img_tok and v_out must be device pointers");
-  if (nt > 0 && !txt) return fail(FLUX_EINVAL, "txt is NULL for %d text tokens", nt);
+  if (nb < 1 || nb > kMaxBatch3) return fail(FLUX_EINVAL, "batch of %d sequences (1..%d)", nb, kMaxBatch3);
+  if (!img_tok) return fail(FLUX_EINVAL, "img_tok must be a device pointer");
+  for (int bb = 0; bb < nb; ++bb) {
+    if (!v_out[bb]) return fail(FLUX_EINVAL, "velocity output %d is NULL", bb);
+    if (nt > 0 && !txt[bb]) return fail(FLUX_EINVAL, "text %d is NULL for %d text tokens", bb, nt);
+    for (int o = 0; o < bb; ++o)
+      if (v_out[o] == v_out[bb]) return fail(FLUX_EINVAL, "the velocity outputs must be distinct buffers");
+  }
   if (gh < 4 || gh > 64 || gw < 4 || gw > 64) return fail(FLUX_EINVAL, "image grid %dx%d outside 4..64", gh, gw);
   if (nt < 0 || nt > 4096) return fail(FLUX_EINVAL, "bad text (n_txt=%d)", nt);
   if (refs.count < 0 || refs.count > kMaxRefs)
@@ -498,12 +525,15 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
   cudaGetDevice(&dev);
   if (dev != m->device) return fail(FLUX_EINVAL, "model lives on device %d, current device is %d", m->device, dev);
 
-  int rc = prepare_shape3(m, nt, gh, gw, refs, s);
+  int rc = prepare_shape3(m, nt, gh, gw, refs, nb, s);
   if (rc) return rc;
   Workspace3& w = m->ws;
-  const int ni = gh * gw, nr = static_cast<int>(ref_tokens(refs)), n = nt + ni + nr;
+  const int ni = gh * gw, nr = static_cast<int>(ref_tokens(refs)), n = nt + ni + nr, rows_all = n * nb;
+  // rows the per-mode blocks touch: all of sequence 0, the text rows of the others
+  const int rows_pm = nb == 1 ? n : (nb - 1) * n + nt;
   const int row0[3] = {0, nt, nt + ni};
-  const int rows[3] = {nt, ni, nr};
+  const int seg[3] = {nt, ni, nr};
+  const size_t sD = D, sDF = static_cast<size_t>(D) + F;
   const float eps_ln = c.eps_ln, eps_rms = c.eps_rms;
   const float* mods = m->mods;
   auto md = [&](int off) { return mods + static_cast<size_t>(off) * D; };
@@ -516,17 +546,22 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
     FD_LAUNCH(m, kProfOther, 0, 6.0 * nr * c.in_ch,
               cast_bf16_launch(ref_tok, w.tokb + static_cast<size_t>(ni) * c.in_ch,
                                static_cast<size_t>(nr) * c.in_ch, s));
-  if (nt)
+  for (int bb = 0; bb < nb && nt; ++bb)
     FD_LAUNCH(m, kProfOther, 0, 6.0 * nt * c.txt_dim,
-              cast_bf16_launch(txt, w.txtb, static_cast<size_t>(nt) * c.txt_dim, s));
-  const double ln_bytes = 6.0 * n * D + 16.0 * D;
+              cast_bf16_launch(txt[bb], w.txtb + static_cast<size_t>(bb) * nt * c.txt_dim,
+                               static_cast<size_t>(nt) * c.txt_dim, s));
+  const bool fp8 = m->precision == FLUX_PRECISION_FP8;
 
+  // input projections: every text, the image and reference tokens once (sequence 0's rows)
   GemmParams P;
   P.num_problems = 2;
-  problem(P, 0, w.a_txtb, m->m_txt_in, nt, D, c.txt_dim, kEpiF32Bias, w.X, D, m->txt_b, nullptr);
-  problem(P, 1, w.a_tokb, m->m_img_in, ni + nr, D, c.in_ch, kEpiF32Bias, w.X + static_cast<size_t>(nt) * D, D,
-          m->img_b, nullptr);
-  FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, false));
+  problem(P, 0, w.a_txtb[0], m->m_txt_in, nt, D, c.txt_dim, kEpiF32Bias, w.X, D, m->txt_b, nullptr);
+  problem(P, 1, w.a_tokb, m->m_img_in, ni + nr, D, c.in_ch, kEpiF32Bias, w.X + nt * sD, D, m->img_b, nullptr);
+  const bool small_in = small_linear(P, m->num_sms, false, 1);
+  for (int bb = 1; bb < nb; ++bb)
+    problem(P, P.num_problems++, w.a_txtb[bb], m->m_txt_in, nt, D, c.txt_dim, kEpiF32Bias, w.X + bb * n * sD, D,
+            m->txt_b, nullptr);
+  FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear_as(P, m->num_sms, s, false, small_in));
 
   AttnParams A;
   A.mapQ = w.qkv; A.mapK = w.qkv; A.mapV = w.qkv;
@@ -534,105 +569,132 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
   A.q_col0 = 0; A.k_col0 = D; A.v_col0 = 2 * D;
   A.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
 
-  // ---------------- per-mode blocks: each stream with its own weights, attention within the stream
-  AttnParams As = A;
-  As.nseg = 3;
-  double seg_flops = 0;
-  for (int sg = 0; sg < 3; ++sg) {
-    As.seg_row0[sg] = row0[sg];
-    As.seg_n[sg] = rows[sg];
-    seg_flops += 4.0 * rows[sg] * static_cast<double>(rows[sg]) * D;
-  }
   // FP8 precision: block linears on e4m3 codes; LN-mod quantises its output, [O | H] is quantised
   // (one scale per row) before linear2
-  const bool fp8 = m->precision == FLUX_PRECISION_FP8;
   auto f8 = [&](int i, const CUtensorMap& a8, const CUtensorMap& w8, const float* sa, const float* sb) {
     P.mapA[i] = a8;
     P.mapB[i] = w8;
     P.prob[i].scale_a = sa;
     P.prob[i].scale_b = sb;
   };
-  auto ln3 = [&](const float* sh0, const float* sc0, const float* sh1, const float* sc1, const float* sh2,
+  // LN + modulation of rows [0, r) (text | image | reference per sequence of n rows)
+  auto ln3 = [&](int r, const float* sh0, const float* sc0, const float* sh1, const float* sc1, const float* sh2,
                  const float* sc2) -> int {
     if (fp8)
-      FD_LAUNCH(m, kProfLnMod, 0, 5.0 * n * D + 4.0 * n,
-                ln_modulate_fp8_launch(w.X, w.Y8, w.sY, n, D, nt, nt + ni, n, sh0, sc0, sh1, sc1, sh2, sc2, eps_ln,
+      FD_LAUNCH(m, kProfLnMod, 0, 5.0 * r * D + 4.0 * r,
+                ln_modulate_fp8_launch(w.X, w.Y8, w.sY, r, D, nt, nt + ni, n, sh0, sc0, sh1, sc1, sh2, sc2, eps_ln,
                                        s));
     else
-      FD_LAUNCH(m, kProfLnMod, 0, ln_bytes,
-                ln_modulate3_launch(w.X, w.Y, n, D, nt, nt + ni, n, sh0, sc0, sh1, sc1, sh2, sc2, eps_ln, s));
+      FD_LAUNCH(m, kProfLnMod, 0, 6.0 * r * D + 16.0 * D,
+                ln_modulate3_launch(w.X, w.Y, r, D, nt, nt + ni, n, sh0, sc0, sh1, sc1, sh2, sc2, eps_ln, s));
     return FLUX_OK;
   };
-  auto quant_cc = [&]() -> int {
-    FD_LAUNCH(m, kProfOther, 0, 3.0 * n * (D + F) + 4.0 * n,
-              quantize_rows_launch(w.CC, D + F, n, D + F, w.C8, D + F, w.sC, s));
+  auto quant_cc = [&](int r) -> int {
+    FD_LAUNCH(m, kProfOther, 0, 3.0 * r * sDF + 4.0 * r, quantize_rows_launch(w.CC, D + F, r, D + F, w.C8, D + F, w.sC, s));
     return FLUX_OK;
   };
+
+  // ---------------- per-mode blocks: each stream with its own weights, attention within the stream.
+  // Segments: sequence 0's text, image and reference rows, then the other sequences' text rows.
+  AttnParams As = A;
+  As.nseg = 2 + nb;
+  double seg_flops = 0;
+  for (int z = 0; z < As.nseg; ++z) {
+    As.seg_row0[z] = z < 3 ? row0[z] : (z - 2) * n;
+    As.seg_n[z] = z < 3 ? seg[z] : nt;
+    seg_flops += 4.0 * As.seg_n[z] * static_cast<double>(As.seg_n[z]) * D;
+  }
   const int mode_set[3] = {kModTxt, kModImg, kModRef};
   for (int i = 0; i < m->act_mode; ++i) {
-    rc = ln3(md(kModTxt), md(kModTxt + 1), md(kModImg), md(kModImg + 1), md(kModRef), md(kModRef + 1));
+    rc = ln3(rows_pm, md(kModTxt), md(kModTxt + 1), md(kModImg), md(kModImg + 1), md(kModRef), md(kModRef + 1));
     if (rc) return rc;
-    P.num_problems = 6;
-    for (int sg = 0; sg < 3; ++sg) {
+    // linear1: (qkv + QK-RMSNorm + RoPE, SwiGLU) per stream of sequence 0, then the other texts
+    P.num_problems = 0;
+    auto lin1 = [&](int sg, size_t r0) {
       const BlockW3& bw = m->mode[3 * i + sg];
-      problem(P, 2 * sg, w.a_Yseg[sg], bw.m_qkv, rows[sg], 3 * D, D, kEpiBf16Bias,
-              w.QKV + static_cast<size_t>(row0[sg]) * 3 * D, 3 * D, bw.qkv_b, nullptr);
-      qk_fuse(P, 2 * sg, bw.q_gain, bw.k_gain, w.rope, row0[sg], eps_rms);
-      problem(P, 2 * sg + 1, w.a_Yseg[sg], bw.m_mlp, rows[sg], 2 * F, D, kEpiSwiGLU,
-              w.CC + static_cast<size_t>(row0[sg]) * (D + F) + D, D + F, bw.mlp_b, nullptr);
+      const int bb = static_cast<int>(r0 / n), j = P.num_problems;
+      problem(P, j, w.a_Yseg[bb][sg], bw.m_qkv, seg[sg], 3 * D, D, kEpiBf16Bias, w.QKV + (r0 + row0[sg]) * 3 * sD,
+              3 * D, bw.qkv_b, nullptr);
+      qk_fuse(P, j, bw.q_gain, bw.k_gain, w.rope, row0[sg], eps_rms);
+      problem(P, j + 1, w.a_Yseg[bb][sg], bw.m_mlp, seg[sg], 2 * F, D, kEpiSwiGLU, w.CC + (r0 + row0[sg]) * sDF + D,
+              D + F, bw.mlp_b, nullptr);
       if (fp8) {
-        f8(2 * sg, w.a8_Yseg[sg], bw.m8_qkv, w.sY + row0[sg], bw.s_qkv);
-        f8(2 * sg + 1, w.a8_Yseg[sg], bw.m8_mlp, w.sY + row0[sg], bw.s_mlp);
+        f8(j, w.a8_Yseg[bb][sg], bw.m8_qkv, w.sY + r0 + row0[sg], bw.s_qkv);
+        f8(j + 1, w.a8_Yseg[bb][sg], bw.m8_mlp, w.sY + r0 + row0[sg], bw.s_mlp);
       }
-    }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8));
-    FD_LAUNCH(m, kProfAttention, seg_flops, 8.0 * n * D, attention_launch(As, s));
-    if (fp8 && (rc = quant_cc())) return rc;
-    P.num_problems = 3;
-    for (int sg = 0; sg < 3; ++sg) {
+      P.num_problems += 2;
+    };
+    for (int sg = 0; sg < 3; ++sg) lin1(sg, 0);
+    for (int bb = 1; bb < nb; ++bb) lin1(kSegTxt, static_cast<size_t>(bb) * n);
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));   // SwiGLU: pair kernel
+    FD_LAUNCH(m, kProfAttention, seg_flops, 8.0 * rows_pm * D, attention_launch(As, s));
+    if (fp8 && (rc = quant_cc(rows_pm))) return rc;
+    // linear2 with each stream's gate into the residual; the kernel is chosen for sequence 0's streams
+    P.num_problems = 0;
+    auto lin2 = [&](int sg, size_t r0) {
       const BlockW3& bw = m->mode[3 * i + sg];
-      problem(P, sg, w.a_CCseg[sg], bw.m_lin2, rows[sg], D, D + F, kEpiResidGate,
-              w.X + static_cast<size_t>(row0[sg]) * D, D, bw.lin2_b, md(mode_set[sg] + 2));
-      if (fp8) f8(sg, w.a8_CCseg[sg], bw.m8_lin2, w.sC + row0[sg], bw.s_lin2);
-    }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8));
+      const int bb = static_cast<int>(r0 / n), j = P.num_problems++;
+      problem(P, j, w.a_CCseg[bb][sg], bw.m_lin2, seg[sg], D, D + F, kEpiResidGate, w.X + (r0 + row0[sg]) * sD, D,
+              bw.lin2_b, md(mode_set[sg] + 2));
+      if (fp8) f8(j, w.a8_CCseg[bb][sg], bw.m8_lin2, w.sC + r0 + row0[sg], bw.s_lin2);
+    };
+    for (int sg = 0; sg < 3; ++sg) lin2(sg, 0);
+    const bool small = small_linear(P, m->num_sms, fp8, 1);
+    for (int bb = 1; bb < nb; ++bb) lin2(kSegTxt, static_cast<size_t>(bb) * n);
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear_as(P, m->num_sms, s, fp8, small));
   }
+  // the image and reference streams of sequence 0 into the other sequences
+  for (int bb = 1; bb < nb; ++bb)
+    FD_LAUNCH(m, kProfOther, 0, 8.0 * (ni + nr) * D,
+              cudaMemcpyAsync(w.X + (static_cast<size_t>(bb) * n + nt) * sD, w.X + nt * sD,
+                              static_cast<size_t>(ni + nr) * sD * sizeof(float), cudaMemcpyDeviceToDevice, s));
 
-  // ---------------- joint blocks: one weight set, attention over the whole sequence, modulation per token type
+  // ---------------- joint blocks: one weight set, attention over each whole sequence, modulation per token type
   const int joint_set[3] = {kModJointCtx, kModJointImg, kModJointCtx};
-  const double at_flops = 4.0 * n * static_cast<double>(n) * D;
+  const double at_flops = 4.0 * nb * n * static_cast<double>(n) * D;
+  A.n = n;
+  A.batch = nb;
   for (int i = 0; i < m->act_joint; ++i) {
     const BlockW3& bw = m->joint[i];
-    rc = ln3(md(kModJointCtx), md(kModJointCtx + 1), md(kModJointImg), md(kModJointImg + 1), md(kModJointCtx),
-             md(kModJointCtx + 1));
+    rc = ln3(rows_all, md(kModJointCtx), md(kModJointCtx + 1), md(kModJointImg), md(kModJointImg + 1),
+             md(kModJointCtx), md(kModJointCtx + 1));
     if (rc) return rc;
-    P.num_problems = 2;
-    problem(P, 0, w.a_Yall, bw.m_qkv, n, 3 * D, D, kEpiBf16Bias, w.QKV, 3 * D, bw.qkv_b, nullptr);
-    qk_fuse(P, 0, bw.q_gain, bw.k_gain, w.rope, 0, eps_rms);
-    problem(P, 1, w.a_Yall, bw.m_mlp, n, 2 * F, D, kEpiSwiGLU, w.CC + D, D + F, bw.mlp_b, nullptr);
-    if (fp8) {
-      f8(0, w.a8_Yall, bw.m8_qkv, w.sY, bw.s_qkv);
-      f8(1, w.a8_Yall, bw.m8_mlp, w.sY, bw.s_mlp);
+    P.num_problems = 2 * nb;
+    for (int bb = 0; bb < nb; ++bb) {
+      const size_t r0 = static_cast<size_t>(bb) * n;
+      problem(P, 2 * bb, w.a_Yall[bb], bw.m_qkv, n, 3 * D, D, kEpiBf16Bias, w.QKV + r0 * 3 * sD, 3 * D, bw.qkv_b,
+              nullptr);
+      qk_fuse(P, 2 * bb, bw.q_gain, bw.k_gain, w.rope, 0, eps_rms);
+      problem(P, 2 * bb + 1, w.a_Yall[bb], bw.m_mlp, n, 2 * F, D, kEpiSwiGLU, w.CC + r0 * sDF + D, D + F, bw.mlp_b,
+              nullptr);
+      if (fp8) {
+        f8(2 * bb, w.a8_Yall[bb], bw.m8_qkv, w.sY + r0, bw.s_qkv);
+        f8(2 * bb + 1, w.a8_Yall[bb], bw.m8_mlp, w.sY + r0, bw.s_mlp);
+      }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8));
-    A.n = n;
-    FD_LAUNCH(m, kProfAttention, at_flops, 8.0 * n * D, attention_launch(A, s));
-    if (fp8 && (rc = quant_cc())) return rc;
-    P.num_problems = 3;
-    for (int sg = 0; sg < 3; ++sg) {
-      problem(P, sg, w.a_CCseg[sg], bw.m_lin2, rows[sg], D, D + F, kEpiResidGate,
-              w.X + static_cast<size_t>(row0[sg]) * D, D, bw.lin2_b, md(joint_set[sg] + 2));
-      if (fp8) f8(sg, w.a8_CCseg[sg], bw.m8_lin2, w.sC + row0[sg], bw.s_lin2);
-    }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
+    FD_LAUNCH(m, kProfAttention, at_flops, 8.0 * rows_all * D, attention_launch(A, s));
+    if (fp8 && (rc = quant_cc(rows_all))) return rc;
+    P.num_problems = 3 * nb;
+    for (int bb = 0; bb < nb; ++bb)
+      for (int sg = 0; sg < 3; ++sg) {
+        const size_t r = static_cast<size_t>(bb) * n + row0[sg];
+        problem(P, 3 * bb + sg, w.a_CCseg[bb][sg], bw.m_lin2, seg[sg], D, D + F, kEpiResidGate, w.X + r * sD, D,
+                bw.lin2_b, md(joint_set[sg] + 2));
+        if (fp8) f8(3 * bb + sg, w.a8_CCseg[bb][sg], bw.m8_lin2, w.sC + r, bw.s_lin2);
+      }
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
   }
 
   // ---------------- output layer on the image rows (text and reference tokens are dropped)
-  FD_LAUNCH(m, kProfLnMod, 0, 6.0 * ni * D + 8.0 * D,
-            ln_modulate_launch(w.X + static_cast<size_t>(nt) * D, w.Y, ni, D, ni, ni, md(kModFinal),
-                               md(kModFinal + 1), md(kModFinal), md(kModFinal + 1), eps_ln, s));
-  P.num_problems = 1;
-  problem(P, 0, w.a_Yout, m->m_fin, ni, c.in_ch, D, kEpiF32Bias, v_out, c.in_ch, m->fin_b, nullptr);
+  P.num_problems = nb;
+  for (int bb = 0; bb < nb; ++bb) {
+    FD_LAUNCH(m, kProfLnMod, 0, 6.0 * ni * D + 8.0 * D,
+              ln_modulate_launch(w.X + (static_cast<size_t>(bb) * n + nt) * sD, w.Y + static_cast<size_t>(bb) * ni * sD,
+                                 ni, D, ni, ni, md(kModFinal), md(kModFinal + 1), md(kModFinal), md(kModFinal + 1),
+                                 eps_ln, s));
+    problem(P, bb, w.a_Yout[bb], m->m_fin, ni, c.in_ch, D, kEpiF32Bias, v_out[bb], c.in_ch, m->fin_b, nullptr);
+  }
   FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm_launch(P, 128, m->num_sms, s));
   return FLUX_OK;
 }
@@ -678,7 +740,20 @@ int flux3_dit_forward(flux3_dit* m, const float* img_tok, int grid_h, int grid_w
   RefGrids refs;
   const int rc = read_ref_grids(n_refs, ref_grids, &refs);
   if (rc) return rc;
-  return forward3_impl(m, img_tok, grid_h, grid_w, txt, n_txt, ref_tok, refs, t, t_target, v_out,
+  return forward3_impl(m, img_tok, grid_h, grid_w, &txt, n_txt, ref_tok, refs, t, t_target, &v_out, 1,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int flux3_dit_forward_cfg(flux3_dit* m, const float* img_tok, int grid_h, int grid_w, const float* txt_cond,
+                          const float* txt_uncond, int n_txt, const float* ref_tok, int n_refs, const int* ref_grids,
+                          float t, float t_target, float* v_cond, float* v_uncond, void* stream) {
+  if (!m) return fail(FLUX_EINVAL, "model is NULL");
+  RefGrids refs;
+  const int rc = read_ref_grids(n_refs, ref_grids, &refs);
+  if (rc) return rc;
+  const float* txt[2] = {txt_cond, txt_uncond};
+  float* out[2] = {v_cond, v_uncond};
+  return forward3_impl(m, img_tok, grid_h, grid_w, txt, n_txt, ref_tok, refs, t, t_target, out, 2,
                        static_cast<cudaStream_t>(stream));
 }
 

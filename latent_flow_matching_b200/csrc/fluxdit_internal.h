@@ -11,7 +11,7 @@ namespace fdit {
 
 // ------------------------------------------------------------------ GEMM
 enum EpiMode : int { kEpiBf16Bias = 0, kEpiF32Bias = 1, kEpiSwiGLU = 2, kEpiResidGate = 3, kEpiQKNormRope = 4 };
-constexpr int kMaxProblems = 6;
+constexpr int kMaxProblems = 8;
 
 struct GemmProblem {
   int M, N, K;                    // out rows, W rows, reduction (K % 64 == 0, N % 32 == 0)

@@ -133,29 +133,35 @@ inline void qk_fuse(GemmParams& P, int i, const bf16* gq, const bf16* gk, const 
   pr.eps = eps;
 }
 
-// Launch the linear layers of one grouped GEMM.  The CTA-pair kernel (256 x 256 tiles) is the
-// faster one per SM, but when its tiles would leave more than half of the 74 pairs idle (few
-// token rows and N = hidden, e.g. linear2 and the projections at 256^2) the one-CTA kernel with
-// 128 x 128 tiles (four times as many) fills the GPU.  SwiGLU problems and 8-bit operands stay on
-// the pair kernel (a SwiGLU tile must hold 128 a-rows and their 128 b-rows).  `nb`: sequences in
-// the batch; the choice is made per sequence, so a batch and its sequences run alone take the
-// same kernel (and produce the same bits).
-inline cudaError_t launch_linear(GemmParams& P, int num_sms, cudaStream_t s, bool fp8, int nb = 1) {
-  if (!fp8) {
-    long pair_tiles = 0, small_tiles = 0;
-    bool swiglu = false;
-    for (int i = 0; i < P.num_problems; ++i) {
-      const GemmProblem& pr = P.prob[i];
-      if (pr.M <= 0 || pr.N <= 0) continue;
-      pair_tiles += static_cast<long>((pr.M + 255) / 256) * ((pr.N + 255) / 256);
-      small_tiles += static_cast<long>((pr.M + 127) / 128) * ((pr.N + 127) / 128);
-      swiglu |= pr.mode == kEpiSwiGLU;
-    }
-    if (!swiglu && pair_tiles > 0 && 4 * pair_tiles <= static_cast<long>(num_sms) * nb &&
-        small_tiles <= static_cast<long>(num_sms) * nb)
-      return gemm_launch(P, 128, num_sms, s);
+// Kernel choice for the linear layers of one grouped GEMM.  The CTA-pair kernel (256 x 256
+// tiles) is the faster one per SM, but when its tiles would leave more than half of the 74 pairs
+// idle (few token rows and N = hidden, e.g. linear2 and the projections at 256^2) the one-CTA
+// kernel with 128 x 128 tiles (four times as many) fills the GPU.  SwiGLU problems and 8-bit
+// operands stay on the pair kernel (a SwiGLU tile must hold 128 a-rows and their 128 b-rows).
+// `nb`: sequences in the batch; the choice is made per sequence, so a batch and its sequences run
+// alone take the same kernel (and produce the same bits).  True: the one-CTA kernel.
+inline bool small_linear(const GemmParams& P, int num_sms, bool fp8, int nb) {
+  if (fp8) return false;
+  long pair_tiles = 0, small_tiles = 0;
+  bool swiglu = false;
+  for (int i = 0; i < P.num_problems; ++i) {
+    const GemmProblem& pr = P.prob[i];
+    if (pr.M <= 0 || pr.N <= 0) continue;
+    pair_tiles += static_cast<long>((pr.M + 255) / 256) * ((pr.N + 255) / 256);
+    small_tiles += static_cast<long>((pr.M + 127) / 128) * ((pr.N + 127) / 128);
+    swiglu |= pr.mode == kEpiSwiGLU;
   }
-  return gemm2_launch(P, num_sms, s, fp8);
+  return !swiglu && pair_tiles > 0 && 4 * pair_tiles <= static_cast<long>(num_sms) * nb &&
+         small_tiles <= static_cast<long>(num_sms) * nb;
+}
+
+// Launch with a kernel chosen by the caller (small_linear of the problems that fix the choice).
+inline cudaError_t launch_linear_as(GemmParams& P, int num_sms, cudaStream_t s, bool fp8, bool small) {
+  return small && !fp8 ? gemm_launch(P, 128, num_sms, s) : gemm2_launch(P, num_sms, s, fp8);
+}
+
+inline cudaError_t launch_linear(GemmParams& P, int num_sms, cudaStream_t s, bool fp8, int nb = 1) {
+  return launch_linear_as(P, num_sms, s, fp8, small_linear(P, num_sms, fp8, nb));
 }
 
 // Grow a device buffer to `need` elements (contents are not kept).

@@ -127,6 +127,8 @@ TINY_DIMS = FluxDims(n_double=1, n_single=1)
 FULL_DIMS = FluxDims()
 F3_TINY_DIMS = Flux3Dims(n_mode=1, n_joint=1)
 F3_FULL_DIMS = Flux3Dims()
+F3_BASE_DIMS = Flux3Dims(flow_map=False)
+F3_TINY_BASE_DIMS = Flux3Dims(n_mode=1, n_joint=1, flow_map=False)
 
 WORKLOADS = {
     "tiny64": Workload("tiny64", 0, 64, 16, 0, 1, TINY_DIMS),
@@ -147,6 +149,11 @@ WORKLOADS = {
     "f3i2i256": Workload("f3i2i256", 22, 256, 80, 256, 4, F3_FULL_DIMS),
     "f3t2i1024": Workload("f3t2i1024", 23, 1024, 160, 0, 16, F3_FULL_DIMS),
     "f3i2i1024": Workload("f3i2i1024", 24, 1024, 80, 1024, 16, F3_FULL_DIMS),
+    # FLUX.3 Image Klein base checkpoint (no flow-map embedding): 50 steps at guidance 3.5 (we0.ai
+    # FLUX 3 Image Klein article, checkpoint table); the 256^2 golden case keeps 4 steps
+    "f3cfgtiny64": Workload("f3cfgtiny64", 26, 64, 16, 64, 4, F3_TINY_BASE_DIMS, guidance=3.5),
+    "f3cfg256": Workload("f3cfg256", 27, 256, 160, 0, 4, F3_BASE_DIMS, guidance=3.5),
+    "f3cfg1024": Workload("f3cfg1024", 28, 1024, 160, 0, 50, F3_BASE_DIMS, guidance=3.5),
 }
 
 

@@ -13,6 +13,8 @@ the stored velocities are the guided ones.
 FLUX.3 workloads (``f3*``) use the FLUX.3 oracle with the flow-map target time t_{i+1}; the
 8272-token image-to-image case runs the first STEPS_RUN steps of its 16-step schedule (``v`` then
 holds those steps and ``final`` the packed state after them, ``meta.steps_run`` says how many).
+The base-checkpoint workload (``f3cfg256``, no target time) is guided: each step evaluates the
+prompt and the unconditional text and stores the guided velocity.
 
 Usage: python tests/golden/make_goldens.py [workload ...]   (about an hour on 8 cores)
 """
@@ -32,7 +34,7 @@ from oracle import flux_oracle as O  # noqa: E402
 from oracle import flux3_oracle as O3  # noqa: E402
 
 ROW_STRIDE = {"t2i256": 1, "t2i512": 2, "t2i1024": 8, "i2i1024": 8, "mref1024": 8, "cfg256": 1,
-              "f3t2i256": 1, "f3i2i256": 1, "f3t2i1024": 8, "f3i2i1024": 8}
+              "f3t2i256": 1, "f3i2i256": 1, "f3t2i1024": 8, "f3i2i1024": 8, "f3cfg256": 1}
 STEPS_RUN = {"f3i2i1024": 4}
 
 
@@ -55,15 +57,21 @@ def make3(name):
     refs = [] if ref is None else (ref if isinstance(ref, list) else [ref])
     ref_toks = [O.pack_latents(torch.from_numpy(r)).float() for r in refs]
     ref_grids = [(r.shape[1] // 2, r.shape[2] // 2) for r in refs]
+    txt_u = torch.from_numpy(make_uncond_text(w)) if w.guidance is not None else None
     vs = []
     for i in range(k):
+        tt = ts[i + 1] if w.dims.flow_map else None
         v = O3.forward3(p, hp, tok, torch.from_numpy(txt), ts[i], (w.grid, w.grid), ref_toks, ref_grids,
-                        t_target=ts[i + 1] if w.dims.flow_map else None, dtype=torch.float32)
+                        t_target=tt, dtype=torch.float32)
+        if txt_u is not None:
+            v_u = O3.forward3(p, hp, tok, txt_u, ts[i], (w.grid, w.grid), ref_toks, ref_grids, t_target=tt,
+                              dtype=torch.float32)
+            v = O.guided_velocity(v, v_u, w.guidance)
         vs.append(v[rows].float().numpy())
         tok = O.euler_update(tok, v, ts[i + 1] - ts[i])
         print(f"  {name} step {i} done at {time.time() - t0:.0f}s", flush=True)
     meta = {"workload": name, "seed": w.seed, "oracle_dtype": "float32", "n_steps": w.n_steps, "steps_run": k,
-            "flow_map": bool(w.dims.flow_map), "row_stride": ROW_STRIDE[name],
+            "flow_map": bool(w.dims.flow_map), "guidance": w.guidance, "row_stride": ROW_STRIDE[name],
             "seconds": round(time.time() - t0, 1)}
     np.savez(os.path.join(HERE, f"{name}.npz"), rows=rows, v=np.stack(vs), final=tok[rows].float().numpy(),
              meta=np.array(json.dumps(meta)))

@@ -19,7 +19,7 @@ import torch
 import latent_flow_matching_b200 as F
 from oracle import flux_oracle as O
 from oracle import flux3_oracle as O3
-from synthetic import WORKLOADS, make_weights, make_inputs
+from synthetic import WORKLOADS, make_weights, make_inputs, make_uncond_text
 
 pytestmark = pytest.mark.gpu
 torch.set_grad_enabled(False)
@@ -277,6 +277,158 @@ def test_flux3_fp8_full_size_against_bf16():
         torch.cuda.synchronize()
         err = rel_l2(v8, v16)
         assert 1e-3 < err < 0.1, err
+    finally:
+        model.close()
+    assert F.flux_device_error() == 0
+
+
+# ---------------------------------------------------------------------------- classifier-free guidance
+@pytest.fixture(scope="module")
+def tiny3_base():
+    """The tiny model without the flow-map embedding (the base checkpoint's structure)."""
+    w = WORKLOADS["f3cfgtiny64"]
+    blob, p = make_weights(w.dims, w.seed)
+    model = F.Flux3DiT(blob, w.dims)
+    yield w, p, model
+    model.close()
+
+
+def _cfg_pair(model, tok, grid, txt_c, txt_u, t, refs, ref_grids, t_target):
+    vc = torch.full((grid[0] * grid[1], 128), float("nan"), device=DEV)
+    vu = torch.full_like(vc, float("nan"))
+    ref_tok = torch.cat(refs).to(DEV) if refs else None
+    nt = txt_c.shape[0]
+    model.forward_cfg(tok.to(DEV), grid, txt_c.to(DEV) if nt else None, txt_u.to(DEV) if nt else None, t, vc, vu,
+                      ref_tok, ref_grids, t_target=t_target)
+    return vc, vu
+
+
+@pytest.mark.parametrize("which", ["flow_map", "base"])
+@pytest.mark.parametrize("precision", ["bf16", "fp8"])
+@pytest.mark.parametrize("nt,grid,ref_grids", [(16, (4, 4), [(4, 4)]), (131, (8, 8), [(4, 8), (4, 4)]),
+                                               (0, (4, 6), []), (200, (12, 12), [(12, 12)]), (5, (6, 4), [])])
+def test_tiny3_guided_batch_is_bit_identical_to_two_forwards(tiny3, tiny3_base, which, precision, nt, grid,
+                                                               ref_grids):
+    """The batch-2 forward (per-mode image and reference streams computed once) returns, bit for
+    bit, the velocities of two single-text forwards; the base model matches the oracle."""
+    w, p, model = tiny3 if which == "flow_map" else tiny3_base
+    tok, txt_c, refs = _tiny_inputs(400 + nt, nt, grid, ref_grids)
+    txt_u = bf16r(torch.randn(nt, 20480, generator=torch.Generator().manual_seed(401 + nt)))
+    if precision == "fp8":
+        model.set_precision(F.PRECISION_FP8)
+    try:
+        vc, vu = _cfg_pair(model, tok, grid, txt_c, txt_u, 0.7, refs, ref_grids, 0.45)
+        sc = _gpu_forward(model, tok, grid, txt_c, 0.7, refs, ref_grids, 0.45)
+        su = _gpu_forward(model, tok, grid, txt_u, 0.7, refs, ref_grids, 0.45)
+    finally:
+        model.set_precision(F.PRECISION_BF16)
+    torch.cuda.synchronize()
+    assert torch.equal(vc, sc) and torch.equal(vu, su)
+    if nt:
+        assert rel_l2(vc, vu) > 1e-4                     # the texts differ, so do the velocities
+    if which == "base" and precision == "bf16":
+        want = O3.forward3(p, O.hyper(w.dims), tok, txt_u, 0.7, grid, refs, ref_grids)
+        assert rel_l2(vu, want) <= V_TOL
+    assert F.flux_device_error() == 0
+
+
+@pytest.mark.parametrize("strength", [1.0, 0.5])
+def test_tiny3_base_guided_sampler_matches_oracle(tiny3_base, strength):
+    """The base checkpoint's sampler: guidance 3.5, a reference image, text-to-image and image
+    editing (strength 0.5 starts at step 2 from the blended latent); every guided velocity and the
+    final latent against the oracle's guided sampler."""
+    w, p, model = tiny3_base
+    lat, txt, ref = make_inputs(w)
+    txt_u = make_uncond_text(w)
+    init = bf16r(torch.randn(*lat.shape, generator=torch.Generator().manual_seed(402))).numpy()
+    edit = {} if strength == 1.0 else {"init_latent": torch.from_numpy(init), "strength": strength}
+    ref_final, ref_vs = O3.sample3(p, O.hyper(w.dims), torch.from_numpy(lat), torch.from_numpy(txt), w.n_steps,
+                                   ref_latent=torch.from_numpy(ref), txt_uncond=torch.from_numpy(txt_u),
+                                   guidance=w.guidance, **edit)
+    vs = []
+    final = F.flux3_sample(model, torch.from_numpy(lat).to(DEV), torch.from_numpy(txt).to(DEV), w.n_steps,
+                           ref_latent=torch.from_numpy(ref).to(DEV), txt_uncond=torch.from_numpy(txt_u).to(DEV),
+                           guidance=w.guidance, on_step=lambda i, v: vs.append(v.cpu().clone()),
+                           **{k: (v.to(DEV) if torch.is_tensor(v) else v) for k, v in edit.items()})
+    assert len(vs) == len(ref_vs) == (w.n_steps if strength == 1.0 else 2)
+    for i in range(len(vs)):
+        assert rel_l2(vs[i], ref_vs[i]) <= V_TOL, i
+    assert rel_l2(final.cpu(), ref_final) <= X_TOL
+    assert F.flux_device_error() == 0
+
+
+def test_flux3_guided_batch_rejects_bad_arguments(tiny3):
+    w, p, model = tiny3
+    tok = torch.zeros(16, 128, device=DEV)
+    v = torch.empty(16, 128, device=DEV)
+    v2 = torch.empty(16, 128, device=DEV)
+    txt = torch.zeros(4, 20480, device=DEV)
+    with pytest.raises(F.FluxError):
+        model.forward_cfg(tok, (4, 4), txt, txt, 1.0, v, v, t_target=0.5)            # one buffer for both
+    rc = F.lib().flux3_dit_forward_cfg(model._h, tok.data_ptr(), 4, 4, txt.data_ptr(), None, 4, None, 0, None,
+                                       1.0, 0.5, v.data_ptr(), v2.data_ptr(), None)
+    assert rc != 0                                                                  # NULL unconditional text
+    with pytest.raises(ValueError):
+        model.forward_cfg(tok, (4, 4), txt, None, 1.0, v, v2, t_target=0.5)
+        model.forward_cfg(tok, (4, 4), txt, txt[:3], 1.0, v, v2, t_target=0.5)       # different token counts
+    model.forward_cfg(tok, (4, 4), txt, txt, 1.0, v, v2, t_target=0.5)              # still usable afterwards
+    torch.cuda.synchronize()
+    assert torch.equal(v, v2)
+    assert F.flux_device_error() == 0
+
+
+def test_flux3_base_guided_full_size_bit_identical():
+    """FLUX.3 base checkpoint at 1024^2 (4096 image + 160 text tokens, 5 + 28 blocks): the guided
+    batch equals two single forwards bit for bit, in bf16 and in FP8."""
+    w = WORKLOADS["f3cfg1024"]
+    blob, _ = make_weights(w.dims, w.seed)
+    lat, txt, _ = make_inputs(w)
+    txt_u = make_uncond_text(w)
+    model = F.Flux3DiT(blob, w.dims)
+    del blob
+    try:
+        tok = O.pack_latents(torch.from_numpy(lat)).float().to(DEV)
+        tc, tu = torch.from_numpy(txt).to(DEV), torch.from_numpy(txt_u).to(DEV)
+        for prec in (F.PRECISION_BF16, F.PRECISION_FP8):
+            model.set_precision(prec)
+            vc, vu = torch.empty(w.n_img, 128, device=DEV), torch.empty(w.n_img, 128, device=DEV)
+            sc, su = torch.empty_like(vc), torch.empty_like(vc)
+            model.forward_cfg(tok, (w.grid, w.grid), tc, tu, 0.8, vc, vu)
+            model.forward(tok, (w.grid, w.grid), tc, 0.8, sc)
+            model.forward(tok, (w.grid, w.grid), tu, 0.8, su)
+            torch.cuda.synchronize()
+            assert torch.equal(vc, sc) and torch.equal(vu, su), prec
+            assert torch.isfinite(vc).all() and rel_l2(vc, vu) > 1e-3
+    finally:
+        model.close()
+    assert F.flux_device_error() == 0
+
+
+def test_flux3_base_guided_sampler_against_oracle_golden():
+    """FLUX.3 base checkpoint at 256^2 (256 image + 160 text tokens), guidance 3.5, 4 steps: every
+    guided velocity and the final latent against the oracle's rows (tests/golden/f3cfg256.npz)."""
+    gd = _golden("f3cfg256")
+    g = WORKLOADS["f3cfg256"]
+    meta = json.loads(str(gd["meta"]))
+    assert meta["workload"] == "f3cfg256" and meta["seed"] == g.seed and meta["guidance"] == g.guidance
+    blob, _ = make_weights(g.dims, g.seed)
+    glat, gtxt, _ = make_inputs(g)
+    gtxt_u = make_uncond_text(g)
+    model = F.Flux3DiT(blob, g.dims)
+    del blob
+    try:
+        ts = F.euler_schedule(g.n_steps)
+        tok = O.pack_latents(torch.from_numpy(glat)).float().to(DEV)
+        tc, tu = torch.from_numpy(gtxt).to(DEV), torch.from_numpy(gtxt_u).to(DEV)
+        vc, vu = torch.empty(g.n_img, 128, device=DEV), torch.empty(g.n_img, 128, device=DEV)
+        rows = torch.from_numpy(gd["rows"]).long()
+        for i in range(g.n_steps):
+            model.forward_cfg(tok, (g.grid, g.grid), tc, tu, ts[i], vc, vu)
+            err = rel_l2((vu + g.guidance * (vc - vu)).cpu()[rows], gd["v"][i])
+            assert err <= V_TOL, (i, err)
+            F.flux_cfg_euler_step(tok, vc, vu, g.guidance, ts[i + 1] - ts[i])
+        err = rel_l2(tok.cpu()[rows], gd["final"])
+        assert err <= X_TOL, err
     finally:
         model.close()
     assert F.flux_device_error() == 0
