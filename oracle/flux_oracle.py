@@ -216,11 +216,15 @@ def timestep_embedding(t: float, dim: int = 256, max_period: float = 10000.0,
 
 
 def block_linear(hp):
-    """The linear layer used inside the transformer blocks: the plain definition, or the
-    row-wise FP8 one (``oracle/fp8_oracle.py``) when ``hp["fp8"]`` is set."""
+    """The linear layer used inside the transformer blocks: the plain definition, the row-wise
+    FP8 one (``oracle/fp8_oracle.py``) when ``hp["fp8"]`` is set, or the NVFP4 one
+    (``oracle/nvfp4_oracle.py``) when ``hp["nvfp4"]`` is set."""
     if hp.get("fp8"):
         from .fp8_oracle import linear_fp8
         return linear_fp8
+    if hp.get("nvfp4"):
+        from .nvfp4_oracle import linear_nvfp4
+        return linear_nvfp4
     return linear
 
 
