@@ -258,6 +258,30 @@ FLUX_API int flux_qk_rmsnorm_rope(uint16_t *qkv, int rows, int ld, int k_col, in
 FLUX_API int flux_quantize_rows_e4m3(const uint16_t *x, int rows, int cols, int ldx, uint8_t *q, int ldq,
                                      float *scale, void *stream);
 
+/* NVFP4 quantisation of rows (see flux_dit_set_precision with FLUX_PRECISION_NVFP4): x bf16 [rows, k]
+ * (row stride ldx elements) to 4-bit e2m1 codes q ([rows, k/2] bytes, row stride ldq bytes,
+ * element 2i in the low nibble of byte i), e4m3 block scales sf (one per 16 elements, in the
+ * tensor-core layout: byte ((r/128)*(k/64) + j/64)*512 + 16*(r%32) + 4*((r%128)/32) + (j/16)%4
+ * for element j of row r; flux_nvfp4_scale_bytes(rows, k) bytes, padding rows untouched) and fp32
+ * row scales S: amax = max |x|, S = amax / 2688, s_b = e4m3(amax_b * (448 / amax)),
+ * code = e2m1(x * (1 / (s_b * S))), each step rounded to float32, round to nearest even and
+ * saturating; a zero row or a block whose scale rounds to 0 gets codes 0 (the nvfp4 checkpoint
+ * format, "FLUX.3 Image Klein in Diffusers: ...", section "Hardwareanforderungen, Quantisierung
+ * und Inferenzlatenz"; block size and block-scale type as in NVIDIA's NVFP4).
+ * k % 64 == 0, k <= 16384, ldx % 8 == 0, ldq % 16 == 0; pointers 16-byte aligned. */
+FLUX_API size_t flux_nvfp4_scale_bytes(int rows, int k);
+FLUX_API int flux_quantize_rows_nvfp4(const uint16_t *x, int rows, int k, int ldx, uint8_t *q, int ldq, uint8_t *sf,
+                                      float *row_scale, void *stream);
+
+/* NVFP4 linear layer on the tensor cores (tcgen05 kind::mxf4nvf4 with block scales, CTA pairs):
+ * acc = sum over 16-element blocks of (codes_A . codes_W) * s_A * s_W for A [m, k] (codes with row
+ * stride lda bytes, scales a_sf) and W [n, k] (codes row stride k/2), both as written by
+ * flux_quantize_rows_nvfp4; then acc[i][j] * a_scale[i] * w_scale[j] goes through the epilogue
+ * `mode` of flux_linear.  k % 256 == 0, n % 32 == 0, lda % 16 == 0; pointers 16-byte aligned. */
+FLUX_API int flux_linear_nvfp4(const uint8_t *a, const uint8_t *a_sf, const float *a_scale, int m, int k, int lda,
+                               const uint8_t *w, const uint8_t *w_sf, const float *w_scale, int n,
+                               const uint16_t *bias, int mode, void *out, int ldo, const float *gate, void *stream);
+
 /* flux_layernorm_modulate with its output quantised row-wise to e4m3 in the same pass: q uint8
  * [rows, dim] codes and q_scale fp32 [rows] as in flux_quantize_rows_e4m3 (the modulated values
  * are quantised from float32).  dim in {1024, 2048, 3072, 4096}. */

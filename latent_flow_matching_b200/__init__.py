@@ -98,6 +98,9 @@ _SIGS = {
     "flux_quantize_rows_e4m3": (_I, [_P, _I, _I, _I, _P, _I, _P, _P]),
     "flux_layernorm_modulate_fp8": (_I, [_P, _P, _P, _I, _I, _P, _P, _F, _P]),
     "flux_linear_fp8": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _P, _I, _P, _I, _P, _P]),
+    "flux_nvfp4_scale_bytes": (_Z, [_I, _I]),
+    "flux_quantize_rows_nvfp4": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _P]),
+    "flux_linear_nvfp4": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _P, _I, _P, _I, _P, _I, _P, _P]),
 }
 EXPORTED = tuple(_SIGS)
 
@@ -486,6 +489,40 @@ def flux_linear_fp8(a, a_scale, w, w_scale, bias, mode, out, gate=None, stream=N
                                  a.stride(0), _u8(w, "w"), _ptr(w_scale, torch.float32, "w_scale"), n,
                                  _bits(bias, "bias"), mode, ctypes.c_void_p(out.data_ptr()), out.stride(0),
                                  _ptr(gate, torch.float32, "gate"), _stream(stream)))
+    return out
+
+
+def flux_nvfp4_scale_bytes(rows, k) -> int:
+    """Bytes of the e4m3 block scales of an NVFP4 matrix [rows, k] (whole 128-row blocks)."""
+    return int(lib().flux_nvfp4_scale_bytes(int(rows), int(k)))
+
+
+def flux_quantize_rows_nvfp4(x, q, sf, row_scale, stream=None):
+    """NVFP4 codes q (uint8 [rows, k/2], two per byte), block scales sf (uint8
+    [flux_nvfp4_scale_bytes(rows, k)]) and row scales (fp32 [rows]) of bf16 x [rows, k]."""
+    import torch
+    rows, k = x.shape
+    if x.stride(1) != 1 or q.stride(1) != 1:
+        raise ValueError("x and q must have unit column stride")
+    _check(lib().flux_quantize_rows_nvfp4(ctypes.c_void_p(x.data_ptr()), rows, k, x.stride(0),
+                                          ctypes.c_void_p(q.data_ptr()), q.stride(0), _u8(sf, "sf"),
+                                          _ptr(row_scale, torch.float32, "row_scale"), _stream(stream)))
+    return q, sf, row_scale
+
+
+def flux_linear_nvfp4(a, a_sf, a_scale, w, w_sf, w_scale, bias, mode, out, gate=None, stream=None):
+    """NVFP4 linear: a, w packed codes [m, k/2] / [n, k/2] with block scales and row scales as
+    written by flux_quantize_rows_nvfp4; epilogue modes as flux_linear."""
+    import torch
+    m, kh = a.shape
+    n = w.shape[0]
+    if a.stride(1) != 1:
+        raise ValueError("a must have unit column stride")
+    _check(lib().flux_linear_nvfp4(ctypes.c_void_p(a.data_ptr()), _u8(a_sf, "a_sf"),
+                                   _ptr(a_scale, torch.float32, "a_scale"), m, 2 * kh, a.stride(0), _u8(w, "w"),
+                                   _u8(w_sf, "w_sf"), _ptr(w_scale, torch.float32, "w_scale"), n,
+                                   _bits(bias, "bias"), mode, ctypes.c_void_p(out.data_ptr()), out.stride(0),
+                                   _ptr(gate, torch.float32, "gate"), _stream(stream)))
     return out
 
 

@@ -68,15 +68,21 @@ static bool encoder_ready() {
 
 // 2D map with a box of 128 bytes along the row (one 128-byte swizzle row) and box_rows rows.
 static bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType type, uint32_t box_cols, const void* base,
-                         uint64_t rows, uint64_t cols, uint64_t row_stride_bytes, uint32_t box_rows) {
+                         uint64_t rows, uint64_t cols, uint64_t row_stride_bytes, uint32_t box_rows,
+                         CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   if (!encoder_ready() || rows == 0 || cols == 0) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {row_stride_bytes};
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return g_encode(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_sf(CUtensorMap* map, const void* base, uint64_t bytes) {
+  if (bytes % 256) return false;
+  return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 256, base, bytes / 256, 256, 256, 8,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
@@ -1104,6 +1110,53 @@ int flux_linear_fp8(const uint8_t* a, const float* a_scale, int m, int k, int ld
   P.prob[0].scale_a = a_scale;
   P.prob[0].scale_b = w_scale;
   FD_CUDA(gemm2_launch(P, num_sms_current(), static_cast<cudaStream_t>(stream), true));
+  return FLUX_OK;
+}
+
+size_t flux_nvfp4_scale_bytes(int rows, int k) {
+  if (rows < 0 || k < 64 || k % 64) return 0;
+  return nvfp4_scale_bytes(static_cast<size_t>(rows), static_cast<size_t>(k));
+}
+
+int flux_quantize_rows_nvfp4(const uint16_t* x, int rows, int k, int ldx, uint8_t* q, int ldq, uint8_t* sf,
+                             float* row_scale, void* stream) {
+  if (!x || !q || !sf || !row_scale) return fail(FLUX_EINVAL, "NULL argument");
+  if (rows < 0 || k < 64 || k % 64 || k > 16384 || ldx < k || ldx % 8 || ldq < k / 2 || ldq % 16)
+    return fail(FLUX_EINVAL, "bad shape rows=%d k=%d ldx=%d ldq=%d (k %% 64, k <= 16384, ldx %% 8, ldq %% 16)", rows,
+                k, ldx, ldq);
+  if (!aligned16(x) || !aligned16(q) || !aligned16(sf) || !aligned16(row_scale))
+    return fail(FLUX_EINVAL, "pointers must be 16-byte aligned");
+  FD_CUDA(quantize_nvfp4_launch(reinterpret_cast<const bf16*>(x), ldx, rows, k, q, ldq, sf, row_scale,
+                                static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_linear_nvfp4(const uint8_t* a, const uint8_t* a_sf, const float* a_scale, int m, int k, int lda,
+                      const uint8_t* w, const uint8_t* w_sf, const float* w_scale, int n, const uint16_t* bias,
+                      int mode, void* out, int ldo, const float* gate, void* stream) {
+  if (!a || !a_sf || !a_scale || !w || !w_sf || !w_scale || !bias || !out) return fail(FLUX_EINVAL, "NULL argument");
+  if (m < 1 || k < 256 || k % 256 || n < 32 || n % 32 || lda < k / 2 || lda % 16)
+    return fail(FLUX_EINVAL, "bad shape m=%d k=%d n=%d lda=%d (k %% 256, n %% 32, lda %% 16 bytes)", m, k, n, lda);
+  if (mode < 0 || mode > 3) return fail(FLUX_EINVAL, "bad mode %d", mode);
+  if (mode == kEpiSwiGLU && n % 256) return fail(FLUX_EINVAL, "SwiGLU mode needs n %% 256 == 0");
+  if (mode == kEpiResidGate && !gate) return fail(FLUX_EINVAL, "gate is NULL");
+  const int out_cols = mode == kEpiSwiGLU ? n / 2 : n;
+  if (ldo < out_cols || ldo % 8) return fail(FLUX_EINVAL, "bad ldo=%d", ldo);
+  if (!aligned16(a) || !aligned16(w) || !aligned16(a_sf) || !aligned16(w_sf) || !aligned16(bias) || !aligned16(out) ||
+      !aligned16(a_scale) || !aligned16(w_scale) || (gate && !aligned16(gate)))
+    return fail(FLUX_EINVAL, "pointers must be 16-byte aligned");
+  GemmParams4 P4;
+  GemmParams& P = P4.g;
+  P.num_problems = 1;
+  if (!make_tmap_u8(&P.mapA[0], a, m, k / 2, static_cast<uint64_t>(lda), 128) ||
+      !make_tmap_u8(&P.mapB[0], w, n, k / 2, static_cast<uint64_t>(k / 2), 128) ||
+      !make_tmap_sf(&P4.mapSFA[0], a_sf, nvfp4_scale_bytes(m, k)) ||
+      !make_tmap_sf(&P4.mapSFB[0], w_sf, nvfp4_scale_bytes(n, k)))
+    return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed");
+  problem(P, 0, P.mapA[0], P.mapB[0], m, n, k, mode, out, ldo, reinterpret_cast<const bf16*>(bias), gate);
+  P.prob[0].scale_a = a_scale;
+  P.prob[0].scale_b = w_scale;
+  FD_CUDA(gemm_fp4_launch(P4, num_sms_current(), static_cast<cudaStream_t>(stream)));
   return FLUX_OK;
 }
 

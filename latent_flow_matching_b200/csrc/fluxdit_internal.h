@@ -135,6 +135,23 @@ cudaError_t ln_modulate_fp8_launch(const float* x, uint8_t* q, float* qscale, in
                                    const float* shift1, const float* scale1, const float* shift2,
                                    const float* scale2, float eps, cudaStream_t s);
 
+// ------------------------------------------------------------------ NVFP4 (nvfp4.cu, gemm_fp4.cu)
+// Rows of x (bf16, stride ldx elements) to e2m1 codes (q, [rows, k/2] bytes, stride ldq), e4m3
+// block scales (sf, nvfp4_scale_bytes(rows, k) bytes, 512-byte blocks of 128 rows x 64 elements)
+// and fp32 row scales; k % 64 == 0, k <= 16384.
+inline size_t nvfp4_scale_bytes(size_t rows, size_t k) { return (rows + 127) / 128 * 128 * (k / 16); }
+cudaError_t quantize_nvfp4_launch(const __nv_bfloat16* x, int ldx, int rows, int k, uint8_t* q, int ldq, uint8_t* sf,
+                                  float* row_scale, cudaStream_t s);
+// Problems of the NVFP4 pair GEMM: mapA / mapB over the codes (u8 maps, 128-byte box), K in elements
+// (K % 256 == 0), scale_a / scale_b the fp32 row scales, and the block scales' maps (make_tmap_sf).
+struct GemmParams4 {
+  GemmParams g;
+  CUtensorMap mapSFA[kMaxProblems];
+  CUtensorMap mapSFB[kMaxProblems];
+};
+cudaError_t gemm_fp4_launch(GemmParams4& P, int num_sms, cudaStream_t stream);
+int gemm_fp4_read_device_error(cudaStream_t stream);
+
 // ------------------------------------------------------------------ host helpers
 // Record `msg` as the calling thread's flux_get_error() message and return `code`.
 int record_error(int code, const char* msg);
@@ -146,6 +163,8 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 // 2D u8 tensor map (e4m3 codes): rows x cols bytes, box {128 bytes, box_rows}, 128B swizzle.
 bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
                   uint32_t box_rows);
+// Block scales of an NVFP4 matrix as 256-byte rows, box 8 rows (2 KB: one stage of 128 rows), no swizzle.
+bool make_tmap_sf(CUtensorMap* map, const void* base, uint64_t bytes);
 int num_sms_current();
 
 }  // namespace fdit

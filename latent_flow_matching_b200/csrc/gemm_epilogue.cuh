@@ -42,10 +42,24 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t
   }
 }
 
-template <int BN, bool kScale = false, int kParts = 1>
+// Overlapping accumulators (kOvl, the NVFP4 kernel): the tile's TMEM columns share 32 columns with
+// the other accumulator buffer, the last 32 (ovl_side 0) or the first 32 (ovl_side 1).  The part
+// that owns them drains that chunk first and then arrives on the barrier at `ovl_bar` (a
+// shared::cluster address), so the next tile's MMAs may start while the rest of this tile drains.
+// Under the fused QK-RMSNorm a head is read twice, so the owning part arrives when its head is done.
+__device__ __forceinline__ void ovl_release(uint32_t ovl_bar) {
+  tc_fence_before();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0)
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(ovl_bar) : "memory");
+}
+
+template <int BN, bool kScale = false, int kParts = 1, bool kOvl = false>
 __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32_t tbase, int m, int n0,
-                                                   int part = 0) {
+                                                   int part = 0, int ovl_side = -1, uint32_t ovl_bar = 0) {
   static_assert(BN % (128 * kParts) == 0, "each part must hold whole 128-wide heads");
+  // this part owns the shared columns: the last part for side 0, the first for side 1
+  const bool ovl_mine = kOvl && ((ovl_side == 0 && part == kParts - 1) || (ovl_side == 1 && part == 0));
   const bool row_ok = m < pr.M;
   // fp32 outputs whose rows start on 32-byte boundaries take 256-bit loads / stores
   const bool v8_ok = ((reinterpret_cast<uintptr_t>(pr.out) | (static_cast<uintptr_t>(pr.ldo) * 4)) & 31) == 0;
@@ -55,12 +69,18 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
   if (pr.mode == kEpiSwiGLU) {
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(pr.out);
     const int on0 = n0 / 2;                // output column of this tile's first pair
+    constexpr int kSw = BN / 2 / kParts;             // pairs per part
 #pragma unroll 1
-    for (int c = part * (BN / 2 / kParts); c < (part + 1) * (BN / 2 / kParts); c += 32) {
+    for (int c0 = part * kSw; c0 < (part + 1) * kSw; c0 += 32) {
+      // side 0 shares the last b chunk: the owning part walks its pairs from the end
+      const int c = (kOvl && ovl_mine && ovl_side == 0) ? (part + 1) * kSw - 32 - (c0 - part * kSw) : c0;
       uint32_t ra[32], rb[32];
       tmem_ld32(tbase + c, ra);
       tmem_ld32(tbase + BN / 2 + c, rb);
       tmem_ld_wait();
+      if constexpr (kOvl) {
+        if (ovl_mine && c0 == part * kSw) ovl_release(ovl_bar);
+      }
       if (row_ok && n0 + c < pr.N) {
         const uint4* ba = reinterpret_cast<const uint4*>(pr.bias + n0 + c);
         const uint4* bb = reinterpret_cast<const uint4*>(pr.bias + n0 + BN / 2 + c);
@@ -163,12 +183,21 @@ __device__ __forceinline__ void gemm_epilogue_tile(const GemmProblem& pr, uint32
         store_bf16x32(dstp, ob, v8b_ok);
       }
     }
+    if constexpr (kOvl) {
+      if (ovl_mine) ovl_release(ovl_bar);
+    }
   } else {
+    constexpr int kCols = BN / kParts;              // columns per part
 #pragma unroll 1
-    for (int c = part * (BN / kParts); c < (part + 1) * (BN / kParts); c += 32) {
+    for (int c0 = part * kCols; c0 < (part + 1) * kCols; c0 += 32) {
+      // side 0 shares the tile's last chunk: the owning part walks its columns from the end
+      const int c = (kOvl && ovl_mine && ovl_side == 0) ? (part + 1) * kCols - 32 - (c0 - part * kCols) : c0;
       uint32_t r[32];
       tmem_ld32(tbase + c, r);
       tmem_ld_wait();
+      if constexpr (kOvl) {
+        if (ovl_mine && c0 == part * kCols) ovl_release(ovl_bar);
+      }
       const int n = n0 + c;
       if (!row_ok || n >= pr.N) continue;
       scale_chunk<kScale>(r, sa, pr.scale_b + n);
