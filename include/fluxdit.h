@@ -147,9 +147,15 @@ FLUX_API int flux_dit_forward_cfg(flux_dit *m, const float *img_tok, int grid_h,
  * switch to FP8 quantises the block weights once (a device allocation of one byte per weight, and
  * a host synchronisation); the input / output projections, the modulation, attention and the
  * residual stream keep their precision.  Needs hidden in {1024, 2048, 3072, 4096} and
- * hidden + mlp_hidden <= 16384. */
+ * hidden + mlp_hidden <= 16384.
+ * FLUX_PRECISION_NVFP4: the "nvfp4" format of the same section, which needs a Blackwell GPU: the
+ * same operands as 4-bit e2m1 codes with one e4m3 scale per 16 elements and one fp32 scale per
+ * row (flux_quantize_rows_nvfp4), multiplied by tcgen05 block-scaled MMAs; the first switch
+ * quantises the block weights once (half a byte per weight plus the scales).  Needs hidden and
+ * mlp_hidden multiples of 256 and hidden + mlp_hidden <= 16384. */
 #define FLUX_PRECISION_BF16 0
 #define FLUX_PRECISION_FP8 1
+#define FLUX_PRECISION_NVFP4 2
 FLUX_API int flux_dit_set_precision(flux_dit *m, int precision);
 
 /* Diagnostic: run only the first n_double double blocks and n_single single
@@ -410,7 +416,8 @@ FLUX_API int flux3_dit_forward_cfg(flux3_dit *m, const float *img_tok, int grid_
                                    void *stream);
 
 /* Precision of the block linears of later FLUX.3 forwards (linear1 / linear2 of the per-mode and
- * joint blocks): FLUX_PRECISION_BF16 or FLUX_PRECISION_FP8, as flux_dit_set_precision. */
+ * joint blocks): FLUX_PRECISION_BF16, FLUX_PRECISION_FP8 or FLUX_PRECISION_NVFP4, as
+ * flux_dit_set_precision. */
 FLUX_API int flux3_dit_set_precision(flux3_dit *m, int precision);
 
 /* Diagnostic: run only the first n_mode per-mode and n_joint joint blocks (-1 = all). */

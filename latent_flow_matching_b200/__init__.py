@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libfluxdit.so")
 FLUX_OK, FLUX_EIO, FLUX_ENOMEM, FLUX_EINVAL = 0, -5, -12, -22
 
 EPI_BF16_BIAS, EPI_F32_BIAS, EPI_SWIGLU, EPI_RESID_GATE = 0, 1, 2, 3
-PRECISION_BF16, PRECISION_FP8 = 0, 1
+PRECISION_BF16, PRECISION_FP8, PRECISION_NVFP4 = 0, 1, 2
 
 
 class FluxConfig(ctypes.Structure):
@@ -227,7 +227,8 @@ class FluxDiT:
         _check(lib().flux_dit_set_active_blocks(self._h, n_double, n_single))
 
     def set_precision(self, precision):
-        """PRECISION_BF16 or PRECISION_FP8 (row-wise e4m3 block linears); see flux_dit_set_precision."""
+        """PRECISION_BF16, PRECISION_FP8 (row-wise e4m3) or PRECISION_NVFP4 (e2m1 with block scales) block
+        linears; see flux_dit_set_precision."""
         _check(lib().flux_dit_set_precision(self._h, int(precision)))
 
     def prepare_timesteps(self, ts, stream=None):
@@ -331,7 +332,7 @@ class Flux3DiT:
         _check(lib().flux3_dit_set_active_blocks(self._h, n_mode, n_joint))
 
     def set_precision(self, precision):
-        """PRECISION_BF16 or PRECISION_FP8 (row-wise e4m3 block linears); see flux3_dit_set_precision."""
+        """PRECISION_BF16, PRECISION_FP8 or PRECISION_NVFP4 block linears; see flux3_dit_set_precision."""
         _check(lib().flux3_dit_set_precision(self._h, int(precision)))
 
     def modulation_size(self) -> int:

@@ -182,6 +182,8 @@ struct StreamW {                       // one stream of a double block
   // FP8 precision: e4m3 codes of the same matrices (same row order) and their row scales
   CUtensorMap m8_qkv, m8_proj, m8_mlp_in, m8_mlp_out;
   const float *s_qkv, *s_proj, *s_mlp_in, *s_mlp_out;
+  // NVFP4 precision: codes, block scales and row scales of the same matrices
+  Fp4Op q4_qkv, q4_proj, q4_mlp_in, q4_mlp_out;
 };
 struct SingleW {
   const bf16 *qkv_b, *mlp_b, *q_gain, *k_gain, *lin2_b;
@@ -190,6 +192,7 @@ struct SingleW {
   CUtensorMap m_qkv, m_mlp, m_lin2;
   CUtensorMap m8_qkv, m8_mlp, m8_lin2;
   const float *s_qkv, *s_mlp, *s_lin2;
+  Fp4Op q4_qkv, q4_mlp, q4_lin2;
 };
 
 constexpr int kMaxBatch = 2;            // sequences of one shape per forward (prompt and unconditional text)
@@ -215,6 +218,17 @@ struct Workspace {
   bool maps8 = false;
   CUtensorMap a8_Yall, a8_CC, a8_Ytxt[kMaxBatch], a8_Yimg[kMaxBatch], a8_Otxt[kMaxBatch], a8_Oimg[kMaxBatch],
       a8_Htxt[kMaxBatch], a8_Himg[kMaxBatch];
+  // NVFP4 precision: codes of the LN-mod output (Y4) and of [O | H] (C4), their block scales
+  // (sfY; sfO, sfH for the double blocks' O and H; sfC for linear2) and row scales.  The double
+  // blocks quantise per stream segment (seg_dbl: text and image rows of every sequence, each
+  // segment's scales starting on a 128-row block), the single blocks the whole batch (seg_all).
+  size_t cap4_rows = 0, cap4_blocks = 0;
+  uint8_t *Y4 = nullptr, *C4 = nullptr, *sfY = nullptr, *sfO = nullptr, *sfH = nullptr, *sfC = nullptr;
+  float *sY4 = nullptr, *sO4 = nullptr, *sH4 = nullptr, *sC4 = nullptr;
+  bool maps4 = false;
+  Q4Segs seg_dbl, seg_all;
+  Fp4Op y4_txt[kMaxBatch], y4_img[kMaxBatch], y4_all, o4_txt[kMaxBatch], o4_img[kMaxBatch], h4_txt[kMaxBatch],
+      h4_img[kMaxBatch], c4_all;
 };
 
 }  // namespace fdit
@@ -242,6 +256,8 @@ struct flux_dit {
   int precision = FLUX_PRECISION_BF16;
   uint8_t* w8 = nullptr;               // e4m3 block linears (allocated on the first switch to FP8)
   float* w8_scale = nullptr;
+  uint8_t* w4 = nullptr;               // NVFP4 block linears: codes and block scales (first switch to NVFP4)
+  float* w4_scale = nullptr;
   fdit::Workspace ws;
   fdit::Profiler prof;
 };
@@ -256,8 +272,18 @@ static void free_ws8(Workspace& w) {
   w.maps8 = false;
 }
 
+static void free_ws4(Workspace& w) {
+  cudaFree(w.Y4); cudaFree(w.C4); cudaFree(w.sfY); cudaFree(w.sfO); cudaFree(w.sfH); cudaFree(w.sfC);
+  cudaFree(w.sY4); cudaFree(w.sO4); cudaFree(w.sH4); cudaFree(w.sC4);
+  w.Y4 = w.C4 = w.sfY = w.sfO = w.sfH = w.sfC = nullptr;
+  w.sY4 = w.sO4 = w.sH4 = w.sC4 = nullptr;
+  w.cap4_rows = w.cap4_blocks = 0;
+  w.maps4 = false;
+}
+
 static void free_ws(Workspace& w) {
   free_ws8(w);
+  free_ws4(w);
   cudaFree(w.X); cudaFree(w.Y); cudaFree(w.QKV); cudaFree(w.CC); cudaFree(w.tokb); cudaFree(w.txtb);
   cudaFree(w.rope);
   w = Workspace();
@@ -268,6 +294,7 @@ static void destroy(flux_dit* m) {
   free_ws(m->ws);
   cudaFree(m->wbuf); cudaFree(m->mods_w); cudaFree(m->mods_b);
   cudaFree(m->w8); cudaFree(m->w8_scale);
+  cudaFree(m->w4); cudaFree(m->w4_scale);
   cudaFree(m->temb); cudaFree(m->th); cudaFree(m->vec); cudaFree(m->mods); cudaFree(m->mods_cache);
   delete m;
 }
@@ -462,6 +489,67 @@ static int prepare_fp8(flux_dit* m, int nt, int nimg, int nb) {
   return FLUX_OK;
 }
 
+// NVFP4 copies of the GEMM A operands for a batch of nb sequences of n = nt + nimg rows, and their maps.
+static int prepare_fp4(flux_dit* m, int nt, int nimg, int nb) {
+  Workspace& w = m->ws;
+  const flux_dit_config& c = m->cfg;
+  const size_t D = c.hidden, F = c.mlp_hidden;
+  const int n = nt + nimg, rows = n * nb;
+  int r0[2 * kMaxBatch], rs[2 * kMaxBatch];
+  for (int b = 0; b < nb; ++b) {
+    r0[2 * b] = b * n;
+    rs[2 * b] = nt;
+    r0[2 * b + 1] = b * n + nt;
+    rs[2 * b + 1] = nimg;
+  }
+  const int zero = 0;
+  w.seg_dbl = q4_segments(r0, rs, 2 * nb);
+  w.seg_all = q4_segments(&zero, &rows, 1);
+  size_t blk_dbl = 0;
+  for (int z = 0; z < 2 * nb; ++z) blk_dbl += (rs[z] + 127) / 128;
+  const size_t blk_all = (rows + 127) / 128, blocks = std::max(blk_dbl, blk_all);
+  if (static_cast<size_t>(rows) > w.cap4_rows || blocks > w.cap4_blocks) {
+    free_ws4(w);
+    const size_t R = rows, B = blocks * 128;
+    const bool ok = cudaMalloc(&w.Y4, R * D / 2) == cudaSuccess && cudaMalloc(&w.C4, R * (D + F) / 2) == cudaSuccess &&
+                    cudaMalloc(&w.sfY, B * D / 16) == cudaSuccess && cudaMalloc(&w.sfO, B * D / 16) == cudaSuccess &&
+                    cudaMalloc(&w.sfH, B * F / 16) == cudaSuccess &&
+                    cudaMalloc(&w.sfC, B * (D + F) / 16) == cudaSuccess && cudaMalloc(&w.sY4, R * 4) == cudaSuccess &&
+                    cudaMalloc(&w.sO4, R * 4) == cudaSuccess && cudaMalloc(&w.sH4, R * 4) == cudaSuccess &&
+                    cudaMalloc(&w.sC4, R * 4) == cudaSuccess;
+    if (!ok) {
+      free_ws4(w);
+      return fail(FLUX_ENOMEM, "NVFP4 workspace allocation for %d tokens failed", rows);
+    }
+    w.cap4_rows = R;
+    w.cap4_blocks = blocks;
+  }
+  if (w.maps4) return FLUX_OK;
+  bool ok = true;
+  const size_t lY = D / 2, lC = (D + F) / 2;
+  for (int b = 0; b < nb; ++b) {
+    const size_t rt = static_cast<size_t>(b) * n, ri = rt + nt;
+    const int zt = 2 * b, zi = 2 * b + 1;
+    ok &= make_fp4_op(&w.y4_txt[b], w.Y4 + rt * lY, nt, D, lY, w.sfY, w.seg_dbl.blk0[zt], w.sY4 + rt);
+    ok &= make_fp4_op(&w.y4_img[b], w.Y4 + ri * lY, nimg, D, lY, w.sfY, w.seg_dbl.blk0[zi], w.sY4 + ri);
+    ok &= make_fp4_op(&w.o4_txt[b], w.C4 + rt * lC, nt, D, lC, w.sfO, w.seg_dbl.blk0[zt], w.sO4 + rt);
+    ok &= make_fp4_op(&w.o4_img[b], w.C4 + ri * lC, nimg, D, lC, w.sfO, w.seg_dbl.blk0[zi], w.sO4 + ri);
+    ok &= make_fp4_op(&w.h4_txt[b], w.C4 + rt * lC + D / 2, nt, F, lC, w.sfH, w.seg_dbl.blk0[zt], w.sH4 + rt);
+    ok &= make_fp4_op(&w.h4_img[b], w.C4 + ri * lC + D / 2, nimg, F, lC, w.sfH, w.seg_dbl.blk0[zi], w.sH4 + ri);
+  }
+  ok &= make_fp4_op(&w.y4_all, w.Y4, rows, D, lY, w.sfY, 0, w.sY4);
+  ok &= make_fp4_op(&w.c4_all, w.C4, rows, D + F, lC, w.sfC, 0, w.sC4);
+  if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an NVFP4 activation buffer");
+  w.maps4 = true;
+  return FLUX_OK;
+}
+
+static int prepare_quant(flux_dit* m, int nt, int nimg, int nb) {
+  if (m->precision == FLUX_PRECISION_FP8) return prepare_fp8(m, nt, nimg, nb);
+  if (m->precision == FLUX_PRECISION_NVFP4) return prepare_fp4(m, nt, nimg, nb);
+  return FLUX_OK;
+}
+
 static int prepare_shape(flux_dit* m, int nt, int gh, int gw, const RefGrids& refs, int nb, cudaStream_t s) {
   Workspace& w = m->ws;
   const flux_dit_config& c = m->cfg;
@@ -486,10 +574,10 @@ static int prepare_shape(flux_dit* m, int nt, int gh, int gw, const RefGrids& re
   if (grow(&w.tokb, &w.cap_tok, (ni + nr) * c.in_ch) != cudaSuccess ||
       grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt * nb, 1) * c.txt_dim) != cudaSuccess)
     return fail(FLUX_ENOMEM, "workspace allocation failed");
-  const bool fp8 = m->precision == FLUX_PRECISION_FP8;
   if (w.nt == nt && w.gh == gh && w.gw == gw && w.nb == nb && same_refs(w.refs, refs))
-    return fp8 ? prepare_fp8(m, nt, static_cast<int>(ni + nr), nb) : FLUX_OK;
+    return prepare_quant(m, nt, static_cast<int>(ni + nr), nb);
   w.maps8 = false;
+  w.maps4 = false;
 
   const size_t nimg = ni + nr;
   const uint64_t ldD = D * 2, ldC = (D + F) * 2;
@@ -524,7 +612,7 @@ static int prepare_shape(flux_dit* m, int nt, int gh, int gw, const RefGrids& re
         cudaSuccess)
       return fail(FLUX_EIO, "rope table copy failed");
   w.nt = nt; w.gh = gh; w.gw = gw; w.nb = nb; w.refs = refs;
-  return fp8 ? prepare_fp8(m, nt, static_cast<int>(nimg), nb) : FLUX_OK;
+  return prepare_quant(m, nt, static_cast<int>(nimg), nb);
 }
 
 // Quantise every block linear to e4m3 with one scale per output row (done once per model).
@@ -592,6 +680,45 @@ static int quantize_block_weights(flux_dit* m, cudaStream_t s) {
     wmap(&sw.m8_lin2, q[i], D, D + F); sw.s_lin2 = sc[i++];
   }
   if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an FP8 weight tensor");
+  FD_CUDA(cudaStreamSynchronize(s));
+  return FLUX_OK;
+}
+
+// Quantise every block linear to NVFP4 (done once per model, on the first switch to NVFP4).
+static int quantize_block_weights_nvfp4(flux_dit* m, cudaStream_t s) {
+  const flux_dit_config& c = m->cfg;
+  const size_t D = c.hidden, F = c.mlp_hidden;
+  std::vector<Fp4Mat> mats;
+  for (const StreamW& sw : m->dbl) {
+    mats.push_back({sw.w_qkv, 3 * D, D});
+    mats.push_back({sw.w_proj, D, D});
+    mats.push_back({sw.w_mlp_in, 2 * F, D});
+    mats.push_back({sw.w_mlp_out, D, F});
+  }
+  for (const SingleW& sw : m->sgl) {
+    mats.push_back({sw.w_lin1, 3 * D + 2 * F, D});
+    mats.push_back({sw.w_lin2, D, D + F});
+  }
+  int rc = quantize_weights_nvfp4(mats, &m->w4, &m->w4_scale, s);
+  if (rc) return rc;
+  bool ok = true;
+  auto op = [&](Fp4Op* o, const Fp4Mat& x, size_t row0, size_t rows) {
+    ok &= make_fp4_op(o, x.codes + row0 * x.cols / 2, rows, x.cols, x.cols / 2, x.sf, row0 / 128, x.scale + row0);
+  };
+  size_t i = 0;
+  for (StreamW& sw : m->dbl) {
+    op(&sw.q4_qkv, mats[i], 0, 3 * D); ++i;
+    op(&sw.q4_proj, mats[i], 0, D); ++i;
+    op(&sw.q4_mlp_in, mats[i], 0, 2 * F); ++i;
+    op(&sw.q4_mlp_out, mats[i], 0, D); ++i;
+  }
+  for (SingleW& sw : m->sgl) {
+    op(&sw.q4_qkv, mats[i], 0, 3 * D);
+    op(&sw.q4_mlp, mats[i], 3 * D, 2 * F);             // the SwiGLU rows start on a 128-row block (D % 128 == 0)
+    ++i;
+    op(&sw.q4_lin2, mats[i], 0, D); ++i;
+  }
+  if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an NVFP4 weight tensor");
   FD_CUDA(cudaStreamSynchronize(s));
   return FLUX_OK;
 }
@@ -667,7 +794,8 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
   const double at_flops = 4.0 * nb * n * static_cast<double>(n) * D, at_bytes = 8.0 * rows * D;
 
   // input projections: text rows with txt_in, image + reference rows with img_in, per sequence
-  GemmParams P;
+  GemmParams4 P4;
+  GemmParams& P = P4.g;
   P.num_problems = 2 * nb;
   for (int b = 0; b < nb; ++b) {
     problem(P, 2 * b, w.a_txtb[b], m->m_txt_in, nt, D, c.txt_dim, kEpiF32Bias, w.X + seq_row(b, 0) * D, D,
@@ -684,16 +812,31 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
   A.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
 
   // FP8 precision: block linears on e4m3 codes (row-wise scales); LN-mod quantises its output,
-  // the attention output and the SwiGLU hidden are quantised before the linears that read them
+  // the attention output and the SwiGLU hidden are quantised before the linears that read them.
+  // NVFP4 precision: the same operands as e2m1 codes with block and row scales (LN-mod writes bf16,
+  // then the rows are quantised per segment).
   const bool fp8 = m->precision == FLUX_PRECISION_FP8;
+  const bool fp4 = m->precision == FLUX_PRECISION_NVFP4;
   auto f8 = [&](int i, const CUtensorMap& a8, const CUtensorMap& w8, const float* sa, const float* sb) {
     P.mapA[i] = a8;
     P.mapB[i] = w8;
     P.prob[i].scale_a = sa;
     P.prob[i].scale_b = sb;
   };
-  // LN-mod of every row: rows r % n < split use (sh0, sc0), the others (sh1, sc1)
-  auto ln_mod = [&](int split, const float* sh0, const float* sc0, const float* sh1, const float* sc1) -> int {
+  auto linear = [&]() -> cudaError_t {
+    return fp4 ? gemm_fp4_launch(P4, m->num_sms, s) : launch_linear(P, m->num_sms, s, fp8, nb);
+  };
+  // NVFP4 codes of bf16 rows (ldx elements apart) into q (ldq bytes apart), one launch over the segments
+  auto quant4 = [&](const bf16* x, int ldx, int k, uint8_t* q, int ldq, uint8_t* sf, float* sc,
+                    const Q4Segs& segs) -> int {
+    FD_LAUNCH(m, kProfOther, 0, 2.5 * rows * k + 4.0 * rows,
+              quantize_nvfp4_launch(x, ldx, k, q, ldq, sf, sc, segs, s));
+    return FLUX_OK;
+  };
+  // LN-mod of every row: rows r % n < split use (sh0, sc0), the others (sh1, sc1); NVFP4 then
+  // quantises Y over the segments `segs`
+  auto ln_mod = [&](int split, const float* sh0, const float* sc0, const float* sh1, const float* sc1,
+                    const Q4Segs& segs) -> int {
     if (fp8)
       FD_LAUNCH(m, kProfLnMod, 0, 5.0 * rows * D + 4.0 * rows,
                 ln_modulate_fp8_launch(w.X, w.Y8, w.sY, rows, D, split, n, n, sh0, sc0, sh1, sc1, sh1, sc1, eps_ln,
@@ -701,6 +844,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
     else
       FD_LAUNCH(m, kProfLnMod, 0, ln_bytes, ln_modulate_launch(w.X, w.Y, rows, D, split, n, sh0, sc0, sh1, sc1,
                                                                eps_ln, s));
+    if (fp4) return quant4(w.Y, D, D, w.Y4, D / 2, w.sfY, w.sY4, segs);
     return FLUX_OK;
   };
   // e4m3 codes of CC columns [col0, col0 + cols) into C8, one scale per row
@@ -715,7 +859,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
     const StreamW& st = m->dbl[2 * i + 1];
     const float* mi = mods + si.mod_off;          // shift1, scale1, gate1, shift2, scale2, gate2
     const float* mt = mods + st.mod_off;
-    rc = ln_mod(nt, mt, mt + D, mi, mi + D);
+    rc = ln_mod(nt, mt, mt + D, mi, mi + D, w.seg_dbl);
     if (rc) return rc;
     P.num_problems = 2 * nb;
     for (int b = 0; b < nb; ++b) {
@@ -729,10 +873,15 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
         f8(2 * b, w.a8_Ytxt[b], st.m8_qkv, w.sY + seq_row(b, 0), st.s_qkv);
         f8(2 * b + 1, w.a8_Yimg[b], si.m8_qkv, w.sY + seq_row(b, nt), si.s_qkv);
       }
+      if (fp4) {
+        fp4_operands(P4, 2 * b, w.y4_txt[b], st.q4_qkv);
+        fp4_operands(P4, 2 * b + 1, w.y4_img[b], si.q4_qkv);
+      }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear());
     FD_LAUNCH(m, kProfAttention, at_flops, at_bytes, attention_launch(A, s));
     if (fp8 && (rc = quant_cc(0, D, w.sO))) return rc;
+    if (fp4 && (rc = quant4(w.CC, D + F, D, w.C4, (D + F) / 2, w.sfO, w.sO4, w.seg_dbl))) return rc;
     P.num_problems = 2 * nb;
     for (int b = 0; b < nb; ++b) {
       problem(P, 2 * b, w.a_Otxt[b], st.m_proj, nt, D, D, kEpiResidGate, w.X + seq_row(b, 0) * D, D, st.proj_b,
@@ -743,9 +892,13 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
         f8(2 * b, w.a8_Otxt[b], st.m8_proj, w.sO + seq_row(b, 0), st.s_proj);
         f8(2 * b + 1, w.a8_Oimg[b], si.m8_proj, w.sO + seq_row(b, nt), si.s_proj);
       }
+      if (fp4) {
+        fp4_operands(P4, 2 * b, w.o4_txt[b], st.q4_proj);
+        fp4_operands(P4, 2 * b + 1, w.o4_img[b], si.q4_proj);
+      }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
-    rc = ln_mod(nt, mt + 3 * D, mt + 4 * D, mi + 3 * D, mi + 4 * D);
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear());
+    rc = ln_mod(nt, mt + 3 * D, mt + 4 * D, mi + 3 * D, mi + 4 * D, w.seg_dbl);
     if (rc) return rc;
     P.num_problems = 2 * nb;
     for (int b = 0; b < nb; ++b) {
@@ -757,9 +910,14 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
         f8(2 * b, w.a8_Ytxt[b], st.m8_mlp_in, w.sY + seq_row(b, 0), st.s_mlp_in);
         f8(2 * b + 1, w.a8_Yimg[b], si.m8_mlp_in, w.sY + seq_row(b, nt), si.s_mlp_in);
       }
+      if (fp4) {
+        fp4_operands(P4, 2 * b, w.y4_txt[b], st.q4_mlp_in);
+        fp4_operands(P4, 2 * b + 1, w.y4_img[b], si.q4_mlp_in);
+      }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear());
     if (fp8 && (rc = quant_cc(D, F, w.sH))) return rc;
+    if (fp4 && (rc = quant4(w.CC + D, D + F, F, w.C4 + D / 2, (D + F) / 2, w.sfH, w.sH4, w.seg_dbl))) return rc;
     P.num_problems = 2 * nb;
     for (int b = 0; b < nb; ++b) {
       problem(P, 2 * b, w.a_Htxt[b], st.m_mlp_out, nt, D, F, kEpiResidGate, w.X + seq_row(b, 0) * D, D,
@@ -770,14 +928,18 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
         f8(2 * b, w.a8_Htxt[b], st.m8_mlp_out, w.sH + seq_row(b, 0), st.s_mlp_out);
         f8(2 * b + 1, w.a8_Himg[b], si.m8_mlp_out, w.sH + seq_row(b, nt), si.s_mlp_out);
       }
+      if (fp4) {
+        fp4_operands(P4, 2 * b, w.h4_txt[b], st.q4_mlp_out);
+        fp4_operands(P4, 2 * b + 1, w.h4_img[b], si.q4_mlp_out);
+      }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear());
   }
   // single blocks: one set of weights for every row, so the whole batch is one problem
   for (int i = 0; i < m->act_single; ++i) {
     const SingleW& sw = m->sgl[i];
     const float* ms = mods + sw.mod_off;          // shift, scale, gate
-    rc = ln_mod(n, ms, ms + D, ms, ms + D);
+    rc = ln_mod(n, ms, ms + D, ms, ms + D, w.seg_all);
     if (rc) return rc;
     P.num_problems = 2;
     problem(P, 0, w.a_Yall, sw.m_qkv, rows, 3 * D, D, kEpiBf16Bias, w.QKV, 3 * D, sw.qkv_b, nullptr);
@@ -787,13 +949,19 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
       f8(0, w.a8_Yall, sw.m8_qkv, w.sY, sw.s_qkv);
       f8(1, w.a8_Yall, sw.m8_mlp, w.sY, sw.s_mlp);
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
+    if (fp4) {
+      fp4_operands(P4, 0, w.y4_all, sw.q4_qkv);
+      fp4_operands(P4, 1, w.y4_all, sw.q4_mlp);
+    }
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear());
     FD_LAUNCH(m, kProfAttention, at_flops, at_bytes, attention_launch(A, s));
     if (fp8 && (rc = quant_cc(0, D + F, w.sC))) return rc;
+    if (fp4 && (rc = quant4(w.CC, D + F, D + F, w.C4, (D + F) / 2, w.sfC, w.sC4, w.seg_all))) return rc;
     P.num_problems = 1;
     problem(P, 0, w.a_CC, sw.m_lin2, rows, D, D + F, kEpiResidGate, w.X, D, sw.lin2_b, ms + 2 * D);
     if (fp8) f8(0, w.a8_CC, sw.m8_lin2, w.sC, sw.s_lin2);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
+    if (fp4) fp4_operands(P4, 0, w.c4_all, sw.q4_lin2);
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear());
   }
   // output layer on the image rows of each sequence
   const float* mf = mods + m->fin_mod_off;         // shift, scale
@@ -898,16 +1066,24 @@ int flux_dit_set_precision(flux_dit* m, int precision) {
     m->precision = precision;
     return FLUX_OK;
   }
-  if (precision != FLUX_PRECISION_FP8) return fail(FLUX_EINVAL, "unknown precision %d", precision);
+  if (precision != FLUX_PRECISION_FP8 && precision != FLUX_PRECISION_NVFP4)
+    return fail(FLUX_EINVAL, "unknown precision %d", precision);
   const flux_dit_config& c = m->cfg;
-  if (c.hidden % 128 || c.mlp_hidden % 128 || (c.hidden != 1024 && c.hidden != 2048 && c.hidden != 3072 &&
-                                                c.hidden != 4096) || c.hidden + c.mlp_hidden > 16384)
+  if (precision == FLUX_PRECISION_FP8 &&
+      (c.hidden % 128 || c.mlp_hidden % 128 || (c.hidden != 1024 && c.hidden != 2048 && c.hidden != 3072 &&
+                                                c.hidden != 4096) || c.hidden + c.mlp_hidden > 16384))
     return fail(FLUX_EINVAL, "FP8 needs hidden in {1024, 2048, 3072, 4096} and hidden + mlp_hidden <= 16384");
+  if (precision == FLUX_PRECISION_NVFP4 && (c.hidden % 256 || c.mlp_hidden % 256 || c.hidden + c.mlp_hidden > 16384))
+    return fail(FLUX_EINVAL, "NVFP4 needs hidden and mlp_hidden multiples of 256 and hidden + mlp_hidden <= 16384");
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev != m->device) return fail(FLUX_EINVAL, "model lives on device %d, current device is %d", m->device, dev);
-  if (!m->w8) {
+  if (precision == FLUX_PRECISION_FP8 && !m->w8) {
     const int rc = quantize_block_weights(m, nullptr);
+    if (rc) return rc;
+  }
+  if (precision == FLUX_PRECISION_NVFP4 && !m->w4) {
+    const int rc = quantize_block_weights_nvfp4(m, nullptr);
     if (rc) return rc;
   }
   m->precision = precision;
@@ -1126,8 +1302,9 @@ int flux_quantize_rows_nvfp4(const uint16_t* x, int rows, int k, int ldx, uint8_
                 k, ldx, ldq);
   if (!aligned16(x) || !aligned16(q) || !aligned16(sf) || !aligned16(row_scale))
     return fail(FLUX_EINVAL, "pointers must be 16-byte aligned");
-  FD_CUDA(quantize_nvfp4_launch(reinterpret_cast<const bf16*>(x), ldx, rows, k, q, ldq, sf, row_scale,
-                                static_cast<cudaStream_t>(stream)));
+  const int r0 = 0;
+  FD_CUDA(quantize_nvfp4_launch(reinterpret_cast<const bf16*>(x), ldx, k, q, ldq, sf, row_scale,
+                                q4_segments(&r0, &rows, 1), static_cast<cudaStream_t>(stream)));
   return FLUX_OK;
 }
 

@@ -129,6 +129,8 @@ struct BlockW3 {
   // FP8 precision: e4m3 codes of linear1 (qkv rows, SwiGLU rows) and linear2, row scales
   CUtensorMap m8_qkv, m8_mlp, m8_lin2;
   const float *s_qkv, *s_mlp, *s_lin2;
+  // NVFP4 precision: codes, block scales and row scales of the same matrices
+  Fp4Op q4_qkv, q4_mlp, q4_lin2;
 };
 
 // Row ranges of the joint sequence: text | image | reference (all references together).
@@ -154,6 +156,17 @@ struct Workspace3 {
   float *sY = nullptr, *sC = nullptr;
   bool maps8 = false;
   CUtensorMap a8_Yall[kMaxBatch3], a8_Yseg[kMaxBatch3][3], a8_CCseg[kMaxBatch3][3];
+  // NVFP4 precision: codes of the LN-mod output (Y4) and of [O | H] (C4), block scales (sfY, sfC)
+  // and row scales.  Each GEMM problem's rows start on a 128-row block of its scales, so the
+  // quantisations follow the problems: per stream segment in the per-mode blocks (seg_pm: text,
+  // image, reference of sequence 0, then the other sequences' text), per sequence for the joint
+  // linear1 (seg_jy) and per token type and sequence for the joint linear2 (seg_jc).
+  size_t cap4_rows = 0, cap4_blocks = 0;
+  uint8_t *Y4 = nullptr, *C4 = nullptr, *sfY = nullptr, *sfC = nullptr;
+  float *sY4 = nullptr, *sC4 = nullptr;
+  bool maps4 = false;
+  Q4Segs seg_pm, seg_jy, seg_jc;
+  Fp4Op y4_pm[kMaxBatch3][3], c4_pm[kMaxBatch3][3], y4_all[kMaxBatch3], c4_seg[kMaxBatch3][3];
 };
 
 // Offsets (in units of D floats) of the modulation vectors in the model's mods buffer.
@@ -181,6 +194,8 @@ struct flux3_dit {
   int precision = FLUX_PRECISION_BF16;
   uint8_t* w8 = nullptr;               // e4m3 block linears (allocated on the first switch to FP8)
   float* w8_scale = nullptr;
+  uint8_t* w4 = nullptr;               // NVFP4 block linears (first switch to NVFP4)
+  float* w4_scale = nullptr;
   fdit::Workspace3 ws;
   fdit::Profiler prof;
 };
@@ -196,8 +211,17 @@ void free_ws3_fp8(Workspace3& w) {
   w.maps8 = false;
 }
 
+void free_ws3_fp4(Workspace3& w) {
+  cudaFree(w.Y4); cudaFree(w.C4); cudaFree(w.sfY); cudaFree(w.sfC); cudaFree(w.sY4); cudaFree(w.sC4);
+  w.Y4 = w.C4 = w.sfY = w.sfC = nullptr;
+  w.sY4 = w.sC4 = nullptr;
+  w.cap4_rows = w.cap4_blocks = 0;
+  w.maps4 = false;
+}
+
 void free_ws3(Workspace3& w) {
   free_ws3_fp8(w);
+  free_ws3_fp4(w);
   cudaFree(w.X); cudaFree(w.Y); cudaFree(w.QKV); cudaFree(w.CC); cudaFree(w.tokb); cudaFree(w.txtb);
   cudaFree(w.rope);
   w = Workspace3();
@@ -208,6 +232,8 @@ void destroy3(flux3_dit* m) {
   free_ws3(m->ws);
   cudaFree(m->w8);
   cudaFree(m->w8_scale);
+  cudaFree(m->w4);
+  cudaFree(m->w4_scale);
   cudaFree(m->wbuf);
   cudaFree(m->scratch);
   delete m;
@@ -351,6 +377,87 @@ int prepare3_fp8(flux3_dit* m, int nt, int ni, int nr, int nb) {
   return FLUX_OK;
 }
 
+// NVFP4 copies of the GEMM A operands and their maps for nb sequences of nt + ni + nr rows.
+int prepare3_fp4(flux3_dit* m, int nt, int ni, int nr, int nb) {
+  Workspace3& w = m->ws;
+  const flux3_dit_config& c = m->cfg;
+  const size_t D = c.hidden, F = c.mlp_hidden;
+  const int n = nt + ni + nr, rows = n * nb;
+  const int row0[3] = {0, nt, nt + ni}, seg[3] = {nt, ni, nr};
+  int r0[2 * kMaxBatch3 * 3], rs[2 * kMaxBatch3 * 3], nz = 0;
+  for (int sg = 0; sg < 3; ++sg, ++nz) {               // per-mode: sequence 0's streams, the others' text
+    r0[nz] = row0[sg];
+    rs[nz] = seg[sg];
+  }
+  for (int bb = 1; bb < nb; ++bb, ++nz) {
+    r0[nz] = bb * n;
+    rs[nz] = nt;
+  }
+  w.seg_pm = q4_segments(r0, rs, nz);
+  for (int bb = 0; bb < nb; ++bb) {
+    r0[bb] = bb * n;
+    rs[bb] = n;
+  }
+  w.seg_jy = q4_segments(r0, rs, nb);
+  for (int bb = 0; bb < nb; ++bb)
+    for (int sg = 0; sg < 3; ++sg) {
+      r0[3 * bb + sg] = bb * n + row0[sg];
+      rs[3 * bb + sg] = seg[sg];
+    }
+  w.seg_jc = q4_segments(r0, rs, 3 * nb);
+  auto blocks_of = [](const Q4Segs& g) {
+    size_t b = 0;
+    for (int z = 0; z < g.n; ++z) b += (g.rows[z] + 127) / 128;
+    return b;
+  };
+  const size_t blocks = std::max(blocks_of(w.seg_pm), std::max(blocks_of(w.seg_jy), blocks_of(w.seg_jc)));
+  if (static_cast<size_t>(rows) > w.cap4_rows || blocks > w.cap4_blocks) {
+    free_ws3_fp4(w);
+    const size_t R = rows, B = blocks * 128;
+    const bool ok = cudaMalloc(&w.Y4, R * D / 2) == cudaSuccess && cudaMalloc(&w.C4, R * (D + F) / 2) == cudaSuccess &&
+                    cudaMalloc(&w.sfY, B * D / 16) == cudaSuccess &&
+                    cudaMalloc(&w.sfC, B * (D + F) / 16) == cudaSuccess && cudaMalloc(&w.sY4, R * 4) == cudaSuccess &&
+                    cudaMalloc(&w.sC4, R * 4) == cudaSuccess;
+    if (!ok) {
+      free_ws3_fp4(w);
+      return fail(FLUX_ENOMEM, "NVFP4 workspace allocation for %d tokens failed", rows);
+    }
+    w.cap4_rows = R;
+    w.cap4_blocks = blocks;
+  }
+  if (w.maps4) return FLUX_OK;
+  bool ok = true;
+  const size_t lY = D / 2, lC = (D + F) / 2;
+  auto y_op = [&](Fp4Op* o, size_t r, int nrows, int blk0) {
+    ok &= make_fp4_op(o, w.Y4 + r * lY, nrows, D, lY, w.sfY, blk0, w.sY4 + r);
+  };
+  auto c_op = [&](Fp4Op* o, size_t r, int nrows, int blk0) {
+    ok &= make_fp4_op(o, w.C4 + r * lC, nrows, D + F, lC, w.sfC, blk0, w.sC4 + r);
+  };
+  for (int sg = 0; sg < 3; ++sg) {
+    y_op(&w.y4_pm[0][sg], row0[sg], seg[sg], w.seg_pm.blk0[sg]);
+    c_op(&w.c4_pm[0][sg], row0[sg], seg[sg], w.seg_pm.blk0[sg]);
+  }
+  for (int bb = 1; bb < nb; ++bb) {
+    y_op(&w.y4_pm[bb][0], static_cast<size_t>(bb) * n, nt, w.seg_pm.blk0[2 + bb]);
+    c_op(&w.c4_pm[bb][0], static_cast<size_t>(bb) * n, nt, w.seg_pm.blk0[2 + bb]);
+  }
+  for (int bb = 0; bb < nb; ++bb) {
+    y_op(&w.y4_all[bb], static_cast<size_t>(bb) * n, n, w.seg_jy.blk0[bb]);
+    for (int sg = 0; sg < 3; ++sg)
+      c_op(&w.c4_seg[bb][sg], static_cast<size_t>(bb) * n + row0[sg], seg[sg], w.seg_jc.blk0[3 * bb + sg]);
+  }
+  if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an NVFP4 activation buffer");
+  w.maps4 = true;
+  return FLUX_OK;
+}
+
+int prepare3_quant(flux3_dit* m, int nt, int ni, int nr, int nb) {
+  if (m->precision == FLUX_PRECISION_FP8) return prepare3_fp8(m, nt, ni, nr, nb);
+  if (m->precision == FLUX_PRECISION_NVFP4) return prepare3_fp4(m, nt, ni, nr, nb);
+  return FLUX_OK;
+}
+
 int prepare_shape3(flux3_dit* m, int nt, int gh, int gw, const RefGrids& refs, int nb, cudaStream_t s) {
   Workspace3& w = m->ws;
   const flux3_dit_config& c = m->cfg;
@@ -373,10 +480,10 @@ int prepare_shape3(flux3_dit* m, int nt, int gh, int gw, const RefGrids& refs, i
   if (grow(&w.tokb, &w.cap_tok, (ni + nr) * c.in_ch) != cudaSuccess ||
       grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt * nb, 1) * c.txt_dim) != cudaSuccess)
     return fail(FLUX_ENOMEM, "workspace allocation failed");
-  const bool fp8 = m->precision == FLUX_PRECISION_FP8;
   if (w.nt == nt && w.gh == gh && w.gw == gw && w.nb == nb && same_refs(w.refs, refs))
-    return fp8 ? prepare3_fp8(m, nt, static_cast<int>(ni), static_cast<int>(nr), nb) : FLUX_OK;
+    return prepare3_quant(m, nt, static_cast<int>(ni), static_cast<int>(nr), nb);
   w.maps8 = false;
+  w.maps4 = false;
 
   const uint64_t ldD = D * 2, ldC = (D + F) * 2;
   bool ok = true;
@@ -406,7 +513,7 @@ int prepare_shape3(flux3_dit* m, int nt, int gh, int gw, const RefGrids& refs, i
   if (rope_table_launch(w.rope, nt, gh, gw, refs, c.rope_theta, s) != cudaSuccess)
     return fail(FLUX_EIO, "rope table launch failed");
   w.nt = nt; w.gh = gh; w.gw = gw; w.nb = nb; w.refs = refs;
-  return fp8 ? prepare3_fp8(m, nt, static_cast<int>(ni), static_cast<int>(nr), nb) : FLUX_OK;
+  return prepare3_quant(m, nt, static_cast<int>(ni), static_cast<int>(nr), nb);
 }
 
 // Quantise every block linear (per-mode streams and joint blocks) to e4m3, one scale per row.
@@ -446,6 +553,34 @@ int quantize3_block_weights(flux3_dit* m, cudaStream_t s) {
     bw.s_lin2 = sc2;
   }
   if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an FP8 weight tensor");
+  FD_CUDA(cudaStreamSynchronize(s));
+  return FLUX_OK;
+}
+
+// Quantise every block linear (per-mode streams and joint blocks) to NVFP4.
+int quantize3_block_weights_nvfp4(flux3_dit* m, cudaStream_t s) {
+  const flux3_dit_config& c = m->cfg;
+  const size_t D = c.hidden, F = c.mlp_hidden;
+  std::vector<BlockW3*> blocks;
+  for (BlockW3& b : m->mode) blocks.push_back(&b);
+  for (BlockW3& b : m->joint) blocks.push_back(&b);
+  std::vector<Fp4Mat> mats;
+  for (BlockW3* b : blocks) {
+    mats.push_back({b->w_lin1, 3 * D + 2 * F, D});
+    mats.push_back({b->w_lin2, D, D + F});
+  }
+  int rc = quantize_weights_nvfp4(mats, &m->w4, &m->w4_scale, s);
+  if (rc) return rc;
+  bool ok = true;
+  auto op = [&](Fp4Op* o, const Fp4Mat& x, size_t row0, size_t rows) {
+    ok &= make_fp4_op(o, x.codes + row0 * x.cols / 2, rows, x.cols, x.cols / 2, x.sf, row0 / 128, x.scale + row0);
+  };
+  for (size_t i = 0; i < blocks.size(); ++i) {
+    op(&blocks[i]->q4_qkv, mats[2 * i], 0, 3 * D);
+    op(&blocks[i]->q4_mlp, mats[2 * i], 3 * D, 2 * F);  // the SwiGLU rows start on a 128-row block
+    op(&blocks[i]->q4_lin2, mats[2 * i + 1], 0, D);
+  }
+  if (!ok) return fail(FLUX_EIO, "cuTensorMapEncodeTiled failed for an NVFP4 weight tensor");
   FD_CUDA(cudaStreamSynchronize(s));
   return FLUX_OK;
 }
@@ -553,7 +688,8 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
   const bool fp8 = m->precision == FLUX_PRECISION_FP8;
 
   // input projections: every text, the image and reference tokens once (sequence 0's rows)
-  GemmParams P;
+  GemmParams4 P4;
+  GemmParams& P = P4.g;
   P.num_problems = 2;
   problem(P, 0, w.a_txtb[0], m->m_txt_in, nt, D, c.txt_dim, kEpiF32Bias, w.X, D, m->txt_b, nullptr);
   problem(P, 1, w.a_tokb, m->m_img_in, ni + nr, D, c.in_ch, kEpiF32Bias, w.X + nt * sD, D, m->img_b, nullptr);
@@ -577,6 +713,20 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
     P.prob[i].scale_a = sa;
     P.prob[i].scale_b = sb;
   };
+  // NVFP4 precision: LN-mod writes bf16 and the rows are quantised per segment (`segs`); [O | H]
+  // likewise before linear2
+  const bool fp4 = m->precision == FLUX_PRECISION_NVFP4;
+  auto linear_as = [&](bool small) -> cudaError_t {
+    return fp4 ? gemm_fp4_launch(P4, m->num_sms, s) : launch_linear_as(P, m->num_sms, s, fp8, small);
+  };
+  auto quant4 = [&](const bf16* x, int k, uint8_t* q, uint8_t* sf, float* sc, const Q4Segs& segs) -> int {
+    double r = 0;
+    for (int z = 0; z < segs.n; ++z) r += segs.rows[z];
+    FD_LAUNCH(m, kProfOther, 0, 2.5 * r * k + 4.0 * r,
+              quantize_nvfp4_launch(x, static_cast<int>(k == D ? D : D + F), k, q, k == D ? D / 2 : (D + F) / 2, sf,
+                                    sc, segs, s));
+    return FLUX_OK;
+  };
   // LN + modulation of rows [0, r) (text | image | reference per sequence of n rows)
   auto ln3 = [&](int r, const float* sh0, const float* sc0, const float* sh1, const float* sc1, const float* sh2,
                  const float* sc2) -> int {
@@ -588,6 +738,12 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
       FD_LAUNCH(m, kProfLnMod, 0, 6.0 * r * D + 16.0 * D,
                 ln_modulate3_launch(w.X, w.Y, r, D, nt, nt + ni, n, sh0, sc0, sh1, sc1, sh2, sc2, eps_ln, s));
     return FLUX_OK;
+  };
+  auto ln3q = [&](int r, const Q4Segs& segs, const float* sh0, const float* sc0, const float* sh1, const float* sc1,
+                  const float* sh2, const float* sc2) -> int {
+    const int rc2 = ln3(r, sh0, sc0, sh1, sc1, sh2, sc2);
+    if (rc2 || !fp4) return rc2;
+    return quant4(w.Y, D, w.Y4, w.sfY, w.sY4, segs);
   };
   auto quant_cc = [&](int r) -> int {
     FD_LAUNCH(m, kProfOther, 0, 3.0 * r * sDF + 4.0 * r, quantize_rows_launch(w.CC, D + F, r, D + F, w.C8, D + F, w.sC, s));
@@ -606,7 +762,8 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
   }
   const int mode_set[3] = {kModTxt, kModImg, kModRef};
   for (int i = 0; i < m->act_mode; ++i) {
-    rc = ln3(rows_pm, md(kModTxt), md(kModTxt + 1), md(kModImg), md(kModImg + 1), md(kModRef), md(kModRef + 1));
+    rc = ln3q(rows_pm, w.seg_pm, md(kModTxt), md(kModTxt + 1), md(kModImg), md(kModImg + 1), md(kModRef),
+              md(kModRef + 1));
     if (rc) return rc;
     // linear1: (qkv + QK-RMSNorm + RoPE, SwiGLU) per stream of sequence 0, then the other texts
     P.num_problems = 0;
@@ -622,13 +779,18 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
         f8(j, w.a8_Yseg[bb][sg], bw.m8_qkv, w.sY + r0 + row0[sg], bw.s_qkv);
         f8(j + 1, w.a8_Yseg[bb][sg], bw.m8_mlp, w.sY + r0 + row0[sg], bw.s_mlp);
       }
+      if (fp4) {
+        fp4_operands(P4, j, w.y4_pm[bb][sg], bw.q4_qkv);
+        fp4_operands(P4, j + 1, w.y4_pm[bb][sg], bw.q4_mlp);
+      }
       P.num_problems += 2;
     };
     for (int sg = 0; sg < 3; ++sg) lin1(sg, 0);
     for (int bb = 1; bb < nb; ++bb) lin1(kSegTxt, static_cast<size_t>(bb) * n);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), gemm2_launch(P, m->num_sms, s, fp8));   // SwiGLU: pair kernel
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear_as(false));   // SwiGLU: pair kernel
     FD_LAUNCH(m, kProfAttention, seg_flops, 8.0 * rows_pm * D, attention_launch(As, s));
     if (fp8 && (rc = quant_cc(rows_pm))) return rc;
+    if (fp4 && (rc = quant4(w.CC, D + F, w.C4, w.sfC, w.sC4, w.seg_pm))) return rc;
     // linear2 with each stream's gate into the residual; the kernel is chosen for sequence 0's streams
     P.num_problems = 0;
     auto lin2 = [&](int sg, size_t r0) {
@@ -637,11 +799,12 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
       problem(P, j, w.a_CCseg[bb][sg], bw.m_lin2, seg[sg], D, D + F, kEpiResidGate, w.X + (r0 + row0[sg]) * sD, D,
               bw.lin2_b, md(mode_set[sg] + 2));
       if (fp8) f8(j, w.a8_CCseg[bb][sg], bw.m8_lin2, w.sC + r0 + row0[sg], bw.s_lin2);
+      if (fp4) fp4_operands(P4, j, w.c4_pm[bb][sg], bw.q4_lin2);
     };
     for (int sg = 0; sg < 3; ++sg) lin2(sg, 0);
     const bool small = small_linear(P, m->num_sms, fp8, 1);
     for (int bb = 1; bb < nb; ++bb) lin2(kSegTxt, static_cast<size_t>(bb) * n);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear_as(P, m->num_sms, s, fp8, small));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear_as(small));
   }
   // the image and reference streams of sequence 0 into the other sequences
   for (int bb = 1; bb < nb; ++bb)
@@ -656,8 +819,8 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
   A.batch = nb;
   for (int i = 0; i < m->act_joint; ++i) {
     const BlockW3& bw = m->joint[i];
-    rc = ln3(rows_all, md(kModJointCtx), md(kModJointCtx + 1), md(kModJointImg), md(kModJointImg + 1),
-             md(kModJointCtx), md(kModJointCtx + 1));
+    rc = ln3q(rows_all, w.seg_jy, md(kModJointCtx), md(kModJointCtx + 1), md(kModJointImg), md(kModJointImg + 1),
+              md(kModJointCtx), md(kModJointCtx + 1));
     if (rc) return rc;
     P.num_problems = 2 * nb;
     for (int bb = 0; bb < nb; ++bb) {
@@ -671,10 +834,15 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
         f8(2 * bb, w.a8_Yall[bb], bw.m8_qkv, w.sY + r0, bw.s_qkv);
         f8(2 * bb + 1, w.a8_Yall[bb], bw.m8_mlp, w.sY + r0, bw.s_mlp);
       }
+      if (fp4) {
+        fp4_operands(P4, 2 * bb, w.y4_all[bb], bw.q4_qkv);
+        fp4_operands(P4, 2 * bb + 1, w.y4_all[bb], bw.q4_mlp);
+      }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear_as(small_linear(P, m->num_sms, fp8, nb)));
     FD_LAUNCH(m, kProfAttention, at_flops, 8.0 * rows_all * D, attention_launch(A, s));
     if (fp8 && (rc = quant_cc(rows_all))) return rc;
+    if (fp4 && (rc = quant4(w.CC, D + F, w.C4, w.sfC, w.sC4, w.seg_jc))) return rc;
     P.num_problems = 3 * nb;
     for (int bb = 0; bb < nb; ++bb)
       for (int sg = 0; sg < 3; ++sg) {
@@ -682,8 +850,9 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
         problem(P, 3 * bb + sg, w.a_CCseg[bb][sg], bw.m_lin2, seg[sg], D, D + F, kEpiResidGate, w.X + r * sD, D,
                 bw.lin2_b, md(joint_set[sg] + 2));
         if (fp8) f8(3 * bb + sg, w.a8_CCseg[bb][sg], bw.m8_lin2, w.sC + r, bw.s_lin2);
+        if (fp4) fp4_operands(P4, 3 * bb + sg, w.c4_seg[bb][sg], bw.q4_lin2);
       }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), launch_linear(P, m->num_sms, s, fp8, nb));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear_as(small_linear(P, m->num_sms, fp8, nb)));
   }
 
   // ---------------- output layer on the image rows (text and reference tokens are dropped)
@@ -763,16 +932,24 @@ int flux3_dit_set_precision(flux3_dit* m, int precision) {
     m->precision = precision;
     return FLUX_OK;
   }
-  if (precision != FLUX_PRECISION_FP8) return fail(FLUX_EINVAL, "unknown precision %d", precision);
+  if (precision != FLUX_PRECISION_FP8 && precision != FLUX_PRECISION_NVFP4)
+    return fail(FLUX_EINVAL, "unknown precision %d", precision);
   const flux3_dit_config& c = m->cfg;
-  if ((c.hidden != 1024 && c.hidden != 2048 && c.hidden != 3072 && c.hidden != 4096) ||
-      c.hidden + c.mlp_hidden > 16384)
+  if (precision == FLUX_PRECISION_FP8 &&
+      ((c.hidden != 1024 && c.hidden != 2048 && c.hidden != 3072 && c.hidden != 4096) ||
+       c.hidden + c.mlp_hidden > 16384))
     return fail(FLUX_EINVAL, "FP8 needs hidden in {1024, 2048, 3072, 4096} and hidden + mlp_hidden <= 16384");
+  if (precision == FLUX_PRECISION_NVFP4 && (c.hidden % 256 || c.mlp_hidden % 256 || c.hidden + c.mlp_hidden > 16384))
+    return fail(FLUX_EINVAL, "NVFP4 needs hidden and mlp_hidden multiples of 256 and hidden + mlp_hidden <= 16384");
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev != m->device) return fail(FLUX_EINVAL, "model lives on device %d, current device is %d", m->device, dev);
-  if (!m->w8) {
+  if (precision == FLUX_PRECISION_FP8 && !m->w8) {
     const int rc = quantize3_block_weights(m, nullptr);
+    if (rc) return rc;
+  }
+  if (precision == FLUX_PRECISION_NVFP4 && !m->w4) {
+    const int rc = quantize3_block_weights_nvfp4(m, nullptr);
     if (rc) return rc;
   }
   m->precision = precision;

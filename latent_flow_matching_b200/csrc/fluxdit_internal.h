@@ -140,8 +140,16 @@ cudaError_t ln_modulate_fp8_launch(const float* x, uint8_t* q, float* qscale, in
 // block scales (sf, nvfp4_scale_bytes(rows, k) bytes, 512-byte blocks of 128 rows x 64 elements)
 // and fp32 row scales; k % 64 == 0, k <= 16384.
 inline size_t nvfp4_scale_bytes(size_t rows, size_t k) { return (rows + 127) / 128 * 128 * (k / 16); }
-cudaError_t quantize_nvfp4_launch(const __nv_bfloat16* x, int ldx, int rows, int k, uint8_t* q, int ldq, uint8_t* sf,
-                                  float* row_scale, cudaStream_t s);
+// Row segments of one quantisation: segment z is rows [row0, row0 + rows) and its block scales
+// start at 128-row block blk0 of the scale buffer (q4_segments packs them one after another).
+constexpr int kMaxQ4Segs = 8;
+struct Q4Segs {
+  int n;
+  int row0[kMaxQ4Segs], rows[kMaxQ4Segs], blk0[kMaxQ4Segs];
+};
+Q4Segs q4_segments(const int* row0, const int* rows, int n);
+cudaError_t quantize_nvfp4_launch(const __nv_bfloat16* x, int ldx, int k, uint8_t* q, int ldq, uint8_t* sf,
+                                  float* row_scale, const Q4Segs& segs, cudaStream_t s);
 // Problems of the NVFP4 pair GEMM: mapA / mapB over the codes (u8 maps, 128-byte box), K in elements
 // (K % 256 == 0), scale_a / scale_b the fp32 row scales, and the block scales' maps (make_tmap_sf).
 struct GemmParams4 {

@@ -34,11 +34,18 @@ __device__ __forceinline__ float bf16_abs_max8(const uint4& w, float m) {
   return m;
 }
 
+// One CTA per row.  Rows come in segments (Q4Segs): segment z is rows [row0, row0 + rows) of x, q
+// and row_scale, and its scales start at 128-row block blk0 of sf, so that a GEMM problem over
+// that segment finds its first row at the start of a scale block.
 __global__ void __launch_bounds__(kQ4Threads) quantize_nvfp4_kernel(const __nv_bfloat16* __restrict__ x, int ldx,
                                                                     int k, uint8_t* __restrict__ q, int ldq,
-                                                                    uint8_t* __restrict__ sf, float* __restrict__ row_scale) {
+                                                                    uint8_t* __restrict__ sf, float* __restrict__ row_scale,
+                                                                    const Q4Segs segs) {
   __shared__ float red[kQ4Threads / 32];
-  const int r = blockIdx.x;
+  int z = 0, l = blockIdx.x;
+  while (z + 1 < segs.n && l >= segs.rows[z]) l -= segs.rows[z++];
+  const int r = segs.row0[z] + l;                  // row of x, q and row_scale
+  const int sfr = segs.blk0[z] * 128 + l;          // row of the scale layout
   const int units = k / 64;
   const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(r) * ldx);
   uint4 v[kQ4MaxUnits][8];
@@ -66,7 +73,7 @@ __global__ void __launch_bounds__(kQ4Threads) quantize_nvfp4_kernel(const __nv_b
   const float S = __fdiv_rn(amax, 2688.0f);
   if (threadIdx.x == 0) row_scale[r] = S;
   uint8_t* qr = q + static_cast<size_t>(r) * ldq;
-  const size_t sf_row = 16 * (r & 31) + 4 * ((r & 127) >> 5);
+  const size_t sf_row = 16 * (sfr & 31) + 4 * ((sfr & 127) >> 5);
 #pragma unroll
   for (int u = 0; u < kQ4MaxUnits; ++u) {
     const int unit = threadIdx.x + u * kQ4Threads;
@@ -96,22 +103,40 @@ __global__ void __launch_bounds__(kQ4Threads) quantize_nvfp4_kernel(const __nv_b
     uint4* dq = reinterpret_cast<uint4*>(qr + unit * 32);
     dq[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
     dq[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-    const size_t blk = static_cast<size_t>(r >> 7) * units + unit;
+    const size_t blk = static_cast<size_t>(sfr >> 7) * units + unit;
     *reinterpret_cast<uint32_t*>(sf + blk * 512 + sf_row) = sfw;
   }
 }
 
 }  // namespace
 
-cudaError_t quantize_nvfp4_launch(const __nv_bfloat16* x, int ldx, int rows, int k, uint8_t* q, int ldq, uint8_t* sf,
-                                  float* row_scale, cudaStream_t s) {
-  if (rows < 0 || k <= 0 || k % 64 != 0 || k > kQ4Threads * 64 * kQ4MaxUnits || ldx < k || ldx % 8 != 0 ||
-      ldq < k / 2 || ldq % 16 != 0)
+cudaError_t quantize_nvfp4_launch(const __nv_bfloat16* x, int ldx, int k, uint8_t* q, int ldq, uint8_t* sf,
+                                  float* row_scale, const Q4Segs& segs, cudaStream_t s) {
+  if (k <= 0 || k % 64 != 0 || k > kQ4Threads * 64 * kQ4MaxUnits || ldx < k || ldx % 8 != 0 || ldq < k / 2 ||
+      ldq % 16 != 0 || segs.n < 1 || segs.n > kMaxQ4Segs)
     return cudaErrorInvalidValue;
-  if (rows == 0) return cudaSuccess;
+  long total = 0;
+  for (int z = 0; z < segs.n; ++z) {
+    if (segs.rows[z] < 0 || segs.row0[z] < 0 || segs.blk0[z] < 0) return cudaErrorInvalidValue;
+    total += segs.rows[z];
+  }
+  if (total == 0) return cudaSuccess;
   count_launch();
-  quantize_nvfp4_kernel<<<rows, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale);
+  quantize_nvfp4_kernel<<<static_cast<unsigned>(total), kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs);
   return cudaGetLastError();
+}
+
+Q4Segs q4_segments(const int* row0, const int* rows, int n) {
+  Q4Segs g{};
+  g.n = n;
+  int blk = 0;
+  for (int z = 0; z < n; ++z) {
+    g.row0[z] = row0[z];
+    g.rows[z] = rows[z];
+    g.blk0[z] = blk;
+    blk += (rows[z] + 127) / 128;
+  }
+  return g;
 }
 
 }  // namespace fdit

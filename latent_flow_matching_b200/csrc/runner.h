@@ -6,6 +6,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <cstring>
 #include <string>
 #include <vector>
 
@@ -162,6 +163,75 @@ inline cudaError_t launch_linear_as(GemmParams& P, int num_sms, cudaStream_t s, 
 
 inline cudaError_t launch_linear(GemmParams& P, int num_sms, cudaStream_t s, bool fp8, int nb = 1) {
   return launch_linear_as(P, num_sms, s, fp8, small_linear(P, num_sms, fp8, nb));
+}
+
+// ------------------------------------------------------------------ NVFP4 operands
+// One NVFP4 GEMM operand: rows [0, rows) of a codes buffer (row stride ldq bytes), its block scales
+// starting at 128-row block blk0 of a scale buffer, and its fp32 row scales.
+struct Fp4Op {
+  CUtensorMap codes, sf;
+  const float* scale = nullptr;
+};
+
+inline bool make_fp4_op(Fp4Op* op, const uint8_t* codes, size_t rows, size_t k, size_t ldq, const uint8_t* sf,
+                        size_t blk0, const float* scale) {
+  op->scale = scale;
+  if (rows == 0) {
+    memset(&op->codes, 0, sizeof(CUtensorMap));
+    memset(&op->sf, 0, sizeof(CUtensorMap));
+    return true;
+  }
+  return make_tmap_u8(&op->codes, codes, rows, k / 2, ldq, 128) &&
+         make_tmap_sf(&op->sf, sf + blk0 * (k / 64) * 512, nvfp4_scale_bytes(rows, k));
+}
+
+// Problem i of an NVFP4 grouped GEMM takes activation operand a and weight operand w.
+inline void fp4_operands(GemmParams4& P4, int i, const Fp4Op& a, const Fp4Op& w) {
+  P4.g.mapA[i] = a.codes;
+  P4.g.mapB[i] = w.codes;
+  P4.mapSFA[i] = a.sf;
+  P4.mapSFB[i] = w.sf;
+  P4.g.prob[i].scale_a = a.scale;
+  P4.g.prob[i].scale_b = w.scale;
+}
+
+// Quantise weight matrices (bf16 [rows, cols], row stride cols) to NVFP4 in one device allocation
+// (*buf: codes and block scales, *scales: row scales).  Fills each matrix's codes / sf / scale.
+struct Fp4Mat {
+  const bf16* w;
+  size_t rows, cols;
+  uint8_t* codes = nullptr;
+  uint8_t* sf = nullptr;
+  float* scale = nullptr;
+};
+inline int quantize_weights_nvfp4(std::vector<Fp4Mat>& mats, uint8_t** buf, float** scales, cudaStream_t s) {
+  auto up = [](size_t v, size_t a) { return (v + a - 1) / a * a; };
+  size_t bytes = 0, rows = 0;
+  for (const Fp4Mat& x : mats) {
+    bytes += up(x.rows * x.cols / 2, 256) + up(nvfp4_scale_bytes(x.rows, x.cols), 256);
+    rows += up(x.rows, 64);
+  }
+  if (cudaMalloc(buf, bytes) != cudaSuccess || cudaMalloc(scales, rows * 4) != cudaSuccess) {
+    cudaFree(*buf);
+    cudaFree(*scales);
+    *buf = nullptr;
+    *scales = nullptr;
+    return fail(FLUX_ENOMEM, "cudaMalloc of the NVFP4 weights (%zu bytes) failed", bytes);
+  }
+  FD_CUDA(cudaMemsetAsync(*buf, 0, bytes, s));       // block-scale padding rows read as 0
+  size_t boff = 0, roff = 0;
+  for (Fp4Mat& x : mats) {
+    x.codes = *buf + boff;
+    boff += up(x.rows * x.cols / 2, 256);
+    x.sf = *buf + boff;
+    boff += up(nvfp4_scale_bytes(x.rows, x.cols), 256);
+    x.scale = *scales + roff;
+    roff += up(x.rows, 64);
+    const int r0 = 0, nr = static_cast<int>(x.rows);
+    FD_CUDA(quantize_nvfp4_launch(x.w, static_cast<int>(x.cols), static_cast<int>(x.cols), x.codes,
+                                  static_cast<int>(x.cols / 2), x.sf, x.scale, q4_segments(&r0, &nr, 1), s));
+  }
+  return FLUX_OK;
 }
 
 // Grow a device buffer to `need` elements (contents are not kept).

@@ -23,7 +23,9 @@ Readings where the pages are silent (each is listed in the design doc):
       value_j = code_j * s_b * S;
   an all-zero row, or a block whose scale rounds to 0, has codes 0;
 * y = sum over blocks of (codes_x . codes_w) s_bx s_bw, times S_x S_w, plus the bias;
-* it applies where the row-wise FP8 format does: the linears inside the transformer blocks.
+* it applies where the row-wise FP8 format does: the linears inside the transformer blocks, whose
+  activations enter the quantiser as bf16 (``flux_oracle.block_linear`` rounds them first: a code
+  is an integer decision, taken in the precision the GPU path quantises from).
 """
 from __future__ import annotations
 

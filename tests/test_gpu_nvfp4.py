@@ -19,6 +19,11 @@ pytestmark = pytest.mark.gpu
 torch.set_grad_enabled(False)
 DEV = "cuda"
 TOL = 1e-2
+# NVFP4 forward against the NVFP4 oracle.  An e2m1 step is 1/4 to 1/2 of the value (e4m3: 1/16 to
+# 1/8), so where the GPU's bf16 intermediates differ from the oracle's float64 ones by an ulp, a
+# code flips with a proportionally larger jump than in FP8 (bar 2e-2); measured 1.5 to 2.2 % on the
+# tiny models, against a format error of 4.3 to 4.7 % (NVFP4 oracle vs exact oracle).
+NV4_V_TOL = 3e-2
 
 
 def nmax(gpu, ref):
@@ -178,3 +183,135 @@ def test_linear_nvfp4_full_size_sampled_rows():
     full = a[rows].double() @ w.double().t() + b.double()
     rel = ((out[rows].cpu().double() - full).norm() / full.norm()).item()
     assert 0.02 < rel < 0.2, rel
+
+
+# ---------------------------------------------------------------------------- forwards in NVFP4
+from oracle import flux3_oracle as O3                      # noqa: E402
+from synthetic import WORKLOADS, make_weights, make_inputs  # noqa: E402
+
+
+def rel_l2(a, b):
+    a = torch.as_tensor(a).double().cpu()
+    b = torch.as_tensor(b).double().cpu()
+    return ((a - b).norm() / b.norm()).item()
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    w = WORKLOADS["tiny64"]
+    blob, p = make_weights(w.dims, w.seed)
+    model = F.FluxDiT(blob, w.dims)
+    yield w, p, model
+    model.close()
+
+
+@pytest.mark.parametrize("n_txt,grid,refs", [(16, (4, 4), []), (131, (8, 8), [(4, 8)]), (0, (4, 6), []),
+                                             (200, (12, 12), [(12, 12)])])
+def test_tiny_nvfp4_forward_against_nvfp4_oracle(tiny, n_txt, grid, refs):
+    w, p, model = tiny
+    g = torch.Generator().manual_seed(180 + n_txt)
+    tok = torch.randn(grid[0] * grid[1], 128, generator=g).to(torch.bfloat16).float()
+    txt = torch.randn(n_txt, 3072, generator=g).to(torch.bfloat16).float()
+    ref_tok = [torch.randn(h * w_, 128, generator=g).to(torch.bfloat16).float() for h, w_ in refs]
+    hq = dict(O.hyper(w.dims), nvfp4=True)
+    want = O.forward(p, hq, tok, txt, 0.6, grid, ref_tok, refs)
+    exact = O.forward(p, O.hyper(w.dims), tok, txt, 0.6, grid, ref_tok, refs)
+    v = torch.empty(grid[0] * grid[1], 128, device=DEV)
+    v16 = torch.empty_like(v)
+    hw = refs if refs else (0, 0)
+    rt = torch.cat(ref_tok).to(DEV) if refs else None
+    model.forward(tok.to(DEV), grid, txt.to(DEV) if n_txt else None, 0.6, v16, rt, hw)
+    model.set_precision(F.PRECISION_NVFP4)
+    try:
+        model.forward(tok.to(DEV), grid, txt.to(DEV) if n_txt else None, 0.6, v, rt, hw)
+    finally:
+        model.set_precision(F.PRECISION_BF16)
+    err = rel_l2(v, want)
+    print(f"nvfp4 forward vs nvfp4 oracle {err:.4f}, vs exact oracle {rel_l2(v, exact):.4f}, "
+          f"nvfp4 oracle vs exact {rel_l2(want, exact):.4f}")
+    assert err <= NV4_V_TOL, err
+    assert err < 0.6 * rel_l2(v, exact)                     # it quantises the way the oracle does
+    assert rel_l2(v, exact) > rel_l2(v16, exact)
+    again = torch.empty_like(v)
+    model.forward(tok.to(DEV), grid, txt.to(DEV) if n_txt else None, 0.6, again, rt, hw)
+    assert torch.equal(again, v16)                          # back to bf16, bit for bit
+
+
+def test_nvfp4_guided_batch_equals_two_single_forwards(tiny):
+    w, p, model = tiny
+    g = torch.Generator().manual_seed(190)
+    grid = (6, 4)
+    tok = torch.randn(24, 128, generator=g).to(torch.bfloat16).float().to(DEV)
+    tc = torch.randn(131, 3072, generator=g).to(torch.bfloat16).float().to(DEV)
+    tu = torch.randn(131, 3072, generator=g).to(torch.bfloat16).float().to(DEV)
+    vc, vu, a, b = (torch.empty(24, 128, device=DEV) for _ in range(4))
+    model.set_precision(F.PRECISION_NVFP4)
+    try:
+        model.forward_cfg(tok, grid, tc, tu, 0.6, vc, vu)
+        model.forward(tok, grid, tc, 0.6, a)
+        model.forward(tok, grid, tu, 0.6, b)
+    finally:
+        model.set_precision(F.PRECISION_BF16)
+    assert torch.equal(vc, a) and torch.equal(vu, b)
+
+
+def test_nvfp4_forward_full_size_against_bf16_and_fp8():
+    """1024^2 workload, full model: NVFP4 is the coarser format, so it lands further from bf16 than FP8."""
+    w = WORKLOADS["t2i1024"]
+    blob, _ = make_weights(w.dims, w.seed)
+    lat, txt, _ = make_inputs(w)
+    model = F.FluxDiT(blob, w.dims)
+    del blob
+    try:
+        tok = O.pack_latents(torch.from_numpy(lat)).float().to(DEV)
+        tx = torch.from_numpy(txt).to(DEV)
+        v16, v8, v4 = (torch.empty(w.n_img, 128, device=DEV) for _ in range(3))
+        model.forward(tok, (w.grid, w.grid), tx, 1.0, v16)
+        model.set_precision(F.PRECISION_FP8)
+        model.forward(tok, (w.grid, w.grid), tx, 1.0, v8)
+        model.set_precision(F.PRECISION_NVFP4)
+        model.forward(tok, (w.grid, w.grid), tx, 1.0, v4)
+        torch.cuda.synchronize()
+        e8, e4 = rel_l2(v8, v16), rel_l2(v4, v16)
+        print(f"1024^2 fp8 vs bf16 {e8:.4f}, nvfp4 vs bf16 {e4:.4f}")
+        assert torch.isfinite(v4).all() and e8 < e4 < 0.5, (e8, e4)
+    finally:
+        model.close()
+
+
+@pytest.fixture(scope="module")
+def tiny3():
+    w = WORKLOADS["f3tiny64"]
+    blob, p = make_weights(w.dims, w.seed)
+    model = F.Flux3DiT(blob, w.dims)
+    yield w, p, model
+    model.close()
+
+
+@pytest.mark.parametrize("nt,grid,ref_grids", [(16, (4, 4), [(4, 4)]), (131, (8, 8), [(4, 8), (4, 4)]),
+                                               (0, (4, 6), [])])
+def test_tiny3_nvfp4_forward_and_guided_batch(tiny3, nt, grid, ref_grids):
+    """FLUX.3: NVFP4 per-mode and joint linears against the NVFP4 oracle; the guided batch equals
+    two single forwards bit for bit."""
+    w, p, model = tiny3
+    g = torch.Generator().manual_seed(500 + nt)
+    tok = torch.randn(grid[0] * grid[1], 128, generator=g).to(torch.bfloat16).float()
+    txt = torch.randn(nt, 20480, generator=g).to(torch.bfloat16).float()
+    txt_u = torch.randn(nt, 20480, generator=g).to(torch.bfloat16).float()
+    refs = [torch.randn(h * w_, 128, generator=g).to(torch.bfloat16).float() for h, w_ in ref_grids]
+    want = O3.forward3(p, dict(O.hyper(w.dims), nvfp4=True), tok, txt, 0.6, grid, refs, ref_grids, t_target=0.35)
+    rt = torch.cat(refs).to(DEV) if refs else None
+    td = txt.to(DEV) if nt else None
+    tud = txt_u.to(DEV) if nt else None
+    v, vc, vu, su = (torch.empty(grid[0] * grid[1], 128, device=DEV) for _ in range(4))
+    model.set_precision(F.PRECISION_NVFP4)
+    try:
+        model.forward(tok.to(DEV), grid, td, 0.6, v, rt, ref_grids, t_target=0.35)
+        model.forward_cfg(tok.to(DEV), grid, td, tud, 0.6, vc, vu, rt, ref_grids, t_target=0.35)
+        model.forward(tok.to(DEV), grid, tud, 0.6, su, rt, ref_grids, t_target=0.35)
+    finally:
+        model.set_precision(F.PRECISION_BF16)
+    err = rel_l2(v, want)
+    print(f"flux3 nvfp4 forward vs nvfp4 oracle {err:.4f}")
+    assert err <= NV4_V_TOL, err
+    assert torch.equal(vc, v) and torch.equal(vu, su)
