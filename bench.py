@@ -195,6 +195,7 @@ def barrier(world):
 
 # the sources whose change invalidates the committed DRAM-traffic figure of the pair GEMM
 GEMM_TRAFFIC_SOURCES = ("gemm_tc2.cu", "gemm_epilogue.cuh", "pair.cuh", "common.cuh")
+GEMM4_TRAFFIC_SOURCES = ("gemm_fp4.cu", "gemm_epilogue.cuh", "pair.cuh", "common.cuh")
 
 
 def profile_traffic(kernel_files, profile):
@@ -347,8 +348,11 @@ def run_ours(args, w):
     model = (F.Flux3DiT if flux3 else F.FluxDiT)(blob, w.dims)
     del blob
     fp8 = args.precision == "fp8"
+    fp4 = args.precision == "nvfp4"
     if fp8:
         model.set_precision(F.PRECISION_FP8)
+    if fp4:
+        model.set_precision(F.PRECISION_NVFP4)
     stream = torch.cuda.current_stream()
     dev = torch.device("cuda", local)
     lat0 = torch.from_numpy(lat_h).to(dev)
@@ -461,16 +465,19 @@ def run_ours(args, w):
     d2h = out_pin.numel() * 4
 
     peaks, peak_src = load_peaks()
-    # FP8 tensor peak: the measured bf16 figure times the nominal dense ratio 4.5 / 2.25 PFLOP/s
-    gemm_peak = peaks["bf16_tflops_sustained"] * (2.0 if fp8 else 1.0)
-    gemm_peak_kind = ("fp8 = 2 x bf16 sustained (nominal dense ratio), " if fp8 else "bf16 sustained, ") + peak_src
+    # FP8 / NVFP4 tensor peaks: the measured bf16 figure times the nominal dense ratios 4.5 / 2.25 and
+    # 9 / 2.25 PFLOP/s
+    gemm_peak = peaks["bf16_tflops_sustained"] * (4.0 if fp4 else 2.0 if fp8 else 1.0)
+    gemm_peak_kind = ("nvfp4 = 4 x bf16 sustained (nominal dense ratio), " if fp4 else
+                      "fp8 = 2 x bf16 sustained (nominal dense ratio), " if fp8 else "bf16 sustained, ") + peak_src
     flops = step_flops(w)
     tflops = flops / (ms_step / 1e3) / 1e12
     g_ms, g_fl, g_by, g_n = prof["gemm"]
     a_ms, a_fl, a_by, a_n = prof["attention"]
     gemm_tflops = g_fl / (g_ms / 1e3) / 1e12
     attn_tflops = a_fl / (a_ms / 1e3) / 1e12
-    traffic_per_gflop, src_sha = profile_traffic(GEMM_TRAFFIC_SOURCES,
+    traffic_per_gflop, src_sha = profile_traffic(GEMM4_TRAFFIC_SOURCES if fp4 else GEMM_TRAFFIC_SOURCES,
+                                                 "gemm_fp4_t2i1024.md" if fp4 else
                                                  "gemm_tc2_fp8_t2i1024.md" if fp8 else "gemm_tc2_t2i1024.md")
     traffic = None if traffic_per_gflop is None else traffic_per_gflop * (g_fl / g_n) / 1e9
     kinds = {k: {"ms_per_forward": round(v_[0] / args.steps, 4), "launches_per_forward": v_[3] // args.steps,
@@ -482,7 +489,8 @@ def run_ours(args, w):
             "metric": METRIC, "value": round(value, 4), "unit": step_unit(w), "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-            "dtype": "fp8-e4m3 row-wise block linears, bf16 attention" if fp8 else "bf16",
+            "dtype": ("nvfp4 (e2m1, e4m3 per 16, fp32 per row) block linears, bf16 attention" if fp4 else
+                      "fp8-e4m3 row-wise block linears, bf16 attention" if fp8 else "bf16"),
             "data": "synthetic (seeded N(0,1) weights scaled 1/sqrt(fan_in), bf16; N(0,1) latent and text)",
             "config": {"workload": f"{w.name}: {w.image}x{w.image}, {w.n_img} image + {w.n_txt} text + {w.n_ref} "
                                    f"reference tokens ({len(w.ref_grids)} reference images), {blocks_text(w)}, "
@@ -497,7 +505,9 @@ def run_ours(args, w):
                                "measured_sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
                                "spec_2250": round(tflops / SPEC_BF16_TFLOPS, 4), "peaks": peak_src},
             "forwards_per_s": round(1e3 / value, 3),
-            "roofline": {"kernel": ("gemm_bf16_tc2<fp8> (CTA-pair tcgen05 kind::f8f6f4) for the block linears, "
+            "roofline": {"kernel": ("gemm_fp4_tc2 (CTA-pair tcgen05 kind::mxf4nvf4 with block scales) for the block "
+                                    "linears, bf16 for the input / output projections" if fp4 else
+                                    "gemm_bf16_tc2<fp8> (CTA-pair tcgen05 kind::f8f6f4) for the block linears, "
                                     "bf16 for the input / output projections" if fp8 else
                                     "gemm_bf16_tc2 (CTA-pair tcgen05 GEMM) + the 128-wide output GEMM, all linear layers"),
                          "bound": "tensor",
@@ -540,8 +550,9 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="t2i1024", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--precision", choices=("bf16", "fp8"), default="bf16",
-                    help="block linears in bf16, or row-wise FP8 (e4m3 codes with per-row scales)")
+    ap.add_argument("--precision", choices=("bf16", "fp8", "nvfp4"), default="bf16",
+                    help="block linears in bf16, row-wise FP8 (e4m3 codes with per-row scales) or NVFP4 "
+                         "(e2m1 codes, e4m3 scales per 16 elements, fp32 per row)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

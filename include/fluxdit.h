@@ -279,6 +279,13 @@ FLUX_API size_t flux_nvfp4_scale_bytes(int rows, int k);
 FLUX_API int flux_quantize_rows_nvfp4(const uint16_t *x, int rows, int k, int ldx, uint8_t *q, int ldq, uint8_t *sf,
                                       float *row_scale, void *stream);
 
+/* flux_layernorm_modulate with its output rounded to bf16 and quantised to NVFP4 in the same pass
+ * (codes [rows, dim/2], block scales and row scales as flux_quantize_rows_nvfp4).  dim % 512 == 0,
+ * dim <= 16384. */
+FLUX_API int flux_layernorm_modulate_nvfp4(const float *x, uint8_t *q, uint8_t *sf, float *row_scale, int rows,
+                                           int dim, const float *shift, const float *scale, float eps,
+                                           void *stream);
+
 /* NVFP4 linear layer on the tensor cores (tcgen05 kind::mxf4nvf4 with block scales, CTA pairs):
  * acc = sum over 16-element blocks of (codes_A . codes_W) * s_A * s_W for A [m, k] (codes with row
  * stride lda bytes, scales a_sf) and W [n, k] (codes row stride k/2), both as written by

@@ -101,6 +101,7 @@ _SIGS = {
     "flux_nvfp4_scale_bytes": (_Z, [_I, _I]),
     "flux_quantize_rows_nvfp4": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _P]),
     "flux_linear_nvfp4": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _P, _I, _P, _I, _P, _I, _P, _P]),
+    "flux_layernorm_modulate_nvfp4": (_I, [_P, _P, _P, _P, _I, _I, _P, _P, _F, _P]),
 }
 EXPORTED = tuple(_SIGS)
 
@@ -508,6 +509,18 @@ def flux_quantize_rows_nvfp4(x, q, sf, row_scale, stream=None):
     _check(lib().flux_quantize_rows_nvfp4(ctypes.c_void_p(x.data_ptr()), rows, k, x.stride(0),
                                           ctypes.c_void_p(q.data_ptr()), q.stride(0), _u8(sf, "sf"),
                                           _ptr(row_scale, torch.float32, "row_scale"), _stream(stream)))
+    return q, sf, row_scale
+
+
+def flux_layernorm_modulate_nvfp4(x, q, sf, row_scale, shift, scale, eps=1e-6, stream=None):
+    """LN + modulation of fp32 x [rows, dim], rounded to bf16 and quantised to NVFP4 (q [rows, dim/2],
+    sf [flux_nvfp4_scale_bytes(rows, dim)], row_scale [rows])."""
+    import torch
+    rows, dim = x.shape
+    _check(lib().flux_layernorm_modulate_nvfp4(_ptr(x, torch.float32, "x"), _u8(q, "q"), _u8(sf, "sf"),
+                                               _ptr(row_scale, torch.float32, "row_scale"), rows, dim,
+                                               _ptr(shift, torch.float32, "shift"), _ptr(scale, torch.float32, "scale"),
+                                               float(eps), _stream(stream)))
     return q, sf, row_scale
 
 

@@ -86,21 +86,8 @@ __global__ void cast_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __r
 // ------------------------------------------------------------------ LayerNorm + adaLN modulation
 // One 256-thread CTA per row: each thread keeps VPT float4 of the row in registers (dim = 1024 VPT),
 // mean and variance come from two block reductions, so many CTAs stay resident per SM.
-// Row r uses modulation set 0 when r % period < split, set 1 when it is < split2, else set 2.
-// (Scalar members: a runtime index into a kernel-parameter array would copy it to the stack.)
-struct LnModSets {
-  int split, split2, period;
-  const float *sh0, *sh1, *sh2;
-  const float *sc0, *sc1, *sc2;
-  __device__ __forceinline__ const float* shift(int row) const {
-    const int r = row % period;
-    return r < split ? sh0 : (r < split2 ? sh1 : sh2);
-  }
-  __device__ __forceinline__ const float* scale(int row) const {
-    const int r = row % period;
-    return r < split ? sc0 : (r < split2 ? sc1 : sc2);
-  }
-};
+// Row r uses modulation set 0 when r % period < split, set 1 when it is < split2, else set 2
+// (LnModSets, fluxdit_internal.h).
 
 template <int VPT>
 __global__ void __launch_bounds__(256) ln_mod_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y,

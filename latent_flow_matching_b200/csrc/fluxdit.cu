@@ -813,8 +813,8 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
 
   // FP8 precision: block linears on e4m3 codes (row-wise scales); LN-mod quantises its output,
   // the attention output and the SwiGLU hidden are quantised before the linears that read them.
-  // NVFP4 precision: the same operands as e2m1 codes with block and row scales (LN-mod writes bf16,
-  // then the rows are quantised per segment).
+  // NVFP4 precision: the same operands as e2m1 codes with block and row scales (LN-mod quantises
+  // its output per segment in the same pass).
   const bool fp8 = m->precision == FLUX_PRECISION_FP8;
   const bool fp4 = m->precision == FLUX_PRECISION_NVFP4;
   auto f8 = [&](int i, const CUtensorMap& a8, const CUtensorMap& w8, const float* sa, const float* sb) {
@@ -837,6 +837,12 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
   // quantises Y over the segments `segs`
   auto ln_mod = [&](int split, const float* sh0, const float* sc0, const float* sh1, const float* sc1,
                     const Q4Segs& segs) -> int {
+    if (fp4) {
+      const LnModSets ms{split, n, n, sh0, sh1, sh1, sc0, sc1, sc1};
+      FD_LAUNCH(m, kProfLnMod, 0, 4.56 * rows * D + 4.0 * rows,
+                ln_modulate_nvfp4_launch(w.X, D, w.Y4, w.sfY, w.sY4, segs, ms, eps_ln, s));
+      return FLUX_OK;
+    }
     if (fp8)
       FD_LAUNCH(m, kProfLnMod, 0, 5.0 * rows * D + 4.0 * rows,
                 ln_modulate_fp8_launch(w.X, w.Y8, w.sY, rows, D, split, n, n, sh0, sc0, sh1, sc1, sh1, sc1, eps_ln,
@@ -844,7 +850,6 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
     else
       FD_LAUNCH(m, kProfLnMod, 0, ln_bytes, ln_modulate_launch(w.X, w.Y, rows, D, split, n, sh0, sc0, sh1, sc1,
                                                                eps_ln, s));
-    if (fp4) return quant4(w.Y, D, D, w.Y4, D / 2, w.sfY, w.sY4, segs);
     return FLUX_OK;
   };
   // e4m3 codes of CC columns [col0, col0 + cols) into C8, one scale per row
@@ -1305,6 +1310,21 @@ int flux_quantize_rows_nvfp4(const uint16_t* x, int rows, int k, int ldx, uint8_
   const int r0 = 0;
   FD_CUDA(quantize_nvfp4_launch(reinterpret_cast<const bf16*>(x), ldx, k, q, ldq, sf, row_scale,
                                 q4_segments(&r0, &rows, 1), static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_layernorm_modulate_nvfp4(const float* x, uint8_t* q, uint8_t* sf, float* row_scale, int rows, int dim,
+                                  const float* shift, const float* scale, float eps, void* stream) {
+  if (!x || !q || !sf || !row_scale || !shift || !scale) return fail(FLUX_EINVAL, "NULL argument");
+  if (rows < 0 || dim < 512 || dim % 512 || dim > 16384)
+    return fail(FLUX_EINVAL, "bad shape rows=%d dim=%d (dim %% 512, dim <= 16384)", rows, dim);
+  if (!aligned16(x) || !aligned16(q) || !aligned16(sf) || !aligned16(row_scale) || !aligned16(shift) ||
+      !aligned16(scale))
+    return fail(FLUX_EINVAL, "pointers must be 16-byte aligned");
+  const int r0 = 0;
+  const LnModSets ms{rows, rows, rows > 0 ? rows : 1, shift, shift, shift, scale, scale, scale};
+  FD_CUDA(ln_modulate_nvfp4_launch(x, dim, q, sf, row_scale, q4_segments(&r0, &rows, 1), ms, eps,
+                                   static_cast<cudaStream_t>(stream)));
   return FLUX_OK;
 }
 

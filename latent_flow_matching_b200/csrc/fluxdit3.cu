@@ -713,8 +713,8 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
     P.prob[i].scale_a = sa;
     P.prob[i].scale_b = sb;
   };
-  // NVFP4 precision: LN-mod writes bf16 and the rows are quantised per segment (`segs`); [O | H]
-  // likewise before linear2
+  // NVFP4 precision: LN-mod quantises its output per segment (`segs`) in the same pass; [O | H] is
+  // quantised per segment before linear2
   const bool fp4 = m->precision == FLUX_PRECISION_NVFP4;
   auto linear_as = [&](bool small) -> cudaError_t {
     return fp4 ? gemm_fp4_launch(P4, m->num_sms, s) : launch_linear_as(P, m->num_sms, s, fp8, small);
@@ -741,9 +741,11 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
   };
   auto ln3q = [&](int r, const Q4Segs& segs, const float* sh0, const float* sc0, const float* sh1, const float* sc1,
                   const float* sh2, const float* sc2) -> int {
-    const int rc2 = ln3(r, sh0, sc0, sh1, sc1, sh2, sc2);
-    if (rc2 || !fp4) return rc2;
-    return quant4(w.Y, D, w.Y4, w.sfY, w.sY4, segs);
+    if (!fp4) return ln3(r, sh0, sc0, sh1, sc1, sh2, sc2);
+    const LnModSets ms{nt, nt + ni, n, sh0, sh1, sh2, sc0, sc1, sc2};
+    FD_LAUNCH(m, kProfLnMod, 0, 4.56 * r * D + 4.0 * r,
+              ln_modulate_nvfp4_launch(w.X, D, w.Y4, w.sfY, w.sY4, segs, ms, eps_ln, s));
+    return FLUX_OK;
   };
   auto quant_cc = [&](int r) -> int {
     FD_LAUNCH(m, kProfOther, 0, 3.0 * r * sDF + 4.0 * r, quantize_rows_launch(w.CC, D + F, r, D + F, w.C8, D + F, w.sC, s));

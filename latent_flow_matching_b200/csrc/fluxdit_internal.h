@@ -78,6 +78,23 @@ cudaError_t cfg_euler_launch(float* x, const float* vc, const float* vu, size_t 
                              cudaStream_t s);
 cudaError_t cast_bf16_launch(const float* x, __nv_bfloat16* y, size_t n, cudaStream_t s);
 
+// Modulation sets of a LayerNorm + modulation launch: row r uses set 0 when r % period < split, set 1
+// when it is < split2, else set 2.  (Scalar members: a runtime index into a kernel-parameter array
+// would copy it to the stack.)
+struct LnModSets {
+  int split, split2, period;
+  const float *sh0, *sh1, *sh2;
+  const float *sc0, *sc1, *sc2;
+  __device__ __forceinline__ const float* shift(int row) const {
+    const int r = row % period;
+    return r < split ? sh0 : (r < split2 ? sh1 : sh2);
+  }
+  __device__ __forceinline__ const float* scale(int row) const {
+    const int r = row % period;
+    return r < split ? sc0 : (r < split2 ? sc1 : sc2);
+  }
+};
+
 // y[r, :] = LN(x[r, :]) * (1 + scale) + shift; rows with r % period < split use (shift0, scale0), the
 // others (shift1, scale1) (period: rows per sequence of a batch, the row count for one sequence)
 cudaError_t ln_modulate_launch(const float* x, __nv_bfloat16* y, int rows, int dim, int split, int period,
@@ -150,6 +167,10 @@ struct Q4Segs {
 Q4Segs q4_segments(const int* row0, const int* rows, int n);
 cudaError_t quantize_nvfp4_launch(const __nv_bfloat16* x, int ldx, int k, uint8_t* q, int ldq, uint8_t* sf,
                                   float* row_scale, const Q4Segs& segs, cudaStream_t s);
+// LayerNorm + modulation (fp32 rows of x, dim values each) rounded to bf16 and quantised to NVFP4 as
+// quantize_nvfp4_launch (codes row stride dim / 2), over the rows of `segs`; dim % 512 == 0.
+cudaError_t ln_modulate_nvfp4_launch(const float* x, int dim, uint8_t* q, uint8_t* sf, float* row_scale,
+                                     const Q4Segs& segs, const LnModSets& ms, float eps, cudaStream_t s);
 // Problems of the NVFP4 pair GEMM: mapA / mapB over the codes (u8 maps, 128-byte box), K in elements
 // (K % 256 == 0), scale_a / scale_b the fp32 row scales, and the block scales' maps (make_tmap_sf).
 struct GemmParams4 {

@@ -24,8 +24,11 @@
 namespace fdit {
 namespace {
 
-constexpr int kQ4Threads = 128;
-constexpr int kQ4MaxUnits = 2;          // 64-element units per thread: k <= 128 * 64 * 2
+// One 256-thread CTA per row.  A row is read with coalesced 16-byte loads (element group j, of 8
+// bf16 values or 4 fp32 values, goes to thread j % 256), kept in registers, and every 16-element
+// block is held by neighbouring threads of one warp (2 threads for bf16 groups, 4 for fp32), so
+// a block's maximum takes one or two shuffles and the row's maximum one CTA reduction.
+constexpr int kQ4Threads = 256;
 
 __device__ __forceinline__ float bf16_abs_max8(const uint4& w, float m) {
   const uint32_t x[4] = {w.x, w.y, w.z, w.w};
@@ -34,95 +37,203 @@ __device__ __forceinline__ float bf16_abs_max8(const uint4& w, float m) {
   return m;
 }
 
-// One CTA per row.  Rows come in segments (Q4Segs): segment z is rows [row0, row0 + rows) of x, q
-// and row_scale, and its scales start at 128-row block blk0 of sf, so that a GEMM problem over
-// that segment finds its first row at the start of a scale block.
-__global__ void __launch_bounds__(kQ4Threads) quantize_nvfp4_kernel(const __nv_bfloat16* __restrict__ x, int ldx,
-                                                                    int k, uint8_t* __restrict__ q, int ldq,
-                                                                    uint8_t* __restrict__ sf, float* __restrict__ row_scale,
-                                                                    const Q4Segs segs) {
-  __shared__ float red[kQ4Threads / 32];
+// Sum (or maximum) over the CTA; every thread gets the result.  red: one float per warp.
+template <bool kMax>
+__device__ __forceinline__ float cta_reduce(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float u = __shfl_xor_sync(0xffffffffu, v, o);
+    v = kMax ? fmaxf(v, u) : v + u;
+  }
+  __syncthreads();                                   // red may still be read by the previous reduction
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  v = red[0];
+#pragma unroll
+  for (int w = 1; w < kQ4Threads / 32; ++w) v = kMax ? fmaxf(v, red[w]) : v + red[w];
+  return v;
+}
+
+// The row and the scale-layout row of CTA blockIdx.x in a segment list.
+struct Q4Row {
+  int r, sfr;
+};
+__device__ __forceinline__ Q4Row q4_row(const Q4Segs& segs) {
   int z = 0, l = blockIdx.x;
   while (z + 1 < segs.n && l >= segs.rows[z]) l -= segs.rows[z++];
-  const int r = segs.row0[z] + l;                  // row of x, q and row_scale
-  const int sfr = segs.blk0[z] * 128 + l;          // row of the scale layout
-  const int units = k / 64;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(r) * ldx);
-  uint4 v[kQ4MaxUnits][8];
-  float bmax[kQ4MaxUnits][4];
+  return {segs.row0[z] + l, segs.blk0[z] * 128 + l};
+}
+
+// Row quantities from the row's absolute maximum: inv = 448 / amax (0 for a zero row), S = amax / 2688.
+__device__ __forceinline__ void q4_row_scales(float amax, float* inv, float* S) {
+  *inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
+  *S = __fdiv_rn(amax, 2688.0f);
+}
+
+// The e4m3 scale of a block with maximum bmax, and the reciprocal of its dequantisation factor.
+__device__ __forceinline__ __nv_fp8_storage_t q4_block_scale(float bmax, float inv, float S, float* rcp) {
+  const __nv_fp8_storage_t s8 = __nv_cvt_float_to_fp8(__fmul_rn(bmax, inv), __NV_SATFINITE, __NV_E4M3);
+  const float sb = __half2float(__half(__nv_cvt_fp8_to_halfraw(s8, __NV_E4M3)));
+  const float d = __fmul_rn(sb, S);
+  *rcp = d > 0.f ? __frcp_rn(d) : 0.f;
+  return s8;
+}
+
+__device__ __forceinline__ uint32_t e2m1x2(float a, float b, float rcp) {
+  return __nv_cvt_float2_to_fp4x2(make_float2(__fmul_rn(a, rcp), __fmul_rn(b, rcp)), __NV_E2M1, cudaRoundNearest);
+}
+
+// Byte offset of the scale of 16-element block g of scale-layout row sfr (k elements per row).
+__device__ __forceinline__ size_t q4_sf_offset(int sfr, int g, int k) {
+  return (static_cast<size_t>(sfr >> 7) * (k / 64) + (g >> 2)) * 512 + 16 * (sfr & 31) + 4 * ((sfr & 127) >> 5) +
+         (g & 3);
+}
+
+// Rows come in segments (Q4Segs): segment z is rows [row0, row0 + rows) of x, q and row_scale, and
+// its scales start at 128-row block blk0 of sf, so that a GEMM problem over that segment finds its
+// first row at the start of a scale block.  U: groups of 8 values per thread (k <= 2048 U).
+template <int U>
+__global__ void __launch_bounds__(kQ4Threads) quantize_nvfp4_kernel(const __nv_bfloat16* __restrict__ x, int ldx,
+                                                                    int k, uint8_t* __restrict__ q, int ldq,
+                                                                    uint8_t* __restrict__ sf,
+                                                                    float* __restrict__ row_scale, const Q4Segs segs) {
+  __shared__ float red[kQ4Threads / 32];
+  const int tid = threadIdx.x;
+  const Q4Row rr = q4_row(segs);
+  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(rr.r) * ldx);
+  const int n8 = k / 8;
+  uint4 v[U];
   float amax = 0.f;
 #pragma unroll
-  for (int u = 0; u < kQ4MaxUnits; ++u) {
-    const int unit = threadIdx.x + u * kQ4Threads;
+  for (int u = 0; u < U; ++u) {
+    const int j = tid + u * kQ4Threads;
+    v[u] = j < n8 ? __ldg(xr + j) : make_uint4(0u, 0u, 0u, 0u);
+    amax = bf16_abs_max8(v[u], amax);
+  }
+  float inv, S;
+  q4_row_scales(cta_reduce<true>(amax, red), &inv, &S);
+  if (tid == 0) row_scale[rr.r] = S;
+  uint32_t* qr = reinterpret_cast<uint32_t*>(q + static_cast<size_t>(rr.r) * ldq);
 #pragma unroll
-    for (int b = 0; b < 4; ++b) bmax[u][b] = 0.f;
-    if (unit < units) {
+  for (int u = 0; u < U; ++u) {
+    const int j = tid + u * kQ4Threads;             // n8 % 8 == 0: both threads of a block agree on j < n8
+    const float m = bf16_abs_max8(v[u], 0.f);
+    float rcp;
+    const __nv_fp8_storage_t s8 = q4_block_scale(fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1)), inv, S, &rcp);
+    const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+    uint32_t c = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[u][i] = __ldg(xr + unit * 8 + i);
-#pragma unroll
-      for (int b = 0; b < 4; ++b) bmax[u][b] = bf16_abs_max8(v[u][2 * b + 1], bf16_abs_max8(v[u][2 * b], 0.f));
-      amax = fmaxf(amax, fmaxf(fmaxf(bmax[u][0], bmax[u][1]), fmaxf(bmax[u][2], bmax[u][3])));
+    for (int e = 0; e < 4; ++e) c |= e2m1x2(bf16lo(w[e]), bf16hi(w[e]), rcp) << (8 * e);
+    if (j < n8) {
+      qr[j] = c;
+      if ((tid & 1) == 0) sf[q4_sf_offset(rr.sfr, j >> 1, k)] = s8;
     }
   }
+}
+
+// LayerNorm + modulation of one row per CTA (dim = 1024 VPT: VPT float4 per thread), the modulated
+// row rounded to bf16 (the block linears' input precision) and quantised to NVFP4 as above; row r
+// uses the modulation set that `ms` gives it.
+template <int VPT>
+__global__ void __launch_bounds__(kQ4Threads) ln_mod_nvfp4_kernel(const float* __restrict__ x,
+                                                                  uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
+                                                                  float* __restrict__ row_scale, const Q4Segs segs,
+                                                                  LnModSets ms, float eps) {
+  constexpr int dim = 1024 * VPT;
+  __shared__ float red[kQ4Threads / 32];
+  const int tid = threadIdx.x;
+  const Q4Row rr = q4_row(segs);
+  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(rr.r) * dim) + tid;
+  float4 v[VPT];
+  float s = 0.f;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
-  __syncthreads();
-  amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
-  const float S = __fdiv_rn(amax, 2688.0f);
-  if (threadIdx.x == 0) row_scale[r] = S;
-  uint8_t* qr = q + static_cast<size_t>(r) * ldq;
-  const size_t sf_row = 16 * (sfr & 31) + 4 * ((sfr & 127) >> 5);
+  for (int i = 0; i < VPT; ++i) {
+    v[i] = __ldcs(xr + i * kQ4Threads);
+    s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+  }
+  const float mean = cta_reduce<false>(s, red) * (1.0f / dim);
+  float qs = 0.f;
 #pragma unroll
-  for (int u = 0; u < kQ4MaxUnits; ++u) {
-    const int unit = threadIdx.x + u * kQ4Threads;
-    if (unit >= units) continue;
-    uint32_t sfw = 0;
-    uint32_t codes[8];                               // 64 codes, 8 per word
+  for (int i = 0; i < VPT; ++i) {
+    const float a = v[i].x - mean, b = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
+    qs += (a * a + b * b) + (c * c + d * d);
+  }
+  const float rstd = rsqrtf(cta_reduce<false>(qs, red) * (1.0f / dim) + eps);
+  const float4* sh = reinterpret_cast<const float4*>(ms.shift(rr.r)) + tid;
+  const float4* sc = reinterpret_cast<const float4*>(ms.scale(rr.r)) + tid;
+  float amax = 0.f;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const __nv_fp8_storage_t s8 = __nv_cvt_float_to_fp8(__fmul_rn(bmax[u][b], inv), __NV_SATFINITE, __NV_E4M3);
-      const float sb = __half2float(__half(__nv_cvt_fp8_to_halfraw(s8, __NV_E4M3)));
-      const float d = __fmul_rn(sb, S);
-      const float rcp = d > 0.f ? __frcp_rn(d) : 0.f;
-      sfw |= static_cast<uint32_t>(s8) << (8 * b);
+  for (int i = 0; i < VPT; ++i) {
+    const float4 a = __ldg(sh + i * kQ4Threads), c = __ldg(sc + i * kQ4Threads);
+    v[i].x = __bfloat162float(__float2bfloat16_rn((v[i].x - mean) * rstd * (1.f + c.x) + a.x));
+    v[i].y = __bfloat162float(__float2bfloat16_rn((v[i].y - mean) * rstd * (1.f + c.y) + a.y));
+    v[i].z = __bfloat162float(__float2bfloat16_rn((v[i].z - mean) * rstd * (1.f + c.z) + a.z));
+    v[i].w = __bfloat162float(__float2bfloat16_rn((v[i].w - mean) * rstd * (1.f + c.w) + a.w));
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+  }
+  float inv, S;
+  q4_row_scales(cta_reduce<true>(amax, red), &inv, &S);
+  if (tid == 0) row_scale[rr.r] = S;
+  uint16_t* qr = reinterpret_cast<uint16_t*>(q + static_cast<size_t>(rr.r) * (dim / 2)) + tid;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {                  // 8 elements per uint4
-        const uint4 w = v[u][2 * b + h];
-        const uint32_t xw[4] = {w.x, w.y, w.z, w.w};
-        uint32_t word = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = make_float2(__fmul_rn(bf16lo(xw[e]), rcp), __fmul_rn(bf16hi(xw[e]), rcp));
-          word |= static_cast<uint32_t>(__nv_cvt_float2_to_fp4x2(f, __NV_E2M1, cudaRoundNearest)) << (8 * e);
-        }
-        codes[2 * b + h] = word;
-      }
-    }
-    uint4* dq = reinterpret_cast<uint4*>(qr + unit * 32);
-    dq[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-    dq[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-    const size_t blk = static_cast<size_t>(sfr >> 7) * units + unit;
-    *reinterpret_cast<uint32_t*>(sf + blk * 512 + sf_row) = sfw;
+  for (int i = 0; i < VPT; ++i) {                    // block of float4 group j = tid + 256 i: threads 4g..4g+3
+    float m = fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w)));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    float rcp;
+    const __nv_fp8_storage_t s8 = q4_block_scale(m, inv, S, &rcp);
+    qr[i * kQ4Threads] = static_cast<uint16_t>(e2m1x2(v[i].x, v[i].y, rcp) | (e2m1x2(v[i].z, v[i].w, rcp) << 8));
+    if ((tid & 3) == 0) sf[q4_sf_offset(rr.sfr, (tid + i * kQ4Threads) >> 2, dim)] = s8;
   }
 }
 
 }  // namespace
 
+static bool q4_segs_ok(const Q4Segs& segs, long* total) {
+  if (segs.n < 1 || segs.n > kMaxQ4Segs) return false;
+  *total = 0;
+  for (int z = 0; z < segs.n; ++z) {
+    if (segs.rows[z] < 0 || segs.row0[z] < 0 || segs.blk0[z] < 0) return false;
+    *total += segs.rows[z];
+  }
+  return *total < (1l << 31);
+}
+
 cudaError_t quantize_nvfp4_launch(const __nv_bfloat16* x, int ldx, int k, uint8_t* q, int ldq, uint8_t* sf,
                                   float* row_scale, const Q4Segs& segs, cudaStream_t s) {
-  if (k <= 0 || k % 64 != 0 || k > kQ4Threads * 64 * kQ4MaxUnits || ldx < k || ldx % 8 != 0 || ldq < k / 2 ||
-      ldq % 16 != 0 || segs.n < 1 || segs.n > kMaxQ4Segs)
-    return cudaErrorInvalidValue;
   long total = 0;
-  for (int z = 0; z < segs.n; ++z) {
-    if (segs.rows[z] < 0 || segs.row0[z] < 0 || segs.blk0[z] < 0) return cudaErrorInvalidValue;
-    total += segs.rows[z];
-  }
+  if (k <= 0 || k % 64 != 0 || k > 16384 || ldx < k || ldx % 8 != 0 || ldq < k / 2 || ldq % 16 != 0 ||
+      !q4_segs_ok(segs, &total))
+    return cudaErrorInvalidValue;
   if (total == 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>(total);
   count_launch();
-  quantize_nvfp4_kernel<<<static_cast<unsigned>(total), kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs);
+  switch ((k / 8 + kQ4Threads - 1) / kQ4Threads) {
+    case 1: quantize_nvfp4_kernel<1><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    case 2: quantize_nvfp4_kernel<2><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    case 3: quantize_nvfp4_kernel<3><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    case 4: quantize_nvfp4_kernel<4><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    case 5: quantize_nvfp4_kernel<5><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    case 6: quantize_nvfp4_kernel<6><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    case 7: quantize_nvfp4_kernel<7><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    default: quantize_nvfp4_kernel<8><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t ln_modulate_nvfp4_launch(const float* x, int dim, uint8_t* q, uint8_t* sf, float* row_scale,
+                                     const Q4Segs& segs, const LnModSets& ms, float eps, cudaStream_t s) {
+  long total = 0;
+  if (!q4_segs_ok(segs, &total)) return cudaErrorInvalidValue;
+  if (total == 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>(total);
+  switch (dim) {
+    case 1024: count_launch(); ln_mod_nvfp4_kernel<1><<<grid, kQ4Threads, 0, s>>>(x, q, sf, row_scale, segs, ms, eps); break;
+    case 2048: count_launch(); ln_mod_nvfp4_kernel<2><<<grid, kQ4Threads, 0, s>>>(x, q, sf, row_scale, segs, ms, eps); break;
+    case 3072: count_launch(); ln_mod_nvfp4_kernel<3><<<grid, kQ4Threads, 0, s>>>(x, q, sf, row_scale, segs, ms, eps); break;
+    case 4096: count_launch(); ln_mod_nvfp4_kernel<4><<<grid, kQ4Threads, 0, s>>>(x, q, sf, row_scale, segs, ms, eps); break;
+    default: return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 
