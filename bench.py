@@ -406,22 +406,50 @@ def run_ours(args, w):
     torch.cuda.synchronize()
     assert F.flux_device_error() == 0
 
+    # ---- every step of one sampling run captured as a CUDA graph (the same launches, replayed
+    # without per-launch host work, so host jitter does not enter the device-timed region)
+    graphs, launch_mode = [], "plain launches"
+    if not args.no_graph:
+        try:
+            for k in range(w.n_steps):
+                g = torch.cuda.CUDAGraph()
+                c0 = F.flux_kernel_launches()
+                with torch.cuda.graph(g):
+                    step(k, lat)
+                graphs.append((g, F.flux_kernel_launches() - c0))
+            for g, _ in graphs:                     # one full sampling run from the graphs
+                g.replay()
+            torch.cuda.synchronize()
+            assert F.flux_device_error() == 0
+            launch_mode = "one CUDA graph per sampling step, replayed"
+        except Exception as ex:                    # capture refused: time plain launches
+            torch.cuda.synchronize()
+            graphs, launch_mode = [], f"plain launches (graph capture failed: {type(ex).__name__})"
+
+    def timed_step(i):
+        if graphs:
+            graphs[i % w.n_steps][0].replay()
+            return graphs[i % w.n_steps][1]
+        c0 = F.flux_kernel_launches()
+        step(i, lat)
+        return F.flux_kernel_launches() - c0
+
     # ---- timed region: K steps, device time, max over ranks
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    launches0 = F.flux_kernel_launches()
+    launches = 0
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     ev0.record(stream)
     for i in range(args.steps):
-        step(i, lat)
+        launches += timed_step(i)
     ev1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     ms_total = ev0.elapsed_time(ev1)
-    launches = F.flux_kernel_launches() - launches0
+    graphs = []                                     # released before the model
     clk = clocks.stop()
     ms_total = max_over_ranks(ms_total, world)
     ms_step = ms_total / args.steps
@@ -523,6 +551,7 @@ def run_ours(args, w):
             "e2e": {"value": round(e2e_ms, 4), "unit": step_unit(w), "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
+            "launch": launch_mode,
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -550,6 +579,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="t2i1024", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time plain per-step launches instead of replaying each step's captured CUDA graph")
     ap.add_argument("--precision", choices=("bf16", "fp8", "nvfp4"), default="bf16",
                     help="block linears in bf16, row-wise FP8 (e4m3 codes with per-row scales) or NVFP4 "
                          "(e2m1 codes, e4m3 scales per 16 elements, fp32 per row)")

@@ -79,6 +79,12 @@ static bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType type, uint32_t bo
                   swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_out(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
+                   bool f32) {
+  return make_tmap_2d(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32, base, rows,
+                      cols, row_stride_bytes, 32, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 bool make_tmap_sf(CUtensorMap* map, const void* base, uint64_t bytes) {
   if (bytes % 256) return false;
   return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 256, base, bytes / 256, 256, 256, 8,

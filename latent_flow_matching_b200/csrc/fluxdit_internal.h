@@ -177,6 +177,7 @@ struct GemmParams4 {
   GemmParams g;
   CUtensorMap mapSFA[kMaxProblems];
   CUtensorMap mapSFB[kMaxProblems];
+  CUtensorMap mapOut[kMaxProblems];     // filled by gemm_fp4_launch: the epilogue writes by TMA
 };
 cudaError_t gemm_fp4_launch(GemmParams4& P, int num_sms, cudaStream_t stream);
 int gemm_fp4_read_device_error(cudaStream_t stream);
@@ -194,6 +195,9 @@ bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t co
                   uint32_t box_rows);
 // Block scales of an NVFP4 matrix as 256-byte rows, box 8 rows (2 KB: one stage of 128 rows), no swizzle.
 bool make_tmap_sf(CUtensorMap* map, const void* base, uint64_t bytes);
+// GEMM output written by TMA: fp32 (128-byte swizzle) or bf16 (64-byte swizzle), box {32 cols, 32 rows}.
+bool make_tmap_out(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
+                   bool f32);
 int num_sms_current();
 
 }  // namespace fdit

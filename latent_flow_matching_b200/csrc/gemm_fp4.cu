@@ -4,7 +4,8 @@
 // Same structure as the bf16 / e4m3 pair kernel (gemm_tc2.cu): CTA r of the pair stages rows
 // [m0 + 128r, +128) of A and [n0 + 128r, +128) of W, one elected lane of the leader issues
 // tcgen05.mma.cta_group::2 with M = N = 256, and eight epilogue warps per CTA drain the
-// accumulator with the shared fused epilogues (the row scales of A and W applied per element).
+// accumulator with the fused epilogues (the row scales of A and W applied per element) and write
+// through shared memory with TMA stores (epilogue_tma.cuh).
 // What the 4-bit path adds:
 //   * kind::mxf4nvf4 MMAs with K = 64 (32 bytes of packed codes per row, so the 128-byte swizzle
 //     row of a stage holds 256 elements and a stage is four MMAs, as for the 8-bit path);
@@ -22,8 +23,10 @@
 //   ovl  leader only: 8 arrivals (the four owning epilogue warps of each CTA) per tile
 #include "common.cuh"
 #include "fluxdit_internal.h"
-#include "gemm_epilogue.cuh"
+#include "epilogue_tma.cuh"
 #include "pair.cuh"
+
+#include <vector>
 
 namespace fdit {
 
@@ -34,7 +37,7 @@ namespace {
 constexpr int BM = 256;
 constexpr int BN = 256;
 constexpr int BKE = 256;                       // K elements per stage (128 bytes of codes per row)
-constexpr int STAGES = 5;
+constexpr int STAGES = 4;
 constexpr int A_BYTES = 128 * 128;             // 16 KB of codes
 constexpr int B_BYTES = 128 * 128;
 constexpr int SFA_BYTES = 128 * BKE / 16;      // 2 KB: 128 rows x 16 scales
@@ -45,9 +48,38 @@ constexpr uint32_t kAcc1Col = 224;             // buffer 1 shares columns [224, 
 constexpr uint32_t kSfCol = 480;               // two scale slots of 16 columns: SFA 4 | SFB 8
 constexpr int kEpiWarps = 8;
 constexpr int kThreads4 = 32 * (2 + kEpiWarps);
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512;
+constexpr int EPI_BYTES = 8192;                // per epilogue warp: two staged {32, 32} fp32 boxes
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + kEpiWarps * EPI_BYTES + 1024 + 512;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 
 static_assert(BN - kAcc1Col == 32 && kAcc1Col + BN <= kSfCol && kSfCol + 28 <= TMEM_COLS, "tensor memory plan");
+static_assert(STAGE_BYTES % 1024 == 0, "the epilogue staging buffers need 1024-byte alignment");
+
+// Output tensor maps of the epilogue's TMA stores, encoded once per (buffer, shape).
+struct OutMapEntry {
+  const void* base;
+  uint64_t rows, cols, stride;
+  bool f32;
+  CUtensorMap map;
+};
+bool out_map(CUtensorMap* dst, const GemmProblem& pr) {
+  static std::vector<OutMapEntry> cache;
+  const bool f32 = pr.mode == kEpiF32Bias || pr.mode == kEpiResidGate;
+  const uint64_t cols = pr.mode == kEpiSwiGLU ? pr.N / 2 : pr.N;
+  const uint64_t stride = static_cast<uint64_t>(pr.ldo) * (f32 ? 4 : 2);
+  for (const OutMapEntry& c : cache)
+    if (c.base == pr.out && c.rows == static_cast<uint64_t>(pr.M) && c.cols == cols && c.stride == stride &&
+        c.f32 == f32) {
+      *dst = c.map;
+      return true;
+    }
+  OutMapEntry c{pr.out, static_cast<uint64_t>(pr.M), cols, stride, f32, {}};
+  if (!make_tmap_out(&c.map, pr.out, c.rows, cols, stride, f32)) return false;
+  if (cache.size() >= 512) cache.erase(cache.begin());
+  cache.push_back(c);
+  *dst = c.map;
+  return true;
+}
 
 __device__ __forceinline__ int find_problem(const GemmParams& P, int tile) {
   int p = 0;
@@ -105,7 +137,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads4, 1)
   uint8_t* sB = sA + STAGES * A_BYTES;
   uint8_t* sSFA = sB + STAGES * B_BYTES;
   uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* sEpi = smem + STAGES * STAGE_BYTES;      // 1024-byte aligned: STAGE_BYTES is a multiple of 1024
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + kEpiWarps * EPI_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
@@ -267,6 +300,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads4, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t acc_empty_leader[2] = {map_to_rank(&acc_empty[0], 0), map_to_rank(&acc_empty[1], 0)};
     const uint32_t ovl_leader = map_to_rank(ovl, 0);
+    const uint32_t epi_buf = smem_u32(sEpi + (warp - 2) * EPI_BYTES);
+    uint32_t epi_which = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < P.total_tiles; tile += num_pairs) {
@@ -281,13 +316,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads4, 1)
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + lane_addr + (acc ? kAcc1Col : 0u);
-      gemm_epilogue_tile<BN, true, 2, true>(pr, tbase, m, n0, part, acc, ovl_leader);
+      const EpiTma et{&P4.mapOut[p], epi_buf, m - lane, pr.M, &epi_which};
+      gemm_epilogue_tile_tma<BN, true, 2, true>(pr, tbase, m, n0, part, acc, ovl_leader, et);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    epi_tma_drain();                                  // this warp's bulk stores are complete
   }
 
   tc_fence_before();
@@ -312,6 +349,7 @@ cudaError_t gemm_fp4_launch(GemmParams4& P4, int num_sms, cudaStream_t stream) {
   for (int i = 0; i < P.num_problems; ++i) {        // K in whole stages, scales present
     const GemmProblem& pr = P.prob[i];
     if (pr.M > 0 && (pr.K % BKE != 0 || !pr.scale_a || !pr.scale_b)) return cudaErrorInvalidValue;
+    if (pr.M > 0 && pr.N > 0 && !out_map(&P4.mapOut[i], pr)) return cudaErrorInvalidValue;
   }
   int w = 0, total = 0;
   for (int i = 0; i < P.num_problems; ++i) {
@@ -326,6 +364,7 @@ cudaError_t gemm_fp4_launch(GemmParams4& P4, int num_sms, cudaStream_t stream) {
       P.mapB[w] = P.mapB[i];
       P4.mapSFA[w] = P4.mapSFA[i];
       P4.mapSFB[w] = P4.mapSFB[i];
+      P4.mapOut[w] = P4.mapOut[i];
     }
     P.prob[w++] = pr;
   }
