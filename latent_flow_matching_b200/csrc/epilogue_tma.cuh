@@ -2,12 +2,12 @@
 //
 // Same modes and arithmetic as gemm_epilogue.cuh, but a warp does not write its 32 accumulator rows
 // with per-thread global stores (one row per thread: 32 separate 32-byte segments per store
-// instruction).  Each 32-column chunk of results is staged in one of this warp's two 4 KB shared
-// memory buffers in the 128-byte (fp32) or 64-byte (bf16) swizzled layout of a {32 columns, 32
-// rows} TMA box and written by one bulk tensor store; the gated residual (X += gate * y) becomes a
-// bulk tensor reduce-add of gate * y into X, so X is never read.  Rows and columns outside the
-// output are clipped by the tensor map.  A buffer is refilled once the store issued from it two
-// chunks earlier has read it.
+// instruction).  Results are staged 64 bytes per row (32 bf16 or 16 fp32 columns) in one of this
+// warp's two 2 KB shared memory buffers, in the 64-byte swizzled layout of a 32-row TMA box, and
+// written by one bulk tensor store per box; the gated residual (X += gate * y) becomes a bulk
+// tensor reduce-add of gate * y into X, so X is never read.  Rows and columns outside the output
+// are clipped by the tensor map.  A buffer is refilled once the store issued from it two boxes
+// earlier has read it.
 #pragma once
 
 #include "common.cuh"
@@ -18,11 +18,11 @@ namespace fdit {
 
 struct EpiTma {
   const CUtensorMap* map;   // output of this problem (make_tmap_out)
-  uint32_t buf0;            // shared address of this warp's two 4 KB staging buffers (1024-byte aligned)
+  uint32_t buf0;            // shared address of this warp's two 2 KB staging buffers (1024-byte aligned)
   int y0;                   // output row of lane 0
   int rows;                 // output rows: a box starting at or past them is not issued
   uint32_t* which;          // the buffer the next chunk fills (0 or 1), kept across tiles
-  __device__ __forceinline__ uint32_t buf() const { return buf0 + (*which << 12); }
+  __device__ __forceinline__ uint32_t buf() const { return buf0 + (*which << 11); }
 };
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -35,13 +35,14 @@ __device__ __forceinline__ void epi_tma_reuse() {
   __syncwarp();
 }
 
-// Row `lane` of a fp32 chunk (32 values) into the 128-byte swizzled box layout.
-__device__ __forceinline__ void epi_stage_f32(const EpiTma& e, const float (&f)[32]) {
+// Row `lane` of half h of a fp32 chunk (16 of its 32 values) into the 64-byte swizzled box layout.
+__device__ __forceinline__ void epi_stage_f32(const EpiTma& e, const float (&f)[32], int h) {
   const uint32_t t = threadIdx.x & 31;
 #pragma unroll
-  for (uint32_t u = 0; u < 8; ++u)
-    st_shared_v4(e.buf() + t * 128 + ((u ^ (t & 7)) << 4), __float_as_uint(f[4 * u]), __float_as_uint(f[4 * u + 1]),
-                 __float_as_uint(f[4 * u + 2]), __float_as_uint(f[4 * u + 3]));
+  for (uint32_t u = 0; u < 4; ++u)
+    st_shared_v4(e.buf() + t * 64 + ((u ^ ((t >> 1) & 3)) << 4), __float_as_uint(f[16 * h + 4 * u]),
+                 __float_as_uint(f[16 * h + 4 * u + 1]), __float_as_uint(f[16 * h + 4 * u + 2]),
+                 __float_as_uint(f[16 * h + 4 * u + 3]));
 }
 // Row `lane` of a bf16 chunk (32 values, 16 packed words) into the 64-byte swizzled box layout.
 __device__ __forceinline__ void epi_stage_bf16(const EpiTma& e, const uint32_t (&w)[16]) {
@@ -51,7 +52,7 @@ __device__ __forceinline__ void epi_stage_bf16(const EpiTma& e, const uint32_t (
     st_shared_v4(e.buf() + t * 64 + ((u ^ ((t >> 1) & 3)) << 4), w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
 }
 
-// Store (or, with add, reduce-add) the staged {32, 32} box at output column x; the next chunk
+// Store (or, with add, reduce-add) the staged 32-row box at output column x; the next box
 // takes the other buffer.  Lane 0 (which issues and waits for every store of the warp) commits a
 // group, possibly empty, per chunk, so that "all but the latest group" is always the buffer being
 // refilled.
@@ -247,8 +248,11 @@ __device__ __forceinline__ void gemm_epilogue_tile_tma(const GemmProblem& pr, ui
             f[4 * v] *= gv.x; f[4 * v + 1] *= gv.y; f[4 * v + 2] *= gv.z; f[4 * v + 3] *= gv.w;
           }
         }
-        epi_stage_f32(e, f);
+        epi_stage_f32(e, f, 0);
         epi_tma_issue(e, n, pr.mode == kEpiResidGate);
+        epi_tma_reuse();
+        epi_stage_f32(e, f, 1);
+        epi_tma_issue(e, n + 16, pr.mode == kEpiResidGate);
       }
     }
   }

@@ -81,8 +81,8 @@ static bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType type, uint32_t bo
 
 bool make_tmap_out(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
                    bool f32) {
-  return make_tmap_2d(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32, base, rows,
-                      cols, row_stride_bytes, 32, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+  return make_tmap_2d(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 ? 16 : 32,
+                      base, rows, cols, row_stride_bytes, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 bool make_tmap_sf(CUtensorMap* map, const void* base, uint64_t bytes) {

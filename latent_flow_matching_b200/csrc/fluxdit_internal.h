@@ -195,7 +195,7 @@ bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t co
                   uint32_t box_rows);
 // Block scales of an NVFP4 matrix as 256-byte rows, box 8 rows (2 KB: one stage of 128 rows), no swizzle.
 bool make_tmap_sf(CUtensorMap* map, const void* base, uint64_t bytes);
-// GEMM output written by TMA: fp32 (128-byte swizzle) or bf16 (64-byte swizzle), box {32 cols, 32 rows}.
+// GEMM output written by TMA: 64-byte box rows (16 fp32 or 32 bf16 columns) x 32 rows, 64-byte swizzle.
 bool make_tmap_out(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
                    bool f32);
 int num_sms_current();

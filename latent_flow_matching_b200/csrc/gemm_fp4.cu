@@ -37,7 +37,7 @@ namespace {
 constexpr int BM = 256;
 constexpr int BN = 256;
 constexpr int BKE = 256;                       // K elements per stage (128 bytes of codes per row)
-constexpr int STAGES = 4;
+constexpr int STAGES = 5;
 constexpr int A_BYTES = 128 * 128;             // 16 KB of codes
 constexpr int B_BYTES = 128 * 128;
 constexpr int SFA_BYTES = 128 * BKE / 16;      // 2 KB: 128 rows x 16 scales
@@ -48,7 +48,7 @@ constexpr uint32_t kAcc1Col = 224;             // buffer 1 shares columns [224, 
 constexpr uint32_t kSfCol = 480;               // two scale slots of 16 columns: SFA 4 | SFB 8
 constexpr int kEpiWarps = 8;
 constexpr int kThreads4 = 32 * (2 + kEpiWarps);
-constexpr int EPI_BYTES = 8192;                // per epilogue warp: two staged {32, 32} fp32 boxes
+constexpr int EPI_BYTES = 4096;                // per epilogue warp: two staged 32-row x 64-byte boxes
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + kEpiWarps * EPI_BYTES + 1024 + 512;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 
