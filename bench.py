@@ -195,7 +195,7 @@ def barrier(world):
 
 # the sources whose change invalidates the committed DRAM-traffic figure of the pair GEMM
 GEMM_TRAFFIC_SOURCES = ("gemm_tc2.cu", "gemm_epilogue.cuh", "pair.cuh", "common.cuh")
-GEMM4_TRAFFIC_SOURCES = ("gemm_fp4.cu", "gemm_epilogue.cuh", "pair.cuh", "common.cuh")
+GEMM4_TRAFFIC_SOURCES = ("gemm_fp4.cu", "epilogue_tma.cuh", "gemm_epilogue.cuh", "pair.cuh", "common.cuh")
 
 
 def profile_traffic(kernel_files, profile):
