@@ -340,3 +340,46 @@ def test_tiny3_nvfp4_forward_and_guided_batch(tiny3, nt, grid, ref_grids):
     print(f"flux3 nvfp4 forward vs nvfp4 oracle {err:.4f}")
     assert err <= NV4_V_TOL, err
     assert torch.equal(vc, v) and torch.equal(vu, su)
+
+
+def test_tiny_nvfp4_sampler_against_nvfp4_oracle(tiny):
+    """Two NVFP4 sampling steps: every velocity and the final latent within the NVFP4 bar."""
+    w, p, model = tiny
+    lat, txt, _ = make_inputs(w)
+    hq = dict(O.hyper(w.dims), nvfp4=True)
+    ref_final, ref_vs = O.sample(p, hq, torch.from_numpy(lat), torch.from_numpy(txt), 2)
+    vs = []
+    model.set_precision(F.PRECISION_NVFP4)
+    try:
+        final = F.flux_sample(model, torch.from_numpy(lat).to(DEV), torch.from_numpy(txt).to(DEV), 2,
+                              on_step=lambda i, v: vs.append(v.cpu().clone()))
+    finally:
+        model.set_precision(F.PRECISION_BF16)
+    assert len(vs) == 2
+    for a, b in zip(vs, ref_vs):
+        assert rel_l2(a, b) <= NV4_V_TOL
+    assert rel_l2(final.cpu(), ref_final) <= NV4_V_TOL
+
+
+def test_flux3_nvfp4_full_size_against_bf16_and_fp8():
+    """FLUX.3 1024^2 workload, full model (5 + 28 blocks): NVFP4 lands further from bf16 than FP8."""
+    w = WORKLOADS["f3t2i1024"]
+    blob, _ = make_weights(w.dims, w.seed)
+    lat, txt, _ = make_inputs(w)
+    model = F.Flux3DiT(blob, w.dims)
+    del blob
+    try:
+        tok = O.pack_latents(torch.from_numpy(lat)).float().to(DEV)
+        tx = torch.from_numpy(txt).to(DEV)
+        v16, v8, v4 = (torch.empty(w.n_img, 128, device=DEV) for _ in range(3))
+        model.forward(tok, (w.grid, w.grid), tx, 1.0, v16, t_target=15 / 16)
+        model.set_precision(F.PRECISION_FP8)
+        model.forward(tok, (w.grid, w.grid), tx, 1.0, v8, t_target=15 / 16)
+        model.set_precision(F.PRECISION_NVFP4)
+        model.forward(tok, (w.grid, w.grid), tx, 1.0, v4, t_target=15 / 16)
+        torch.cuda.synchronize()
+        e8, e4 = rel_l2(v8, v16), rel_l2(v4, v16)
+        print(f"FLUX.3 1024^2 fp8 vs bf16 {e8:.4f}, nvfp4 vs bf16 {e4:.4f}")
+        assert torch.isfinite(v4).all() and e8 < e4 < 0.5, (e8, e4)
+    finally:
+        model.close()
