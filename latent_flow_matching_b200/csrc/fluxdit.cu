@@ -85,6 +85,36 @@ bool make_tmap_out(CUtensorMap* map, const void* base, uint64_t rows, uint64_t c
                       base, rows, cols, row_stride_bytes, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
+namespace {
+struct OutMapEntry {
+  const void* base;
+  uint64_t rows, cols, stride;
+  bool f32;
+  CUtensorMap map;
+};
+}  // namespace
+
+bool gemm_out_map(CUtensorMap* dst, const GemmProblem& pr) {
+  static std::vector<OutMapEntry> cache;
+  static std::mutex mu;
+  const bool f32 = pr.mode == kEpiF32Bias || pr.mode == kEpiResidGate;
+  const uint64_t cols = pr.mode == kEpiSwiGLU ? pr.N / 2 : pr.N;
+  const uint64_t stride = static_cast<uint64_t>(pr.ldo) * (f32 ? 4 : 2);
+  std::lock_guard<std::mutex> lock(mu);
+  for (const OutMapEntry& c : cache)
+    if (c.base == pr.out && c.rows == static_cast<uint64_t>(pr.M) && c.cols == cols && c.stride == stride &&
+        c.f32 == f32) {
+      *dst = c.map;
+      return true;
+    }
+  OutMapEntry c{pr.out, static_cast<uint64_t>(pr.M), cols, stride, f32, {}};
+  if (!make_tmap_out(&c.map, pr.out, c.rows, cols, stride, f32)) return false;
+  if (cache.size() >= 512) cache.erase(cache.begin());
+  cache.push_back(c);
+  *dst = c.map;
+  return true;
+}
+
 bool make_tmap_sf(CUtensorMap* map, const void* base, uint64_t bytes) {
   if (bytes % 256) return false;
   return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 256, base, bytes / 256, 256, 256, 8,

@@ -198,6 +198,9 @@ bool make_tmap_sf(CUtensorMap* map, const void* base, uint64_t bytes);
 // GEMM output written by TMA: 64-byte box rows (16 fp32 or 32 bf16 columns) x 32 rows, 64-byte swizzle.
 bool make_tmap_out(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
                    bool f32);
+// The output map of problem pr for a TMA-store epilogue (fp32 for kEpiF32Bias / kEpiResidGate, N / 2
+// columns for SwiGLU), encoded once per (buffer, shape) and kept.
+bool gemm_out_map(CUtensorMap* map, const GemmProblem& pr);
 int num_sms_current();
 
 }  // namespace fdit

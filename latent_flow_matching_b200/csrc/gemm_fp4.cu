@@ -26,8 +26,6 @@
 #include "epilogue_tma.cuh"
 #include "pair.cuh"
 
-#include <vector>
-
 namespace fdit {
 
 __device__ int g_gemm4_error;
@@ -54,32 +52,6 @@ static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 
 static_assert(BN - kAcc1Col == 32 && kAcc1Col + BN <= kSfCol && kSfCol + 28 <= TMEM_COLS, "tensor memory plan");
 static_assert(STAGE_BYTES % 1024 == 0, "the epilogue staging buffers need 1024-byte alignment");
-
-// Output tensor maps of the epilogue's TMA stores, encoded once per (buffer, shape).
-struct OutMapEntry {
-  const void* base;
-  uint64_t rows, cols, stride;
-  bool f32;
-  CUtensorMap map;
-};
-bool out_map(CUtensorMap* dst, const GemmProblem& pr) {
-  static std::vector<OutMapEntry> cache;
-  const bool f32 = pr.mode == kEpiF32Bias || pr.mode == kEpiResidGate;
-  const uint64_t cols = pr.mode == kEpiSwiGLU ? pr.N / 2 : pr.N;
-  const uint64_t stride = static_cast<uint64_t>(pr.ldo) * (f32 ? 4 : 2);
-  for (const OutMapEntry& c : cache)
-    if (c.base == pr.out && c.rows == static_cast<uint64_t>(pr.M) && c.cols == cols && c.stride == stride &&
-        c.f32 == f32) {
-      *dst = c.map;
-      return true;
-    }
-  OutMapEntry c{pr.out, static_cast<uint64_t>(pr.M), cols, stride, f32, {}};
-  if (!make_tmap_out(&c.map, pr.out, c.rows, cols, stride, f32)) return false;
-  if (cache.size() >= 512) cache.erase(cache.begin());
-  cache.push_back(c);
-  *dst = c.map;
-  return true;
-}
 
 __device__ __forceinline__ int find_problem(const GemmParams& P, int tile) {
   int p = 0;
@@ -349,7 +321,7 @@ cudaError_t gemm_fp4_launch(GemmParams4& P4, int num_sms, cudaStream_t stream) {
   for (int i = 0; i < P.num_problems; ++i) {        // K in whole stages, scales present
     const GemmProblem& pr = P.prob[i];
     if (pr.M > 0 && (pr.K % BKE != 0 || !pr.scale_a || !pr.scale_b)) return cudaErrorInvalidValue;
-    if (pr.M > 0 && pr.N > 0 && !out_map(&P4.mapOut[i], pr)) return cudaErrorInvalidValue;
+    if (pr.M > 0 && pr.N > 0 && !gemm_out_map(&P4.mapOut[i], pr)) return cudaErrorInvalidValue;
   }
   int w = 0, total = 0;
   for (int i = 0; i < P.num_problems; ++i) {
