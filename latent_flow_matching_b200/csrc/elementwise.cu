@@ -185,9 +185,12 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(__nv_bfloat16* __rest
   const float cs[4] = {r01.x, r01.z, r23.x, r23.z};
   const float sn[4] = {r01.y, r01.w, r23.y, r23.w};
   __nv_bfloat16* base = qkv + static_cast<size_t>(row) * ld + (which ? kcol : 0);
-  for (int h = hsub; h < heads; h += 2) {
-    uint4* p = reinterpret_cast<uint4*>(base + h * 128) + hl;
-    const uint4 w = *p;
+  // every lane takes every shuffle: with an odd head count the second half-warp idles on the last pair
+  for (int h0 = 0; h0 < heads; h0 += 2) {
+    const int h = h0 + hsub;
+    const bool act = h < heads;
+    uint4* p = reinterpret_cast<uint4*>(base + (act ? h : 0) * 128) + hl;
+    const uint4 w = act ? *p : make_uint4(0u, 0u, 0u, 0u);
     float x[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
                   bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
     float ss = 0.f;
@@ -203,7 +206,7 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(__nv_bfloat16* __rest
       const float b = x[2 * pr + 1] * r * g[2 * pr + 1];
       out[pr] = pack_bf16x2(a * cs[pr] - b * sn[pr], a * sn[pr] + b * cs[pr]);
     }
-    *p = make_uint4(out[0], out[1], out[2], out[3]);
+    if (act) *p = make_uint4(out[0], out[1], out[2], out[3]);
   }
 }
 

@@ -90,9 +90,11 @@ def test_rope_table_matches_oracle_angles():
     assert (t[..., 1] - torch.sin(ang)).abs().max() < 1e-6
 
 
-@pytest.mark.parametrize("nt,gh,gw,rh,rw", [(7, 5, 6, 4, 4), (512, 16, 16, 0, 0)])
-def test_qk_rmsnorm_rope(nt, gh, gw, rh, rw):
-    heads, D = 24, 3072
+@pytest.mark.parametrize("nt,gh,gw,rh,rw,heads", [(7, 5, 6, 4, 4, 24), (512, 16, 16, 0, 0, 24), (7, 5, 6, 0, 0, 5),
+                                                  (3, 4, 4, 0, 0, 1)])
+def test_qk_rmsnorm_rope(nt, gh, gw, rh, rw, heads):
+    """Odd head counts leave the second half-warp without a head on the last pair."""
+    D = heads * 128
     n = nt + gh * gw + rh * rw
     qkv = bf(rand((n, 3 * D), 6, 1.5))
     gq, gk = bf(rand((128,), 7)), bf(rand((128,), 8))
