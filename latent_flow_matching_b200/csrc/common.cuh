@@ -258,6 +258,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+// silu(x) = x / (1 + e^-x).  The fast division (2 ulp; 0 once the denominator passes 2^126, i.e.
+// for x < -87, where silu is 0 in any output precision used here) instead of the IEEE one: the
+// SwiGLU epilogue divides once per output, and with the IEEE division it bounded the 8-bit GEMMs.
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 }  // namespace fdit
