@@ -151,8 +151,8 @@ FLUX_API int flux_dit_forward_cfg(flux_dit *m, const float *img_tok, int grid_h,
  * FLUX_PRECISION_NVFP4: the "nvfp4" format of the same section, which needs a Blackwell GPU: the
  * same operands as 4-bit e2m1 codes with one e4m3 scale per 16 elements and one fp32 scale per
  * row (flux_quantize_rows_nvfp4), multiplied by tcgen05 block-scaled MMAs; the first switch
- * quantises the block weights once (half a byte per weight plus the scales).  Needs hidden and
- * mlp_hidden multiples of 256 and hidden + mlp_hidden <= 16384. */
+ * quantises the block weights once (half a byte per weight plus the scales).  Needs hidden in
+ * {1024, 2048, 3072, 4096}, mlp_hidden a multiple of 256 and hidden + mlp_hidden <= 16384. */
 #define FLUX_PRECISION_BF16 0
 #define FLUX_PRECISION_FP8 1
 #define FLUX_PRECISION_NVFP4 2
@@ -280,8 +280,8 @@ FLUX_API int flux_quantize_rows_nvfp4(const uint16_t *x, int rows, int k, int ld
                                       float *row_scale, void *stream);
 
 /* flux_layernorm_modulate with its output rounded to bf16 and quantised to NVFP4 in the same pass
- * (codes [rows, dim/2], block scales and row scales as flux_quantize_rows_nvfp4).  dim % 512 == 0,
- * dim <= 16384. */
+ * (codes [rows, dim/2], block scales and row scales as flux_quantize_rows_nvfp4).  dim in
+ * {1024, 2048, 3072, 4096}. */
 FLUX_API int flux_layernorm_modulate_nvfp4(const float *x, uint8_t *q, uint8_t *sf, float *row_scale, int rows,
                                            int dim, const float *shift, const float *scale, float eps,
                                            void *stream);

@@ -1114,8 +1114,11 @@ int flux_dit_set_precision(flux_dit* m, int precision) {
       (c.hidden % 128 || c.mlp_hidden % 128 || (c.hidden != 1024 && c.hidden != 2048 && c.hidden != 3072 &&
                                                 c.hidden != 4096) || c.hidden + c.mlp_hidden > 16384))
     return fail(FLUX_EINVAL, "FP8 needs hidden in {1024, 2048, 3072, 4096} and hidden + mlp_hidden <= 16384");
-  if (precision == FLUX_PRECISION_NVFP4 && (c.hidden % 256 || c.mlp_hidden % 256 || c.hidden + c.mlp_hidden > 16384))
-    return fail(FLUX_EINVAL, "NVFP4 needs hidden and mlp_hidden multiples of 256 and hidden + mlp_hidden <= 16384");
+  if (precision == FLUX_PRECISION_NVFP4 &&
+      ((c.hidden != 1024 && c.hidden != 2048 && c.hidden != 3072 && c.hidden != 4096) || c.mlp_hidden % 256 ||
+       c.hidden + c.mlp_hidden > 16384))
+    return fail(FLUX_EINVAL, "NVFP4 needs hidden in {1024, 2048, 3072, 4096}, mlp_hidden a multiple of 256 and "
+                             "hidden + mlp_hidden <= 16384");
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev != m->device) return fail(FLUX_EINVAL, "model lives on device %d, current device is %d", m->device, dev);
@@ -1352,8 +1355,8 @@ int flux_quantize_rows_nvfp4(const uint16_t* x, int rows, int k, int ldx, uint8_
 int flux_layernorm_modulate_nvfp4(const float* x, uint8_t* q, uint8_t* sf, float* row_scale, int rows, int dim,
                                   const float* shift, const float* scale, float eps, void* stream) {
   if (!x || !q || !sf || !row_scale || !shift || !scale) return fail(FLUX_EINVAL, "NULL argument");
-  if (rows < 0 || dim < 512 || dim % 512 || dim > 16384)
-    return fail(FLUX_EINVAL, "bad shape rows=%d dim=%d (dim %% 512, dim <= 16384)", rows, dim);
+  if (rows < 0 || (dim != 1024 && dim != 2048 && dim != 3072 && dim != 4096))
+    return fail(FLUX_EINVAL, "bad shape rows=%d dim=%d (dim in {1024, 2048, 3072, 4096})", rows, dim);
   if (!aligned16(x) || !aligned16(q) || !aligned16(sf) || !aligned16(row_scale) || !aligned16(shift) ||
       !aligned16(scale))
     return fail(FLUX_EINVAL, "pointers must be 16-byte aligned");

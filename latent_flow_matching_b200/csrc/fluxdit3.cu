@@ -941,8 +941,11 @@ int flux3_dit_set_precision(flux3_dit* m, int precision) {
       ((c.hidden != 1024 && c.hidden != 2048 && c.hidden != 3072 && c.hidden != 4096) ||
        c.hidden + c.mlp_hidden > 16384))
     return fail(FLUX_EINVAL, "FP8 needs hidden in {1024, 2048, 3072, 4096} and hidden + mlp_hidden <= 16384");
-  if (precision == FLUX_PRECISION_NVFP4 && (c.hidden % 256 || c.mlp_hidden % 256 || c.hidden + c.mlp_hidden > 16384))
-    return fail(FLUX_EINVAL, "NVFP4 needs hidden and mlp_hidden multiples of 256 and hidden + mlp_hidden <= 16384");
+  if (precision == FLUX_PRECISION_NVFP4 &&
+      ((c.hidden != 1024 && c.hidden != 2048 && c.hidden != 3072 && c.hidden != 4096) || c.mlp_hidden % 256 ||
+       c.hidden + c.mlp_hidden > 16384))
+    return fail(FLUX_EINVAL, "NVFP4 needs hidden in {1024, 2048, 3072, 4096}, mlp_hidden a multiple of 256 and "
+                             "hidden + mlp_hidden <= 16384");
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev != m->device) return fail(FLUX_EINVAL, "model lives on device %d, current device is %d", m->device, dev);

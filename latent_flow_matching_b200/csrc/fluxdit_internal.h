@@ -168,7 +168,7 @@ Q4Segs q4_segments(const int* row0, const int* rows, int n);
 cudaError_t quantize_nvfp4_launch(const __nv_bfloat16* x, int ldx, int k, uint8_t* q, int ldq, uint8_t* sf,
                                   float* row_scale, const Q4Segs& segs, cudaStream_t s);
 // LayerNorm + modulation (fp32 rows of x, dim values each) rounded to bf16 and quantised to NVFP4 as
-// quantize_nvfp4_launch (codes row stride dim / 2), over the rows of `segs`; dim % 512 == 0.
+// quantize_nvfp4_launch (codes row stride dim / 2), over the rows of `segs`; dim in {1024, 2048, 3072, 4096}.
 cudaError_t ln_modulate_nvfp4_launch(const float* x, int dim, uint8_t* q, uint8_t* sf, float* row_scale,
                                      const Q4Segs& segs, const LnModSets& ms, float eps, cudaStream_t s);
 // Problems of the NVFP4 pair GEMM: mapA / mapB over the codes (u8 maps, 128-byte box), K in elements

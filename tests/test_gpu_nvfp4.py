@@ -110,22 +110,22 @@ def test_quantize_rows_nvfp4_bit_exact_against_oracle(rows, k):
     assert torch.equal(decode_codes(q), qc)
 
 
-@pytest.mark.parametrize("rows", [4608 + 5, 33])
-def test_layernorm_modulate_nvfp4_against_oracle(rows):
+@pytest.mark.parametrize("rows,dim", [(4608 + 5, 3072), (33, 3072), (70, 1024), (40, 2048), (37, 4096)])
+def test_layernorm_modulate_nvfp4_against_oracle(rows, dim):
     """LN-mod rounded to bf16 and quantised in one pass: the codes, block scales and row scales of
     the oracle's quantisation of the same bf16 row, except where the two LayerNorm evaluations
     (float32 here, float64 there) round an element to neighbouring bf16 values, which may move the
     element's code by one step (or a block scale by one e4m3 step when it moves the block maximum)."""
-    x = rand((rows, 3072), 150) * 3 + 0.5
-    shift, scale = rand((3072,), 151), rand((3072,), 152, 0.5)
-    q = torch.empty(rows, 1536, dtype=torch.uint8, device=DEV)
-    sf = torch.zeros(F.flux_nvfp4_scale_bytes(rows, 3072), dtype=torch.uint8, device=DEV)
+    x = rand((rows, dim), 150) * 3 + 0.5
+    shift, scale = rand((dim,), 151), rand((dim,), 152, 0.5)
+    q = torch.empty(rows, dim // 2, dtype=torch.uint8, device=DEV)
+    sf = torch.zeros(F.flux_nvfp4_scale_bytes(rows, dim), dtype=torch.uint8, device=DEV)
     s = torch.empty(rows, dtype=torch.float32, device=DEV)
     F.flux_layernorm_modulate_nvfp4(x.to(DEV), q, sf, s, shift.to(DEV), scale.to(DEV))
     y = O.modulate(O.layer_norm(x.double(), 1e-6), shift.double(), scale.double())
     qc, qsb, qs = Q4.quantize_rows_nvfp4(y.to(torch.bfloat16).float())
     assert torch.allclose(s.cpu().double(), qs.double(), rtol=2 ** -7, atol=0)
-    sb = decode_sf(sf, rows, 3072)
+    sb = decode_sf(sf, rows, dim)
     assert (sb != qsb).double().mean() < 1e-3
     codes = decode_codes(q)
     same_blocks = (sb == qsb).repeat_interleave(16, dim=1) & (s.cpu() == qs)[:, None]
