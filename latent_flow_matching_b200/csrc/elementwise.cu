@@ -25,33 +25,71 @@ inline int blocks_for(size_t n, int per_block) {
 
 // ------------------------------------------------------------------ pack / unpack
 // token (i, j) channel c*4 + py*2 + px  <->  lat[c, 2i+py, 2j+px]
-__global__ void pack_kernel(const float* __restrict__ lat, float* __restrict__ tok, int C, int h8, int w8) {
-  const int gw = w8 / 2;
-  const size_t total = static_cast<size_t>(h8 / 2) * gw * C;
-  for (size_t idx = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; idx < total;
-       idx += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(idx % C);
-    const size_t t = idx / C;
-    const int i = static_cast<int>(t / gw), j = static_cast<int>(t % gw);
-    const float* src = lat + (static_cast<size_t>(c) * h8 + 2 * i) * w8 + 2 * j;
-    const float2 top = *reinterpret_cast<const float2*>(src);
-    const float2 bot = *reinterpret_cast<const float2*>(src + w8);
-    reinterpret_cast<float4*>(tok)[idx] = make_float4(top.x, top.y, bot.x, bot.y);
+//
+// The packing transposes channels and tokens: a latent row is contiguous along j, a token is
+// contiguous along its 128 channels.  One CTA takes a tile of kPackT consecutive tokens of one
+// token row i (all 32 channels, 2 latent rows each) and stages it in shared memory, so that both
+// the latent side (8 bytes per thread, a warp spans 256 contiguous bytes of one latent row) and the
+// token side (16 bytes per thread, the tile is kPackT * 512 contiguous bytes) are coalesced.
+constexpr int kPackC = 32;            // latent channels; 4 * kPackC = 128 token channels
+constexpr int kPackT = 32;            // tokens per tile
+constexpr int kPackLd = 4 * kPackC + 4;   // shared row stride in floats: 16-byte rows, 4-bank skew
+constexpr int kPackThreads = 256;
+
+struct PackTile {
+  int i, j0, gw;
+};
+__device__ __forceinline__ PackTile pack_tile(int w8) {
+  const int gw = w8 / 2, tiles_w = (gw + kPackT - 1) / kPackT;
+  return {static_cast<int>(blockIdx.x / tiles_w), static_cast<int>(blockIdx.x % tiles_w) * kPackT, gw};
+}
+
+__global__ void __launch_bounds__(kPackThreads) pack_kernel(const float* __restrict__ lat, float* __restrict__ tok,
+                                                            int h8, int w8) {
+  __shared__ __align__(16) float st[kPackT * kPackLd];
+  const PackTile tl = pack_tile(w8);
+  // latent side: item (c, py, jj), jj fastest
+#pragma unroll
+  for (int s = 0; s < kPackC * 2 * kPackT / kPackThreads; ++s) {
+    const int item = threadIdx.x + s * kPackThreads;
+    const int jj = item % kPackT, cp = item / kPackT, c = cp >> 1, py = cp & 1;
+    if (tl.j0 + jj < tl.gw) {
+      const float2 v = __ldcs(reinterpret_cast<const float2*>(
+          lat + (static_cast<size_t>(c) * h8 + 2 * tl.i + py) * w8 + 2 * (tl.j0 + jj)));
+      *reinterpret_cast<float2*>(st + jj * kPackLd + c * 4 + py * 2) = v;
+    }
+  }
+  __syncthreads();
+  // token side: item (jj, quad), quad fastest
+  float4* dst = reinterpret_cast<float4*>(tok + (static_cast<size_t>(tl.i) * tl.gw + tl.j0) * (4 * kPackC));
+#pragma unroll
+  for (int s = 0; s < kPackT * kPackC / kPackThreads; ++s) {
+    const int item = threadIdx.x + s * kPackThreads;
+    const int jj = item / kPackC, qd = item % kPackC;
+    if (tl.j0 + jj < tl.gw) dst[item] = *reinterpret_cast<const float4*>(st + jj * kPackLd + qd * 4);
   }
 }
 
-__global__ void unpack_kernel(const float* __restrict__ tok, float* __restrict__ lat, int C, int h8, int w8) {
-  const int gw = w8 / 2;
-  const size_t total = static_cast<size_t>(h8 / 2) * gw * C;
-  for (size_t idx = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; idx < total;
-       idx += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(idx % C);
-    const size_t t = idx / C;
-    const int i = static_cast<int>(t / gw), j = static_cast<int>(t % gw);
-    const float4 v = reinterpret_cast<const float4*>(tok)[idx];
-    float* dst = lat + (static_cast<size_t>(c) * h8 + 2 * i) * w8 + 2 * j;
-    *reinterpret_cast<float2*>(dst) = make_float2(v.x, v.y);
-    *reinterpret_cast<float2*>(dst + w8) = make_float2(v.z, v.w);
+__global__ void __launch_bounds__(kPackThreads) unpack_kernel(const float* __restrict__ tok, float* __restrict__ lat,
+                                                              int h8, int w8) {
+  __shared__ __align__(16) float st[kPackT * kPackLd];
+  const PackTile tl = pack_tile(w8);
+  const float4* src =
+      reinterpret_cast<const float4*>(tok + (static_cast<size_t>(tl.i) * tl.gw + tl.j0) * (4 * kPackC));
+#pragma unroll
+  for (int s = 0; s < kPackT * kPackC / kPackThreads; ++s) {
+    const int item = threadIdx.x + s * kPackThreads;
+    const int jj = item / kPackC, qd = item % kPackC;
+    if (tl.j0 + jj < tl.gw) *reinterpret_cast<float4*>(st + jj * kPackLd + qd * 4) = __ldcs(src + item);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int s = 0; s < kPackC * 2 * kPackT / kPackThreads; ++s) {
+    const int item = threadIdx.x + s * kPackThreads;
+    const int jj = item % kPackT, cp = item / kPackT, c = cp >> 1, py = cp & 1;
+    if (tl.j0 + jj < tl.gw)
+      *reinterpret_cast<float2*>(lat + (static_cast<size_t>(c) * h8 + 2 * tl.i + py) * w8 + 2 * (tl.j0 + jj)) =
+          *reinterpret_cast<const float2*>(st + jj * kPackLd + c * 4 + py * 2);
   }
 }
 
@@ -341,17 +379,28 @@ __global__ void __launch_bounds__(256) gemv_kernel(const __nv_bfloat16* __restri
 
 }  // namespace
 
+// One CTA per tile of kPackT tokens of one token row.
+static cudaError_t pack_grid(int c, int h8, int w8, unsigned* tiles) {
+  if (c != kPackC || h8 < 2 || w8 < 2 || (h8 | w8) & 1) return cudaErrorInvalidValue;
+  const long t = static_cast<long>(h8 / 2) * ((w8 / 2 + kPackT - 1) / kPackT);
+  if (t >= (1l << 31)) return cudaErrorInvalidValue;
+  *tiles = static_cast<unsigned>(t);
+  return cudaSuccess;
+}
+
 cudaError_t pack_latents_launch(const float* lat, float* tok, int c, int h8, int w8, cudaStream_t s) {
-  const size_t total = static_cast<size_t>(h8 / 2) * (w8 / 2) * c;
+  unsigned tiles;
+  if (const cudaError_t e = pack_grid(c, h8, w8, &tiles)) return e;
   count_launch();
-  pack_kernel<<<blocks_for(total, 256), 256, 0, s>>>(lat, tok, c, h8, w8);
+  pack_kernel<<<tiles, kPackThreads, 0, s>>>(lat, tok, h8, w8);
   return cudaGetLastError();
 }
 
 cudaError_t unpack_latents_launch(const float* tok, float* lat, int c, int h8, int w8, cudaStream_t s) {
-  const size_t total = static_cast<size_t>(h8 / 2) * (w8 / 2) * c;
+  unsigned tiles;
+  if (const cudaError_t e = pack_grid(c, h8, w8, &tiles)) return e;
   count_launch();
-  unpack_kernel<<<blocks_for(total, 256), 256, 0, s>>>(tok, lat, c, h8, w8);
+  unpack_kernel<<<tiles, kPackThreads, 0, s>>>(tok, lat, h8, w8);
   return cudaGetLastError();
 }
 
