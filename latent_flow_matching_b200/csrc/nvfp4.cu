@@ -114,19 +114,34 @@ __global__ void __launch_bounds__(kQ4Threads) quantize_nvfp4_kernel(const __nv_b
   q4_row_scales(cta_reduce<true>(amax, red), &inv, &S);
   if (tid == 0) row_scale[rr.r] = S;
   uint32_t* qr = reinterpret_cast<uint32_t*>(q + static_cast<size_t>(rr.r) * ldq);
+  // Group pairs (u0, u1) = (2w, 2w + 1): the two threads of a block each compute one of the pair's
+  // two block scales (thread parity p takes u_p) and exchange the reciprocals.
+  const int p = tid & 1;
 #pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int j = tid + u * kQ4Threads;             // n8 % 8 == 0: both threads of a block agree on j < n8
-    const float m = bf16_abs_max8(v[u], 0.f);
-    float rcp;
-    const __nv_fp8_storage_t s8 = q4_block_scale(fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1)), inv, S, &rcp);
-    const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-    uint32_t c = 0;
+  for (int w = 0; w < (U + 1) / 2; ++w) {
+    float m[2];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) c |= e2m1x2(bf16lo(w[e]), bf16hi(w[e]), rcp) << (8 * e);
-    if (j < n8) {
-      qr[j] = c;
-      if ((tid & 1) == 0) sf[q4_sf_offset(rr.sfr, j >> 1, k)] = s8;
+    for (int h = 0; h < 2; ++h) {
+      const float a = 2 * w + h < U ? bf16_abs_max8(v[2 * w + h], 0.f) : 0.f;
+      m[h] = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    }
+    float my_rcp;
+    const __nv_fp8_storage_t s8 = q4_block_scale(p ? m[1] : m[0], inv, S, &my_rcp);
+    const float other = __shfl_xor_sync(0xffffffffu, my_rcp, 1);
+    const int jp = tid + (2 * w + p) * kQ4Threads;  // n8 % 8 == 0: both threads of a block agree on j < n8
+    if (2 * w + p < U && jp < n8) sf[q4_sf_offset(rr.sfr, jp >> 1, k)] = s8;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int u = 2 * w + h;
+      if (u < U) {
+        const int j = tid + u * kQ4Threads;
+        const float rcp = h == p ? my_rcp : other;
+        const uint32_t e4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        uint32_t c = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c |= e2m1x2(bf16lo(e4[e]), bf16hi(e4[e]), rcp) << (8 * e);
+        if (j < n8) qr[j] = c;
+      }
     }
   }
 }
@@ -139,6 +154,7 @@ __global__ void __launch_bounds__(kQ4Threads) ln_mod_nvfp4_kernel(const float* _
                                                                   uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
                                                                   float* __restrict__ row_scale, const Q4Segs segs,
                                                                   LnModSets ms, float eps) {
+  static_assert(VPT >= 1 && VPT <= 4, "one block scale per quad lane");
   constexpr int dim = 1024 * VPT;
   __shared__ float red[kQ4Threads / 32];
   const int tid = threadIdx.x;
@@ -174,16 +190,26 @@ __global__ void __launch_bounds__(kQ4Threads) ln_mod_nvfp4_kernel(const float* _
   float inv, S;
   q4_row_scales(cta_reduce<true>(amax, red), &inv, &S);
   if (tid == 0) row_scale[rr.r] = S;
-  uint16_t* qr = reinterpret_cast<uint16_t*>(q + static_cast<size_t>(rr.r) * (dim / 2)) + tid;
+  // Float4 group g = tid + 256 i belongs to block g / 4: the quad of threads 4b..4b+3 shares block
+  // b + 64 i for every i.  Thread 4b + i computes the scale of the quad's i-th block once and the
+  // quad exchanges the reciprocals (lanes with 4b + i, i >= VPT, compute a spare copy of block 0).
+  const int quad_lane = tid & 3;
+  float mine = 0.f;
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {                    // block of float4 group j = tid + 256 i: threads 4g..4g+3
+  for (int i = 0; i < VPT; ++i) {
     float m = fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w)));
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    float rcp;
-    const __nv_fp8_storage_t s8 = q4_block_scale(m, inv, S, &rcp);
+    mine = (i == 0 || quad_lane == i) ? m : mine;
+  }
+  float my_rcp;
+  const __nv_fp8_storage_t s8 = q4_block_scale(mine, inv, S, &my_rcp);
+  if (quad_lane < VPT) sf[q4_sf_offset(rr.sfr, (tid >> 2) + 64 * quad_lane, dim)] = s8;
+  uint16_t* qr = reinterpret_cast<uint16_t*>(q + static_cast<size_t>(rr.r) * (dim / 2)) + tid;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const float rcp = __shfl_sync(0xffffffffu, my_rcp, (tid & 28) | i);
     qr[i * kQ4Threads] = static_cast<uint16_t>(e2m1x2(v[i].x, v[i].y, rcp) | (e2m1x2(v[i].z, v[i].w, rcp) << 8));
-    if ((tid & 3) == 0) sf[q4_sf_offset(rr.sfr, (tid + i * kQ4Threads) >> 2, dim)] = s8;
   }
 }
 
