@@ -198,7 +198,9 @@ FLUX_API int flux_blend_latents(const float *x, const float *noise, float t, flo
 
 /* 2x2 latent packing ("Zweistufiger Transformer und Tokenisierung"):
  *   lat fp32 [32, h8, w8]  <->  tok fp32 [(h8/2)*(w8/2), 128],
- *   tok[i*(w8/2)+j][c*4 + py*2 + px] = lat[c][2i+py][2j+px].  h8, w8 even, >= 2. */
+ *   tok[i*(w8/2)+j][c*4 + py*2 + px] = lat[c][2i+py][2j+px].  h8, w8 even, >= 2.
+ * Device pointers, 16-byte aligned, owned by the caller; the call is asynchronous on `stream`.
+ * FLUX_EINVAL (nothing launched) for a NULL or misaligned pointer or an odd / too small size. */
 FLUX_API int flux_pack_latents(const float *lat, float *tok, int h8, int w8, void *stream);
 FLUX_API int flux_unpack_latents(const float *tok, float *lat, int h8, int w8, void *stream);
 

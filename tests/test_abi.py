@@ -104,6 +104,9 @@ def test_entry_points_reject_bad_arguments(L):
     assert L.flux_pack_latents(p, p, 7, 8, None) == F.FLUX_EINVAL
     assert "even" in F.get_error()
     assert L.flux_unpack_latents(p, p, 8, 0, None) == F.FLUX_EINVAL
+    assert L.flux_pack_latents(ctypes.c_void_p(24), p, 8, 8, None) == F.FLUX_EINVAL   # 8-byte aligned only
+    assert "aligned" in F.get_error()
+    assert L.flux_unpack_latents(p, ctypes.c_void_p(20), 8, 8, None) == F.FLUX_EINVAL
     assert L.flux_joint_attention(p, p, p, p, 10, 2, 64, 0.1, None) == F.FLUX_EINVAL
     assert "head_dim" in F.get_error()
     assert L.flux_joint_attention(p, p, p, p, 0, 2, 128, 0.1, None) == F.FLUX_EINVAL
