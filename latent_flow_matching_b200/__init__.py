@@ -48,6 +48,14 @@ class FluxError(RuntimeError):
         self.code = code
 
 
+class FluxShapeError(FluxError, ValueError):
+    """A buffer whose shape, size or dtype does not fit the call (found before anything is launched;
+    code FLUX_EINVAL, like the library's own argument checks)."""
+
+    def __init__(self, msg):
+        super().__init__(FLUX_EINVAL, msg)
+
+
 _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 _SIGS = {
     "flux_get_error": (ctypes.c_char_p, []),
@@ -159,9 +167,83 @@ def _bits(t, what):
     return _ptr(t, None, what)
 
 
+# Size checks: the C ABI takes plain pointers, so the binding checks every buffer against the
+# sizes the call will touch before anything is launched (a short buffer would be read or written
+# past its end on the device).
+def _need_numel(t, n, what):
+    if t is not None and t.numel() < n:
+        raise FluxShapeError(f"{what} holds {t.numel()} elements; the call needs {n}")
+
+
+def _need_same(t, ref, what):
+    if t is None or tuple(t.shape) != tuple(ref.shape):
+        raise FluxShapeError(f"{what} must have shape {tuple(ref.shape)}")
+
+
+def _need_rows_cols(t, rows, cols, what):
+    if t.dim() != 2 or t.shape[0] < rows or t.shape[1] < cols or t.stride(1) != 1:
+        raise FluxShapeError(f"{what} must be 2-D with at least [{rows}, {cols}] and unit column stride, "
+                         f"got {tuple(t.shape)}")
+
+
+def _need_linear_out(out, gate, m, n, mode):
+    import torch
+    if mode not in (EPI_BF16_BIAS, EPI_F32_BIAS, EPI_SWIGLU, EPI_RESID_GATE):
+        return                                  # the library rejects it
+    bf = mode in (EPI_BF16_BIAS, EPI_SWIGLU)
+    if bf and out.dtype not in (torch.bfloat16, torch.uint16, torch.int16):
+        raise FluxShapeError("out must be bf16 for this mode")
+    if not bf and out.dtype != torch.float32:
+        raise FluxShapeError("out must be float32 for this mode")
+    _need_rows_cols(out, m, n // 2 if mode == EPI_SWIGLU else n, "out")
+    if mode == EPI_RESID_GATE:
+        if gate is None:
+            raise FluxShapeError("the gated residual mode needs gate")
+        _need_numel(gate, n, "gate")
+
+
+def _check_strided(t, kind, what):
+    """A 2-D buffer whose rows may be strided (unit column stride); kind "bf16", "u8" or None
+    (dtype checked elsewhere)."""
+    import torch
+    kinds = {"bf16": (torch.bfloat16, torch.uint16, torch.int16), "u8": (torch.uint8, torch.float8_e4m3fn)}
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise FluxShapeError(f"{what} must be 2-D with unit column stride")
+    if kind is not None and t.dtype not in kinds[kind]:
+        raise FluxShapeError(f"{what} must be {kind}, got {t.dtype}")
+
+
+def _strided(t, kind, what):
+    """_check_strided, then the device pointer."""
+    _check_strided(t, kind, what)
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _need_tokens(t, rows, what, width=128):
+    if t is None or t.numel() != rows * width:
+        raise FluxShapeError(f"{what} must hold {rows} x {width} values")
+
+
 def flux_blob_expected_bytes(dims) -> int:
     cfg = FluxConfig.from_dims(dims)
     return lib().flux_blob_expected_bytes(ctypes.byref(cfg))
+
+
+def _check_forward_shapes(dims, img_tok, grid_hw, txts, hw_list, ref_tok, outs):
+    """Token buffers of a forward: image tokens and every output [gh*gw, 128], each text
+    [n_txt, txt_dim] (txt_dim checked when the model's dims are known), references [sum h*w, 128]."""
+    n_img = int(grid_hw[0]) * int(grid_hw[1])
+    _need_tokens(img_tok, n_img, "img_tok")
+    for o in outs:
+        _need_tokens(o, n_img, "velocity output")
+    for txt in txts:
+        if txt is not None and (txt.dim() != 2 or (dims is not None and txt.shape[1] != dims.txt_dim)):
+            raise FluxShapeError("txt must be [n_txt, txt_dim]")
+    n_ref = sum(int(h) * int(w) for h, w in hw_list)
+    if n_ref:
+        _need_tokens(ref_tok, n_ref, "ref_tok")
 
 
 class FluxDiT:
@@ -192,6 +274,9 @@ class FluxDiT:
         reference's packed tokens, concatenated in order)."""
         import torch
         n_txt = 0 if txt is None else txt.shape[0]
+        hw_list = list(ref_hw) if ref_hw and isinstance(ref_hw[0], (tuple, list)) else \
+            ([tuple(ref_hw)] if ref_hw and ref_hw[0] else [])
+        self._check_shapes(img_tok, grid_hw, [txt], hw_list, ref_tok, [v_out])
         if ref_hw and isinstance(ref_hw[0], (tuple, list)):
             grids = (ctypes.c_int * (2 * len(ref_hw)))(*[v for hw in ref_hw for v in hw])
             _check(lib().flux_dit_forward_refs(self._h, _ptr(img_tok, torch.float32, "img_tok"), grid_hw[0],
@@ -215,6 +300,7 @@ class FluxDiT:
             raise ValueError("txt_cond and txt_uncond must have the same token count")
         if ref_hw and not isinstance(ref_hw[0], (tuple, list)):
             ref_hw = [tuple(ref_hw)] if ref_hw[0] else []
+        self._check_shapes(img_tok, grid_hw, [txt_cond, txt_uncond], list(ref_hw), ref_tok, [v_cond, v_uncond])
         grids = (ctypes.c_int * max(1, 2 * len(ref_hw)))(*[v for hw in ref_hw for v in hw])
         _check(lib().flux_dit_forward_cfg(self._h, _ptr(img_tok, torch.float32, "img_tok"), grid_hw[0], grid_hw[1],
                                           _ptr(txt_cond, torch.float32, "txt_cond"),
@@ -223,6 +309,9 @@ class FluxDiT:
                                           _ptr(v_cond, torch.float32, "v_cond"),
                                           _ptr(v_uncond, torch.float32, "v_uncond"), _stream(stream)))
         return v_cond, v_uncond
+
+    def _check_shapes(self, img_tok, grid_hw, txts, hw_list, ref_tok, outs):
+        _check_forward_shapes(self.dims, img_tok, grid_hw, txts, hw_list, ref_tok, outs)
 
     def set_active_blocks(self, n_double=-1, n_single=-1):
         _check(lib().flux_dit_set_active_blocks(self._h, n_double, n_single))
@@ -257,6 +346,7 @@ class FluxDiT:
 
     def modulation(self, t, out, stream=None):
         import torch
+        _need_numel(out, self.modulation_size(), "out")
         _check(lib().flux_dit_modulation(self._h, float(t), _ptr(out, torch.float32, "mods"), _stream(stream)))
         return out
 
@@ -306,6 +396,8 @@ class Flux3DiT:
         import torch
         n_txt = 0 if txt is None else txt.shape[0]
         n_refs, grids = _grids(ref_hw)
+        _check_forward_shapes(self.dims, img_tok, grid_hw, [txt], list(zip(grids[0::2], grids[1::2]))[:n_refs],
+                              ref_tok, [v_out])
         _check(lib().flux3_dit_forward(self._h, _ptr(img_tok, torch.float32, "img_tok"), grid_hw[0], grid_hw[1],
                                        _ptr(txt, torch.float32, "txt"), n_txt,
                                        _ptr(ref_tok, torch.float32, "ref_tok"), n_refs, grids, float(t),
@@ -321,6 +413,8 @@ class Flux3DiT:
         if (0 if txt_uncond is None else txt_uncond.shape[0]) != n_txt:
             raise ValueError("txt_cond and txt_uncond must have the same token count")
         n_refs, grids = _grids(ref_hw)
+        _check_forward_shapes(self.dims, img_tok, grid_hw, [txt_cond, txt_uncond],
+                              list(zip(grids[0::2], grids[1::2]))[:n_refs], ref_tok, [v_cond, v_uncond])
         _check(lib().flux3_dit_forward_cfg(self._h, _ptr(img_tok, torch.float32, "img_tok"), grid_hw[0], grid_hw[1],
                                            _ptr(txt_cond, torch.float32, "txt_cond"),
                                            _ptr(txt_uncond, torch.float32, "txt_uncond"), n_txt,
@@ -341,6 +435,7 @@ class Flux3DiT:
 
     def modulation(self, t, t_target, out, stream=None):
         import torch
+        _need_numel(out, self.modulation_size(), "out")
         _check(lib().flux3_dit_modulation(self._h, float(t), float(t_target), _ptr(out, torch.float32, "mods"),
                                           _stream(stream)))
         return out
@@ -372,6 +467,8 @@ def img2img_first_step(n_steps: int, strength: float) -> int:
 def flux_blend_latents(x, noise, t, out, stream=None):
     """out = (1 - t) x + t noise (img2img start state)."""
     import torch
+    _need_same(noise, x, "noise")
+    _need_same(out, x, "out")
     _check(lib().flux_blend_latents(_ptr(x, torch.float32, "x"), _ptr(noise, torch.float32, "noise"), float(t),
                                     _ptr(out, torch.float32, "out"), x.numel(), _stream(stream)))
     return out
@@ -379,6 +476,7 @@ def flux_blend_latents(x, noise, t, out, stream=None):
 
 def flux_euler_step(x, v, dt, stream=None):
     import torch
+    _need_same(v, x, "v")
     _check(lib().flux_euler_step(_ptr(x, torch.float32, "x"), _ptr(v, torch.float32, "v"), x.numel(),
                                  float(dt), _stream(stream)))
     return x
@@ -387,14 +485,23 @@ def flux_euler_step(x, v, dt, stream=None):
 def flux_cfg_euler_step(x, v_cond, v_uncond, guidance, dt, stream=None):
     """x += dt * (v_uncond + guidance * (v_cond - v_uncond)), in place."""
     import torch
+    _need_same(v_cond, x, "v_cond")
+    _need_same(v_uncond, x, "v_uncond")
     _check(lib().flux_cfg_euler_step(_ptr(x, torch.float32, "x"), _ptr(v_cond, torch.float32, "v_cond"),
                                      _ptr(v_uncond, torch.float32, "v_uncond"), x.numel(), float(guidance),
                                      float(dt), _stream(stream)))
     return x
 
 
+def _latent_tokens(lat, tok):
+    if lat.dim() != 3 or lat.shape[0] != 32:
+        raise FluxShapeError("lat must be [32, h8, w8]")
+    _need_tokens(tok, (lat.shape[1] // 2) * (lat.shape[2] // 2), "tok")
+
+
 def flux_pack_latents(lat, tok, stream=None):
     import torch
+    _latent_tokens(lat, tok)
     _check(lib().flux_pack_latents(_ptr(lat, torch.float32, "lat"), _ptr(tok, torch.float32, "tok"),
                                    lat.shape[1], lat.shape[2], _stream(stream)))
     return tok
@@ -402,12 +509,21 @@ def flux_pack_latents(lat, tok, stream=None):
 
 def flux_unpack_latents(tok, lat, stream=None):
     import torch
+    _latent_tokens(lat, tok)
     _check(lib().flux_unpack_latents(_ptr(tok, torch.float32, "tok"), _ptr(lat, torch.float32, "lat"),
                                      lat.shape[1], lat.shape[2], _stream(stream)))
     return lat
 
 
+def _qkvo(q, k, v, o):
+    if q.dim() != 3:
+        raise FluxShapeError("q must be [n, heads, head_dim]")
+    for t, name in ((k, "k"), (v, "v"), (o, "o")):
+        _need_same(t, q, name)
+
+
 def flux_joint_attention(q, k, v, o, scale=None, stream=None):
+    _qkvo(q, k, v, o)
     n, heads, hd = q.shape
     scale = hd ** -0.5 if scale is None else scale
     _check(lib().flux_joint_attention(_bits(q, "q"), _bits(k, "k"), _bits(v, "v"), _bits(o, "o"), n, heads, hd,
@@ -417,6 +533,7 @@ def flux_joint_attention(q, k, v, o, scale=None, stream=None):
 
 def flux_joint_attention_batch(q, k, v, o, batch, scale=None, stream=None):
     """q, k, v, o bf16 [batch * n, heads, 128]; sequence b attends within rows [b n, (b + 1) n)."""
+    _qkvo(q, k, v, o)
     rows, heads, hd = q.shape
     if rows % batch:
         raise ValueError("rows must be a multiple of batch")
@@ -428,6 +545,7 @@ def flux_joint_attention_batch(q, k, v, o, batch, scale=None, stream=None):
 
 def flux_joint_attention_segments(q, k, v, o, seg_len, scale=None, stream=None):
     """q, k, v, o bf16 [sum(seg_len), heads, 128]; each segment attends only within itself."""
+    _qkvo(q, k, v, o)
     rows, heads, hd = q.shape
     if sum(seg_len) != rows:
         raise ValueError("segment lengths must add up to the row count")
@@ -442,11 +560,16 @@ def flux_linear(a, w, bias, mode, out, gate=None, stream=None):
     import torch
     m, k = a.shape
     n = w.shape[0]
+    if w.dim() != 2 or w.shape[1] != k:
+        raise FluxShapeError("w must be [n, k] with the k of a")
+    _check_strided(a, "bf16", "a")
+    _need_numel(bias, n, "bias")
+    _need_linear_out(out, gate, m, n, mode)
     lda = a.stride(0)
     if a.stride(1) != 1:
         raise ValueError("a must have unit column stride")
-    _check(lib().flux_linear(ctypes.c_void_p(a.data_ptr()), m, k, lda, _bits(w, "w"), n, _bits(bias, "bias"), mode,
-                             ctypes.c_void_p(out.data_ptr()), out.stride(0),
+    _check(lib().flux_linear(_strided(a, "bf16", "a"), m, k, lda, _bits(w, "w"), n, _bits(bias, "bias"), mode,
+                             _strided(out, None, "out"), out.stride(0),
                              _ptr(gate, torch.float32, "gate"), _stream(stream)))
     return out
 
@@ -464,8 +587,12 @@ def flux_quantize_rows_e4m3(x, q, scale, stream=None):
     rows, cols = x.shape
     if x.stride(1) != 1 or q.stride(1) != 1:
         raise ValueError("x and q must have unit column stride")
-    _check(lib().flux_quantize_rows_e4m3(ctypes.c_void_p(x.data_ptr()), rows, cols, x.stride(0),
-                                         ctypes.c_void_p(q.data_ptr()), q.stride(0),
+    _check_strided(x, "bf16", "x")
+    _check_strided(q, "u8", "q")
+    _need_rows_cols(q, rows, cols, "q")
+    _need_numel(scale, rows, "scale")
+    _check(lib().flux_quantize_rows_e4m3(_strided(x, "bf16", "x"), rows, cols, x.stride(0),
+                                         _strided(q, "u8", "q"), q.stride(0),
                                          _ptr(scale, torch.float32, "scale"), _stream(stream)))
     return q, scale
 
@@ -473,6 +600,10 @@ def flux_quantize_rows_e4m3(x, q, scale, stream=None):
 def flux_layernorm_modulate_fp8(x, q, q_scale, shift, scale, eps=1e-6, stream=None):
     import torch
     rows, dim = x.shape
+    _need_numel(q, rows * dim, "q")
+    _need_numel(q_scale, rows, "q_scale")
+    _need_numel(shift, dim, "shift")
+    _need_numel(scale, dim, "scale")
     _check(lib().flux_layernorm_modulate_fp8(_ptr(x, torch.float32, "x"), _u8(q, "q"),
                                              _ptr(q_scale, torch.float32, "q_scale"), rows, dim,
                                              _ptr(shift, torch.float32, "shift"), _ptr(scale, torch.float32, "scale"),
@@ -487,9 +618,16 @@ def flux_linear_fp8(a, a_scale, w, w_scale, bias, mode, out, gate=None, stream=N
     n = w.shape[0]
     if a.stride(1) != 1:
         raise ValueError("a must have unit column stride")
-    _check(lib().flux_linear_fp8(ctypes.c_void_p(a.data_ptr()), _ptr(a_scale, torch.float32, "a_scale"), m, k,
+    if w.dim() != 2 or w.shape[1] != k:
+        raise FluxShapeError("w must be [n, k] with the k of a")
+    _check_strided(a, "u8", "a")
+    _need_numel(a_scale, m, "a_scale")
+    _need_numel(w_scale, n, "w_scale")
+    _need_numel(bias, n, "bias")
+    _need_linear_out(out, gate, m, n, mode)
+    _check(lib().flux_linear_fp8(_strided(a, "u8", "a"), _ptr(a_scale, torch.float32, "a_scale"), m, k,
                                  a.stride(0), _u8(w, "w"), _ptr(w_scale, torch.float32, "w_scale"), n,
-                                 _bits(bias, "bias"), mode, ctypes.c_void_p(out.data_ptr()), out.stride(0),
+                                 _bits(bias, "bias"), mode, _strided(out, None, "out"), out.stride(0),
                                  _ptr(gate, torch.float32, "gate"), _stream(stream)))
     return out
 
@@ -506,8 +644,13 @@ def flux_quantize_rows_nvfp4(x, q, sf, row_scale, stream=None):
     rows, k = x.shape
     if x.stride(1) != 1 or q.stride(1) != 1:
         raise ValueError("x and q must have unit column stride")
-    _check(lib().flux_quantize_rows_nvfp4(ctypes.c_void_p(x.data_ptr()), rows, k, x.stride(0),
-                                          ctypes.c_void_p(q.data_ptr()), q.stride(0), _u8(sf, "sf"),
+    _check_strided(x, "bf16", "x")
+    _check_strided(q, "u8", "q")
+    _need_rows_cols(q, rows, k // 2, "q")
+    _need_numel(sf, flux_nvfp4_scale_bytes(rows, k), "sf")
+    _need_numel(row_scale, rows, "row_scale")
+    _check(lib().flux_quantize_rows_nvfp4(_strided(x, "bf16", "x"), rows, k, x.stride(0),
+                                          _strided(q, "u8", "q"), q.stride(0), _u8(sf, "sf"),
                                           _ptr(row_scale, torch.float32, "row_scale"), _stream(stream)))
     return q, sf, row_scale
 
@@ -517,6 +660,11 @@ def flux_layernorm_modulate_nvfp4(x, q, sf, row_scale, shift, scale, eps=1e-6, s
     sf [flux_nvfp4_scale_bytes(rows, dim)], row_scale [rows])."""
     import torch
     rows, dim = x.shape
+    _need_numel(q, rows * dim // 2, "q")
+    _need_numel(sf, flux_nvfp4_scale_bytes(rows, dim), "sf")
+    _need_numel(row_scale, rows, "row_scale")
+    _need_numel(shift, dim, "shift")
+    _need_numel(scale, dim, "scale")
     _check(lib().flux_layernorm_modulate_nvfp4(_ptr(x, torch.float32, "x"), _u8(q, "q"), _u8(sf, "sf"),
                                                _ptr(row_scale, torch.float32, "row_scale"), rows, dim,
                                                _ptr(shift, torch.float32, "shift"), _ptr(scale, torch.float32, "scale"),
@@ -532,10 +680,19 @@ def flux_linear_nvfp4(a, a_sf, a_scale, w, w_sf, w_scale, bias, mode, out, gate=
     n = w.shape[0]
     if a.stride(1) != 1:
         raise ValueError("a must have unit column stride")
-    _check(lib().flux_linear_nvfp4(ctypes.c_void_p(a.data_ptr()), _u8(a_sf, "a_sf"),
+    if w.dim() != 2 or w.shape[1] != kh:
+        raise FluxShapeError("w must be [n, k/2] with the k of a")
+    _check_strided(a, "u8", "a")
+    _need_numel(a_sf, flux_nvfp4_scale_bytes(m, 2 * kh), "a_sf")
+    _need_numel(w_sf, flux_nvfp4_scale_bytes(n, 2 * kh), "w_sf")
+    _need_numel(a_scale, m, "a_scale")
+    _need_numel(w_scale, n, "w_scale")
+    _need_numel(bias, n, "bias")
+    _need_linear_out(out, gate, m, n, mode)
+    _check(lib().flux_linear_nvfp4(_strided(a, "u8", "a"), _u8(a_sf, "a_sf"),
                                    _ptr(a_scale, torch.float32, "a_scale"), m, 2 * kh, a.stride(0), _u8(w, "w"),
                                    _u8(w_sf, "w_sf"), _ptr(w_scale, torch.float32, "w_scale"), n,
-                                   _bits(bias, "bias"), mode, ctypes.c_void_p(out.data_ptr()), out.stride(0),
+                                   _bits(bias, "bias"), mode, _strided(out, None, "out"), out.stride(0),
                                    _ptr(gate, torch.float32, "gate"), _stream(stream)))
     return out
 
@@ -546,7 +703,16 @@ def flux_qkv_projection(a, w, bias, heads, q_gain, k_gain, table, qkv, table_row
     m, k = a.shape
     if a.stride(1) != 1:
         raise ValueError("a must have unit column stride")
-    _check(lib().flux_qkv_projection(ctypes.c_void_p(a.data_ptr()), m, k, a.stride(0), _bits(w, "w"),
+    n = 3 * heads * 128
+    _check_strided(a, "bf16", "a")
+    if w.dim() != 2 or tuple(w.shape) != (n, k):
+        raise FluxShapeError(f"w must be [{n}, {k}]")
+    _need_numel(bias, n, "bias")
+    _need_numel(q_gain, 128, "q_gain")
+    _need_numel(k_gain, 128, "k_gain")
+    _need_rows_cols(qkv, m, n, "qkv")
+    _need_numel(table, (table_row0 + m) * 128, "table")
+    _check(lib().flux_qkv_projection(_strided(a, "bf16", "a"), m, k, a.stride(0), _bits(w, "w"),
                                      _bits(bias, "bias"), heads, _bits(q_gain, "q_gain"), _bits(k_gain, "k_gain"),
                                      _ptr(table, torch.float32, "table"), table_row0, float(eps), _bits(qkv, "qkv"),
                                      _stream(stream)))
@@ -556,6 +722,9 @@ def flux_qkv_projection(a, w, bias, heads, q_gain, k_gain, table, qkv, table_row
 def flux_layernorm_modulate(x, y, shift, scale, eps=1e-6, stream=None):
     import torch
     rows, dim = x.shape
+    _need_same(y, x, "y")
+    _need_numel(shift, dim, "shift")
+    _need_numel(scale, dim, "scale")
     _check(lib().flux_layernorm_modulate(_ptr(x, torch.float32, "x"), _bits(y, "y"), rows, dim,
                                          _ptr(shift, torch.float32, "shift"), _ptr(scale, torch.float32, "scale"),
                                          float(eps), _stream(stream)))
@@ -564,6 +733,7 @@ def flux_layernorm_modulate(x, y, shift, scale, eps=1e-6, stream=None):
 
 def flux_rope_table(table, n_txt, grid_hw, ref_hw=(0, 0), theta=1e4, stream=None):
     import torch
+    _need_numel(table, (n_txt + grid_hw[0] * grid_hw[1] + ref_hw[0] * ref_hw[1]) * 128, "table")
     _check(lib().flux_rope_table(_ptr(table, torch.float32, "table"), n_txt, grid_hw[0], grid_hw[1], ref_hw[0],
                                  ref_hw[1], float(theta), _stream(stream)))
     return table
@@ -572,6 +742,11 @@ def flux_rope_table(table, n_txt, grid_hw, ref_hw=(0, 0), theta=1e4, stream=None
 def flux_qk_rmsnorm_rope(qkv, k_col, heads, q_gain, k_gain, table, eps=1e-6, stream=None):
     import torch
     rows, ld = qkv.shape
+    if heads * 128 > ld or k_col < 0 or k_col + heads * 128 > ld:
+        raise FluxShapeError("q and k heads must lie inside the row")
+    _need_numel(q_gain, 128, "q_gain")
+    _need_numel(k_gain, 128, "k_gain")
+    _need_numel(table, rows * 128, "table")
     _check(lib().flux_qk_rmsnorm_rope(_bits(qkv, "qkv"), rows, ld, k_col, heads, _bits(q_gain, "q_gain"),
                                       _bits(k_gain, "k_gain"), _ptr(table, torch.float32, "table"), float(eps),
                                       _stream(stream)))
