@@ -41,8 +41,9 @@ def _device_clean():
 
 
 # ---------------------------------------------------------------------------- pack / unpack / Euler
-@pytest.mark.parametrize("h8,w8", [(8, 8), (128, 128), (6, 10), (2, 2), (64, 32)])
+@pytest.mark.parametrize("h8,w8", [(8, 8), (128, 128), (6, 10), (2, 2), (64, 32), (4, 66), (2, 130)])
 def test_pack_unpack_bit_exact(h8, w8):
+    """Pack tiles hold 32 tokens of one token row: 33 and 65 tokens per row leave a ragged tile."""
     lat = rand((32, h8, w8), h8 * 100 + w8)
     tok = torch.empty((h8 // 2) * (w8 // 2), 128, device=DEV)
     F.flux_pack_latents(lat.to(DEV), tok)
