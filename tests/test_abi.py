@@ -193,3 +193,35 @@ def test_flux3_entry_points_reject_bad_arguments(L):
     assert L.flux3_dit_set_active_blocks(None, 1, 1) == F.FLUX_EINVAL
     assert L.flux3_dit_modulation_size(None) == 0
     L.flux3_dit_destroy(None)
+
+
+@pytest.mark.parametrize("rows,k", [(1, 64), (128, 64), (129, 3072), (4608, 12288), (0, 256), (300, 16384)])
+def test_nvfp4_scale_bytes_is_whole_128_row_blocks(L, rows, k):
+    """One 512-byte tile per 128 rows (rounded up) and 64 elements of the row."""
+    assert F.flux_nvfp4_scale_bytes(rows, k) == -(-rows // 128) * (k // 64) * 512
+
+
+def test_nvfp4_scale_bytes_rejects_bad_sizes(L):
+    for rows, k in ((10, 32), (10, 100), (-1, 64), (10, 0)):
+        assert F.flux_nvfp4_scale_bytes(rows, k) == 0
+
+
+def test_low_precision_entry_points_reject_bad_arguments(L):
+    """Shape, mode and alignment checks of the FP8 and NVFP4 entry points fail before any launch."""
+    p, p8 = ctypes.c_void_p(16), ctypes.c_void_p(24)
+    E = F.FLUX_EINVAL
+    assert L.flux_quantize_rows_e4m3(p, 4, 12, 16, p, 16, p, None) == E                  # cols % 8
+    assert L.flux_quantize_rows_e4m3(p, 4, 16, 8, p, 16, p, None) == E                   # ldx < cols
+    assert L.flux_quantize_rows_e4m3(p8, 4, 16, 16, p, 16, p, None) == E                 # x 8-byte aligned
+    assert L.flux_layernorm_modulate_fp8(p, p, p, 4, 3000, p, p, 1e-6, None) == E
+    assert L.flux_linear_fp8(p, p, 4, 64, 64, p, p, 32, p, 1, p, 32, None, None) == E     # k % 128
+    assert L.flux_linear_fp8(p, p, 4, 128, 128, p, p, 32, p, 3, p, 32, None, None) == E   # gate missing
+    assert L.flux_linear_fp8(p, p, 4, 128, 128, p, p, 64, p, 2, p, 32, None, None) == E   # SwiGLU n % 256
+    assert L.flux_quantize_rows_nvfp4(p, 4, 96, 96, p, 48, p, p, None) == E              # k % 64
+    assert L.flux_quantize_rows_nvfp4(p, 4, 16448, 16448, p, 8224, p, p, None) == E      # k > 16384
+    assert L.flux_quantize_rows_nvfp4(p, 4, 128, 128, p, 72, p, p, None) == E            # ldq % 16
+    assert L.flux_layernorm_modulate_nvfp4(p, p, p, p, 4, 1536, p, p, 1e-6, None) == E
+    assert "dim" in F.get_error()
+    assert L.flux_linear_nvfp4(p, p, p, 4, 128, 64, p, p, p, 32, p, 1, p, 32, None, None) == E    # k % 256
+    assert L.flux_linear_nvfp4(p, p, p, 4, 256, 128, p, p, p, 32, p, 4, p, 32, None, None) == E   # mode
+    assert L.flux_linear_nvfp4(p8, p, p, 4, 256, 128, p, p, p, 32, p, 1, p, 32, None, None) == E  # alignment
