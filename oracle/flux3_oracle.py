@@ -24,7 +24,7 @@ Systemanforderungen im Überblick" (mindverse), sections
 "FLUX.3 Image Klein: offene Gewichte ..." (kimiseek): the distilled checkpoint samples 16
 steps without guidance.  we0.ai FLUX 3 Image Klein article: 5.6 B generator parameters.
 
-Readings where the page is silent (each is listed in the design doc):
+Readings where the page is silent:
 * modulation linears are shared by the blocks of a phase: one Linear(3072 -> 3*3072) per
   stream for the per-mode blocks, one for the joint blocks, Linear(3072 -> 2*3072) for the
   output layer.  With per-block linears the model would have 6.7 B parameters; shared, it

@@ -26,7 +26,7 @@ Sources (web pages, by title and section):
   from the timestep embedding, one timestep for all tokens in FLUX.2, 4-axis
   RoPE with 32 dims per axis and its coordinate table).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 * timestep embedding: 256 dims, t scaled by 1000, max period 1e4, [cos, sin];
   MLP 256 -> 3072 -> 3072 with SiLU between.
 * modulation: one Linear(3072 -> k*3072) per block and stream applied to

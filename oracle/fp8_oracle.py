@@ -9,7 +9,7 @@ Inferenzlatenz": the transformer ships as fp8r, row-wise FP8, with fast kernels 
 capability 8.9 on (Blackwell included); the we0.ai FLUX 3 Image Klein article lists 11.2 GB of
 generator weights in BF16 and 5.6 GB in FP8 (one byte per weight).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 * the format is e4m3 ("fn": no infinities, largest finite 448), round to nearest even,
   saturating at +-448;
 * row-wise means one fp32 scale per row of every operand: per output row of a weight matrix and

@@ -11,7 +11,7 @@ values (1 sign, 2 exponent bits with bias 1, 1 mantissa bit: magnitudes 0, 0.5, 
 4, 6), one e4m3 scale per block of 16 consecutive elements along the reduction dimension, and
 a second-level fp32 scale.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 * the second-level scale is per row (per output row of a weight matrix and per token row of an
   activation), like the row-wise FP8 format, instead of per tensor;
 * quantisation of one row x (all values rounded to float32 as below):
