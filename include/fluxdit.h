@@ -189,6 +189,13 @@ FLUX_API int flux_euler_step(float *x, const float *v, size_t n, float dt, void 
 FLUX_API int flux_cfg_euler_step(float *x, const float *v_cond, const float *v_uncond, size_t n, float guidance,
                                  float dt, void *stream);
 
+/* flux_cfg_euler_step that also writes the guided velocity v_uncond + guidance * (v_cond - v_uncond)
+ * to v_guided (fp32, n values, a distinct 16-byte aligned device buffer, caller-owned), the same
+ * values the update adds to x, for a sampler that reports each step's velocity.  Errors as
+ * flux_cfg_euler_step; a NULL v_guided is FLUX_EINVAL. */
+FLUX_API int flux_cfg_euler_step_out(float *x, const float *v_cond, const float *v_uncond, float *v_guided,
+                                     size_t n, float guidance, float dt, void *stream);
+
 /* img2img start state: out = (1 - t) x + t noise over n fp32 values (x the latent of the
  * image to edit, noise N(0,1)): the flow-matching state at time t.  With strength s the
  * sampler starts at the first of the last floor(S*s) schedule times; s = 0 keeps the image
@@ -281,9 +288,9 @@ FLUX_API size_t flux_nvfp4_scale_bytes(int rows, int k);
 FLUX_API int flux_quantize_rows_nvfp4(const uint16_t *x, int rows, int k, int ldx, uint8_t *q, int ldq, uint8_t *sf,
                                       float *row_scale, void *stream);
 
-/* flux_layernorm_modulate with its output rounded to bf16 and quantised to NVFP4 in the same pass
- * (codes [rows, dim/2], block scales and row scales as flux_quantize_rows_nvfp4).  dim in
- * {1024, 2048, 3072, 4096}. */
+/* flux_layernorm_modulate with its output quantised to NVFP4 in the same pass (codes [rows, dim/2],
+ * block scales and row scales as flux_quantize_rows_nvfp4; the modulated values are quantised from
+ * float32).  dim in {1024, 2048, 3072, 4096}. */
 FLUX_API int flux_layernorm_modulate_nvfp4(const float *x, uint8_t *q, uint8_t *sf, float *row_scale, int rows,
                                            int dim, const float *shift, const float *scale, float eps,
                                            void *stream);
@@ -338,9 +345,10 @@ FLUX_API unsigned long long flux_kernel_launches(void);
  * Limits: hidden <= 8192 and t_freq_dim <= 1024, both multiples of 8; larger
  * sizes return FLUX_EINVAL.  The intermediates live in one 68 KiB device array
  * inside the library, which every GPU that loads the library holds until the
- * process exits.  The first call on a device looks up that array's address
- * (cudaGetSymbolAddress) with the device current; make that first call before
- * any stream capture.  All calls on a device share the array: calls whose
+ * process exits.  The first call in a CUDA context (normally a device's primary
+ * context) looks up that array's address (cudaGetSymbolAddress) with the device
+ * current and keeps it for that context; make that first call before any stream
+ * capture.  All calls on a device share the array: calls whose
  * kernels overlap on the GPU (different streams without ordering) race.  Each
  * call writes every scratch element before reading it, so nothing is cleared. */
 FLUX_API int flux_timestep_modulation_noalloc(const uint16_t *w1, const uint16_t *b1, const uint16_t *w2,
@@ -453,8 +461,26 @@ FLUX_API int flux_joint_attention_segments(const uint16_t *q, const uint16_t *k,
                                            void *stream);
 
 /* Synchronise `stream`, then read and clear the kernels' device error words:
- * 0 when no kernel gave up waiting, else the first nonzero code. */
+ * 0 when no kernel gave up waiting, else the first nonzero code (FLUX_DEVERR_*). */
 FLUX_API int flux_device_error(void *stream);
+
+/* Device error codes: which role of a kernel gave up waiting. */
+#define FLUX_DEVERR_TIMEOUT_PRODUCER 1 /* a TMA producer waited for a free stage */
+#define FLUX_DEVERR_TIMEOUT_MMA 2      /* the MMA issuer waited for operands or an empty accumulator */
+#define FLUX_DEVERR_TIMEOUT_EPILOGUE 3 /* the epilogue waited for a finished accumulator */
+#define FLUX_DEVERR_TIMEOUT_SOFTMAX 4  /* an attention softmax warpgroup waited for scores */
+#define FLUX_DEVERR_BAD_LAUNCH 5       /* a kernel found its launch shape inconsistent */
+#define FLUX_DEVERR_TIMEOUT_SELFTEST 6 /* flux_selftest_bounded_wait gave up, as asked */
+
+/* Check of the error path above, with no kernel stalled for real (hakusoku.com story 4662,
+ * "エラーハンドリング": failures surface as a status code and a message).  Launches one CTA
+ * that waits on a shared-memory mbarrier through the bounded wait every pipeline uses.  With
+ * arrive = 1 the CTA first arrives on the barrier, so the wait succeeds at once and nothing is
+ * recorded.  With arrive = 0 nothing ever arrives: the wait gives up after limit_ns nanoseconds
+ * (0 < limit_ns <= 1e9, else FLUX_EINVAL), the kernel records FLUX_DEVERR_TIMEOUT_SELFTEST in its
+ * device error word and returns normally, leaving the context usable; flux_device_error() then
+ * reports and clears it.  Asynchronous on `stream`; no memory arguments. */
+FLUX_API int flux_selftest_bounded_wait(unsigned long long limit_ns, int arrive, void *stream);
 
 #ifdef __cplusplus
 }

@@ -147,8 +147,7 @@ __global__ void __launch_bounds__(kQ4Threads) quantize_nvfp4_kernel(const __nv_b
 }
 
 // LayerNorm + modulation of one row per CTA (dim = 1024 VPT: VPT float4 per thread), the modulated
-// row rounded to bf16 (the block linears' input precision) and quantised to NVFP4 as above; row r
-// uses the modulation set that `ms` gives it.
+// float32 row quantised to NVFP4 as above; row r uses the modulation set that `ms` gives it.
 template <int VPT>
 __global__ void __launch_bounds__(kQ4Threads) ln_mod_nvfp4_kernel(const float* __restrict__ x,
                                                                   uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
@@ -181,10 +180,10 @@ __global__ void __launch_bounds__(kQ4Threads) ln_mod_nvfp4_kernel(const float* _
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const float4 a = __ldg(sh + i * kQ4Threads), c = __ldg(sc + i * kQ4Threads);
-    v[i].x = __bfloat162float(__float2bfloat16_rn((v[i].x - mean) * rstd * (1.f + c.x) + a.x));
-    v[i].y = __bfloat162float(__float2bfloat16_rn((v[i].y - mean) * rstd * (1.f + c.y) + a.y));
-    v[i].z = __bfloat162float(__float2bfloat16_rn((v[i].z - mean) * rstd * (1.f + c.z) + a.z));
-    v[i].w = __bfloat162float(__float2bfloat16_rn((v[i].w - mean) * rstd * (1.f + c.w) + a.w));
+    v[i].x = (v[i].x - mean) * rstd * (1.f + c.x) + a.x;
+    v[i].y = (v[i].y - mean) * rstd * (1.f + c.y) + a.y;
+    v[i].z = (v[i].z - mean) * rstd * (1.f + c.z) + a.z;
+    v[i].w = (v[i].w - mean) * rstd * (1.f + c.w) + a.w;
     amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
   }
   float inv, S;

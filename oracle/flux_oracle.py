@@ -224,12 +224,7 @@ def block_linear(hp):
         return linear_fp8
     if hp.get("nvfp4"):
         from .nvfp4_oracle import linear_nvfp4
-
-        def lin4(x, w, b):
-            # a quantised code is an integer decision, taken in the precision the GPU path
-            # quantises from: its block inputs are bf16 activations
-            return linear_nvfp4(torch.as_tensor(x).to(torch.bfloat16).to(torch.as_tensor(x).dtype), w, b)
-        return lin4
+        return linear_nvfp4
     return linear
 
 

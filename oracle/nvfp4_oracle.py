@@ -23,9 +23,9 @@ Readings where the pages are silent:
       value_j = code_j * s_b * S;
   an all-zero row, or a block whose scale rounds to 0, has codes 0;
 * y = sum over blocks of (codes_x . codes_w) s_bx s_bw, times S_x S_w, plus the bias;
-* it applies where the row-wise FP8 format does: the linears inside the transformer blocks, whose
-  activations enter the quantiser as bf16 (``flux_oracle.block_linear`` rounds them first: a code
-  is an integer decision, taken in the precision the GPU path quantises from).
+* it applies where the row-wise FP8 format does: the linears inside the transformer blocks; an
+  activation row is quantised from the values the layer receives (the format defines no other
+  rounding before the quantiser), its scale and code decisions taken in float32 as above.
 """
 from __future__ import annotations
 

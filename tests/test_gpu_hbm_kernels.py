@@ -199,8 +199,8 @@ def test_quantize_rows_nvfp4_larger_than_l2():
 
 
 def test_layernorm_modulate_nvfp4_larger_than_l2():
-    """Same allowance as at small sizes: the float32 and float64 LayerNorms may round an element
-    to neighbouring bf16 values, which can move its code by one e2m1 step."""
+    """Same allowance as at small sizes: the float32 and float64 LayerNorms may land on opposite
+    sides of a rounding boundary, which moves that element's code by one e2m1 step (rare)."""
     x, shift, scale = _ln_inputs(360)
     q = torch.empty(ROWS, 1536, dtype=torch.uint8, device=DEV)
     sf = torch.zeros(F.flux_nvfp4_scale_bytes(ROWS, 3072), dtype=torch.uint8, device=DEV)
@@ -209,13 +209,13 @@ def test_layernorm_modulate_nvfp4_larger_than_l2():
     for blk in _nvfp4_blocks(ROWS):
         r0, r1 = 128 * blk, min(128 * blk + 128, ROWS)
         y = _ln_ref(x, shift, scale, torch.arange(r0, r1))
-        qc, qsb, qs = Q4.quantize_rows_nvfp4(y.to(torch.bfloat16).float())
+        qc, qsb, qs = Q4.quantize_rows_nvfp4(y)
         got_s = s.cpu()[r0:r1]
-        assert torch.allclose(got_s.double(), qs.double(), rtol=2 ** -7, atol=0)
+        assert torch.allclose(got_s.double(), qs.double(), rtol=1e-5, atol=0)
         sb = _sf_block(sf, blk, 3072)[:r1 - r0]
-        assert (sb != qsb).double().mean() < 1e-3
+        assert (sb != qsb).double().mean() < 1e-4
         codes = _codes(q[r0:r1])
-        same = (sb == qsb).repeat_interleave(16, dim=1) & (got_s == qs)[:, None]
+        same = (sb == qsb).repeat_interleave(16, dim=1)
         diff = (codes != qc) & same
-        assert diff.double().mean() < 2e-3
+        assert diff.double().mean() < 1e-4
         assert ((codes - qc).abs()[diff] <= 2.0).all()

@@ -19,11 +19,16 @@ pytestmark = pytest.mark.gpu
 torch.set_grad_enabled(False)
 DEV = "cuda"
 TOL = 1e-2
-# NVFP4 forward against the NVFP4 oracle.  An e2m1 step is 1/4 to 1/2 of the value (e4m3: 1/16 to
-# 1/8), so where the GPU's bf16 intermediates differ from the oracle's float64 ones by an ulp, a
-# code flips with a proportionally larger jump than in FP8 (bar 2e-2); measured 1.5 to 2.2 % on the
-# tiny models, against a format error of 4.3 to 4.7 % (NVFP4 oracle vs exact oracle).
+# NVFP4 forward against the NVFP4 oracle.  The NVFP4 forward is not continuous in its quantiser
+# inputs: a value that crosses a rounding boundary moves by a whole e2m1 step (1/4 to 1/2 of it).
+# On the CPU the oracle alone moves by sigma = 2-3 % when every quantiser input is perturbed by one
+# bf16 rounding, and sits eps = 3.5-6 % from the exact forward (tests/test_oracle_nvfp4_pins.py).
+# The GPU path's attention runs on bf16 operands, so its quantiser inputs carry at least that
+# perturbation and the bf16 path's 2e-2 is below this format's noise floor.  The bar is 3e-2, the
+# top of the pinned sigma range and below the smallest eps (a path that did not quantise fails it),
+# and the GPU must sit nearer the NVFP4 oracle than the exact forward by NV4_RATIO.
 NV4_V_TOL = 3e-2
+NV4_RATIO = 0.6
 
 
 def nmax(gpu, ref):
@@ -112,10 +117,11 @@ def test_quantize_rows_nvfp4_bit_exact_against_oracle(rows, k):
 
 @pytest.mark.parametrize("rows,dim", [(4608 + 5, 3072), (33, 3072), (70, 1024), (40, 2048), (37, 4096)])
 def test_layernorm_modulate_nvfp4_against_oracle(rows, dim):
-    """LN-mod rounded to bf16 and quantised in one pass: the codes, block scales and row scales of
-    the oracle's quantisation of the same bf16 row, except where the two LayerNorm evaluations
-    (float32 here, float64 there) round an element to neighbouring bf16 values, which may move the
-    element's code by one step (or a block scale by one e4m3 step when it moves the block maximum)."""
+    """LN-mod quantised to NVFP4 in one pass, from the float32 modulated values: the codes, block
+    scales and row scales of the oracle's quantisation of the same row, except where the two LayerNorm
+    evaluations (float32 here, float64 there) land on opposite sides of a rounding boundary, which
+    moves one code by one e2m1 step (or a block scale by one e4m3 step); that needs a value within a
+    few float32 ulps of the boundary, so it is rare."""
     x = rand((rows, dim), 150) * 3 + 0.5
     shift, scale = rand((dim,), 151), rand((dim,), 152, 0.5)
     q = torch.empty(rows, dim // 2, dtype=torch.uint8, device=DEV)
@@ -123,14 +129,14 @@ def test_layernorm_modulate_nvfp4_against_oracle(rows, dim):
     s = torch.empty(rows, dtype=torch.float32, device=DEV)
     F.flux_layernorm_modulate_nvfp4(x.to(DEV), q, sf, s, shift.to(DEV), scale.to(DEV))
     y = O.modulate(O.layer_norm(x.double(), 1e-6), shift.double(), scale.double())
-    qc, qsb, qs = Q4.quantize_rows_nvfp4(y.to(torch.bfloat16).float())
-    assert torch.allclose(s.cpu().double(), qs.double(), rtol=2 ** -7, atol=0)
+    qc, qsb, qs = Q4.quantize_rows_nvfp4(y)
+    assert torch.allclose(s.cpu().double(), qs.double(), rtol=1e-5, atol=0)
     sb = decode_sf(sf, rows, dim)
-    assert (sb != qsb).double().mean() < 1e-3
+    assert (sb != qsb).double().mean() < 1e-4
     codes = decode_codes(q)
-    same_blocks = (sb == qsb).repeat_interleave(16, dim=1) & (s.cpu() == qs)[:, None]
+    same_blocks = (sb == qsb).repeat_interleave(16, dim=1)
     diff = (codes != qc) & same_blocks
-    assert diff.double().mean() < 2e-3
+    assert diff.double().mean() < 1e-4
     steps = (codes - qc).abs()[diff]
     assert (steps <= 2.0).all()                             # neighbouring e2m1 values (spacing <= 2)
 
@@ -255,7 +261,7 @@ def test_tiny_nvfp4_forward_against_nvfp4_oracle(tiny, n_txt, grid, refs):
     print(f"nvfp4 forward vs nvfp4 oracle {err:.4f}, vs exact oracle {rel_l2(v, exact):.4f}, "
           f"nvfp4 oracle vs exact {rel_l2(want, exact):.4f}")
     assert err <= NV4_V_TOL, err
-    assert err < 0.6 * rel_l2(v, exact)                     # it quantises the way the oracle does
+    assert err < NV4_RATIO * rel_l2(v, exact)               # it quantises the way the oracle does
     assert rel_l2(v, exact) > rel_l2(v16, exact)
     again = torch.empty_like(v)
     model.forward(tok.to(DEV), grid, txt.to(DEV) if n_txt else None, 0.6, again, rt, hw)
@@ -357,7 +363,9 @@ def test_tiny_nvfp4_sampler_against_nvfp4_oracle(tiny):
         model.set_precision(F.PRECISION_BF16)
     assert len(vs) == 2
     for a, b in zip(vs, ref_vs):
+        print(f"nvfp4 sampler step velocity vs nvfp4 oracle {rel_l2(a, b):.4f}")
         assert rel_l2(a, b) <= NV4_V_TOL
+    print(f"nvfp4 sampler final latent vs nvfp4 oracle {rel_l2(final.cpu(), ref_final):.4f}")
     assert rel_l2(final.cpu(), ref_final) <= NV4_V_TOL
 
 

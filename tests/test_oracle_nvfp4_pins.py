@@ -114,3 +114,44 @@ def test_block_scale_is_the_e4m3_of_the_scaled_block_maximum():
     assert sb[0].tolist() == [448.0, 112.0, 28.0]
     assert q[0, 0] == 6.0 and q[0, 16] == 6.0 and q[0, 32] == -6.0
     assert [e for e in itertools.islice(q[0].tolist(), 1, 16)] == [0.0] * 15
+
+
+def test_nvfp4_forward_error_and_its_sensitivity_to_bf16_sized_perturbations(monkeypatch):
+    """Two properties of the NVFP4 forward itself (oracle only, tiny 1 + 1 block workload), which
+    fix the tolerance of the GPU's NVFP4 forward:
+
+    * eps: the NVFP4 forward is 3.5-6 % (rel-L2) from the exact forward (the format's own error);
+    * sigma: perturbing every quantiser input by at most one bf16 rounding (relative 2^-9, seeded
+      uniform) moves the NVFP4 forward by 2-3 %, more than the bf16 path's 2e-2 bar.  A code
+      sits on one side of a rounding boundary; an input that crosses it moves the value by a whole
+      e2m1 step (1/4 to 1/2 of the value), so the forward is not continuous in its quantiser inputs,
+      and any path whose attention runs on bf16 operands carries at least this perturbation.
+    Also sigma < 0.7 eps: a forward that did not quantise at all would sit eps away, well outside a
+    bar set from sigma."""
+    from oracle import flux_oracle as O
+    from synthetic import WORKLOADS, make_weights
+    torch.set_grad_enabled(False)
+    w = WORKLOADS["tiny64"]
+    _, p = make_weights(w.dims, w.seed)
+    g = torch.Generator().manual_seed(196)
+    tok = torch.randn(16, 128, generator=g).to(torch.bfloat16).float()
+    txt = torch.randn(16, 3072, generator=g).to(torch.bfloat16).float()
+    exact = O.forward(p, O.hyper(w.dims), tok, txt, 0.6, (4, 4))
+    hq = dict(O.hyper(w.dims), nvfp4=True)
+    pure = O.forward(p, hq, tok, txt, 0.6, (4, 4))
+    plain = Q4.linear_nvfp4
+    gp = torch.Generator().manual_seed(0)
+
+    def perturbed(x, wt, b):
+        x = torch.as_tensor(x)
+        u = torch.rand(x.shape, generator=gp, dtype=torch.float64) * 2 - 1
+        return plain(x * (1 + u * 2.0 ** -9).to(x.dtype), wt, b)
+    monkeypatch.setattr(Q4, "linear_nvfp4", perturbed)
+    pert = O.forward(p, hq, tok, txt, 0.6, (4, 4))
+
+    def rel(a, b):
+        return ((a - b).norm() / b.norm()).item()
+    eps, sigma = rel(pure, exact), rel(pert, pure)
+    assert 0.035 <= eps <= 0.06, eps
+    assert 0.02 <= sigma <= 0.03, sigma
+    assert sigma < 0.7 * eps, (sigma, eps)
