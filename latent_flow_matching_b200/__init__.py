@@ -67,6 +67,8 @@ _SIGS = {
     "flux_dit_forward_cfg": (_I, [_P, _P, _I, _I, _P, _P, _I, _P, _I, ctypes.POINTER(ctypes.c_int), _F, _P, _P,
                                   _P]),
     "flux_cfg_euler_step": (_I, [_P, _P, _P, _Z, _F, _F, _P]),
+    "flux_cfg_euler_step_out": (_I, [_P, _P, _P, _P, _Z, _F, _F, _P]),
+    "flux_selftest_bounded_wait": (_I, [ctypes.c_ulonglong, _I, _P]),
     "flux_blend_latents": (_I, [_P, _P, _F, _P, _Z, _P]),
     "flux_dit_set_active_blocks": (_I, [_P, _I, _I]),
     "flux_dit_modulation_size": (_Z, [_P]),
@@ -482,14 +484,22 @@ def flux_euler_step(x, v, dt, stream=None):
     return x
 
 
-def flux_cfg_euler_step(x, v_cond, v_uncond, guidance, dt, stream=None):
-    """x += dt * (v_uncond + guidance * (v_cond - v_uncond)), in place."""
+def flux_cfg_euler_step(x, v_cond, v_uncond, guidance, dt, stream=None, v_guided=None):
+    """x += dt * (v_uncond + guidance * (v_cond - v_uncond)), in place; with ``v_guided`` (a tensor
+    like x) the kernel also writes the guided velocity there."""
     import torch
     _need_same(v_cond, x, "v_cond")
     _need_same(v_uncond, x, "v_uncond")
-    _check(lib().flux_cfg_euler_step(_ptr(x, torch.float32, "x"), _ptr(v_cond, torch.float32, "v_cond"),
-                                     _ptr(v_uncond, torch.float32, "v_uncond"), x.numel(), float(guidance),
-                                     float(dt), _stream(stream)))
+    if v_guided is None:
+        _check(lib().flux_cfg_euler_step(_ptr(x, torch.float32, "x"), _ptr(v_cond, torch.float32, "v_cond"),
+                                         _ptr(v_uncond, torch.float32, "v_uncond"), x.numel(), float(guidance),
+                                         float(dt), _stream(stream)))
+        return x
+    _need_same(v_guided, x, "v_guided")
+    _check(lib().flux_cfg_euler_step_out(_ptr(x, torch.float32, "x"), _ptr(v_cond, torch.float32, "v_cond"),
+                                         _ptr(v_uncond, torch.float32, "v_uncond"),
+                                         _ptr(v_guided, torch.float32, "v_guided"), x.numel(), float(guidance),
+                                         float(dt), _stream(stream)))
     return x
 
 
@@ -772,6 +782,15 @@ def flux_device_error(stream=None) -> int:
     return lib().flux_device_error(_stream(stream))
 
 
+DEVERR_TIMEOUT_SELFTEST = 6
+
+
+def flux_selftest_bounded_wait(limit_ns: int, arrive: bool, stream=None):
+    """One CTA waits on an mbarrier through the pipelines' bounded wait; with arrive=False nothing
+    arrives and the kernel gives up after limit_ns, recording DEVERR_TIMEOUT_SELFTEST."""
+    _check(lib().flux_selftest_bounded_wait(int(limit_ns), 1 if arrive else 0, _stream(stream)))
+
+
 def flux_sample(model: FluxDiT, latent, txt, n_steps, ref_latent=None, on_step=None, stream=None,
                 init_latent=None, strength=1.0, txt_uncond=None, guidance=None):
     """Euler sampling on the device: pack -> S x (forward, Euler) -> unpack.
@@ -812,11 +831,12 @@ def flux_sample(model: FluxDiT, latent, txt, n_steps, ref_latent=None, on_step=N
             raise ValueError("guidance needs txt_uncond")
         v_u = torch.empty_like(tok)
         hw_list = ref_hw if (ref_hw and isinstance(ref_hw[0], (tuple, list))) else ([ref_hw] if ref_hw[0] else [])
+        v_g = torch.empty_like(tok) if on_step is not None else None
         for i in range(start, n_steps):
             model.forward_cfg(tok, (gh, gw), txt, txt_uncond, ts[i], v, v_u, ref_tok, hw_list, stream)
+            flux_cfg_euler_step(tok, v, v_u, guidance, ts[i + 1] - ts[i], stream, v_guided=v_g)
             if on_step is not None:
-                on_step(i, v_u + guidance * (v - v_u))
-            flux_cfg_euler_step(tok, v, v_u, guidance, ts[i + 1] - ts[i], stream)
+                on_step(i, v_g)
         out = torch.empty_like(latent)
         flux_unpack_latents(tok, out, stream)
         return out
@@ -865,12 +885,13 @@ def flux3_sample(model: Flux3DiT, latent, txt, n_steps, ref_latent=None, on_step
         if txt_uncond is None:
             raise ValueError("guidance needs txt_uncond")
         v_u = torch.empty_like(tok)
+        v_g = torch.empty_like(tok) if on_step is not None else None
         for i in range(start, n_steps):
             model.forward_cfg(tok, (gh, gw), txt, txt_uncond, ts[i], v, v_u, ref_tok, grids, t_target=ts[i + 1],
                               stream=stream)
+            flux_cfg_euler_step(tok, v, v_u, guidance, ts[i + 1] - ts[i], stream, v_guided=v_g)
             if on_step is not None:
-                on_step(i, v_u + guidance * (v - v_u))
-            flux_cfg_euler_step(tok, v, v_u, guidance, ts[i + 1] - ts[i], stream)
+                on_step(i, v_g)
     else:
         for i in range(start, n_steps):
             model.forward(tok, (gh, gw), txt, ts[i], v, ref_tok, grids, t_target=ts[i + 1], stream=stream)

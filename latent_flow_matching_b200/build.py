@@ -8,7 +8,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = ["fluxdit.cu", "fluxdit3.cu", "gemm_tc.cu", "gemm_tc2.cu", "gemm_fp4.cu", "attention_tc.cu", "elementwise.cu", "fp8.cu",
-           "nvfp4.cu", "noalloc.cu"]
+           "nvfp4.cu", "noalloc.cu", "selftest.cu"]
 LIB = os.path.join(HERE, "libfluxdit.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -24,6 +24,7 @@ enum DeviceError : int {
   kErrTimeoutEpilogue = 3,
   kErrTimeoutSoftmax = 4,
   kErrBadLaunch = 5,
+  kErrTimeoutSelftest = 6,
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -63,20 +64,27 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Returns false if
-// the CTA abort flag is (or becomes) set or the wait exceeds kWaitTimeoutNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// the CTA abort flag is (or becomes) set or the wait exceeds limit_ns, in which
+// case it raises the abort flag itself.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                uint64_t limit_ns) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_test(bar, parity)) return true;
     if ((it & 15u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         return false;
       }
     }
   }
+}
+
+// The pipelines' wait: bounded by kWaitTimeoutNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return mbar_wait_limit(bar, parity, abort_flag, kWaitTimeoutNs);
 }
 
 // Bounded wait used while draining after an abort (ignores the abort flag).

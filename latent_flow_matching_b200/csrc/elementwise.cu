@@ -285,21 +285,27 @@ __global__ void rope_table_kernel(float2* __restrict__ table, int n_txt, int gh,
 // (1 - t) x + t noise: the flow-matching state at time t between data (t = 0) and noise (t = 1)
 // x += dt * (v_u + g (v_c - v_u)): the guided velocity and the Euler step in one pass.
 __global__ void cfg_euler_kernel(float* __restrict__ x, const float* __restrict__ vc, const float* __restrict__ vu,
-                                 size_t n, float g, float dt) {
+                                 float* __restrict__ vg, size_t n, float g, float dt) {
   const size_t n4 = n / 4;
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4; i += stride) {
     float4 a = reinterpret_cast<float4*>(x)[i];
     const float4 c = reinterpret_cast<const float4*>(vc)[i];
     const float4 u = reinterpret_cast<const float4*>(vu)[i];
-    a.x = fmaf(dt, fmaf(g, c.x - u.x, u.x), a.x);
-    a.y = fmaf(dt, fmaf(g, c.y - u.y, u.y), a.y);
-    a.z = fmaf(dt, fmaf(g, c.z - u.z, u.z), a.z);
-    a.w = fmaf(dt, fmaf(g, c.w - u.w, u.w), a.w);
+    const float4 v = make_float4(fmaf(g, c.x - u.x, u.x), fmaf(g, c.y - u.y, u.y), fmaf(g, c.z - u.z, u.z),
+                                 fmaf(g, c.w - u.w, u.w));
+    a.x = fmaf(dt, v.x, a.x);
+    a.y = fmaf(dt, v.y, a.y);
+    a.z = fmaf(dt, v.z, a.z);
+    a.w = fmaf(dt, v.w, a.w);
     reinterpret_cast<float4*>(x)[i] = a;
+    if (vg) reinterpret_cast<float4*>(vg)[i] = v;
   }
-  for (size_t i = n4 * 4 + blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n; i += stride)
-    x[i] = fmaf(dt, fmaf(g, vc[i] - vu[i], vu[i]), x[i]);
+  for (size_t i = n4 * 4 + blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n; i += stride) {
+    const float v = fmaf(g, vc[i] - vu[i], vu[i]);
+    x[i] = fmaf(dt, v, x[i]);
+    if (vg) vg[i] = v;
+  }
 }
 
 __global__ void blend_kernel(const float* __restrict__ x, const float* __restrict__ noise, float t,
@@ -411,11 +417,11 @@ cudaError_t euler_launch(float* x, const float* v, size_t n, float dt, cudaStrea
   return cudaGetLastError();
 }
 
-cudaError_t cfg_euler_launch(float* x, const float* vc, const float* vu, size_t n, float g, float dt,
+cudaError_t cfg_euler_launch(float* x, const float* vc, const float* vu, float* vg, size_t n, float g, float dt,
                              cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   count_launch();
-  cfg_euler_kernel<<<blocks_for((n + 3) / 4, 256), 256, 0, s>>>(x, vc, vu, n, g, dt);
+  cfg_euler_kernel<<<blocks_for((n + 3) / 4, 256), 256, 0, s>>>(x, vc, vu, vg, n, g, dt);
   return cudaGetLastError();
 }
 

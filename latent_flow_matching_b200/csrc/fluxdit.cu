@@ -152,8 +152,10 @@ struct BlobTensor {
 int device_error_words(cudaStream_t s) {
   const int g = gemm_read_device_error(s);
   const int g2 = gemm2_read_device_error(s);
+  const int g4 = gemm_fp4_read_device_error(s);
   const int a = attention_read_device_error(s);
-  return g ? g : (g2 ? g2 : a);
+  const int t = selftest_read_device_error(s);
+  return g ? g : (g2 ? g2 : (g4 ? g4 : (a ? a : t)));
 }
 
 static bool valid_cfg(const flux_dit_config& c) {
@@ -896,6 +898,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
   };
 
   for (int i = 0; i < m->act_double; ++i) {
+    const NvtxRange range("double block %d", i);
     const StreamW& si = m->dbl[2 * i];
     const StreamW& st = m->dbl[2 * i + 1];
     const float* mi = mods + si.mod_off;          // shift1, scale1, gate1, shift2, scale2, gate2
@@ -978,6 +981,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
   }
   // single blocks: one set of weights for every row, so the whole batch is one problem
   for (int i = 0; i < m->act_single; ++i) {
+    const NvtxRange range("single block %d", i);
     const SingleW& sw = m->sgl[i];
     const float* ms = mods + sw.mod_off;          // shift, scale, gate
     rc = ln_mod(n, ms, ms + D, ms, ms + D, w.seg_all);
@@ -1005,6 +1009,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
     FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear());
   }
   // output layer on the image rows of each sequence
+  const NvtxRange range("output layer");
   const float* mf = mods + m->fin_mod_off;         // shift, scale
   for (int b = 0; b < nb; ++b)
     FD_LAUNCH(m, kProfLnMod, 0, ln_bytes_img,
@@ -1090,7 +1095,17 @@ int flux_cfg_euler_step(float* x, const float* v_cond, const float* v_uncond, si
   if (!aligned16(x) || !aligned16(v_cond) || !aligned16(v_uncond))
     return fail(FLUX_EINVAL, "x, v_cond and v_uncond must be 16-byte aligned");
   if (!std::isfinite(guidance) || !std::isfinite(dt)) return fail(FLUX_EINVAL, "guidance and dt must be finite");
-  FD_CUDA(cfg_euler_launch(x, v_cond, v_uncond, n, guidance, dt, static_cast<cudaStream_t>(stream)));
+  FD_CUDA(cfg_euler_launch(x, v_cond, v_uncond, nullptr, n, guidance, dt, static_cast<cudaStream_t>(stream)));
+  return FLUX_OK;
+}
+
+int flux_cfg_euler_step_out(float* x, const float* v_cond, const float* v_uncond, float* v_guided, size_t n,
+                            float guidance, float dt, void* stream) {
+  if (n && (!x || !v_cond || !v_uncond || !v_guided)) return fail(FLUX_EINVAL, "NULL argument");
+  if (!aligned16(x) || !aligned16(v_cond) || !aligned16(v_uncond) || !aligned16(v_guided))
+    return fail(FLUX_EINVAL, "x, v_cond, v_uncond and v_guided must be 16-byte aligned");
+  if (!std::isfinite(guidance) || !std::isfinite(dt)) return fail(FLUX_EINVAL, "guidance and dt must be finite");
+  FD_CUDA(cfg_euler_launch(x, v_cond, v_uncond, v_guided, n, guidance, dt, static_cast<cudaStream_t>(stream)));
   return FLUX_OK;
 }
 

@@ -764,6 +764,7 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
   }
   const int mode_set[3] = {kModTxt, kModImg, kModRef};
   for (int i = 0; i < m->act_mode; ++i) {
+    const NvtxRange range("per-mode block %d", i);
     rc = ln3q(rows_pm, w.seg_pm, md(kModTxt), md(kModTxt + 1), md(kModImg), md(kModImg + 1), md(kModRef),
               md(kModRef + 1));
     if (rc) return rc;
@@ -820,6 +821,7 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
   A.n = n;
   A.batch = nb;
   for (int i = 0; i < m->act_joint; ++i) {
+    const NvtxRange range("joint block %d", i);
     const BlockW3& bw = m->joint[i];
     rc = ln3q(rows_all, w.seg_jy, md(kModJointCtx), md(kModJointCtx + 1), md(kModJointImg), md(kModJointImg + 1),
               md(kModJointCtx), md(kModJointCtx + 1));
@@ -858,6 +860,7 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
   }
 
   // ---------------- output layer on the image rows (text and reference tokens are dropped)
+  const NvtxRange range("output layer");
   P.num_problems = nb;
   for (int bb = 0; bb < nb; ++bb) {
     FD_LAUNCH(m, kProfLnMod, 0, 6.0 * ni * D + 8.0 * D,

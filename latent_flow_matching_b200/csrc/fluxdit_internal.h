@@ -73,8 +73,8 @@ int attention_read_device_error(cudaStream_t stream);
 cudaError_t pack_latents_launch(const float* lat, float* tok, int c, int h8, int w8, cudaStream_t s);
 cudaError_t unpack_latents_launch(const float* tok, float* lat, int c, int h8, int w8, cudaStream_t s);
 cudaError_t euler_launch(float* x, const float* v, size_t n, float dt, cudaStream_t s);
-// x += dt * (vu + g * (vc - vu)), element-wise
-cudaError_t cfg_euler_launch(float* x, const float* vc, const float* vu, size_t n, float g, float dt,
+// v = vu + g * (vc - vu) and x += dt * v, element-wise; v is also written to vg unless vg is null
+cudaError_t cfg_euler_launch(float* x, const float* vc, const float* vu, float* vg, size_t n, float g, float dt,
                              cudaStream_t s);
 cudaError_t cast_bf16_launch(const float* x, __nv_bfloat16* y, size_t n, cudaStream_t s);
 
@@ -187,6 +187,8 @@ int gemm_fp4_read_device_error(cudaStream_t stream);
 int record_error(int code, const char* msg);
 // Counts kernel launches enqueued by the library (reported by flux_kernel_launches).
 void count_launch();
+// the bounded-wait self-test kernel's device error word (read and cleared)
+int selftest_read_device_error(cudaStream_t stream);
 // 2D bf16 tensor map: rows x cols, row stride in bytes, box {64 cols, box_rows}, 128B swizzle.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
                     uint32_t box_rows);

@@ -5,6 +5,9 @@
 // synchronise the whole device).  The two hidden-size intermediates and the
 // embedding live in a fixed device array that is part of this library's image,
 // so a call allocates nothing.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <cmath>
 #include <mutex>
 
@@ -22,24 +25,67 @@ constexpr int kNoAllocFloats = kNoAllocMaxFreq + 2 * kNoAllocMaxHidden;   // 174
 // call reads was written earlier by the same call, so nothing needs clearing.
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocFloats];
 
-constexpr int kMaxDevices = 64;
+// The array's device address differs per CUDA context (each context loads its own copy of
+// the library's device image), so the address is looked up once per context and kept under
+// the context's process-unique ID: a context created later on the same device (after
+// cudaDeviceReset, or a caller-made context) gets a fresh lookup instead of a stale address.
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  float* ptr;
+};
+constexpr int kMaxContexts = 64;
 std::mutex g_noalloc_mutex;
-float* g_noalloc_ptr[kMaxDevices] = {};
+ScratchEntry g_noalloc_cache[kMaxContexts];
+int g_noalloc_entries = 0;
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
 
-// Device address of the scratch array for the current device (looked up once per device).
-int scratch_for_current_device(float** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return FLUX_EIO;
-  if (dev < 0 || dev >= kMaxDevices) return FLUX_EINVAL;
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p) return FLUX_EIO;
-    g_noalloc_ptr[dev] = static_cast<float*>(p);
+// ID of the calling thread's current context (0 if none is current yet).
+int current_context_id(unsigned long long* id) {
+  if (!g_ctx_current || !g_ctx_id) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess || !f1 ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess || !f2)
+      return FLUX_EIO;
+    g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f1);
+    g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f2);
   }
-  *out = g_noalloc_ptr[dev];
+  CUcontext ctx = nullptr;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS) return FLUX_EIO;
+  *id = 0;
+  if (ctx && g_ctx_id(ctx, id) != CUDA_SUCCESS) return FLUX_EIO;
+  return FLUX_OK;
+}
+
+// Device address of the scratch array in the current context (looked up once per context, with
+// the caller's device current).
+int scratch_for_current_context(float** out, const char** why) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  unsigned long long id = 0;
+  if (current_context_id(&id)) {
+    *why = "could not read the current CUDA context";
+    return FLUX_EIO;
+  }
+  for (int i = 0; id && i < g_noalloc_entries; ++i)
+    if (g_noalloc_cache[i].ctx_id == id) {
+      *out = g_noalloc_cache[i].ptr;
+      return FLUX_OK;
+    }
+  void* p = nullptr;
+  // With no context current yet this also makes the device's primary context current.
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || !p) {
+    *why = "cudaGetSymbolAddress of the no-allocation scratch failed";
+    return FLUX_EIO;
+  }
+  if (!id && current_context_id(&id)) {
+    *why = "could not read the current CUDA context";
+    return FLUX_EIO;
+  }
+  if (id && g_noalloc_entries < kMaxContexts) g_noalloc_cache[g_noalloc_entries++] = {id, static_cast<float*>(p)};
+  *out = static_cast<float*>(p);
   return FLUX_OK;
 }
 
@@ -64,8 +110,9 @@ extern "C" int flux_timestep_modulation_noalloc(const uint16_t* w1, const uint16
   if (!al16(w1) || !al16(w2) || !al16(wmod) || !al16(mods_out))
     return record_error(FLUX_EINVAL, "weight and output pointers must be 16-byte aligned");
   float* scratch = nullptr;
-  const int rc = scratch_for_current_device(&scratch);
-  if (rc) return record_error(rc, "cudaGetSymbolAddress of the no-allocation scratch failed");
+  const char* why = "";
+  const int rc = scratch_for_current_context(&scratch, &why);
+  if (rc) return record_error(rc, why);
   float* temb = scratch;
   float* h = scratch + kNoAllocMaxFreq;
   float* vec = h + kNoAllocMaxHidden;

@@ -6,6 +6,9 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <nvtx3/nvToolsExt.h>
+
+#include <cstdio>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -16,6 +19,21 @@
 namespace fdit {
 
 using bf16 = __nv_bfloat16;
+
+// A named NVTX range over one scope of host code (the launches of one transformer block, the
+// modulation, the input or output layers), so a profiler's timeline groups the kernels by block.
+// Without a profiler attached a push / pop is a check of one function pointer.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  NvtxRange(const char* fmt, int i) {
+    char buf[48];
+    snprintf(buf, sizeof(buf), fmt, i);
+    nvtxRangePushA(buf);
+  }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // printf-style flux_get_error() message for the calling thread; returns `code`.
 int fail(int code, const char* fmt, ...);

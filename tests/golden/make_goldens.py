@@ -10,6 +10,10 @@ step's velocity and the final packed latent:
 Row sets: all rows at 256^2, every 2nd at 512^2, every 8th at 1024^2.  For a guided workload
 the stored velocities are the guided ones.
 
+Quantised goldens (``<workload>_fp8``, ``<workload>_nvfp4``) run the same sampler with the block
+linears in row-wise FP8 or NVFP4 (the oracle's ``hp["fp8"]`` / ``hp["nvfp4"]``), on the same seeded
+weights and inputs as the bf16 workload they name; ``meta.precision`` says which.
+
 FLUX.3 workloads (``f3*``) use the FLUX.3 oracle with the flow-map target time t_{i+1}; the
 8272-token image-to-image case runs the first STEPS_RUN steps of its 16-step schedule (``v`` then
 holds those steps and ``final`` the packed state after them, ``meta.steps_run`` says how many).
@@ -34,12 +38,20 @@ from oracle import flux_oracle as O  # noqa: E402
 from oracle import flux3_oracle as O3  # noqa: E402
 
 ROW_STRIDE = {"t2i256": 1, "t2i512": 2, "t2i1024": 8, "i2i1024": 8, "mref1024": 8, "cfg256": 1,
-              "f3t2i256": 1, "f3i2i256": 1, "f3t2i1024": 8, "f3i2i1024": 8, "f3cfg256": 1}
+              "f3t2i256": 1, "f3i2i256": 1, "f3t2i1024": 8, "f3i2i1024": 8, "f3cfg256": 1,
+              "t2i256_fp8": 1, "t2i256_nvfp4": 1, "t2i1024_fp8": 8, "t2i1024_nvfp4": 8}
 STEPS_RUN = {"f3i2i1024": 4}
+PRECISIONS = ("fp8", "nvfp4")
+
+
+def split_name(name):
+    """(workload, precision): 't2i256_nvfp4' -> ('t2i256', 'nvfp4'); plain names are bf16."""
+    base, _, prec = name.rpartition("_")
+    return (base, prec) if prec in PRECISIONS else (name, "bf16")
 
 
 def rows_for(name):
-    w = WORKLOADS[name]
+    w = WORKLOADS[split_name(name)[0]]
     return np.arange(0, w.n_img, ROW_STRIDE[name], dtype=np.int32)
 
 
@@ -81,7 +93,8 @@ def make3(name):
 def make(name):
     if name.startswith("f3"):
         return make3(name)
-    w = WORKLOADS[name]
+    base, precision = split_name(name)
+    w = WORKLOADS[base]
     t0 = time.time()
     _, p = make_weights(w.dims, w.seed)
     lat, txt, ref = make_inputs(w)
@@ -100,11 +113,15 @@ def make(name):
         guided = {}
         if w.guidance is not None:
             guided = {"txt_uncond": torch.from_numpy(make_uncond_text(w)), "guidance": w.guidance}
-        final, _ = O.sample(p, O.hyper(w.dims), torch.from_numpy(lat), torch.from_numpy(txt),
+        hp = O.hyper(w.dims)
+        if precision != "bf16":
+            hp[precision] = True
+        final, _ = O.sample(p, hp, torch.from_numpy(lat), torch.from_numpy(txt),
                             w.n_steps, ref, dtype=torch.float32, on_step=on_step, **guided)
     final_tok = O.pack_latents(final)[rows].float().numpy()
-    meta = {"workload": name, "seed": w.seed, "oracle_dtype": "float32", "n_steps": w.n_steps, "guidance": w.guidance,
-            "row_stride": ROW_STRIDE[name], "seconds": round(time.time() - t0, 1)}
+    meta = {"workload": base, "precision": precision, "seed": w.seed, "oracle_dtype": "float32",
+            "n_steps": w.n_steps, "guidance": w.guidance, "row_stride": ROW_STRIDE[name],
+            "seconds": round(time.time() - t0, 1)}
     np.savez(os.path.join(HERE, f"{name}.npz"), rows=rows, v=np.stack(vs), final=final_tok,
              meta=np.array(json.dumps(meta)))
     print(f"{name}: wrote {len(rows)} rows x {w.n_steps} steps in {time.time() - t0:.0f}s", flush=True)

@@ -47,6 +47,8 @@ def test_latent_space_kernels():
     shape_error(F.flux_euler_step, z(10), z(9), 0.5)
     passes_size_checks(F.flux_cfg_euler_step, z(10), z(10), z(10), 2.0, 0.5)
     shape_error(F.flux_cfg_euler_step, z(10), z(10), z(5), 2.0, 0.5)
+    passes_size_checks(F.flux_cfg_euler_step, z(10), z(10), z(10), 2.0, 0.5, None, z(10))
+    shape_error(F.flux_cfg_euler_step, z(10), z(10), z(10), 2.0, 0.5, None, z(9))
     passes_size_checks(F.flux_blend_latents, z(4, 4), z(4, 4), 0.3, z(4, 4))
     shape_error(F.flux_blend_latents, z(4, 4), z(4, 4), 0.3, z(4, 3))
 

@@ -258,8 +258,14 @@ def test_cfg_euler_step(n):
     vu = torch.randn(n, generator=g)
     xd = x.to(DEV)
     F.flux_cfg_euler_step(xd, vc.to(DEV), vu.to(DEV), 3.5, -0.25)
-    ref = O.euler_update(x.double(), O.guided_velocity(vc.double(), vu.double(), 3.5), -0.25)
+    v_ref = O.guided_velocity(vc.double(), vu.double(), 3.5)
+    ref = O.euler_update(x.double(), v_ref, -0.25)
     assert (xd.cpu().double() - ref).abs().max().item() <= 1e-5
+    # the same update with the guided velocity written out: the same x, and v within fp32 rounding
+    xo, vg = x.to(DEV), torch.full((n,), float("nan"), device=DEV)
+    F.flux_cfg_euler_step(xo, vc.to(DEV), vu.to(DEV), 3.5, -0.25, v_guided=vg)
+    assert torch.equal(xo, xd)
+    assert (vg.cpu().double() - v_ref).abs().max().item() <= 1e-5 * v_ref.abs().max().item()
 
 
 @pytest.mark.parametrize("batch,n", [(2, 77), (2, 300), (3, 129), (2, 4608)])
@@ -279,3 +285,25 @@ def test_attention_batch_sequences_are_independent(batch, n):
         rows = torch.arange(0, n, max(1, n // 40))
         ref = O.attention(q[sl][rows].double(), k[sl].double(), v[sl].double())
         assert nmax(o[sl].cpu()[rows].reshape(len(rows), -1), ref) <= TOL
+
+
+# ---------------------------------------------------------------------------- bounded waits
+def test_bounded_wait_gives_up_records_the_code_and_leaves_the_context_usable():
+    """A wait on an mbarrier that nothing arrives on returns after its limit; the kernel records its
+    code, flux_device_error reports it once (and clears it), and the next launches run normally."""
+    assert F.flux_device_error() == 0
+    F.flux_selftest_bounded_wait(20_000_000, arrive=True)          # the phase completes: no error
+    assert F.flux_device_error() == 0
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    F.flux_selftest_bounded_wait(20_000_000, arrive=False)         # nothing arrives: gives up after 20 ms
+    ev1.record()
+    torch.cuda.synchronize()
+    assert ev0.elapsed_time(ev1) >= 19.0
+    assert F.flux_device_error() == F.DEVERR_TIMEOUT_SELFTEST
+    assert F.flux_device_error() == 0                               # read and cleared
+    x = torch.zeros(1000, device=DEV)
+    F.flux_euler_step(x, torch.ones(1000, device=DEV), -0.5)        # the context still works
+    assert torch.equal(x.cpu(), torch.full((1000,), -0.5))
+    with pytest.raises(F.FluxError):
+        F.flux_selftest_bounded_wait(2_000_000_000, arrive=False)   # above the pipelines' 1 s limit
