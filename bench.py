@@ -191,28 +191,36 @@ def barrier(world):
         dist.barrier()
 
 
+CPU_SAMPLE_BLOCKS = 3      # double and single blocks the CPU sample runs (FLUX.2)
+
+
 def cpu_oracle_sample(w, params, lat, txt, ref):
-    """Oracle time of one double and one single block at full size (fp32, host cores), scaled to a forward
-    (FLUX.3: one joint block, scaled by forward FLOPs / block FLOPs)."""
+    """The fp32 oracle on host cores, on this workload's own latent and text: a forward of the model
+    cut to its first CPU_SAMPLE_BLOCKS double and single blocks (time MLP, input projections, those
+    blocks in order on the real activations, output layer), scaled to the full forward by algorithmic
+    FLOPs (FLUX.3: one joint block, scaled the same way)."""
+    import dataclasses
     from oracle import flux_oracle as O
     torch.set_grad_enabled(False)
     if is_flux3(w):
         ms_block, secs = oracle_joint_block_ms(w, params)
         return ms_block * forward_flops(w) / single_block_flops(w), secs
-    hp = O.hyper(w.dims)
-    D = w.dims.hidden
-    g = torch.Generator().manual_seed(0)
-    x_txt = torch.randn(w.n_txt, D, generator=g)
-    x_img = torch.randn(w.n_img + w.n_ref, D, generator=g)
-    s = torch.randn(D, generator=g)
-    ang = O.rope_angles(O.token_positions(w.n_txt, w.grid, w.grid, ref_grids=w.ref_grids), 128, 1e4).float()
+    k = CPU_SAMPLE_BLOCKS
+    keep = {name: v for name, v in params.items()
+            if not ((name.startswith("double.") and int(name.split(".")[1]) >= k) or
+                    (name.startswith("single.") and int(name.split(".")[1]) >= k))}
+    cut = dataclasses.replace(w, dims=dataclasses.replace(w.dims, n_double=k, n_single=k))
+    tok = O.pack_latents(torch.from_numpy(lat)).float()
+    refs, ref_grids = [], []
+    if ref is not None:
+        for r in (ref if isinstance(ref, list) else [ref]):
+            refs.append(O.pack_latents(torch.from_numpy(r)).float())
+            ref_grids.append((r.shape[1] // 2, r.shape[2] // 2))
     t0 = time.perf_counter()
-    O.double_block(params, 0, x_txt, x_img, s, ang, hp, torch.float32)
-    t1 = time.perf_counter()
-    O.single_block(params, 0, torch.cat([x_txt, x_img]), s, ang, hp, torch.float32)
-    t2 = time.perf_counter()
-    ms = 1e3 * (w.dims.n_double * (t1 - t0) + w.dims.n_single * (t2 - t1))
-    return ms, t2 - t0
+    O.forward(keep, O.hyper(w.dims), tok, torch.from_numpy(txt), 1.0, (w.grid, w.grid), refs, ref_grids,
+              dtype=torch.float32)
+    secs = time.perf_counter() - t0
+    return 1e3 * secs * forward_flops(w) / forward_flops(cut), secs
 
 
 def oracle_joint_block_ms(w, params, repeats=1):
@@ -565,8 +573,10 @@ def run_ours(args, w):
                                     "cores": torch.get_num_threads(), "kind": "oracle",
                                     "sample": (f"one joint block at full {w.name} size, fp32 oracle ({secs:.1f} s), "
                                                f"scaled by forward FLOPs / block FLOPs" if flux3 else
-                                               f"one double + one single block at full {w.name} size, fp32 oracle "
-                                               f"({secs:.1f} s), scaled x5 and x20 to a forward")
+                                               f"the {w.name} forward on its own latent and text, cut to its first "
+                                               f"{CPU_SAMPLE_BLOCKS} double + {CPU_SAMPLE_BLOCKS} single blocks, fp32 "
+                                               f"oracle ({secs:.1f} s), scaled by algorithmic FLOPs to the "
+                                               f"{n_blocks(w)}-block forward")
                                               + ("" if not guided else ", x2 for the two guided sequences")}
         print(json.dumps(line), flush=True)
     model.close()
