@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
   uint64_t* v_full = k_empty + kStagesK;                 // [kStagesV]
   uint64_t* v_empty = v_full + kStagesV;                 // [kStagesV]
   uint64_t* s_full = v_empty + kStagesV;                 // [query tile]
-  uint64_t* p_full = s_full + 2;                         // [query tile], 4 arrivals
+  uint64_t* p_full = s_full + 2;                         // [query tile], 128 arrivals (every softmax thread)
   uint64_t* o_final = p_full + 2;                        // [query tile]
   uint64_t* drain = o_final + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_full[i], 128);
       mbar_init(&o_final[i], 1);
     }
     mbar_init(drain, 1);
@@ -357,8 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
       tmem_st32(s_addr + 32, *reinterpret_cast<const uint32_t(*)[32]>(&s[32]));
       tmem_st_wait();
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[t]);
+      mbar_arrive(&p_full[t]);
       const float2 s01 = __fadd2_rn(__fadd2_rn(sp[0], sp[1]), __fadd2_rn(sp[2], sp[3]));
       l_run = l_run * alpha + (s01.x + s01.y);
       m_run = m_use;
