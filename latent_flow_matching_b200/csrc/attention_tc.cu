@@ -401,15 +401,15 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
 }  // namespace
 
 cudaError_t attention_launch(const AttnParams& P, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
+  static std::atomic<unsigned long long> attr_done{0};
+  const cudaError_t ea = once_per_device(attr_done, [] {
     cudaError_t e =
         cudaFuncSetAttribute(attention_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(attention_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+    return e;
+  });
+  if (ea != cudaSuccess) return ea;
   int n_max = P.n, nz = P.batch;
   if (P.nseg) {
     if (P.nseg < 0 || P.nseg > kMaxSegs) return cudaErrorInvalidValue;

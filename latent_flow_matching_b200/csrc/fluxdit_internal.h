@@ -7,7 +7,24 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace fdit {
+
+// Kernel attributes (the dynamic shared-memory size) are a per-device setting: cudaFuncSetAttribute
+// applies to the current device.  `set` runs once per device ordinal (below 64; beyond that, on
+// every call), and again after a failure.
+template <class SetAttributes>
+cudaError_t once_per_device(std::atomic<unsigned long long>& done, SetAttributes set) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = set();
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // ------------------------------------------------------------------ GEMM
 enum EpiMode : int { kEpiBf16Bias = 0, kEpiF32Bias = 1, kEpiSwiGLU = 2, kEpiResidGate = 3, kEpiQKNormRope = 4 };

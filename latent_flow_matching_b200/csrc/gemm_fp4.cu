@@ -310,13 +310,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads4, 1)
 }  // namespace
 
 cudaError_t gemm_fp4_launch(GemmParams4& P4, int num_sms, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(gemm_fp4_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};
+  const cudaError_t ea = once_per_device(attr_done, [] {
+    return cudaFuncSetAttribute(gemm_fp4_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  });
+  if (ea != cudaSuccess) return ea;
   GemmParams& P = P4.g;
   for (int i = 0; i < P.num_problems; ++i) {        // K in whole stages, scales present
     const GemmProblem& pr = P.prob[i];

@@ -227,13 +227,12 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
 template <int BN>
 cudaError_t launch_bn(GemmParams& P, int num_sms, cudaStream_t stream) {
   using C = GemmCfg<BN>;
-  static bool attr_set = false;          // per process; the attribute is per function
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_done{0};   // one per tile width: the attribute is per function
+  const cudaError_t ea = once_per_device(attr_done, [] {
+    return cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                C::SMEM_BYTES);
+  });
+  if (ea != cudaSuccess) return ea;
   const int grid = P.total_tiles < num_sms ? P.total_tiles : num_sms;
   count_launch();
   gemm_bf16_tc_kernel<BN><<<grid, 192, C::SMEM_BYTES, stream>>>(P);

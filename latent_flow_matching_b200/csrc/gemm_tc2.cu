@@ -232,15 +232,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
 }  // namespace
 
 cudaError_t gemm2_launch(GemmParams& P, int num_sms, cudaStream_t stream, bool fp8) {
-  static bool attr_set = false;
-  if (!attr_set) {
+  static std::atomic<unsigned long long> attr_done{0};
+  const cudaError_t ea = once_per_device(attr_done, [] {
     cudaError_t e =
         cudaFuncSetAttribute(gemm_bf16_tc2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(gemm_bf16_tc2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+    return e;
+  });
+  if (ea != cudaSuccess) return ea;
   for (int i = 0; i < P.num_problems; ++i) {        // 8-bit problems: K in whole stages, scales present
     const GemmProblem& pr = P.prob[i];
     if (pr.M > 0 && (pr.K % (fp8 ? 2 * BK : BK) != 0 || (fp8 && (!pr.scale_a || !pr.scale_b))))

@@ -125,3 +125,41 @@ def test_quantised_sampler_against_quantised_oracle_golden(name):
         e0, x0 = rel_l2(vs[0][rows], gd["v"][0]), rel_l2(vs[0][rows], ex["v"][0])
         print(f"{name} step 0: vs quantised golden {e0:.4f}, vs exact golden {x0:.4f}")
         assert e0 < EXACT_RATIO * x0
+
+
+@pytest.mark.parametrize("precision", ["fp8", "nvfp4"])
+def test_flux3_one_per_mode_one_joint_block_at_full_token_count(precision):
+    """FLUX.3 image editing at 1024^2 with a 1024^2 reference (4096 + 80 + 4096 = 8272 tokens: every
+    per-mode segment and joint-block GEMM at full size), 1 per-mode + 1 joint block, quantised
+    block linears against the FLUX.3 oracle run live in float64, at the tiny models' bars."""
+    from oracle import flux3_oracle as O3
+    w = WORKLOADS["f3i2i1024"]
+    blob, p = make_weights(w.dims, w.seed)
+    lat, txt, ref = make_inputs(w)
+    keep = {k: v for k, v in p.items()
+            if not ((k.startswith("mode.") and int(k.split(".")[1]) >= 1) or
+                    (k.startswith("joint.") and int(k.split(".")[1]) >= 1))}
+    tok = O.pack_latents(torch.from_numpy(lat))
+    rtok = O.pack_latents(torch.from_numpy(ref))
+    tx = torch.from_numpy(txt)
+    grids = [(w.ref_grid, w.ref_grid)]
+    want = O3.forward3(keep, dict(O.hyper(w.dims), **{precision: True}), tok, tx, 0.75, (w.grid, w.grid), [rtok],
+                       grids, t_target=0.5)
+    exact = O3.forward3(keep, O.hyper(w.dims), tok, tx, 0.75, (w.grid, w.grid), [rtok], grids, t_target=0.5)
+    model = F.Flux3DiT(blob, w.dims)
+    del blob
+    v = torch.empty(w.n_img, 128, device=DEV)
+    try:
+        model.set_active_blocks(1, 1)
+        model.set_precision(PRECISION[precision])
+        model.forward(tok.float().to(DEV), (w.grid, w.grid), tx.to(DEV), 0.75, v, rtok.float().to(DEV), grids,
+                      t_target=0.5)
+        torch.cuda.synchronize()
+        assert F.flux_device_error() == 0
+    finally:
+        model.close()
+    err = rel_l2(v, want)
+    print(f"FLUX.3 {precision} 1+1 blocks at {w.n_tokens} tokens: vs quantised oracle {err:.4f}, "
+          f"vs exact {rel_l2(v, exact):.4f}, quantised oracle vs exact {rel_l2(want, exact):.4f}")
+    assert err <= BLOCK_BARS[precision], err
+    assert err < 0.6 * rel_l2(v, exact)
