@@ -158,6 +158,8 @@ __global__ void __launch_bounds__(kThreads, 1) attention_tc_kernel(const __grid_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();                                    // after this CTA's tensor-memory allocation
+  pdl_wait();                                       // the previous kernel's writes are visible
 
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
@@ -424,9 +426,9 @@ cudaError_t attention_launch(const AttnParams& P, cudaStream_t stream) {
   dim3 grid((n_max + kQTiles * kTile - 1) / (kQTiles * kTile), P.heads, nz);
   count_launch();
   if (P.nseg)
-    attention_tc_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(P);
+    launch_kernel(attention_tc_kernel<true>, grid, kThreads, kSmemBytes, stream, P);
   else
-    attention_tc_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(P);
+    launch_kernel(attention_tc_kernel<false>, grid, kThreads, kSmemBytes, stream, P);
   return cudaGetLastError();
 }
 

@@ -37,6 +37,18 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with launch_kernel() (fluxdit_internal.h) may start while the previous kernel
+// on its stream is still finishing, so that its set-up (barrier initialisation, tensor-memory
+// allocation, tensor-map prefetch) overlaps that kernel's last CTAs.  pdl_wait() returns once the
+// previous kernel has completed and its memory writes are visible: every kernel calls it before its
+// first global-memory access.  pdl_trigger() lets the next kernel's CTAs be scheduled once every
+// CTA of this grid has called it (or exited); a kernel that allocates tensor memory calls it only
+// after its allocation, so a waiting next kernel can never hold columns this one still needs.
+// Without a programmatic launch both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

@@ -46,6 +46,8 @@ __device__ __forceinline__ PackTile pack_tile(int w8) {
 
 __global__ void __launch_bounds__(kPackThreads) pack_kernel(const float* __restrict__ lat, float* __restrict__ tok,
                                                             int h8, int w8) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ __align__(16) float st[kPackT * kPackLd];
   const PackTile tl = pack_tile(w8);
   // latent side: item (c, py, jj), jj fastest
@@ -72,6 +74,8 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const float* __restr
 
 __global__ void __launch_bounds__(kPackThreads) unpack_kernel(const float* __restrict__ tok, float* __restrict__ lat,
                                                               int h8, int w8) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ __align__(16) float st[kPackT * kPackLd];
   const PackTile tl = pack_tile(w8);
   const float4* src =
@@ -95,6 +99,8 @@ __global__ void __launch_bounds__(kPackThreads) unpack_kernel(const float* __res
 
 // ------------------------------------------------------------------ Euler, casts
 __global__ void euler_kernel(float* __restrict__ x, const float* __restrict__ v, size_t n, float dt) {
+  pdl_trigger();
+  pdl_wait();
   const size_t n4 = n / 4;
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4; i += stride) {
@@ -111,6 +117,8 @@ __global__ void euler_kernel(float* __restrict__ x, const float* __restrict__ v,
 }
 
 __global__ void cast_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y, size_t n) {
+  pdl_trigger();
+  pdl_wait();
   const size_t n4 = n / 4;
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4; i += stride) {
@@ -130,6 +138,8 @@ __global__ void cast_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __r
 template <int VPT>
 __global__ void __launch_bounds__(256) ln_mod_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y,
                                                      int rows, const LnModSets m, float eps) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int dim = 1024 * VPT;
   __shared__ float red[2][8];
   const int row = blockIdx.x;
@@ -181,6 +191,8 @@ __global__ void __launch_bounds__(256) ln_mod_kernel(const float* __restrict__ x
 // Any dim that is a multiple of 4: three passes over the row in global memory.
 __global__ void ln_mod_generic_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y, int rows, int dim,
                                       const LnModSets m, float eps) {
+  pdl_trigger();
+  pdl_wait();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= rows) return;
@@ -207,6 +219,8 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(__nv_bfloat16* __rest
                                                            const __nv_bfloat16* __restrict__ gq1,
                                                            const __nv_bfloat16* __restrict__ gk1,
                                                            const float2* __restrict__ rope, float eps) {
+  pdl_trigger();
+  pdl_wait();
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int row = gw >> 1;
@@ -252,6 +266,8 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(__nv_bfloat16* __rest
 // text i: (0,0,0,i); image (r,c): (0,r,c,0); reference k (r,c): (0,r,c,-(k+1)).
 __global__ void rope_table_kernel(float2* __restrict__ table, int n_txt, int gh, int gw, RefGrids refs,
                                   float theta) {
+  pdl_trigger();
+  pdl_wait();
   int n = n_txt + gh * gw;
   for (int k = 0; k < refs.count; ++k) n += refs.h[k] * refs.w[k];
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
@@ -286,6 +302,8 @@ __global__ void rope_table_kernel(float2* __restrict__ table, int n_txt, int gh,
 // x += dt * (v_u + g (v_c - v_u)): the guided velocity and the Euler step in one pass.
 __global__ void cfg_euler_kernel(float* __restrict__ x, const float* __restrict__ vc, const float* __restrict__ vu,
                                  float* __restrict__ vg, size_t n, float g, float dt) {
+  pdl_trigger();
+  pdl_wait();
   const size_t n4 = n / 4;
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4; i += stride) {
@@ -310,6 +328,8 @@ __global__ void cfg_euler_kernel(float* __restrict__ x, const float* __restrict_
 
 __global__ void blend_kernel(const float* __restrict__ x, const float* __restrict__ noise, float t,
                              float* __restrict__ out, size_t n) {
+  pdl_trigger();
+  pdl_wait();
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n; i += stride)
     out[i] = (1.0f - t) * x[i] + t * noise[i];
@@ -317,6 +337,8 @@ __global__ void blend_kernel(const float* __restrict__ x, const float* __restric
 
 // ------------------------------------------------------------------ timestep embedding, GEMV
 __global__ void timestep_embed_kernel(float* __restrict__ out, float t, int dim) {
+  pdl_trigger();
+  pdl_wait();
   const int half = dim / 2;
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= half) return;
@@ -338,6 +360,8 @@ __global__ void __launch_bounds__(256) gemv_kernel(const __nv_bfloat16* __restri
                                                    const __nv_bfloat16* __restrict__ b, const float* __restrict__ x,
                                                    float* __restrict__ y, const float* __restrict__ add, int rows,
                                                    int k, int silu_in, int silu_out) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float xs[];
   for (int i = threadIdx.x; i < NV * k; i += blockDim.x) {
     const float v = x[i];
@@ -398,7 +422,7 @@ cudaError_t pack_latents_launch(const float* lat, float* tok, int c, int h8, int
   unsigned tiles;
   if (const cudaError_t e = pack_grid(c, h8, w8, &tiles)) return e;
   count_launch();
-  pack_kernel<<<tiles, kPackThreads, 0, s>>>(lat, tok, h8, w8);
+  launch_kernel(pack_kernel, tiles, kPackThreads, 0, s, lat, tok, h8, w8);
   return cudaGetLastError();
 }
 
@@ -406,14 +430,14 @@ cudaError_t unpack_latents_launch(const float* tok, float* lat, int c, int h8, i
   unsigned tiles;
   if (const cudaError_t e = pack_grid(c, h8, w8, &tiles)) return e;
   count_launch();
-  unpack_kernel<<<tiles, kPackThreads, 0, s>>>(tok, lat, h8, w8);
+  launch_kernel(unpack_kernel, tiles, kPackThreads, 0, s, tok, lat, h8, w8);
   return cudaGetLastError();
 }
 
 cudaError_t euler_launch(float* x, const float* v, size_t n, float dt, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   count_launch();
-  euler_kernel<<<blocks_for((n + 3) / 4, 256), 256, 0, s>>>(x, v, n, dt);
+  launch_kernel(euler_kernel, blocks_for((n + 3) / 4, 256), 256, 0, s, x, v, n, dt);
   return cudaGetLastError();
 }
 
@@ -421,14 +445,14 @@ cudaError_t cfg_euler_launch(float* x, const float* vc, const float* vu, float* 
                              cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   count_launch();
-  cfg_euler_kernel<<<blocks_for((n + 3) / 4, 256), 256, 0, s>>>(x, vc, vu, vg, n, g, dt);
+  launch_kernel(cfg_euler_kernel, blocks_for((n + 3) / 4, 256), 256, 0, s, x, vc, vu, vg, n, g, dt);
   return cudaGetLastError();
 }
 
 cudaError_t cast_bf16_launch(const float* x, __nv_bfloat16* y, size_t n, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   count_launch();
-  cast_bf16_kernel<<<blocks_for((n + 3) / 4, 256), 256, 0, s>>>(x, y, n);
+  launch_kernel(cast_bf16_kernel, blocks_for((n + 3) / 4, 256), 256, 0, s, x, y, n);
   return cudaGetLastError();
 }
 
@@ -441,9 +465,9 @@ cudaError_t ln_modulate3_launch(const float* x, __nv_bfloat16* y, int rows, int 
   const LnModSets m = {split, split2, period, shift0, shift1, shift2, scale0, scale1, scale2};
   count_launch();
   if (dim == 3072)
-    ln_mod_kernel<3><<<rows, 256, 0, s>>>(x, y, rows, m, eps);
+    launch_kernel(ln_mod_kernel<3>, rows, 256, 0, s, x, y, rows, m, eps);
   else
-    ln_mod_generic_kernel<<<(rows + 7) / 8, 256, 0, s>>>(x, y, rows, dim, m, eps);
+    launch_kernel(ln_mod_generic_kernel, (rows + 7) / 8, 256, 0, s, x, y, rows, dim, m, eps);
   return cudaGetLastError();
 }
 
@@ -460,7 +484,7 @@ cudaError_t qk_norm_rope_launch(__nv_bfloat16* qkv, int rows, int ld, int kcol, 
   if (rows <= 0) return cudaSuccess;
   const int warps = rows * 2;
   count_launch();
-  qk_norm_rope_kernel<<<(warps + 7) / 8, 256, 0, s>>>(qkv, rows, ld, kcol, heads, split, gq0, gk0, gq1, gk1, rope,
+  launch_kernel(qk_norm_rope_kernel, (warps + 7) / 8, 256, 0, s, qkv, rows, ld, kcol, heads, split, gq0, gk0, gq1, gk1, rope,
                                                       eps);
   return cudaGetLastError();
 }
@@ -471,20 +495,20 @@ cudaError_t rope_table_launch(float2* table, int n_txt, int gh, int gw, const Re
   for (int k = 0; k < refs.count; ++k) n += refs.h[k] * refs.w[k];
   if (n <= 0) return cudaSuccess;
   count_launch();
-  rope_table_kernel<<<(n * 64 + 255) / 256, 256, 0, s>>>(table, n_txt, gh, gw, refs, theta);
+  launch_kernel(rope_table_kernel, (n * 64 + 255) / 256, 256, 0, s, table, n_txt, gh, gw, refs, theta);
   return cudaGetLastError();
 }
 
 cudaError_t blend_launch(const float* x, const float* noise, float t, float* out, size_t n, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   count_launch();
-  blend_kernel<<<blocks_for(n, 256), 256, 0, s>>>(x, noise, t, out, n);
+  launch_kernel(blend_kernel, blocks_for(n, 256), 256, 0, s, x, noise, t, out, n);
   return cudaGetLastError();
 }
 
 cudaError_t timestep_embed_launch(float* temb, float t, int dim, cudaStream_t s) {
   count_launch();
-  timestep_embed_kernel<<<(dim / 2 + 127) / 128, 128, 0, s>>>(temb, t, dim);
+  launch_kernel(timestep_embed_kernel, (dim / 2 + 127) / 128, 128, 0, s, temb, t, dim);
   return cudaGetLastError();
 }
 
@@ -500,13 +524,13 @@ cudaError_t gemv_multi_launch(const __nv_bfloat16* W, const __nv_bfloat16* b, co
   if (smem > 48 * 1024) return cudaErrorInvalidValue;
   count_launch();
   if (nvec == 1)
-    gemv_kernel<1><<<grid, 256, smem, s>>>(W, b, x, y, add, rows, k, silu_in, silu_out);
+    launch_kernel(gemv_kernel<1>, grid, 256, smem, s, W, b, x, y, add, rows, k, silu_in, silu_out);
   else if (nvec == 2)
-    gemv_kernel<2><<<grid, 256, smem, s>>>(W, b, x, y, add, rows, k, silu_in, silu_out);
+    launch_kernel(gemv_kernel<2>, grid, 256, smem, s, W, b, x, y, add, rows, k, silu_in, silu_out);
   else if (nvec == 3)
-    gemv_kernel<3><<<grid, 256, smem, s>>>(W, b, x, y, add, rows, k, silu_in, silu_out);
+    launch_kernel(gemv_kernel<3>, grid, 256, smem, s, W, b, x, y, add, rows, k, silu_in, silu_out);
   else
-    gemv_kernel<4><<<grid, 256, smem, s>>>(W, b, x, y, add, rows, k, silu_in, silu_out);
+    launch_kernel(gemv_kernel<4>, grid, 256, smem, s, W, b, x, y, add, rows, k, silu_in, silu_out);
   return cudaGetLastError();
 }
 

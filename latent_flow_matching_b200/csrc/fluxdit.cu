@@ -21,6 +21,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -141,6 +142,11 @@ int num_sms_current() {
 // ------------------------------------------------------------------ launch counter
 static std::atomic<unsigned long long> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+bool pdl_enabled() {
+  const char* v = std::getenv("FLUX_PDL");
+  return !(v && v[0] == '0' && v[1] == 0);
+}
 
 // ------------------------------------------------------------------ blob layout
 struct BlobTensor {

@@ -199,6 +199,30 @@ struct GemmParams4 {
 cudaError_t gemm_fp4_launch(GemmParams4& P, int num_sms, cudaStream_t stream);
 int gemm_fp4_read_device_error(cudaStream_t stream);
 
+// ------------------------------------------------------------------ kernel launches
+// Programmatic dependent launches are on unless the environment sets FLUX_PDL=0 (read at every
+// launch, so a process can compare both; a CUDA graph keeps what was set when it was captured).
+bool pdl_enabled();
+// Launch `kernel` on `s` with programmatic stream serialisation (when enabled): the kernel may be
+// scheduled before the previous kernel on the stream has finished, and waits for it with
+// pdl_wait() (common.cuh) before touching global memory.  Only kernels that call pdl_wait()
+// before their first global access may be launched this way.
+template <typename... KernelArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KernelArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // ------------------------------------------------------------------ host helpers
 // Record `msg` as the calling thread's flux_get_error() message and return `code`.
 int record_error(int code, const char* msg);

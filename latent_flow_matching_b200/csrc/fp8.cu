@@ -48,6 +48,8 @@ __device__ __forceinline__ void row_scale(float amax, float* scale, float* inv) 
 __global__ void __launch_bounds__(kQThreads) quantize_rows_kernel(const __nv_bfloat16* __restrict__ x, int ldx,
                                                                   int cols, uint8_t* __restrict__ q, int ldq,
                                                                   float* __restrict__ scale) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[kQThreads / 32];
   const int row = blockIdx.x;
   const int nch = cols / 8;
@@ -94,6 +96,8 @@ __global__ void __launch_bounds__(kQThreads) ln_mod_fp8_kernel(const float* __re
                                                                const float* __restrict__ sc1,
                                                                const float* __restrict__ sh2,
                                                                const float* __restrict__ sc2, float eps) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int dim = 1024 * VPT;
   __shared__ float red[3][kQThreads / 32];
   const int row = blockIdx.x;
@@ -169,7 +173,7 @@ cudaError_t quantize_rows_launch(const __nv_bfloat16* x, int ldx, int rows, int 
   if (cols <= 0 || cols % 8 || cols > kQThreads * kQMaxChunks * 8 || ldx % 8 || ldq % 8)
     return cudaErrorInvalidValue;
   count_launch();
-  quantize_rows_kernel<<<rows, kQThreads, 0, s>>>(x, ldx, cols, q, ldq, scale);
+  launch_kernel(quantize_rows_kernel, rows, kQThreads, 0, s, x, ldx, cols, q, ldq, scale);
   return cudaGetLastError();
 }
 
@@ -182,19 +186,19 @@ cudaError_t ln_modulate_fp8_launch(const float* x, uint8_t* q, float* qscale, in
   count_launch();
   switch (dim) {
     case 1024:
-      ln_mod_fp8_kernel<1><<<rows, kQThreads, 0, s>>>(x, q, qscale, split, split2, period, shift0, scale0, shift1,
+      launch_kernel(ln_mod_fp8_kernel<1>, rows, kQThreads, 0, s, x, q, qscale, split, split2, period, shift0, scale0, shift1,
                                                        scale1, shift2, scale2, eps);
       break;
     case 2048:
-      ln_mod_fp8_kernel<2><<<rows, kQThreads, 0, s>>>(x, q, qscale, split, split2, period, shift0, scale0, shift1,
+      launch_kernel(ln_mod_fp8_kernel<2>, rows, kQThreads, 0, s, x, q, qscale, split, split2, period, shift0, scale0, shift1,
                                                        scale1, shift2, scale2, eps);
       break;
     case 3072:
-      ln_mod_fp8_kernel<3><<<rows, kQThreads, 0, s>>>(x, q, qscale, split, split2, period, shift0, scale0, shift1,
+      launch_kernel(ln_mod_fp8_kernel<3>, rows, kQThreads, 0, s, x, q, qscale, split, split2, period, shift0, scale0, shift1,
                                                        scale1, shift2, scale2, eps);
       break;
     case 4096:
-      ln_mod_fp8_kernel<4><<<rows, kQThreads, 0, s>>>(x, q, qscale, split, split2, period, shift0, scale0, shift1,
+      launch_kernel(ln_mod_fp8_kernel<4>, rows, kQThreads, 0, s, x, q, qscale, split, split2, period, shift0, scale0, shift1,
                                                        scale1, shift2, scale2, eps);
       break;
     default:

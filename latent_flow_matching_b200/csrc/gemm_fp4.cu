@@ -155,6 +155,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads4, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();                                    // after this CTA's tensor-memory allocation
+  pdl_wait();                                       // the previous kernel's writes are visible
 
   if (warp == 0) {
     if (lane == 0) {
@@ -344,7 +346,7 @@ cudaError_t gemm_fp4_launch(GemmParams4& P4, int num_sms, cudaStream_t stream) {
   int pairs = num_sms / 2;
   if (pairs > total) pairs = total;
   count_launch();
-  gemm_fp4_tc2_kernel<<<2 * pairs, kThreads4, SMEM_BYTES, stream>>>(P4);
+  launch_kernel(gemm_fp4_tc2_kernel, 2 * pairs, kThreads4, SMEM_BYTES, stream, P4);
   return cudaGetLastError();
 }
 

@@ -104,6 +104,8 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();                                    // after this CTA's tensor-memory allocation
+  pdl_wait();                                       // the previous kernel's writes are visible
 
   if (warp == 0) {
     if (lane == 0) {
@@ -235,7 +237,7 @@ cudaError_t launch_bn(GemmParams& P, int num_sms, cudaStream_t stream) {
   if (ea != cudaSuccess) return ea;
   const int grid = P.total_tiles < num_sms ? P.total_tiles : num_sms;
   count_launch();
-  gemm_bf16_tc_kernel<BN><<<grid, 192, C::SMEM_BYTES, stream>>>(P);
+  launch_kernel(gemm_bf16_tc_kernel<BN>, grid, 192, C::SMEM_BYTES, stream, P);
   return cudaGetLastError();
 }
 

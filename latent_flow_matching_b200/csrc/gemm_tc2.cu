@@ -102,6 +102,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
   cluster_sync();                                   // both CTAs' barriers exist before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();                                    // after this CTA's tensor-memory allocation
+  pdl_wait();                                       // the previous kernel's writes are visible
 
   if (warp == 0) {
     if (lane == 0) {
@@ -267,9 +269,9 @@ cudaError_t gemm2_launch(GemmParams& P, int num_sms, cudaStream_t stream, bool f
   if (pairs > total) pairs = total;
   count_launch();
   if (fp8)
-    gemm_bf16_tc2_kernel<true><<<2 * pairs, kThreads2, SMEM_BYTES, stream>>>(P);
+    launch_kernel(gemm_bf16_tc2_kernel<true>, 2 * pairs, kThreads2, SMEM_BYTES, stream, P);
   else
-    gemm_bf16_tc2_kernel<false><<<2 * pairs, kThreads2, SMEM_BYTES, stream>>>(P);
+    launch_kernel(gemm_bf16_tc2_kernel<false>, 2 * pairs, kThreads2, SMEM_BYTES, stream, P);
   return cudaGetLastError();
 }
 

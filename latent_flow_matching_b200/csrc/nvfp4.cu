@@ -97,6 +97,8 @@ __global__ void __launch_bounds__(kQ4Threads) quantize_nvfp4_kernel(const __nv_b
                                                                     int k, uint8_t* __restrict__ q, int ldq,
                                                                     uint8_t* __restrict__ sf,
                                                                     float* __restrict__ row_scale, const Q4Segs segs) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[kQ4Threads / 32];
   const int tid = threadIdx.x;
   const Q4Row rr = q4_row(segs);
@@ -153,6 +155,8 @@ __global__ void __launch_bounds__(kQ4Threads) ln_mod_nvfp4_kernel(const float* _
                                                                   uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
                                                                   float* __restrict__ row_scale, const Q4Segs segs,
                                                                   LnModSets ms, float eps) {
+  pdl_trigger();
+  pdl_wait();
   static_assert(VPT >= 1 && VPT <= 4, "one block scale per quad lane");
   constexpr int dim = 1024 * VPT;
   __shared__ float red[kQ4Threads / 32];
@@ -234,14 +238,14 @@ cudaError_t quantize_nvfp4_launch(const __nv_bfloat16* x, int ldx, int k, uint8_
   const unsigned grid = static_cast<unsigned>(total);
   count_launch();
   switch ((k / 8 + kQ4Threads - 1) / kQ4Threads) {
-    case 1: quantize_nvfp4_kernel<1><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
-    case 2: quantize_nvfp4_kernel<2><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
-    case 3: quantize_nvfp4_kernel<3><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
-    case 4: quantize_nvfp4_kernel<4><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
-    case 5: quantize_nvfp4_kernel<5><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
-    case 6: quantize_nvfp4_kernel<6><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
-    case 7: quantize_nvfp4_kernel<7><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
-    default: quantize_nvfp4_kernel<8><<<grid, kQ4Threads, 0, s>>>(x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    case 1: launch_kernel(quantize_nvfp4_kernel<1>, grid, kQ4Threads, 0, s, x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    case 2: launch_kernel(quantize_nvfp4_kernel<2>, grid, kQ4Threads, 0, s, x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    case 3: launch_kernel(quantize_nvfp4_kernel<3>, grid, kQ4Threads, 0, s, x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    case 4: launch_kernel(quantize_nvfp4_kernel<4>, grid, kQ4Threads, 0, s, x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    case 5: launch_kernel(quantize_nvfp4_kernel<5>, grid, kQ4Threads, 0, s, x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    case 6: launch_kernel(quantize_nvfp4_kernel<6>, grid, kQ4Threads, 0, s, x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    case 7: launch_kernel(quantize_nvfp4_kernel<7>, grid, kQ4Threads, 0, s, x, ldx, k, q, ldq, sf, row_scale, segs); break;
+    default: launch_kernel(quantize_nvfp4_kernel<8>, grid, kQ4Threads, 0, s, x, ldx, k, q, ldq, sf, row_scale, segs); break;
   }
   return cudaGetLastError();
 }
@@ -253,10 +257,10 @@ cudaError_t ln_modulate_nvfp4_launch(const float* x, int dim, uint8_t* q, uint8_
   if (total == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>(total);
   switch (dim) {
-    case 1024: count_launch(); ln_mod_nvfp4_kernel<1><<<grid, kQ4Threads, 0, s>>>(x, q, sf, row_scale, segs, ms, eps); break;
-    case 2048: count_launch(); ln_mod_nvfp4_kernel<2><<<grid, kQ4Threads, 0, s>>>(x, q, sf, row_scale, segs, ms, eps); break;
-    case 3072: count_launch(); ln_mod_nvfp4_kernel<3><<<grid, kQ4Threads, 0, s>>>(x, q, sf, row_scale, segs, ms, eps); break;
-    case 4096: count_launch(); ln_mod_nvfp4_kernel<4><<<grid, kQ4Threads, 0, s>>>(x, q, sf, row_scale, segs, ms, eps); break;
+    case 1024: count_launch(); launch_kernel(ln_mod_nvfp4_kernel<1>, grid, kQ4Threads, 0, s, x, q, sf, row_scale, segs, ms, eps); break;
+    case 2048: count_launch(); launch_kernel(ln_mod_nvfp4_kernel<2>, grid, kQ4Threads, 0, s, x, q, sf, row_scale, segs, ms, eps); break;
+    case 3072: count_launch(); launch_kernel(ln_mod_nvfp4_kernel<3>, grid, kQ4Threads, 0, s, x, q, sf, row_scale, segs, ms, eps); break;
+    case 4096: count_launch(); launch_kernel(ln_mod_nvfp4_kernel<4>, grid, kQ4Threads, 0, s, x, q, sf, row_scale, segs, ms, eps); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
