@@ -191,7 +191,7 @@ def barrier(world):
         dist.barrier()
 
 
-CPU_SAMPLE_BLOCKS = 3      # double and single blocks the CPU sample runs (FLUX.2)
+CPU_SAMPLE_BLOCKS = 4      # double and single blocks the CPU sample runs (FLUX.2): about 12 s on 16 cores
 
 
 def cpu_oracle_sample(w, params, lat, txt, ref):
