@@ -137,6 +137,26 @@ def test_forward_is_deterministic(tiny):
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("precision", ["bf16", "fp8", "nvfp4"])
+def test_programmatic_launches_change_nothing(tiny, precision, monkeypatch):
+    """With programmatic dependent launches (the default) every kernel waits for its predecessor
+    before touching memory, so the sampler's output is bit-identical to plain stream order."""
+    w, p, model = tiny
+    lat, txt, _ = make_inputs(w)
+    prec = {"bf16": F.PRECISION_BF16, "fp8": F.PRECISION_FP8, "nvfp4": F.PRECISION_NVFP4}[precision]
+    model.set_precision(prec)
+    try:
+        monkeypatch.setenv("FLUX_PDL", "0")
+        plain, vs_plain = gpu_sample(model, w, lat, txt, None)
+        monkeypatch.setenv("FLUX_PDL", "1")
+        pdl, vs_pdl = gpu_sample(model, w, lat, txt, None)
+    finally:
+        model.set_precision(F.PRECISION_BF16)
+    assert torch.equal(plain, pdl)
+    assert all(torch.equal(a, b) for a, b in zip(vs_plain, vs_pdl))
+    assert F.flux_device_error() == 0
+
+
 @pytest.mark.parametrize("n_txt,grid,ref_grid", [(0, (4, 6), (0, 0)), (5, (6, 4), (4, 4)), (131, (8, 8), (4, 8))])
 def test_tiny_forward_ragged_and_degenerate_shapes(tiny, n_txt, grid, ref_grid):
     """No text, non-square grids, a reference of another size, sequence lengths off the 128-row tiles."""
