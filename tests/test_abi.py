@@ -122,6 +122,17 @@ def test_entry_points_reject_bad_arguments(L):
     L.flux_dit_destroy(None)
 
 
+def test_guided_update_and_wait_self_test_reject_bad_arguments(L):
+    p = ctypes.c_void_p(16)            # never dereferenced: validation fails first
+    assert L.flux_cfg_euler_step_out(p, p, p, None, 8, 3.5, -0.25, None) == F.FLUX_EINVAL     # no v_guided
+    assert L.flux_cfg_euler_step_out(p, p, p, ctypes.c_void_p(20), 8, 3.5, -0.25, None) == F.FLUX_EINVAL
+    assert "aligned" in F.get_error()
+    assert L.flux_cfg_euler_step_out(p, p, p, p, 8, float("inf"), -0.25, None) == F.FLUX_EINVAL
+    assert L.flux_selftest_bounded_wait(0, 0, None) == F.FLUX_EINVAL                        # no limit
+    assert L.flux_selftest_bounded_wait(2_000_000_000, 0, None) == F.FLUX_EINVAL            # above 1 s
+    assert L.flux_selftest_bounded_wait(1000, 2, None) == F.FLUX_EINVAL
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(4, 4)
