@@ -121,6 +121,25 @@ def _gpu_forward(model, tok, grid, txt, t, refs, ref_grids, t_target):
     return v
 
 
+@pytest.mark.parametrize("precision", ["bf16", "nvfp4"])
+def test_tiny3_programmatic_launches_change_nothing(tiny3, precision, monkeypatch):
+    """FLUX.3 forward with a reference (segmented per-mode attention, three-region LN-mod) with and
+    without programmatic dependent launches: bit-identical."""
+    w, p, model = tiny3
+    tok, txt, refs = _tiny_inputs(7, 16, (4, 4), [(4, 4)])
+    model.set_precision(F.PRECISION_NVFP4 if precision == "nvfp4" else F.PRECISION_BF16)
+    try:
+        monkeypatch.setenv("FLUX_PDL", "0")
+        plain = _gpu_forward(model, tok, (4, 4), txt, 0.6, refs, [(4, 4)], 0.35)
+        monkeypatch.setenv("FLUX_PDL", "1")
+        pdl = _gpu_forward(model, tok, (4, 4), txt, 0.6, refs, [(4, 4)], 0.35)
+        torch.cuda.synchronize()
+    finally:
+        model.set_precision(F.PRECISION_BF16)
+    assert torch.equal(plain, pdl)
+    assert F.flux_device_error() == 0
+
+
 @pytest.mark.parametrize("n_mode,n_joint", [(0, 0), (1, 0), (0, 1), (1, 1)])
 def test_tiny3_forward_block_by_block(tiny3, n_mode, n_joint):
     w, p, model = tiny3
