@@ -157,6 +157,42 @@ def test_programmatic_launches_change_nothing(tiny, precision, monkeypatch):
     assert F.flux_device_error() == 0
 
 
+def test_sampling_step_replayed_from_a_cuda_graph_equals_plain_launches(tiny):
+    """One sampling step as the benchmark times it (a device copy of the noise, the run's modulation
+    vectors, pack, forward, Euler, unpack), captured in a CUDA graph with programmatic launches and
+    replayed, against the same launches run directly: bit-identical latents."""
+    w, p, model = tiny
+    lat_h, txt_h, _ = make_inputs(w)
+    lat0 = torch.from_numpy(lat_h).to(DEV)
+    txt = torch.from_numpy(txt_h).to(DEV)
+    ts = F.euler_schedule(w.n_steps)
+    tok = torch.empty(w.n_img, 128, device=DEV)
+    v = torch.empty_like(tok)
+    lat = torch.empty_like(lat0)
+
+    def step():
+        lat.copy_(lat0)
+        model.prepare_timesteps(ts[:-1])
+        F.flux_pack_latents(lat, tok)
+        model.forward(tok, (w.grid, w.grid), txt, ts[0], v)
+        F.flux_euler_step(tok, v, ts[1] - ts[0])
+        F.flux_unpack_latents(tok, lat)
+
+    step()
+    torch.cuda.synchronize()
+    plain = lat.clone()
+    lat.fill_(float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    lat.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(lat, plain)
+    del g
+    assert F.flux_device_error() == 0
+
+
 @pytest.mark.parametrize("n_txt,grid,ref_grid", [(0, (4, 6), (0, 0)), (5, (6, 4), (4, 4)), (131, (8, 8), (4, 8))])
 def test_tiny_forward_ragged_and_degenerate_shapes(tiny, n_txt, grid, ref_grid):
     """No text, non-square grids, a reference of another size, sequence lengths off the 128-row tiles."""
