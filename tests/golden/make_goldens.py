@@ -45,7 +45,8 @@ from oracle import flux3_oracle as O3  # noqa: E402
 
 ROW_STRIDE = {"t2i256": 1, "t2i512": 2, "t2i1024": 8, "i2i1024": 8, "mref1024": 8, "cfg256": 1,
               "f3t2i256": 1, "f3i2i256": 1, "f3t2i1024": 8, "f3i2i1024": 8, "f3cfg256": 1,
-              "t2i256_fp8": 1, "t2i256_nvfp4": 1, "t2i1024_fp8": 8, "t2i1024_nvfp4": 8}
+              "t2i256_fp8": 1, "t2i256_nvfp4": 1, "t2i1024_fp8": 8, "t2i1024_nvfp4": 8,
+              "f3t2i256_fp8": 1, "f3t2i256_nvfp4": 1}
 STEPS_RUN = {"f3i2i1024": 4, "t2i1024_fp8": 2, "t2i1024_nvfp4": 2}
 PRECISIONS = ("fp8", "nvfp4")
 
@@ -63,19 +64,29 @@ def rows_for(name):
 
 def make3(name):
     """FLUX.3 sampler: forward3 with target time t_{i+1}, Euler update, for the first k steps."""
-    w = WORKLOADS[name]
+    base, precision = split_name(name)
+    w = WORKLOADS[base]
     t0 = time.time()
     _, p = make_weights(w.dims, w.seed)
     lat, txt, ref = make_inputs(w)
     rows = rows_for(name)
     k = STEPS_RUN.get(name, w.n_steps)
     hp = O.hyper(w.dims)
+    if precision != "bf16":
+        hp[precision] = True
     ts = O.schedule(w.n_steps)
     tok = O.pack_latents(torch.from_numpy(lat)).float()
     refs = [] if ref is None else (ref if isinstance(ref, list) else [ref])
     ref_toks = [O.pack_latents(torch.from_numpy(r)).float() for r in refs]
     ref_grids = [(r.shape[1] // 2, r.shape[2] // 2) for r in refs]
     txt_u = torch.from_numpy(make_uncond_text(w)) if w.guidance is not None else None
+    extra = {}
+    if precision != "bf16":
+        tt = ts[1] if w.dims.flow_map else None
+        extra["v_pert"] = perturbed(precision, lambda: O3.forward3(
+            p, hp, tok, torch.from_numpy(txt), ts[0], (w.grid, w.grid), ref_toks, ref_grids, t_target=tt,
+            dtype=torch.float32))[rows].float().numpy()[None]
+        print(f"  {name} perturbed step 0 done at {time.time() - t0:.0f}s", flush=True)
     vs = []
     for i in range(k):
         tt = ts[i + 1] if w.dims.flow_map else None
@@ -88,38 +99,43 @@ def make3(name):
         vs.append(v[rows].float().numpy())
         tok = O.euler_update(tok, v, ts[i + 1] - ts[i])
         print(f"  {name} step {i} done at {time.time() - t0:.0f}s", flush=True)
-    meta = {"workload": name, "seed": w.seed, "oracle_dtype": "float32", "n_steps": w.n_steps, "steps_run": k,
-            "flow_map": bool(w.dims.flow_map), "guidance": w.guidance, "row_stride": ROW_STRIDE[name],
-            "seconds": round(time.time() - t0, 1)}
+    meta = {"workload": base, "precision": precision, "seed": w.seed, "oracle_dtype": "float32",
+            "n_steps": w.n_steps, "steps_run": k, "flow_map": bool(w.dims.flow_map), "guidance": w.guidance,
+            "row_stride": ROW_STRIDE[name], "seconds": round(time.time() - t0, 1)}
     np.savez(os.path.join(HERE, f"{name}.npz"), rows=rows, v=np.stack(vs), final=tok[rows].float().numpy(),
-             meta=np.array(json.dumps(meta)))
+             meta=np.array(json.dumps(meta)), **extra)
     print(f"{name}: wrote {len(rows)} rows x {k} steps in {time.time() - t0:.0f}s", flush=True)
 
 
-def perturbed_step0(p, hp, precision, lat, txt, ref, w):
-    """Step-0 velocity of the quantised oracle with every quantiser input perturbed by at most one
-    bf16 rounding (relative 2^-9, seeded uniform)."""
+def perturbed(precision, run):
+    """run() with every quantiser input of the oracle's FP8 / NVFP4 linears multiplied by
+    (1 + u 2^-9), u uniform in [-1, 1] from a generator seeded with 0 (one bf16 rounding's worth)."""
     from oracle import fp8_oracle as Q8
     from oracle import nvfp4_oracle as Q4
     mod, attr = (Q8, "linear_fp8") if precision == "fp8" else (Q4, "linear_nvfp4")
     plain = getattr(mod, attr)
     g = torch.Generator().manual_seed(0)
 
-    def perturbed(x, wt, b):
+    def perturbed_linear(x, wt, b):
         x = torch.as_tensor(x)
         u = torch.rand(x.shape, generator=g, dtype=torch.float64) * 2 - 1
         return plain(x * (1 + u * 2.0 ** -9).to(x.dtype), wt, b)
-    setattr(mod, attr, perturbed)
+    setattr(mod, attr, perturbed_linear)
     try:
-        tok = O.pack_latents(torch.from_numpy(lat)).float()
-        refs, grids = [], []
-        for r in ([] if ref is None else (ref if isinstance(ref, list) else [ref])):
-            refs.append(O.pack_latents(torch.from_numpy(r)).float())
-            grids.append((r.shape[1] // 2, r.shape[2] // 2))
-        return O.forward(p, hp, tok, torch.from_numpy(txt), O.schedule(w.n_steps)[0], (w.grid, w.grid), refs,
-                         grids, dtype=torch.float32)
+        return run()
     finally:
         setattr(mod, attr, plain)
+
+
+def perturbed_step0(p, hp, precision, lat, txt, ref, w):
+    """Step-0 velocity of the quantised FLUX.2 oracle with its quantiser inputs perturbed."""
+    tok = O.pack_latents(torch.from_numpy(lat)).float()
+    refs, grids = [], []
+    for r in ([] if ref is None else (ref if isinstance(ref, list) else [ref])):
+        refs.append(O.pack_latents(torch.from_numpy(r)).float())
+        grids.append((r.shape[1] // 2, r.shape[2] // 2))
+    return perturbed(precision, lambda: O.forward(p, hp, tok, torch.from_numpy(txt), O.schedule(w.n_steps)[0],
+                                                  (w.grid, w.grid), refs, grids, dtype=torch.float32))
 
 
 def make(name):

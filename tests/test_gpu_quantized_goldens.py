@@ -3,8 +3,8 @@
 * 1 double + 1 single block at the full 1024^2 token count (4608 rows: every GEMM segment, scale
   block and tile offset of the full-size path), against the oracle run live in float64, at the
   tiny models' bars (FP8 2e-2, NVFP4 3e-2; ratio to the exact forward below 0.6).
-* The whole 25-block sampler against the oracle's quantised goldens (tests/golden/<workload>_fp8,
-  _nvfp4, written by tests/golden/make_goldens.py from the oracle alone).  Over 25 blocks a
+* The whole 25-block sampler (FLUX.3: 33 blocks) against the oracle's quantised goldens
+  (tests/golden/<workload>_fp8, _nvfp4, written by tests/golden/make_goldens.py from the oracle alone).  Over 25 blocks a
   quantised forward is not continuous in its quantiser inputs: a bf16-sized perturbation of them
   moves the oracle's own step-0 velocity by sigma (FP8 about 3 %, NVFP4 about 12 % at 256^2), and
   the GPU path's bf16 attention operands are such a perturbation.  The golden stores the perturbed
@@ -163,3 +163,56 @@ def test_flux3_one_per_mode_one_joint_block_at_full_token_count(precision):
           f"vs exact {rel_l2(v, exact):.4f}, quantised oracle vs exact {rel_l2(want, exact):.4f}")
     assert err <= BLOCK_BARS[precision], err
     assert err < 0.6 * rel_l2(v, exact)
+
+
+@pytest.mark.parametrize("name", ["f3t2i256_fp8", "f3t2i256_nvfp4"])
+def test_flux3_quantised_sampler_against_quantised_oracle_golden(name):
+    """FLUX.3 Image Klein at 256^2 (5 per-mode + 28 joint blocks, flow-map target time), 4 steps with
+    quantised block linears, against the FLUX.3 oracle's quantised golden; bar 1.25 sigma as above."""
+    path = os.path.join(GOLDEN, f"{name}.npz")
+    if not os.path.exists(path):
+        pytest.skip(f"golden {path} not generated")
+    gd = np.load(path)
+    base, precision = name.rsplit("_", 1)
+    w = WORKLOADS[base]
+    meta = json.loads(str(gd["meta"]))
+    assert meta["workload"] == base and meta["precision"] == precision and meta["seed"] == w.seed
+    k = meta["steps_run"]
+    sigma = rel_l2(gd["v_pert"][0], gd["v"][0])
+    bar = SIGMA_FACTOR * sigma
+    blob, _ = make_weights(w.dims, w.seed)
+    lat, txt, _ = make_inputs(w)
+    model = F.Flux3DiT(blob, w.dims)
+    del blob
+    vs = []
+    try:
+        model.set_precision(PRECISION[precision])
+        ts = F.euler_schedule(w.n_steps)
+        tok = O.pack_latents(torch.from_numpy(lat)).float().to(DEV)
+        tx = torch.from_numpy(txt).to(DEV)
+        v = torch.empty(w.n_img, 128, device=DEV)
+        for i in range(k):
+            model.forward(tok, (w.grid, w.grid), tx, ts[i], v, t_target=ts[i + 1])
+            vs.append(v.cpu().clone())
+            F.flux_euler_step(tok, v, ts[i + 1] - ts[i])
+        final = tok.cpu()
+        torch.cuda.synchronize()
+        assert F.flux_device_error() == 0
+    finally:
+        model.close()
+    rows = torch.from_numpy(gd["rows"]).long()
+    print(f"{name}: sigma {sigma:.4f}, bar {bar:.4f}")
+    for i in range(k):
+        err = rel_l2(vs[i][rows], gd["v"][i])
+        print(f"{name} step {i} velocity vs golden {err:.4f}")
+        assert err <= bar, (i, err, bar)
+    err = rel_l2(final[rows], gd["final"])
+    print(f"{name} latent after {k} steps vs golden {err:.4f}")
+    assert err <= bar, err
+    exact_path = os.path.join(GOLDEN, f"{base}.npz")
+    if os.path.exists(exact_path):
+        ex = np.load(exact_path)
+        assert np.array_equal(ex["rows"], gd["rows"])
+        e0, x0 = rel_l2(vs[0][rows], gd["v"][0]), rel_l2(vs[0][rows], ex["v"][0])
+        print(f"{name} step 0: vs quantised golden {e0:.4f}, vs exact golden {x0:.4f}")
+        assert e0 < EXACT_RATIO * x0
