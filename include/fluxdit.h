@@ -26,6 +26,10 @@
  *   - Kernels never trap: a pipeline wait that exceeds one second makes the
  *     kernel stop, record a code in a device error word and return;
  *     flux_device_error() reads and clears it.
+ *   - Kernels are launched with programmatic dependent launch: a kernel's set-up
+ *     may overlap the end of the previous kernel on the stream, and it waits for
+ *     that kernel's completion before touching memory, so results do not change.
+ *     FLUX_PDL=0 in the environment (read at every launch) turns this off.
  */
 #ifndef FLUXDIT_H
 #define FLUXDIT_H
