@@ -666,7 +666,7 @@ def flux_quantize_rows_nvfp4(x, q, sf, row_scale, stream=None):
 
 
 def flux_layernorm_modulate_nvfp4(x, q, sf, row_scale, shift, scale, eps=1e-6, stream=None):
-    """LN + modulation of fp32 x [rows, dim], rounded to bf16 and quantised to NVFP4 (q [rows, dim/2],
+    """LN + modulation of fp32 x [rows, dim], the float32 results quantised to NVFP4 (q [rows, dim/2],
     sf [flux_nvfp4_scale_bytes(rows, dim)], row_scale [rows])."""
     import torch
     rows, dim = x.shape

@@ -15,7 +15,6 @@
 //          so that 32 rows of 16 bytes, copied to tensor memory and broadcast to the four lane
 //          quarters, put row r's four scales in lane r, column r/32 of the block's four columns;
 //   row scales fp32 [rows].
-#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -79,8 +78,16 @@ __device__ __forceinline__ __nv_fp8_storage_t q4_block_scale(float bmax, float i
   return s8;
 }
 
+// Two e2m1 codes, a * rcp in the low nibble and b * rcp in the high one, by the sm_100a conversion
+// instruction (nearest even, saturating at +-6; it places its first source in the high nibble).
+// The toolkit's conversion helper emulates this in integer arithmetic unless the family-specific
+// target macro is defined, which an sm_100a build does not define.
 __device__ __forceinline__ uint32_t e2m1x2(float a, float b, float rcp) {
-  return __nv_cvt_float2_to_fp4x2(make_float2(__fmul_rn(a, rcp), __fmul_rn(b, rcp)), __NV_E2M1, cudaRoundNearest);
+  uint32_t r;
+  asm("{\n\t.reg .b8 c;\n\tcvt.rn.satfinite.e2m1x2.f32 c, %2, %1;\n\tcvt.u32.u8 %0, c;\n}"
+      : "=r"(r)
+      : "f"(__fmul_rn(a, rcp)), "f"(__fmul_rn(b, rcp)));
+  return r;
 }
 
 // Byte offset of the scale of 16-element block g of scale-layout row sfr (k elements per row).
