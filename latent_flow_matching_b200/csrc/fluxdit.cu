@@ -861,6 +861,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
   // its output per segment in the same pass).
   const bool fp8 = m->precision == FLUX_PRECISION_FP8;
   const bool fp4 = m->precision == FLUX_PRECISION_NVFP4;
+  const OpFormat lin_fmt = fp4 ? OpFormat::kNvfp4 : fp8 ? OpFormat::kE4M3 : OpFormat::kBf16;
   auto f8 = [&](int i, const CUtensorMap& a8, const CUtensorMap& w8, const float* sa, const float* sb) {
     P.mapA[i] = a8;
     P.mapB[i] = w8;
@@ -928,7 +929,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
         fp4_operands(P4, 2 * b + 1, w.y4_img[b], si.q4_qkv);
       }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear());
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P, lin_fmt), linear());
     FD_LAUNCH(m, kProfAttention, at_flops, at_bytes, attention_launch(A, s));
     if (fp8 && (rc = quant_cc(0, D, w.sO))) return rc;
     if (fp4 && (rc = quant4(w.CC, D + F, D, w.C4, (D + F) / 2, w.sfO, w.sO4, w.seg_dbl))) return rc;
@@ -947,7 +948,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
         fp4_operands(P4, 2 * b + 1, w.o4_img[b], si.q4_proj);
       }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear());
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P, lin_fmt), linear());
     rc = ln_mod(nt, mt + 3 * D, mt + 4 * D, mi + 3 * D, mi + 4 * D, w.seg_dbl);
     if (rc) return rc;
     P.num_problems = 2 * nb;
@@ -965,7 +966,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
         fp4_operands(P4, 2 * b + 1, w.y4_img[b], si.q4_mlp_in);
       }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear());
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P, lin_fmt), linear());
     if (fp8 && (rc = quant_cc(D, F, w.sH))) return rc;
     if (fp4 && (rc = quant4(w.CC + D, D + F, F, w.C4 + D / 2, (D + F) / 2, w.sfH, w.sH4, w.seg_dbl))) return rc;
     P.num_problems = 2 * nb;
@@ -983,7 +984,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
         fp4_operands(P4, 2 * b + 1, w.h4_img[b], si.q4_mlp_out);
       }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear());
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P, lin_fmt), linear());
   }
   // single blocks: one set of weights for every row, so the whole batch is one problem
   for (int i = 0; i < m->act_single; ++i) {
@@ -1004,7 +1005,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
       fp4_operands(P4, 0, w.y4_all, sw.q4_qkv);
       fp4_operands(P4, 1, w.y4_all, sw.q4_mlp);
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear());
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P, lin_fmt), linear());
     FD_LAUNCH(m, kProfAttention, at_flops, at_bytes, attention_launch(A, s));
     if (fp8 && (rc = quant_cc(0, D + F, w.sC))) return rc;
     if (fp4 && (rc = quant4(w.CC, D + F, D + F, w.C4, (D + F) / 2, w.sfC, w.sC4, w.seg_all))) return rc;
@@ -1012,7 +1013,7 @@ static int forward_impl(flux_dit* m, const float* img_tok, int gh, int gw, const
     problem(P, 0, w.a_CC, sw.m_lin2, rows, D, D + F, kEpiResidGate, w.X, D, sw.lin2_b, ms + 2 * D);
     if (fp8) f8(0, w.a8_CC, sw.m8_lin2, w.sC, sw.s_lin2);
     if (fp4) fp4_operands(P4, 0, w.c4_all, sw.q4_lin2);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear());
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P, lin_fmt), linear());
   }
   // output layer on the image rows of each sequence
   const NvtxRange range("output layer");

@@ -716,6 +716,7 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
   // NVFP4 precision: LN-mod quantises its output per segment (`segs`) in the same pass; [O | H] is
   // quantised per segment before linear2
   const bool fp4 = m->precision == FLUX_PRECISION_NVFP4;
+  const OpFormat lin_fmt = fp4 ? OpFormat::kNvfp4 : fp8 ? OpFormat::kE4M3 : OpFormat::kBf16;
   auto linear_as = [&](bool small) -> cudaError_t {
     return fp4 ? gemm_fp4_launch(P4, m->num_sms, s) : launch_linear_as(P, m->num_sms, s, fp8, small);
   };
@@ -790,7 +791,7 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
     };
     for (int sg = 0; sg < 3; ++sg) lin1(sg, 0);
     for (int bb = 1; bb < nb; ++bb) lin1(kSegTxt, static_cast<size_t>(bb) * n);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear_as(false));   // SwiGLU: pair kernel
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P, lin_fmt), linear_as(false));   // SwiGLU: pair kernel
     FD_LAUNCH(m, kProfAttention, seg_flops, 8.0 * rows_pm * D, attention_launch(As, s));
     if (fp8 && (rc = quant_cc(rows_pm))) return rc;
     if (fp4 && (rc = quant4(w.CC, D + F, w.C4, w.sfC, w.sC4, w.seg_pm))) return rc;
@@ -807,7 +808,7 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
     for (int sg = 0; sg < 3; ++sg) lin2(sg, 0);
     const bool small = small_linear(P, m->num_sms, fp8, 1);
     for (int bb = 1; bb < nb; ++bb) lin2(kSegTxt, static_cast<size_t>(bb) * n);
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear_as(small));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P, lin_fmt), linear_as(small));
   }
   // the image and reference streams of sequence 0 into the other sequences
   for (int bb = 1; bb < nb; ++bb)
@@ -843,7 +844,7 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
         fp4_operands(P4, 2 * bb + 1, w.y4_all[bb], bw.q4_mlp);
       }
     }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear_as(small_linear(P, m->num_sms, fp8, nb)));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P, lin_fmt), linear_as(small_linear(P, m->num_sms, fp8, nb)));
     FD_LAUNCH(m, kProfAttention, at_flops, 8.0 * rows_all * D, attention_launch(A, s));
     if (fp8 && (rc = quant_cc(rows_all))) return rc;
     if (fp4 && (rc = quant4(w.CC, D + F, w.C4, w.sfC, w.sC4, w.seg_jc))) return rc;
@@ -856,7 +857,7 @@ int forward3_impl(flux3_dit* m, const float* img_tok, int gh, int gw, const floa
         if (fp8) f8(3 * bb + sg, w.a8_CCseg[bb][sg], bw.m8_lin2, w.sC + r, bw.s_lin2);
         if (fp4) fp4_operands(P4, 3 * bb + sg, w.c4_seg[bb][sg], bw.q4_lin2);
       }
-    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P), linear_as(small_linear(P, m->num_sms, fp8, nb)));
+    FD_LAUNCH(m, kProfGemm, gemm_flops(P), gemm_bytes(P, lin_fmt), linear_as(small_linear(P, m->num_sms, fp8, nb)));
   }
 
   // ---------------- output layer on the image rows (text and reference tokens are dropped)

@@ -103,13 +103,26 @@ inline double gemm_flops(const GemmParams& P) {
     if (P.prob[i].M > 0) f += 2.0 * P.prob[i].M * static_cast<double>(P.prob[i].N) * P.prob[i].K;
   return f;
 }
-inline double gemm_bytes(const GemmParams& P) {
+// Operand storage of a linear: bf16 (2 bytes per element), e4m3 codes (1 byte) or NVFP4 (half a
+// byte of code plus one e4m3 block scale per 16 elements); the quantised formats also read one
+// fp32 row scale per row of A and of W.
+enum class OpFormat { kBf16, kE4M3, kNvfp4 };
+// Algorithmic bytes of a launch: A and W read once, the output written once (bf16 for the bias and
+// the fused QK-norm + RoPE modes; the SwiGLU writes half the columns in bf16; fp32; the gated
+// residual reads and writes its fp32 rows).
+inline double gemm_bytes(const GemmParams& P, OpFormat f = OpFormat::kBf16) {
+  const double elt = f == OpFormat::kBf16 ? 2.0 : f == OpFormat::kE4M3 ? 1.0 : 0.5 + 1.0 / 16.0;
+  const double row = f == OpFormat::kBf16 ? 0.0 : 4.0;
   double b = 0;
   for (int i = 0; i < P.num_problems; ++i) {
     const GemmProblem& pr = P.prob[i];
     if (pr.M <= 0) continue;
-    const double out_elt = pr.mode == kEpiBf16Bias ? 2 : pr.mode == kEpiSwiGLU ? 1 : pr.mode == kEpiF32Bias ? 4 : 8;
-    b += 2.0 * pr.M * pr.K + 2.0 * pr.N * pr.K + out_elt * pr.M * pr.N;
+    const double out_elt = pr.mode == kEpiBf16Bias || pr.mode == kEpiQKNormRope ? 2
+                           : pr.mode == kEpiSwiGLU                             ? 1
+                           : pr.mode == kEpiF32Bias                            ? 4
+                                                                               : 8;   // gated residual
+    b += elt * (static_cast<double>(pr.M) * pr.K + static_cast<double>(pr.N) * pr.K) + row * (pr.M + pr.N) +
+         out_elt * pr.M * static_cast<double>(pr.N);
   }
   return b;
 }

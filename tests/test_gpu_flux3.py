@@ -121,6 +121,51 @@ def _gpu_forward(model, tok, grid, txt, t, refs, ref_grids, t_target):
     return v
 
 
+@pytest.mark.parametrize("precision", [F.PRECISION_BF16, F.PRECISION_FP8, F.PRECISION_NVFP4])
+def test_tiny3_profile_counts_the_algorithmic_work(tiny3, precision):
+    """The profiling hook's FLOPs and bytes for a forward with a reference equal the closed forms:
+    per block N 2D(4D + 3F) of linears; attention 4 D (Nt^2 + Ni^2 + Nr^2) in a per-mode block (each
+    stream within itself) and 4 N^2 D in a joint block; GEMM bytes with A and W read once in the
+    format that runs and each output written once (bf16 2 bytes; the SwiGLU half the columns in
+    bf16; fp32 4; the gated residual's fp32 rows read and written)."""
+    w, p, model = tiny3
+    d = w.dims
+    D, Fh, C, T = d.hidden, d.mlp_hidden, d.in_ch, d.txt_dim
+    tok, txt, refs = _tiny_inputs(11, 16, (4, 4), [(4, 4)])
+    nt, ni, nr = 16, 16, 16
+    n = nt + ni + nr
+    elt, row = {F.PRECISION_BF16: (2.0, 0.0), F.PRECISION_FP8: (1.0, 4.0),
+                F.PRECISION_NVFP4: (0.5 + 1.0 / 16.0, 4.0)}[precision]
+
+    def lb(m, k, nn, out_per_elt, e=elt, r=row):
+        return e * (m * k + nn * k) + r * (m + nn) + out_per_elt * m * nn
+
+    segs = (nt, ni, nr)
+    mode_bytes = sum(lb(g, D, 3 * D, 2) + lb(g, D, 2 * Fh, 1) + lb(g, D + Fh, D, 8) for g in segs)
+    joint_bytes = lb(n, D, 3 * D, 2) + lb(n, D, 2 * Fh, 1) + sum(lb(g, D + Fh, D, 8) for g in segs)
+    io = lb(nt, T, D, 4, 2.0, 0.0) + lb(ni + nr, C, D, 4, 2.0, 0.0) + lb(ni, D, C, 4, 2.0, 0.0)
+    want_bytes = d.n_mode * mode_bytes + d.n_joint * joint_bytes + io
+    want_flops = ((d.n_mode + d.n_joint) * n * 2.0 * D * (4 * D + 3 * Fh) + 2.0 * (ni + nr) * C * D +
+                  2.0 * nt * T * D + 2.0 * ni * D * C)
+    want_attn = d.n_mode * 4.0 * D * sum(g * g for g in segs) + d.n_joint * 4.0 * n * n * D
+    model.set_precision(precision)
+    try:
+        _gpu_forward(model, tok, (4, 4), txt, 0.6, refs, [(4, 4)], 0.35)
+        model.profile(True)
+        _gpu_forward(model, tok, (4, 4), txt, 0.6, refs, [(4, 4)], 0.35)
+        prof = model.profile_read()
+    finally:
+        model.profile(False)
+        model.set_precision(F.PRECISION_BF16)
+    _, g_fl, g_by, g_n = prof["gemm"]
+    _, a_fl, _, a_n = prof["attention"]
+    assert g_n == 2 * (d.n_mode + d.n_joint) + 2
+    assert a_n == d.n_mode + d.n_joint
+    assert g_fl == pytest.approx(want_flops, rel=1e-12)
+    assert a_fl == pytest.approx(want_attn, rel=1e-12)
+    assert g_by == pytest.approx(want_bytes, rel=1e-12)
+
+
 @pytest.mark.parametrize("precision", ["bf16", "nvfp4"])
 def test_tiny3_programmatic_launches_change_nothing(tiny3, precision, monkeypatch):
     """FLUX.3 forward with a reference (segmented per-mode attention, three-region LN-mod) with and

@@ -193,6 +193,56 @@ def test_sampling_step_replayed_from_a_cuda_graph_equals_plain_launches(tiny):
     assert F.flux_device_error() == 0
 
 
+@pytest.mark.parametrize("precision", [F.PRECISION_BF16, F.PRECISION_FP8, F.PRECISION_NVFP4])
+def test_profile_counts_the_algorithmic_work(tiny, precision):
+    """The profiling hook's FLOPs and bytes (from which the benchmark's rooflines are computed) equal
+    the closed forms for the tiny model: per block N 2D(4D + 3F) of linears and 4 N^2 D of attention,
+    the input and output projections; GEMM bytes read A and W once in the format that runs (bf16 2
+    bytes, e4m3 1, NVFP4 1/2 + 1/16 per element, the quantised formats plus a 4-byte scale per row)
+    and write each output once (bf16 2 bytes, SwiGLU half the columns in bf16, fp32 4, the gated
+    residual's fp32 rows read and written)."""
+    w, p, model = tiny
+    d = w.dims
+    D, Fh, C, T = d.hidden, d.mlp_hidden, d.in_ch, d.txt_dim
+    ni, nt = w.n_img, w.n_txt
+    n = ni + nt
+    blocks = d.n_double + d.n_single
+    lat, txt, _ = make_inputs(w)
+    tok = O.pack_latents(torch.from_numpy(lat)).float().to(DEV)
+    v = torch.empty(ni, 128, device=DEV)
+    elt, row = {F.PRECISION_BF16: (2.0, 0.0), F.PRECISION_FP8: (1.0, 4.0),
+                F.PRECISION_NVFP4: (0.5 + 1.0 / 16.0, 4.0)}[precision]
+
+    def linear_bytes(m, k, nn, out_per_elt, e=elt, r=row):
+        return e * (m * k + nn * k) + r * (m + nn) + out_per_elt * m * nn
+
+    blk = 0.0
+    for rows in (nt, ni):                       # double block, per stream
+        blk += linear_bytes(rows, D, 3 * D, 2) + linear_bytes(rows, D, D, 8)
+        blk += linear_bytes(rows, D, 2 * Fh, 1) + linear_bytes(rows, Fh, D, 8)
+    sgl = linear_bytes(n, D, 3 * D, 2) + linear_bytes(n, D, 2 * Fh, 1) + linear_bytes(n, D + Fh, D, 8)
+    io = (linear_bytes(nt, T, D, 4, 2.0, 0.0) + linear_bytes(ni, C, D, 4, 2.0, 0.0) +
+          linear_bytes(ni, D, C, 4, 2.0, 0.0))
+    want_bytes = d.n_double * blk + d.n_single * sgl + io
+    want_flops = blocks * n * 2.0 * D * (4 * D + 3 * Fh) + 2.0 * ni * C * D + 2.0 * nt * T * D + 2.0 * ni * D * C
+    model.set_precision(precision)
+    try:
+        model.forward(tok, (w.grid, w.grid), torch.from_numpy(txt).to(DEV), 0.5, v)
+        model.profile(True)
+        model.forward(tok, (w.grid, w.grid), torch.from_numpy(txt).to(DEV), 0.5, v)
+        prof = model.profile_read()
+    finally:
+        model.profile(False)
+        model.set_precision(F.PRECISION_BF16)
+    _, g_fl, g_by, g_n = prof["gemm"]
+    _, a_fl, _, a_n = prof["attention"]
+    assert g_n == 4 * d.n_double + 2 * d.n_single + 2
+    assert a_n == blocks
+    assert g_fl == pytest.approx(want_flops, rel=1e-12)
+    assert a_fl == pytest.approx(blocks * 4.0 * n * n * D, rel=1e-12)
+    assert g_by == pytest.approx(want_bytes, rel=1e-12)
+
+
 @pytest.mark.parametrize("n_txt,grid,ref_grid", [(0, (4, 6), (0, 0)), (5, (6, 4), (4, 4)), (131, (8, 8), (4, 8))])
 def test_tiny_forward_ragged_and_degenerate_shapes(tiny, n_txt, grid, ref_grid):
     """No text, non-square grids, a reference of another size, sequence lengths off the 128-row tiles."""
