@@ -13,7 +13,10 @@
 //     of all 256 tile columns (4 KB, the MMA of each CTA multiplies by every column's scales);
 //     before every MMA the issuing lane copies that MMA's scales from shared to tensor memory
 //     (tcgen05.cp 32x128b.warpx4: 32 rows of 16 bytes broadcast to the four lane quarters, one
-//     copy per 128 rows), into one of two 12-column slots used in turn;
+//     copy per 128 rows), into one of two 12-column slots used in turn.  A stage's four MMAs and
+//     twelve copies go out from one elected lane in a single block (one election, descriptor
+//     offsets added in place): the issuing thread takes about 100 cycles per MMA with its copies
+//     against the MMA's 128 tensor cycles, so its issue rate bounds how far it runs ahead;
 //   * tensor memory holds two 256-column accumulators and the scale slots in 512 columns only
 //     if the accumulators overlap: buffer 0 is columns [0, 256), buffer 1 [224, 480), the scale
 //     slots [480, 512).  The epilogue part that owns the 32 shared columns drains them first and
@@ -78,26 +81,43 @@ __device__ __forceinline__ uint64_t sf_desc(uint32_t smem_addr) {
   return d;                                         // layout type 0: no swizzle
 }
 
-// Warp-collective scale copy on the pair (one elected lane issues; both CTAs copy from their own
-// shared memory into their own tensor memory).
-__device__ __forceinline__ void sf_copy_pair_warp(uint32_t taddr, uint64_t sdesc) {
+// One stage's four MMAs and their scale copies, issued by one elected lane in a single block:
+// MMA k (K elements 64k..64k+63) takes its A/W descriptors advanced by 32k bytes and its scale
+// blocks advanced by 512k bytes (W's second 128 columns 2048 bytes further), and uses scale slot
+// k & 1 (sf0 / sf1: SFA at +0, the two SFB halves at +4 and +8 columns).  acc0 = 0 only for the
+// first stage of a tile.
+__device__ __forceinline__ void stage_issue_nvf4(uint32_t d_tmem, uint64_t ad, uint64_t bd, uint64_t sad, uint64_t sbd,
+                                                 uint32_t idesc, uint32_t acc0, uint32_t sf0, uint32_t sf1) {
   asm volatile(
-      "{\n\t.reg .pred e;\n\t"
+      "{\n\t.reg .pred p, t, e;\n\t"
+      ".reg .b64 a, b, sa, sb, sc;\n\t"
+      ".reg .b32 f0b, f0c, f1b, f1c;\n\t"
       "elect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr),
-      "l"(sdesc)
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "setp.eq.b32 t, %6, %6;\n\t"
+      "add.u32 f0b, %7, 4;\n\tadd.u32 f0c, %7, 8;\n\tadd.u32 f1b, %8, 4;\n\tadd.u32 f1c, %8, 8;\n\t"
+      "add.s64 sc, %4, 128;\n\t"
+      "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [%7], %3;\n\t"
+      "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [f0b], %4;\n\t"
+      "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [f0c], sc;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %5, [%7], [f0b], p;\n\t"
+      "add.s64 a, %1, 2;\n\tadd.s64 b, %2, 2;\n\tadd.s64 sa, %3, 32;\n\tadd.s64 sb, %4, 32;\n\tadd.s64 sc, %4, 160;\n\t"
+      "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [%8], sa;\n\t"
+      "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [f1b], sb;\n\t"
+      "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [f1c], sc;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], a, b, %5, [%8], [f1b], t;\n\t"
+      "add.s64 a, %1, 4;\n\tadd.s64 b, %2, 4;\n\tadd.s64 sa, %3, 64;\n\tadd.s64 sb, %4, 64;\n\tadd.s64 sc, %4, 192;\n\t"
+      "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [%7], sa;\n\t"
+      "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [f0b], sb;\n\t"
+      "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [f0c], sc;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], a, b, %5, [%7], [f0b], t;\n\t"
+      "add.s64 a, %1, 6;\n\tadd.s64 b, %2, 6;\n\tadd.s64 sa, %3, 96;\n\tadd.s64 sb, %4, 96;\n\tadd.s64 sc, %4, 224;\n\t"
+      "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [%8], sa;\n\t"
+      "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [f1b], sb;\n\t"
+      "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [f1c], sc;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], a, b, %5, [%8], [f1b], t;\n\t}" ::"r"(d_tmem),
+      "l"(ad), "l"(bd), "l"(sad), "l"(sbd), "r"(idesc), "r"(acc0), "r"(sf0), "r"(sf1)
       : "memory");
-}
-
-__device__ __forceinline__ void mma_pair_nvf4_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                                   uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
-          d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb));
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads4, 1)
@@ -213,7 +233,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads4, 1)
       const uint64_t b_desc0 = sw128_desc(smem_u32(sB), 16, 1024);
       const uint64_t sfa_desc0 = sf_desc(smem_u32(sSFA));
       const uint64_t sfb_desc0 = sf_desc(smem_u32(sSFB));
-      uint32_t slot = 0;
       for (int tile = pair; ok && tile < P.total_tiles; tile += num_pairs) {
         const int p = find_problem(P, tile);
         const int nk = P.prob[p].K / BKE;
@@ -241,16 +260,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads4, 1)
           const uint64_t bd = desc_advance(b_desc0, stage * B_BYTES);
           const uint64_t sad = desc_advance(sfa_desc0, stage * SFA_BYTES);
           const uint64_t sbd = desc_advance(sfb_desc0, stage * SFB_BYTES);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {                  // 64 elements (32 bytes) of K per MMA
-            const uint32_t sfa = tmem_base + kSfCol + 16 * slot;
-            sf_copy_pair_warp(sfa, desc_advance(sad, k * 512));
-            sf_copy_pair_warp(sfa + 4, desc_advance(sbd, k * 512));
-            sf_copy_pair_warp(sfa + 8, desc_advance(sbd, SFB_BYTES / 2 + k * 512));
-            mma_pair_nvf4_warp(d_tmem, desc_advance(ad, k * 32), desc_advance(bd, k * 32), idesc, sfa, sfa + 4,
-                               (kb | k) != 0 ? 1u : 0u);
-            slot ^= 1u;
-          }
+          stage_issue_nvf4(d_tmem, ad, bd, sad, sbd, idesc, kb != 0 ? 1u : 0u, tmem_base + kSfCol,
+                           tmem_base + kSfCol + 16);
           mma_commit_pair_warp(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
