@@ -64,6 +64,11 @@ typedef struct {
 /* Last error message of the calling thread ("" if none).  Valid until the next call. */
 FLUX_API const char *flux_get_error(void);
 
+/* Code (FLUX_EINVAL, FLUX_ENOMEM, FLUX_EIO) of the calling thread's last failure, 0 if none has
+ * happened: lets a caller of a pointer-returning call (flux_dit_create, flux3_dit_create) tell a
+ * device out of memory from a bad argument. */
+FLUX_API int flux_get_error_code(void);
+
 /* Bytes of a weight blob for `cfg` (header + tensors), or 0 if cfg is invalid.
  *
  * Blob format (little endian): a 256-byte header
@@ -485,6 +490,16 @@ FLUX_API int flux_device_error(void *stream);
  * device error word and returns normally, leaving the context usable; flux_device_error() then
  * reports and clears it.  Asynchronous on `stream`; no memory arguments. */
 FLUX_API int flux_selftest_bounded_wait(unsigned long long limit_ns, int arrive, void *stream);
+
+/* Test hook for the out-of-memory path (same convention: hakusoku.com story 4662,
+ * "エラーハンドリング").  After this call the library's next n device allocations succeed and
+ * the one after them fails as if the device were out of memory (n = 0: the very next one); the
+ * hook then disarms itself.  n < 0 disarms it at once.  Every entry point that allocates (model
+ * creation, the first forward at a larger token count or a new precision, timestep preparation)
+ * then returns FLUX_ENOMEM with a message in flux_get_error(), frees what it had allocated in that
+ * call and leaves the model as it was, so that a later call succeeds.  Process-wide; no device
+ * work. */
+FLUX_API void flux_test_fail_alloc_after(long long n);
 
 #ifdef __cplusplus
 }

@@ -59,6 +59,7 @@ class FluxShapeError(FluxError, ValueError):
 _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 _SIGS = {
     "flux_get_error": (ctypes.c_char_p, []),
+    "flux_get_error_code": (_I, []),
     "flux_blob_expected_bytes": (_Z, [ctypes.POINTER(FluxConfig)]),
     "flux_dit_create": (_P, [_P, _Z, ctypes.POINTER(FluxConfig), _P]),
     "flux_dit_destroy": (None, [_P]),
@@ -69,6 +70,7 @@ _SIGS = {
     "flux_cfg_euler_step": (_I, [_P, _P, _P, _Z, _F, _F, _P]),
     "flux_cfg_euler_step_out": (_I, [_P, _P, _P, _P, _Z, _F, _F, _P]),
     "flux_selftest_bounded_wait": (_I, [ctypes.c_ulonglong, _I, _P]),
+    "flux_test_fail_alloc_after": (None, [ctypes.c_longlong]),
     "flux_blend_latents": (_I, [_P, _P, _F, _P, _Z, _P]),
     "flux_dit_set_active_blocks": (_I, [_P, _I, _I]),
     "flux_dit_modulation_size": (_Z, [_P]),
@@ -256,7 +258,7 @@ class FluxDiT:
         cfg = ctypes.byref(FluxConfig.from_dims(dims)) if dims is not None else None
         h = lib().flux_dit_create(ctypes.c_void_p(blob.ctypes.data), blob.nbytes, cfg, _stream(stream))
         if not h:
-            raise FluxError(FLUX_EINVAL, get_error())
+            raise FluxError(lib().flux_get_error_code() or FLUX_EINVAL, get_error())
         self._h = ctypes.c_void_p(h)
         self.dims = dims
 
@@ -376,7 +378,7 @@ class Flux3DiT:
         cfg = ctypes.byref(Flux3Config.from_dims(dims)) if dims is not None else None
         h = lib().flux3_dit_create(ctypes.c_void_p(blob.ctypes.data), blob.nbytes, cfg, _stream(stream))
         if not h:
-            raise FluxError(FLUX_EINVAL, get_error())
+            raise FluxError(lib().flux_get_error_code() or FLUX_EINVAL, get_error())
         self._h = ctypes.c_void_p(h)
         self.dims = dims
         self.flow_map = bool(dims.flow_map) if dims is not None else True
@@ -789,6 +791,12 @@ def flux_selftest_bounded_wait(limit_ns: int, arrive: bool, stream=None):
     """One CTA waits on an mbarrier through the pipelines' bounded wait; with arrive=False nothing
     arrives and the kernel gives up after limit_ns, recording DEVERR_TIMEOUT_SELFTEST."""
     _check(lib().flux_selftest_bounded_wait(int(limit_ns), 1 if arrive else 0, _stream(stream)))
+
+
+def flux_test_fail_alloc_after(n: int):
+    """Test hook: the library's next n device allocations succeed and the one after them fails as
+    if the device were out of memory (then the hook disarms itself); n < 0 disarms it."""
+    lib().flux_test_fail_alloc_after(int(n))
 
 
 def flux_sample(model: FluxDiT, latent, txt, n_steps, ref_latent=None, on_step=None, stream=None,

@@ -37,6 +37,7 @@ namespace fdit {
 
 // ------------------------------------------------------------------ errors
 static thread_local std::string g_error;
+static thread_local int g_error_code = 0;
 
 int fail(int code, const char* fmt, ...) {
   char buf[512];
@@ -45,12 +46,14 @@ int fail(int code, const char* fmt, ...) {
   vsnprintf(buf, sizeof(buf), fmt, ap);
   va_end(ap);
   g_error = buf;
+  g_error_code = code;
   return code;
 }
 
 int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
 
 const char* last_error() { return g_error.c_str(); }
+int last_error_code() { return g_error_code; }
 
 // ------------------------------------------------------------------ tensor maps
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -146,6 +149,38 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 bool pdl_enabled() {
   const char* v = std::getenv("FLUX_PDL");
   return !(v && v[0] == '0' && v[1] == 0);
+}
+
+// Allocations that still succeed before the injected failure (-1: none injected).
+static std::atomic<long long> g_fail_alloc_after{-1};
+
+static bool injected_alloc_failure() {
+  long long n = g_fail_alloc_after.load();
+  while (n >= 0)
+    if (g_fail_alloc_after.compare_exchange_weak(n, n - 1)) return n == 0;
+  return false;
+}
+
+cudaError_t dev_alloc(void** p, size_t bytes) {
+  *p = nullptr;
+  if (injected_alloc_failure()) return cudaErrorMemoryAllocation;
+  const cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    *p = nullptr;
+    cudaGetLastError();
+  }
+  return e;
+}
+
+cudaError_t dev_alloc_async(void** p, size_t bytes, cudaStream_t s) {
+  *p = nullptr;
+  if (injected_alloc_failure()) return cudaErrorMemoryAllocation;
+  const cudaError_t e = cudaMallocAsync(p, bytes, s);
+  if (e != cudaSuccess) {
+    *p = nullptr;
+    cudaGetLastError();
+  }
+  return e;
 }
 
 // ------------------------------------------------------------------ blob layout
@@ -394,11 +429,11 @@ static int create_impl(const void* blob, size_t blob_bytes, const flux_dit_confi
     destroy(m);
     return fail(code, "%s", what);
   };
-  if (cudaMalloc(&m->wbuf, wbytes) != cudaSuccess || cudaMalloc(&m->mods_w, mrows * D * 2) != cudaSuccess ||
-      cudaMalloc(&m->mods_b, mrows * 2) != cudaSuccess || cudaMalloc(&m->temb, c.t_freq_dim * 4) != cudaSuccess ||
-      cudaMalloc(&m->th, D * 4) != cudaSuccess || cudaMalloc(&m->vec, D * 4) != cudaSuccess ||
-      cudaMalloc(&m->mods, mrows * 4) != cudaSuccess)
-    return cleanup(FLUX_ENOMEM, "cudaMalloc of model weights failed");
+  if (dev_alloc(&m->wbuf, wbytes) != cudaSuccess || dev_alloc(&m->mods_w, mrows * D * 2) != cudaSuccess ||
+      dev_alloc(&m->mods_b, mrows * 2) != cudaSuccess || dev_alloc(&m->temb, c.t_freq_dim * 4) != cudaSuccess ||
+      dev_alloc(&m->th, D * 4) != cudaSuccess || dev_alloc(&m->vec, D * 4) != cudaSuccess ||
+      dev_alloc(&m->mods, mrows * 4) != cudaSuccess)
+    return cleanup(FLUX_ENOMEM, "device allocation of the model weights failed");
 
   uint8_t* wb = static_cast<uint8_t*>(m->wbuf);
   size_t mrow = 0;
@@ -499,9 +534,9 @@ static int prepare_fp8(flux_dit* m, int nt, int nimg, int nb) {
   const size_t n = nt + nimg, rows = n * nb;
   if (rows > w.cap8) {
     free_ws8(w);
-    bool ok = cudaMalloc(&w.Y8, rows * D) == cudaSuccess && cudaMalloc(&w.C8, rows * (D + F)) == cudaSuccess &&
-              cudaMalloc(&w.sY, rows * 4) == cudaSuccess && cudaMalloc(&w.sC, rows * 4) == cudaSuccess &&
-              cudaMalloc(&w.sO, rows * 4) == cudaSuccess && cudaMalloc(&w.sH, rows * 4) == cudaSuccess;
+    bool ok = dev_alloc(&w.Y8, rows * D) == cudaSuccess && dev_alloc(&w.C8, rows * (D + F)) == cudaSuccess &&
+              dev_alloc(&w.sY, rows * 4) == cudaSuccess && dev_alloc(&w.sC, rows * 4) == cudaSuccess &&
+              dev_alloc(&w.sO, rows * 4) == cudaSuccess && dev_alloc(&w.sH, rows * 4) == cudaSuccess;
     if (!ok) {
       free_ws8(w);
       return fail(FLUX_ENOMEM, "FP8 workspace allocation for %zu tokens failed", rows);
@@ -555,12 +590,12 @@ static int prepare_fp4(flux_dit* m, int nt, int nimg, int nb) {
   if (static_cast<size_t>(rows) > w.cap4_rows || blocks > w.cap4_blocks) {
     free_ws4(w);
     const size_t R = rows, B = blocks * 128;
-    const bool ok = cudaMalloc(&w.Y4, R * D / 2) == cudaSuccess && cudaMalloc(&w.C4, R * (D + F) / 2) == cudaSuccess &&
-                    cudaMalloc(&w.sfY, B * D / 16) == cudaSuccess && cudaMalloc(&w.sfO, B * D / 16) == cudaSuccess &&
-                    cudaMalloc(&w.sfH, B * F / 16) == cudaSuccess &&
-                    cudaMalloc(&w.sfC, B * (D + F) / 16) == cudaSuccess && cudaMalloc(&w.sY4, R * 4) == cudaSuccess &&
-                    cudaMalloc(&w.sO4, R * 4) == cudaSuccess && cudaMalloc(&w.sH4, R * 4) == cudaSuccess &&
-                    cudaMalloc(&w.sC4, R * 4) == cudaSuccess;
+    const bool ok = dev_alloc(&w.Y4, R * D / 2) == cudaSuccess && dev_alloc(&w.C4, R * (D + F) / 2) == cudaSuccess &&
+                    dev_alloc(&w.sfY, B * D / 16) == cudaSuccess && dev_alloc(&w.sfO, B * D / 16) == cudaSuccess &&
+                    dev_alloc(&w.sfH, B * F / 16) == cudaSuccess &&
+                    dev_alloc(&w.sfC, B * (D + F) / 16) == cudaSuccess && dev_alloc(&w.sY4, R * 4) == cudaSuccess &&
+                    dev_alloc(&w.sO4, R * 4) == cudaSuccess && dev_alloc(&w.sH4, R * 4) == cudaSuccess &&
+                    dev_alloc(&w.sC4, R * 4) == cudaSuccess;
     if (!ok) {
       free_ws4(w);
       return fail(FLUX_ENOMEM, "NVFP4 workspace allocation for %d tokens failed", rows);
@@ -603,12 +638,12 @@ static int prepare_shape(flux_dit* m, int nt, int gh, int gw, const RefGrids& re
   if (rows > w.cap_n) {
     float* X = nullptr;
     free_ws(w);
-    bool ok = cudaMalloc(&X, rows * D * 4) == cudaSuccess;
+    bool ok = dev_alloc(&X, rows * D * 4) == cudaSuccess;
     w.X = X;
-    ok = ok && cudaMalloc(&w.Y, rows * D * 2) == cudaSuccess;
-    ok = ok && cudaMalloc(&w.QKV, rows * 3 * D * 2) == cudaSuccess;
-    ok = ok && cudaMalloc(&w.CC, rows * (D + F) * 2) == cudaSuccess;
-    ok = ok && cudaMalloc(&w.rope, rows * 64 * sizeof(float2)) == cudaSuccess;
+    ok = ok && dev_alloc(&w.Y, rows * D * 2) == cudaSuccess;
+    ok = ok && dev_alloc(&w.QKV, rows * 3 * D * 2) == cudaSuccess;
+    ok = ok && dev_alloc(&w.CC, rows * (D + F) * 2) == cudaSuccess;
+    ok = ok && dev_alloc(&w.rope, rows * 64 * sizeof(float2)) == cudaSuccess;
     if (!ok) {
       free_ws(w);
       return fail(FLUX_ENOMEM, "workspace allocation for %zu tokens failed", rows);
@@ -616,8 +651,10 @@ static int prepare_shape(flux_dit* m, int nt, int gh, int gw, const RefGrids& re
     w.cap_n = rows;
   }
   if (grow(&w.tokb, &w.cap_tok, (ni + nr) * c.in_ch) != cudaSuccess ||
-      grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt * nb, 1) * c.txt_dim) != cudaSuccess)
+      grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt * nb, 1) * c.txt_dim) != cudaSuccess) {
+    w.nt = -1;                                  // the maps may name a buffer grow() released: rebuild them
     return fail(FLUX_ENOMEM, "workspace allocation failed");
+  }
   if (w.nt == nt && w.gh == gh && w.gw == gw && w.nb == nb && same_refs(w.refs, refs))
     return prepare_quant(m, nt, static_cast<int>(ni + nr), nb);
   w.maps8 = false;
@@ -683,12 +720,12 @@ static int quantize_block_weights(flux_dit* m, cudaStream_t s) {
     bytes += (x.rows * x.cols + 255) / 256 * 256;
     rows += (x.rows + 63) / 64 * 64;
   }
-  if (cudaMalloc(&m->w8, bytes) != cudaSuccess || cudaMalloc(&m->w8_scale, rows * 4) != cudaSuccess) {
+  if (dev_alloc(&m->w8, bytes) != cudaSuccess || dev_alloc(&m->w8_scale, rows * 4) != cudaSuccess) {
     cudaFree(m->w8);
     cudaFree(m->w8_scale);
     m->w8 = nullptr;
     m->w8_scale = nullptr;
-    return fail(FLUX_ENOMEM, "cudaMalloc of the FP8 weights (%zu bytes) failed", bytes);
+    return fail(FLUX_ENOMEM, "device allocation of the FP8 weights (%zu bytes) failed", bytes);
   }
   std::vector<const uint8_t*> q(mats.size());
   std::vector<const float*> sc(mats.size());
@@ -1038,6 +1075,8 @@ extern "C" {
 
 const char* flux_get_error(void) { return last_error(); }
 
+int flux_get_error_code(void) { return last_error_code(); }
+
 size_t flux_blob_expected_bytes(const flux_dit_config* cfg) {
   if (!cfg || !valid_cfg(*cfg)) return 0;
   size_t total = 0;
@@ -1175,16 +1214,16 @@ int flux_dit_prepare_timesteps(flux_dit* m, const float* ts, int n, void* stream
   m->cache_n = 0;
   if (n == 0) return FLUX_OK;
   if (!m->mods_cache &&
-      cudaMalloc(&m->mods_cache, static_cast<size_t>(flux_dit::kMaxCachedT) * m->mods_rows * 4) != cudaSuccess)
-    return fail(FLUX_ENOMEM, "cudaMalloc of the modulation cache failed");
+      dev_alloc(&m->mods_cache, static_cast<size_t>(flux_dit::kMaxCachedT) * m->mods_rows * 4) != cudaSuccess)
+    return fail(FLUX_ENOMEM, "device allocation of the modulation cache failed");
   // up to four timesteps per pass: the embeddings, the time MLP and every modulation linear read
   // their weights once for the group (the GEMV takes the group's vectors together)
   float* temb = nullptr;
   float* th = nullptr;
   float* vec = nullptr;
   const size_t scratch = 4 * (static_cast<size_t>(tf) + 2 * D);
-  if (cudaMallocAsync(&temb, scratch * sizeof(float), s) != cudaSuccess)
-    return fail(FLUX_ENOMEM, "cudaMallocAsync of the timestep scratch failed");
+  if (dev_alloc_async(&temb, scratch * sizeof(float), s) != cudaSuccess)
+    return fail(FLUX_ENOMEM, "device allocation of the timestep scratch failed");
   th = temb + 4 * tf;
   vec = th + 4 * D;
   auto gv = [](double rows, double k, double nvec) { return rows * k * 2 + nvec * (rows * 6 + k * 4); };
@@ -1495,6 +1534,8 @@ int flux_dit_profile_read(flux_dit* m, int kind, double* ms, double* flops, doub
 }
 
 unsigned long long flux_kernel_launches(void) { return g_launches.load(); }
+
+void flux_test_fail_alloc_after(long long n) { g_fail_alloc_after.store(n < 0 ? -1 : n); }
 
 int flux_device_error(void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);

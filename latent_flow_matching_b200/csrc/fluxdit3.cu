@@ -264,9 +264,9 @@ int create3_impl(const void* blob, size_t blob_bytes, const flux3_dit_config* cf
   };
   // device copy: the blob's tensor area as is (same offsets), SwiGLU rows of linear1 re-interleaved
   const size_t scratch_floats = 3 * c.t_freq_dim + 3 * D + D + 2 * D + kModRowsD * D;
-  if (cudaMalloc(&m->wbuf, total - kHeaderBytes) != cudaSuccess ||
-      cudaMalloc(&m->scratch, scratch_floats * sizeof(float)) != cudaSuccess)
-    return cleanup(FLUX_ENOMEM, "cudaMalloc of model weights failed");
+  if (dev_alloc(&m->wbuf, total - kHeaderBytes) != cudaSuccess ||
+      dev_alloc(&m->scratch, scratch_floats * sizeof(float)) != cudaSuccess)
+    return cleanup(FLUX_ENOMEM, "device allocation of the model weights failed");
   m->temb = m->scratch;
   m->th = m->temb + 3 * c.t_freq_dim;
   m->tt = m->th + 3 * D;
@@ -344,9 +344,9 @@ int prepare3_fp8(flux3_dit* m, int nt, int ni, int nr, int nb) {
   const size_t n = static_cast<size_t>(nt) + ni + nr, rows = n * nb;
   if (rows > w.cap8) {
     free_ws3_fp8(w);
-    const bool ok = cudaMalloc(&w.Y8, rows * D) == cudaSuccess &&
-                    cudaMalloc(&w.C8, rows * (D + F)) == cudaSuccess && cudaMalloc(&w.sY, rows * 4) == cudaSuccess &&
-                    cudaMalloc(&w.sC, rows * 4) == cudaSuccess;
+    const bool ok = dev_alloc(&w.Y8, rows * D) == cudaSuccess &&
+                    dev_alloc(&w.C8, rows * (D + F)) == cudaSuccess && dev_alloc(&w.sY, rows * 4) == cudaSuccess &&
+                    dev_alloc(&w.sC, rows * 4) == cudaSuccess;
     if (!ok) {
       free_ws3_fp8(w);
       return fail(FLUX_ENOMEM, "FP8 workspace allocation for %zu tokens failed", rows);
@@ -414,10 +414,10 @@ int prepare3_fp4(flux3_dit* m, int nt, int ni, int nr, int nb) {
   if (static_cast<size_t>(rows) > w.cap4_rows || blocks > w.cap4_blocks) {
     free_ws3_fp4(w);
     const size_t R = rows, B = blocks * 128;
-    const bool ok = cudaMalloc(&w.Y4, R * D / 2) == cudaSuccess && cudaMalloc(&w.C4, R * (D + F) / 2) == cudaSuccess &&
-                    cudaMalloc(&w.sfY, B * D / 16) == cudaSuccess &&
-                    cudaMalloc(&w.sfC, B * (D + F) / 16) == cudaSuccess && cudaMalloc(&w.sY4, R * 4) == cudaSuccess &&
-                    cudaMalloc(&w.sC4, R * 4) == cudaSuccess;
+    const bool ok = dev_alloc(&w.Y4, R * D / 2) == cudaSuccess && dev_alloc(&w.C4, R * (D + F) / 2) == cudaSuccess &&
+                    dev_alloc(&w.sfY, B * D / 16) == cudaSuccess &&
+                    dev_alloc(&w.sfC, B * (D + F) / 16) == cudaSuccess && dev_alloc(&w.sY4, R * 4) == cudaSuccess &&
+                    dev_alloc(&w.sC4, R * 4) == cudaSuccess;
     if (!ok) {
       free_ws3_fp4(w);
       return fail(FLUX_ENOMEM, "NVFP4 workspace allocation for %d tokens failed", rows);
@@ -466,11 +466,11 @@ int prepare_shape3(flux3_dit* m, int nt, int gh, int gw, const RefGrids& refs, i
   const size_t n = nt + ni + nr, rows = n * nb;
   if (rows > w.cap_n) {
     free_ws3(w);
-    bool ok = cudaMalloc(&w.X, rows * D * 4) == cudaSuccess;
-    ok = ok && cudaMalloc(&w.Y, rows * D * 2) == cudaSuccess;
-    ok = ok && cudaMalloc(&w.QKV, rows * 3 * D * 2) == cudaSuccess;
-    ok = ok && cudaMalloc(&w.CC, rows * (D + F) * 2) == cudaSuccess;
-    ok = ok && cudaMalloc(&w.rope, rows * 64 * sizeof(float2)) == cudaSuccess;
+    bool ok = dev_alloc(&w.X, rows * D * 4) == cudaSuccess;
+    ok = ok && dev_alloc(&w.Y, rows * D * 2) == cudaSuccess;
+    ok = ok && dev_alloc(&w.QKV, rows * 3 * D * 2) == cudaSuccess;
+    ok = ok && dev_alloc(&w.CC, rows * (D + F) * 2) == cudaSuccess;
+    ok = ok && dev_alloc(&w.rope, rows * 64 * sizeof(float2)) == cudaSuccess;
     if (!ok) {
       free_ws3(w);
       return fail(FLUX_ENOMEM, "workspace allocation for %zu tokens failed", rows);
@@ -478,8 +478,10 @@ int prepare_shape3(flux3_dit* m, int nt, int gh, int gw, const RefGrids& refs, i
     w.cap_n = rows;
   }
   if (grow(&w.tokb, &w.cap_tok, (ni + nr) * c.in_ch) != cudaSuccess ||
-      grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt * nb, 1) * c.txt_dim) != cudaSuccess)
+      grow(&w.txtb, &w.cap_txt, std::max<size_t>(nt * nb, 1) * c.txt_dim) != cudaSuccess) {
+    w.nt = -1;                                  // the maps may name a buffer grow() released: rebuild them
     return fail(FLUX_ENOMEM, "workspace allocation failed");
+  }
   if (w.nt == nt && w.gh == gh && w.gw == gw && w.nb == nb && same_refs(w.refs, refs))
     return prepare3_quant(m, nt, static_cast<int>(ni), static_cast<int>(nr), nb);
   w.maps8 = false;
@@ -527,12 +529,12 @@ int quantize3_block_weights(flux3_dit* m, cudaStream_t s) {
   const size_t b1 = (r1 * D + 255) / 256 * 256, b2 = (r2 * (D + F) + 255) / 256 * 256;
   const size_t s1 = (r1 + 63) / 64 * 64, s2 = (r2 + 63) / 64 * 64;
   const size_t nb = blocks.size();
-  if (cudaMalloc(&m->w8, nb * (b1 + b2)) != cudaSuccess || cudaMalloc(&m->w8_scale, nb * (s1 + s2) * 4) != cudaSuccess) {
+  if (dev_alloc(&m->w8, nb * (b1 + b2)) != cudaSuccess || dev_alloc(&m->w8_scale, nb * (s1 + s2) * 4) != cudaSuccess) {
     cudaFree(m->w8);
     cudaFree(m->w8_scale);
     m->w8 = nullptr;
     m->w8_scale = nullptr;
-    return fail(FLUX_ENOMEM, "cudaMalloc of the FP8 weights failed");
+    return fail(FLUX_ENOMEM, "device allocation of the FP8 weights failed");
   }
   bool ok = true;
   for (size_t i = 0; i < nb; ++i) {

@@ -203,6 +203,21 @@ int gemm_fp4_read_device_error(cudaStream_t stream);
 // Programmatic dependent launches are on unless the environment sets FLUX_PDL=0 (read at every
 // launch, so a process can compare both; a CUDA graph keeps what was set when it was captured).
 bool pdl_enabled();
+
+// Every device allocation of the library goes through dev_alloc / dev_alloc_async: a failed
+// cudaMalloc leaves *p null and its error is cleared from the runtime's last-error state (so that a
+// later launch check does not report it again), and flux_test_fail_alloc_after can make the n-th
+// following allocation fail the same way without asking the driver.
+cudaError_t dev_alloc(void** p, size_t bytes);
+cudaError_t dev_alloc_async(void** p, size_t bytes, cudaStream_t s);
+template <typename T>
+cudaError_t dev_alloc(T** p, size_t bytes) {
+  return dev_alloc(reinterpret_cast<void**>(p), bytes);
+}
+template <typename T>
+cudaError_t dev_alloc_async(T** p, size_t bytes, cudaStream_t s) {
+  return dev_alloc_async(reinterpret_cast<void**>(p), bytes, s);
+}
 // Launch `kernel` on `s` with programmatic stream serialisation (when enabled): the kernel may be
 // scheduled before the previous kernel on the stream has finished, and waits for it with
 // pdl_wait() (common.cuh) before touching global memory.  Only kernels that call pdl_wait()

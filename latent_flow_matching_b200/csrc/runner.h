@@ -38,6 +38,7 @@ struct NvtxRange {
 // printf-style flux_get_error() message for the calling thread; returns `code`.
 int fail(int code, const char* fmt, ...);
 const char* last_error();
+int last_error_code();
 
 #define FD_CUDA(expr)                                                                          \
   do {                                                                                         \
@@ -242,12 +243,12 @@ inline int quantize_weights_nvfp4(std::vector<Fp4Mat>& mats, uint8_t** buf, floa
     bytes += up(x.rows * x.cols / 2, 256) + up(nvfp4_scale_bytes(x.rows, x.cols), 256);
     rows += up(x.rows, 64);
   }
-  if (cudaMalloc(buf, bytes) != cudaSuccess || cudaMalloc(scales, rows * 4) != cudaSuccess) {
+  if (dev_alloc(buf, bytes) != cudaSuccess || dev_alloc(scales, rows * 4) != cudaSuccess) {
     cudaFree(*buf);
     cudaFree(*scales);
     *buf = nullptr;
     *scales = nullptr;
-    return fail(FLUX_ENOMEM, "cudaMalloc of the NVFP4 weights (%zu bytes) failed", bytes);
+    return fail(FLUX_ENOMEM, "device allocation of the NVFP4 weights (%zu bytes) failed", bytes);
   }
   FD_CUDA(cudaMemsetAsync(*buf, 0, bytes, s));       // block-scale padding rows read as 0
   size_t boff = 0, roff = 0;
@@ -272,7 +273,7 @@ cudaError_t grow(T** p, size_t* cap, size_t need) {
   cudaFree(*p);
   *p = nullptr;
   *cap = 0;
-  cudaError_t e = cudaMalloc(p, need * sizeof(T));
+  cudaError_t e = dev_alloc(p, need * sizeof(T));
   if (e == cudaSuccess) *cap = need;
   return e;
 }

@@ -87,6 +87,17 @@ def test_create_rejects_corrupt_blob(L):
     assert "size" in F.get_error()
     h = L.flux_dit_create(None, 0, None, None)
     assert not h
+    assert L.flux_get_error_code() == F.FLUX_EINVAL          # a bad argument, not an allocation
+
+
+def test_allocation_hook_needs_no_device(L):
+    """Arming and disarming the out-of-memory test hook touch no device (this runs without a GPU),
+    and a call rejected for its arguments while the hook is armed still reports FLUX_EINVAL."""
+    L.flux_test_fail_alloc_after(0)
+    h = L.flux_dit_create(None, 0, None, None)
+    assert not h and L.flux_get_error_code() == F.FLUX_EINVAL
+    L.flux_test_fail_alloc_after(-1)
+    L.flux_test_fail_alloc_after(-5)
 
 
 def test_create_rejects_config_mismatch(L):
