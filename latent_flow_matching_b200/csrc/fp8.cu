@@ -29,8 +29,7 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
 
 // Maximum over the CTA (256 threads); `red` holds 8 floats.
 __device__ __forceinline__ float block_max(float v, float* red) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  v = redux_max(v, 0xffffffffu);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) red[warp] = v;
   __syncthreads();
@@ -146,8 +145,7 @@ __global__ void __launch_bounds__(kQThreads) ln_mod_fp8_kernel(const float* __re
     v[i].w = (v[i].w - mean) * rstd * (1.f + sc.w) + sh.w;
     amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
   }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  amax = redux_max(amax, 0xffffffffu);
   if (lane == 0) red[2][warp] = amax;
   __syncthreads();
   amax = red[2][0];

@@ -39,10 +39,11 @@ __device__ __forceinline__ float bf16_abs_max8(const uint4& w, float m) {
 // Sum (or maximum) over the CTA; every thread gets the result.  red: one float per warp.
 template <bool kMax>
 __device__ __forceinline__ float cta_reduce(float v, float* red) {
+  if constexpr (kMax) {
+    v = redux_max(v, 0xffffffffu);
+  } else {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float u = __shfl_xor_sync(0xffffffffu, v, o);
-    v = kMax ? fmaxf(v, u) : v + u;
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   }
   __syncthreads();                                   // red may still be read by the previous reduction
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
