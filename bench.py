@@ -517,7 +517,7 @@ def run_ours(args, w):
     gemm_gbs = g_by / (g_ms / 1e3) / 1e9
     # the linears' FLOPs per algorithmic byte against the ridge where the tensor and HBM roofs meet:
     # below it (the tiny model's 16-row problems) the weights' read bounds the launch
-    intensity = g_fl / g_by
+    intensity = g_fl / g_by if g_by else float("inf")
     ridge = gemm_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     hbm_bound = intensity < ridge
     attn_tflops = a_fl / (a_ms / 1e3) / 1e12

@@ -120,6 +120,11 @@ __device__ __forceinline__ void stage_issue_nvf4(uint32_t d_tmem, uint64_t ad, u
       : "memory");
 }
 
+// The offsets written into stage_issue_nvf4 (in the descriptors' 16-byte units: 2 per MMA for A
+// and W, 32 per MMA for a 512-byte scale block, 128 for W's second 128 columns of scales).
+static_assert(BKE == 4 * 64 && SFA_BYTES == 4 * 512 && SFB_BYTES == 2 * 2048 && kSfCol % 16 == 0,
+              "stage_issue_nvf4 assumes four K = 64 MMAs per stage and 512-byte scale blocks");
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads4, 1)
     gemm_fp4_tc2_kernel(const __grid_constant__ GemmParams4 P4) {
   const GemmParams& P = P4.g;
