@@ -46,8 +46,8 @@ from oracle import flux3_oracle as O3  # noqa: E402
 ROW_STRIDE = {"t2i256": 1, "t2i512": 2, "t2i1024": 8, "i2i1024": 8, "mref1024": 8, "cfg256": 1,
               "f3t2i256": 1, "f3i2i256": 1, "f3t2i1024": 8, "f3i2i1024": 8, "f3cfg256": 1,
               "t2i256_fp8": 1, "t2i256_nvfp4": 1, "t2i1024_fp8": 8, "t2i1024_nvfp4": 8,
-              "f3t2i256_fp8": 1, "f3t2i256_nvfp4": 1}
-STEPS_RUN = {"f3i2i1024": 4, "t2i1024_fp8": 2, "t2i1024_nvfp4": 2}
+              "f3t2i256_fp8": 1, "f3t2i256_nvfp4": 1, "f3t2i1024_fp8": 8, "f3t2i1024_nvfp4": 8}
+STEPS_RUN = {"f3i2i1024": 4, "t2i1024_fp8": 2, "t2i1024_nvfp4": 2, "f3t2i1024_fp8": 2, "f3t2i1024_nvfp4": 2}
 PRECISIONS = ("fp8", "nvfp4")
 
 

@@ -165,10 +165,11 @@ def test_flux3_one_per_mode_one_joint_block_at_full_token_count(precision):
     assert err < 0.6 * rel_l2(v, exact)
 
 
-@pytest.mark.parametrize("name", ["f3t2i256_fp8", "f3t2i256_nvfp4"])
+@pytest.mark.parametrize("name", ["f3t2i256_fp8", "f3t2i256_nvfp4", "f3t2i1024_fp8", "f3t2i1024_nvfp4"])
 def test_flux3_quantised_sampler_against_quantised_oracle_golden(name):
-    """FLUX.3 Image Klein at 256^2 (5 per-mode + 28 joint blocks, flow-map target time), 4 steps with
-    quantised block linears, against the FLUX.3 oracle's quantised golden; bar 1.25 sigma as above."""
+    """FLUX.3 Image Klein (5 per-mode + 28 joint blocks, flow-map target time) with quantised block
+    linears against the FLUX.3 oracle's quantised golden: at 256^2 all 4 steps, at 1024^2 (4256
+    tokens) the first 2 of the 16 steps on every 8th image row; bar 1.25 sigma as above."""
     path = os.path.join(GOLDEN, f"{name}.npz")
     if not os.path.exists(path):
         pytest.skip(f"golden {path} not generated")
