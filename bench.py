@@ -322,6 +322,32 @@ def fractions(tflops, peaks, fp4=False, fp8=False):
             "spec_2250": round(tflops / (mult * SPEC_BF16_TFLOPS), 4)}
 
 
+def gemm_roofline(g_ms, g_fl, g_by, peaks, peak_src, fp4=False, fp8=False):
+    """The linears' roofline entries from their summed device time, FLOPs and algorithmic bytes.
+
+    The GEMM peak is the measured sustained bf16 rate (2x for FP8, 4x for NVFP4: the nominal dense
+    ratios).  When the FLOPs per algorithmic byte fall below the ridge point (peak / measured copy
+    bandwidth), as on the tiny model's 16-row problems where the weights' read bounds each launch,
+    the entries are the HBM roofline in GB/s; otherwise the tensor roofline in TFLOP/s."""
+    gemm_peak = peaks["bf16_tflops_sustained"] * (4.0 if fp4 else 2.0 if fp8 else 1.0)
+    peak_kind = ("nvfp4 = 4 x bf16 sustained (nominal dense ratio), " if fp4 else
+                 "fp8 = 2 x bf16 sustained (nominal dense ratio), " if fp8 else "bf16 sustained, ") + peak_src
+    tflops = g_fl / (g_ms / 1e3) / 1e12
+    gbs = g_by / (g_ms / 1e3) / 1e9
+    intensity = g_fl / g_by if g_by else float("inf")
+    ridge = gemm_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if intensity < ridge:
+        out = {"bound": "hbm", "achieved": round(gbs, 1), "peak": round(peaks["hbm_gbs"], 1), "unit": "GB/s",
+               "frac": round(gbs / peaks["hbm_gbs"], 4), "peak_kind": f"HBM copy, {peak_src}",
+               "tflops": round(tflops, 2)}
+    else:
+        out = {"bound": "tensor", "achieved": round(tflops, 1), "peak": round(gemm_peak, 1), "unit": "TFLOP/s",
+               "frac": round(tflops / gemm_peak, 4), "peak_kind": peak_kind,
+               "frac_of": fractions(tflops, peaks, fp4=fp4, fp8=fp8)}
+    out.update(flop_per_byte=round(intensity, 1), ridge_flop_per_byte=round(ridge, 1))
+    return out
+
+
 TENSOR_KINDS = ("gemm", "attention")
 
 
@@ -504,22 +530,10 @@ def run_ours(args, w):
     d2h = out_pin.numel() * 4
 
     peaks, peak_src = load_peaks()
-    # FP8 / NVFP4 tensor peaks: the measured bf16 figure times the nominal dense ratios 4.5 / 2.25 and
-    # 9 / 2.25 PFLOP/s
-    gemm_peak = peaks["bf16_tflops_sustained"] * (4.0 if fp4 else 2.0 if fp8 else 1.0)
-    gemm_peak_kind = ("nvfp4 = 4 x bf16 sustained (nominal dense ratio), " if fp4 else
-                      "fp8 = 2 x bf16 sustained (nominal dense ratio), " if fp8 else "bf16 sustained, ") + peak_src
     flops = step_flops(w)
     tflops = flops / (ms_step / 1e3) / 1e12
     g_ms, g_fl, g_by, g_n = prof["gemm"]
     a_ms, a_fl, a_by, a_n = prof["attention"]
-    gemm_tflops = g_fl / (g_ms / 1e3) / 1e12
-    gemm_gbs = g_by / (g_ms / 1e3) / 1e9
-    # the linears' FLOPs per algorithmic byte against the ridge where the tensor and HBM roofs meet:
-    # below it (the tiny model's 16-row problems) the weights' read bounds the launch
-    intensity = g_fl / g_by if g_by else float("inf")
-    ridge = gemm_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    hbm_bound = intensity < ridge
     attn_tflops = a_fl / (a_ms / 1e3) / 1e12
     kinds = {k: kernel_kind_line(k, v_, args.steps, peaks) for k, v_ in prof.items() if v_[3]}
 
@@ -549,15 +563,7 @@ def run_ours(args, w):
                                     "gemm_bf16_tc2<fp8> (CTA-pair tcgen05 kind::f8f6f4) for the block linears, "
                                     "bf16 for the input / output projections" if fp8 else
                                     "gemm_bf16_tc2 (CTA-pair tcgen05 GEMM) + the 128-wide output GEMM, all linear layers"),
-                         **({"bound": "hbm", "achieved": round(gemm_gbs, 1), "peak": round(peaks["hbm_gbs"], 1),
-                             "unit": "GB/s", "frac": round(gemm_gbs / peaks["hbm_gbs"], 4),
-                             "peak_kind": f"HBM copy, {peak_src}", "tflops": round(gemm_tflops, 2)}
-                            if hbm_bound else
-                            {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(gemm_peak, 1),
-                             "unit": "TFLOP/s", "frac": round(gemm_tflops / gemm_peak, 4),
-                             "peak_kind": gemm_peak_kind,
-                             "frac_of": fractions(gemm_tflops, peaks, fp4=fp4, fp8=fp8)}),
-                         "flop_per_byte": round(intensity, 1), "ridge_flop_per_byte": round(ridge, 1),
+                         **gemm_roofline(g_ms, g_fl, g_by, peaks, peak_src, fp4=fp4, fp8=fp8),
                          "traffic": None,
                          "traffic_note": ("DRAM bytes need a profiler's counters, which this timed run does "
                                           "not take; the ncu capture of the same kernel is kept beside the "
